@@ -1,0 +1,414 @@
+"""Pins for the CPU oracle: each check ties an oracle function to something
+other than itself (an independent Philox implementation, closed forms,
+hand-derived worked examples, brute-force enumeration with exact rationals,
+numpy), so that a dropped term, a wrong sign or index or a transposed operand
+fails at least one of them. CPU only."""
+import json
+import math
+import subprocess
+import sys
+from fractions import Fraction
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import oracle
+from quantized_lora_merge_b200 import workloads as wl
+
+GOLDEN = Path(__file__).resolve().parent / "golden"
+
+
+# ---------------------------------------------------------------------------
+# a1: Philox4x32-10 against Triton's independent implementation
+# ---------------------------------------------------------------------------
+def test_philox_matches_independent_implementation():
+    rng = np.random.default_rng(12345)
+    cases = [[0, 0, 0, 0, 0, 0], [2**32 - 1] * 6, [1, 0, 0, 0, 1, 0], [0, 1, 0, 0, 0, 0],
+             [0, 0, 7, 0, 1, 0], [123, 0, 5, 0, 1, 0]]
+    cases += rng.integers(0, 2**32, size=(26, 6), dtype=np.uint64).tolist()
+    script = Path(__file__).resolve().parent / "philox_triton_reference.py"
+    res = subprocess.run([sys.executable, str(script), json.dumps(cases)], check=True,
+                         capture_output=True, text=True, timeout=600)
+    expected = json.loads(res.stdout.strip().splitlines()[-1])
+    for case, exp in zip(cases, expected):
+        got = oracle.philox4x32_10(case[:4], case[4:]).tolist()
+        assert got == exp, f"Philox mismatch for counter/key {case}"
+
+
+def test_aux_word_counter_layout():
+    """Element e of stream (seed, sid) is word e%4 of the block whose counter
+    is (e//4 low, e//4 high, sid, 0) under key (seed low, seed high); checked
+    through the independently pinned block function, including a block index
+    above 2^32 and a seed above 2^32."""
+    for seed, sid, e in [(1, 0, 0), (1, 0, 7), (1, 3, 1023), (2**40 + 5, 9, 2**34 + 6),
+                         (1, 2**32 - 1, 5)]:
+        block = e >> 2
+        words = oracle.philox4x32_10([block & 0xFFFFFFFF, block >> 32, sid, 0],
+                                     [seed & 0xFFFFFFFF, seed >> 32])
+        assert oracle.aux_word(seed, sid, e) == int(words[e & 3])
+
+
+def test_philox_output_is_uniform():
+    """Chi-square of 2^16 words over 256 top-byte bins, and bit balance."""
+    words = np.concatenate([oracle.philox4x32_10([b, 0, 1, 0], [7, 0]) for b in range(1 << 14)])
+    words = words.astype(np.uint64)
+    counts = np.bincount((words >> 24).astype(np.int64), minlength=256)
+    expected = words.size / 256
+    chi2 = float(((counts - expected) ** 2 / expected).sum())
+    assert chi2 < 256 + 6 * math.sqrt(2 * 256)
+    bits = np.unpackbits(words.astype(np.uint32).view(np.uint8))
+    assert abs(bits.mean() - 0.5) < 4 * 0.5 / math.sqrt(bits.size)
+
+
+# ---------------------------------------------------------------------------
+# a1: the Laplace sampler
+# ---------------------------------------------------------------------------
+def test_laplace_closed_forms():
+    g = json.loads((GOLDEN / "laplace_closed_form.json").read_text())
+    for case in g["cases"]:
+        expected = eval(case["R_expr"], {"ln": math.log, "log": math.log, "log1p": math.log1p})
+        got = float(oracle.laplace_from_word(case["x"])[0])
+        assert got == pytest.approx(expected, rel=1e-15, abs=1e-300), case
+
+
+def test_laplace_inverse_cdf_round_trip():
+    """F(R(x)) = u(x) with F the textbook Laplace(0,1) CDF."""
+    rng = np.random.default_rng(5)
+    xs = rng.integers(0, 2**32, size=4000, dtype=np.uint64).astype(np.uint32)
+    R = oracle.laplace_from_word(xs)
+    u = (2.0 * (xs >> 9).astype(np.float64) + 1.0) * 2.0**-24
+    F = np.where(R < 0, 0.5 * np.exp(R), 1.0 - 0.5 * np.exp(-R))
+    assert np.max(np.abs(F - u)) < 1e-15
+
+
+def test_laplace_symmetry_exact():
+    """Complementing the 23 uniform bits maps u to 1-u, hence R to -R exactly."""
+    rng = np.random.default_rng(6)
+    xs = rng.integers(0, 2**32, size=2000, dtype=np.uint64).astype(np.uint32)
+    assert np.array_equal(oracle.laplace_from_word(xs ^ np.uint32(0xFFFFFE00)),
+                          -oracle.laplace_from_word(xs))
+
+
+def test_laplace_moments():
+    """Laplace(0,1): mean 0, variance 2, excess kurtosis 3, P(|R|>t)=e^-t."""
+    R = oracle.aux_R(1024, 1024, seed=1, stream_id=0).ravel()
+    N = R.size
+    assert abs(R.mean()) < 4 * math.sqrt(2.0 / N)
+    var = R.var()
+    assert abs(var - 2.0) < 4 * math.sqrt(20.0 / N)
+    kurt = np.mean(R**4) / var**2 - 3.0
+    assert abs(kurt - 3.0) < 0.1
+    for t in (0.5, 1.0, 2.0, 4.0):
+        p = math.exp(-t)
+        assert abs(np.mean(np.abs(R) > t) - p) < 5 * math.sqrt(p * (1 - p) / N)
+    assert np.max(np.abs(R)) <= 23 * math.log(2) + 1e-12
+
+
+# ---------------------------------------------------------------------------
+# a2: sigma and VMC
+# ---------------------------------------------------------------------------
+def test_population_std_closed_form_ramp():
+    for N in (1, 2, 10, 1001):
+        x = np.arange(N, dtype=np.float64) * 3.0 + 7.0
+        assert oracle.population_std(x) == pytest.approx(3.0 * math.sqrt((N * N - 1) / 12.0),
+                                                         rel=1e-14, abs=1e-14)
+
+
+def test_std_f32_and_sigma_r_against_numpy():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((37, 53)) * 0.02 + 0.5).astype(np.float32)
+    assert oracle.std_f32(W) == pytest.approx(float(np.std(W.astype(np.float64))), rel=1e-12)
+    R = oracle.aux_R(37, 53, 1, 4)
+    assert oracle.sigma_r(37, 53, 1, 4) == pytest.approx(float(np.std(R)), rel=1e-12)
+
+
+def test_vmc_scale_laws():
+    sw, sr = 0.02, 1.41
+    assert oracle.vmc_scale(sw, sr, 0.0) == 1.0
+    # alpha = 1 matches sigma exactly: std(c R) = sigma_W
+    R = oracle.aux_R(64, 64, 1, 0)
+    c1 = oracle.vmc_scale(sw, float(np.std(R)), 1.0)
+    assert np.std(c1 * R) == pytest.approx(sw, rel=1e-13)
+    # exponent law: c(2a) = c(a)^2, and c < 1 grows toward 1 as alpha shrinks
+    assert oracle.vmc_scale(sw, sr, 3.0) == pytest.approx(oracle.vmc_scale(sw, sr, 1.5) ** 2,
+                                                          rel=1e-14)
+    assert oracle.vmc_scale(sw, sr, 0.5) > oracle.vmc_scale(sw, sr, 1.5)
+
+
+# ---------------------------------------------------------------------------
+# a3 / a6: the affine quantizer
+# ---------------------------------------------------------------------------
+def test_affine_quantizer_worked_examples():
+    g = json.loads((GOLDEN / "affine_quantizer_worked.json").read_text())
+    for case in g["cases"]:
+        q = oracle.affine_quantize_row(case["x"], case["bits"])
+        assert q["scale"] == pytest.approx(case["scale"], rel=1e-15), case
+        assert q["zero"] == case["zero"], case
+        assert q["codes"].tolist() == case["codes"], case
+
+
+def _brute_force_code(x: Fraction, scale: Fraction, zero: int, qmax: int) -> int:
+    best, best_err = None, None
+    for q in range(qmax + 1):
+        err = abs(x - scale * (q - zero))
+        if best is None or err < best_err or (err == best_err and (q - zero) % 2 == 0):
+            best, best_err = q, err
+    return best
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_affine_quantizer_brute_force(bits):
+    """Every code is the exact argmin over all 2^b codes of |x - s(q - z)|,
+    ties to the even (q - z); zero is exactly representable; the extremes of a
+    row that spans both signs land on codes 0 and 2^b - 1 (the grid is tight);
+    every value inside the range is reproduced within s/2."""
+    rng = np.random.default_rng(bits)
+    qmax = 2**bits - 1
+    for trial in range(60):
+        n = int(rng.integers(1, 17))
+        x = rng.standard_normal(n) * 10 ** rng.uniform(-3, 1)
+        if trial % 7 == 0:
+            x = np.abs(x)
+        if trial % 11 == 0:
+            x = -np.abs(x)
+        q = oracle.affine_quantize_row(x, bits)
+        scale, zero = Fraction(q["scale"]), q["zero"]
+        assert 0 <= zero <= qmax
+        for xi, ci in zip(x, q["codes"]):
+            assert ci == _brute_force_code(Fraction(float(xi)), scale, zero, qmax)
+            assert abs(Fraction(float(xi)) - scale * (ci - zero)) <= scale / 2 * (1 + 1e-12)
+        if x.min() < 0 < x.max():
+            assert q["codes"][int(np.argmin(x))] == 0
+            assert q["codes"][int(np.argmax(x))] == qmax
+
+
+# ---------------------------------------------------------------------------
+# a1-a3: layer preparation (AQS + VMC)
+# ---------------------------------------------------------------------------
+def _small_layer(d, n, r, w_bits, sid, variant="mul", out_bits=8):
+    spec = wl.LayerSpec("t", d, n, r, w_bits, variant, out_bits, stream_id=sid)
+    return spec, wl.host_W(spec), wl.host_A(spec), wl.host_B(spec)
+
+
+@pytest.mark.parametrize("w_bits", [4, 8])
+def test_gen_aux_composition(w_bits):
+    """sigma_W, sigma_R against numpy; R* = c R; each row is the pinned affine
+    quantizer of W - R*; and the AQS reconstruction s(W_round - z) + R*
+    reproduces W within s/2 (a wrong sign on R* would miss by ~2|R*|)."""
+    spec, W, _, _ = _small_layer(24, 40, 4, w_bits, sid=3)
+    g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, w_bits, want_r_star=True)
+    R = oracle.aux_R(24, 40, spec.seed, spec.stream_id)
+    assert g["sigma_w"] == pytest.approx(float(np.std(W.astype(np.float64))), rel=1e-12)
+    assert g["sigma_r"] == pytest.approx(float(np.std(R)), rel=1e-12)
+    assert g["c"] == pytest.approx((g["sigma_w"] / g["sigma_r"]) ** spec.alpha, rel=1e-14)
+    np.testing.assert_allclose(g["r_star"], g["c"] * R, rtol=1e-15, atol=0)
+    for i in range(24):
+        q = oracle.affine_quantize_row(W[i].astype(np.float64) - g["r_star"][i], w_bits)
+        assert g["codes"][i].tolist() == q["codes"].tolist()
+        assert g["s"][i] == q["scale"] and g["z"][i] == q["zero"]
+    recon = g["s"][:, None] * (g["codes"] - g["z"][:, None]) + g["r_star"]
+    assert np.all(np.abs(recon - W) <= g["s"][:, None] / 2 * (1 + 1e-9))
+
+
+def test_gen_aux_row_subset_matches_full():
+    spec, W, _, _ = _small_layer(20, 16, 4, 8, sid=1)
+    full = oracle.gen_aux(W, 1, 1, 1.5, 8)
+    part = oracle.gen_aux(W, 1, 1, 1.5, 8, row_begin=7, row_count=5)
+    assert np.array_equal(full["codes"][7:12], part["codes"])
+    assert np.array_equal(full["s"][7:12], part["s"])
+
+
+# ---------------------------------------------------------------------------
+# a4-a5: the MLA adaptation term
+# ---------------------------------------------------------------------------
+def _prepared(d, n, r, w_bits, sid):
+    spec, W, A, B = _small_layer(d, n, r, w_bits, sid)
+    g = oracle.gen_aux(W, spec.seed, sid, spec.alpha, w_bits, want_r_star=True)
+    return spec, W, A, B, g
+
+
+@pytest.mark.parametrize("w_bits,d,n,r", [(8, 16, 16, 4), (4, 12, 20, 3), (8, 9, 33, 16)])
+def test_mla_identity(w_bits, d, n, r):
+    """[s + (R* + AB)/D] * D = Q[W - R*] + R* + AB on D != 0 (AQS and MLA give
+    the same pre-quantization weight), with AB from numpy and R* from the
+    pinned sampler; U = s where D = 0."""
+    spec, W, A, B, g = _prepared(d, n, r, w_bits, sid=2)
+    s32 = g["s"].astype(np.float32)
+    U, D = oracle.mla_rows(g["codes"], s32, g["z"], A, B, spec.seed, 2, g["sigma_w"],
+                           g["sigma_r"], spec.alpha)
+    AB = A.astype(np.float64) @ B.astype(np.float64)
+    rhs = s32.astype(np.float64)[:, None] * D + g["r_star"] + AB
+    nz = D != 0
+    scale = np.abs(s32.astype(np.float64)[:, None] * D) + np.abs(g["r_star"]) + np.abs(AB)
+    assert np.all(np.abs(U * D - rhs)[nz] <= 1e-13 * scale[nz])
+    assert np.array_equal(U[~nz], np.broadcast_to(s32.astype(np.float64)[:, None], U.shape)[~nz])
+    assert np.array_equal(D, g["codes"].astype(np.int64) - g["z"][:, None])
+
+
+def test_mla_exact_rational_on_4x4():
+    """The same identity term by term in exact rationals on a 4x4 layer: the
+    oracle's fp64 U differs from the exact quotient by at most one rounding."""
+    spec, W, A, B, g = _prepared(4, 4, 2, 8, sid=5)
+    s32 = g["s"].astype(np.float32)
+    U, D = oracle.mla_rows(g["codes"], s32, g["z"], A, B, spec.seed, 5, g["sigma_w"],
+                           g["sigma_r"], spec.alpha)
+    for i in range(4):
+        for j in range(4):
+            if D[i, j] == 0:
+                continue
+            ab = sum(Fraction(float(A[i, k])) * Fraction(float(B[k, j])) for k in range(2))
+            exact = (Fraction(float(s32[i])) + (Fraction(float(g["r_star"][i, j])) + ab)
+                     / int(D[i, j]))
+            assert abs(Fraction(float(U[i, j])) - exact) <= abs(exact) * Fraction(1, 2**50)
+
+
+# ---------------------------------------------------------------------------
+# a6: IntLoRA_MUL
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w_bits,u_bits", [(8, 8), (4, 4)])
+def test_merge_mul_composition(w_bits, u_bits):
+    """U_round, s_bar, z_bar are the pinned affine quantizer applied to the
+    pinned U row; P = (U_round - z_bar) * D in integer arithmetic."""
+    spec, W, A, B, g = _prepared(10, 24, 4, w_bits, sid=7)
+    s32 = g["s"].astype(np.float32)
+    m = oracle.merge_mul(g["codes"], s32, g["z"], A, B, spec.seed, 7, g["sigma_w"], g["sigma_r"],
+                         spec.alpha, u_bits)
+    U, D = oracle.mla_rows(g["codes"], s32, g["z"], A, B, spec.seed, 7, g["sigma_w"],
+                           g["sigma_r"], spec.alpha)
+    for i in range(10):
+        q = oracle.affine_quantize_row(U[i], u_bits)
+        assert m["u_round"][i].tolist() == q["codes"].tolist()
+        assert m["sbar"][i] == q["scale"] and m["zbar"][i] == q["zero"]
+        want = [(int(a) - q["zero"]) * int(b) for a, b in zip(q["codes"], D[i])]
+        assert m["P"][i].tolist() == want
+    lim = (2**w_bits - 1) * (2**u_bits - 1)
+    assert np.abs(m["P"]).max() <= lim
+
+
+def test_merge_mul_ab_zero_special_case():
+    """AB zero-initialised: W'_pre = Q[W - R*] + R*, and after MUL quantization
+    |s_bar P - (Q[W-R*] + R*)| <= s_bar |D| / 2 on D != 0, P = 0 on D = 0."""
+    spec, W, A, B, g = _prepared(12, 32, 4, 8, sid=11)
+    s32 = g["s"].astype(np.float32).astype(np.float64)
+    A0 = np.zeros_like(A)
+    m = oracle.merge_mul(g["codes"], s32.astype(np.float32), g["z"], A0, B, spec.seed, 11,
+                         g["sigma_w"], g["sigma_r"], spec.alpha, 8)
+    D = g["codes"].astype(np.int64) - g["z"][:, None]
+    target = s32[:, None] * D + g["r_star"]
+    err = np.abs(m["sbar"][:, None] * m["P"] - target)
+    nz = D != 0
+    assert np.all(err[nz] <= (m["sbar"][:, None] * np.abs(D) / 2 * (1 + 1e-9))[nz])
+    assert np.all(m["P"][~nz] == 0)
+
+
+def test_merge_mul_bit_width_limit():
+    """W' -> W + AB as the bit widths grow. At a fixed base width the MUL
+    output converges to the MLA weight Q[W-R*] + R* + AB like 2^-b_U; growing
+    the base width as well (with b_U = b_W + 12) drives it to W + AB."""
+    spec, W, A, B = _small_layer(16, 48, 4, 8, sid=13)
+    AB = A.astype(np.float64) @ B.astype(np.float64)
+    errs_u = []
+    g8 = oracle.gen_aux(W, spec.seed, 13, spec.alpha, 8, want_r_star=True)
+    s8 = g8["s"].astype(np.float32)
+    D8 = g8["codes"].astype(np.int64) - g8["z"][:, None]
+    mla = s8.astype(np.float64)[:, None] * D8 + g8["r_star"] + AB
+    for ub in (8, 12, 16, 20):
+        m = oracle.merge_mul(g8["codes"], s8, g8["z"], A, B, spec.seed, 13, g8["sigma_w"],
+                             g8["sigma_r"], spec.alpha, ub)
+        nz = D8 != 0
+        errs_u.append(np.linalg.norm((m["sbar"][:, None] * m["P"] - mla)[nz])
+                      / np.linalg.norm(mla[nz]))
+    for a, b in zip(errs_u, errs_u[1:]):
+        assert b < a / 8          # 4 more bits: at least 8x smaller
+    errs_w = []
+    for wb in (4, 8, 12, 16):
+        g = oracle.gen_aux(W, spec.seed, 13, spec.alpha, wb, want_r_star=True)
+        s = g["s"].astype(np.float32)
+        m = oracle.merge_mul(g["codes"], s, g["z"], A, B, spec.seed, 13, g["sigma_w"],
+                             g["sigma_r"], spec.alpha, wb + 12)
+        D = g["codes"].astype(np.int64) - g["z"][:, None]
+        nz = D != 0
+        target = W.astype(np.float64) + AB
+        errs_w.append(np.linalg.norm((m["sbar"][:, None] * m["P"] - target)[nz])
+                      / np.linalg.norm(target[nz]))
+    for a, b in zip(errs_w, errs_w[1:]):
+        assert b < a / 8
+    assert errs_w[-1] < 1e-4
+
+
+# ---------------------------------------------------------------------------
+# a7: IntLoRA_SHIFT
+# ---------------------------------------------------------------------------
+def test_shift_quantizer_worked_examples():
+    g = json.loads((GOLDEN / "shift_quantizer_worked.json").read_text())
+    for case in g["cases"]:
+        q = oracle.shift_quantize_row(case["U"], case["D"], case["bits"])
+        assert q["sbar"] == case["sbar"], case
+        assert q["shift"].tolist() == case["shift"], case
+        assert q["M"].tolist() == case["M"], case
+
+
+def _brute_force_shift(v: Fraction, kmax: int) -> int:
+    """Nearest integer to -log2|v| by exact comparisons of v^2 with the
+    half-integer powers 2^-(2k+1), clamped to [0, kmax]."""
+    if v == 0:
+        return kmax
+    v2 = v * v
+    k = 0
+    while k < kmax and v2 <= Fraction(1, 2 ** (2 * k + 1)):
+        k += 1
+    return k
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_shift_quantizer_brute_force(bits):
+    rng = np.random.default_rng(40 + bits)
+    kmax = 2**bits - 1
+    for _ in range(60):
+        n = int(rng.integers(1, 17))
+        U = rng.standard_normal(n) * np.exp(rng.uniform(-6, 0, n))
+        D = rng.integers(-15, 16, n)
+        if n > 2:
+            U[0] = 0.0
+        q = oracle.shift_quantize_row(U, D, bits)
+        sbar = Fraction(float(np.max(np.abs(U)))) if np.any(U != 0) else Fraction(1)
+        assert Fraction(q["sbar"]) == sbar
+        for u, dv, k, m in zip(U, D, q["shift"], q["M"]):
+            v = Fraction(float(u)) / sbar
+            assert k == _brute_force_shift(v, kmax)
+            sign = (v > 0) - (v < 0)
+            assert m == sign * (int(dv) >> int(k))   # Python >> is a floor shift
+
+
+def test_merge_shift_composition():
+    spec, W, A, B, g = _prepared(10, 24, 8, 4, sid=17)
+    s32 = g["s"].astype(np.float32)
+    m = oracle.merge_shift(g["codes"], s32, g["z"], A, B, spec.seed, 17, g["sigma_w"],
+                           g["sigma_r"], spec.alpha, 4)
+    U, D = oracle.mla_rows(g["codes"], s32, g["z"], A, B, spec.seed, 17, g["sigma_w"],
+                           g["sigma_r"], spec.alpha)
+    for i in range(10):
+        q = oracle.shift_quantize_row(U[i], D[i], 4)
+        assert m["sbar"][i] == q["sbar"]
+        assert m["shift"][i].tolist() == q["shift"].tolist()
+        assert m["M"][i].tolist() == q["M"].tolist()
+    assert np.abs(m["M"]).max() <= 15
+
+
+# ---------------------------------------------------------------------------
+# a8: STE backward
+# ---------------------------------------------------------------------------
+def test_ste_backward_against_numpy():
+    spec = wl.LayerSpec("t", 19, 45, 6, 8, "mul", 8, stream_id=21)
+    Gb = wl.host_G_bits(spec)
+    Ab = wl.to_bf16_bits(wl.host_A(spec))
+    Bb = wl.to_bf16_bits(wl.host_B(spec))
+    G, A, B = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+    dA, dB = oracle.ste_backward(G, A, B)
+    np.testing.assert_allclose(dA, G @ B.T, rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(dB, A.T @ G, rtol=1e-12, atol=1e-18)
+    rows, cols = np.array([0, 5, 18]), np.array([0, 44, 7])
+    sA, sB = oracle.ste_sampled(Gb, Ab, Bb, rows, cols)
+    np.testing.assert_allclose(sA, dA[rows], rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(sB, dB[:, cols], rtol=1e-12, atol=1e-18)

@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the IntLoRA merge hot path on B200.
+
+One step = the whole per-layer path over every layer of the workload:
+layer preparation (Philox/Laplace R, sigma_W and sigma_R, VMC, base
+quantization of W - R*), the merge (MUL for the default workload) and the STE
+backward (dA = G B^T, dB = A^T G), each stage one batched call of the C ABI.
+
+Default workload: 128 SD-v1.5-UNet-shaped linears (16 transformer blocks, 8
+linears each), int4 base codes, rank 4, alpha 1.5, MUL with a 4-bit U
+quantizer, 217,415,680 merged weight elements per step (synthetic inputs drawn
+on the device). Metric: merged weight elements per second (whole job), with the
+dominant kernel's HBM roofline fraction reported beside it.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: one process per GPU under torch.distributed.run; every rank runs its
+own copy of the workload (weak scaling; layers are independent, no collective
+on the data path), timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "merged weight elements/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "elements/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="sd_unet")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_desc(name, layers):
+    from quantized_lora_merge_b200 import workloads as wl
+    l0 = layers[0]
+    total = sum(l.numel for l in layers)
+    return {
+        "workload": f"{name}: {len(layers)} linears, int{l0.w_bits} base codes, r={l0.r}, "
+                    f"alpha={l0.alpha}, {l0.variant.upper()} {l0.out_bits}-bit; prepare + merge "
+                    f"+ STE backward per step",
+        "layers": len(layers),
+        "merged_elements_per_step": total,
+        "l2": "inputs larger than L2 (fp32 W 4 B/elem + bf16 G 2 B/elem per step, "
+              f"{(6 * total) / 1e9:.2f} GB)",
+        "data": "synthetic (seeded device draws, shapes of the named model)",
+    }
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (unit of work: one merged element)
+# ---------------------------------------------------------------------------
+def merge_bytes(l):
+    code = 0.5 if l.w_bits == 4 else 1.0
+    if l.variant == "mul":
+        out = 2 if ((2**l.w_bits - 1) * (2**l.out_bits - 1) <= 32767) else 4
+        per_row = 4 + 4 + 4 + 4           # s, z in; s_bar, z_bar out
+    else:
+        out = 1 if l.w_bits <= 7 else 2
+        per_row = 4 + 4 + 4
+    return l.numel * (code + out) + l.d * per_row + 4 * l.r * (l.d + l.n)
+
+
+def prepare_bytes(l):
+    code = 0.5 if l.w_bits == 4 else 1.0
+    # statistics pass reads W; quantization pass reads W and writes codes, s, z
+    return l.numel * (4 + 4 + code) + l.d * 8
+
+
+def ste_bytes(l):
+    # G read once per contraction (the CUDA-core path reads it twice), A, B, dA, dB
+    return l.numel * 2 + l.r * (l.d + l.n) * (2 + 4)
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def oracle_sample(layers, seconds):
+    """Run the oracle's whole path (prepare, merge, STE) layer by layer in
+    workload order until `seconds` have passed; returns (elements, time)."""
+    import numpy as np
+
+    import oracle
+    from quantized_lora_merge_b200 import workloads as wl
+    done, t_total, names = 0, 0.0, []
+    for spec in layers:
+        W, A, Bm = wl.host_W(spec), wl.host_A(spec), wl.host_B(spec)
+        Gb = wl.host_G_bits(spec)
+        A16, B16 = wl.to_bf16_bits(A), wl.to_bf16_bits(Bm)
+        t0 = time.perf_counter()
+        g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits)
+        s32 = g["s"].astype(np.float32)
+        if spec.variant == "mul":
+            oracle.merge_mul(g["codes"], s32, g["z"], A, Bm, spec.seed, spec.stream_id,
+                             g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits)
+        else:
+            oracle.merge_shift(g["codes"], s32, g["z"], A, Bm, spec.seed, spec.stream_id,
+                               g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits)
+        oracle.ste_backward(wl.bf16_bits_to_f32(Gb).astype(np.float64),
+                            wl.bf16_bits_to_f32(A16).astype(np.float64),
+                            wl.bf16_bits_to_f32(B16).astype(np.float64))
+        t_total += time.perf_counter() - t0
+        done += spec.numel
+        names.append(spec.name)
+        if t_total >= seconds:
+            break
+    return done, t_total, names
+
+
+def cpu_baseline(layers, seconds):
+    import oracle
+    done, t, names = oracle_sample(layers, seconds)
+    return {"value": done / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {len(names)} of {len(layers)} layers in workload order "
+                      f"({done} merged elements, prepare + merge + STE, {t:.1f} s)"}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle as it stands on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args, layers, desc):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    per_step_seconds = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(layers, per_step_seconds)
+    done = t = 0.0
+    names = []
+    for _ in range(args.steps):
+        d, tt, names = oracle_sample(layers, per_step_seconds)
+        done += d
+        t += tt
+    import oracle
+    value = done / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": desc,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: first {len(names)} layers in workload "
+                                       f"order, prepare + merge + STE"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    from quantized_lora_merge_b200 import workloads as wl
+    layers_base = wl.CONFIGS[args.config]()
+    desc = workload_desc(args.config, layers_base)
+    if args.impl == "reference":
+        run_reference(args, layers_base, desc)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    from dataclasses import replace
+
+    from quantized_lora_merge_b200 import build as qbuild
+    from quantized_lora_merge_b200 import pipeline as P
+    qbuild.build()
+    # weak scaling: every rank owns its own copy of the workload (own R streams)
+    layers = [replace(l, stream_id=l.stream_id + 1000 * rank, ste=True) for l in layers_base]
+
+    states = []
+    for spec in layers:
+        t = wl.device_inputs(spec, device, with_grad=True, salt=rank)
+        states.append(P.allocate(spec, t["W"], t["A"], t["B"], device, G=t["G"], A16=t["A16"],
+                                 B16=t["B16"]))
+    path = P.Path(states, device)
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(max(3, args.warmup)):
+        path.step()
+    torch.cuda.synchronize(device)
+
+    # timed region: whole steps, plus per-stage events on the launching stream
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(device)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        path.prepare()
+        ev[k][1].record(stream)
+        path.merge()
+        ev[k][2].record(stream)
+        path.backward()
+        ev[k][3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_end)
+    stage_ms = {name: sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps))
+                / args.steps for i, name in enumerate(["prepare", "merge", "ste_backward"])}
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    elements = sum(l.numel for l in layers) * world
+    value = elements / (ms_step / 1000.0)
+    hbm_peak, peak_kind = peaks()
+
+    per_stage_bytes = {"prepare": sum(prepare_bytes(l) for l in layers),
+                       "merge": sum(merge_bytes(l) for l in layers),
+                       "ste_backward": sum(ste_bytes(l) for l in layers)}
+    stages = {}
+    for name, ms in stage_ms.items():
+        gbs = per_stage_bytes[name] / (ms / 1000.0) / 1e9
+        stages[name] = {"ms": ms, "algorithmic_GB": per_stage_bytes[name] / 1e9,
+                        "GB_s": gbs, "frac_of_hbm": gbs / hbm_peak}
+    stages["merge"]["elements_per_s"] = sum(l.numel for l in layers) / (stage_ms["merge"] / 1e3)
+    dominant = max(stage_ms, key=stage_ms.get)
+    roof_gbs = per_stage_bytes[dominant] / (stage_ms[dominant] / 1000.0) / 1e9
+    launches_per_step = {"prepare": 3, "merge": 1, "ste_backward": 4}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": desc,
+        "hbm_GB_s_merge": stages["merge"]["GB_s"],
+        "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": roof_gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": roof_gbs / hbm_peak,
+                     "peak_source": peak_kind, "traffic": None},
+        "stages": stages,
+        "clocks": clk,
+        "gpu_launches": args.steps * sum(launches_per_step.values()),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e(path, states, device, stream, max(2, min(args.steps, 5)), world,
+                          elements)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def e2e(path, states, device, stream, steps, world, elements):
+    """Same step through the public API with HOST buffers: every step copies
+    the step's inputs from pinned host memory, runs the path and reads the
+    merged weights, scales and gradients back."""
+    import torch
+    import torch.distributed as dist
+    host_in, host_out = [], []
+    for st in states:
+        hi = {k: torch.empty(getattr(st, k).shape, dtype=getattr(st, k).dtype, pin_memory=True)
+              for k in ("W", "A", "B", "G", "A16", "B16")}
+        for k, v in hi.items():
+            v.copy_(getattr(st, k))
+        ho = {k: torch.empty(getattr(st, k).shape, dtype=getattr(st, k).dtype, pin_memory=True)
+              for k in ("out", "sbar", "zbar", "dA", "dB")}
+        host_in.append(hi)
+        host_out.append(ho)
+    h2d = sum(v.numel() * v.element_size() for hi in host_in for v in hi.values())
+    d2h = sum(v.numel() * v.element_size() for ho in host_out for v in ho.values())
+
+    def one():
+        for st, hi in zip(states, host_in):
+            for k, v in hi.items():
+                getattr(st, k).copy_(v, non_blocking=True)
+        path.step()
+        for st, ho in zip(states, host_out):
+            for k, v in ho.items():
+                v.copy_(getattr(st, k), non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": elements / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,243 @@
+/*
+ * intlora.h - C ABI of the IntLoRA integer low-rank merge library (B200, sm_100a).
+ *
+ * IntLoRA adapts a quantized linear layer with integer-type low-rank factors
+ * so that the merged weight comes out already quantized, with no post-training
+ * quantization step. This library implements the per-layer hot path of that
+ * method on the GPU:
+ *
+ *   - intlora_gen_aux       auxiliary matrix R (seeded Philox4x32-10 Laplace
+ *                           noise, never stored), its variance-matched copy
+ *                           R* = (sigma_W / sigma_R)^alpha * R, and the base
+ *                           quantization W_round, s, z of W - R*;
+ *   - intlora_merge_mul     IntLoRA_MUL: the adaptation term
+ *                           U = s + (R* + A B) / (W_round - z) quantized per row
+ *                           by a uniform affine quantizer, merged by an integer
+ *                           Hadamard product;
+ *   - intlora_merge_shift   IntLoRA_SHIFT: U quantized by a log2 quantizer,
+ *                           merged by arithmetic shifts;
+ *   - intlora_ste_backward  straight-through backward dA = G B^T, dB = A^T G.
+ *
+ * Sources, cited by page title and section:
+ *   [notes]   "IntLoRA: Integral Low-rank Adaptation of Quantized Diffusion
+ *             Models", Paper-Notes page (ICML2025), section 方法详解:
+ *             1. AQS (W' = Q[W - sg(R)] + sg(R) + AB; R regenerated online from
+ *             a fixed seed and distribution statistics, no storage),
+ *             2. MLA (W' = [s + (R + AB) / (W_round - z)] (.) (W_round - z)),
+ *             3. VMC (R* = r^alpha R, r = sigma_W / sigma_R),
+ *             两种实现版本 (IntLoRA_MUL: W' = s_bar (U_round - z_bar) (.)
+ *             (W_round - z); IntLoRA_SHIFT: W' = sign(V) (.) [(W_round - z) >>
+ *             shift]; training through the quantizers with the STE).
+ *   [summary] atlas.scime.ai summary of the same paper, "Measured effects":
+ *             Laplace is the auxiliary distribution.
+ *   [Philox]  Salmon et al., SC'11, Philox4x32-10.
+ *
+ * Conventions (fixed here where the pages are silent):
+ *   - Layer W is d x n, row-major: d output channels (rows i), n inputs
+ *     (columns j). Flat index e = i * n + j. A is d x r, B is r x n, both
+ *     dense row-major (leading dimensions r and n).
+ *   - W_round codes are unsigned: 8-bit codes one per byte; 4-bit codes two per
+ *     byte, even column in the low nibble. Row i starts at byte i * ld_w.
+ *   - R_ij = Laplace(0,1) from word (e mod 4) of Philox4x32-10 with key
+ *     (seed low 32 bits, seed high 32 bits) and counter (e/4 low, e/4 high,
+ *     stream_id, 0). u = (2 (x >> 9) + 1) 2^-24, v = u - 1/2,
+ *     R = -sign(v) ln(1 - 2|v|).
+ *   - sigma_W, sigma_R are population standard deviations over the whole
+ *     d x n layer. c = (sigma_W / sigma_R)^alpha is formed in fp64.
+ *   - Affine quantizer of a row x (b bits): range [min(0, min x), max(0, max x)],
+ *     scale = range / (2^b - 1) (a row whose range is {0} gets scale 1, zero 0),
+ *     zero = clamp(rne(-min / scale), 0, 2^b - 1),
+ *     code = clamp(rne(x / scale) + zero, 0, 2^b - 1); rne = round to nearest,
+ *     ties to even.
+ *   - D_ij = W_round_ij - z_i. Where D_ij = 0 the quotient term of U is 0.
+ *   - SHIFT: s_bar_i = max_j |U_ij|, V = U / s_bar, shift = nearest integer
+ *     of -log2|V| clamped to [0, 2^shift_bits - 1], M = sign(V) (D >> shift)
+ *     with an arithmetic (floor) shift. The merged weight is s_bar_i M_ij.
+ *   - MUL: the merged weight is s_bar_i P_ij with P = (U_round - z_bar) D.
+ *   - GPU arithmetic is fp32 (fp64 for the sigma reductions and c). A code
+ *     may differ by one from an fp64 evaluation only where the fp64 pre-round
+ *     value lies within ~1e-5 relative of a rounding boundary.
+ *
+ * Ownership and execution:
+ *   - Every data pointer is a DEVICE pointer (or managed memory) on the
+ *     current device, allocated and owned by the caller. sigma scalars are
+ *     device doubles. The library keeps no state between calls and allocates
+ *     nothing; scratch space is the caller's workspace (ws, ws_bytes), whose
+ *     required size the *_workspace_size queries return.
+ *   - Every call validates its arguments on the host and returns a status
+ *     before launching anything. Work is then enqueued asynchronously on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream). A launch
+ *     failure returns INTLORA_ERR_CUDA. No call synchronizes the device.
+ *   - Outputs must not alias inputs. Calls on different streams that share a
+ *     workspace race.
+ *   - intlora_last_error() returns a thread-local description of the most
+ *     recent failure in the calling thread.
+ */
+#ifndef INTLORA_H
+#define INTLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum intlora_status {
+    INTLORA_OK = 0,
+    INTLORA_ERR_INVALID_ARG = 1,  /* bad pointer, size, bit width, alignment */
+    INTLORA_ERR_UNSUPPORTED = 2,  /* valid but outside what this build handles */
+    INTLORA_ERR_WORKSPACE = 3,    /* ws NULL or ws_bytes below the query's value */
+    INTLORA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    INTLORA_ERR_TIMEOUT = 5       /* a bounded device wait gave up */
+} intlora_status;
+
+/* Static description of a status code. */
+const char* intlora_status_string(int status);
+/* Thread-local message of the last failure in this thread ("" if none). */
+const char* intlora_last_error(void);
+/* Library version, major * 10000 + minor * 100 + patch. */
+int intlora_version(void);
+
+/* Limits of this build. */
+#define INTLORA_MAX_RANK 256
+#define INTLORA_MAX_BATCH 128     /* descriptors per batched call */
+
+/* --------------------------------------------------------------------------
+ * Layer preparation [notes, AQS and VMC].
+ *
+ * From the fp32 weight W (d x n, dense row-major) computes, for one layer:
+ *   sigma_w_out  = std(W), sigma_r_out = std(R)            (device doubles)
+ *   r_star_out   = R* = c R            (optional, fp32 d x n dense; may be NULL)
+ *   w_round_out  = codes of W - R*     (optional; w_bits 4 or 8, row stride
+ *                                       ld_w_out bytes; may be NULL)
+ *   s_out, z_out = per-row scale (fp32) and zero-point (int32) of W - R*
+ *                  (required when w_round_out is given, else may be NULL)
+ * alpha >= 0. With alpha = 0 (c = 1) r_star_out is R itself.
+ * Requirements: d, n >= 1; d * n < 2^40; w_bits in {4, 8}; n even when
+ * w_bits = 4; ld_w_out >= n * w_bits / 8; W, w_round_out, r_star_out 16-byte
+ * aligned; ws of at least intlora_gen_aux_workspace_size bytes, 256-byte
+ * aligned.
+ * ------------------------------------------------------------------------ */
+typedef struct intlora_aux_job {
+    const float* W;
+    int64_t d, n;
+    uint64_t seed;
+    uint32_t stream_id;
+    float alpha;
+    int32_t w_bits;
+    double* sigma_w_out;
+    double* sigma_r_out;
+    float* r_star_out;
+    void* w_round_out;
+    int64_t ld_w_out;
+    float* s_out;
+    int32_t* z_out;
+} intlora_aux_job;
+
+size_t intlora_gen_aux_workspace_size(const intlora_aux_job* jobs, int32_t count);
+
+intlora_status intlora_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed,
+                               uint32_t stream_id, float alpha, int32_t w_bits,
+                               double* sigma_w_out, double* sigma_r_out, float* r_star_out,
+                               void* w_round_out, int64_t ld_w_out, float* s_out,
+                               int32_t* z_out, void* ws, size_t ws_bytes, void* stream);
+
+/* `count` jobs (a host array) in three launches in total. */
+intlora_status intlora_gen_aux_batched(const intlora_aux_job* jobs, int32_t count, void* ws,
+                                       size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * Merges [notes, MLA and 两种实现版本].
+ *
+ * One quantized layer with its LoRA factors. All pointers are device pointers.
+ * sigma_w is required (from intlora_gen_aux); sigma_r may be NULL, in which
+ * case the call regenerates R once more to reduce it on the device (this
+ * needs workspace). r in [1, INTLORA_MAX_RANK].
+ * ------------------------------------------------------------------------ */
+typedef struct intlora_layer {
+    int64_t d, n;
+    int32_t r;
+    int32_t w_bits;             /* 4 (packed nibbles) or 8 */
+    const void* w_round;        /* 16-byte aligned; row i at byte i * ld_w */
+    int64_t ld_w;               /* bytes per row, >= n * w_bits / 8 */
+    const float* s;             /* [d] base scales */
+    const int32_t* z;           /* [d] base zero-points, in [0, 2^w_bits - 1] */
+    const float* A;             /* d x r fp32 */
+    const float* B;             /* r x n fp32 */
+    uint64_t seed;              /* Philox key of R */
+    uint32_t stream_id;         /* Philox counter word 2 */
+    float alpha;                /* VMC exponent */
+    const double* sigma_w;      /* device scalar */
+    const double* sigma_r;      /* device scalar or NULL */
+} intlora_layer;
+
+/* Outputs of one merge.
+ *   out:  MUL: P = (U_round - z_bar) D, int16 when
+ *         (2^w_bits - 1)(2^u_bits - 1) <= 32767, else int32, d x n dense;
+ *         SHIFT: M = sign(V) (D >> shift), int8 when w_bits <= 7, else int16.
+ *   sbar: [d] fp32 per-row scale of the merged weight (W' = sbar_i * out_ij).
+ *   zbar: [d] int32 MUL zero-point of U (ignored by SHIFT, may be NULL there).
+ *   code: optional uint8 d x n: MUL U_round, SHIFT shift; may be NULL.
+ * out and code must be 16-byte aligned. */
+typedef struct intlora_merge_out {
+    void* out;
+    float* sbar;
+    int32_t* zbar;
+    uint8_t* code;
+} intlora_merge_out;
+
+/* Bytes per element of `out`: MUL (variant 0) or SHIFT (variant 1). */
+int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits);
+
+size_t intlora_merge_workspace_size(const intlora_layer* layers, int32_t count);
+
+/* IntLoRA_MUL, u_bits in [2, 8]. */
+intlora_status intlora_merge_mul(const intlora_layer* layer, int32_t u_bits, void* prod_out,
+                                 float* sbar_out, int32_t* zbar_out, uint8_t* u_round_out,
+                                 void* ws, size_t ws_bytes, void* stream);
+/* IntLoRA_SHIFT, shift_bits in [1, 5] (shift codes 0 .. 2^shift_bits - 1). */
+intlora_status intlora_merge_shift(const intlora_layer* layer, int32_t shift_bits, void* m_out,
+                                   float* sbar_out, uint8_t* shift_out, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* `count` layers (host arrays `layers` and `outs`) in one grouped launch. */
+intlora_status intlora_merge_mul_batched(const intlora_layer* layers,
+                                         const intlora_merge_out* outs, int32_t count,
+                                         int32_t u_bits, void* ws, size_t ws_bytes,
+                                         void* stream);
+intlora_status intlora_merge_shift_batched(const intlora_layer* layers,
+                                           const intlora_merge_out* outs, int32_t count,
+                                           int32_t shift_bits, void* ws, size_t ws_bytes,
+                                           void* stream);
+
+/* --------------------------------------------------------------------------
+ * STE backward [notes, 两种实现版本: training through the quantizers with the
+ * straight-through estimator]. With G the upstream gradient on W' (d x n),
+ *   dA = G B^T   (d x r, fp32),     dB = A^T G   (r x n, fp32).
+ * G, A, B are bf16 (raw 16-bit patterns), dense row-major, 16-byte aligned;
+ * accumulation is fp32. dA and dB are overwritten.
+ * ------------------------------------------------------------------------ */
+typedef struct intlora_ste_job {
+    const void* G;
+    const void* A;
+    const void* B;
+    int64_t d, n;
+    int32_t r;
+    float* dA;
+    float* dB;
+} intlora_ste_job;
+
+size_t intlora_ste_workspace_size(const intlora_ste_job* jobs, int32_t count);
+
+intlora_status intlora_ste_backward(const void* G, const void* A, const void* B, int64_t d,
+                                    int64_t n, int32_t r, float* dA, float* dB, void* ws,
+                                    size_t ws_bytes, void* stream);
+intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t count,
+                                            void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INTLORA_H */

@@ -1,0 +1,605 @@
+// C ABI of the IntLoRA merge library: host-side validation, launch geometry
+// and kernel launches. Every entry point validates all of its arguments before
+// enqueuing anything, never synchronizes, and never allocates: scratch space is
+// the caller's workspace. See include/intlora.h for the contract.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "intlora.h"
+#include "intlora_kernels.h"
+
+using namespace intlora;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+intlora_status fail(intlora_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+intlora_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(INTLORA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+constexpr int64_t kMaxElements = int64_t{1} << 40;
+constexpr int kStatsThreadsHost = 256;
+constexpr int kStatsGroupsPerThread = 8;
+constexpr int kStatsMaxBlocksPerJob = 148 * 8;
+
+int64_t stats_blocks(int64_t numel) {
+  const int64_t groups = ceil_div(numel, 4);
+  return std::min<int64_t>(kStatsMaxBlocksPerJob,
+                           std::max<int64_t>(1, ceil_div(groups, kStatsThreadsHost * kStatsGroupsPerThread)));
+}
+size_t stats_partial_bytes(int64_t numel) { return round256(static_cast<size_t>(stats_blocks(numel)) * 4 * sizeof(double)); }
+
+// ------------------------------------------------------------------------
+// tile geometry: cluster size, column slice, rows per tile
+// ------------------------------------------------------------------------
+struct Geometry {
+  int cluster = 1;
+  int num_clusters = 0;
+};
+
+int max_active_clusters_cached(int variant, int w_bits, int rank_ct, int cluster) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, cluster);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int v = tile_max_active_clusters(variant, w_bits, rank_ct, cluster);
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = v;
+  return v;
+}
+
+int slice_cols(int64_t n, int cluster) { return static_cast<int>(ceil_div(ceil_div(n, cluster), 4) * 4); }
+
+// Fill n_c, m, b_resident, kc, aligned and tile_begin of every layer for a
+// cluster size; returns the total number of tiles or -1 if a slice is too wide.
+int64_t plan_layers(int variant, std::vector<TileLayer>& L, int cluster, bool* all_resident) {
+  int64_t tiles = 0;
+  bool resident = true;
+  for (auto& l : L) {
+    const int n_c = slice_cols(l.n, cluster);
+    const int quads = n_c / 4;
+    if (quads > kMaxQuads) return -1;
+    int groups = std::max(1, kMaxQuads / quads);
+    int m = kRowsPerItem * groups;
+    m = std::min(m, kMaxTileRows);
+    if (variant != kGen) {
+      const int a_rows = (kASmemFloats / std::max(1, l.r)) / kRowsPerItem * kRowsPerItem;
+      m = std::min(m, std::max(kRowsPerItem, a_rows));
+      l.b_resident = static_cast<int64_t>(l.r) * n_c <= kBSmemFloats ? 1 : 0;
+      l.kc = std::max(1, kBSmemFloats / n_c);
+      resident = resident && l.b_resident;
+    } else {
+      l.b_resident = 0;
+      l.kc = 0;
+    }
+    // do not make tiles much taller than the layer
+    m = std::min<int64_t>(m, ceil_div(l.d, kRowsPerItem) * kRowsPerItem);
+    l.n_c = n_c;
+    l.m = m;
+    l.aligned = (l.n % 4 == 0) ? 1 : 0;
+    l.tile_begin = tiles;
+    tiles += ceil_div(l.d, m);
+  }
+  if (all_resident) *all_resident = resident;
+  return tiles;
+}
+
+intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bits, int w_bits,
+                                 int out_bytes, cudaStream_t stream) {
+  int rank_ct = 0;
+  if (variant != kGen) {
+    rank_ct = L[0].r;
+    for (auto& l : L)
+      if (l.r != rank_ct) rank_ct = 0;
+    if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16 && rank_ct != 32) rank_ct = 0;
+  }
+  static const int kClusters[] = {1, 2, 4, 8, 16};
+  int chosen = -1;
+  int64_t total = -1;
+  // smallest cluster whose slices fit and keep B resident; else smallest that fits
+  for (int pass = 0; pass < 2 && chosen < 0; ++pass) {
+    for (int c : kClusters) {
+      bool resident = false;
+      const int64_t t = plan_layers(variant, L, c, &resident);
+      if (t < 0) continue;
+      if (pass == 0 && variant != kGen && !resident) continue;
+      if (max_active_clusters_cached(variant, w_bits, rank_ct, c) <= 0) continue;
+      chosen = c;
+      total = t;
+      break;
+    }
+  }
+  if (chosen < 0) return fail(INTLORA_ERR_UNSUPPORTED, "no launchable cluster size for this batch");
+  total = plan_layers(variant, L, chosen, nullptr);
+  TileBatch b;
+  std::memset(&b, 0, sizeof b);
+  for (size_t k = 0; k < L.size(); ++k) b.layer[k] = L[k];
+  b.count = static_cast<int32_t>(L.size());
+  b.cluster = chosen;
+  b.total_tiles = total;
+  b.num_clusters = static_cast<int32_t>(
+      std::min<int64_t>(total, max_active_clusters_cached(variant, w_bits, rank_ct, chosen)));
+  b.bits = bits;
+  b.w_bits = w_bits;
+  b.out_bytes = out_bytes;
+  cudaError_t e = launch_tiles(variant, b, rank_ct, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "row-tile kernel launch");
+  return INTLORA_OK;
+}
+
+uint32_t lo32(uint64_t v) { return static_cast<uint32_t>(v); }
+uint32_t hi32(uint64_t v) { return static_cast<uint32_t>(v >> 32); }
+
+// ------------------------------------------------------------------------
+// gen_aux
+// ------------------------------------------------------------------------
+intlora_status check_aux_job(const intlora_aux_job& j, int idx) {
+  if (j.W == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "job %d: W is NULL", idx);
+  if (j.d < 1 || j.n < 1) return fail(INTLORA_ERR_INVALID_ARG, "job %d: d and n must be >= 1", idx);
+  if (j.d > kMaxElements / j.n) return fail(INTLORA_ERR_INVALID_ARG, "job %d: d*n exceeds 2^40", idx);
+  if (j.w_bits != 4 && j.w_bits != 8)
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: w_bits must be 4 or 8", idx);
+  if (j.w_bits == 4 && (j.n % 2) != 0)
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: n must be even for 4-bit codes", idx);
+  if (!(j.alpha >= 0.0f) || !std::isfinite(j.alpha))
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: alpha must be finite and >= 0", idx);
+  if (j.sigma_w_out == nullptr || j.sigma_r_out == nullptr)
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: sigma outputs are required", idx);
+  if (!aligned16(j.W)) return fail(INTLORA_ERR_INVALID_ARG, "job %d: W must be 16-byte aligned", idx);
+  if (j.r_star_out != nullptr && !aligned16(j.r_star_out))
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: r_star_out must be 16-byte aligned", idx);
+  if (j.w_round_out != nullptr) {
+    const int64_t need = j.w_bits == 8 ? j.n : j.n / 2;
+    if (j.ld_w_out < need || j.ld_w_out % 16 != 0)
+      return fail(INTLORA_ERR_INVALID_ARG,
+                  "job %d: ld_w_out must be >= %lld bytes and a multiple of 16", idx,
+                  static_cast<long long>(need));
+    if (!aligned16(j.w_round_out))
+      return fail(INTLORA_ERR_INVALID_ARG, "job %d: w_round_out must be 16-byte aligned", idx);
+    if (j.s_out == nullptr || j.z_out == nullptr)
+      return fail(INTLORA_ERR_INVALID_ARG, "job %d: s_out and z_out are required with w_round_out", idx);
+  }
+  return INTLORA_OK;
+}
+
+size_t aux_ws_bytes(const intlora_aux_job* jobs, int32_t count) {
+  size_t total = 0;
+  for (int32_t k = 0; k < count; ++k) total += stats_partial_bytes(jobs[k].d * jobs[k].n);
+  return total;
+}
+
+// The three launches of one chunk of at most kMaxBatch jobs.
+intlora_status gen_aux_chunk(const intlora_aux_job* jobs, int32_t count, char* ws, cudaStream_t st) {
+  StatsBatch sb;
+  std::memset(&sb, 0, sizeof sb);
+  int64_t blocks = 0;
+  size_t off = 0;
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_aux_job& j = jobs[k];
+    StatsJob& s = sb.job[k];
+    s.W = j.W;
+    s.numel = j.d * j.n;
+    s.key0 = lo32(j.seed);
+    s.key1 = hi32(j.seed);
+    s.stream_id = j.stream_id;
+    s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
+    s.block_begin = blocks;
+    s.partial = reinterpret_cast<double*>(ws + off);
+    s.sigma_w_out = j.sigma_w_out;
+    s.sigma_r_out = j.sigma_r_out;
+    blocks += s.nblocks;
+    off += stats_partial_bytes(s.numel);
+  }
+  sb.count = count;
+  cudaError_t e = launch_stats(sb, blocks, st);
+  if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
+  e = launch_stats_finalize(sb, st);
+  if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
+
+  // base quantization for the jobs that want codes or R*, grouped by w_bits
+  for (int wb : {4, 8}) {
+    std::vector<TileLayer> L;
+    for (int32_t k = 0; k < count; ++k) {
+      const intlora_aux_job& j = jobs[k];
+      if (j.w_bits != wb || (j.w_round_out == nullptr && j.r_star_out == nullptr)) continue;
+      TileLayer l;
+      std::memset(&l, 0, sizeof l);
+      l.src = j.W;
+      l.ld_src = j.n * 4;
+      l.sigma_w = j.sigma_w_out;
+      l.sigma_r = j.sigma_r_out;
+      l.alpha = j.alpha;
+      l.key0 = lo32(j.seed);
+      l.key1 = hi32(j.seed);
+      l.stream_id = j.stream_id;
+      l.out = j.w_round_out;
+      l.ld_out = j.ld_w_out;
+      l.scale_out = j.s_out;
+      l.zero_out = j.z_out;
+      l.r_star_out = j.r_star_out;
+      l.d = j.d;
+      l.n = j.n;
+      L.push_back(l);
+    }
+    if (L.empty()) continue;
+    const intlora_status s = launch_tile_batch(kGen, L, wb, wb, 1, st);
+    if (s != INTLORA_OK) return s;
+  }
+  return INTLORA_OK;
+}
+
+// ------------------------------------------------------------------------
+// merges
+// ------------------------------------------------------------------------
+intlora_status check_layer(const intlora_layer* l, int idx) {
+  if (l == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "layer %d is NULL", idx);
+  if (l->d < 1 || l->n < 1) return fail(INTLORA_ERR_INVALID_ARG, "layer %d: d and n must be >= 1", idx);
+  if (l->d > kMaxElements / l->n) return fail(INTLORA_ERR_INVALID_ARG, "layer %d: d*n exceeds 2^40", idx);
+  if (l->r < 1 || l->r > INTLORA_MAX_RANK)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: r must be in [1, %d]", idx, INTLORA_MAX_RANK);
+  if (l->w_bits != 4 && l->w_bits != 8)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: w_bits must be 4 or 8", idx);
+  if (l->w_bits == 4 && (l->n % 2) != 0)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: n must be even for 4-bit codes", idx);
+  if (l->w_round == nullptr || l->s == nullptr || l->z == nullptr || l->A == nullptr ||
+      l->B == nullptr || l->sigma_w == nullptr)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: w_round, s, z, A, B and sigma_w are required", idx);
+  const int64_t need = l->w_bits == 8 ? l->n : l->n / 2;
+  if (l->ld_w < need || l->ld_w % 16 != 0)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: ld_w must be >= %lld bytes and a multiple of 16",
+                idx, static_cast<long long>(need));
+  if (!aligned16(l->w_round)) return fail(INTLORA_ERR_INVALID_ARG, "layer %d: w_round must be 16-byte aligned", idx);
+  if (!(l->alpha >= 0.0f) || !std::isfinite(l->alpha))
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: alpha must be finite and >= 0", idx);
+  return INTLORA_OK;
+}
+
+intlora_status check_out(const intlora_merge_out* o, bool mul, int idx) {
+  if (o == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "output %d is NULL", idx);
+  if (o->out == nullptr || o->sbar == nullptr)
+    return fail(INTLORA_ERR_INVALID_ARG, "output %d: out and sbar are required", idx);
+  if (mul && o->zbar == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "output %d: zbar is required for MUL", idx);
+  if (!aligned16(o->out) || (o->code != nullptr && !aligned16(o->code)))
+    return fail(INTLORA_ERR_INVALID_ARG, "output %d: out and code must be 16-byte aligned", idx);
+  return INTLORA_OK;
+}
+
+size_t merge_ws_bytes(const intlora_layer* layers, int32_t count) {
+  size_t total = 0;
+  for (int32_t k = 0; k < count; ++k) {
+    if (layers[k].sigma_r != nullptr) continue;
+    total += 256 + stats_partial_bytes(layers[k].d * layers[k].n);
+  }
+  return total;
+}
+
+int32_t out_bytes_for(int variant, int w_bits, int out_bits) {
+  if (variant == 0) {
+    const int64_t bound = ((int64_t{1} << w_bits) - 1) * ((int64_t{1} << out_bits) - 1);
+    return bound <= 32767 ? 2 : 4;
+  }
+  return w_bits <= 7 ? 1 : 2;
+}
+
+intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlora_merge_out* outs,
+                           int32_t count, int32_t bits, char* ws, cudaStream_t st) {
+  // sigma_R on the device for layers that did not pass it in
+  StatsBatch sb;
+  std::memset(&sb, 0, sizeof sb);
+  int32_t ns = 0;
+  int64_t blocks = 0;
+  size_t off = 0;
+  std::vector<const double*> sig_r(count);
+  for (int32_t k = 0; k < count; ++k) {
+    sig_r[k] = layers[k].sigma_r;
+    if (layers[k].sigma_r != nullptr) continue;
+    StatsJob& s = sb.job[ns++];
+    s.W = nullptr;
+    s.numel = layers[k].d * layers[k].n;
+    s.key0 = lo32(layers[k].seed);
+    s.key1 = hi32(layers[k].seed);
+    s.stream_id = layers[k].stream_id;
+    s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
+    s.block_begin = blocks;
+    s.sigma_w_out = nullptr;
+    s.sigma_r_out = reinterpret_cast<double*>(ws + off);
+    s.partial = reinterpret_cast<double*>(ws + off + 256);
+    sig_r[k] = s.sigma_r_out;
+    blocks += s.nblocks;
+    off += 256 + stats_partial_bytes(s.numel);
+  }
+  if (ns > 0) {
+    sb.count = ns;
+    cudaError_t e = launch_stats(sb, blocks, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
+    e = launch_stats_finalize(sb, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
+  }
+  for (int wb : {4, 8}) {
+    std::vector<TileLayer> L;
+    for (int32_t k = 0; k < count; ++k) {
+      const intlora_layer& y = layers[k];
+      if (y.w_bits != wb) continue;
+      TileLayer l;
+      std::memset(&l, 0, sizeof l);
+      l.src = y.w_round;
+      l.ld_src = y.ld_w;
+      l.s = y.s;
+      l.z = y.z;
+      l.A = y.A;
+      l.B = y.B;
+      l.sigma_w = y.sigma_w;
+      l.sigma_r = sig_r[k];
+      l.alpha = y.alpha;
+      l.key0 = lo32(y.seed);
+      l.key1 = hi32(y.seed);
+      l.stream_id = y.stream_id;
+      l.out = outs[k].out;
+      l.ld_out = y.n;
+      l.scale_out = outs[k].sbar;
+      l.zero_out = variant == kMul ? outs[k].zbar : nullptr;
+      l.code_out = outs[k].code;
+      l.d = y.d;
+      l.n = y.n;
+      l.r = y.r;
+      L.push_back(l);
+    }
+    if (L.empty()) continue;
+    const intlora_status s = launch_tile_batch(variant, L, bits, wb,
+                                               out_bytes_for(variant == kMul ? 0 : 1, wb, bits), st);
+    if (s != INTLORA_OK) return s;
+  }
+  return INTLORA_OK;
+}
+
+intlora_status merge_batched(int variant, const intlora_layer* layers, const intlora_merge_out* outs,
+                             int32_t count, int32_t bits, void* ws, size_t ws_bytes, void* stream) {
+  if (count < 0 || (count > 0 && (layers == nullptr || outs == nullptr)))
+    return fail(INTLORA_ERR_INVALID_ARG, "layers/outs must be non-NULL arrays, count >= 0");
+  if (variant == kMul && (bits < 2 || bits > 8))
+    return fail(INTLORA_ERR_INVALID_ARG, "u_bits must be in [2, 8]");
+  if (variant == kShift && (bits < 1 || bits > 5))
+    return fail(INTLORA_ERR_INVALID_ARG, "shift_bits must be in [1, 5]");
+  for (int32_t k = 0; k < count; ++k) {
+    intlora_status s = check_layer(&layers[k], k);
+    if (s != INTLORA_OK) return s;
+    s = check_out(&outs[k], variant == kMul, k);
+    if (s != INTLORA_OK) return s;
+  }
+  const size_t need = merge_ws_bytes(layers, count);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(INTLORA_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+  char* w = static_cast<char*>(ws);
+  for (int32_t k0 = 0; k0 < count; k0 += kMaxBatch) {
+    const int32_t c = std::min<int32_t>(kMaxBatch, count - k0);
+    const intlora_status s = merge_chunk(variant, layers + k0, outs + k0, c, bits, w,
+                                         static_cast<cudaStream_t>(stream));
+    if (s != INTLORA_OK) return s;
+    w += merge_ws_bytes(layers + k0, c);
+  }
+  return INTLORA_OK;
+}
+
+// ------------------------------------------------------------------------
+// STE
+// ------------------------------------------------------------------------
+intlora_status check_ste(const intlora_ste_job& j, int idx) {
+  if (j.G == nullptr || j.A == nullptr || j.B == nullptr || j.dA == nullptr || j.dB == nullptr)
+    return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: G, A, B, dA, dB are required", idx);
+  if (j.d < 1 || j.n < 1) return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: d and n must be >= 1", idx);
+  if (j.d > kMaxElements / j.n) return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: d*n exceeds 2^40", idx);
+  if (j.r < 1 || j.r > INTLORA_MAX_RANK)
+    return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: r must be in [1, %d]", idx, INTLORA_MAX_RANK);
+  if (!aligned16(j.G) || !aligned16(j.A) || !aligned16(j.B))
+    return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: G, A, B must be 16-byte aligned", idx);
+  return INTLORA_OK;
+}
+
+constexpr int kSteBM = 64, kSteRB = 32, kSteTargetCtas = 148 * 4;
+
+intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_t st) {
+  for (int dir = 0; dir < 2; ++dir) {
+    SteBatch b;
+    std::memset(&b, 0, sizeof b);
+    int64_t tiles = 0;
+    for (int32_t k = 0; k < count; ++k) {
+      const intlora_ste_job& j = jobs[k];
+      SteJob& s = b.job[k];
+      s.G = static_cast<const uint16_t*>(j.G);
+      s.A = static_cast<const uint16_t*>(j.A);
+      s.B = static_cast<const uint16_t*>(j.B);
+      s.d = j.d;
+      s.n = j.n;
+      s.r = j.r;
+      s.dA = j.dA;
+      s.dB = j.dB;
+      const int64_t M = dir ? j.n : j.d, K = dir ? j.d : j.n;
+      const int64_t base = ceil_div(M, kSteBM) * ceil_div(j.r, kSteRB);
+      int64_t ks = std::max<int64_t>(1, ceil_div(kSteTargetCtas, base));
+      ks = std::min<int64_t>(ks, std::max<int64_t>(1, ceil_div(K, 512)));
+      s.ksplit = static_cast<int32_t>(ks);
+      s.tile_begin = tiles;
+      tiles += base * ks;
+    }
+    b.count = count;
+    b.transposed = dir;
+    b.total_tiles = tiles;
+    cudaError_t e = launch_ste(b, st);
+    if (e != cudaSuccess) return cuda_fail(e, "STE kernel launch");
+  }
+  return INTLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* intlora_status_string(int status) {
+  switch (status) {
+    case INTLORA_OK: return "ok";
+    case INTLORA_ERR_INVALID_ARG: return "invalid argument";
+    case INTLORA_ERR_UNSUPPORTED: return "unsupported";
+    case INTLORA_ERR_WORKSPACE: return "workspace missing or too small";
+    case INTLORA_ERR_CUDA: return "CUDA error";
+    case INTLORA_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* intlora_last_error(void) { return g_last_error; }
+
+int intlora_version(void) { return 100; }
+
+int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits) {
+  if ((variant != 0 && variant != 1) || (w_bits != 4 && w_bits != 8)) return 0;
+  return out_bytes_for(variant, w_bits, out_bits);
+}
+
+size_t intlora_gen_aux_workspace_size(const intlora_aux_job* jobs, int32_t count) {
+  if (jobs == nullptr || count <= 0) return 0;
+  return aux_ws_bytes(jobs, count);
+}
+
+intlora_status intlora_gen_aux_batched(const intlora_aux_job* jobs, int32_t count, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_status s = check_aux_job(jobs[k], k);
+    if (s != INTLORA_OK) return s;
+  }
+  const size_t need = aux_ws_bytes(jobs, count);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
+    return fail(INTLORA_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+  char* w = static_cast<char*>(ws);
+  for (int32_t k0 = 0; k0 < count; k0 += kMaxBatch) {
+    const int32_t c = std::min<int32_t>(kMaxBatch, count - k0);
+    const intlora_status s = gen_aux_chunk(jobs + k0, c, w, static_cast<cudaStream_t>(stream));
+    if (s != INTLORA_OK) return s;
+    w += aux_ws_bytes(jobs + k0, c);
+  }
+  return INTLORA_OK;
+}
+
+intlora_status intlora_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t stream_id,
+                               float alpha, int32_t w_bits, double* sigma_w_out, double* sigma_r_out,
+                               float* r_star_out, void* w_round_out, int64_t ld_w_out, float* s_out,
+                               int32_t* z_out, void* ws, size_t ws_bytes, void* stream) {
+  intlora_aux_job j;
+  j.W = W;
+  j.d = d;
+  j.n = n;
+  j.seed = seed;
+  j.stream_id = stream_id;
+  j.alpha = alpha;
+  j.w_bits = w_bits;
+  j.sigma_w_out = sigma_w_out;
+  j.sigma_r_out = sigma_r_out;
+  j.r_star_out = r_star_out;
+  j.w_round_out = w_round_out;
+  j.ld_w_out = ld_w_out;
+  j.s_out = s_out;
+  j.z_out = z_out;
+  return intlora_gen_aux_batched(&j, 1, ws, ws_bytes, stream);
+}
+
+size_t intlora_merge_workspace_size(const intlora_layer* layers, int32_t count) {
+  if (layers == nullptr || count <= 0) return 0;
+  return merge_ws_bytes(layers, count);
+}
+
+intlora_status intlora_merge_mul_batched(const intlora_layer* layers, const intlora_merge_out* outs,
+                                         int32_t count, int32_t u_bits, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  g_last_error[0] = '\0';
+  return merge_batched(kMul, layers, outs, count, u_bits, ws, ws_bytes, stream);
+}
+
+intlora_status intlora_merge_shift_batched(const intlora_layer* layers, const intlora_merge_out* outs,
+                                           int32_t count, int32_t shift_bits, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  return merge_batched(kShift, layers, outs, count, shift_bits, ws, ws_bytes, stream);
+}
+
+intlora_status intlora_merge_mul(const intlora_layer* layer, int32_t u_bits, void* prod_out,
+                                 float* sbar_out, int32_t* zbar_out, uint8_t* u_round_out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  intlora_merge_out o{prod_out, sbar_out, zbar_out, u_round_out};
+  g_last_error[0] = '\0';
+  if (layer == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "layer is NULL");
+  return merge_batched(kMul, layer, &o, 1, u_bits, ws, ws_bytes, stream);
+}
+
+intlora_status intlora_merge_shift(const intlora_layer* layer, int32_t shift_bits, void* m_out,
+                                   float* sbar_out, uint8_t* shift_out, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  intlora_merge_out o{m_out, sbar_out, nullptr, shift_out};
+  g_last_error[0] = '\0';
+  if (layer == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "layer is NULL");
+  return merge_batched(kShift, layer, &o, 1, shift_bits, ws, ws_bytes, stream);
+}
+
+size_t intlora_ste_workspace_size(const intlora_ste_job* jobs, int32_t count) {
+  (void)jobs;
+  (void)count;
+  return 0;
+}
+
+intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t count, void* ws,
+                                            size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_status s = check_ste(jobs[k], k);
+    if (s != INTLORA_OK) return s;
+  }
+  for (int32_t k0 = 0; k0 < count; k0 += kMaxBatch) {
+    const int32_t c = std::min<int32_t>(kMaxBatch, count - k0);
+    const intlora_status s = ste_chunk(jobs + k0, c, static_cast<cudaStream_t>(stream));
+    if (s != INTLORA_OK) return s;
+  }
+  return INTLORA_OK;
+}
+
+intlora_status intlora_ste_backward(const void* G, const void* A, const void* B, int64_t d, int64_t n,
+                                    int32_t r, float* dA, float* dB, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  intlora_ste_job j{G, A, B, d, n, r, dA, dB};
+  return intlora_ste_backward_batched(&j, 1, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+// Device-side building blocks of the IntLoRA merge kernels (sm_100a).
+//
+//  * Philox4x32-10 counter-based generator [Salmon et al., SC'11]: the
+//    auxiliary matrix R is regenerated from (seed, stream id, element index)
+//    instead of being stored ("R is generated online from distribution
+//    statistics and a fixed seed, with no extra storage": IntLoRA paper notes,
+//    ICML2025, method section 1, AQS).
+//  * Laplace(0,1) by the inverse CDF (the auxiliary law the IntLoRA ablation
+//    selects: atlas.scime.ai summary, "Measured effects").
+//  * Rounding and order-preserving helpers used by the row quantizers.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace intlora {
+
+// Philox4x32 multipliers and Weyl key increments (published constants of the
+// generator).
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u;
+constexpr uint32_t kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u;
+constexpr uint32_t kPhiloxW1 = 0xBB67AE85u;
+
+// Ten rounds of Philox4x32 on counter (c0, c1, c2, c3) under key (k0, k1).
+// Each round multiplies words 0 and 2 by the two constants (32x32 -> 64),
+// swaps the halves around with words 1 and 3 and the round key, and bumps
+// the key by the Weyl increments.
+__device__ __forceinline__ uint4 philox10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                          uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t hi0 = __umulhi(kPhiloxM0, c0);
+    const uint32_t lo0 = kPhiloxM0 * c0;
+    const uint32_t hi1 = __umulhi(kPhiloxM1, c2);
+    const uint32_t lo1 = kPhiloxM1 * c2;
+    c0 = hi1 ^ c1 ^ k0;
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ k1;
+    c3 = lo0;
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+  return make_uint4(c0, c1, c2, c3);
+}
+
+// Four consecutive words of the auxiliary stream, starting at a flat index
+// that is a multiple of 4: block = e / 4, counter (block lo, block hi,
+// stream id, 0).
+__device__ __forceinline__ uint4 aux_block(uint64_t block, uint32_t stream_id, uint32_t k0,
+                                           uint32_t k1) {
+  return philox10(static_cast<uint32_t>(block), static_cast<uint32_t>(block >> 32), stream_id,
+                  0u, k0, k1);
+}
+
+// One word of the auxiliary stream at any flat index (ragged shapes).
+__device__ __forceinline__ uint32_t aux_word(uint64_t e, uint32_t stream_id, uint32_t k0,
+                                             uint32_t k1) {
+  const uint4 w = aux_block(e >> 2, stream_id, k0, k1);
+  const uint32_t sel = static_cast<uint32_t>(e & 3u);
+  return sel == 0 ? w.x : sel == 1 ? w.y : sel == 2 ? w.z : w.w;
+}
+
+// c * R for the Laplace sample of word x, with c_ln2 = c * ln 2 (fp32).
+//
+// With k = x >> 9 (23 bits), u = (2k + 1) 2^-24 and v = u - 1/2, the inverse
+// CDF gives R = -sign(v) ln(1 - 2|v|). Folding the sign: 1 - 2|v| = m 2^-23
+// with m = 2k' + 1, k' = k for v < 0 and 2^23 - 1 - k for v > 0, i.e. k' is
+// bits 9..30 of x XOR (x's sign bit replicated). m 2^-23 is built exactly as
+// the float (1 + m 2^-23) - 1. sign(v) = +1 exactly when bit 31 of x is set,
+// so R = ln2 * log2(m 2^-23) with the sign flipped for those words.
+__device__ __forceinline__ float laplace_scaled(uint32_t x, float c_ln2) {
+  const uint32_t sign_mask = static_cast<uint32_t>(static_cast<int32_t>(x) >> 31);
+  const uint32_t folded = x ^ sign_mask;                       // bit 31 now clear
+  const float one_plus = __uint_as_float((folded >> 8) | 0x3F800001u);
+  const float y = one_plus - 1.0f;                             // exact, in (0, 1)
+  const float lg = __log2f(y);                                 // < 0
+  const float cs = __uint_as_float(__float_as_uint(c_ln2) ^ (sign_mask & 0x80000000u));
+  return lg * cs;
+}
+
+// Round to nearest, ties to even, for |x| < 2^22, via the 1.5 * 2^23 bias:
+// the fused multiply-add rounds x * inv + bias once, leaving the integer in
+// the low mantissa bits.
+constexpr float kRoundBias = 12582912.0f;          // 1.5 * 2^23
+constexpr int32_t kRoundBiasBits = 0x4B400000;
+__device__ __forceinline__ int32_t rne_scaled(float x, float inv) {
+  return __float_as_int(fmaf(x, inv, kRoundBias)) - kRoundBiasBits;
+}
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ int32_t clamp_i(int32_t v, int32_t lo, int32_t hi) {
+  return min(max(v, lo), hi);
+}
+
+// Non-negative floats order like their bit patterns: row maxima of
+// non-negative quantities are reduced as unsigned integers.
+__device__ __forceinline__ uint32_t nonneg_bits(float v) { return __float_as_uint(fmaxf(v, 0.0f)); }
+
+// Threshold on the fp32 mantissa for "1.f > sqrt(2)": floor((sqrt2 - 1) 2^23).
+constexpr uint32_t kSqrt2Mantissa = 0x3504F3u;
+
+// Nearest integer of -log2|v| for 0 < |v| <= 1 (and +large for v = 0 or
+// subnormal v), decided exactly on the exponent and mantissa bits: with
+// |v| = 2^E * 1.f, -log2|v| = -E - log2(1.f) rounds to -E - 1 exactly when
+// 1.f > sqrt(2) (the half-integer threshold of the log domain).
+__device__ __forceinline__ int32_t neg_log2_round(float v) {
+  const uint32_t a = __float_as_uint(v) & 0x7FFFFFFFu;
+  const int32_t e = static_cast<int32_t>(a >> 23) - 127;
+  const int32_t up = (a & 0x7FFFFFu) > kSqrt2Mantissa ? 1 : 0;
+  return -e - up;
+}
+
+__device__ __forceinline__ void warp_sum2(double& a, double& b) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+}
+
+// Cluster helpers (inline PTX; sm_90+).
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_smem_to_rank(const void* p, uint32_t rank) {
+  uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+}  // namespace intlora

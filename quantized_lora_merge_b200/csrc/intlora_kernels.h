@@ -1,0 +1,122 @@
+// Internal descriptors and launchers of the IntLoRA kernels. The public C ABI
+// (include/intlora.h) validates arguments, fills these descriptors and calls
+// the launchers; descriptors travel to the device as kernel parameters, so a
+// batched call needs no device-side table and no host-to-device copy.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace intlora {
+
+constexpr int kMaxBatch = 128;          // descriptors per launch
+
+// ---------------------------------------------------------------------------
+// Whole-layer statistics (sigma_W and sigma_R): one partial per CTA, reduced
+// in a fixed order by the finalize kernel, so sigma is bit-reproducible.
+// ---------------------------------------------------------------------------
+struct StatsJob {
+  const float* W;            // nullptr: R statistics only
+  int64_t numel;
+  uint32_t key0, key1, stream_id;
+  int32_t nblocks;           // CTAs working on this job
+  int64_t block_begin;       // index of the job's first CTA in the grid
+  double* partial;           // [nblocks][4]: sum(w-K), sum((w-K)^2), sum R, sum R^2
+  double* sigma_w_out;       // may be nullptr
+  double* sigma_r_out;
+};
+struct StatsBatch {
+  StatsJob job[kMaxBatch];
+  int32_t count;
+};
+
+// ---------------------------------------------------------------------------
+// Row-tile kernels (base quantization, MUL merge, SHIFT merge). A layer is cut
+// into tiles of m rows; a cluster of C CTAs covers one tile, CTA k of the
+// cluster owning the column slice [k n_c, (k+1) n_c). Row minima and maxima
+// are reduced inside the CTA and then across the cluster through distributed
+// shared memory, so every tile is finished in one pass.
+// ---------------------------------------------------------------------------
+enum Variant : int { kGen = 0, kMul = 1, kShift = 2 };
+
+struct TileLayer {
+  // inputs
+  const void* src;           // kGen: fp32 W; merges: W_round codes
+  int64_t ld_src;            // bytes per row of src
+  const float* s;            // merges: base scales
+  const int32_t* z;          // merges: base zero-points
+  const float* A;            // merges: d x r
+  const float* B;            // merges: r x n
+  const double* sigma_w;
+  const double* sigma_r;
+  float alpha;
+  uint32_t key0, key1, stream_id;
+  // outputs
+  void* out;                 // kGen: codes; kMul: P; kShift: M
+  int64_t ld_out;            // kGen: bytes per code row; merges: elements (= n)
+  float* scale_out;          // kGen: s; merges: s_bar
+  int32_t* zero_out;         // kGen: z; kMul: z_bar
+  uint8_t* code_out;         // kMul: U_round; kShift: shift (optional)
+  float* r_star_out;         // kGen only, optional
+  // geometry
+  int64_t d, n;
+  int32_t r;
+  int32_t n_c;               // columns per CTA (multiple of 4)
+  int32_t m;                 // rows per tile (multiple of kRowsPerItem)
+  int32_t b_resident;        // B slice stays in shared memory across tiles
+  int32_t kc;                // B rows per staged chunk
+  int32_t aligned;           // n % 4 == 0: one Philox block per 4 columns
+  int64_t tile_begin;        // global index of the layer's first tile
+};
+struct TileBatch {
+  TileLayer layer[kMaxBatch];
+  int32_t count;
+  int32_t cluster;           // C
+  int32_t num_clusters;
+  int64_t total_tiles;
+  int32_t bits;              // kGen: w_bits; kMul: u_bits; kShift: shift_bits
+  int32_t w_bits;            // code width of the input W_round (merges)
+  int32_t out_bytes;         // merges: bytes per element of `out` (1, 2 or 4)
+};
+
+constexpr int kTileThreads = 256;
+constexpr int kRowsPerItem = 4;                     // rows of one work item
+constexpr int kItemsPerThread = 3;
+constexpr int kMaxQuads = kTileThreads * kItemsPerThread;   // 4-column groups per tile
+constexpr int kMaxTileRows = 128;
+constexpr int kBSmemFloats = 16384;                 // B slice capacity (64 KB)
+constexpr int kASmemFloats = 8192;                  // A rows of a tile (32 KB)
+
+size_t tile_kernel_smem_bytes();
+
+// ---------------------------------------------------------------------------
+// STE backward.
+// ---------------------------------------------------------------------------
+struct SteJob {
+  const uint16_t* G;
+  const uint16_t* A;
+  const uint16_t* B;
+  int64_t d, n;
+  int32_t r;
+  float* dA;
+  float* dB;
+  int64_t tile_begin;        // first CTA of this job in the grid
+  int32_t ksplit;            // CTAs sharing one output tile (split reduction)
+};
+struct SteBatch {
+  SteJob job[kMaxBatch];
+  int32_t count;
+  int32_t transposed;        // 0: dA = G B^T; 1: dB^T = G^T A
+  int64_t total_tiles;
+};
+
+// Launchers: return the cudaError_t of the launch.
+cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t s);
+cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s);
+cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, cudaStream_t s);
+int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int cluster);
+cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
+cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
+
+}  // namespace intlora

@@ -1,0 +1,131 @@
+// Whole-layer statistics for VMC [IntLoRA paper notes (ICML2025), method
+// section 3: R* = r^alpha R with r = sigma_W / sigma_R]. sigma is the
+// population standard deviation over the d x n layer.
+//
+// One pass reads W (16-byte vector loads) and regenerates R (Philox + Laplace)
+// for the same elements; each CTA accumulates shifted sums in fp64 (shift K =
+// W[0] for W, 0 for R, whose mean is 0 by symmetry), writes one partial, and
+// a finalize kernel adds the partials in a fixed order, so sigma does not
+// depend on scheduling. var = (S2 - S1^2 / N) / N.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "intlora_device.cuh"
+#include "intlora_kernels.h"
+
+namespace intlora {
+
+namespace {
+
+constexpr int kStatsThreads = 256;
+constexpr float kLn2f = 0.693147180559945309f;
+
+__device__ __forceinline__ void block_sum4(double v[4], double* red /* [4][32] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  warp_sum2(v[0], v[1]);
+  warp_sum2(v[2], v[3]);
+  if (lane == 0)
+    for (int q = 0; q < 4; ++q) red[q * 32 + warp] = v[q];
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    for (int q = 0; q < 4; ++q) v[q] = lane < nw ? red[q * 32 + lane] : 0.0;
+    warp_sum2(v[0], v[1]);
+    warp_sum2(v[2], v[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_constant__ StatsBatch b) {
+  __shared__ double red[4 * 32];
+  const int64_t bid = blockIdx.x;
+  int j = 0;
+  while (j + 1 < b.count && b.job[j + 1].block_begin <= bid) ++j;
+  const StatsJob& J = b.job[j];
+  const int64_t local = bid - J.block_begin;
+  const int64_t groups = (J.numel + 3) >> 2;
+  const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
+  const float K = J.W != nullptr ? __ldg(J.W) : 0.0f;
+
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int64_t g = local * kStatsThreads + threadIdx.x; g < groups; g += stride) {
+    const int64_t e = g << 2;
+    const int valid = static_cast<int>(min64(4, J.numel - e));
+    const uint4 w = aux_block(static_cast<uint64_t>(g), J.stream_id, J.key0, J.key1);
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    float rs = 0.0f, rq = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c < valid) {
+        const float rv = laplace_scaled(words[c], kLn2f);
+        rs += rv;
+        rq = fmaf(rv, rv, rq);
+      }
+    }
+    acc[2] += static_cast<double>(rs);
+    acc[3] += static_cast<double>(rq);
+    if (J.W != nullptr) {
+      float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (valid == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(J.W + e));
+        x[0] = v.x - K; x[1] = v.y - K; x[2] = v.z - K; x[3] = v.w - K;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < valid) x[c] = __ldg(J.W + e + c) - K;
+      }
+      acc[0] += static_cast<double>((x[0] + x[1]) + (x[2] + x[3]));
+      acc[1] += static_cast<double>(fmaf(x[0], x[0], x[1] * x[1]) + fmaf(x[2], x[2], x[3] * x[3]));
+    }
+  }
+  block_sum4(acc, red);
+  if (threadIdx.x == 0)
+    for (int q = 0; q < 4; ++q) J.partial[local * 4 + q] = acc[q];
+}
+
+__global__ void __launch_bounds__(kStatsThreads) stats_finalize_kernel(const __grid_constant__ StatsBatch b) {
+  __shared__ double red[4 * 32];
+  const StatsJob& J = b.job[blockIdx.x];
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int64_t k = threadIdx.x; k < J.nblocks; k += kStatsThreads)
+    for (int q = 0; q < 4; ++q) acc[q] += J.partial[k * 4 + q];
+  block_sum4(acc, red);
+  if (threadIdx.x == 0) {
+    const double N = static_cast<double>(J.numel);
+    if (J.W != nullptr && J.sigma_w_out != nullptr) {
+      const double var = (acc[1] - acc[0] * acc[0] / N) / N;
+      *J.sigma_w_out = sqrt(fmax(var, 0.0));
+    }
+    if (J.sigma_r_out != nullptr) {
+      const double var = (acc[3] - acc[2] * acc[2] / N) / N;
+      *J.sigma_r_out = sqrt(fmax(var, 0.0));
+    }
+  }
+}
+
+__global__ void zero_kernel(float* p, int64_t count) {
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < count;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[k] = 0.0f;
+}
+
+}  // namespace
+
+cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t s) {
+  stats_kernel<<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s) {
+  stats_finalize_kernel<<<static_cast<unsigned>(b.count), kStatsThreads, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  const int64_t blocks = min64((count + 255) / 256, 148 * 8);
+  zero_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p, count);
+  return cudaGetLastError();
+}
+
+}  // namespace intlora

@@ -1,0 +1,132 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+public header declares, and rejects bad arguments on the host with the right
+status before any CUDA call (these calls never reach a launch)."""
+import ctypes
+
+import pytest
+
+from quantized_lora_merge_b200 import binding as B
+from quantized_lora_merge_b200.build import build
+
+FAKE = 0x100000  # 16-byte-aligned dummy address; never dereferenced by validation
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.lib()
+
+
+def test_every_header_function_is_exported(lib):
+    names = B.header_functions()
+    assert len(names) >= 15
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/intlora.h but not exported"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.intlora_status_string(0) == b"ok"
+    assert lib.intlora_status_string(1) == b"invalid argument"
+    assert lib.intlora_status_string(99) == b"unknown status"
+    assert lib.intlora_version() >= 100
+
+
+def test_merge_out_bytes(lib):
+    assert lib.intlora_merge_out_bytes(0, 4, 4) == 2     # 15*15 fits int16
+    assert lib.intlora_merge_out_bytes(0, 8, 8) == 4     # 255*255 does not
+    assert lib.intlora_merge_out_bytes(0, 8, 7) == 2     # 255*127 = 32385
+    assert lib.intlora_merge_out_bytes(1, 4, 4) == 1
+    assert lib.intlora_merge_out_bytes(1, 8, 4) == 2
+    assert lib.intlora_merge_out_bytes(2, 8, 4) == 0
+
+
+def _aux(**kw):
+    j = B.intlora_aux_job(W=FAKE, d=4, n=8, seed=1, stream_id=0, alpha=1.5, w_bits=8,
+                          sigma_w_out=FAKE, sigma_r_out=FAKE, r_star_out=None,
+                          w_round_out=FAKE, ld_w_out=16, s_out=FAKE, z_out=FAKE)
+    for k, v in kw.items():
+        setattr(j, k, v)
+    return j
+
+
+@pytest.mark.parametrize("field,value,needle", [
+    ("W", None, "W is NULL"),
+    ("d", 0, "d and n"),
+    ("n", -3, "d and n"),
+    ("w_bits", 3, "w_bits"),
+    ("alpha", -1.0, "alpha"),
+    ("alpha", float("nan"), "alpha"),
+    ("sigma_r_out", None, "sigma"),
+    ("ld_w_out", 8, "ld_w_out"),
+    ("ld_w_out", 24, "ld_w_out"),
+    ("W", FAKE + 4, "16-byte"),
+    ("s_out", None, "s_out"),
+])
+def test_gen_aux_rejects(lib, field, value, needle):
+    jobs = (B.intlora_aux_job * 1)(_aux(**{field: value}))
+    st = lib.intlora_gen_aux_batched(jobs, 1, None, 0, None)
+    assert st == 1
+    assert needle in lib.intlora_last_error().decode()
+
+
+def test_gen_aux_4bit_needs_even_n(lib):
+    jobs = (B.intlora_aux_job * 1)(_aux(w_bits=4, n=7))
+    assert lib.intlora_gen_aux_batched(jobs, 1, None, 0, None) == 1
+    assert "even" in lib.intlora_last_error().decode()
+
+
+def test_gen_aux_workspace_checked(lib):
+    jobs = (B.intlora_aux_job * 1)(_aux())
+    need = lib.intlora_gen_aux_workspace_size(jobs, 1)
+    assert need > 0
+    assert lib.intlora_gen_aux_batched(jobs, 1, None, 0, None) == 3
+    assert lib.intlora_gen_aux_batched(jobs, 1, FAKE, need - 1, None) == 3
+
+
+def _layer(**kw):
+    l = B.intlora_layer(d=4, n=8, r=4, w_bits=8, w_round=FAKE, ld_w=16, s=FAKE, z=FAKE, A=FAKE,
+                        B=FAKE, seed=1, stream_id=0, alpha=1.5, sigma_w=FAKE, sigma_r=FAKE)
+    for k, v in kw.items():
+        setattr(l, k, v)
+    return l
+
+
+@pytest.mark.parametrize("field,value", [
+    ("d", 0), ("r", 0), ("r", 257), ("w_bits", 2), ("w_round", None), ("B", None),
+    ("sigma_w", None), ("ld_w", 4), ("w_round", FAKE + 1), ("alpha", -0.5)])
+def test_merge_rejects_bad_layer(lib, field, value):
+    layer = _layer(**{field: value})
+    st = lib.intlora_merge_mul(ctypes.byref(layer), 8, FAKE, FAKE, FAKE, None, None, 0, None)
+    assert st == 1, lib.intlora_last_error()
+
+
+def test_merge_rejects_bad_bits_and_outputs(lib):
+    layer = _layer()
+    assert lib.intlora_merge_mul(ctypes.byref(layer), 9, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+    assert lib.intlora_merge_mul(ctypes.byref(layer), 8, FAKE, FAKE, None, None, None, 0, None) == 1
+    assert lib.intlora_merge_shift(ctypes.byref(layer), 6, FAKE, FAKE, None, None, 0, None) == 1
+    assert lib.intlora_merge_shift(ctypes.byref(layer), 4, FAKE + 8, FAKE, None, None, 0, None) == 1
+    assert lib.intlora_merge_mul(None, 8, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+
+
+def test_merge_without_sigma_r_needs_workspace(lib):
+    layer = _layer(sigma_r=None)
+    arr = (B.intlora_layer * 1)(layer)
+    need = lib.intlora_merge_workspace_size(arr, 1)
+    assert need > 0
+    assert lib.intlora_merge_workspace_size((B.intlora_layer * 1)(_layer()), 1) == 0
+    st = lib.intlora_merge_mul(ctypes.byref(layer), 8, FAKE, FAKE, FAKE, None, None, 0, None)
+    assert st == 3
+
+
+def test_ste_rejects(lib):
+    assert lib.intlora_ste_backward(None, FAKE, FAKE, 4, 8, 4, FAKE, FAKE, None, 0, None) == 1
+    assert lib.intlora_ste_backward(FAKE, FAKE, FAKE, 4, 8, 0, FAKE, FAKE, None, 0, None) == 1
+    assert lib.intlora_ste_backward(FAKE, FAKE, FAKE, 0, 8, 4, FAKE, FAKE, None, 0, None) == 1
+    assert lib.intlora_ste_backward(FAKE + 2, FAKE, FAKE, 4, 8, 4, FAKE, FAKE, None, 0, None) == 1
+
+
+def test_empty_batches_are_no_ops(lib):
+    assert lib.intlora_gen_aux_batched(None, 0, None, 0, None) == 0
+    assert lib.intlora_merge_mul_batched(None, None, 0, 8, None, 0, None) == 0
+    assert lib.intlora_ste_backward_batched(None, 0, None, 0, None) == 0

@@ -1,0 +1,181 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle on the same
+seeded inputs, through the C ABI. Each stage is fed the oracle's inputs, so a
+difference in one stage cannot cascade into the next."""
+import numpy as np
+import pytest
+
+import oracle
+from quantized_lora_merge_b200 import workloads as wl
+
+from .parity import (STE_RTOL, assert_affine, assert_scale, assert_shift, gpu_gen_aux,
+                     gpu_merge, gpu_ste, rel_fro, spec_for)
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------------------
+# a1: Philox + Laplace, materialised through gen_aux with alpha = 0 (R* = R)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,n", [(256, 1024), (37, 50), (3, 6)])
+def test_aux_matrix_matches_oracle(d, n):
+    spec = spec_for(d, n, 4, 8, alpha=0.0, sid=5)
+    W = wl.host_W(spec)
+    g = gpu_gen_aux([spec], [W], want_r_star=True)[0]
+    R = oracle.aux_R(d, n, spec.seed, spec.stream_id)
+    err = np.abs(g["r_star"].astype(np.float64) - R)
+    assert np.max(err / np.maximum(1.0, np.abs(R))) < 2e-6
+    assert np.array_equal(np.sign(g["r_star"]), np.sign(R))
+
+
+# ---------------------------------------------------------------------------
+# a1-a3: layer preparation
+# ---------------------------------------------------------------------------
+GEN_SHAPES = [(320, 320, 8), (64, 768, 4), (33, 100, 8), (7, 10, 4), (5, 6, 8), (1, 4, 8),
+              (130, 5120, 4), (20, 14336, 8), (9, 2, 4)]
+
+
+@pytest.mark.parametrize("d,n,w_bits", GEN_SHAPES)
+def test_gen_aux_parity(d, n, w_bits):
+    spec = spec_for(d, n, 4, w_bits, sid=d + n)
+    W = wl.host_W(spec)
+    g = gpu_gen_aux([spec], [W])[0]
+    o = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, w_bits)
+    assert_scale("sigma_w", g["sigma_w"], o["sigma_w"])
+    assert_scale("sigma_r", g["sigma_r"], o["sigma_r"])
+    assert_scale("s", g["s"], o["s"])
+    assert_affine("W_round", g["codes"], g["z"], o["codes"], o["z"], o["pre"], o["zpre"],
+                  2**w_bits - 1)
+
+
+def test_gen_aux_batched_equals_single():
+    specs = [spec_for(d, n, 4, b, sid=k) for k, (d, n, b) in enumerate(GEN_SHAPES[:5])]
+    Ws = [wl.host_W(s) for s in specs]
+    a = gpu_gen_aux(specs, Ws, batched=True)
+    b = gpu_gen_aux(specs, Ws, batched=False)
+    for x, y in zip(a, b):
+        assert x["sigma_w"] == y["sigma_w"] and x["sigma_r"] == y["sigma_r"]
+        assert np.array_equal(x["codes"], y["codes"]) and np.array_equal(x["s"], y["s"])
+
+
+# ---------------------------------------------------------------------------
+# a4-a7: merges, on the oracle's prepared layers
+# ---------------------------------------------------------------------------
+def _oracle_prepared(spec):
+    W = wl.host_W(spec)
+    g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits)
+    return dict(codes=g["codes"], s=g["s"].astype(np.float32), z=g["z"], A=wl.host_A(spec),
+                B=wl.host_B(spec), sigma_w=g["sigma_w"], sigma_r=g["sigma_r"])
+
+
+def _check_mul(spec, inp, got):
+    o = oracle.merge_mul(inp["codes"], inp["s"], inp["z"], inp["A"], inp["B"], spec.seed,
+                         spec.stream_id, inp["sigma_w"], inp["sigma_r"], spec.alpha,
+                         spec.out_bits)
+    qmax = 2**spec.out_bits - 1
+    assert_scale("s_bar", got["sbar"], o["sbar"])
+    assert_affine("U_round", got["code"], got["zbar"], o["u_round"], o["zbar"], o["pre"],
+                  o["zpre"], qmax)
+    D = inp["codes"].astype(np.int64) - inp["z"][:, None]
+    # the products are exactly (U_round - z_bar) * D of the GPU's own codes ...
+    assert np.array_equal(got["out"], (got["code"].astype(np.int64) - got["zbar"][:, None]) * D)
+    # ... and equal to the oracle's wherever the codes agree
+    same = (got["code"] == o["u_round"]) & (got["zbar"] == o["zbar"])[:, None]
+    assert np.array_equal(got["out"][same], o["P"][same])
+    assert np.all(got["out"][D == 0] == 0)
+
+
+def _check_shift(spec, inp, got):
+    o = oracle.merge_shift(inp["codes"], inp["s"], inp["z"], inp["A"], inp["B"], spec.seed,
+                           spec.stream_id, inp["sigma_w"], inp["sigma_r"], spec.alpha,
+                           spec.out_bits)
+    assert_scale("s_bar", got["sbar"], o["sbar"])
+    assert_shift("shift", got["code"], o["shift"], o["pre"], 2**spec.out_bits - 1)
+    D = inp["codes"].astype(np.int64) - inp["z"][:, None]
+    sign = np.sign(o["U"]).astype(np.int64)
+    assert np.array_equal(got["out"], sign * (D >> got["code"].astype(np.int64)))
+    same = got["code"] == o["shift"]
+    assert np.array_equal(got["out"][same], o["M"][same])
+
+
+MUL_CASES = [
+    # d, n, r, w_bits, u_bits
+    (320, 320, 4, 8, 8),      # the single 320x320 layer
+    (64, 768, 4, 4, 4),       # SD cross-attention shape, int4
+    (40, 4096, 16, 8, 8),     # Llama width, cluster of CTAs over the columns
+    (24, 14336, 16, 8, 8),    # Llama down-projection width
+    (12, 4096, 128, 8, 8),    # rank 128: B streamed through shared memory
+    (9, 50, 3, 8, 8),         # ragged: n % 4 != 0, rank not a template
+    (130, 5120, 4, 4, 4),     # FF width 4d at d = 1280
+    (1, 8, 1, 4, 4),          # single row, rank 1
+    (17, 64, 8, 8, 6),        # 6-bit U quantizer (int16 products)
+]
+
+
+@pytest.mark.parametrize("d,n,r,w_bits,u_bits", MUL_CASES)
+def test_merge_mul_parity(d, n, r, w_bits, u_bits):
+    spec = spec_for(d, n, r, w_bits, "mul", u_bits, sid=7 + d)
+    inp = _oracle_prepared(spec)
+    got = gpu_merge([spec], [inp])[0]
+    _check_mul(spec, inp, got)
+
+
+SHIFT_CASES = [
+    (32, 3072, 64, 4, 4),     # DiT width, r = 64, 4-bit base, 4-bit shift
+    (16, 12288, 64, 4, 4),    # DiT fc2 width
+    (48, 320, 4, 8, 4),       # 8-bit base: int16 merged codes
+    (5, 6, 2, 4, 2),          # ragged, 2-bit shift code (clamps at 3)
+    (3, 40, 32, 8, 5),
+]
+
+
+@pytest.mark.parametrize("d,n,r,w_bits,shift_bits", SHIFT_CASES)
+def test_merge_shift_parity(d, n, r, w_bits, shift_bits):
+    spec = spec_for(d, n, r, w_bits, "shift", shift_bits, sid=11 + d)
+    inp = _oracle_prepared(spec)
+    got = gpu_merge([spec], [inp])[0]
+    _check_shift(spec, inp, got)
+
+
+def test_merge_reduces_sigma_r_on_device_when_not_given():
+    spec = spec_for(50, 256, 8, 8, "mul", 8, sid=3)
+    inp = _oracle_prepared(spec)
+    a = gpu_merge([spec], [inp], pass_sigma_r=True)[0]
+    b = gpu_merge([spec], [inp], pass_sigma_r=False)[0]
+    _check_mul(spec, inp, b)
+    assert np.array_equal(a["sbar"], b["sbar"]) or np.max(np.abs(a["sbar"] / b["sbar"] - 1)) < 1e-6
+
+
+def test_merge_batched_equals_single():
+    specs = [spec_for(d, n, r, wb, "mul", ub, sid=k)
+             for k, (d, n, r, wb, ub) in enumerate([(64, 768, 4, 4, 4), (30, 320, 4, 4, 4),
+                                                     (130, 5120, 4, 4, 4)])]
+    inps = [_oracle_prepared(s) for s in specs]
+    a = gpu_merge(specs, inps, batched=True)
+    b = gpu_merge(specs, inps, batched=False)
+    for x, y in zip(a, b):
+        assert np.array_equal(x["out"], y["out"]) and np.array_equal(x["sbar"], y["sbar"])
+
+
+def test_merge_without_code_output():
+    spec = spec_for(20, 128, 4, 8, "mul", 8, sid=2)
+    inp = _oracle_prepared(spec)
+    a = gpu_merge([spec], [inp], want_code=False)[0]
+    b = gpu_merge([spec], [inp], want_code=True)[0]
+    assert np.array_equal(a["out"], b["out"])
+
+
+# ---------------------------------------------------------------------------
+# a8: STE backward
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,n,r", [(320, 320, 4), (64, 768, 16), (100, 300, 128), (1, 5, 1),
+                                   (257, 1030, 33)])
+def test_ste_parity(d, n, r):
+    spec = spec_for(d, n, r, 8, sid=d)
+    Gb = wl.host_G_bits(spec)
+    Ab = wl.to_bf16_bits(wl.host_A(spec))
+    Bb = wl.to_bf16_bits(wl.host_B(spec))
+    dA, dB = gpu_ste(Gb, Ab, Bb)
+    G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+    oA, oB = oracle.ste_backward(G, A, Bm)
+    assert rel_fro(dA, oA) < STE_RTOL
+    assert rel_fro(dB, oB) < STE_RTOL

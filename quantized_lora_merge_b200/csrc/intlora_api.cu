@@ -55,23 +55,18 @@ size_t stats_partial_bytes(int64_t numel) { return round256(static_cast<size_t>(
 // ------------------------------------------------------------------------
 // tile geometry: cluster size, column slice, rows per tile
 // ------------------------------------------------------------------------
-struct Geometry {
-  int cluster = 1;
-  int num_clusters = 0;
-};
-
-int max_active_clusters_cached(int variant, int w_bits, int rank_ct, int cluster) {
+int max_active_clusters_cached(int variant, int w_bits, int rank_ct, bool aligned, int cluster) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int>, int> cache;
+  static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, cluster);
+  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, aligned ? 1 : 0, cluster);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
   }
-  const int v = tile_max_active_clusters(variant, w_bits, rank_ct, cluster);
+  const int v = tile_max_active_clusters(variant, w_bits, rank_ct, aligned, cluster);
   std::lock_guard<std::mutex> lock(mu);
   cache[key] = v;
   return v;
@@ -122,6 +117,8 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
       if (l.r != rank_ct) rank_ct = 0;
     if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16 && rank_ct != 32) rank_ct = 0;
   }
+  bool aligned = true;
+  for (auto& l : L) aligned = aligned && (l.n % 4 == 0);
   static const int kClusters[] = {1, 2, 4, 8, 16};
   int chosen = -1;
   int64_t total = -1;
@@ -132,7 +129,7 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
       const int64_t t = plan_layers(variant, L, c, &resident);
       if (t < 0) continue;
       if (pass == 0 && variant != kGen && !resident) continue;
-      if (max_active_clusters_cached(variant, w_bits, rank_ct, c) <= 0) continue;
+      if (max_active_clusters_cached(variant, w_bits, rank_ct, aligned, c) <= 0) continue;
       chosen = c;
       total = t;
       break;
@@ -147,11 +144,11 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
   b.cluster = chosen;
   b.total_tiles = total;
   b.num_clusters = static_cast<int32_t>(
-      std::min<int64_t>(total, max_active_clusters_cached(variant, w_bits, rank_ct, chosen)));
+      std::min<int64_t>(total, max_active_clusters_cached(variant, w_bits, rank_ct, aligned, chosen)));
   b.bits = bits;
   b.w_bits = w_bits;
   b.out_bytes = out_bytes;
-  cudaError_t e = launch_tiles(variant, b, rank_ct, stream);
+  cudaError_t e = launch_tiles(variant, b, rank_ct, aligned, stream);
   if (e != cudaSuccess) return cuda_fail(e, "row-tile kernel launch");
   return INTLORA_OK;
 }

@@ -30,16 +30,12 @@ __device__ __forceinline__ uint4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
                                           uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
-    const uint32_t hi0 = __umulhi(kPhiloxM0, c0);
-    const uint32_t lo0 = kPhiloxM0 * c0;
-    const uint32_t hi1 = __umulhi(kPhiloxM1, c2);
-    const uint32_t lo1 = kPhiloxM1 * c2;
-    c0 = hi1 ^ c1 ^ k0;
-    c1 = lo1;
-    c2 = hi0 ^ c3 ^ k1;
-    c3 = lo0;
-    k0 += kPhiloxW0;
-    k1 += kPhiloxW1;
+    const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * c0;   // one wide multiply each
+    const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * c2;
+    c0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ (k0 + round * kPhiloxW0);
+    c2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ (k1 + round * kPhiloxW1);
+    c1 = static_cast<uint32_t>(p1);
+    c3 = static_cast<uint32_t>(p0);
   }
   return make_uint4(c0, c1, c2, c3);
 }
@@ -69,14 +65,18 @@ __device__ __forceinline__ uint32_t aux_word(uint64_t e, uint32_t stream_id, uin
 // bits 9..30 of x XOR (x's sign bit replicated). m 2^-23 is built exactly as
 // the float (1 + m 2^-23) - 1. sign(v) = +1 exactly when bit 31 of x is set,
 // so R = ln2 * log2(m 2^-23) with the sign flipped for those words.
-__device__ __forceinline__ float laplace_scaled(uint32_t x, float c_ln2) {
+__device__ __forceinline__ float laplace_log2(uint32_t x) {
   const uint32_t sign_mask = static_cast<uint32_t>(static_cast<int32_t>(x) >> 31);
   const uint32_t folded = x ^ sign_mask;                       // bit 31 now clear
   const float one_plus = __uint_as_float((folded >> 8) | 0x3F800001u);
-  const float y = one_plus - 1.0f;                             // exact, in (0, 1)
-  const float lg = __log2f(y);                                 // < 0
-  const float cs = __uint_as_float(__float_as_uint(c_ln2) ^ (sign_mask & 0x80000000u));
-  return lg * cs;
+  return __log2f(one_plus - 1.0f);                             // log2(m 2^-23) < 0, exact input
+}
+// +-c ln2: the factor that turns laplace_log2(x) into c * R.
+__device__ __forceinline__ float laplace_sign(uint32_t x, float c_ln2) {
+  return __uint_as_float(__float_as_uint(c_ln2) ^ (x & 0x80000000u));
+}
+__device__ __forceinline__ float laplace_scaled(uint32_t x, float c_ln2) {
+  return laplace_log2(x) * laplace_sign(x, c_ln2);
 }
 
 // Round to nearest, ties to even, for |x| < 2^22, via the 1.5 * 2^23 bias:

@@ -114,8 +114,8 @@ struct SteBatch {
 // Launchers: return the cudaError_t of the launch.
 cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t s);
 cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s);
-cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, cudaStream_t s);
-int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int cluster);
+cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s);
+int tile_max_active_clusters(int variant, int w_bits, int rank_ct, bool aligned, int cluster);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 

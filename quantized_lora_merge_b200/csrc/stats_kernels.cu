@@ -36,6 +36,68 @@ __device__ __forceinline__ void block_sum4(double v[4], double* red /* [4][32] *
   }
 }
 
+// Sums of one group of 4 consecutive elements (one Philox block). fp32 partial
+// sums of a few groups are flushed into the fp64 accumulators.
+struct GroupSums {
+  float w1 = 0.f, w2 = 0.f, r1 = 0.f, r2 = 0.f;
+};
+
+template <bool HAS_W>
+__device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64_t group, float K,
+                                          int valid) {
+  const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, J.key0, J.key1);
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  if (HAS_W) {
+    const int64_t e = group << 2;
+    if (valid == 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(J.W + e));
+      x[0] = v.x - K; x[1] = v.y - K; x[2] = v.z - K; x[3] = v.w - K;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < valid) x[c] = __ldg(J.W + e + c) - K;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float rv = c < valid ? laplace_scaled(words[c], kLn2f) : 0.0f;
+    g.r1 += rv;
+    g.r2 = fmaf(rv, rv, g.r2);
+    if (HAS_W) {
+      g.w1 += x[c];
+      g.w2 = fmaf(x[c], x[c], g.w2);
+    }
+  }
+}
+
+template <bool HAS_W>
+__device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4]) {
+  constexpr int kFlush = 8;   // groups per fp32 partial
+  const int64_t full = J.numel >> 2;                 // complete groups
+  const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
+  const float K = HAS_W ? __ldg(J.W) : 0.0f;
+  int64_t g = local * kStatsThreads + threadIdx.x;
+  while (g < full) {
+    GroupSums s;
+#pragma unroll 2
+    for (int u = 0; u < kFlush && g < full; ++u, g += stride) add_group<HAS_W>(s, J, g, K, 4);
+    acc[0] += static_cast<double>(s.w1);
+    acc[1] += static_cast<double>(s.w2);
+    acc[2] += static_cast<double>(s.r1);
+    acc[3] += static_cast<double>(s.r2);
+  }
+  const int tail = static_cast<int>(J.numel & 3);
+  if (tail != 0 && local == 0 && threadIdx.x == 0) {
+    GroupSums s;
+    add_group<HAS_W>(s, J, full, K, tail);
+    acc[0] += static_cast<double>(s.w1);
+    acc[1] += static_cast<double>(s.w2);
+    acc[2] += static_cast<double>(s.r1);
+    acc[3] += static_cast<double>(s.r2);
+  }
+}
+
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_constant__ StatsBatch b) {
   __shared__ double red[4 * 32];
   const int64_t bid = blockIdx.x;
@@ -43,41 +105,9 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_const
   while (j + 1 < b.count && b.job[j + 1].block_begin <= bid) ++j;
   const StatsJob& J = b.job[j];
   const int64_t local = bid - J.block_begin;
-  const int64_t groups = (J.numel + 3) >> 2;
-  const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
-  const float K = J.W != nullptr ? __ldg(J.W) : 0.0f;
-
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int64_t g = local * kStatsThreads + threadIdx.x; g < groups; g += stride) {
-    const int64_t e = g << 2;
-    const int valid = static_cast<int>(min64(4, J.numel - e));
-    const uint4 w = aux_block(static_cast<uint64_t>(g), J.stream_id, J.key0, J.key1);
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-    float rs = 0.0f, rq = 0.0f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (c < valid) {
-        const float rv = laplace_scaled(words[c], kLn2f);
-        rs += rv;
-        rq = fmaf(rv, rv, rq);
-      }
-    }
-    acc[2] += static_cast<double>(rs);
-    acc[3] += static_cast<double>(rq);
-    if (J.W != nullptr) {
-      float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (valid == 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(J.W + e));
-        x[0] = v.x - K; x[1] = v.y - K; x[2] = v.z - K; x[3] = v.w - K;
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < valid) x[c] = __ldg(J.W + e + c) - K;
-      }
-      acc[0] += static_cast<double>((x[0] + x[1]) + (x[2] + x[3]));
-      acc[1] += static_cast<double>(fmaf(x[0], x[0], x[1] * x[1]) + fmaf(x[2], x[2], x[3] * x[3]));
-    }
-  }
+  if (J.W != nullptr) stats_body<true>(J, local, acc);
+  else stats_body<false>(J, local, acc);
   block_sum4(acc, red);
   if (threadIdx.x == 0)
     for (int q = 0; q < 4; ++q) J.partial[local * 4 + q] = acc[q];

@@ -77,9 +77,100 @@ __device__ __forceinline__ int32_t code_at(uint32_t packed, int c) {
                     : static_cast<int32_t>((packed >> (4 * c)) & 0xFu);
 }
 
-template <int VARIANT, int WBITS, int RANK>
+// Stores of one item row (4 columns): codes (kGen), P (kMul) or M (kShift),
+// plus the optional per-element code output of the merges.
+template <int VARIANT, int WBITS, bool ALIGNED>
+__device__ __forceinline__ void store_item(const TileLayer& L, int out_bytes, int64_t i, int64_t j,
+                                           int vcols, const int32_t res[4], const uint32_t code8[4]) {
+  if (VARIANT == kGen) {
+    if (L.out == nullptr) return;
+    uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
+    if (WBITS == 8) {
+      const uint32_t packed = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
+      if (ALIGNED || vcols == 4) {
+        *reinterpret_cast<uint32_t*>(orow + j) = packed;
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < vcols) orow[j + c] = static_cast<uint8_t>(code8[c]);
+      }
+    } else {
+      const uint32_t packed = code8[0] | (code8[1] << 4) | (code8[2] << 8) | (code8[3] << 12);
+      if (ALIGNED || vcols == 4) {
+        *reinterpret_cast<uint16_t*>(orow + (j >> 1)) = static_cast<uint16_t>(packed);
+      } else {
+        // n is even for 4-bit codes, so a ragged quad holds exactly 2 columns
+        orow[j >> 1] = static_cast<uint8_t>(packed & 0xFFu);
+      }
+    }
+    return;
+  }
+  const int64_t e0 = i * L.n + j;
+  const bool vec = ALIGNED || vcols == 4;
+  if (vec && !ALIGNED) {
+    // an unaligned layer has row starts off the vector boundary
+    for (int c = 0; c < 4; ++c) {
+      if (out_bytes == 4) static_cast<int32_t*>(L.out)[e0 + c] = res[c];
+      else if (out_bytes == 2) static_cast<int16_t*>(L.out)[e0 + c] = static_cast<int16_t>(res[c]);
+      else static_cast<int8_t*>(L.out)[e0 + c] = static_cast<int8_t>(res[c]);
+      if (L.code_out != nullptr) L.code_out[e0 + c] = static_cast<uint8_t>(code8[c]);
+    }
+    return;
+  }
+  if (out_bytes == 4) {   // MUL products beyond the int16 bound
+    int32_t* o = static_cast<int32_t*>(L.out) + e0;
+    if (vec) {
+      *reinterpret_cast<int4*>(o) = make_int4(res[0], res[1], res[2], res[3]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < vcols) o[c] = res[c];
+    }
+  } else if (out_bytes == 2) {   // int16 products or merged codes
+    int16_t* o = static_cast<int16_t*>(L.out) + e0;
+    if (vec) {
+      const uint32_t lo = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
+      const uint32_t hi = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
+      *reinterpret_cast<uint2*>(o) = make_uint2(lo, hi);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < vcols) o[c] = static_cast<int16_t>(res[c]);
+    }
+  } else {   // int8 merged codes (SHIFT with a base of at most 7 bits)
+    int8_t* o = static_cast<int8_t*>(L.out) + e0;
+    if (vec) {
+      *reinterpret_cast<uint32_t*>(o) = (static_cast<uint32_t>(res[0]) & 0xFFu) |
+                                        ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
+                                        ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) |
+                                        (static_cast<uint32_t>(res[3]) << 24);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < vcols) o[c] = static_cast<int8_t>(res[c]);
+    }
+  }
+  if (L.code_out != nullptr) {
+    uint8_t* co = L.code_out + e0;
+    if (vec) {
+      *reinterpret_cast<uint32_t*>(co) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (c < vcols) co[c] = static_cast<uint8_t>(code8[c]);
+    }
+  }
+}
+
+// Non-negative floats (sign bit clear) order like their bit patterns, so row
+// maxima are reduced as unsigned integers (REDUX, shared atomics, DSMEM).
+__device__ __forceinline__ uint32_t ord(float v) { return __float_as_uint(v); }
+
+template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
 __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_constant__ TileBatch p) {
   constexpr SmemLayout lay = layout_for(VARIANT);
+  constexpr int IPT = kItemsPerThread;
+  constexpr int RPI = kRowsPerItem;
   extern __shared__ __align__(16) float smem[];
   float* Bs = smem + lay.b_off();
   float* At = smem + lay.a_off();
@@ -118,7 +209,6 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
     const int r = (VARIANT == kGen) ? 0 : (RANK > 0 ? RANK : L.r);
     const int m = L.m;
     const int n_c = L.n_c;
-    const bool aligned = L.aligned != 0;
 
     __syncthreads();  // previous tile is done with At, row params and q params
     if (li != cur) {
@@ -127,10 +217,9 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
         s_cln2 = static_cast<float>(c * kLn2);
       }
       if (VARIANT != kGen && L.b_resident) {
-        const float* Bg = L.B;
         for (int idx = tid; idx < r * n_c; idx += kTileThreads) {
           const int k = idx / n_c, jj = idx - k * n_c;
-          Bs[idx] = jj < ncols ? __ldg(Bg + static_cast<int64_t>(k) * L.n + col0 + jj) : 0.0f;
+          Bs[idx] = jj < ncols ? __ldg(L.B + static_cast<int64_t>(k) * L.n + col0 + jj) : 0.0f;
         }
       }
       cur = li;
@@ -138,42 +227,56 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
     if (VARIANT != kGen) {
       for (int rr = tid; rr < m; rr += kTileThreads) {
         row_s[rr] = rr < rows ? __ldg(L.s + row0 + rr) : 0.0f;
-        row_z[rr] = rr < rows ? __ldg(L.z + row0 + rr) : 0;
+        // zero-points outside the code range are clamped into it, so the
+        // reciprocal table is never indexed outside [-2^b + 1, 2^b - 1]
+        row_z[rr] = rr < rows ? clamp_i(__ldg(L.z + row0 + rr), 0, (1 << p.w_bits) - 1) : 0;
       }
+      // A rows of the tile, read along the rank (coalesced), stored k-major
       for (int idx = tid; idx < r * m; idx += kTileThreads) {
-        const int k = idx / m, rr = idx - k * m;
-        At[idx] = rr < rows ? __ldg(L.A + (row0 + rr) * static_cast<int64_t>(L.r) + k) : 0.0f;
+        const int rr = idx / max(r, 1), k = idx - rr * max(r, 1);
+        At[k * m + rr] = rr < rows ? __ldg(L.A + (row0 + rr) * static_cast<int64_t>(L.r) + k) : 0.0f;
       }
     }
     __syncthreads();
     const float c_ln2 = s_cln2;
 
+    // ---- work items of this thread: 4 rows x 4 columns each
     const int quads = n_c >> 2;
-    const int nitems = (m / kRowsPerItem) * quads;
-
-    float acc[kItemsPerThread][kRowsPerItem][4];
-    uint32_t cw[kItemsPerThread][kRowsPerItem];
-
-    // ---- phase A.1: loads of the codes (merges) or of W (base quantization)
+    const int G = m / RPI;
+    const int nitems = G * quads;
+    int ig[IPT], iq[IPT];
+    bool iok[IPT];
 #pragma unroll
-    for (int k = 0; k < kItemsPerThread; ++k) {
+    for (int k = 0; k < IPT; ++k) {
       const int it = tid + k * kTileThreads;
-      const int g = it / quads, q = it - (it / quads) * quads;
-      const int jl = 4 * q;
-      const int vcols = min(4, ncols - jl);
+      const int g = it / quads;
+      iq[k] = it - g * quads;
+      iok[k] = it < nitems && 4 * iq[k] < ncols;
+      ig[k] = min(g, G - 1);
+    }
+
+    float acc[IPT][RPI][4];
+    uint32_t cw[IPT][RPI];
+
+    // ---- phase A.1: codes (merges) or W (base quantization); rows past the
+    // layer's end read the last row (their results are masked out)
 #pragma unroll
-      for (int ml = 0; ml < kRowsPerItem; ++ml) {
-        const int rr = g * kRowsPerItem + ml;
-        const bool ok = it < nitems && rr < rows && vcols > 0;
+    for (int k = 0; k < IPT; ++k) {
+#pragma unroll
+      for (int ml = 0; ml < RPI; ++ml) {
         cw[k][ml] = 0u;
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[k][ml][c] = 0.0f;
-        if (!ok) continue;
-        const int64_t i = row0 + rr;
-        const int64_t j = col0 + jl;
+      }
+      if (!iok[k]) continue;
+      const int64_t j = col0 + 4 * iq[k];
+      const int vcols = ALIGNED ? 4 : min(4, ncols - 4 * iq[k]);
+#pragma unroll
+      for (int ml = 0; ml < RPI; ++ml) {
+        const int64_t i = row0 + min(ig[k] * RPI + ml, rows - 1);
         if (VARIANT == kGen) {
           const float* wr = static_cast<const float*>(L.src) + i * L.n;
-          if (aligned && vcols == 4) {
+          if (ALIGNED) {
             const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + j));
             acc[k][ml][0] = w4.x; acc[k][ml][1] = w4.y; acc[k][ml][2] = w4.z; acc[k][ml][3] = w4.w;
           } else {
@@ -183,17 +286,37 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
           }
         } else {
           const uint8_t* wr = static_cast<const uint8_t*>(L.src) + i * L.ld_src;
-          cw[k][ml] = load_codes<WBITS>(wr, j, vcols, aligned);
+          cw[k][ml] = load_codes<WBITS>(wr, j, vcols, ALIGNED);
         }
       }
     }
 
     // ---- phase A.2: T = A B on the tile (CUDA-core FMA), B from shared memory
     if (VARIANT != kGen) {
-      const int kc = L.b_resident ? r : L.kc;
-      for (int k0 = 0; k0 < r; k0 += kc) {
-        const int kn = min(kc, r - k0);
-        if (!L.b_resident) {
+      auto fma_tile = [&](const float* arow, const float* brow) {
+#pragma unroll
+        for (int k = 0; k < IPT; ++k) {
+          const float4 a4 = *reinterpret_cast<const float4*>(arow + ig[k] * RPI);
+          const float4 b4 = *reinterpret_cast<const float4*>(brow + 4 * iq[k]);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int ml = 0; ml < RPI; ++ml)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[k][ml][c] = fmaf(av[ml], bv[c], acc[k][ml][c]);
+        }
+      };
+      if (L.b_resident) {
+        if (RANK > 0) {
+#pragma unroll
+          for (int kk = 0; kk < RANK; ++kk) fma_tile(At + kk * m, Bs + kk * n_c);
+        } else {
+#pragma unroll 4
+          for (int kk = 0; kk < r; ++kk) fma_tile(At + kk * m, Bs + kk * n_c);
+        }
+      } else {
+        for (int k0 = 0; k0 < r; k0 += L.kc) {
+          const int kn = min(L.kc, r - k0);
           __syncthreads();
           for (int idx = tid; idx < kn * n_c; idx += kTileThreads) {
             const int kk = idx / n_c, jj = idx - kk * n_c;
@@ -201,100 +324,79 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
                                  : 0.0f;
           }
           __syncthreads();
-        }
-        const int boff = L.b_resident ? k0 : 0;
 #pragma unroll 4
-        for (int kk = 0; kk < kn; ++kk) {
-          const float* brow = Bs + (boff + kk) * n_c;
-          const float* arow = At + (k0 + kk) * m;
-#pragma unroll
-          for (int k = 0; k < kItemsPerThread; ++k) {
-            const int it = tid + k * kTileThreads;
-            if (it < nitems) {
-              const int g = it / quads, q = it - (it / quads) * quads;
-              const float4 a4 = *reinterpret_cast<const float4*>(arow + g * kRowsPerItem);
-              const float4 b4 = *reinterpret_cast<const float4*>(brow + 4 * q);
-              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-              const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-              for (int ml = 0; ml < kRowsPerItem; ++ml)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[k][ml][c] = fmaf(av[ml], bv[c], acc[k][ml][c]);
-            }
-          }
+          for (int kk = 0; kk < kn; ++kk) fma_tile(At + (k0 + kk) * m, Bs + kk * n_c);
         }
       }
     }
 
-    // ---- phase A.3: R*, the value to quantize, row maxima
+    // ---- phase A.3: R*, the value to quantize, and the row maxima
 #pragma unroll
-    for (int k = 0; k < kItemsPerThread; ++k) {
-      const int it = tid + k * kTileThreads;
-      const int g = it / quads, q = it - (it / quads) * quads;
-      const int jl = 4 * q;
-      const int vcols = min(4, ncols - jl);
-      uint32_t mx[kRowsPerItem], nm[kRowsPerItem];
+    for (int k = 0; k < IPT; ++k) {
+      float hi[RPI], lo[RPI];
 #pragma unroll
-      for (int ml = 0; ml < kRowsPerItem; ++ml) {
-        mx[ml] = 0u;
-        nm[ml] = 0u;
-        const int rr = g * kRowsPerItem + ml;
-        const bool ok = it < nitems && rr < rows && vcols > 0;
-        if (!ok) {
+      for (int ml = 0; ml < RPI; ++ml) hi[ml] = lo[ml] = 0.0f;
+      if (iok[k]) {
+        const int jl = 4 * iq[k];
+        const int vcols = ALIGNED ? 4 : min(4, ncols - jl);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[k][ml][c] = 0.0f;
-          continue;
-        }
-        const int64_t i = row0 + rr;
-        const int64_t e0 = i * L.n + col0 + jl;
-        uint32_t words[4];
-        if (aligned) {
-          const uint4 w4 = aux_block(static_cast<uint64_t>(e0) >> 2, L.stream_id, L.key0, L.key1);
-          words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
-        } else {
+        for (int ml = 0; ml < RPI; ++ml) {
+          const int rr = ig[k] * RPI + ml;
+          const bool row_ok = rr < rows;
+          const int64_t e0 = (row0 + min(rr, rows - 1)) * L.n + col0 + jl;
+          uint32_t words[4];
+          if (ALIGNED) {
+            const uint4 w4 = aux_block(static_cast<uint64_t>(e0) >> 2, L.stream_id, L.key0, L.key1);
+            words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
+          } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            words[c] = c < vcols ? aux_word(static_cast<uint64_t>(e0 + c), L.stream_id, L.key0,
-                                            L.key1)
-                                 : 0u;
-        }
-        float sv = 0.0f;
-        int32_t zv = 0;
-        if (VARIANT != kGen) {
-          sv = row_s[rr];
-          zv = row_z[rr];
-        }
+            for (int c = 0; c < 4; ++c)
+              words[c] = c < vcols ? aux_word(static_cast<uint64_t>(e0 + c), L.stream_id, L.key0,
+                                              L.key1)
+                                   : 0u;
+          }
+          float sv = 0.0f;
+          int32_t zv = 0;
+          if (VARIANT != kGen) {
+            sv = row_s[rr];
+            zv = row_z[rr];
+          }
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v = 0.0f;
-          if (c < vcols) {
-            const float rs = laplace_scaled(words[c], c_ln2);
+          for (int c = 0; c < 4; ++c) {
+            const float lg = laplace_log2(words[c]);
+            const float cs = laplace_sign(words[c], c_ln2);   // +-c ln2
+            float v;
             if (VARIANT == kGen) {
-              if (L.r_star_out != nullptr) L.r_star_out[e0 + c] = rs;
-              v = acc[k][ml][c] - rs;
+              if (L.r_star_out != nullptr && row_ok && (ALIGNED || c < vcols))
+                L.r_star_out[e0 + c] = lg * cs;
+              v = fmaf(-lg, cs, acc[k][ml][c]);                // W - R*
             } else {
               const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
-              v = fmaf(acc[k][ml][c] + rs, rcp_tab[dcode + 255], sv);
+              v = fmaf(fmaf(lg, cs, acc[k][ml][c]), rcp_tab[dcode + 255], sv);
             }
-          }
-          acc[k][ml][c] = v;
-          if (VARIANT == kShift) {
-            mx[ml] = max(mx[ml], __float_as_uint(fabsf(v)));
-          } else {
-            mx[ml] = max(mx[ml], nonneg_bits(v));
-            nm[ml] = max(nm[ml], nonneg_bits(-v));
+            const bool ok = row_ok && (ALIGNED || c < vcols);
+            v = ok ? v : 0.0f;
+            acc[k][ml][c] = v;
+            if (VARIANT == kShift) {
+              hi[ml] = fmaxf(hi[ml], fabsf(v));
+            } else {
+              hi[ml] = fmaxf(hi[ml], v);
+              lo[ml] = fminf(lo[ml], v);
+            }
           }
         }
       }
-      // reduce over lanes holding the same rows, then one atomic per group
-      const int key = it < nitems ? g : -1;
+      // reduce over the lanes holding the same rows, then one atomic per group
+      const int key = iok[k] ? ig[k] : -1;
       const unsigned peers = __match_any_sync(0xffffffffu, key);
       const int leader = __ffs(peers) - 1;
 #pragma unroll
-      for (int ml = 0; ml < kRowsPerItem; ++ml) {
-        const uint32_t a = __reduce_max_sync(peers, mx[ml]);
-        const uint32_t b = (VARIANT == kShift) ? 0u : __reduce_max_sync(peers, nm[ml]);
-        const int rr = g * kRowsPerItem + ml;
+      for (int ml = 0; ml < RPI; ++ml) {
+        // hi >= 0 >= lo in value; fabsf drops a possible -0.0, whose bit
+        // pattern would otherwise win the unsigned maximum
+        const uint32_t a = __reduce_max_sync(peers, ord(fabsf(hi[ml])));
+        const uint32_t b = (VARIANT == kShift) ? 0u : __reduce_max_sync(peers, ord(fabsf(lo[ml])));
+        const int rr = ig[k] * RPI + ml;
         if (lane == leader && key >= 0 && rr < rows) {
           atomicMax(&slots[(buf * kMaxTileRows + rr) * 2 + 0], a);
           if (VARIANT != kShift) atomicMax(&slots[(buf * kMaxTileRows + rr) * 2 + 1], b);
@@ -324,21 +426,20 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
         a = sp[0];
         b = sp[1];
       }
-      const float hi = __uint_as_float(a), neg_lo = __uint_as_float(b);
-      float scale, inv;
+      const float top = __uint_as_float(a), neg_bottom = __uint_as_float(b);
+      float scale;
       int32_t zero = 0;
       if (VARIANT == kShift) {
-        scale = hi > 0.0f ? hi : 1.0f;
+        scale = top > 0.0f ? top : 1.0f;
       } else {
-        scale = __fdiv_rn(hi + neg_lo, static_cast<float>(qmax));
+        scale = __fdiv_rn(top + neg_bottom, static_cast<float>(qmax));
         if (scale > 0.0f) {
-          zero = clamp_i(static_cast<int32_t>(rintf(__fdiv_rn(neg_lo, scale))), 0, qmax);
+          zero = clamp_i(static_cast<int32_t>(rintf(__fdiv_rn(neg_bottom, scale))), 0, qmax);
         } else {
           scale = 1.0f;
         }
       }
-      inv = __frcp_rn(scale);
-      q_inv[rr] = inv;
+      q_inv[rr] = __frcp_rn(scale);
       q_zero[rr] = zero;
       if (crank == 0) {
         if (L.scale_out != nullptr) L.scale_out[row0 + rr] = scale;
@@ -349,22 +450,21 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
 
     // ---- phase B: quantize from registers and store
 #pragma unroll
-    for (int k = 0; k < kItemsPerThread; ++k) {
-      const int it = tid + k * kTileThreads;
-      const int g = it / quads, q = it - (it / quads) * quads;
-      const int jl = 4 * q;
-      const int vcols = min(4, ncols - jl);
+    for (int k = 0; k < IPT; ++k) {
+      if (!iok[k]) continue;
+      const int jl = 4 * iq[k];
+      const int vcols = ALIGNED ? 4 : min(4, ncols - jl);
+      const int64_t j = col0 + jl;
 #pragma unroll
-      for (int ml = 0; ml < kRowsPerItem; ++ml) {
-        const int rr = g * kRowsPerItem + ml;
-        if (!(it < nitems && rr < rows && vcols > 0)) continue;
+      for (int ml = 0; ml < RPI; ++ml) {
+        const int rr = ig[k] * RPI + ml;
+        if (rr >= rows) continue;
         const int64_t i = row0 + rr;
-        const int64_t j = col0 + jl;
         const float inv = q_inv[rr];
         const int32_t zero = q_zero[rr];
+        const int32_t zv = VARIANT == kGen ? 0 : row_z[rr];
         int32_t res[4];
         uint32_t code8[4];
-        const int32_t zv = VARIANT == kGen ? 0 : row_z[rr];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const float v = acc[k][ml][c];
@@ -375,88 +475,17 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
             const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
             res[c] = sgn * (dcode >> sh);
             code8[c] = static_cast<uint32_t>(sh);
+          } else if (VARIANT == kMul) {
+            const int32_t centred = clamp_i(rne_scaled(v, inv), -zero, qmax - zero);
+            const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
+            res[c] = centred * dcode;
+            code8[c] = static_cast<uint32_t>(centred + zero);
           } else {
-            const int32_t qc = clamp_i(rne_scaled(v, inv) + zero, 0, qmax);
-            code8[c] = static_cast<uint32_t>(qc);
-            if (VARIANT == kMul) {
-              const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
-              res[c] = (qc - zero) * dcode;
-            } else {
-              res[c] = qc;
-            }
+            code8[c] = static_cast<uint32_t>(clamp_i(rne_scaled(v, inv) + zero, 0, qmax));
+            res[c] = 0;
           }
         }
-        if (VARIANT == kGen) {
-          if (L.out == nullptr) continue;
-          uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
-          if (WBITS == 8) {
-            const uint32_t packed = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
-            if (vcols == 4) {
-              *reinterpret_cast<uint32_t*>(orow + j) = packed;
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < vcols) orow[j + c] = static_cast<uint8_t>(code8[c]);
-            }
-          } else {
-            const uint32_t packed = code8[0] | (code8[1] << 4) | (code8[2] << 8) | (code8[3] << 12);
-            if (vcols == 4) {
-              *reinterpret_cast<uint16_t*>(orow + (j >> 1)) = static_cast<uint16_t>(packed);
-            } else {
-              // n is even for 4-bit codes, so a ragged quad holds exactly 2 columns
-              orow[j >> 1] = static_cast<uint8_t>(packed & 0xFFu);
-            }
-          }
-        } else {
-          const int64_t e0 = i * L.n + j;
-          const bool vec = aligned && vcols == 4;
-          if (p.out_bytes == 4) {   // MUL products beyond the int16 bound
-            int32_t* o = static_cast<int32_t*>(L.out) + e0;
-            if (vec) *reinterpret_cast<int4*>(o) = make_int4(res[0], res[1], res[2], res[3]);
-            else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < vcols) o[c] = res[c];
-            }
-          } else if (p.out_bytes == 2) {   // int16 products or merged codes
-            int16_t* o = static_cast<int16_t*>(L.out) + e0;
-            if (vec) {
-              const uint32_t lo = (static_cast<uint32_t>(res[0]) & 0xFFFFu) |
-                                  (static_cast<uint32_t>(res[1]) << 16);
-              const uint32_t hi = (static_cast<uint32_t>(res[2]) & 0xFFFFu) |
-                                  (static_cast<uint32_t>(res[3]) << 16);
-              *reinterpret_cast<uint2*>(o) = make_uint2(lo, hi);
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < vcols) o[c] = static_cast<int16_t>(res[c]);
-            }
-          } else {   // int8 merged codes (SHIFT with a base of at most 7 bits)
-            int8_t* o = static_cast<int8_t*>(L.out) + e0;
-            if (vec) {
-              const uint32_t packed = (static_cast<uint32_t>(res[0]) & 0xFFu) |
-                                      ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
-                                      ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) |
-                                      (static_cast<uint32_t>(res[3]) << 24);
-              *reinterpret_cast<uint32_t*>(o) = packed;
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < vcols) o[c] = static_cast<int8_t>(res[c]);
-            }
-          }
-          if (L.code_out != nullptr) {
-            uint8_t* co = L.code_out + e0;
-            if (vec) {
-              *reinterpret_cast<uint32_t*>(co) =
-                  code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
-            } else {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                if (c < vcols) co[c] = static_cast<uint8_t>(code8[c]);
-            }
-          }
-        }
+        store_item<VARIANT, WBITS, ALIGNED>(L, p.out_bytes, i, j, vcols, res, code8);
       }
     }
   }
@@ -467,9 +496,9 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
   }
 }
 
-template <int VARIANT, int WBITS, int RANK>
+template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
 cudaError_t launch_one(const TileBatch& b, cudaStream_t s) {
-  auto kern = tile_kernel<VARIANT, WBITS, RANK>;
+  auto kern = tile_kernel<VARIANT, WBITS, RANK, ALIGNED>;
   const size_t smem = static_cast<size_t>(layout_for(VARIANT).total_words()) * 4;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -493,9 +522,9 @@ cudaError_t launch_one(const TileBatch& b, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, b);
 }
 
-template <int VARIANT, int WBITS, int RANK>
+template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
 int max_clusters_one(int cluster) {
-  auto kern = tile_kernel<VARIANT, WBITS, RANK>;
+  auto kern = tile_kernel<VARIANT, WBITS, RANK, ALIGNED>;
   const size_t smem = static_cast<size_t>(layout_for(VARIANT).total_words()) * 4;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
@@ -522,25 +551,46 @@ int max_clusters_one(int cluster) {
   return n;
 }
 
-template <int VARIANT, int WBITS>
+template <int VARIANT, int WBITS, bool ALIGNED>
 cudaError_t dispatch_rank(const TileBatch& b, int rank_ct, cudaStream_t s) {
   switch (rank_ct) {
-    case 4: return launch_one<VARIANT, WBITS, 4>(b, s);
-    case 8: return launch_one<VARIANT, WBITS, 8>(b, s);
-    case 16: return launch_one<VARIANT, WBITS, 16>(b, s);
-    case 32: return launch_one<VARIANT, WBITS, 32>(b, s);
-    default: return launch_one<VARIANT, WBITS, 0>(b, s);
+    case 4: return launch_one<VARIANT, WBITS, 4, ALIGNED>(b, s);
+    case 8: return launch_one<VARIANT, WBITS, 8, ALIGNED>(b, s);
+    case 16: return launch_one<VARIANT, WBITS, 16, ALIGNED>(b, s);
+    case 32: return launch_one<VARIANT, WBITS, 32, ALIGNED>(b, s);
+    default: return launch_one<VARIANT, WBITS, 0, ALIGNED>(b, s);
   }
 }
 
-template <int VARIANT, int WBITS>
+template <int VARIANT, int WBITS, bool ALIGNED>
 int clusters_rank(int rank_ct, int cluster) {
   switch (rank_ct) {
-    case 4: return max_clusters_one<VARIANT, WBITS, 4>(cluster);
-    case 8: return max_clusters_one<VARIANT, WBITS, 8>(cluster);
-    case 16: return max_clusters_one<VARIANT, WBITS, 16>(cluster);
-    case 32: return max_clusters_one<VARIANT, WBITS, 32>(cluster);
-    default: return max_clusters_one<VARIANT, WBITS, 0>(cluster);
+    case 4: return max_clusters_one<VARIANT, WBITS, 4, ALIGNED>(cluster);
+    case 8: return max_clusters_one<VARIANT, WBITS, 8, ALIGNED>(cluster);
+    case 16: return max_clusters_one<VARIANT, WBITS, 16, ALIGNED>(cluster);
+    case 32: return max_clusters_one<VARIANT, WBITS, 32, ALIGNED>(cluster);
+    default: return max_clusters_one<VARIANT, WBITS, 0, ALIGNED>(cluster);
+  }
+}
+
+template <int VARIANT, bool ALIGNED>
+cudaError_t dispatch_bits(const TileBatch& b, int wb, int rank_ct, cudaStream_t s) {
+  if constexpr (VARIANT == kGen) {
+    return wb == 8 ? launch_one<kGen, 8, 0, ALIGNED>(b, s) : launch_one<kGen, 4, 0, ALIGNED>(b, s);
+  } else {
+    return wb == 8 ? dispatch_rank<VARIANT, 8, ALIGNED>(b, rank_ct, s)
+                   : dispatch_rank<VARIANT, 4, ALIGNED>(b, rank_ct, s);
+  }
+}
+
+template <int VARIANT, bool ALIGNED>
+int clusters_bits(int wb, int rank_ct, int cluster) {
+  if constexpr (VARIANT == kGen) {
+    return wb == 8 ? max_clusters_one<kGen, 8, 0, ALIGNED>(cluster)
+                   : max_clusters_one<kGen, 4, 0, ALIGNED>(cluster);
+  } else {
+    return wb == 8 ? clusters_rank<VARIANT, 8, ALIGNED>(rank_ct, cluster)
+                   : clusters_rank<VARIANT, 4, ALIGNED>(rank_ct, cluster);
   }
 }
 
@@ -548,24 +598,26 @@ int clusters_rank(int rank_ct, int cluster) {
 
 size_t tile_kernel_smem_bytes() { return static_cast<size_t>(layout_for(kMul).total_words()) * 4; }
 
-cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, cudaStream_t s) {
+cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s) {
   const int wb = variant == kGen ? b.bits : b.w_bits;
-  if (variant == kGen) {
-    return wb == 8 ? launch_one<kGen, 8, 0>(b, s) : launch_one<kGen, 4, 0>(b, s);
-  }
-  if (variant == kMul) {
-    return wb == 8 ? dispatch_rank<kMul, 8>(b, rank_ct, s) : dispatch_rank<kMul, 4>(b, rank_ct, s);
-  }
-  return wb == 8 ? dispatch_rank<kShift, 8>(b, rank_ct, s) : dispatch_rank<kShift, 4>(b, rank_ct, s);
+  if (variant == kGen)
+    return aligned ? dispatch_bits<kGen, true>(b, wb, 0, s) : dispatch_bits<kGen, false>(b, wb, 0, s);
+  if (variant == kMul)
+    return aligned ? dispatch_bits<kMul, true>(b, wb, rank_ct, s)
+                   : dispatch_bits<kMul, false>(b, wb, rank_ct, s);
+  return aligned ? dispatch_bits<kShift, true>(b, wb, rank_ct, s)
+                 : dispatch_bits<kShift, false>(b, wb, rank_ct, s);
 }
 
-int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int cluster) {
+int tile_max_active_clusters(int variant, int w_bits, int rank_ct, bool aligned, int cluster) {
   if (variant == kGen)
-    return w_bits == 8 ? max_clusters_one<kGen, 8, 0>(cluster) : max_clusters_one<kGen, 4, 0>(cluster);
+    return aligned ? clusters_bits<kGen, true>(w_bits, 0, cluster)
+                   : clusters_bits<kGen, false>(w_bits, 0, cluster);
   if (variant == kMul)
-    return w_bits == 8 ? clusters_rank<kMul, 8>(rank_ct, cluster) : clusters_rank<kMul, 4>(rank_ct, cluster);
-  return w_bits == 8 ? clusters_rank<kShift, 8>(rank_ct, cluster)
-                     : clusters_rank<kShift, 4>(rank_ct, cluster);
+    return aligned ? clusters_bits<kMul, true>(w_bits, rank_ct, cluster)
+                   : clusters_bits<kMul, false>(w_bits, rank_ct, cluster);
+  return aligned ? clusters_bits<kShift, true>(w_bits, rank_ct, cluster)
+                 : clusters_bits<kShift, false>(w_bits, rank_ct, cluster);
 }
 
 }  // namespace intlora

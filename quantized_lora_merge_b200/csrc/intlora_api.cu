@@ -55,18 +55,20 @@ size_t stats_partial_bytes(int64_t numel) { return round256(static_cast<size_t>(
 // ------------------------------------------------------------------------
 // tile geometry: cluster size, column slice, rows per tile
 // ------------------------------------------------------------------------
-int max_active_clusters_cached(int variant, int w_bits, int rank_ct, bool aligned, int cluster) {
+int max_active_clusters_cached(int variant, int w_bits, int rank_ct, int out_bytes, bool aligned,
+                               int cluster, size_t smem) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
+  static std::map<std::tuple<int, int, int, int, int, int, size_t>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, aligned ? 1 : 0, cluster);
+  const auto key = std::make_tuple(dev, variant * 16 + w_bits, rank_ct, out_bytes, aligned ? 1 : 0,
+                                   cluster, smem);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
   }
-  const int v = tile_max_active_clusters(variant, w_bits, rank_ct, aligned, cluster);
+  const int v = tile_max_active_clusters(variant, w_bits, rank_ct, out_bytes, aligned, cluster, smem);
   std::lock_guard<std::mutex> lock(mu);
   cache[key] = v;
   return v;
@@ -74,81 +76,123 @@ int max_active_clusters_cached(int variant, int w_bits, int rank_ct, bool aligne
 
 int slice_cols(int64_t n, int cluster) { return static_cast<int>(ceil_div(ceil_div(n, cluster), 4) * 4); }
 
-// Fill n_c, m, b_resident, kc, aligned and tile_begin of every layer for a
-// cluster size; returns the total number of tiles or -1 if a slice is too wide.
-int64_t plan_layers(int variant, std::vector<TileLayer>& L, int cluster, bool* all_resident) {
-  int64_t tiles = 0;
-  bool resident = true;
+// Shared memory an SM offers to `occ` CTAs of the tile kernel (B200: 228 KB
+// per SM, 1 KB reserved per CTA, 227 KB per CTA at most).
+constexpr int64_t kSmemPerSm = 233472;
+constexpr int64_t kSmemPerCtaMax = 232448;
+constexpr int kMiscWords = 512 + 8 * kMaxTileRows;
+
+// Geometry of every layer for one (cluster, occupancy) choice. Returns false
+// when the slices do not fit. B stays resident when `resident` is asked for.
+// *efficiency receives the element-weighted fraction of thread slots that do
+// useful work in the item loops (the tile's items spread over kTileThreads).
+bool plan_layers(int variant, std::vector<TileLayer>& L, int cluster, int occ, bool resident,
+                 TileBatch* b, int64_t* tiles_out, double* efficiency) {
+  const int64_t budget_words = (std::min(kSmemPerCtaMax, kSmemPerSm / occ - 1024) - 64) / 4;
+  int64_t max_nc = 0, max_b = 0, max_r = 1;
   for (auto& l : L) {
     const int n_c = slice_cols(l.n, cluster);
-    const int quads = n_c / 4;
-    if (quads > kMaxQuads) return -1;
-    int groups = std::max(1, kMaxQuads / quads);
-    int m = kRowsPerItem * groups;
-    m = std::min(m, kMaxTileRows);
+    max_nc = std::max<int64_t>(max_nc, n_c);
     if (variant != kGen) {
-      const int a_rows = (kASmemFloats / std::max(1, l.r)) / kRowsPerItem * kRowsPerItem;
-      m = std::min(m, std::max(kRowsPerItem, a_rows));
-      l.b_resident = static_cast<int64_t>(l.r) * n_c <= kBSmemFloats ? 1 : 0;
-      l.kc = std::max(1, kBSmemFloats / n_c);
-      resident = resident && l.b_resident;
-    } else {
-      l.b_resident = 0;
-      l.kc = 0;
+      max_r = std::max<int64_t>(max_r, l.r);
+      max_b = std::max<int64_t>(max_b, resident ? int64_t{l.r} * n_c : int64_t{n_c} * std::min(l.r, 8));
     }
-    // do not make tiles much taller than the layer
-    m = std::min<int64_t>(m, ceil_div(l.d, kRowsPerItem) * kRowsPerItem);
+  }
+  // rows of A a tile may stage: all kMaxTileRows up to rank 32, fewer above
+  const int64_t a_rows = variant == kGen ? kMaxTileRows
+      : std::min<int64_t>(kMaxTileRows, std::max<int64_t>(kRowsPerItem, (4096 / max_r) / 4 * 4));
+  const int64_t free_words = budget_words - max_b - (variant == kGen ? 0 : max_r * a_rows) - kMiscWords;
+  // merges stash one code word per 4 tile values next to the tile buffer
+  const int64_t u_words = (variant == kGen ? free_words : free_words * 4 / 5) / 16 * 16;
+  if (u_words < kRowsPerItem * max_nc) return false;
+  int64_t smem_a = 0, tiles = 0;
+  double useful = 0.0, total = 0.0;
+  for (auto& l : L) {
+    const int n_c = slice_cols(l.n, cluster);
+    const int64_t quads = n_c / 4;
+    int64_t gmax = std::min<int64_t>(u_words / n_c, std::min<int64_t>(kMaxTileRows, a_rows)) / kRowsPerItem;
+    gmax = std::max<int64_t>(1, std::min<int64_t>(gmax, ceil_div(l.d, kRowsPerItem)));
+    // rows per tile: the item count that fills whole rounds of the block best,
+    // then the largest such tile
+    int64_t best_g = 1;
+    double best_e = -1.0;
+    for (int64_t g = 1; g <= gmax; ++g) {
+      const int64_t items = g * quads;
+      const double e = static_cast<double>(items) / static_cast<double>(ceil_div(items, kTileThreads) * kTileThreads);
+      if (e > best_e + 1e-9 || (e > best_e - 1e-9 && g > best_g)) {
+        best_e = e;
+        best_g = g;
+      }
+    }
+    const int m = static_cast<int>(best_g * kRowsPerItem);
     l.n_c = n_c;
     l.m = m;
     l.aligned = (l.n % 4 == 0) ? 1 : 0;
+    if (variant != kGen) {
+      l.b_resident = resident ? 1 : 0;
+      l.kc = resident ? l.r : static_cast<int>(std::max<int64_t>(1, max_b / n_c));
+      smem_a = std::max<int64_t>(smem_a, int64_t{l.r} * m);
+    }
     l.tile_begin = tiles;
-    tiles += ceil_div(l.d, m);
+    const int64_t nt = ceil_div(l.d, m);
+    tiles += nt;
+    const double numel = static_cast<double>(l.d) * static_cast<double>(l.n);
+    useful += numel * best_e * (static_cast<double>(l.d) / static_cast<double>(nt * m));
+    total += numel;
   }
-  if (all_resident) *all_resident = resident;
-  return tiles;
+  b->smem_u = static_cast<int32_t>(u_words);
+  b->smem_b = static_cast<int32_t>(max_b);
+  b->smem_a = static_cast<int32_t>(smem_a);
+  *tiles_out = tiles;
+  if (efficiency) *efficiency = total > 0 ? useful / total : 0.0;
+  return true;
 }
 
 intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bits, int w_bits,
-                                 int out_bytes, cudaStream_t stream) {
+                                 int out_bytes, uint64_t seed, cudaStream_t stream) {
   int rank_ct = 0;
   if (variant != kGen) {
     rank_ct = L[0].r;
     for (auto& l : L)
       if (l.r != rank_ct) rank_ct = 0;
-    if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16 && rank_ct != 32) rank_ct = 0;
+    if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16) rank_ct = 0;
   }
   bool aligned = true;
   for (auto& l : L) aligned = aligned && (l.n % 4 == 0);
-  static const int kClusters[] = {1, 2, 4, 8, 16};
-  int chosen = -1;
-  int64_t total = -1;
-  // smallest cluster whose slices fit and keep B resident; else smallest that fits
-  for (int pass = 0; pass < 2 && chosen < 0; ++pass) {
-    for (int c : kClusters) {
-      bool resident = false;
-      const int64_t t = plan_layers(variant, L, c, &resident);
-      if (t < 0) continue;
-      if (pass == 0 && variant != kGen && !resident) continue;
-      if (max_active_clusters_cached(variant, w_bits, rank_ct, aligned, c) <= 0) continue;
-      chosen = c;
-      total = t;
-      break;
-    }
-  }
-  if (chosen < 0) return fail(INTLORA_ERR_UNSUPPORTED, "no launchable cluster size for this batch");
-  total = plan_layers(variant, L, chosen, nullptr);
   TileBatch b;
   std::memset(&b, 0, sizeof b);
+  static const int kClusters[] = {1, 2, 4, 8, 16};
+  bool found = false;
+  int64_t total = 0;
+  int max_clusters = 0;
+  // Prefer B resident, then more CTAs per SM, then the smaller cluster; the
+  // rows per tile of each layer are picked for balanced item rounds.
+  for (int pass = 0; pass < 2 && !found; ++pass) {
+    const bool resident = (pass == 0) || variant == kGen;
+    for (int occ = 3; occ >= 1 && !found; --occ) {
+      for (int c : kClusters) {
+        if (!plan_layers(variant, L, c, occ, resident, &b, &total, nullptr)) continue;
+        const size_t smem = tile_smem_bytes(variant, b.smem_u, b.smem_b, b.smem_a);
+        max_clusters = max_active_clusters_cached(variant, w_bits, rank_ct, out_bytes, aligned, c, smem);
+        if (max_clusters <= 0) continue;
+        b.cluster = c;
+        found = true;
+        break;
+      }
+    }
+  }
+  if (!found) return fail(INTLORA_ERR_UNSUPPORTED, "no launchable tile geometry for this batch");
   for (size_t k = 0; k < L.size(); ++k) b.layer[k] = L[k];
   b.count = static_cast<int32_t>(L.size());
-  b.cluster = chosen;
+  b.variant = variant;
   b.total_tiles = total;
-  b.num_clusters = static_cast<int32_t>(
-      std::min<int64_t>(total, max_active_clusters_cached(variant, w_bits, rank_ct, aligned, chosen)));
+  b.num_clusters = static_cast<int32_t>(std::min<int64_t>(total, max_clusters));
   b.bits = bits;
   b.w_bits = w_bits;
   b.out_bytes = out_bytes;
-  cudaError_t e = launch_tiles(variant, b, rank_ct, aligned, stream);
+  b.key0 = static_cast<uint32_t>(seed);
+  b.key1 = static_cast<uint32_t>(seed >> 32);
+  cudaError_t e = launch_tiles(b, rank_ct, aligned, stream);
   if (e != cudaSuccess) return cuda_fail(e, "row-tile kernel launch");
   return INTLORA_OK;
 }
@@ -194,62 +238,85 @@ size_t aux_ws_bytes(const intlora_aux_job* jobs, int32_t count) {
   return total;
 }
 
-// The three launches of one chunk of at most kMaxBatch jobs.
+// Indices of `count` items grouped by seed, in first-appearance order: every
+// launch carries one Philox key at batch level (uniform round keys).
+template <typename T>
+std::vector<std::vector<int32_t>> group_by_seed(const T* items, int32_t count) {
+  std::vector<uint64_t> seeds;
+  std::vector<std::vector<int32_t>> groups;
+  for (int32_t k = 0; k < count; ++k) {
+    size_t g = 0;
+    while (g < seeds.size() && seeds[g] != items[k].seed) ++g;
+    if (g == seeds.size()) {
+      seeds.push_back(items[k].seed);
+      groups.emplace_back();
+    }
+    groups[g].push_back(k);
+  }
+  return groups;
+}
+
+// The launches of one chunk of at most kMaxBatch jobs: per seed, statistics,
+// finalize and the base quantization (grouped by code width).
 intlora_status gen_aux_chunk(const intlora_aux_job* jobs, int32_t count, char* ws, cudaStream_t st) {
-  StatsBatch sb;
-  std::memset(&sb, 0, sizeof sb);
-  int64_t blocks = 0;
+  std::vector<size_t> offset(count);
   size_t off = 0;
   for (int32_t k = 0; k < count; ++k) {
-    const intlora_aux_job& j = jobs[k];
-    StatsJob& s = sb.job[k];
-    s.W = j.W;
-    s.numel = j.d * j.n;
-    s.key0 = lo32(j.seed);
-    s.key1 = hi32(j.seed);
-    s.stream_id = j.stream_id;
-    s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
-    s.block_begin = blocks;
-    s.partial = reinterpret_cast<double*>(ws + off);
-    s.sigma_w_out = j.sigma_w_out;
-    s.sigma_r_out = j.sigma_r_out;
-    blocks += s.nblocks;
-    off += stats_partial_bytes(s.numel);
+    offset[k] = off;
+    off += stats_partial_bytes(jobs[k].d * jobs[k].n);
   }
-  sb.count = count;
-  cudaError_t e = launch_stats(sb, blocks, st);
-  if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
-  e = launch_stats_finalize(sb, st);
-  if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
-
-  // base quantization for the jobs that want codes or R*, grouped by w_bits
-  for (int wb : {4, 8}) {
-    std::vector<TileLayer> L;
-    for (int32_t k = 0; k < count; ++k) {
-      const intlora_aux_job& j = jobs[k];
-      if (j.w_bits != wb || (j.w_round_out == nullptr && j.r_star_out == nullptr)) continue;
-      TileLayer l;
-      std::memset(&l, 0, sizeof l);
-      l.src = j.W;
-      l.ld_src = j.n * 4;
-      l.sigma_w = j.sigma_w_out;
-      l.sigma_r = j.sigma_r_out;
-      l.alpha = j.alpha;
-      l.key0 = lo32(j.seed);
-      l.key1 = hi32(j.seed);
-      l.stream_id = j.stream_id;
-      l.out = j.w_round_out;
-      l.ld_out = j.ld_w_out;
-      l.scale_out = j.s_out;
-      l.zero_out = j.z_out;
-      l.r_star_out = j.r_star_out;
-      l.d = j.d;
-      l.n = j.n;
-      L.push_back(l);
+  for (const auto& grp : group_by_seed(jobs, count)) {
+    StatsBatch sb;
+    std::memset(&sb, 0, sizeof sb);
+    int64_t blocks = 0;
+    for (size_t q = 0; q < grp.size(); ++q) {
+      const intlora_aux_job& j = jobs[grp[q]];
+      StatsJob& s = sb.job[q];
+      s.W = j.W;
+      s.numel = j.d * j.n;
+      s.stream_id = j.stream_id;
+      s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
+      s.block_begin = blocks;
+      s.partial = reinterpret_cast<double*>(ws + offset[grp[q]]);
+      s.sigma_w_out = j.sigma_w_out;
+      s.sigma_r_out = j.sigma_r_out;
+      blocks += s.nblocks;
     }
-    if (L.empty()) continue;
-    const intlora_status s = launch_tile_batch(kGen, L, wb, wb, 1, st);
-    if (s != INTLORA_OK) return s;
+    sb.count = static_cast<int32_t>(grp.size());
+    sb.key0 = lo32(jobs[grp[0]].seed);
+    sb.key1 = hi32(jobs[grp[0]].seed);
+    cudaError_t e = launch_stats(sb, blocks, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
+    e = launch_stats_finalize(sb, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
+
+    // base quantization for the jobs that want codes or R*, grouped by w_bits
+    for (int wb : {4, 8}) {
+      std::vector<TileLayer> L;
+      for (int32_t k : grp) {
+        const intlora_aux_job& j = jobs[k];
+        if (j.w_bits != wb || (j.w_round_out == nullptr && j.r_star_out == nullptr)) continue;
+        TileLayer l;
+        std::memset(&l, 0, sizeof l);
+        l.src = j.W;
+        l.ld_src = j.n * 4;
+        l.sigma_w = j.sigma_w_out;
+        l.sigma_r = j.sigma_r_out;
+        l.alpha = j.alpha;
+        l.stream_id = j.stream_id;
+        l.out = j.w_round_out;
+        l.ld_out = j.ld_w_out;
+        l.scale_out = j.s_out;
+        l.zero_out = j.z_out;
+        l.r_star_out = j.r_star_out;
+        l.d = j.d;
+        l.n = j.n;
+        L.push_back(l);
+      }
+      if (L.empty()) continue;
+      const intlora_status s = launch_tile_batch(kGen, L, wb, wb, 1, jobs[grp[0]].seed, st);
+      if (s != INTLORA_OK) return s;
+    }
   }
   return INTLORA_OK;
 }
@@ -309,71 +376,76 @@ int32_t out_bytes_for(int variant, int w_bits, int out_bits) {
 
 intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlora_merge_out* outs,
                            int32_t count, int32_t bits, char* ws, cudaStream_t st) {
-  // sigma_R on the device for layers that did not pass it in
-  StatsBatch sb;
-  std::memset(&sb, 0, sizeof sb);
-  int32_t ns = 0;
-  int64_t blocks = 0;
-  size_t off = 0;
   std::vector<const double*> sig_r(count);
+  std::vector<size_t> offset(count);
+  size_t off = 0;
   for (int32_t k = 0; k < count; ++k) {
     sig_r[k] = layers[k].sigma_r;
-    if (layers[k].sigma_r != nullptr) continue;
-    StatsJob& s = sb.job[ns++];
-    s.W = nullptr;
-    s.numel = layers[k].d * layers[k].n;
-    s.key0 = lo32(layers[k].seed);
-    s.key1 = hi32(layers[k].seed);
-    s.stream_id = layers[k].stream_id;
-    s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
-    s.block_begin = blocks;
-    s.sigma_w_out = nullptr;
-    s.sigma_r_out = reinterpret_cast<double*>(ws + off);
-    s.partial = reinterpret_cast<double*>(ws + off + 256);
-    sig_r[k] = s.sigma_r_out;
-    blocks += s.nblocks;
-    off += 256 + stats_partial_bytes(s.numel);
+    offset[k] = off;
+    if (layers[k].sigma_r == nullptr) off += 256 + stats_partial_bytes(layers[k].d * layers[k].n);
   }
-  if (ns > 0) {
-    sb.count = ns;
-    cudaError_t e = launch_stats(sb, blocks, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
-    e = launch_stats_finalize(sb, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
-  }
-  for (int wb : {4, 8}) {
-    std::vector<TileLayer> L;
-    for (int32_t k = 0; k < count; ++k) {
-      const intlora_layer& y = layers[k];
-      if (y.w_bits != wb) continue;
-      TileLayer l;
-      std::memset(&l, 0, sizeof l);
-      l.src = y.w_round;
-      l.ld_src = y.ld_w;
-      l.s = y.s;
-      l.z = y.z;
-      l.A = y.A;
-      l.B = y.B;
-      l.sigma_w = y.sigma_w;
-      l.sigma_r = sig_r[k];
-      l.alpha = y.alpha;
-      l.key0 = lo32(y.seed);
-      l.key1 = hi32(y.seed);
-      l.stream_id = y.stream_id;
-      l.out = outs[k].out;
-      l.ld_out = y.n;
-      l.scale_out = outs[k].sbar;
-      l.zero_out = variant == kMul ? outs[k].zbar : nullptr;
-      l.code_out = outs[k].code;
-      l.d = y.d;
-      l.n = y.n;
-      l.r = y.r;
-      L.push_back(l);
+  for (const auto& grp : group_by_seed(layers, count)) {
+    // sigma_R on the device for layers that did not pass it in
+    StatsBatch sb;
+    std::memset(&sb, 0, sizeof sb);
+    int32_t ns = 0;
+    int64_t blocks = 0;
+    for (int32_t k : grp) {
+      if (layers[k].sigma_r != nullptr) continue;
+      StatsJob& s = sb.job[ns++];
+      s.W = nullptr;
+      s.numel = layers[k].d * layers[k].n;
+      s.stream_id = layers[k].stream_id;
+      s.nblocks = static_cast<int32_t>(stats_blocks(s.numel));
+      s.block_begin = blocks;
+      s.sigma_w_out = nullptr;
+      s.sigma_r_out = reinterpret_cast<double*>(ws + offset[k]);
+      s.partial = reinterpret_cast<double*>(ws + offset[k] + 256);
+      sig_r[k] = s.sigma_r_out;
+      blocks += s.nblocks;
     }
-    if (L.empty()) continue;
-    const intlora_status s = launch_tile_batch(variant, L, bits, wb,
-                                               out_bytes_for(variant == kMul ? 0 : 1, wb, bits), st);
-    if (s != INTLORA_OK) return s;
+    if (ns > 0) {
+      sb.count = ns;
+      sb.key0 = lo32(layers[grp[0]].seed);
+      sb.key1 = hi32(layers[grp[0]].seed);
+      cudaError_t e = launch_stats(sb, blocks, st);
+      if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
+      e = launch_stats_finalize(sb, st);
+      if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
+    }
+    for (int wb : {4, 8}) {
+      std::vector<TileLayer> L;
+      for (int32_t k : grp) {
+        const intlora_layer& y = layers[k];
+        if (y.w_bits != wb) continue;
+        TileLayer l;
+        std::memset(&l, 0, sizeof l);
+        l.src = y.w_round;
+        l.ld_src = y.ld_w;
+        l.s = y.s;
+        l.z = y.z;
+        l.A = y.A;
+        l.B = y.B;
+        l.sigma_w = y.sigma_w;
+        l.sigma_r = sig_r[k];
+        l.alpha = y.alpha;
+        l.stream_id = y.stream_id;
+        l.out = outs[k].out;
+        l.ld_out = y.n;
+        l.scale_out = outs[k].sbar;
+        l.zero_out = variant == kMul ? outs[k].zbar : nullptr;
+        l.code_out = outs[k].code;
+        l.d = y.d;
+        l.n = y.n;
+        l.r = y.r;
+        L.push_back(l);
+      }
+      if (L.empty()) continue;
+      const intlora_status s = launch_tile_batch(variant, L, bits, wb,
+                                                 out_bytes_for(variant == kMul ? 0 : 1, wb, bits),
+                                                 layers[grp[0]].seed, st);
+      if (s != INTLORA_OK) return s;
+    }
   }
   return INTLORA_OK;
 }
@@ -424,6 +496,44 @@ intlora_status check_ste(const intlora_ste_job& j, int idx) {
 constexpr int kSteBM = 64, kSteRB = 32, kSteTargetCtas = 148 * 4;
 
 intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_t st) {
+  // Ranks up to 8 with n % 8 == 0: one fused pass over G (both outputs).
+  int max_r = 0;
+  bool fusable = true;
+  for (int32_t k = 0; k < count; ++k) {
+    max_r = std::max(max_r, jobs[k].r);
+    fusable = fusable && jobs[k].n % 8 == 0;
+  }
+  fusable = fusable && max_r <= 8;
+  if (fusable) {
+    SteBatch b;
+    std::memset(&b, 0, sizeof b);
+    int64_t tiles = 0;
+    for (int32_t k = 0; k < count; ++k) {
+      const intlora_ste_job& j = jobs[k];
+      SteJob& s = b.job[k];
+      s.G = static_cast<const uint16_t*>(j.G);
+      s.A = static_cast<const uint16_t*>(j.A);
+      s.B = static_cast<const uint16_t*>(j.B);
+      s.d = j.d;
+      s.n = j.n;
+      s.r = j.r;
+      s.dA = j.dA;
+      s.dB = j.dB;
+      const int64_t strips = ceil_div(j.n, 128);
+      // row ranges of at least 256 rows, enough CTAs to fill the GPU a few times
+      int64_t ranges = std::max<int64_t>(1, ceil_div(kSteTargetCtas * 2, strips));
+      ranges = std::min<int64_t>(ranges, std::max<int64_t>(1, ceil_div(j.d, 256)));
+      s.ksplit = static_cast<int32_t>(ranges);
+      s.tile_begin = tiles;
+      tiles += strips * ranges;
+    }
+    b.count = count;
+    b.fused = max_r <= 4 ? 4 : 8;
+    b.total_tiles = tiles;
+    cudaError_t e = launch_ste(b, st);
+    if (e != cudaSuccess) return cuda_fail(e, "STE kernel launch");
+    return INTLORA_OK;
+  }
   for (int dir = 0; dir < 2; ++dir) {
     SteBatch b;
     std::memset(&b, 0, sizeof b);

@@ -19,7 +19,7 @@ constexpr int kMaxBatch = 128;          // descriptors per launch
 struct StatsJob {
   const float* W;            // nullptr: R statistics only
   int64_t numel;
-  uint32_t key0, key1, stream_id;
+  uint32_t stream_id;        // Philox counter word 2 (the key is batch level)
   int32_t nblocks;           // CTAs working on this job
   int64_t block_begin;       // index of the job's first CTA in the grid
   double* partial;           // [nblocks][4]: sum(w-K), sum((w-K)^2), sum R, sum R^2
@@ -29,6 +29,8 @@ struct StatsJob {
 struct StatsBatch {
   StatsJob job[kMaxBatch];
   int32_t count;
+  uint32_t key0, key1;       // Philox key shared by every job of the batch (kept
+                             // at batch level so the round keys stay uniform)
 };
 
 // ---------------------------------------------------------------------------
@@ -51,7 +53,7 @@ struct TileLayer {
   const double* sigma_w;
   const double* sigma_r;
   float alpha;
-  uint32_t key0, key1, stream_id;
+  uint32_t stream_id;        // Philox counter word 2 (the key is batch level)
   // outputs
   void* out;                 // kGen: codes; kMul: P; kShift: M
   int64_t ld_out;            // kGen: bytes per code row; merges: elements (= n)
@@ -72,23 +74,25 @@ struct TileLayer {
 struct TileBatch {
   TileLayer layer[kMaxBatch];
   int32_t count;
+  uint32_t key0, key1;       // Philox key shared by every layer of the batch
+  int32_t variant;           // kGen, kMul or kShift
   int32_t cluster;           // C
   int32_t num_clusters;
   int64_t total_tiles;
   int32_t bits;              // kGen: w_bits; kMul: u_bits; kShift: shift_bits
   int32_t w_bits;            // code width of the input W_round (merges)
   int32_t out_bytes;         // merges: bytes per element of `out` (1, 2 or 4)
+  int32_t smem_u;            // floats of the tile buffer (>= m n_c of every layer)
+  int32_t smem_b;            // floats of the B buffer
+  int32_t smem_a;            // floats of the A-rows buffer (>= r m)
 };
 
 constexpr int kTileThreads = 256;
 constexpr int kRowsPerItem = 4;                     // rows of one work item
-constexpr int kItemsPerThread = 3;
-constexpr int kMaxQuads = kTileThreads * kItemsPerThread;   // 4-column groups per tile
 constexpr int kMaxTileRows = 128;
-constexpr int kBSmemFloats = 16384;                 // B slice capacity (64 KB)
-constexpr int kASmemFloats = 8192;                  // A rows of a tile (32 KB)
 
-size_t tile_kernel_smem_bytes();
+// Dynamic shared memory of a tile launch with the given carve-up.
+size_t tile_smem_bytes(int variant, int smem_u, int smem_b, int smem_a);
 
 // ---------------------------------------------------------------------------
 // STE backward.
@@ -102,20 +106,23 @@ struct SteJob {
   float* dA;
   float* dB;
   int64_t tile_begin;        // first CTA of this job in the grid
-  int32_t ksplit;            // CTAs sharing one output tile (split reduction)
+  int32_t ksplit;            // CTAs sharing one output tile (split reduction); fused
+                             // pass: row ranges per column strip
 };
 struct SteBatch {
   SteJob job[kMaxBatch];
   int32_t count;
   int32_t transposed;        // 0: dA = G B^T; 1: dB^T = G^T A
+  int32_t fused;             // 4 or 8: one fused pass (both outputs) at that rank bound
   int64_t total_tiles;
 };
 
 // Launchers: return the cudaError_t of the launch.
 cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t s);
 cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s);
-cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s);
-int tile_max_active_clusters(int variant, int w_bits, int rank_ct, bool aligned, int cluster);
+cudaError_t launch_tiles(const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s);
+int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes, bool aligned,
+                             int cluster, size_t smem);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 

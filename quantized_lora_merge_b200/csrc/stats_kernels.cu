@@ -44,8 +44,8 @@ struct GroupSums {
 
 template <bool HAS_W>
 __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64_t group, float K,
-                                          int valid) {
-  const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, J.key0, J.key1);
+                                          int valid, uint32_t k0, uint32_t k1) {
+  const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
   float x[4] = {0.f, 0.f, 0.f, 0.f};
   if (HAS_W) {
@@ -72,7 +72,8 @@ __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64
 }
 
 template <bool HAS_W>
-__device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4]) {
+__device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4],
+                                           uint32_t k0, uint32_t k1) {
   constexpr int kFlush = 8;   // groups per fp32 partial
   const int64_t full = J.numel >> 2;                 // complete groups
   const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
@@ -81,7 +82,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   while (g < full) {
     GroupSums s;
 #pragma unroll 2
-    for (int u = 0; u < kFlush && g < full; ++u, g += stride) add_group<HAS_W>(s, J, g, K, 4);
+    for (int u = 0; u < kFlush && g < full; ++u, g += stride) add_group<HAS_W>(s, J, g, K, 4, k0, k1);
     acc[0] += static_cast<double>(s.w1);
     acc[1] += static_cast<double>(s.w2);
     acc[2] += static_cast<double>(s.r1);
@@ -90,7 +91,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
-    add_group<HAS_W>(s, J, full, K, tail);
+    add_group<HAS_W>(s, J, full, K, tail, k0, k1);
     acc[0] += static_cast<double>(s.w1);
     acc[1] += static_cast<double>(s.w2);
     acc[2] += static_cast<double>(s.r1);
@@ -106,8 +107,8 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_const
   const StatsJob& J = b.job[j];
   const int64_t local = bid - J.block_begin;
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  if (J.W != nullptr) stats_body<true>(J, local, acc);
-  else stats_body<false>(J, local, acc);
+  if (J.W != nullptr) stats_body<true>(J, local, acc, b.key0, b.key1);
+  else stats_body<false>(J, local, acc, b.key0, b.key1);
   block_sum4(acc, red);
   if (threadIdx.x == 0)
     for (int q = 0; q < 4; ++q) J.partial[local * 4 + q] = acc[q];

@@ -111,16 +111,159 @@ __global__ void __launch_bounds__(kSteThreads) ste_gemm_kernel(const __grid_cons
   }
 }
 
+// Fused single pass over G for ranks up to 8 (CUDA cores). A CTA owns a strip
+// of 128 columns and a range of rows; each lane owns 4 consecutive columns
+// (one 8-byte load of G per row), keeps B[:, its columns] and its dB partial
+// sums in registers, and forms the dA partial dot products of every row over
+// its columns, which a warp shuffle tree sums over the strip. Partial sums of
+// dA (per row and strip) and dB (per strip and row range) are added with fp32
+// atomics into the zero-initialized outputs. G is read exactly once.
+constexpr int kStripCols = 128;
+
+__device__ __forceinline__ void unpack_bf16x4(uint2 raw, float out[4]) {
+  out[0] = __uint_as_float(raw.x << 16);
+  out[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+  out[2] = __uint_as_float(raw.y << 16);
+  out[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+}
+
+// A[i, 0..RB) as floats (zero past r); one vector load when r == RB.
+template <int RB>
+__device__ __forceinline__ void load_a_row(const uint16_t* A, int64_t i, int r, float a[RB]) {
+  if (r == RB && RB == 4) {
+    unpack_bf16x4(__ldg(reinterpret_cast<const uint2*>(A + i * 4)), a);
+  } else if (r == RB && RB == 8) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(A + i * 8));
+    unpack_bf16x4(make_uint2(raw.x, raw.y), a);
+    unpack_bf16x4(make_uint2(raw.z, raw.w), a + 4);
+  } else {
+#pragma unroll
+    for (int k = 0; k < RB; ++k) a[k] = k < r ? bf16f(A[i * r + k]) : 0.0f;
+  }
+}
+
+// Sum over the 32 lanes of each of the 32 values v[0..31] that every lane
+// holds; lane L ends with the total of value index (L's bits in the order the
+// halvings visit them). 31 shuffles for 32 sums instead of 5 per sum.
+__device__ __forceinline__ float transpose_reduce32(float v[32], int lane) {
+#pragma unroll
+  for (int s = 16, half = 16; s >= 1; s >>= 1, half >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return v[0];
+}
+
+// Value index whose total lane L holds after transpose_reduce32: at the step
+// with shuffle distance s the lanes with bit s set keep the upper half.
+__device__ __forceinline__ int transpose_index(int lane) {
+  int idx = 0;
+#pragma unroll
+  for (int s = 16, half = 16; s >= 1; s >>= 1, half >>= 1)
+    if (lane & s) idx += half;
+  return idx;
+}
+
+template <int RB>
+__global__ void __launch_bounds__(kSteThreads, 2) ste_fused_kernel(const __grid_constant__ SteBatch b) {
+  int64_t t = blockIdx.x;
+  int j = 0;
+  while (j + 1 < b.count && b.job[j + 1].tile_begin <= t) ++j;
+  const SteJob& J = b.job[j];
+  t -= J.tile_begin;
+  const int64_t n = J.n;
+  const int r = J.r;
+  const uint16_t* __restrict__ G = J.G;
+  const uint16_t* __restrict__ A = J.A;
+  const int strips = static_cast<int>((n + kStripCols - 1) / kStripCols);
+  const int strip = static_cast<int>(t % strips);
+  const int rchunk = static_cast<int>(t / strips);
+  const int64_t rows_per = (J.d + J.ksplit - 1) / J.ksplit;
+  const int64_t i_begin = rchunk * rows_per;
+  const int64_t i_end = min64(J.d, i_begin + rows_per);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t c0 = static_cast<int64_t>(strip) * kStripCols + lane * 4;
+  const bool col_ok = c0 < n;               // n % 8 == 0: a lane's 4 columns are all in or out
+
+  float bv[RB][4];
+#pragma unroll
+  for (int k = 0; k < RB; ++k) {
+    if (k < r && col_ok) unpack_bf16x4(__ldg(reinterpret_cast<const uint2*>(J.B + static_cast<int64_t>(k) * n + c0)), bv[k]);
+    else bv[k][0] = bv[k][1] = bv[k][2] = bv[k][3] = 0.0f;
+  }
+  float dbacc[RB][4];
+#pragma unroll
+  for (int k = 0; k < RB; ++k) dbacc[k][0] = dbacc[k][1] = dbacc[k][2] = dbacc[k][3] = 0.0f;
+
+  // Rows in groups of RG = 32 / RB per warp: the RG x RB partial dot products
+  // of dA are summed over the lanes by one transpose-reduce.
+  constexpr int RG = 32 / RB;
+  constexpr int kWarps = kSteThreads / 32;
+  const int my_idx = transpose_index(lane);
+  const int my_row = my_idx / RB, my_k = my_idx % RB;
+  for (int64_t i0 = i_begin + warp * RG; i0 < i_end; i0 += kWarps * RG) {
+    float P[32];
+    // all RG rows of G are requested before any is used (RG loads in flight)
+    uint2 graw[RG];
+#pragma unroll
+    for (int u = 0; u < RG; ++u) {
+      const int64_t i = i0 + u;
+      graw[u] = (i < i_end && col_ok) ? __ldg(reinterpret_cast<const uint2*>(G + i * n + c0))
+                                      : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < RG; ++u) {
+      const int64_t i = i0 + u;
+      float a[RB];
+      if (i < i_end) load_a_row<RB>(A, i, r, a);
+      else
+#pragma unroll
+        for (int k = 0; k < RB; ++k) a[k] = 0.0f;
+      float g[4];
+      unpack_bf16x4(graw[u], g);
+#pragma unroll
+      for (int k = 0; k < RB; ++k) {
+        float acc = g[0] * bv[k][0];
+#pragma unroll
+        for (int c = 1; c < 4; ++c) acc = fmaf(g[c], bv[k][c], acc);
+        P[u * RB + k] = acc;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dbacc[k][c] = fmaf(a[k], g[c], dbacc[k][c]);
+      }
+    }
+    const float total = transpose_reduce32(P, lane);
+    const int64_t row = i0 + my_row;
+    if (row < i_end && my_k < r) atomicAdd(&J.dA[row * r + my_k], total);
+  }
+  if (col_ok) {
+#pragma unroll
+    for (int k = 0; k < RB; ++k) {
+      if (k >= r) break;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) atomicAdd(&J.dB[static_cast<int64_t>(k) * n + c0 + c], dbacc[k][c]);
+    }
+  }
+}
+
 // Zero the outputs that split-K CTAs accumulate into (one launch per batch).
 __global__ void ste_zero_kernel(const __grid_constant__ SteBatch b) {
   for (int j = 0; j < b.count; ++j) {
     const SteJob& J = b.job[j];
-    if (J.ksplit <= 1) continue;
-    float* p = b.transposed ? J.dB : J.dA;
-    const int64_t count = b.transposed ? static_cast<int64_t>(J.r) * J.n : J.d * J.r;
-    for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < count;
-         k += static_cast<int64_t>(gridDim.x) * blockDim.x)
-      p[k] = 0.0f;
+    const bool both = b.fused != 0;
+    for (int which = 0; which < 2; ++which) {
+      const bool is_db = which == 1;
+      if (!both && (J.ksplit <= 1 || is_db != (b.transposed != 0))) continue;
+      float* p = is_db ? J.dB : J.dA;
+      const int64_t count = is_db ? static_cast<int64_t>(J.r) * J.n : J.d * J.r;
+      for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < count;
+           k += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        p[k] = 0.0f;
+    }
   }
 }
 
@@ -128,6 +271,14 @@ __global__ void ste_zero_kernel(const __grid_constant__ SteBatch b) {
 
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s) {
   if (b.count <= 0) return cudaSuccess;
+  if (b.fused) {
+    ste_zero_kernel<<<148 * 4, 256, 0, s>>>(b);
+    if (b.fused == 4)
+      ste_fused_kernel<4><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
+    else
+      ste_fused_kernel<8><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
+    return cudaGetLastError();
+  }
   bool any_split = false;
   for (int j = 0; j < b.count; ++j) any_split = any_split || b.job[j].ksplit > 1;
   if (any_split) ste_zero_kernel<<<148 * 4, 256, 0, s>>>(b);

@@ -12,15 +12,16 @@
 //         shift = nearest integer of -log2|V| (clamped), M = sign(V) (D >> shift).
 //
 // Design. A tile is m rows of one layer; a cluster of C CTAs covers it, CTA k
-// owning the column slice [k n_c, (k+1) n_c). Every value of the tile (U or X)
-// stays in registers between the two phases: phase A computes it and the
-// per-row maxima (reduced with warp REDUX, shared-memory atomics and then
-// across the cluster through distributed shared memory), phase B quantizes
-// and stores. The layer is therefore read once and R is generated once. The
-// B slice stays in shared memory across the tiles of a layer when it fits;
-// work items are 4 rows x 4 columns so one B load and one A load feed 16 FMAs
-// and one Philox call yields the 4 words of a row's 4 columns. Clusters keep a
-// contiguous range of tiles, so B is restaged only at layer changes.
+// owning the column slice [k n_c, (k+1) n_c). Phase A computes the tile's
+// values (U or X) into a shared-memory tile; a warp per row then reduces the
+// row extrema (REDUX), which are combined across the cluster through
+// distributed shared memory; phase B quantizes the tile from shared memory and
+// stores. The layer is therefore read once and R generated once. Work items
+// are 4 rows x 4 columns: one A load and one B load feed 16 FMAs and one
+// Philox call yields the 4 words of a row's 4 columns. The B slice stays in
+// shared memory across the tiles of a layer when it fits; clusters walk a
+// contiguous range of tiles, so B is restaged only at layer changes. The
+// shared-memory carve-up (tile, codes, B, A) is chosen per launch by the host.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -33,34 +34,19 @@ namespace intlora {
 namespace {
 
 constexpr double kLn2 = 0.69314718055994530942;
-
-struct SmemLayout {
-  int b_floats, a_floats, rcp_floats;
-  __host__ __device__ constexpr int b_off() const { return 0; }
-  __host__ __device__ constexpr int a_off() const { return b_floats; }
-  __host__ __device__ constexpr int rcp_off() const { return b_floats + a_floats; }
-  __host__ __device__ constexpr int rows_off() const { return rcp_off() + rcp_floats; }
-  // per-row area: s, z, q_inv, q_zero (4 words) + 2 x 2 slots (4 words)
-  __host__ __device__ constexpr int total_words() const { return rows_off() + 8 * kMaxTileRows; }
-};
-
-__host__ __device__ constexpr SmemLayout layout_for(int variant) {
-  return variant == kGen ? SmemLayout{0, 0, 0} : SmemLayout{kBSmemFloats, kASmemFloats, 512};
-}
+constexpr int RPI = kRowsPerItem;
 
 // Load the 4 codes of one item row (columns j .. j+3). aligned: one 32-bit
 // (8-bit codes) or 16-bit (4-bit codes) load; otherwise per element.
-template <int WBITS>
-__device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int64_t j, int valid,
-                                               bool aligned) {
+template <int WBITS, bool ALIGNED>
+__device__ __forceinline__ uint32_t load_codes(const uint8_t* row, int64_t j, int valid) {
   if (WBITS == 8) {
-    if (aligned && valid == 4) return __ldg(reinterpret_cast<const uint32_t*>(row + j));
+    if (ALIGNED) return __ldg(reinterpret_cast<const uint32_t*>(row + j));
     uint32_t v = 0;
     for (int c = 0; c < valid; ++c) v |= static_cast<uint32_t>(__ldg(row + j + c)) << (8 * c);
     return v;
   } else {
-    if (aligned && valid == 4)
-      return __ldg(reinterpret_cast<const uint16_t*>(row + (j >> 1)));
+    if (ALIGNED) return __ldg(reinterpret_cast<const uint16_t*>(row + (j >> 1)));
     uint32_t v = 0;
     for (int c = 0; c < valid; ++c) {
       const int64_t jj = j + c;
@@ -78,21 +64,20 @@ __device__ __forceinline__ int32_t code_at(uint32_t packed, int c) {
 }
 
 // Stores of one item row (4 columns): codes (kGen), P (kMul) or M (kShift),
-// plus the optional per-element code output of the merges.
-template <int VARIANT, int WBITS, bool ALIGNED>
-__device__ __forceinline__ void store_item(const TileLayer& L, int out_bytes, int64_t i, int64_t j,
-                                           int vcols, const int32_t res[4], const uint32_t code8[4]) {
+// plus the optional per-element code output of the merges. OUTB = bytes per
+// element of `out` for the merges.
+template <int VARIANT, int WBITS, int OUTB, bool ALIGNED>
+__device__ __forceinline__ void store_item(void* out, uint8_t* code_out, int64_t ld_out, int64_t n,
+                                           int64_t i, int64_t j, int vcols, const int32_t res[4],
+                                           const uint32_t code8[4]) {
   if (VARIANT == kGen) {
-    if (L.out == nullptr) return;
-    uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
+    uint8_t* orow = static_cast<uint8_t*>(out) + i * ld_out;
     if (WBITS == 8) {
       const uint32_t packed = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
       if (ALIGNED || vcols == 4) {
         *reinterpret_cast<uint32_t*>(orow + j) = packed;
       } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < vcols) orow[j + c] = static_cast<uint8_t>(code8[c]);
+        for (int c = 0; c < vcols; ++c) orow[j + c] = static_cast<uint8_t>(code8[c]);
       }
     } else {
       const uint32_t packed = code8[0] | (code8[1] << 4) | (code8[2] << 8) | (code8[3] << 12);
@@ -105,81 +90,72 @@ __device__ __forceinline__ void store_item(const TileLayer& L, int out_bytes, in
     }
     return;
   }
-  const int64_t e0 = i * L.n + j;
-  const bool vec = ALIGNED || vcols == 4;
-  if (vec && !ALIGNED) {
-    // an unaligned layer has row starts off the vector boundary
-    for (int c = 0; c < 4; ++c) {
-      if (out_bytes == 4) static_cast<int32_t*>(L.out)[e0 + c] = res[c];
-      else if (out_bytes == 2) static_cast<int16_t*>(L.out)[e0 + c] = static_cast<int16_t>(res[c]);
-      else static_cast<int8_t*>(L.out)[e0 + c] = static_cast<int8_t>(res[c]);
-      if (L.code_out != nullptr) L.code_out[e0 + c] = static_cast<uint8_t>(code8[c]);
+  const int64_t e0 = i * n + j;
+  if (!ALIGNED) {   // row starts are off the vector boundary: element stores
+    for (int c = 0; c < vcols; ++c) {
+      if (OUTB == 4) static_cast<int32_t*>(out)[e0 + c] = res[c];
+      else if (OUTB == 2) static_cast<int16_t*>(out)[e0 + c] = static_cast<int16_t>(res[c]);
+      else static_cast<int8_t*>(out)[e0 + c] = static_cast<int8_t>(res[c]);
+      if (code_out != nullptr) code_out[e0 + c] = static_cast<uint8_t>(code8[c]);
     }
     return;
   }
-  if (out_bytes == 4) {   // MUL products beyond the int16 bound
-    int32_t* o = static_cast<int32_t*>(L.out) + e0;
-    if (vec) {
-      *reinterpret_cast<int4*>(o) = make_int4(res[0], res[1], res[2], res[3]);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < vcols) o[c] = res[c];
-    }
-  } else if (out_bytes == 2) {   // int16 products or merged codes
-    int16_t* o = static_cast<int16_t*>(L.out) + e0;
-    if (vec) {
-      const uint32_t lo = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
-      const uint32_t hi = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
-      *reinterpret_cast<uint2*>(o) = make_uint2(lo, hi);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < vcols) o[c] = static_cast<int16_t>(res[c]);
-    }
-  } else {   // int8 merged codes (SHIFT with a base of at most 7 bits)
-    int8_t* o = static_cast<int8_t*>(L.out) + e0;
-    if (vec) {
-      *reinterpret_cast<uint32_t*>(o) = (static_cast<uint32_t>(res[0]) & 0xFFu) |
-                                        ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
-                                        ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) |
-                                        (static_cast<uint32_t>(res[3]) << 24);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < vcols) o[c] = static_cast<int8_t>(res[c]);
-    }
+  if (OUTB == 4) {
+    *reinterpret_cast<int4*>(static_cast<int32_t*>(out) + e0) = make_int4(res[0], res[1], res[2], res[3]);
+  } else if (OUTB == 2) {
+    const uint32_t lo = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
+    const uint32_t hi = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
+    *reinterpret_cast<uint2*>(static_cast<int16_t*>(out) + e0) = make_uint2(lo, hi);
+  } else {
+    *reinterpret_cast<uint32_t*>(static_cast<int8_t*>(out) + e0) =
+        (static_cast<uint32_t>(res[0]) & 0xFFu) | ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
+        ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) | (static_cast<uint32_t>(res[3]) << 24);
   }
-  if (L.code_out != nullptr) {
-    uint8_t* co = L.code_out + e0;
-    if (vec) {
-      *reinterpret_cast<uint32_t*>(co) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (c < vcols) co[c] = static_cast<uint8_t>(code8[c]);
-    }
-  }
+  if (code_out != nullptr)
+    *reinterpret_cast<uint32_t*>(code_out + e0) =
+        code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
 }
 
 // Non-negative floats (sign bit clear) order like their bit patterns, so row
-// maxima are reduced as unsigned integers (REDUX, shared atomics, DSMEM).
-__device__ __forceinline__ uint32_t ord(float v) { return __float_as_uint(v); }
+// extrema are reduced as unsigned integers (REDUX, shared atomics, DSMEM).
+// fabsf also drops a -0.0, whose pattern would otherwise win the maximum.
+__device__ __forceinline__ uint32_t ord(float v) { return __float_as_uint(fabsf(v)); }
 
-template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
-__global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_constant__ TileBatch p) {
-  constexpr SmemLayout lay = layout_for(VARIANT);
-  constexpr int IPT = kItemsPerThread;
-  constexpr int RPI = kRowsPerItem;
+// Walk of the items a thread owns: item it = tid + k T, i.e. (g, q) with
+// it = g quads + q, advanced without division.
+struct ItemWalk {
+  int g, q, dg, dq, quads;
+  __device__ __forceinline__ void init(int tid, int T, int quads_) {
+    quads = quads_;
+    g = tid / quads;
+    q = tid - g * quads;
+    dg = T / quads;
+    dq = T - dg * quads;
+  }
+  __device__ __forceinline__ void next() {
+    g += dg;
+    q += dq;
+    if (q >= quads) {
+      q -= quads;
+      ++g;
+    }
+  }
+};
+
+template <int VARIANT, int WBITS, int RANK, int OUTB, bool ALIGNED>
+__global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_constant__ TileBatch p) {
   extern __shared__ __align__(16) float smem[];
-  float* Bs = smem + lay.b_off();
-  float* At = smem + lay.a_off();
-  float* rcp_tab = smem + lay.rcp_off();
-  float* row_s = smem + lay.rows_off();
+  float* Us = smem;                                   // m x n_c tile of U (or X)
+  uint32_t* Cs = reinterpret_cast<uint32_t*>(Us + p.smem_u);   // codes, one word per item row
+  float* Bs = Us + p.smem_u + (VARIANT == kGen ? 0 : p.smem_u / 4);   // B slice, k-major
+  float* At = Bs + p.smem_b;                          // A rows of the tile, k-major
+  float* rcp_tab = At + p.smem_a;                     // 1/D for D in [-255, 255]
+  float* row_s = rcp_tab + (VARIANT == kGen ? 0 : 512);
   int32_t* row_z = reinterpret_cast<int32_t*>(row_s + kMaxTileRows);
   float* q_inv = row_s + 2 * kMaxTileRows;
   int32_t* q_zero = reinterpret_cast<int32_t*>(row_s + 3 * kMaxTileRows);
   uint32_t* slots = reinterpret_cast<uint32_t*>(row_s + 4 * kMaxTileRows);  // [2][rows][2]
+  const int warp = threadIdx.x >> 5;
   __shared__ float s_cln2;
 
   const int tid = threadIdx.x;
@@ -206,11 +182,20 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
     const int rows = static_cast<int>(min64(L.m, L.d - row0));
     const int64_t col0 = static_cast<int64_t>(crank) * L.n_c;
     const int ncols = static_cast<int>(max64(0, min64(L.n_c, L.n - col0)));
-    const int r = (VARIANT == kGen) ? 0 : (RANK > 0 ? RANK : L.r);
+    const int r = (VARIANT == kGen) ? 1 : (RANK > 0 ? RANK : L.r);
     const int m = L.m;
     const int n_c = L.n_c;
+    // per-layer values used inside the item loops, read once per tile
+    const int64_t n = L.n;
+    const int64_t ld_src = L.ld_src;
+    const uint8_t* __restrict__ src = static_cast<const uint8_t*>(L.src);
+    const uint32_t sid = L.stream_id;
+    void* const out = L.out;
+    uint8_t* const code_out = VARIANT == kGen ? nullptr : L.code_out;
+    const int64_t ld_out = L.ld_out;
+    float* const r_star_out = VARIANT == kGen ? L.r_star_out : nullptr;
 
-    __syncthreads();  // previous tile is done with At, row params and q params
+    __syncthreads();  // previous tile is done with the tile buffer and row params
     if (li != cur) {
       if (tid == 0) {
         const double c = pow(*L.sigma_w / *L.sigma_r, static_cast<double>(L.alpha));
@@ -233,126 +218,127 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
       }
       // A rows of the tile, read along the rank (coalesced), stored k-major
       for (int idx = tid; idx < r * m; idx += kTileThreads) {
-        const int rr = idx / max(r, 1), k = idx - rr * max(r, 1);
+        const int rr = idx / r, k = idx - rr * r;
         At[k * m + rr] = rr < rows ? __ldg(L.A + (row0 + rr) * static_cast<int64_t>(L.r) + k) : 0.0f;
       }
     }
     __syncthreads();
     const float c_ln2 = s_cln2;
 
-    // ---- work items of this thread: 4 rows x 4 columns each
     const int quads = n_c >> 2;
     const int G = m / RPI;
     const int nitems = G * quads;
-    int ig[IPT], iq[IPT];
-    bool iok[IPT];
-#pragma unroll
-    for (int k = 0; k < IPT; ++k) {
-      const int it = tid + k * kTileThreads;
-      const int g = it / quads;
-      iq[k] = it - g * quads;
-      iok[k] = it < nitems && 4 * iq[k] < ncols;
-      ig[k] = min(g, G - 1);
-    }
 
-    float acc[IPT][RPI][4];
-    uint32_t cw[IPT][RPI];
-
-    // ---- phase A.1: codes (merges) or W (base quantization); rows past the
-    // layer's end read the last row (their results are masked out)
-#pragma unroll
-    for (int k = 0; k < IPT; ++k) {
-#pragma unroll
-      for (int ml = 0; ml < RPI; ++ml) {
-        cw[k][ml] = 0u;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[k][ml][c] = 0.0f;
-      }
-      if (!iok[k]) continue;
-      const int64_t j = col0 + 4 * iq[k];
-      const int vcols = ALIGNED ? 4 : min(4, ncols - 4 * iq[k]);
-#pragma unroll
-      for (int ml = 0; ml < RPI; ++ml) {
-        const int64_t i = row0 + min(ig[k] * RPI + ml, rows - 1);
-        if (VARIANT == kGen) {
-          const float* wr = static_cast<const float*>(L.src) + i * L.n;
-          if (ALIGNED) {
-            const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + j));
-            acc[k][ml][0] = w4.x; acc[k][ml][1] = w4.y; acc[k][ml][2] = w4.z; acc[k][ml][3] = w4.w;
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              if (c < vcols) acc[k][ml][c] = __ldg(wr + j + c);
-          }
-        } else {
-          const uint8_t* wr = static_cast<const uint8_t*>(L.src) + i * L.ld_src;
-          cw[k][ml] = load_codes<WBITS>(wr, j, vcols, ALIGNED);
+    // B slices that do not stay resident are streamed in chunks; then the
+    // items accumulate A B into the tile buffer chunk by chunk first.
+    const bool streamed = VARIANT != kGen && !L.b_resident;
+    if (streamed) {
+      for (int k0 = 0; k0 < r; k0 += L.kc) {
+        const int kn = min(L.kc, r - k0);
+        __syncthreads();
+        for (int idx = tid; idx < kn * n_c; idx += kTileThreads) {
+          const int kk = idx / n_c, jj = idx - kk * n_c;
+          Bs[idx] = jj < ncols ? __ldg(L.B + static_cast<int64_t>(k0 + kk) * L.n + col0 + jj) : 0.0f;
         }
-      }
-    }
-
-    // ---- phase A.2: T = A B on the tile (CUDA-core FMA), B from shared memory
-    if (VARIANT != kGen) {
-      auto fma_tile = [&](const float* arow, const float* brow) {
+        __syncthreads();
+        ItemWalk w;
+        w.init(tid, kTileThreads, quads);
+        for (int it = tid; it < nitems; it += kTileThreads, w.next()) {
+          float acc[RPI][4];
 #pragma unroll
-        for (int k = 0; k < IPT; ++k) {
-          const float4 a4 = *reinterpret_cast<const float4*>(arow + ig[k] * RPI);
-          const float4 b4 = *reinterpret_cast<const float4*>(brow + 4 * iq[k]);
-          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-          const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+          for (int ml = 0; ml < RPI; ++ml) {
+            const float4 u = k0 == 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                     : *reinterpret_cast<const float4*>(Us + (w.g * RPI + ml) * n_c + 4 * w.q);
+            acc[ml][0] = u.x; acc[ml][1] = u.y; acc[ml][2] = u.z; acc[ml][3] = u.w;
+          }
+          for (int kk = 0; kk < kn; ++kk) {
+            const float4 a4 = *reinterpret_cast<const float4*>(At + (k0 + kk) * m + w.g * RPI);
+            const float4 b4 = *reinterpret_cast<const float4*>(Bs + kk * n_c + 4 * w.q);
+            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int ml = 0; ml < RPI; ++ml)
+#pragma unroll
+              for (int c = 0; c < 4; ++c) acc[ml][c] = fmaf(av[ml], bv[c], acc[ml][c]);
+          }
 #pragma unroll
           for (int ml = 0; ml < RPI; ++ml)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[k][ml][c] = fmaf(av[ml], bv[c], acc[k][ml][c]);
-        }
-      };
-      if (L.b_resident) {
-        if (RANK > 0) {
-#pragma unroll
-          for (int kk = 0; kk < RANK; ++kk) fma_tile(At + kk * m, Bs + kk * n_c);
-        } else {
-#pragma unroll 4
-          for (int kk = 0; kk < r; ++kk) fma_tile(At + kk * m, Bs + kk * n_c);
-        }
-      } else {
-        for (int k0 = 0; k0 < r; k0 += L.kc) {
-          const int kn = min(L.kc, r - k0);
-          __syncthreads();
-          for (int idx = tid; idx < kn * n_c; idx += kTileThreads) {
-            const int kk = idx / n_c, jj = idx - kk * n_c;
-            Bs[idx] = jj < ncols ? __ldg(L.B + static_cast<int64_t>(k0 + kk) * L.n + col0 + jj)
-                                 : 0.0f;
-          }
-          __syncthreads();
-#pragma unroll 4
-          for (int kk = 0; kk < kn; ++kk) fma_tile(At + (k0 + kk) * m, Bs + kk * n_c);
+            *reinterpret_cast<float4*>(Us + (w.g * RPI + ml) * n_c + 4 * w.q) =
+                make_float4(acc[ml][0], acc[ml][1], acc[ml][2], acc[ml][3]);
         }
       }
     }
 
-    // ---- phase A.3: R*, the value to quantize, and the row maxima
-#pragma unroll
-    for (int k = 0; k < IPT; ++k) {
-      float hi[RPI], lo[RPI];
-#pragma unroll
-      for (int ml = 0; ml < RPI; ++ml) hi[ml] = lo[ml] = 0.0f;
-      if (iok[k]) {
-        const int jl = 4 * iq[k];
+    // ---- phase A: values of the tile (and the code words of the merges)
+    {
+      const int64_t nq = n >> 2;   // Philox blocks per row (aligned layers)
+      ItemWalk w;
+      w.init(tid, kTileThreads, quads);
+      for (int it = tid; it < nitems; it += kTileThreads, w.next()) {
+        const int jl = 4 * w.q;
+        if (jl >= ncols) continue;
         const int vcols = ALIGNED ? 4 : min(4, ncols - jl);
+        const int64_t j = col0 + jl;
+        float acc[RPI][4];
+        uint32_t cw[RPI];
+        // inputs: codes (merges) or W (base quantization); rows past the
+        // layer's end read the last row (those values are never used)
 #pragma unroll
         for (int ml = 0; ml < RPI; ++ml) {
-          const int rr = ig[k] * RPI + ml;
-          const bool row_ok = rr < rows;
-          const int64_t e0 = (row0 + min(rr, rows - 1)) * L.n + col0 + jl;
+          const int64_t i = row0 + min(w.g * RPI + ml, rows - 1);
+          cw[ml] = 0u;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[ml][c] = 0.0f;
+          if (VARIANT == kGen) {
+            const float* wr = reinterpret_cast<const float*>(src) + i * n;
+            if (ALIGNED) {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(wr + j));
+              acc[ml][0] = w4.x; acc[ml][1] = w4.y; acc[ml][2] = w4.z; acc[ml][3] = w4.w;
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                if (c < vcols) acc[ml][c] = __ldg(wr + j + c);
+            }
+          } else {
+            cw[ml] = load_codes<WBITS, ALIGNED>(src + i * ld_src, j, vcols);
+          }
+        }
+        // T = A B on the item (CUDA-core FMA)
+        if (VARIANT != kGen) {
+          if (streamed) {
+#pragma unroll
+            for (int ml = 0; ml < RPI; ++ml) {
+              const float4 u = *reinterpret_cast<const float4*>(Us + (w.g * RPI + ml) * n_c + jl);
+              acc[ml][0] = u.x; acc[ml][1] = u.y; acc[ml][2] = u.z; acc[ml][3] = u.w;
+            }
+          } else {
+#pragma unroll 4
+            for (int kk = 0; kk < r; ++kk) {
+              const float4 a4 = *reinterpret_cast<const float4*>(At + kk * m + w.g * RPI);
+              const float4 b4 = *reinterpret_cast<const float4*>(Bs + kk * n_c + jl);
+              const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+              const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+              for (int ml = 0; ml < RPI; ++ml)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[ml][c] = fmaf(av[ml], bv[c], acc[ml][c]);
+            }
+          }
+        }
+        // R* and the value to quantize
+        const int64_t blk0 = (row0 + w.g * RPI) * nq + (j >> 2);   // aligned layers only
+#pragma unroll
+        for (int ml = 0; ml < RPI; ++ml) {
+          const int rr = w.g * RPI + ml;
+          const int64_t e0 = (row0 + min(rr, rows - 1)) * n + j;
           uint32_t words[4];
           if (ALIGNED) {
-            const uint4 w4 = aux_block(static_cast<uint64_t>(e0) >> 2, L.stream_id, L.key0, L.key1);
+            const uint4 w4 = aux_block(static_cast<uint64_t>(blk0 + ml * nq), sid, p.key0, p.key1);
             words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
           } else {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              words[c] = c < vcols ? aux_word(static_cast<uint64_t>(e0 + c), L.stream_id, L.key0,
-                                              L.key1)
+              words[c] = c < vcols ? aux_word(static_cast<uint64_t>(e0 + c), sid, p.key0, p.key1)
                                    : 0u;
           }
           float sv = 0.0f;
@@ -361,46 +347,50 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
             sv = row_s[rr];
             zv = row_z[rr];
           }
+          float v[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const float lg = laplace_log2(words[c]);
             const float cs = laplace_sign(words[c], c_ln2);   // +-c ln2
-            float v;
+            float x;
             if (VARIANT == kGen) {
-              if (L.r_star_out != nullptr && row_ok && (ALIGNED || c < vcols))
-                L.r_star_out[e0 + c] = lg * cs;
-              v = fmaf(-lg, cs, acc[k][ml][c]);                // W - R*
+              x = fmaf(-lg, cs, acc[ml][c]);                   // W - R*
             } else {
-              const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
-              v = fmaf(fmaf(lg, cs, acc[k][ml][c]), rcp_tab[dcode + 255], sv);
+              const int32_t dcode = code_at<WBITS>(cw[ml], c) - zv;
+              x = fmaf(fmaf(lg, cs, acc[ml][c]), rcp_tab[dcode + 255], sv);
             }
-            const bool ok = row_ok && (ALIGNED || c < vcols);
-            v = ok ? v : 0.0f;
-            acc[k][ml][c] = v;
-            if (VARIANT == kShift) {
-              hi[ml] = fmaxf(hi[ml], fabsf(v));
-            } else {
-              hi[ml] = fmaxf(hi[ml], v);
-              lo[ml] = fminf(lo[ml], v);
-            }
+            // columns past a ragged layer's end must not reach the extrema
+            v[c] = (ALIGNED || c < vcols) ? x : 0.0f;
+          }
+          *reinterpret_cast<float4*>(Us + rr * n_c + jl) = make_float4(v[0], v[1], v[2], v[3]);
+          if (VARIANT != kGen) Cs[rr * quads + w.q] = cw[ml];
+          if (VARIANT == kGen && r_star_out != nullptr && rr < rows) {
+            for (int c = 0; c < vcols; ++c)
+              r_star_out[e0 + c] = laplace_log2(words[c]) * laplace_sign(words[c], c_ln2);
           }
         }
       }
-      // reduce over the lanes holding the same rows, then one atomic per group
-      const int key = iok[k] ? ig[k] : -1;
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      const int leader = __ffs(peers) - 1;
-#pragma unroll
-      for (int ml = 0; ml < RPI; ++ml) {
-        // hi >= 0 >= lo in value; fabsf drops a possible -0.0, whose bit
-        // pattern would otherwise win the unsigned maximum
-        const uint32_t a = __reduce_max_sync(peers, ord(fabsf(hi[ml])));
-        const uint32_t b = (VARIANT == kShift) ? 0u : __reduce_max_sync(peers, ord(fabsf(lo[ml])));
-        const int rr = ig[k] * RPI + ml;
-        if (lane == leader && key >= 0 && rr < rows) {
-          atomicMax(&slots[(buf * kMaxTileRows + rr) * 2 + 0], a);
-          if (VARIANT != kShift) atomicMax(&slots[(buf * kMaxTileRows + rr) * 2 + 1], b);
+    }
+    __syncthreads();
+
+    // ---- row extrema of the tile: one warp per row, REDUX over the lanes
+    for (int rr = warp; rr < rows; rr += kTileThreads / 32) {
+      float hi = 0.0f, lo = 0.0f;
+      const float* urow = Us + rr * n_c;
+      for (int q = lane; 4 * q < ncols; q += 32) {
+        const float4 u = *reinterpret_cast<const float4*>(urow + 4 * q);
+        if (VARIANT == kShift) {
+          hi = fmaxf(hi, fmaxf(fmaxf(fabsf(u.x), fabsf(u.y)), fmaxf(fabsf(u.z), fabsf(u.w))));
+        } else {
+          hi = fmaxf(hi, fmaxf(fmaxf(u.x, u.y), fmaxf(u.z, u.w)));
+          lo = fminf(lo, fminf(fminf(u.x, u.y), fminf(u.z, u.w)));
         }
+      }
+      const uint32_t a = __reduce_max_sync(0xffffffffu, ord(hi));
+      const uint32_t b = (VARIANT == kShift) ? 0u : __reduce_max_sync(0xffffffffu, ord(lo));
+      if (lane == 0) {
+        slots[(buf * kMaxTileRows + rr) * 2 + 0] = a;
+        slots[(buf * kMaxTileRows + rr) * 2 + 1] = b;
       }
     }
 
@@ -448,44 +438,51 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
     }
     __syncthreads();
 
-    // ---- phase B: quantize from registers and store
-#pragma unroll
-    for (int k = 0; k < IPT; ++k) {
-      if (!iok[k]) continue;
-      const int jl = 4 * iq[k];
-      const int vcols = ALIGNED ? 4 : min(4, ncols - jl);
-      const int64_t j = col0 + jl;
-#pragma unroll
-      for (int ml = 0; ml < RPI; ++ml) {
-        const int rr = ig[k] * RPI + ml;
-        if (rr >= rows) continue;
+    // ---- phase B: quantize the tile and store (one item row per step)
+    if (VARIANT == kGen && out == nullptr) continue;
+    {
+      const int nrow_items = rows * quads;
+      ItemWalk w;                            // (row, quad) walk: g is the row here
+      w.init(tid, kTileThreads, quads);
+      for (int ir = tid; ir < nrow_items; ir += kTileThreads, w.next()) {
+        const int rr = w.g;
+        const int jl = 4 * w.q;
+        if (jl >= ncols) continue;
+        const int vcols = ALIGNED ? 4 : min(4, ncols - jl);
         const int64_t i = row0 + rr;
+        const int64_t j = col0 + jl;
+        const float4 u = *reinterpret_cast<const float4*>(Us + rr * n_c + jl);
+        const float uv[4] = {u.x, u.y, u.z, u.w};
         const float inv = q_inv[rr];
         const int32_t zero = q_zero[rr];
-        const int32_t zv = VARIANT == kGen ? 0 : row_z[rr];
+        uint32_t cw = 0u;
+        int32_t zv = 0;
+        if (VARIANT != kGen) {
+          cw = Cs[rr * quads + w.q];
+          zv = row_z[rr];
+        }
         int32_t res[4];
         uint32_t code8[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const float v = acc[k][ml][c];
           if (VARIANT == kShift) {
-            const float vn = v * inv;
+            const float vn = uv[c] * inv;
             const int32_t sh = clamp_i(neg_log2_round(vn), 0, qmax);
-            const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
+            const int32_t dcode = code_at<WBITS>(cw, c) - zv;
             const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
             res[c] = sgn * (dcode >> sh);
             code8[c] = static_cast<uint32_t>(sh);
           } else if (VARIANT == kMul) {
-            const int32_t centred = clamp_i(rne_scaled(v, inv), -zero, qmax - zero);
-            const int32_t dcode = code_at<WBITS>(cw[k][ml], c) - zv;
+            const int32_t centred = clamp_i(rne_scaled(uv[c], inv), -zero, qmax - zero);
+            const int32_t dcode = code_at<WBITS>(cw, c) - zv;
             res[c] = centred * dcode;
             code8[c] = static_cast<uint32_t>(centred + zero);
           } else {
-            code8[c] = static_cast<uint32_t>(clamp_i(rne_scaled(v, inv) + zero, 0, qmax));
+            code8[c] = static_cast<uint32_t>(clamp_i(rne_scaled(uv[c], inv) + zero, 0, qmax));
             res[c] = 0;
           }
         }
-        store_item<VARIANT, WBITS, ALIGNED>(L, p.out_bytes, i, j, vcols, res, code8);
+        store_item<VARIANT, WBITS, OUTB, ALIGNED>(out, code_out, ld_out, n, i, j, vcols, res, code8);
       }
     }
   }
@@ -496,128 +493,130 @@ __global__ void __launch_bounds__(kTileThreads, 2) tile_kernel(const __grid_cons
   }
 }
 
-template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
-cudaError_t launch_one(const TileBatch& b, cudaStream_t s) {
-  auto kern = tile_kernel<VARIANT, WBITS, RANK, ALIGNED>;
-  const size_t smem = static_cast<size_t>(layout_for(VARIANT).total_words()) * 4;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  if (b.cluster > 8) {
-    err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+template <int VARIANT, int WBITS, int RANK, int OUTB, bool ALIGNED>
+struct TileLaunch {
+  static constexpr auto kernel() { return tile_kernel<VARIANT, WBITS, RANK, OUTB, ALIGNED>; }
+
+  static cudaError_t prepare(int cluster, size_t smem) {
+    auto kern = kernel();
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
     if (err != cudaSuccess) return err;
+    if (cluster > 8) err = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return err;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(b.num_clusters * b.cluster));
-  cfg.blockDim = dim3(kTileThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(b.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, b);
+
+  static cudaLaunchConfig_t config(int grid, int cluster, size_t smem, cudaStream_t s,
+                                   cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kTileThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+  }
+
+  static cudaError_t launch(const TileBatch& b, cudaStream_t s) {
+    const size_t smem = tile_smem_bytes(b.variant, b.smem_u, b.smem_b, b.smem_a);
+    cudaError_t err = prepare(b.cluster, smem);
+    if (err != cudaSuccess) return err;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = config(b.num_clusters * b.cluster, b.cluster, smem, s, attr);
+    return cudaLaunchKernelEx(&cfg, kernel(), b);
+  }
+
+  static int max_clusters(int cluster, size_t smem) {
+    if (prepare(cluster, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = config(cluster, cluster, smem, nullptr, attr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel(), &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return n;
+  }
+};
+
+// Dispatch over the compile-time parameters. op = 0: launch, 1: occupancy.
+struct TileQuery {
+  int op;
+  int cluster;
+  size_t smem;
+  const TileBatch* batch;
+  cudaStream_t stream;
+  int result;
+  cudaError_t err;
+};
+
+template <int VARIANT, int WBITS, int RANK, int OUTB, bool ALIGNED>
+void run_query(TileQuery& q) {
+  using T = TileLaunch<VARIANT, WBITS, RANK, OUTB, ALIGNED>;
+  if (q.op == 0) q.err = T::launch(*q.batch, q.stream);
+  else q.result = T::max_clusters(q.cluster, q.smem);
 }
 
-template <int VARIANT, int WBITS, int RANK, bool ALIGNED>
-int max_clusters_one(int cluster) {
-  auto kern = tile_kernel<VARIANT, WBITS, RANK, ALIGNED>;
-  const size_t smem = static_cast<size_t>(layout_for(VARIANT).total_words()) * 4;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return 0;
-  if (cluster > 8 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    return 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(cluster));
-  cfg.blockDim = dim3(kTileThreads);
-  cfg.dynamicSmemBytes = smem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  return n;
-}
-
-template <int VARIANT, int WBITS, bool ALIGNED>
-cudaError_t dispatch_rank(const TileBatch& b, int rank_ct, cudaStream_t s) {
+template <int VARIANT, int WBITS, int OUTB, bool ALIGNED>
+void by_rank(TileQuery& q, int rank_ct) {
   switch (rank_ct) {
-    case 4: return launch_one<VARIANT, WBITS, 4, ALIGNED>(b, s);
-    case 8: return launch_one<VARIANT, WBITS, 8, ALIGNED>(b, s);
-    case 16: return launch_one<VARIANT, WBITS, 16, ALIGNED>(b, s);
-    case 32: return launch_one<VARIANT, WBITS, 32, ALIGNED>(b, s);
-    default: return launch_one<VARIANT, WBITS, 0, ALIGNED>(b, s);
+    case 4: run_query<VARIANT, WBITS, 4, OUTB, ALIGNED>(q); break;
+    case 8: run_query<VARIANT, WBITS, 8, OUTB, ALIGNED>(q); break;
+    case 16: run_query<VARIANT, WBITS, 16, OUTB, ALIGNED>(q); break;
+    default: run_query<VARIANT, WBITS, 0, OUTB, ALIGNED>(q); break;
   }
 }
 
-template <int VARIANT, int WBITS, bool ALIGNED>
-int clusters_rank(int rank_ct, int cluster) {
-  switch (rank_ct) {
-    case 4: return max_clusters_one<VARIANT, WBITS, 4, ALIGNED>(cluster);
-    case 8: return max_clusters_one<VARIANT, WBITS, 8, ALIGNED>(cluster);
-    case 16: return max_clusters_one<VARIANT, WBITS, 16, ALIGNED>(cluster);
-    case 32: return max_clusters_one<VARIANT, WBITS, 32, ALIGNED>(cluster);
-    default: return max_clusters_one<VARIANT, WBITS, 0, ALIGNED>(cluster);
-  }
-}
-
-template <int VARIANT, bool ALIGNED>
-cudaError_t dispatch_bits(const TileBatch& b, int wb, int rank_ct, cudaStream_t s) {
-  if constexpr (VARIANT == kGen) {
-    return wb == 8 ? launch_one<kGen, 8, 0, ALIGNED>(b, s) : launch_one<kGen, 4, 0, ALIGNED>(b, s);
+template <bool ALIGNED>
+void by_variant(TileQuery& q, int variant, int w_bits, int rank_ct, int out_bytes) {
+  if (variant == kGen) {
+    if (w_bits == 8) run_query<kGen, 8, 0, 1, ALIGNED>(q);
+    else run_query<kGen, 4, 0, 1, ALIGNED>(q);
+  } else if (variant == kMul) {
+    if (w_bits == 8) {
+      if (out_bytes == 4) by_rank<kMul, 8, 4, ALIGNED>(q, rank_ct);
+      else by_rank<kMul, 8, 2, ALIGNED>(q, rank_ct);
+    } else {
+      by_rank<kMul, 4, 2, ALIGNED>(q, rank_ct);
+    }
   } else {
-    return wb == 8 ? dispatch_rank<VARIANT, 8, ALIGNED>(b, rank_ct, s)
-                   : dispatch_rank<VARIANT, 4, ALIGNED>(b, rank_ct, s);
+    if (w_bits == 8) by_rank<kShift, 8, 2, ALIGNED>(q, rank_ct);
+    else by_rank<kShift, 4, 1, ALIGNED>(q, rank_ct);
   }
 }
 
-template <int VARIANT, bool ALIGNED>
-int clusters_bits(int wb, int rank_ct, int cluster) {
-  if constexpr (VARIANT == kGen) {
-    return wb == 8 ? max_clusters_one<kGen, 8, 0, ALIGNED>(cluster)
-                   : max_clusters_one<kGen, 4, 0, ALIGNED>(cluster);
-  } else {
-    return wb == 8 ? clusters_rank<VARIANT, 8, ALIGNED>(rank_ct, cluster)
-                   : clusters_rank<VARIANT, 4, ALIGNED>(rank_ct, cluster);
-  }
+void dispatch(TileQuery& q, int variant, int w_bits, int rank_ct, int out_bytes, bool aligned) {
+  if (aligned) by_variant<true>(q, variant, w_bits, rank_ct, out_bytes);
+  else by_variant<false>(q, variant, w_bits, rank_ct, out_bytes);
 }
 
 }  // namespace
 
-size_t tile_kernel_smem_bytes() { return static_cast<size_t>(layout_for(kMul).total_words()) * 4; }
-
-cudaError_t launch_tiles(int variant, const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s) {
-  const int wb = variant == kGen ? b.bits : b.w_bits;
-  if (variant == kGen)
-    return aligned ? dispatch_bits<kGen, true>(b, wb, 0, s) : dispatch_bits<kGen, false>(b, wb, 0, s);
-  if (variant == kMul)
-    return aligned ? dispatch_bits<kMul, true>(b, wb, rank_ct, s)
-                   : dispatch_bits<kMul, false>(b, wb, rank_ct, s);
-  return aligned ? dispatch_bits<kShift, true>(b, wb, rank_ct, s)
-                 : dispatch_bits<kShift, false>(b, wb, rank_ct, s);
+size_t tile_smem_bytes(int variant, int smem_u, int smem_b, int smem_a) {
+  const int codes = variant == kGen ? 0 : smem_u / 4;   // one code word per 4 tile values
+  const int words = smem_u + codes + smem_b + smem_a + (variant == kGen ? 0 : 512) + 8 * kMaxTileRows;
+  return static_cast<size_t>(words) * 4;
 }
 
-int tile_max_active_clusters(int variant, int w_bits, int rank_ct, bool aligned, int cluster) {
-  if (variant == kGen)
-    return aligned ? clusters_bits<kGen, true>(w_bits, 0, cluster)
-                   : clusters_bits<kGen, false>(w_bits, 0, cluster);
-  if (variant == kMul)
-    return aligned ? clusters_bits<kMul, true>(w_bits, rank_ct, cluster)
-                   : clusters_bits<kMul, false>(w_bits, rank_ct, cluster);
-  return aligned ? clusters_bits<kShift, true>(w_bits, rank_ct, cluster)
-                 : clusters_bits<kShift, false>(w_bits, rank_ct, cluster);
+cudaError_t launch_tiles(const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s) {
+  TileQuery q{0, b.cluster, 0, &b, s, 0, cudaSuccess};
+  dispatch(q, b.variant, b.variant == kGen ? b.bits : b.w_bits, rank_ct, b.out_bytes, aligned);
+  return q.err;
+}
+
+int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes, bool aligned,
+                             int cluster, size_t smem) {
+  TileQuery q{1, cluster, smem, nullptr, nullptr, 0, cudaSuccess};
+  dispatch(q, variant, w_bits, rank_ct, out_bytes, aligned);
+  return q.result;
 }
 
 }  // namespace intlora

@@ -179,3 +179,24 @@ def test_ste_parity(d, n, r):
     oA, oB = oracle.ste_backward(G, A, Bm)
     assert rel_fro(dA, oA) < STE_RTOL
     assert rel_fro(dB, oB) < STE_RTOL
+
+
+def test_batches_with_mixed_seeds():
+    """Layers with different Philox keys in one batched call (the library
+    launches one group per key) match the oracle and single-layer calls."""
+    specs = [spec_for(48, 320, 4, 4, "mul", 4, sid=k, seed=seed)
+             for k, seed in enumerate([1, 7, 2**40 + 3])]
+    Ws = [wl.host_W(s) for s in specs]
+    g_b = gpu_gen_aux(specs, Ws, batched=True)
+    g_s = gpu_gen_aux(specs, Ws, batched=False)
+    for spec, W, x, y in zip(specs, Ws, g_b, g_s):
+        assert np.array_equal(x["codes"], y["codes"]) and x["sigma_r"] == y["sigma_r"]
+        o = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits)
+        assert_scale("sigma_r", x["sigma_r"], o["sigma_r"])
+        assert_affine("W_round", x["codes"], x["z"], o["codes"], o["z"], o["pre"], o["zpre"], 15)
+    inps = [_oracle_prepared(s) for s in specs]
+    a = gpu_merge(specs, inps, batched=True)
+    b = gpu_merge(specs, inps, batched=False)
+    for spec, inp, x, y in zip(specs, inps, a, b):
+        assert np.array_equal(x["out"], y["out"])
+        _check_mul(spec, inp, x)

@@ -148,6 +148,34 @@ intlora_status intlora_gen_aux_batched(const intlora_aux_job* jobs, int32_t coun
                                        size_t ws_bytes, void* stream);
 
 /* --------------------------------------------------------------------------
+ * Layer preparation without a workspace argument. The paper has no
+ * counterpart: this serves callers that cannot allocate device memory, such
+ * as a host framework whose memory manager owns every device allocation, or a
+ * latency-critical loop where cudaMalloc (which may synchronize the device) is
+ * not allowed.
+ *
+ * Same arguments, results and validation as intlora_gen_aux, minus ws and
+ * ws_bytes: the scratch it needs comes from a fixed array compiled into the
+ * library (16 KB of device memory on every GPU that loads the library, held
+ * until the process exits). Hence a size limit: d * n must not exceed
+ * INTLORA_NOALLOC_MAX_ELEMENTS, else INTLORA_ERR_UNSUPPORTED with a message in
+ * intlora_last_error(). Allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array: calls whose GPU work can overlap
+ * (different streams without ordering) race on it and must be serialized by
+ * the caller. Nothing in the array needs clearing between calls.
+ * ------------------------------------------------------------------------ */
+#define INTLORA_NOALLOC_MAX_ELEMENTS 4194304
+
+intlora_status intlora_gen_aux_noalloc(const float* W, int64_t d, int64_t n, uint64_t seed,
+                                       uint32_t stream_id, float alpha, int32_t w_bits,
+                                       double* sigma_w_out, double* sigma_r_out,
+                                       float* r_star_out, void* w_round_out, int64_t ld_w_out,
+                                       float* s_out, int32_t* z_out, void* stream);
+
+/* --------------------------------------------------------------------------
  * Merges [notes, MLA and 两种实现版本].
  *
  * One quantized layer with its LoRA factors. All pointers are device pointers.

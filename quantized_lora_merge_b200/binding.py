@@ -67,6 +67,9 @@ _SIGNATURES = {
                                        _c_ptr, _c_size, _c_ptr]),
     "intlora_gen_aux_batched": (ctypes.c_int, [_P(intlora_aux_job), _c_i32, _c_ptr, _c_size,
                                                _c_ptr]),
+    "intlora_gen_aux_noalloc": (ctypes.c_int, [_c_ptr, _c_i64, _c_i64, _c_u64, _c_u32, _c_f32,
+                                               _c_i32, _c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i64,
+                                               _c_ptr, _c_ptr, _c_ptr]),
     "intlora_merge_workspace_size": (_c_size, [_P(intlora_layer), _c_i32]),
     "intlora_merge_mul": (ctypes.c_int, [_P(intlora_layer), _c_i32, _c_ptr, _c_ptr, _c_ptr,
                                          _c_ptr, _c_ptr, _c_size, _c_ptr]),
@@ -242,6 +245,15 @@ def intlora_gen_aux(job: AuxJob, ws=None, stream=None) -> None:
     _check(lib().intlora_gen_aux(c.W, c.d, c.n, c.seed, c.stream_id, c.alpha, c.w_bits,
                                  c.sigma_w_out, c.sigma_r_out, c.r_star_out, c.w_round_out,
                                  c.ld_w_out, c.s_out, c.z_out, p, nb, _stream(stream)))
+
+
+def intlora_gen_aux_noalloc(job: AuxJob, stream=None) -> None:
+    """Layer preparation with the library's built-in scratch (no workspace)."""
+    c = job.to_c()
+    _check(lib().intlora_gen_aux_noalloc(c.W, c.d, c.n, c.seed, c.stream_id, c.alpha, c.w_bits,
+                                         c.sigma_w_out, c.sigma_r_out, c.r_star_out,
+                                         c.w_round_out, c.ld_w_out, c.s_out, c.z_out,
+                                         _stream(stream)))
 
 
 def intlora_merge_workspace_size(layers: Sequence[Layer]) -> int:

@@ -568,6 +568,10 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
 
 }  // namespace
 
+void intlora::set_last_error(const char* message) {
+  snprintf(g_last_error, sizeof g_last_error, "%s", message);
+}
+
 extern "C" {
 
 const char* intlora_status_string(int status) {

@@ -126,4 +126,7 @@ int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 
+// Sets the calling thread's intlora_last_error() message.
+void set_last_error(const char* message);
+
 }  // namespace intlora

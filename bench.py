@@ -9,8 +9,10 @@ backward (dA = G B^T, dB = A^T G), each stage one batched call of the C ABI.
 Default workload: 128 SD-v1.5-UNet-shaped linears (16 transformer blocks, 8
 linears each), int4 base codes, rank 4, alpha 1.5, MUL with a 4-bit U
 quantizer, 217,415,680 merged weight elements per step (synthetic inputs drawn
-on the device). Metric: merged weight elements per second (whole job), with the
-dominant kernel's HBM roofline fraction reported beside it.
+on the device). Metric: merged weight elements per second (whole job). The
+roofline line is the merge kernel's: it is bound by lane issue (Philox and the
+Laplace inverse CDF per element), so it is reported against the SM lane-issue
+rate at the sampled SM clock, with its HBM fraction beside it.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: one process per GPU under torch.distributed.run; every rank runs its
@@ -39,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="sd_unet")
@@ -91,6 +93,54 @@ def prepare_bytes(l):
     code = 0.5 if l.w_bits == 4 else 1.0
     # statistics pass reads W; quantization pass reads W and writes codes, s, z
     return l.numel * (4 + 4 + code) + l.d * 8
+
+
+def merge_ops(l):
+    """Algorithmic lane operations of the merge kernel, per element x numel:
+    Philox4x32-10 share (10 rounds x 4 ops / 4 words = 10), Laplace inverse CDF
+    (6: shift, int->float, fma, log2, scale, sign), T = A.B (r FMAs), U (4: add,
+    fma, reciprocal multiply, select), row extrema (2), quantize + product
+    (MUL 5.5: fma, round, clamp x2, sub, half an IMAD; SHIFT 8: abs, exponent,
+    mantissa compare, clamps, shift, sign)."""
+    quant = 5.5 if l.variant == "mul" else 8.0
+    return l.numel * (10 + 6 + l.r + 4 + 2 + quant)
+
+
+ALU_LANES_PER_SM_CLK = 128       # FP32/INT32 lanes per SM per clock on sm_100
+NUM_SMS = 148
+
+
+def csrc_hash():
+    """Hash of the CUDA sources, so a stored ncu traffic figure is only used
+    while the kernels it was taken on are unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    root = Path(__file__).resolve().parent / "quantized_lora_merge_b200" / "csrc"
+    for p in sorted(root.iterdir()):
+        if p.suffix in (".cu", ".cuh", ".h"):
+            h.update(p.name.encode())
+            h.update(p.read_bytes())
+    return h.hexdigest()
+
+
+def profiled_traffic(name):
+    """dram__bytes_read.sum + dram__bytes_write.sum per launch from the ncu
+    summary profiles/<name>.md, or None when absent or when the kernels have
+    changed since it was taken."""
+    p = Path(__file__).resolve().parent / "profiles" / f"{name}.md"
+    if not p.exists():
+        return None
+    fields = {}
+    for line in p.read_text().splitlines():
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip().strip("-* `")] = v.strip().strip("` ")
+    if fields.get("csrc_sha256") != csrc_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def ste_bytes(l):
@@ -316,9 +366,13 @@ def main():
         stages[name] = {"ms": ms, "algorithmic_GB": per_stage_bytes[name] / 1e9,
                         "GB_s": gbs, "frac_of_hbm": gbs / hbm_peak}
     stages["merge"]["elements_per_s"] = sum(l.numel for l in layers) / (stage_ms["merge"] / 1e3)
-    dominant = max(stage_ms, key=stage_ms.get)
-    roof_gbs = per_stage_bytes[dominant] / (stage_ms[dominant] / 1000.0) / 1e9
-    launches_per_step = {"prepare": 3, "merge": 1, "ste_backward": 4}
+    # dominant kernel: the merge's row-tile kernel (one launch per step); it is
+    # bound by ALU issue (Philox + Laplace per element), so its roofline is the
+    # SM lane-issue rate at the measured SM clock; HBM fraction reported beside
+    sm_mhz = clk.get("sm_mhz") or 1965.0
+    alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
+    alu_achieved = sum(merge_ops(l) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
+    launches_per_step = {"prepare": 3, "merge": 1, "ste_backward": 2}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -327,9 +381,14 @@ def main():
         "config": desc,
         "hbm_GB_s_merge": stages["merge"]["GB_s"],
         "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
-        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": roof_gbs,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": roof_gbs / hbm_peak,
-                     "peak_source": peak_kind, "traffic": None},
+        "roofline": {"bound": "alu", "kernel": "merge row-tile kernel (MUL, 1 launch per step)",
+                     "achieved": alu_achieved, "peak": alu_peak, "unit": "Top/s",
+                     "frac": alu_achieved / alu_peak,
+                     "peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
+                     "ops_per_element": merge_ops(layers[0]) / layers[0].numel,
+                     "hbm_achieved_GB_s": stages["merge"]["GB_s"], "hbm_peak_GB_s": hbm_peak,
+                     "hbm_peak_source": peak_kind, "hbm_frac": stages["merge"]["frac_of_hbm"],
+                     "traffic": profiled_traffic("tile_kernel_mul_sd_unet")},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": args.steps * sum(launches_per_step.values()),

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -148,8 +149,163 @@ bool plan_layers(int variant, std::vector<TileLayer>& L, int cluster, int occ, b
   return true;
 }
 
+// ------------------------------------------------------------------------
+// team kernels: layers with n % 4 == 0 and n <= kTeamMaxCols
+// ------------------------------------------------------------------------
+// INTLORA_ROW_KERNEL=tile sends every layer to the row-tile kernels (both
+// kernel families stay testable on the same shapes); unset or "auto": the
+// team kernels take the layers they support.
+bool team_path_enabled() {
+  const char* v = std::getenv("INTLORA_ROW_KERNEL");
+  return v == nullptr || std::strcmp(v, "tile") != 0;
+}
+
+bool team_eligible(int variant, const TileLayer& l) {
+  if (l.n % 4 != 0 || l.n > kTeamMaxCols) return false;
+  if (l.d > (int64_t{1} << 24)) return false;      // keeps tile indices of a batch in int32
+  if (variant != kGen && !aligned16(l.B)) return false;
+  return true;
+}
+
+// Team width and sweeps of one layer: the most even spread of the row's
+// column quads over the team's lanes, then the fewest sweeps (less shared
+// memory, more resident CTAs), then the narrower team.
+void team_shape(int64_t n, int* tw_out, int* sweeps_out) {
+  const int64_t quads = n / 4;
+  double best_e = -1.0;
+  int best_tw = kTeamWarps, best_s = kTeamMaxSweeps;
+  for (int tw = 1; tw <= kTeamWarps; tw *= 2) {
+    const int64_t s = ceil_div(quads, int64_t{32} * tw);
+    if (s > kTeamMaxSweeps) continue;
+    const double e = static_cast<double>(quads) / static_cast<double>(32 * tw * s);
+    const bool better = e > best_e + 0.1 || (e > best_e - 0.1 && s < best_s);
+    if (better) {
+      best_e = std::max(best_e, e);
+      best_tw = tw;
+      best_s = static_cast<int>(s);
+    }
+  }
+  *tw_out = best_tw;
+  *sweeps_out = best_s;
+}
+
+int team_ctas_cached(int variant, int w_bits, int rank_ct, int out_bytes, int sweeps_max) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, out_bytes, sweeps_max);
+  {
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int v = team_max_active_ctas(variant, w_bits, rank_ct, out_bytes,
+                                     team_smem_bytes(variant, sweeps_max));
+  std::lock_guard<std::mutex> g(mu);
+  cache[key] = v;
+  return v;
+}
+
+intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, int rank_ct, int bits,
+                                 int w_bits, int out_bytes, uint64_t seed, cudaStream_t stream) {
+  static thread_local TeamBatch b;
+  std::memset(&b, 0, sizeof b);
+  int smax = 1;
+  int64_t tiles = 0;
+  std::vector<double> layer_cost(L.size()), tile_cost(L.size());
+  std::vector<int64_t> layer_tiles(L.size());
+  double total_cost = 0.0;
+  for (size_t k = 0; k < L.size(); ++k) {
+    const TileLayer& s = L[k];
+    TeamLayer& t = b.layer[k];
+    t.src = s.src;
+    t.ld_src = s.ld_src;
+    t.s = s.s;
+    t.z = s.z;
+    t.A = s.A;
+    t.B = s.B;
+    t.sigma_w = s.sigma_w;
+    t.sigma_r = s.sigma_r;
+    t.alpha = s.alpha;
+    t.stream_id = s.stream_id;
+    t.out = s.out;
+    t.ld_out = s.ld_out;
+    t.scale_out = s.scale_out;
+    t.zero_out = s.zero_out;
+    t.code_out = s.code_out;
+    t.r_star_out = s.r_star_out;
+    t.d = s.d;
+    t.n = s.n;
+    t.r = s.r;
+    team_shape(s.n, &t.team_warps, &t.sweeps);
+    smax = std::max(smax, t.sweeps);
+    const int64_t groups = ceil_div(s.d, kTeamRows);
+    const int64_t teams = kTeamWarps / t.team_warps;
+    t.tile_begin = tiles;
+    layer_tiles[k] = ceil_div(groups, teams);
+    tiles += layer_tiles[k];
+    // cost of a tile: its elements plus a fixed per-row-group overhead
+    tile_cost[k] = static_cast<double>(teams) * (kTeamRows * static_cast<double>(s.n) + 512.0);
+    layer_cost[k] = tile_cost[k] * static_cast<double>(layer_tiles[k]);
+    total_cost += layer_cost[k];
+  }
+  const int resident = team_ctas_cached(variant, w_bits, rank_ct, out_bytes, smax);
+  if (resident <= 0) return fail(INTLORA_ERR_UNSUPPORTED, "team kernel cannot be made resident");
+  const int ctas = static_cast<int>(std::min<int64_t>({int64_t{resident}, int64_t{kTeamMaxCtas}, tiles}));
+  // contiguous tile ranges of about equal cost, one per CTA
+  size_t li = 0;
+  double c_acc = 0.0;
+  int64_t t_acc = 0;
+  for (int k = 0; k < ctas; ++k) {
+    const double target = total_cost * static_cast<double>(k) / static_cast<double>(ctas);
+    while (li < L.size() && c_acc + layer_cost[li] <= target) {
+      c_acc += layer_cost[li];
+      t_acc += layer_tiles[li];
+      ++li;
+    }
+    int64_t begin = tiles;
+    if (li < L.size())
+      begin = t_acc + std::min<int64_t>(layer_tiles[li],
+                                        static_cast<int64_t>(std::ceil((target - c_acc) / tile_cost[li] - 1e-9)));
+    if (k > 0) begin = std::max<int64_t>(begin, b.cta_begin[k - 1]);
+    b.cta_begin[k] = static_cast<int32_t>(begin);
+  }
+  b.cta_begin[0] = 0;
+  b.cta_begin[ctas] = static_cast<int32_t>(tiles);
+  b.count = static_cast<int32_t>(L.size());
+  b.key0 = static_cast<uint32_t>(seed);
+  b.key1 = static_cast<uint32_t>(seed >> 32);
+  b.bits = bits;
+  b.w_bits = w_bits;
+  b.sweeps_max = smax;
+  b.num_ctas = ctas;
+  b.total_tiles = tiles;
+  cudaError_t e = launch_team(b, variant, rank_ct, out_bytes, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "team kernel launch");
+  return INTLORA_OK;
+}
+
 intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bits, int w_bits,
                                  int out_bytes, uint64_t seed, cudaStream_t stream) {
+  // layers the team kernel takes go there (one launch); the rest stay here
+  if (team_path_enabled()) {
+    std::vector<TileLayer> team, rest;
+    for (auto& l : L) (team_eligible(variant, l) ? team : rest).push_back(l);
+    if (!team.empty()) {
+      int rank_t = 0;
+      if (variant != kGen) {
+        rank_t = team[0].r;
+        for (auto& l : team)
+          if (l.r != rank_t) rank_t = 0;
+        if (rank_t != 4 && rank_t != 8 && rank_t != 16) rank_t = 0;
+      }
+      const intlora_status s = launch_team_batch(variant, team, rank_t, bits, w_bits, out_bytes, seed, stream);
+      if (s != INTLORA_OK) return s;
+    }
+    if (rest.empty()) return INTLORA_OK;
+    L = rest;
+  }
   int rank_ct = 0;
   if (variant != kGen) {
     rank_ct = L[0].r;

@@ -95,6 +95,58 @@ constexpr int kMaxTileRows = 128;
 size_t tile_smem_bytes(int variant, int smem_u, int smem_b, int smem_a);
 
 // ---------------------------------------------------------------------------
+// Team kernels (same three operations, rows up to kTeamMaxCols columns with
+// n % 4 == 0). A team of TW warps of one CTA owns a group of 4 rows across the
+// whole row: lane l of the team takes the column quads l, l + 32 TW, ... (at
+// most kTeamMaxSweeps of them), keeps its values in a lane-private stretch of
+// shared memory, and the team combines its row extrema with one named barrier
+// (none for TW = 1). Warps never wait on the rest of the CTA inside a layer.
+// ---------------------------------------------------------------------------
+constexpr int kTeamThreads = 256;
+constexpr int kTeamWarps = kTeamThreads / 32;
+constexpr int kTeamRows = 4;
+constexpr int kTeamMaxSweeps = 6;
+constexpr int64_t kTeamMaxCols = int64_t{4} * kTeamThreads * kTeamMaxSweeps;
+constexpr int kTeamMaxCtas = 148 * 4;
+
+struct TeamLayer {
+  const void* src;           // kGen: fp32 W; merges: W_round codes
+  int64_t ld_src;            // bytes per row of src
+  const float* s;            // merges: base scales
+  const int32_t* z;          // merges: base zero-points
+  const float* A;            // merges: d x r
+  const float* B;            // merges: r x n (16-byte aligned)
+  const double* sigma_w;
+  const double* sigma_r;
+  float alpha;
+  uint32_t stream_id;
+  void* out;
+  int64_t ld_out;            // kGen: bytes per code row; merges: elements (= n)
+  float* scale_out;
+  int32_t* zero_out;
+  uint8_t* code_out;
+  float* r_star_out;
+  int64_t d, n;
+  int32_t r;
+  int32_t team_warps;        // TW: 1, 2, 4 or 8
+  int32_t sweeps;            // column quads per lane: ceil(n / (128 TW))
+  int64_t tile_begin;        // a tile is the kTeamWarps / TW row groups of one CTA step
+};
+struct TeamBatch {
+  TeamLayer layer[kMaxBatch];
+  int32_t count;
+  uint32_t key0, key1;
+  int32_t bits;              // kGen: w_bits; kMul: u_bits; kShift: shift_bits
+  int32_t w_bits;
+  int32_t sweeps_max;        // shared memory is carved for this many sweeps
+  int32_t num_ctas;
+  int64_t total_tiles;
+  int32_t cta_begin[kTeamMaxCtas + 1];   // tiles of CTA k: [cta_begin[k], cta_begin[k+1])
+};
+
+size_t team_smem_bytes(int variant, int sweeps_max);
+
+// ---------------------------------------------------------------------------
 // STE backward.
 // ---------------------------------------------------------------------------
 struct SteJob {
@@ -123,6 +175,8 @@ cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s);
 cudaError_t launch_tiles(const TileBatch& b, int rank_ct, bool aligned, cudaStream_t s);
 int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes, bool aligned,
                              int cluster, size_t smem);
+cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s);
+int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 

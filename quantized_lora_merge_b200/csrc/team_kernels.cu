@@ -1,0 +1,431 @@
+// Team kernels of the IntLoRA merge path (sm_100a): the same three per-row
+// operations as the row-tile kernels (base quantization of W - R*, the MUL
+// merge and the SHIFT merge; IntLoRA paper notes (ICML2025), method sections
+// 1-3), laid out so that warps do not wait on one another inside a layer.
+//
+// A team of TW warps owns a group of 4 rows across the whole row. Lane l of
+// the team takes the column quads q = l, l + 32 TW, ... ("sweeps"). Phase A
+// computes an item of 4 rows x 4 columns (one Philox block per row: the 4
+// words of its 4 columns), keeps the running row extrema in registers and
+// parks the values (and the code words of the merges) in a lane-private
+// stretch of shared memory: only the lane that wrote a value reads it back,
+// so no synchronisation is needed for it. The row extrema are reduced over
+// the warp with REDUX and over the team through a small slot array and one
+// named barrier (none when TW = 1). Phase B quantizes the parked values and
+// stores. B is read through the L1 cache (16-byte loads), A and the row
+// parameters once per row group.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "intlora_device.cuh"
+#include "intlora_kernels.h"
+
+namespace intlora {
+
+namespace {
+
+constexpr double kLn2 = 0.69314718055994530942;
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ uint32_t ord(float v) { return __float_as_uint(fabsf(v)); }
+
+__device__ __forceinline__ void team_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int WBITS>
+__device__ __forceinline__ int32_t nib(uint32_t packed, int c) {
+  return WBITS == 8 ? static_cast<int32_t>((packed >> (8 * c)) & 0xFFu)
+                    : static_cast<int32_t>((packed >> (4 * c)) & 0xFu);
+}
+
+template <int WBITS>
+__device__ __forceinline__ uint32_t load_quad_codes(const uint8_t* row, int64_t j) {
+  return WBITS == 8 ? __ldg(reinterpret_cast<const uint32_t*>(row + j))
+                    : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(row + (j >> 1))));
+}
+
+// One of the four values selected by a small runtime index, without a local
+// array (keeps the operands in registers).
+template <typename T>
+__device__ __forceinline__ T pick4(const T v[4], int k) {
+  T x = v[0];
+  x = k == 1 ? v[1] : x;
+  x = k == 2 ? v[2] : x;
+  x = k == 3 ? v[3] : x;
+  return x;
+}
+
+template <int VARIANT, int WBITS, int RANK, int OUTB>
+__global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_constant__ TeamBatch p) {
+  extern __shared__ __align__(16) float4 smem4[];
+  const int smax = p.sweeps_max;
+  float4* Ubuf = smem4;                                              // [smax][4][256]
+  uint4* Cbuf = reinterpret_cast<uint4*>(smem4 + smax * kTeamRows * kTeamThreads);   // [smax][256]
+  uint32_t* slots = reinterpret_cast<uint32_t*>(Cbuf + (VARIANT == kGen ? 0 : smax * kTeamThreads));
+  float* rcp_tab = reinterpret_cast<float*>(slots + 2 * kTeamWarps * 8);   // 1/D, D in [-255, 255]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qmax = (1 << p.bits) - 1;
+  if (VARIANT != kGen)
+    for (int k = tid; k < 511; k += kTeamThreads)
+      rcp_tab[k] = (k == 255) ? 0.0f : __frcp_rn(static_cast<float>(k - 255));
+  __syncthreads();
+
+  const int64_t t_begin = p.cta_begin[blockIdx.x];
+  const int64_t t_end = p.cta_begin[blockIdx.x + 1];
+  int li = 0, cur = -1, cur_tw = 0;
+  uint32_t phase = 0;
+  float c_ln2 = 0.0f;
+  for (int64_t t = t_begin; t < t_end; ++t) {
+    while (li + 1 < p.count && p.layer[li + 1].tile_begin <= t) ++li;
+    const TeamLayer& L = p.layer[li];
+    if (li != cur) {
+      if (L.team_warps != cur_tw) {
+        // teams regroup: nobody may still be reading the slots of the old teams
+        __syncthreads();
+        cur_tw = L.team_warps;
+        phase = 0;
+      }
+      const double c = pow(*L.sigma_w / *L.sigma_r, static_cast<double>(L.alpha));
+      c_ln2 = static_cast<float>(c * kLn2);
+      cur = li;
+    }
+    const int TW = cur_tw;
+    const int teams = kTeamWarps / TW;
+    const int team = warp / TW;
+    const int wi = warp - team * TW;
+    const int LT = TW * 32;
+    const int lt = wi * 32 + lane;
+    const int64_t row0 = ((t - L.tile_begin) * teams + team) * kTeamRows;
+    if (row0 >= L.d) continue;                  // the whole team skips together
+    const int rows = static_cast<int>(min64(kTeamRows, L.d - row0));
+    const int64_t n = L.n;
+    const int quads = static_cast<int>(n >> 2);
+    const int S = L.sweeps;
+    const uint8_t* __restrict__ src = static_cast<const uint8_t*>(L.src);
+    const int64_t ld_src = L.ld_src;
+    const uint32_t sid = L.stream_id;
+    const int r = VARIANT == kGen ? 0 : (RANK > 0 ? RANK : L.r);
+
+    // row parameters and (small fixed rank) the A rows of the group
+    int64_t irow[kTeamRows];
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) irow[ml] = row0 + min(ml, rows - 1);
+    float sv[kTeamRows];
+    int32_t zv[kTeamRows];
+    constexpr int AREG = (RANK > 0 && RANK <= 8) ? RANK : 1;
+    float areg[kTeamRows][AREG];
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) {
+      sv[ml] = 0.0f;
+      zv[ml] = 0;
+      if (VARIANT != kGen) {
+        sv[ml] = __ldg(L.s + irow[ml]);
+        zv[ml] = clamp_i(__ldg(L.z + irow[ml]), 0, (1 << WBITS) - 1);
+        if (RANK > 0 && RANK <= 8) {
+#pragma unroll
+          for (int kk = 0; kk < AREG; ++kk) areg[ml][kk] = __ldg(L.A + irow[ml] * RANK + kk);
+        }
+      }
+    }
+
+    // ---- phase A
+    float hi[kTeamRows], lo[kTeamRows];
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) hi[ml] = lo[ml] = 0.0f;
+    for (int k = 0; k < S; ++k) {
+      const int q = lt + k * LT;
+      if (q >= quads) break;
+      const int64_t j = 4 * static_cast<int64_t>(q);
+      float acc[kTeamRows][4];
+      uint32_t cw[kTeamRows];
+#pragma unroll
+      for (int ml = 0; ml < kTeamRows; ++ml) {
+        cw[ml] = 0u;
+        if (VARIANT == kGen) {
+          const float4 w4 = __ldg(reinterpret_cast<const float4*>(src + irow[ml] * ld_src) + q);
+          acc[ml][0] = w4.x; acc[ml][1] = w4.y; acc[ml][2] = w4.z; acc[ml][3] = w4.w;
+        } else {
+          cw[ml] = load_quad_codes<WBITS>(src + irow[ml] * ld_src, j);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[ml][c] = 0.0f;
+        }
+      }
+      if (VARIANT != kGen) {
+        if (RANK > 0 && RANK <= 8) {
+#pragma unroll
+          for (int kk = 0; kk < AREG; ++kk) {
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(L.B + kk * n) + q);
+#pragma unroll
+            for (int ml = 0; ml < kTeamRows; ++ml) {
+              acc[ml][0] = fmaf(areg[ml][kk], b4.x, acc[ml][0]);
+              acc[ml][1] = fmaf(areg[ml][kk], b4.y, acc[ml][1]);
+              acc[ml][2] = fmaf(areg[ml][kk], b4.z, acc[ml][2]);
+              acc[ml][3] = fmaf(areg[ml][kk], b4.w, acc[ml][3]);
+            }
+          }
+        } else {
+#pragma unroll 4
+          for (int kk = 0; kk < r; ++kk) {
+            const float4 b4 = __ldg(reinterpret_cast<const float4*>(L.B + kk * n) + q);
+#pragma unroll
+            for (int ml = 0; ml < kTeamRows; ++ml) {
+              const float a = __ldg(L.A + irow[ml] * r + kk);
+              acc[ml][0] = fmaf(a, b4.x, acc[ml][0]);
+              acc[ml][1] = fmaf(a, b4.y, acc[ml][1]);
+              acc[ml][2] = fmaf(a, b4.z, acc[ml][2]);
+              acc[ml][3] = fmaf(a, b4.w, acc[ml][3]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int ml = 0; ml < kTeamRows; ++ml) {
+        const uint4 w4 = aux_block(static_cast<uint64_t>(irow[ml] * quads + q), sid, p.key0, p.key1);
+        const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
+        float v[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float lg = laplace_log2(words[c]);
+          const float cs = laplace_sign(words[c], c_ln2);
+          if (VARIANT == kGen) {
+            v[c] = fmaf(-lg, cs, acc[ml][c]);                     // W - R*
+          } else {
+            const int32_t dcode = nib<WBITS>(cw[ml], c) - zv[ml];
+            v[c] = fmaf(fmaf(lg, cs, acc[ml][c]), rcp_tab[dcode + 255], sv[ml]);
+          }
+          if (VARIANT == kShift) {
+            hi[ml] = fmaxf(hi[ml], fabsf(v[c]));
+          } else {
+            hi[ml] = fmaxf(hi[ml], v[c]);
+            lo[ml] = fminf(lo[ml], v[c]);
+          }
+        }
+        Ubuf[(k * kTeamRows + ml) * kTeamThreads + tid] = make_float4(v[0], v[1], v[2], v[3]);
+        if (VARIANT == kGen && L.r_star_out != nullptr && ml < rows) {
+          float* rs = L.r_star_out + irow[ml] * n + j;
+          *reinterpret_cast<float4*>(rs) =
+              make_float4(laplace_scaled(words[0], c_ln2), laplace_scaled(words[1], c_ln2),
+                          laplace_scaled(words[2], c_ln2), laplace_scaled(words[3], c_ln2));
+        }
+      }
+      if (VARIANT != kGen) Cbuf[k * kTeamThreads + tid] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    }
+
+    // ---- row extrema: over the warp (REDUX), then over the team
+    uint32_t ehi[kTeamRows], elo[kTeamRows];
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) {
+      ehi[ml] = __reduce_max_sync(kFull, ord(hi[ml]));
+      elo[ml] = VARIANT == kShift ? 0u : __reduce_max_sync(kFull, ord(lo[ml]));
+    }
+    if (TW > 1) {
+      uint32_t* mine = slots + ((phase & 1u) * kTeamWarps + warp) * 8;
+      if (lane == 0) {
+#pragma unroll
+        for (int ml = 0; ml < kTeamRows; ++ml) {
+          mine[ml] = ehi[ml];
+          mine[kTeamRows + ml] = elo[ml];
+        }
+      }
+      team_barrier(1 + team, LT);
+      // lane v < 8 gathers value v over the team's warps, then every lane
+      // takes the 8 combined values by shuffles
+      uint32_t acc = 0u;
+      if (lane < 8) {
+        const uint32_t* base = slots + ((phase & 1u) * kTeamWarps + team * TW) * 8 + lane;
+        for (int w2 = 0; w2 < TW; ++w2) acc = max(acc, base[w2 * 8]);
+      }
+#pragma unroll
+      for (int ml = 0; ml < kTeamRows; ++ml) {
+        ehi[ml] = __shfl_sync(kFull, acc, ml);
+        elo[ml] = __shfl_sync(kFull, acc, kTeamRows + ml);
+      }
+      ++phase;
+    }
+
+    // ---- quantizer parameters: lane ml < 4 works out row ml, then broadcast
+    float scale = 1.0f;
+    int32_t zero = 0;
+    {
+      const float top = __uint_as_float(pick4(ehi, lane & 3));
+      const float neg_bottom = __uint_as_float(pick4(elo, lane & 3));
+      if (VARIANT == kShift) {
+        scale = top > 0.0f ? top : 1.0f;
+      } else {
+        scale = __fdiv_rn(top + neg_bottom, static_cast<float>(qmax));
+        if (scale > 0.0f) zero = clamp_i(static_cast<int32_t>(rintf(__fdiv_rn(neg_bottom, scale))), 0, qmax);
+        else scale = 1.0f;
+      }
+    }
+    const float inv_own = __frcp_rn(scale);
+    if (wi == 0 && lane < rows) {
+      if (L.scale_out != nullptr) L.scale_out[row0 + lane] = scale;
+      if (VARIANT != kShift && L.zero_out != nullptr) L.zero_out[row0 + lane] = zero;
+    }
+    float inv[kTeamRows];
+    int32_t zq[kTeamRows];
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) {
+      inv[ml] = __shfl_sync(kFull, inv_own, ml);
+      zq[ml] = __shfl_sync(kFull, zero, ml);
+    }
+
+    // ---- phase B: quantize the parked values and store
+    if (VARIANT == kGen && L.out == nullptr) continue;
+    for (int k = 0; k < S; ++k) {
+      const int q = lt + k * LT;
+      if (q >= quads) break;
+      const int64_t j = 4 * static_cast<int64_t>(q);
+      uint4 cw4 = make_uint4(0u, 0u, 0u, 0u);
+      if (VARIANT != kGen) cw4 = Cbuf[k * kTeamThreads + tid];
+      const uint32_t cw[kTeamRows] = {cw4.x, cw4.y, cw4.z, cw4.w};
+#pragma unroll
+      for (int ml = 0; ml < kTeamRows; ++ml) {
+        if (ml >= rows) break;
+        const float4 u4 = Ubuf[(k * kTeamRows + ml) * kTeamThreads + tid];
+        const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+        const int64_t i = row0 + ml;
+        int32_t res[4];
+        uint32_t code8[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (VARIANT == kShift) {
+            const float vn = uv[c] * inv[ml];
+            const int32_t sh = clamp_i(neg_log2_round(vn), 0, qmax);
+            const int32_t dcode = nib<WBITS>(cw[ml], c) - zv[ml];
+            const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
+            res[c] = sgn * (dcode >> sh);
+            code8[c] = static_cast<uint32_t>(sh);
+          } else if (VARIANT == kMul) {
+            const int32_t centred = clamp_i(rne_scaled(uv[c], inv[ml]), -zq[ml], qmax - zq[ml]);
+            res[c] = centred * (nib<WBITS>(cw[ml], c) - zv[ml]);
+            code8[c] = static_cast<uint32_t>(centred + zq[ml]);
+          } else {
+            code8[c] = static_cast<uint32_t>(clamp_i(rne_scaled(uv[c], inv[ml]) + zq[ml], 0, qmax));
+            res[c] = 0;
+          }
+        }
+        if (VARIANT == kGen) {
+          uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
+          if (WBITS == 8)
+            *reinterpret_cast<uint32_t*>(orow + j) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
+          else
+            *reinterpret_cast<uint16_t*>(orow + (j >> 1)) =
+                static_cast<uint16_t>(code8[0] | (code8[1] << 4) | (code8[2] << 8) | (code8[3] << 12));
+          continue;
+        }
+        const int64_t e0 = i * n + j;
+        if (OUTB == 4) {
+          *reinterpret_cast<int4*>(static_cast<int32_t*>(L.out) + e0) = make_int4(res[0], res[1], res[2], res[3]);
+        } else if (OUTB == 2) {
+          const uint32_t w0 = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
+          const uint32_t w1 = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
+          *reinterpret_cast<uint2*>(static_cast<int16_t*>(L.out) + e0) = make_uint2(w0, w1);
+        } else {
+          *reinterpret_cast<uint32_t*>(static_cast<int8_t*>(L.out) + e0) =
+              (static_cast<uint32_t>(res[0]) & 0xFFu) | ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
+              ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) | (static_cast<uint32_t>(res[3]) << 24);
+        }
+        if (L.code_out != nullptr)
+          *reinterpret_cast<uint32_t*>(L.code_out + e0) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
+      }
+    }
+  }
+}
+
+template <int VARIANT, int WBITS, int RANK, int OUTB>
+struct TeamLaunch {
+  static constexpr auto kernel() { return team_kernel<VARIANT, WBITS, RANK, OUTB>; }
+  static cudaError_t launch(const TeamBatch& b, cudaStream_t s) {
+    const size_t smem = team_smem_bytes(VARIANT, b.sweeps_max);
+    cudaError_t err = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    kernel()<<<b.num_ctas, kTeamThreads, smem, s>>>(b);
+    return cudaGetLastError();
+  }
+  static int max_ctas(size_t smem) {
+    if (cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel(), kTeamThreads, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return per_sm * sms;
+  }
+};
+
+struct TeamQuery {
+  int op;                    // 0: launch, 1: resident CTAs
+  size_t smem;
+  const TeamBatch* batch;
+  cudaStream_t stream;
+  int result;
+  cudaError_t err;
+};
+
+template <int VARIANT, int WBITS, int RANK, int OUTB>
+void team_run(TeamQuery& q) {
+  using T = TeamLaunch<VARIANT, WBITS, RANK, OUTB>;
+  if (q.op == 0) q.err = T::launch(*q.batch, q.stream);
+  else q.result = T::max_ctas(q.smem);
+}
+
+template <int VARIANT, int WBITS, int OUTB>
+void team_by_rank(TeamQuery& q, int rank_ct) {
+  switch (rank_ct) {
+    case 4: team_run<VARIANT, WBITS, 4, OUTB>(q); break;
+    case 8: team_run<VARIANT, WBITS, 8, OUTB>(q); break;
+    case 16: team_run<VARIANT, WBITS, 16, OUTB>(q); break;
+    default: team_run<VARIANT, WBITS, 0, OUTB>(q); break;
+  }
+}
+
+void team_dispatch(TeamQuery& q, int variant, int w_bits, int rank_ct, int out_bytes) {
+  if (variant == kGen) {
+    if (w_bits == 8) team_run<kGen, 8, 0, 1>(q);
+    else team_run<kGen, 4, 0, 1>(q);
+  } else if (variant == kMul) {
+    if (w_bits == 8) {
+      if (out_bytes == 4) team_by_rank<kMul, 8, 4>(q, rank_ct);
+      else team_by_rank<kMul, 8, 2>(q, rank_ct);
+    } else {
+      team_by_rank<kMul, 4, 2>(q, rank_ct);
+    }
+  } else {
+    if (w_bits == 8) team_by_rank<kShift, 8, 2>(q, rank_ct);
+    else team_by_rank<kShift, 4, 1>(q, rank_ct);
+  }
+}
+
+}  // namespace
+
+size_t team_smem_bytes(int variant, int sweeps_max) {
+  const size_t per_sweep = static_cast<size_t>(kTeamRows) * kTeamThreads * 16 +
+                           (variant == kGen ? 0 : static_cast<size_t>(kTeamThreads) * 16);
+  return per_sweep * sweeps_max + 2 * kTeamWarps * 8 * 4 + (variant == kGen ? 0 : 512 * 4);
+}
+
+cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s) {
+  TeamQuery q{0, 0, &b, s, 0, cudaSuccess};
+  team_dispatch(q, variant, variant == kGen ? b.bits : b.w_bits, rank_ct, out_bytes);
+  return q.err;
+}
+
+int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem) {
+  TeamQuery q{1, smem, nullptr, nullptr, 0, cudaSuccess};
+  team_dispatch(q, variant, w_bits, rank_ct, out_bytes);
+  return q.result;
+}
+
+}  // namespace intlora

@@ -212,10 +212,41 @@ class SteJob:
 
 
 def _array(struct, items):
+    if isinstance(items, Descriptors):
+        if items.struct is not struct:
+            raise TypeError(f"descriptors of {items.struct.__name__}, expected {struct.__name__}")
+        return items.arr
     arr = (struct * max(1, len(items)))()
     for k, it in enumerate(items):
         arr[k] = it.to_c()
     return arr
+
+
+class Descriptors:
+    """A list of descriptors converted to their C structs once, for calls that
+    repeat on the same buffers (the per-call conversion of a 128-layer list
+    costs milliseconds of Python). Pass it wherever a list is accepted."""
+
+    _STRUCT = {}
+
+    def __init__(self, items):
+        items = list(items)
+        if not items:
+            raise ValueError("empty descriptor list")
+        self.struct = self._STRUCT[type(items[0])]
+        self.arr = (self.struct * len(items))()
+        for k, it in enumerate(items):
+            if type(it) is not type(items[0]):
+                raise TypeError("mixed descriptor types")
+            self.arr[k] = it.to_c()
+        self.count = len(items)
+
+    def __len__(self):
+        return self.count
+
+
+Descriptors._STRUCT = {AuxJob: intlora_aux_job, Layer: intlora_layer,
+                       MergeOut: intlora_merge_out, SteJob: intlora_ste_job}
 
 
 # ---------------------------------------------------------------------------

@@ -34,6 +34,10 @@ __device__ __forceinline__ void team_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 template <int WBITS>
 __device__ __forceinline__ int32_t nib(uint32_t packed, int c) {
   return WBITS == 8 ? static_cast<int32_t>((packed >> (8 * c)) & 0xFFu)
@@ -130,6 +134,29 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         }
       }
     }
+
+#ifndef TEAM_NO_PREFETCH
+    // The team's next row group of this layer is brought into L2 now (its
+    // source rows and, for the merges, its row parameters and A rows), so the
+    // next tile starts on L2 hits instead of HBM misses.
+    {
+      const int64_t nrow0 = row0 + static_cast<int64_t>(teams) * kTeamRows;
+      if (t + 1 < t_end && nrow0 < L.d) {
+        const int nrows = static_cast<int>(min64(kTeamRows, L.d - nrow0));
+        const int64_t row_bytes = VARIANT == kGen ? 4 * n : (WBITS == 8 ? n : n / 2);
+        const int lines = static_cast<int>((row_bytes + 127) / 128);
+        for (int idx = lt; idx < nrows * lines; idx += LT) {
+          const int rr = idx / lines;
+          prefetch_l2(src + (nrow0 + rr) * ld_src + static_cast<int64_t>(idx - rr * lines) * 128);
+        }
+        if (VARIANT != kGen && lt == 0) {
+          prefetch_l2(L.s + nrow0);
+          prefetch_l2(L.z + nrow0);
+          prefetch_l2(L.A + nrow0 * r);
+        }
+      }
+    }
+#endif
 
     // ---- phase A
     float hi[kTeamRows], lo[kTeamRows];

@@ -100,34 +100,37 @@ class Path:
     def __init__(self, states: list[LayerState], device):
         self.states = states
         self.device = device
-        self.aux_jobs = [s.aux_job() for s in states]
         self.mul = [s for s in states if s.spec.variant == "mul"]
         self.shift = [s for s in states if s.spec.variant == "shift"]
         self.ste = [s for s in states if s.G is not None]
+        # descriptors are converted to C structs once: the buffers never move
+        self.aux_jobs = B.Descriptors(s.aux_job() for s in states)
         self.ws_aux = workspace(B.intlora_gen_aux_workspace_size(self.aux_jobs), device)
         self.ws_merge = workspace(B.intlora_merge_workspace_size(
             [s.layer() for s in states]), device)
-
-    def prepare(self, stream=None):
-        B.intlora_gen_aux_batched(self.aux_jobs, self.ws_aux, stream)
-
-    def merge(self, stream=None):
         groups = {}
         for s in self.mul:
             groups.setdefault(("mul", s.spec.out_bits), []).append(s)
         for s in self.shift:
             groups.setdefault(("shift", s.spec.out_bits), []).append(s)
-        for (kind, bits), sts in groups.items():
-            layers = [s.layer() for s in sts]
-            outs = [s.merge_out() for s in sts]
+        self.merge_groups = [(kind, bits, B.Descriptors(s.layer() for s in sts),
+                              B.Descriptors(s.merge_out() for s in sts))
+                             for (kind, bits), sts in groups.items()]
+        self.ste_jobs = B.Descriptors(s.ste_job() for s in self.ste) if self.ste else None
+
+    def prepare(self, stream=None):
+        B.intlora_gen_aux_batched(self.aux_jobs, self.ws_aux, stream)
+
+    def merge(self, stream=None):
+        for kind, bits, layers, outs in self.merge_groups:
             if kind == "mul":
                 B.intlora_merge_mul_batched(layers, outs, bits, self.ws_merge, stream)
             else:
                 B.intlora_merge_shift_batched(layers, outs, bits, self.ws_merge, stream)
 
     def backward(self, stream=None):
-        if self.ste:
-            B.intlora_ste_backward_batched([s.ste_job() for s in self.ste], None, stream)
+        if self.ste_jobs is not None:
+            B.intlora_ste_backward_batched(self.ste_jobs, None, stream)
 
     def step(self, stream=None):
         self.prepare(stream)

@@ -264,6 +264,14 @@ intlora_status intlora_ste_backward(const void* G, const void* A, const void* B,
 intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t count,
                                             void* ws, size_t ws_bytes, void* stream);
 
+/* Number of bounded device-side waits that gave up since the library was
+ * loaded: 0 in a healthy run. The tensor-core STE kernel bounds every wait on
+ * an mbarrier (2 s); a wait that gives up is counted here, the CTA stops, releases its
+ * tensor memory and returns, so a broken run shows up as a nonzero count and
+ * wrong outputs instead of a hung device. Synchronous (reads one device
+ * word); the library has no counterpart of this on the pages. */
+uint32_t intlora_device_timeouts(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -651,7 +651,41 @@ intlora_status check_ste(const intlora_ste_job& j, int idx) {
 
 constexpr int kSteBM = 64, kSteRB = 32, kSteTargetCtas = 148 * 4;
 
+// INTLORA_STE_KERNEL=cuda keeps the STE backward on the CUDA-core kernels;
+// unset or "auto": the tensor-core kernel takes every batch it supports.
+bool ste_tc_enabled() {
+  const char* v = std::getenv("INTLORA_STE_KERNEL");
+  return v == nullptr || std::strcmp(v, "cuda") != 0;
+}
+
 intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_t st) {
+  if (ste_tc_enabled()) {
+    // tensor-core pass: both products from one read of G
+    SteBatch b;
+    std::memset(&b, 0, sizeof b);
+    bool ok = true;
+    for (int32_t k = 0; k < count && ok; ++k) {
+      const intlora_ste_job& j = jobs[k];
+      SteJob& s = b.job[k];
+      s.G = static_cast<const uint16_t*>(j.G);
+      s.A = static_cast<const uint16_t*>(j.A);
+      s.B = static_cast<const uint16_t*>(j.B);
+      s.d = j.d;
+      s.n = j.n;
+      s.r = j.r;
+      s.dA = j.dA;
+      s.dB = j.dB;
+      ok = ste_tc_supported(s);
+    }
+    if (ok) {
+      b.count = count;
+      cudaError_t e = launch_ste_zero(b, st);
+      if (e != cudaSuccess) return cuda_fail(e, "STE zero launch");
+      e = launch_ste_tc(b.job, count, st);
+      if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE kernel launch");
+      return INTLORA_OK;
+    }
+  }
   // Ranks up to 8 with n % 8 == 0: one fused pass over G (both outputs).
   int max_r = 0;
   bool fusable = true;
@@ -745,6 +779,8 @@ const char* intlora_status_string(int status) {
 const char* intlora_last_error(void) { return g_last_error; }
 
 int intlora_version(void) { return 100; }
+
+uint32_t intlora_device_timeouts(void) { return intlora::ste_tc_timeouts(); }
 
 int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits) {
   if ((variant != 0 && variant != 1) || (w_bits != 4 && w_bits != 8)) return 0;

@@ -178,6 +178,13 @@ int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes
 cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s);
 int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
+cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s);   // dA and dB of every job
+// tcgen05 path of the STE backward (one pass over G, both products on the
+// tensor cores); outputs must be zeroed first.
+constexpr int kSteTcMaxRank = 128;
+bool ste_tc_supported(const SteJob& j);
+cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s);
+unsigned int ste_tc_timeouts();
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 
 // Sets the calling thread's intlora_last_error() message.

@@ -269,6 +269,14 @@ __global__ void ste_zero_kernel(const __grid_constant__ SteBatch b) {
 
 }  // namespace
 
+cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s) {
+  if (b.count <= 0) return cudaSuccess;
+  SteBatch z = b;
+  z.fused = 1;                     // both outputs
+  ste_zero_kernel<<<148 * 4, 256, 0, s>>>(z);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s) {
   if (b.count <= 0) return cudaSuccess;
   if (b.fused) {

@@ -27,6 +27,7 @@ namespace {
 
 constexpr double kLn2 = 0.69314718055994530942;
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kSlotWords = 2 * kTeamRows;      // row maxima and negated minima of one warp
 
 __device__ __forceinline__ uint32_t ord(float v) { return __float_as_uint(fabsf(v)); }
 
@@ -50,14 +51,13 @@ __device__ __forceinline__ uint32_t load_quad_codes(const uint8_t* row, int64_t 
                     : static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(row + (j >> 1))));
 }
 
-// One of the four values selected by a small runtime index, without a local
-// array (keeps the operands in registers).
+// One of the kTeamRows values selected by a small runtime index, without a
+// local array (keeps the operands in registers).
 template <typename T>
-__device__ __forceinline__ T pick4(const T v[4], int k) {
+__device__ __forceinline__ T pick_row(const T v[kTeamRows], int k) {
   T x = v[0];
-  x = k == 1 ? v[1] : x;
-  x = k == 2 ? v[2] : x;
-  x = k == 3 ? v[3] : x;
+#pragma unroll
+  for (int ml = 1; ml < kTeamRows; ++ml) x = k == ml ? v[ml] : x;
   return x;
 }
 
@@ -66,9 +66,11 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
   extern __shared__ __align__(16) float4 smem4[];
   const int smax = p.sweeps_max;
   float4* Ubuf = smem4;                                              // [smax][4][256]
-  uint4* Cbuf = reinterpret_cast<uint4*>(smem4 + smax * kTeamRows * kTeamThreads);   // [smax][256]
-  uint32_t* slots = reinterpret_cast<uint32_t*>(Cbuf + (VARIANT == kGen ? 0 : smax * kTeamThreads));
-  float* rcp_tab = reinterpret_cast<float*>(slots + 2 * kTeamWarps * 8);   // 1/D, D in [-255, 255]
+  // code words of the merges: [smax][kTeamRows][256]
+  uint32_t* Cbuf = reinterpret_cast<uint32_t*>(smem4 + smax * kTeamRows * kTeamThreads);
+  // row extrema of every warp: [2][warps][2 kTeamRows] (double buffered)
+  uint32_t* slots = Cbuf + (VARIANT == kGen ? 0 : smax * kTeamRows * kTeamThreads);
+  float* rcp_tab = reinterpret_cast<float*>(slots + 2 * kTeamWarps * kSlotWords);   // 1/D, D in [-255, 255]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qmax = (1 << p.bits) - 1;
@@ -238,7 +240,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
                           laplace_scaled(words[2], c_ln2), laplace_scaled(words[3], c_ln2));
         }
       }
-      if (VARIANT != kGen) Cbuf[k * kTeamThreads + tid] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      if (VARIANT != kGen) {
+#pragma unroll
+        for (int ml = 0; ml < kTeamRows; ++ml) Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] = cw[ml];
+      }
     }
 
     // ---- row extrema: over the warp (REDUX), then over the team
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       elo[ml] = VARIANT == kShift ? 0u : __reduce_max_sync(kFull, ord(lo[ml]));
     }
     if (TW > 1) {
-      uint32_t* mine = slots + ((phase & 1u) * kTeamWarps + warp) * 8;
+      uint32_t* mine = slots + ((phase & 1u) * kTeamWarps + warp) * kSlotWords;
       if (lane == 0) {
 #pragma unroll
         for (int ml = 0; ml < kTeamRows; ++ml) {
@@ -258,12 +263,12 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         }
       }
       team_barrier(1 + team, LT);
-      // lane v < 8 gathers value v over the team's warps, then every lane
-      // takes the 8 combined values by shuffles
+      // lane v < 2 kTeamRows gathers value v over the team's warps, then
+      // every lane takes the combined values by shuffles
       uint32_t acc = 0u;
-      if (lane < 8) {
-        const uint32_t* base = slots + ((phase & 1u) * kTeamWarps + team * TW) * 8 + lane;
-        for (int w2 = 0; w2 < TW; ++w2) acc = max(acc, base[w2 * 8]);
+      if (lane < kSlotWords) {
+        const uint32_t* base = slots + ((phase & 1u) * kTeamWarps + team * TW) * kSlotWords + lane;
+        for (int w2 = 0; w2 < TW; ++w2) acc = max(acc, base[w2 * kSlotWords]);
       }
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml) {
@@ -277,8 +282,8 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
     float scale = 1.0f;
     int32_t zero = 0;
     {
-      const float top = __uint_as_float(pick4(ehi, lane & 3));
-      const float neg_bottom = __uint_as_float(pick4(elo, lane & 3));
+      const float top = __uint_as_float(pick_row(ehi, lane & (kTeamRows - 1)));
+      const float neg_bottom = __uint_as_float(pick_row(elo, lane & (kTeamRows - 1)));
       if (VARIANT == kShift) {
         scale = top > 0.0f ? top : 1.0f;
       } else {
@@ -306,9 +311,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       const int q = lt + k * LT;
       if (q >= quads) break;
       const int64_t j = 4 * static_cast<int64_t>(q);
-      uint4 cw4 = make_uint4(0u, 0u, 0u, 0u);
-      if (VARIANT != kGen) cw4 = Cbuf[k * kTeamThreads + tid];
-      const uint32_t cw[kTeamRows] = {cw4.x, cw4.y, cw4.z, cw4.w};
+      uint32_t cw[kTeamRows];
+#pragma unroll
+      for (int ml = 0; ml < kTeamRows; ++ml)
+        cw[ml] = VARIANT != kGen ? Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] : 0u;
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml) {
         if (ml >= rows) break;
@@ -439,8 +445,8 @@ void team_dispatch(TeamQuery& q, int variant, int w_bits, int rank_ct, int out_b
 
 size_t team_smem_bytes(int variant, int sweeps_max) {
   const size_t per_sweep = static_cast<size_t>(kTeamRows) * kTeamThreads * 16 +
-                           (variant == kGen ? 0 : static_cast<size_t>(kTeamThreads) * 16);
-  return per_sweep * sweeps_max + 2 * kTeamWarps * 8 * 4 + (variant == kGen ? 0 : 512 * 4);
+                           (variant == kGen ? 0 : static_cast<size_t>(kTeamRows) * kTeamThreads * 4);
+  return per_sweep * sweeps_max + 2 * kTeamWarps * kSlotWords * 4 + (variant == kGen ? 0 : 512 * 4);
 }
 
 cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s) {

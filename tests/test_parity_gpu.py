@@ -3,11 +3,13 @@ seeded inputs, through the C ABI. Each stage is fed the oracle's inputs, so a
 difference in one stage cannot cascade into the next."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
+from quantized_lora_merge_b200 import binding as B
 from quantized_lora_merge_b200 import workloads as wl
 
-from .parity import (STE_RTOL, assert_affine, assert_scale, assert_shift, gpu_gen_aux,
+from .parity import (STE_RTOL, assert_affine, assert_scale, assert_shift, dev, gpu_gen_aux,
                      gpu_merge, gpu_ste, rel_fro, spec_for)
 
 pytestmark = pytest.mark.gpu
@@ -179,6 +181,51 @@ def test_ste_parity(d, n, r):
     oA, oB = oracle.ste_backward(G, A, Bm)
     assert rel_fro(dA, oA) < STE_RTOL
     assert rel_fro(dB, oB) < STE_RTOL
+
+
+@pytest.mark.parametrize("d,n,r", [(100, 304, 128), (257, 1032, 33), (129, 136, 1), (1, 8, 4),
+                                   (4096, 1024, 64), (130, 4104, 8)])
+def test_ste_tensor_core_parity(d, n, r):
+    """Shapes the tensor-core pass takes (n % 8 == 0, r <= 128): ragged row
+    blocks and column tiles, padded ranks (1, 8, 33 -> 16, 16, 48)."""
+    spec = spec_for(d, n, r, 8, sid=d + 1)
+    Gb = wl.host_G_bits(spec)
+    Ab = wl.to_bf16_bits(wl.host_A(spec))
+    Bb = wl.to_bf16_bits(wl.host_B(spec))
+    dA, dB = gpu_ste(Gb, Ab, Bb)
+    G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+    oA, oB = oracle.ste_backward(G, A, Bm)
+    assert rel_fro(dA, oA) < STE_RTOL
+    assert rel_fro(dB, oB) < STE_RTOL
+
+
+def test_ste_batched_mixed_ranks_both_kernels(monkeypatch):
+    """One batched call over layers of different shapes and ranks, through the
+    tensor-core pass and through the CUDA-core kernels: both match the oracle."""
+    specs = [spec_for(d, n, r, 8, sid=40 + k) for k, (d, n, r) in
+             enumerate([(320, 320, 4), (200, 768, 8), (64, 1280, 16), (384, 256, 2)])]
+    host = [(wl.host_G_bits(s), wl.to_bf16_bits(wl.host_A(s)), wl.to_bf16_bits(wl.host_B(s)))
+            for s in specs]
+    for kernel in ("auto", "cuda"):
+        monkeypatch.setenv("INTLORA_STE_KERNEL", kernel)
+        jobs = []
+        for spec, (Gb, Ab, Bb) in zip(specs, host):
+            t = [torch.from_numpy(x.view(np.int16)).to(dev()).view(torch.bfloat16) for x in (Gb, Ab, Bb)]
+            jobs.append(B.SteJob(t[0], t[1], t[2],
+                                 torch.full((spec.d, spec.r), np.nan, device=dev()),
+                                 torch.full((spec.r, spec.n), np.nan, device=dev())))
+        B.intlora_ste_backward_batched(jobs)
+        torch.cuda.synchronize()
+        for job, (Gb, Ab, Bb) in zip(jobs, host):
+            G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+            oA, oB = oracle.ste_backward(G, A, Bm)
+            assert rel_fro(job.dA.cpu().numpy(), oA) < STE_RTOL, kernel
+            assert rel_fro(job.dB.cpu().numpy(), oB) < STE_RTOL, kernel
+
+
+def test_no_device_wait_gave_up():
+    """Every bounded wait of the tensor-core kernels finished in time."""
+    assert B.intlora_device_timeouts() == 0
 
 
 def test_batches_with_mixed_seeds():

@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "intlora_device.cuh"
 #include "intlora_kernels.h"
@@ -269,18 +270,65 @@ __global__ void ste_zero_kernel(const __grid_constant__ SteBatch b) {
 
 }  // namespace
 
+namespace {
+
+// Zeroing of many small buffers in one launch: every CTA clears one chunk of
+// kZeroChunk floats of one segment.
+constexpr int kZeroSegments = 2 * kMaxBatch;
+constexpr int kZeroChunk = 4096;
+struct ZeroBatch {
+  float* ptr[kZeroSegments];
+  int64_t count[kZeroSegments];
+  int32_t block_begin[kZeroSegments + 1];
+  int32_t segments;
+};
+
+__global__ void __launch_bounds__(256) zero_segments_kernel(const __grid_constant__ ZeroBatch z) {
+  const int bid = blockIdx.x;
+  int lo = 0, hi = z.segments - 1;         // last segment whose first block <= bid
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (z.block_begin[mid] <= bid) lo = mid;
+    else hi = mid - 1;
+  }
+  const int64_t base = static_cast<int64_t>(bid - z.block_begin[lo]) * kZeroChunk;
+  const int64_t end = min64(z.count[lo], base + kZeroChunk);
+  float* p = z.ptr[lo];
+  for (int64_t k = base + threadIdx.x; k < end; k += 256) p[k] = 0.0f;
+}
+
+}  // namespace
+
 cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s) {
   if (b.count <= 0) return cudaSuccess;
-  SteBatch z = b;
-  z.fused = 1;                     // both outputs
-  ste_zero_kernel<<<148 * 4, 256, 0, s>>>(z);
+  ZeroBatch z;
+  std::memset(&z, 0, sizeof z);
+  int blocks = 0, seg = 0;
+  for (int j = 0; j < b.count; ++j) {
+    const SteJob& J = b.job[j];
+    const int64_t counts[2] = {J.d * J.r, static_cast<int64_t>(J.r) * J.n};
+    float* ptrs[2] = {J.dA, J.dB};
+    for (int w = 0; w < 2; ++w) {
+      if (counts[w] <= 0) continue;
+      z.ptr[seg] = ptrs[w];
+      z.count[seg] = counts[w];
+      z.block_begin[seg] = blocks;
+      blocks += static_cast<int>((counts[w] + kZeroChunk - 1) / kZeroChunk);
+      ++seg;
+    }
+  }
+  z.segments = seg;
+  z.block_begin[seg] = blocks;
+  if (blocks == 0) return cudaSuccess;
+  zero_segments_kernel<<<blocks, 256, 0, s>>>(z);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s) {
   if (b.count <= 0) return cudaSuccess;
   if (b.fused) {
-    ste_zero_kernel<<<148 * 4, 256, 0, s>>>(b);
+    cudaError_t e = launch_ste_zero(b, s);
+    if (e != cudaSuccess) return e;
     if (b.fused == 4)
       ste_fused_kernel<4><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
     else

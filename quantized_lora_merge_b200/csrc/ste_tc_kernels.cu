@@ -35,6 +35,7 @@ constexpr int kTileCols = 128;                 // columns of G per tile (GEMM1 K
 constexpr uint32_t kGBytes = kTileRows * kTileCols * 2;
 constexpr uint32_t kBoxBytes = kTileRows * 64 * 2;    // one 64-column box of the G tile
 constexpr int kMaxTcJobs = 64;
+constexpr int kMaxD2 = 8;                      // D2 accumulators (tile epilogues in flight)
 constexpr uint64_t kWaitNs = 2000000000ull;  // a wait gives up after 2 s
 
 struct alignas(64) SteTcJob {
@@ -56,6 +57,8 @@ struct SteTcBatch {
   int32_t rp;                 // r rounded up to a multiple of 16 (MMA N)
   int32_t tiles_per_unit;
   int32_t stages;
+  int32_t nd2;
+  int32_t ctas_per_sm;
   int64_t total_units;
   uint32_t tmem_cols;
   unsigned int* timeouts;
@@ -199,7 +202,7 @@ __device__ __forceinline__ Unit decode_unit(const SteTcBatch& b, int64_t u) {
   return x;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_constant__ SteTcBatch b) {
+__global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_constant__ SteTcBatch b) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -213,12 +216,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
   uint64_t* bars = reinterpret_cast<uint64_t*>(sA + 2 * b_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
+  const int ND2 = b.nd2;                                       // D2 accumulators in the ring
   uint64_t* d2_full = bars + 2 * S;
-  uint64_t* d2_empty = d2_full + 2;
-  uint64_t* d1_full = d2_full + 4;
-  uint64_t* d1_empty = d2_full + 6;
-  uint64_t* a_full = d2_full + 8;
-  uint64_t* a_empty = d2_full + 10;
+  uint64_t* d2_empty = d2_full + kMaxD2;
+  uint64_t* d1_full = d2_empty + kMaxD2;
+  uint64_t* d1_empty = d1_full + 2;
+  uint64_t* a_full = d1_full + 4;
+  uint64_t* a_empty = d1_full + 6;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -226,9 +230,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int q = 0; q < 2; ++q) {
+    for (int q = 0; q < ND2; ++q) {
       mbar_init(&d2_full[q], 1);
       mbar_init(&d2_empty[q], 128);
+    }
+    for (int q = 0; q < 2; ++q) {
       mbar_init(&d1_full[q], 1);
       mbar_init(&d1_empty[q], 128);
       mbar_init(&a_full[q], 64);
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  // TMEM columns: D1[2] at 0 and RP, D2[2] at 2 RP and 3 RP
+  // TMEM columns: D1[2] at 0 and RP, D2[q] at (2 + q) RP
   const uint32_t idesc1 = instr_desc(RP, false);
   const uint32_t idesc2 = instr_desc(RP, true);
 
@@ -289,7 +295,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
         if (!mbar_wait(&d1_empty[ab], aph ^ 1u, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d1 = tmem + static_cast<uint32_t>(ab * RP);
-        const uint32_t a_addr = smem_u32(sA + ab * b_bytes);
+        const uint64_t a0 = smem_desc(smem_u32(sA + ab * b_bytes), 16, 1024);
         bool ok = true;
         for (int ct = x.ct0; ct < x.ct1; ++ct) {
           if (!mbar_wait(&full[stage], ph, &abort_flag) || !mbar_wait(&d2_empty[d2], d2ph ^ 1u, &abort_flag)) {
@@ -297,24 +303,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
-          const uint32_t g_addr = smem_u32(sG + stage * kGBytes);
-          const uint32_t bt_addr = smem_u32(sB + stage * b_bytes);
+          // descriptors of this stage; the K steps only move the start address
+          // (16-byte units): 32 bytes per K step inside a 128-byte row, one
+          // 64-column atom further every 4 steps; 16 rows per GEMM2 step
+          const uint64_t gk0 = smem_desc(smem_u32(sG + stage * kGBytes), 16, 1024);
+          const uint64_t gm0 = smem_desc(smem_u32(sG + stage * kGBytes), kBoxBytes, 1024);
+          const uint64_t bt0 = smem_desc(smem_u32(sB + stage * b_bytes), 16, 1024);
           const uint32_t d2t = tmem + static_cast<uint32_t>((2 + d2) * RP);
+          const uint32_t acc1 = ct > x.ct0 ? 1u : 0u;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             // GEMM1: K = 16 columns of the tile; both operands K-major
-            const uint32_t koff = (ks & 3) * 32u;             // 16 bf16 inside the 128-byte row
-            const uint64_t ga = smem_desc(g_addr + (ks >> 2) * kBoxBytes + koff, 16, 1024);
-            const uint64_t bb = smem_desc(bt_addr + (ks >> 2) * (RP * 128) + koff, 16, 1024);
-            tc_mma(d1, ga, bb, idesc1, (ct > x.ct0 || ks > 0) ? 1u : 0u);
+            const uint64_t koff = static_cast<uint64_t>((ks & 3) * 2);
+            tc_mma(d1, gk0 + static_cast<uint64_t>((ks >> 2) * (kBoxBytes >> 4)) + koff,
+                   bt0 + static_cast<uint64_t>((ks >> 2) * (RP * 8)) + koff, idesc1,
+                   (acc1 | static_cast<uint32_t>(ks)) != 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             // GEMM2: K = 16 rows of the tile; A = G tile MN-major (64-column
             // atoms kBoxBytes apart, 8-row groups 1024 bytes apart), B = A block
-            const uint64_t ga = smem_desc(g_addr + ks * 2048, kBoxBytes, 1024);
-            const uint64_t ab_desc = smem_desc(a_addr + (ks >> 2) * (RP * 128) + (ks & 3) * 32, 16, 1024);
-            tc_mma(d2t, ga, ab_desc, idesc2, ks > 0 ? 1u : 0u);
+            tc_mma(d2t, gm0 + static_cast<uint64_t>(ks * 128),
+                   a0 + static_cast<uint64_t>((ks >> 2) * (RP * 8) + (ks & 3) * 2), idesc2, ks > 0 ? 1u : 0u);
           }
           tc_commit(&empty[stage]);
           tc_commit(&d2_full[d2]);
@@ -322,7 +332,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
             stage = 0;
             ph ^= 1u;
           }
-          if (++d2 == 2) {
+          if (++d2 == ND2) {
             d2 = 0;
             d2ph ^= 1u;
           }
@@ -386,7 +396,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ste_tc_kernel(const __grid_cons
         }
         tc_fence_before();
         mbar_arrive(&d2_empty[d2]);
-        if (++d2 == 2) {
+        if (++d2 == ND2) {
           d2 = 0;
           d2ph ^= 1u;
         }
@@ -453,7 +463,7 @@ bool encode_bf16(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, 
 
 size_t tc_smem_bytes(int rp, int stages) {
   const size_t b_bytes = static_cast<size_t>(rp) * 256;
-  return 1024 + stages * (kGBytes + b_bytes) + 2 * b_bytes + (2 * stages + 12) * 8;
+  return 1024 + stages * (kGBytes + b_bytes) + 2 * b_bytes + (2 * stages + 2 * kMaxD2 + 8) * 8;
 }
 
 }  // namespace
@@ -475,8 +485,9 @@ cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s) {
     int max_r = 1;
     for (int k = 0; k < m; ++k) max_r = jobs[base + k].r > max_r ? jobs[base + k].r : max_r;
     const int rp = (max_r + 15) / 16 * 16;
-    // about 1 MB of G per unit keeps units many and epilogues rare
-    b.tiles_per_unit = 8;
+    // 128 x 2048 of G (512 KB) per unit at most: units many enough to balance,
+    // D1 epilogues rare
+    b.tiles_per_unit = 16;
     int64_t units = 0;
     for (int k = 0; k < m; ++k) {
       const SteJob& j = jobs[base + k];
@@ -496,18 +507,27 @@ cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s) {
     }
     b.count = m;
     b.rp = rp;
-    int stages = 4;
-    while (stages > 2 && tc_smem_bytes(rp, stages) > 232448 - 1024) --stages;
+    // two CTAs per SM when their tensor memory fits (two independent
+    // load -> MMA -> epilogue chains per SM), else one with deeper buffers
+    const int per_sm = 6 * rp <= 256 ? 2 : 1;
+    const uint32_t col_budget = 512 / per_sm;
+    int nd2 = static_cast<int>(col_budget / rp) - 2;
+    nd2 = nd2 > kMaxD2 ? kMaxD2 : nd2;
+    int stages = per_sm == 2 ? 3 : 4;
+    const size_t smem_cap = (233472 / per_sm) - 1024;
+    while (stages > 2 && tc_smem_bytes(rp, stages) > smem_cap) --stages;
     b.stages = stages;
+    b.nd2 = nd2;
+    b.ctas_per_sm = per_sm;
     b.total_units = units;
     uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(4 * rp)) cols <<= 1;
+    while (cols < static_cast<uint32_t>((2 + nd2) * rp)) cols <<= 1;
     b.tmem_cols = cols;
     const size_t smem = tc_smem_bytes(rp, stages);
     cudaError_t e = cudaFuncSetAttribute(ste_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int64_t grid = units < sms ? units : sms;
+    const int64_t grid = units < int64_t{per_sm} * sms ? units : int64_t{per_sm} * sms;
     ste_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(b);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

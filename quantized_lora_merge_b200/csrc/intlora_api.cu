@@ -43,7 +43,7 @@ size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 constexpr int64_t kMaxElements = int64_t{1} << 40;
 constexpr int kStatsThreadsHost = 256;
-constexpr int kStatsGroupsPerThread = 8;
+constexpr int kStatsGroupsPerThread = 64;
 constexpr int kStatsMaxBlocksPerJob = 148 * 8;
 
 int64_t stats_blocks(int64_t numel) {

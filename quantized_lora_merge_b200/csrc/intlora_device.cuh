@@ -60,16 +60,19 @@ __device__ __forceinline__ uint32_t aux_word(uint64_t e, uint32_t stream_id, uin
 // c * R for the Laplace sample of word x, with c_ln2 = c * ln 2 (fp32).
 //
 // With k = x >> 9 (23 bits), u = (2k + 1) 2^-24 and v = u - 1/2, the inverse
-// CDF gives R = -sign(v) ln(1 - 2|v|). Folding the sign: 1 - 2|v| = m 2^-23
-// with m = 2k' + 1, k' = k for v < 0 and 2^23 - 1 - k for v > 0, i.e. k' is
-// bits 9..30 of x XOR (x's sign bit replicated). m 2^-23 is built exactly as
-// the float (1 + m 2^-23) - 1. sign(v) = +1 exactly when bit 31 of x is set,
-// so R = ln2 * log2(m 2^-23) with the sign flipped for those words.
+// CDF gives R = -sign(v) ln(1 - 2|v|). Every step below is exact in fp32:
+//   f  = 1 + k 2^-23                     (the bits 0x3F800000 | k, built by one
+//                                         funnel shift of 0x7F:x by 9)
+//   u2 = 2 f - (2 - 2^-23) = (2k + 1) 2^-23 = 2u
+//   w  = 1 - |u2 - 1|      = 1 - 2|v|   (an odd multiple of 2^-23 in (0, 1))
+// so log2(w) is taken of the exact argument; the sign of R is that of -v,
+// i.e. + exactly when bit 31 of x is clear. Most of the work sits on the FMA
+// pipe rather than the integer/logic pipe.
 __device__ __forceinline__ float laplace_log2(uint32_t x) {
-  const uint32_t sign_mask = static_cast<uint32_t>(static_cast<int32_t>(x) >> 31);
-  const uint32_t folded = x ^ sign_mask;                       // bit 31 now clear
-  const float one_plus = __uint_as_float((folded >> 8) | 0x3F800001u);
-  return __log2f(one_plus - 1.0f);                             // log2(m 2^-23) < 0, exact input
+  const float f = __uint_as_float(__funnelshift_r(x, 0x7Fu, 9));
+  const float u2 = fmaf(2.0f, f, -1.99999988079071044921875f);   // -(2 - 2^-23)
+  const float w = 1.0f - fabsf(u2 - 1.0f);
+  return __log2f(w);                                              // log2(1 - 2|v|) < 0
 }
 // +-c ln2: the factor that turns laplace_log2(x) into c * R.
 __device__ __forceinline__ float laplace_sign(uint32_t x, float c_ln2) {

@@ -41,7 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="sd_unet")
@@ -144,7 +144,7 @@ def profiled_traffic(name):
 
 
 def ste_bytes(l):
-    # G read once per contraction (the CUDA-core path reads it twice), A, B, dA, dB
+    # G read once (both products from one pass), A, B, dA, dB
     return l.numel * 2 + l.r * (l.d + l.n) * (2 + 4)
 
 
@@ -310,6 +310,10 @@ def main():
         t = wl.device_inputs(spec, device, with_grad=True, salt=rank)
         states.append(P.allocate(spec, t["W"], t["A"], t["B"], device, G=t["G"], A16=t["A16"],
                                  B16=t["B16"]))
+    # inputs and outputs each live in one arena, so the end-to-end leg moves
+    # them with one host<->device copy per direction
+    arena_in, arena_out = P.pack_io(states, device)
+    torch.cuda.empty_cache()
     path = P.Path(states, device)
     stream = torch.cuda.current_stream(device)
 
@@ -366,13 +370,16 @@ def main():
         stages[name] = {"ms": ms, "algorithmic_GB": per_stage_bytes[name] / 1e9,
                         "GB_s": gbs, "frac_of_hbm": gbs / hbm_peak}
     stages["merge"]["elements_per_s"] = sum(l.numel for l in layers) / (stage_ms["merge"] / 1e3)
-    # dominant kernel: the merge's row-tile kernel (one launch per step); it is
+    # dominant kernel: the merge's team kernel (one launch per step); it is
     # bound by ALU issue (Philox + Laplace per element), so its roofline is the
     # SM lane-issue rate at the measured SM clock; HBM fraction reported beside
     sm_mhz = clk.get("sm_mhz") or 1965.0
     alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
     alu_achieved = sum(merge_ops(l) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
-    launches_per_step = {"prepare": 3, "merge": 1, "ste_backward": 2}
+    # prepare: statistics + finalize + base quantization; merge: one team
+    # launch; STE: zeroing + one tensor-core launch per 64 layers
+    launches_per_step = {"prepare": 3, "merge": 1,
+                         "ste_backward": 1 + (len(layers) + 63) // 64}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -381,22 +388,22 @@ def main():
         "config": desc,
         "hbm_GB_s_merge": stages["merge"]["GB_s"],
         "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
-        "roofline": {"bound": "alu", "kernel": "merge row-tile kernel (MUL, 1 launch per step)",
+        "roofline": {"bound": "alu", "kernel": "merge team kernel (MUL, 1 launch per step)",
                      "achieved": alu_achieved, "peak": alu_peak, "unit": "Top/s",
                      "frac": alu_achieved / alu_peak,
                      "peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
                      "ops_per_element": merge_ops(layers[0]) / layers[0].numel,
                      "hbm_achieved_GB_s": stages["merge"]["GB_s"], "hbm_peak_GB_s": hbm_peak,
                      "hbm_peak_source": peak_kind, "hbm_frac": stages["merge"]["frac_of_hbm"],
-                     "traffic": profiled_traffic("tile_kernel_mul_sd_unet")},
+                     "traffic": profiled_traffic("team_kernel_mul_sd_unet")},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": args.steps * sum(launches_per_step.values()),
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e(path, states, device, stream, max(2, min(args.steps, 5)), world,
-                          elements)
+        line["e2e"] = e2e(path, arena_in, arena_out, device, stream, max(2, min(args.steps, 5)),
+                          world, elements)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
     if rank == 0:
@@ -405,33 +412,23 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e(path, states, device, stream, steps, world, elements):
+def e2e(path, arena_in, arena_out, device, stream, steps, world, elements):
     """Same step through the public API with HOST buffers: every step copies
-    the step's inputs from pinned host memory, runs the path and reads the
-    merged weights, scales and gradients back."""
+    the step's inputs (one pinned host arena holding every layer's W, A, B, G
+    and bf16 A, B) to the device, runs the path and reads the merged weights,
+    scales, zero-points and gradients back (one arena)."""
     import torch
     import torch.distributed as dist
-    host_in, host_out = [], []
-    for st in states:
-        hi = {k: torch.empty(getattr(st, k).shape, dtype=getattr(st, k).dtype, pin_memory=True)
-              for k in ("W", "A", "B", "G", "A16", "B16")}
-        for k, v in hi.items():
-            v.copy_(getattr(st, k))
-        ho = {k: torch.empty(getattr(st, k).shape, dtype=getattr(st, k).dtype, pin_memory=True)
-              for k in ("out", "sbar", "zbar", "dA", "dB")}
-        host_in.append(hi)
-        host_out.append(ho)
-    h2d = sum(v.numel() * v.element_size() for hi in host_in for v in hi.values())
-    d2h = sum(v.numel() * v.element_size() for ho in host_out for v in ho.values())
+    host_in = torch.empty(arena_in.numel(), dtype=torch.uint8, pin_memory=True)
+    host_in.copy_(arena_in)
+    host_out = torch.empty(arena_out.numel(), dtype=torch.uint8, pin_memory=True)
+    h2d = host_in.numel()
+    d2h = host_out.numel()
 
     def one():
-        for st, hi in zip(states, host_in):
-            for k, v in hi.items():
-                getattr(st, k).copy_(v, non_blocking=True)
+        arena_in.copy_(host_in, non_blocking=True)
         path.step()
-        for st, ho in zip(states, host_out):
-            for k, v in ho.items():
-                v.copy_(getattr(st, k), non_blocking=True)
+        host_out.copy_(arena_out, non_blocking=True)
 
     one()
     torch.cuda.synchronize(device)

@@ -86,6 +86,40 @@ def allocate(spec: LayerSpec, W, A, Bm, device, G=None, A16=None, B16=None,
     return st
 
 
+def arena(tensors: list[torch.Tensor], device) -> tuple[torch.Tensor, list[torch.Tensor]]:
+    """One device buffer holding copies of `tensors` (each at a 256-byte
+    aligned offset) and views of it with the tensors' shapes and dtypes: a
+    host mirror of the buffer then moves with one copy per direction."""
+    offsets, total = [], 0
+    for t in tensors:
+        offsets.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    buf = torch.empty(max(total, 256), dtype=torch.uint8, device=device)
+    views = []
+    for t, off in zip(tensors, offsets):
+        nb = t.numel() * t.element_size()
+        v = buf[off:off + nb].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return buf, views
+
+
+def pack_io(states: list[LayerState], device) -> tuple[torch.Tensor, torch.Tensor]:
+    """Moves every layer's inputs (W, A, B and the STE operands) into one
+    arena and its outputs (merged weights, scales, zero-points, gradients)
+    into another; returns (inputs, outputs). Build the Path afterwards."""
+    in_keys = ("W", "A", "B", "G", "A16", "B16")
+    out_keys = ("out", "sbar", "zbar", "dA", "dB")
+    groups = []
+    for keys in (in_keys, out_keys):
+        slots = [(st, k) for st in states for k in keys if getattr(st, k) is not None]
+        buf, views = arena([getattr(st, k) for st, k in slots], device)
+        for (st, k), v in zip(slots, views):
+            setattr(st, k, v)
+        groups.append(buf)
+    return groups[0], groups[1]
+
+
 def workspace(nbytes: int, device) -> torch.Tensor | None:
     if nbytes <= 0:
         return None

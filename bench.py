@@ -402,8 +402,8 @@ def main():
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e(path, arena_in, arena_out, device, stream, max(2, min(args.steps, 5)),
-                          world, elements)
+        line["e2e"] = e2e(layers, path, arena_in, arena_out, device,
+                          max(4, min(args.steps, 10)), world, elements)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
     if rank == 0:
@@ -412,34 +412,78 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e(path, arena_in, arena_out, device, stream, steps, world, elements):
+def e2e(layers, path, arena_in, arena_out, device, steps, world, elements):
     """Same step through the public API with HOST buffers: every step copies
     the step's inputs (one pinned host arena holding every layer's W, A, B, G
     and bf16 A, B) to the device, runs the path and reads the merged weights,
-    scales, zero-points and gradients back (one arena)."""
+    scales, zero-points and gradients back (one arena).
+
+    Steps are pipelined over two device copies of the workload and three
+    streams, as a streaming caller would run them: the inputs of step k+1
+    travel host->device while step k computes and step k-1's results travel
+    device->host. Every step still moves all of its bytes both ways inside
+    the timed region."""
     import torch
     import torch.distributed as dist
+    from quantized_lora_merge_b200 import pipeline as P
+    # second device copy of the workload (same layers, own buffers)
+    states2 = [P.allocate(l, torch.empty(l.d, l.n, device=device),
+                          torch.empty(l.d, l.r, device=device),
+                          torch.empty(l.r, l.n, device=device), device,
+                          G=torch.empty(l.d, l.n, dtype=torch.bfloat16, device=device),
+                          A16=torch.empty(l.d, l.r, dtype=torch.bfloat16, device=device),
+                          B16=torch.empty(l.r, l.n, dtype=torch.bfloat16, device=device))
+               for l in layers]
+    in2, out2 = P.pack_io(states2, device)
+    assert in2.numel() == arena_in.numel() and out2.numel() == arena_out.numel()
+    path2 = P.Path(states2, device)
+    sets = [(path, arena_in, arena_out), (path2, in2, out2)]
+
     host_in = torch.empty(arena_in.numel(), dtype=torch.uint8, pin_memory=True)
     host_in.copy_(arena_in)
-    host_out = torch.empty(arena_out.numel(), dtype=torch.uint8, pin_memory=True)
+    host_out = [torch.empty(arena_out.numel(), dtype=torch.uint8, pin_memory=True)
+                for _ in range(2)]
     h2d = host_in.numel()
-    d2h = host_out.numel()
+    d2h = arena_out.numel()
+    s_h2d, s_run, s_d2h = (torch.cuda.Stream(device) for _ in range(3))
+    ev = lambda: torch.cuda.Event()                       # noqa: E731
+    copied_in = [ev(), ev()]
+    computed = [ev(), ev()]
+    copied_out = [ev(), ev()]
+    used = [False, False]
 
-    def one():
-        arena_in.copy_(host_in, non_blocking=True)
-        path.step()
-        host_out.copy_(arena_out, non_blocking=True)
+    def one(k):
+        q = k & 1
+        pth, a_in, a_out = sets[q]
+        with torch.cuda.stream(s_h2d):
+            if used[q]:
+                s_h2d.wait_event(computed[q])             # step k-2 has read its inputs
+            a_in.copy_(host_in, non_blocking=True)
+            copied_in[q].record(s_h2d)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(copied_in[q])
+            if used[q]:
+                s_run.wait_event(copied_out[q])           # step k-2's outputs are home
+            pth.step()
+            computed[q].record(s_run)
+        with torch.cuda.stream(s_d2h):
+            s_d2h.wait_event(computed[q])
+            host_out[q].copy_(a_out, non_blocking=True)
+            copied_out[q].record(s_d2h)
+        used[q] = True
 
-    one()
+    for k in range(2):
+        one(k)
     torch.cuda.synchronize(device)
     if world > 1:
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    a.record(s_h2d)
+    for k in range(steps):
+        one(k)
+    s_d2h.wait_event(copied_out[(steps - 2) & 1])
+    b.record(s_d2h)
     torch.cuda.synchronize(device)
     ms = a.elapsed_time(b) / steps
     if world > 1:
@@ -447,7 +491,8 @@ def e2e(path, arena_in, arena_out, device, stream, steps, world, elements):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     return {"value": elements / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "pipelined": "2 device copies, 3 streams"}
 
 
 if __name__ == "__main__":

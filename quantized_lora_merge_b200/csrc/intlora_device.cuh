@@ -82,6 +82,51 @@ __device__ __forceinline__ float laplace_scaled(uint32_t x, float c_ln2) {
   return laplace_log2(x) * laplace_sign(x, c_ln2);
 }
 
+// Packed pairs of fp32 (sm_100 f32x2 instructions): two lanes' worth of
+// fma/add/mul per instruction, each half rounded exactly like its scalar
+// counterpart (round to nearest even).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a;
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return b;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Two Laplace log2 values (laplace_log2 of words x and y) with the FMA-pipe
+// steps done pairwise; bit-identical to two laplace_log2 calls.
+__device__ __forceinline__ uint64_t laplace_log2_x2(uint32_t x, uint32_t y) {
+  const uint64_t f = f2_pack(__uint_as_float(__funnelshift_r(x, 0x7Fu, 9)),
+                             __uint_as_float(__funnelshift_r(y, 0x7Fu, 9)));
+  const uint64_t u2 = f2_fma(f2_pack(2.0f, 2.0f), f, f2_pack(-1.99999988079071044921875f,
+                                                           -1.99999988079071044921875f));
+  const uint64_t t = f2_add(u2, f2_pack(-1.0f, -1.0f));
+  return f2_pack(__log2f(1.0f - fabsf(f2_lo(t))), __log2f(1.0f - fabsf(f2_hi(t))));
+}
+
 // Round to nearest, ties to even, for |x| < 2^22, via the 1.5 * 2^23 bias:
 // the fused multiply-add rounds x * inv + bias once, leaving the integer in
 // the low mantissa bits.

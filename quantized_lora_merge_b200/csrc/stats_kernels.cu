@@ -37,38 +37,55 @@ __device__ __forceinline__ void block_sum4(double v[4], double* red /* [4][32] *
 }
 
 // Sums of one group of 4 consecutive elements (one Philox block). fp32 partial
-// sums of a few groups are flushed into the fp64 accumulators.
+// sums of a few groups are flushed into the fp64 accumulators. Each sum is a
+// pair of fp32 lanes (f32x2 instructions): words 0 and 2 feed the low half,
+// words 1 and 3 the high half.
 struct GroupSums {
-  float w1 = 0.f, w2 = 0.f, r1 = 0.f, r2 = 0.f;
+  uint64_t w1 = 0, w2 = 0, r1 = 0, r2 = 0;
 };
 
 template <bool HAS_W>
 __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64_t group, float K,
                                           int valid, uint32_t k0, uint32_t k1) {
   const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
-  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-  float x[4] = {0.f, 0.f, 0.f, 0.f};
+  uint64_t r01, r23;
+  if (valid == 4) {
+    const uint64_t l01 = laplace_log2_x2(w.x, w.y), l23 = laplace_log2_x2(w.z, w.w);
+    r01 = f2_mul(l01, f2_pack(laplace_sign(w.x, kLn2f), laplace_sign(w.y, kLn2f)));
+    r23 = f2_mul(l23, f2_pack(laplace_sign(w.z, kLn2f), laplace_sign(w.w, kLn2f)));
+  } else {
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    float rv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) rv[c] = c < valid ? laplace_scaled(words[c], kLn2f) : 0.0f;
+    r01 = f2_pack(rv[0], rv[1]);
+    r23 = f2_pack(rv[2], rv[3]);
+  }
+  g.r1 = f2_add(f2_add(g.r1, r01), r23);
+  g.r2 = f2_fma(r23, r23, f2_fma(r01, r01, g.r2));
   if (HAS_W) {
     const int64_t e = group << 2;
+    uint64_t x01, x23;                   // W - K, elements past the tail left at 0
     if (valid == 4) {
       const float4 v = __ldg(reinterpret_cast<const float4*>(J.W + e));
-      x[0] = v.x - K; x[1] = v.y - K; x[2] = v.z - K; x[3] = v.w - K;
+      const uint64_t nk = f2_pack(-K, -K);
+      x01 = f2_add(f2_pack(v.x, v.y), nk);
+      x23 = f2_add(f2_pack(v.z, v.w), nk);
     } else {
+      float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         if (c < valid) x[c] = __ldg(J.W + e + c) - K;
+      x01 = f2_pack(x[0], x[1]);
+      x23 = f2_pack(x[2], x[3]);
     }
+    g.w1 = f2_add(f2_add(g.w1, x01), x23);
+    g.w2 = f2_fma(x23, x23, f2_fma(x01, x01, g.w2));
   }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const float rv = c < valid ? laplace_scaled(words[c], kLn2f) : 0.0f;
-    g.r1 += rv;
-    g.r2 = fmaf(rv, rv, g.r2);
-    if (HAS_W) {
-      g.w1 += x[c];
-      g.w2 = fmaf(x[c], x[c], g.w2);
-    }
-  }
+}
+
+__device__ __forceinline__ double f2_sum(uint64_t v) {
+  return static_cast<double>(f2_lo(v)) + static_cast<double>(f2_hi(v));
 }
 
 template <bool HAS_W>
@@ -83,19 +100,19 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
     GroupSums s;
 #pragma unroll 2
     for (int u = 0; u < kFlush && g < full; ++u, g += stride) add_group<HAS_W>(s, J, g, K, 4, k0, k1);
-    acc[0] += static_cast<double>(s.w1);
-    acc[1] += static_cast<double>(s.w2);
-    acc[2] += static_cast<double>(s.r1);
-    acc[3] += static_cast<double>(s.r2);
+    acc[0] += f2_sum(s.w1);
+    acc[1] += f2_sum(s.w2);
+    acc[2] += f2_sum(s.r1);
+    acc[3] += f2_sum(s.r2);
   }
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
     add_group<HAS_W>(s, J, full, K, tail, k0, k1);
-    acc[0] += static_cast<double>(s.w1);
-    acc[1] += static_cast<double>(s.w2);
-    acc[2] += static_cast<double>(s.r1);
-    acc[3] += static_cast<double>(s.r2);
+    acc[0] += f2_sum(s.w1);
+    acc[1] += f2_sum(s.w2);
+    acc[2] += f2_sum(s.r1);
+    acc[3] += f2_sum(s.r2);
   }
 }
 

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
     float sv[kTeamRows];
     int32_t zv[kTeamRows];
     constexpr int AREG = (RANK > 0 && RANK <= 8) ? RANK : 1;
-    float areg[kTeamRows][AREG];
+    uint64_t areg[kTeamRows][AREG];          // (a, a) pairs for the f32x2 FMAs
 #pragma unroll
     for (int ml = 0; ml < kTeamRows; ++ml) {
       sv[ml] = 0.0f;
@@ -132,7 +132,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         zv[ml] = clamp_i(__ldg(L.z + irow[ml]), 0, (1 << WBITS) - 1);
         if (RANK > 0 && RANK <= 8) {
 #pragma unroll
-          for (int kk = 0; kk < AREG; ++kk) areg[ml][kk] = __ldg(L.A + irow[ml] * RANK + kk);
+          for (int kk = 0; kk < AREG; ++kk) {
+            const float a = __ldg(L.A + irow[ml] * RANK + kk);
+            areg[ml][kk] = f2_pack(a, a);
+          }
         }
       }
     }
@@ -168,18 +171,18 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       const int q = lt + k * LT;
       if (q >= quads) break;
       const int64_t j = 4 * static_cast<int64_t>(q);
-      float acc[kTeamRows][4];
+      uint64_t acc[kTeamRows][2];            // columns (0, 1) and (2, 3) as f32x2 pairs
       uint32_t cw[kTeamRows];
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml) {
         cw[ml] = 0u;
         if (VARIANT == kGen) {
           const float4 w4 = __ldg(reinterpret_cast<const float4*>(src + irow[ml] * ld_src) + q);
-          acc[ml][0] = w4.x; acc[ml][1] = w4.y; acc[ml][2] = w4.z; acc[ml][3] = w4.w;
+          acc[ml][0] = f2_pack(w4.x, w4.y);
+          acc[ml][1] = f2_pack(w4.z, w4.w);
         } else {
           cw[ml] = load_quad_codes<WBITS>(src + irow[ml] * ld_src, j);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[ml][c] = 0.0f;
+          acc[ml][0] = acc[ml][1] = 0ull;
         }
       }
       if (VARIANT != kGen) {
@@ -187,25 +190,24 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
 #pragma unroll
           for (int kk = 0; kk < AREG; ++kk) {
             const float4 b4 = __ldg(reinterpret_cast<const float4*>(L.B + kk * n) + q);
+            const uint64_t b01 = f2_pack(b4.x, b4.y), b23 = f2_pack(b4.z, b4.w);
 #pragma unroll
             for (int ml = 0; ml < kTeamRows; ++ml) {
-              acc[ml][0] = fmaf(areg[ml][kk], b4.x, acc[ml][0]);
-              acc[ml][1] = fmaf(areg[ml][kk], b4.y, acc[ml][1]);
-              acc[ml][2] = fmaf(areg[ml][kk], b4.z, acc[ml][2]);
-              acc[ml][3] = fmaf(areg[ml][kk], b4.w, acc[ml][3]);
+              acc[ml][0] = f2_fma(areg[ml][kk], b01, acc[ml][0]);
+              acc[ml][1] = f2_fma(areg[ml][kk], b23, acc[ml][1]);
             }
           }
         } else {
 #pragma unroll 4
           for (int kk = 0; kk < r; ++kk) {
             const float4 b4 = __ldg(reinterpret_cast<const float4*>(L.B + kk * n) + q);
+            const uint64_t b01 = f2_pack(b4.x, b4.y), b23 = f2_pack(b4.z, b4.w);
 #pragma unroll
             for (int ml = 0; ml < kTeamRows; ++ml) {
               const float a = __ldg(L.A + irow[ml] * r + kk);
-              acc[ml][0] = fmaf(a, b4.x, acc[ml][0]);
-              acc[ml][1] = fmaf(a, b4.y, acc[ml][1]);
-              acc[ml][2] = fmaf(a, b4.z, acc[ml][2]);
-              acc[ml][3] = fmaf(a, b4.w, acc[ml][3]);
+              const uint64_t a2 = f2_pack(a, a);
+              acc[ml][0] = f2_fma(a2, b01, acc[ml][0]);
+              acc[ml][1] = f2_fma(a2, b23, acc[ml][1]);
             }
           }
         }
@@ -216,15 +218,28 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
         float v[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float lg = laplace_log2(words[c]);
-          const float cs = laplace_sign(words[c], c_ln2);
+        for (int h = 0; h < 2; ++h) {
+          // columns 2h and 2h + 1 as one f32x2 pair
+          const uint32_t wa = words[2 * h], wb = words[2 * h + 1];
+          const uint64_t lg = laplace_log2_x2(wa, wb);
+          uint64_t vp;
           if (VARIANT == kGen) {
-            v[c] = fmaf(-lg, cs, acc[ml][c]);                     // W - R*
+            // W - R*: the sign factor negated (bit 31 of the word flipped)
+            const uint64_t ncs = f2_pack(laplace_sign(wa ^ 0x80000000u, c_ln2),
+                                         laplace_sign(wb ^ 0x80000000u, c_ln2));
+            vp = f2_fma(lg, ncs, acc[ml][h]);
           } else {
-            const int32_t dcode = nib<WBITS>(cw[ml], c) - zv[ml];
-            v[c] = fmaf(fmaf(lg, cs, acc[ml][c]), rcp_tab[dcode + 255], sv[ml]);
+            const uint64_t cs = f2_pack(laplace_sign(wa, c_ln2), laplace_sign(wb, c_ln2));
+            const int32_t d0 = nib<WBITS>(cw[ml], 2 * h) - zv[ml];
+            const int32_t d1 = nib<WBITS>(cw[ml], 2 * h + 1) - zv[ml];
+            vp = f2_fma(f2_fma(lg, cs, acc[ml][h]), f2_pack(rcp_tab[d0 + 255], rcp_tab[d1 + 255]),
+                        f2_pack(sv[ml], sv[ml]));
           }
+          v[2 * h] = f2_lo(vp);
+          v[2 * h + 1] = f2_hi(vp);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
           if (VARIANT == kShift) {
             hi[ml] = fmaxf(hi[ml], fabsf(v[c]));
           } else {

@@ -91,14 +91,10 @@ __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
   return r;
 }
 __device__ __forceinline__ float f2_lo(uint64_t v) {
-  float a, b;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-  return a;
+  return __uint_as_float(static_cast<uint32_t>(v));
 }
 __device__ __forceinline__ float f2_hi(uint64_t v) {
-  float a, b;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-  return b;
+  return __uint_as_float(static_cast<uint32_t>(v >> 32));
 }
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;

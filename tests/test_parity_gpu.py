@@ -223,6 +223,41 @@ def test_ste_batched_mixed_ranks_both_kernels(monkeypatch):
             assert rel_fro(job.dB.cpu().numpy(), oB) < STE_RTOL, kernel
 
 
+def test_batches_beyond_one_launch_table():
+    """130 layers in one batched call of every stage: the library splits the
+    call into chunks of 128 descriptors (and the tensor-core STE into launches
+    of 64); every layer still matches its single-layer call and the oracle."""
+    specs = [spec_for(8 + 4 * (k % 3), 64 + 16 * (k % 5), 4, 4, "mul", 4, sid=200 + k)
+             for k in range(130)]
+    Ws = [wl.host_W(s) for s in specs]
+    g_b = gpu_gen_aux(specs, Ws, batched=True)
+    for k in (0, 64, 127, 128, 129):
+        o = oracle.gen_aux(Ws[k], specs[k].seed, specs[k].stream_id, specs[k].alpha, 4)
+        assert_scale("sigma_r", g_b[k]["sigma_r"], o["sigma_r"])
+        assert_affine("W_round", g_b[k]["codes"], g_b[k]["z"], o["codes"], o["z"], o["pre"],
+                      o["zpre"], 15)
+    inps = [_oracle_prepared(s) for s in specs]
+    a = gpu_merge(specs, inps, batched=True)
+    for k in (0, 127, 128, 129):
+        b = gpu_merge([specs[k]], [inps[k]], batched=False)[0]
+        assert np.array_equal(a[k]["out"], b["out"]) and np.array_equal(a[k]["zbar"], b["zbar"])
+    jobs, host = [], []
+    for spec in specs:
+        Gb, Ab, Bb = (wl.host_G_bits(spec), wl.to_bf16_bits(wl.host_A(spec)),
+                      wl.to_bf16_bits(wl.host_B(spec)))
+        t = [torch.from_numpy(x.view(np.int16)).to(dev()).view(torch.bfloat16) for x in (Gb, Ab, Bb)]
+        jobs.append(B.SteJob(t[0], t[1], t[2], torch.full((spec.d, spec.r), np.nan, device=dev()),
+                             torch.full((spec.r, spec.n), np.nan, device=dev())))
+        host.append((Gb, Ab, Bb))
+    B.intlora_ste_backward_batched(jobs)
+    torch.cuda.synchronize()
+    for k in (0, 63, 64, 127, 128, 129):
+        G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in host[k])
+        oA, oB = oracle.ste_backward(G, A, Bm)
+        assert rel_fro(jobs[k].dA.cpu().numpy(), oA) < STE_RTOL
+        assert rel_fro(jobs[k].dB.cpu().numpy(), oB) < STE_RTOL
+
+
 def test_no_device_wait_gave_up():
     """Every bounded wait of the tensor-core kernels finished in time."""
     assert B.intlora_device_timeouts() == 0

@@ -163,7 +163,8 @@ bool team_path_enabled() {
 bool team_eligible(int variant, const TileLayer& l) {
   if (l.n % 4 != 0 || l.n > kTeamMaxCols) return false;
   if (l.d > (int64_t{1} << 24)) return false;      // keeps tile indices of a batch in int32
-  if (variant != kGen && !aligned16(l.B)) return false;
+  if (variant != kGen && l.r > 0 && !aligned16(l.B)) return false;
+  if (l.T != nullptr && !aligned16(l.T)) return false;
   return true;
 }
 
@@ -235,6 +236,7 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
     t.zero_out = s.zero_out;
     t.code_out = s.code_out;
     t.r_star_out = s.r_star_out;
+    t.T = s.T;
     t.d = s.d;
     t.n = s.n;
     t.r = s.r;
@@ -288,6 +290,20 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
 
 intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bits, int w_bits,
                                  int out_bytes, uint64_t seed, cudaStream_t stream) {
+  // layers whose A B was precomputed run in launches of their own (the
+  // kernels' rank-free specialisation)
+  bool any_t = false, all_t = true;
+  for (auto& l : L) {
+    any_t = any_t || l.T != nullptr;
+    all_t = all_t && l.T != nullptr;
+  }
+  if (any_t && !all_t) {
+    std::vector<TileLayer> with_t, without;
+    for (auto& l : L) (l.T != nullptr ? with_t : without).push_back(l);
+    const intlora_status s = launch_tile_batch(variant, with_t, bits, w_bits, out_bytes, seed, stream);
+    if (s != INTLORA_OK) return s;
+    return launch_tile_batch(variant, without, bits, w_bits, out_bytes, seed, stream);
+  }
   // layers the team kernel takes go there (one launch); the rest stay here
   if (team_path_enabled()) {
     std::vector<TileLayer> team, rest;
@@ -299,6 +315,7 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
         for (auto& l : team)
           if (l.r != rank_t) rank_t = 0;
         if (rank_t != 4 && rank_t != 8 && rank_t != 16) rank_t = 0;
+        if (all_t) rank_t = -1;
       }
       const intlora_status s = launch_team_batch(variant, team, rank_t, bits, w_bits, out_bytes, seed, stream);
       if (s != INTLORA_OK) return s;
@@ -312,6 +329,7 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
     for (auto& l : L)
       if (l.r != rank_ct) rank_ct = 0;
     if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16) rank_ct = 0;
+    if (all_t) rank_ct = -1;
   }
   bool aligned = true;
   for (auto& l : L) aligned = aligned && (l.n % 4 == 0);
@@ -513,12 +531,41 @@ intlora_status check_out(const intlora_merge_out* o, bool mul, int idx) {
   return INTLORA_OK;
 }
 
+// INTLORA_T_KERNEL=cuda keeps T = A B on the CUDA cores inside the row
+// kernels; unset or "auto": ranks in [kTensorTMinRank, kTensorTMaxRank] get T
+// from the tensor-core pass.
+bool tensor_t_enabled() {
+  const char* v = std::getenv("INTLORA_T_KERNEL");
+  return v == nullptr || std::strcmp(v, "cuda") != 0;
+}
+bool uses_tensor_t(const intlora_layer& l) {
+  return tensor_t_enabled() && t_gemm_supported(l.d, l.n, l.r);
+}
+// A call whose workspace does not cover the tensor-core T buffers still runs,
+// with A B on the CUDA cores (set per call by merge_batched).
+thread_local bool g_t_allowed = true;
+
+// Workspace of one layer of a merge: the sigma_R scratch when sigma_r is not
+// passed, then (tensor-core T) T, A_hi, A_lo, B^T_hi, B^T_lo.
+struct MergeWs {
+  size_t sigma, T, a, bt, total;
+};
+MergeWs merge_ws_layout(const intlora_layer& l) {
+  MergeWs w{0, 0, 0, 0, 0};
+  if (l.sigma_r == nullptr) w.sigma = 256 + stats_partial_bytes(l.d * l.n);
+  if (g_t_allowed && uses_tensor_t(l)) {
+    const int64_t kp = t_gemm_kp(l.r);
+    w.T = round256(static_cast<size_t>(l.d * l.n) * 4);
+    w.a = round256(static_cast<size_t>(l.d * kp) * 4);
+    w.bt = round256(static_cast<size_t>(l.n * kp) * 4);
+  }
+  w.total = w.sigma + w.T + 2 * w.a + 2 * w.bt;
+  return w;
+}
+
 size_t merge_ws_bytes(const intlora_layer* layers, int32_t count) {
   size_t total = 0;
-  for (int32_t k = 0; k < count; ++k) {
-    if (layers[k].sigma_r != nullptr) continue;
-    total += 256 + stats_partial_bytes(layers[k].d * layers[k].n);
-  }
+  for (int32_t k = 0; k < count; ++k) total += merge_ws_layout(layers[k]).total;
   return total;
 }
 
@@ -534,11 +581,35 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
                            int32_t count, int32_t bits, char* ws, cudaStream_t st) {
   std::vector<const double*> sig_r(count);
   std::vector<size_t> offset(count);
+  std::vector<const float*> t_of(count, nullptr);
+  std::vector<TGemmJob> tjobs;
   size_t off = 0;
   for (int32_t k = 0; k < count; ++k) {
     sig_r[k] = layers[k].sigma_r;
     offset[k] = off;
-    if (layers[k].sigma_r == nullptr) off += 256 + stats_partial_bytes(layers[k].d * layers[k].n);
+    const MergeWs w = merge_ws_layout(layers[k]);
+    if (w.T > 0) {
+      char* p = ws + off + w.sigma;
+      TGemmJob j;
+      j.A = layers[k].A;
+      j.B = layers[k].B;
+      j.d = layers[k].d;
+      j.n = layers[k].n;
+      j.r = layers[k].r;
+      j.kp = static_cast<int32_t>(t_gemm_kp(layers[k].r));
+      j.T = reinterpret_cast<float*>(p);
+      j.a_hi = reinterpret_cast<float*>(p + w.T);
+      j.a_lo = reinterpret_cast<float*>(p + w.T + w.a);
+      j.b_hi = reinterpret_cast<float*>(p + w.T + 2 * w.a);
+      j.b_lo = reinterpret_cast<float*>(p + w.T + 2 * w.a + w.bt);
+      t_of[k] = j.T;
+      tjobs.push_back(j);
+    }
+    off += w.total;
+  }
+  if (!tjobs.empty()) {
+    cudaError_t e = launch_t_gemm(tjobs.data(), static_cast<int>(tjobs.size()), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core A B launch");
   }
   for (const auto& grp : group_by_seed(layers, count)) {
     // sigma_R on the device for layers that did not pass it in
@@ -594,6 +665,10 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
         l.d = y.d;
         l.n = y.n;
         l.r = y.r;
+        if (t_of[k] != nullptr) {          // the row kernels read T, no A B on the CUDA cores
+          l.T = t_of[k];
+          l.r = 0;
+        }
         L.push_back(l);
       }
       if (L.empty()) continue;
@@ -620,9 +695,17 @@ intlora_status merge_batched(int variant, const intlora_layer* layers, const int
     s = check_out(&outs[k], variant == kMul, k);
     if (s != INTLORA_OK) return s;
   }
-  const size_t need = merge_ws_bytes(layers, count);
-  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws)))
-    return fail(INTLORA_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+  g_t_allowed = true;
+  size_t need = merge_ws_bytes(layers, count);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) {
+    // without room for the tensor-core T buffers, form A B on the CUDA cores
+    g_t_allowed = false;
+    need = merge_ws_bytes(layers, count);
+    if (need > 0 && (ws == nullptr || ws_bytes < need || !aligned16(ws))) {
+      g_t_allowed = true;
+      return fail(INTLORA_ERR_WORKSPACE, "workspace of %zu bytes (16-byte aligned) required", need);
+    }
+  }
   char* w = static_cast<char*>(ws);
   for (int32_t k0 = 0; k0 < count; k0 += kMaxBatch) {
     const int32_t c = std::min<int32_t>(kMaxBatch, count - k0);
@@ -631,6 +714,7 @@ intlora_status merge_batched(int variant, const intlora_layer* layers, const int
     if (s != INTLORA_OK) return s;
     w += merge_ws_bytes(layers + k0, c);
   }
+  g_t_allowed = true;
   return INTLORA_OK;
 }
 
@@ -780,7 +864,7 @@ const char* intlora_last_error(void) { return g_last_error; }
 
 int intlora_version(void) { return 100; }
 
-uint32_t intlora_device_timeouts(void) { return intlora::ste_tc_timeouts(); }
+uint32_t intlora_device_timeouts(void) { return intlora::ste_tc_timeouts() + intlora::t_gemm_timeouts(); }
 
 int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits) {
   if ((variant != 0 && variant != 1) || (w_bits != 4 && w_bits != 8)) return 0;

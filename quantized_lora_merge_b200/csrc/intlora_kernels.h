@@ -61,6 +61,7 @@ struct TileLayer {
   int32_t* zero_out;         // kGen: z; kMul: z_bar
   uint8_t* code_out;         // kMul: U_round; kShift: shift (optional)
   float* r_star_out;         // kGen only, optional
+  const float* T;            // merges: precomputed A B (d x n) or nullptr (then r = 0)
   // geometry
   int64_t d, n;
   int32_t r;
@@ -126,6 +127,7 @@ struct TeamLayer {
   int32_t* zero_out;
   uint8_t* code_out;
   float* r_star_out;
+  const float* T;            // merges: precomputed A B (d x n) or nullptr
   int64_t d, n;
   int32_t r;
   int32_t team_warps;        // TW: 1, 2, 4 or 8
@@ -185,6 +187,27 @@ constexpr int kSteTcMaxRank = 128;
 bool ste_tc_supported(const SteJob& j);
 cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s);
 unsigned int ste_tc_timeouts();
+
+// T = A B on the tensor cores (tf32 three-term split) for ranks in
+// [kTensorTMinRank, kTensorTMaxRank]: the row kernels then read T instead of
+// forming it on the CUDA cores.
+constexpr int kTensorTMinRank = 32;
+constexpr int kTensorTMaxRank = 64;
+struct TGemmJob {
+  const float* A;            // d x r
+  const float* B;            // r x n
+  int64_t d, n;
+  int32_t r, kp;             // kp = t_gemm_kp(r)
+  float* T;                  // d x n (workspace)
+  float* a_hi;               // d x kp (workspace), 16-byte aligned like the others
+  float* a_lo;
+  float* b_hi;               // n x kp: B transposed
+  float* b_lo;
+};
+int64_t t_gemm_kp(int32_t r);
+bool t_gemm_supported(int64_t d, int64_t n, int32_t r);
+cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s);
+unsigned int t_gemm_timeouts();
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 
 // Sets the calling thread's intlora_last_error() message.

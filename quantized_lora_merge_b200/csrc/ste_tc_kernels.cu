@@ -24,10 +24,13 @@
 #include <mutex>
 
 #include "intlora_kernels.h"
+#include "tcgen05_util.cuh"
 
 namespace intlora {
 
 namespace {
+
+using namespace tc;
 
 constexpr int kTcThreads = 256;
 constexpr int kTileRows = 128;                 // rows of G per unit (GEMM1 M, GEMM2 K)
@@ -36,7 +39,6 @@ constexpr uint32_t kGBytes = kTileRows * kTileCols * 2;
 constexpr uint32_t kBoxBytes = kTileRows * 64 * 2;    // one 64-column box of the G tile
 constexpr int kMaxTcJobs = 64;
 constexpr int kMaxD2 = 8;                      // D2 accumulators (tile epilogues in flight)
-constexpr uint64_t kWaitNs = 2000000000ull;  // a wait gives up after 2 s
 
 struct alignas(64) SteTcJob {
   CUtensorMap g_map;          // G: dims {n, d}, box {64, 128}, 128B swizzle
@@ -66,108 +68,11 @@ struct SteTcBatch {
 
 __device__ unsigned int g_tc_timeouts;
 
-// ---- PTX wrappers ----------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait: false once kWaitNs have passed (the wait is counted in a
-// device word and the CTA is told to stop) or when another role of the CTA
-// has given up already.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitNs) break;
-    }
-  }
-  atomicAdd(&g_tc_timeouts, 1u);
-  *abort_flag = 1;
-  return false;
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void red_add(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+// Bounded mbarrier wait counted in this kernel family's timeout word.
+__device__ __forceinline__ bool mbar_wait_c(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait(bar, parity, abort_flag, &g_tc_timeouts);
 }
 
-// Shared-memory matrix descriptor (tcgen05): start address, leading and
-// stride byte offsets (16-byte units), descriptor version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= uint64_t{1} << 46;                 // version
-  d |= uint64_t{2} << 61;                 // SWIZZLE_128B
-  return d;
-}
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M = 128, N = rp.
 __host__ __device__ constexpr uint32_t instr_desc(int rp, bool a_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major ? (1u << 15) : 0u) |
@@ -265,7 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
         const Unit x = decode_unit(b, u);
         const SteTcJob& J = b.job[x.job];
         for (int ct = x.ct0; ct < x.ct1; ++ct) {
-          if (!mbar_wait(&empty[stage], ph ^ 1u, &abort_flag)) break;
+          if (!mbar_wait_c(&empty[stage], ph ^ 1u, &abort_flag)) break;
           mbar_arrive_tx(&full[stage], kGBytes + b_bytes);
           uint8_t* g = sG + stage * kGBytes;
           uint8_t* bt = sB + stage * b_bytes;
@@ -291,14 +196,14 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
         const Unit x = decode_unit(b, u);
         const int ab = ucount & 1;
         const uint32_t aph = static_cast<uint32_t>(ucount >> 1) & 1u;
-        if (!mbar_wait(&a_full[ab], aph, &abort_flag)) break;
-        if (!mbar_wait(&d1_empty[ab], aph ^ 1u, &abort_flag)) break;
+        if (!mbar_wait_c(&a_full[ab], aph, &abort_flag)) break;
+        if (!mbar_wait_c(&d1_empty[ab], aph ^ 1u, &abort_flag)) break;
         tc_fence_after();
         const uint32_t d1 = tmem + static_cast<uint32_t>(ab * RP);
         const uint64_t a0 = smem_desc(smem_u32(sA + ab * b_bytes), 16, 1024);
         bool ok = true;
         for (int ct = x.ct0; ct < x.ct1; ++ct) {
-          if (!mbar_wait(&full[stage], ph, &abort_flag) || !mbar_wait(&d2_empty[d2], d2ph ^ 1u, &abort_flag)) {
+          if (!mbar_wait_c(&full[stage], ph, &abort_flag) || !mbar_wait_c(&d2_empty[d2], d2ph ^ 1u, &abort_flag)) {
             ok = false;
             break;
           }
@@ -351,7 +256,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
       const SteTcJob& J = b.job[x.job];
       const int ab = ucount & 1;
       const uint32_t aph = static_cast<uint32_t>(ucount >> 1) & 1u;
-      if (!mbar_wait(&a_empty[ab], aph ^ 1u, &abort_flag)) break;
+      if (!mbar_wait_c(&a_empty[ab], aph ^ 1u, &abort_flag)) break;
       uint8_t* dst = sA + ab * b_bytes;
       for (int rr = t; rr < kTileRows; rr += 64) {
         const int64_t i = x.i0 + rr;
@@ -379,7 +284,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
       const int64_t n = J.n;
       bool ok = true;
       for (int ct = x.ct0; ct < x.ct1; ++ct) {
-        if (!mbar_wait(&d2_full[d2], d2ph, &abort_flag)) {
+        if (!mbar_wait_c(&d2_full[d2], d2ph, &abort_flag)) {
           ok = false;
           break;
         }
@@ -403,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
       }
       if (!ok) break;
       const int ab = ucount & 1;
-      if (!mbar_wait(&d1_full[ab], static_cast<uint32_t>(ucount >> 1) & 1u, &abort_flag)) break;
+      if (!mbar_wait_c(&d1_full[ab], static_cast<uint32_t>(ucount >> 1) & 1u, &abort_flag)) break;
       tc_fence_after();
       const int64_t i = x.i0 + e;
       for (int c0 = 0; c0 < RP; c0 += 16) {
@@ -434,31 +339,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
 }
 
 // ---- host side ---------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor map of a row-major rows x cols matrix, box {64, box_rows},
-// 128-byte swizzle, zero fill outside the matrix.
 bool encode_bf16(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tc::encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, rows, cols, 64, box_rows);
 }
 
 size_t tc_smem_bytes(int rp, int stages) {
@@ -471,7 +353,7 @@ size_t tc_smem_bytes(int rp, int stages) {
 bool ste_tc_supported(const SteJob& j) {
   const auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   return j.n % 8 == 0 && j.r >= 1 && j.r <= kSteTcMaxRank && al(j.G) && al(j.B) && j.d <= (int64_t{1} << 31) &&
-         j.n <= (int64_t{1} << 31) && encode_fn() != nullptr;
+         j.n <= (int64_t{1} << 31) && tc::encode_fn() != nullptr;
 }
 
 cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s) {

@@ -113,7 +113,8 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
     const uint8_t* __restrict__ src = static_cast<const uint8_t*>(L.src);
     const int64_t ld_src = L.ld_src;
     const uint32_t sid = L.stream_id;
-    const int r = VARIANT == kGen ? 0 : (RANK > 0 ? RANK : L.r);
+    // RANK > 0: fixed rank; 0: any rank; < 0: A B precomputed (L.T), no rank loop
+    const int r = (VARIANT == kGen || RANK < 0) ? 0 : (RANK > 0 ? RANK : L.r);
 
     // row parameters and (small fixed rank) the A rows of the group
     int64_t irow[kTeamRows];
@@ -182,7 +183,13 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
           acc[ml][1] = f2_pack(w4.z, w4.w);
         } else {
           cw[ml] = load_quad_codes<WBITS>(src + irow[ml] * ld_src, j);
-          acc[ml][0] = acc[ml][1] = 0ull;
+          if (RANK < 0) {                        // A B precomputed on the tensor cores
+            const float4 t4 = __ldg(reinterpret_cast<const float4*>(L.T + irow[ml] * n) + q);
+            acc[ml][0] = f2_pack(t4.x, t4.y);
+            acc[ml][1] = f2_pack(t4.z, t4.w);
+          } else {
+            acc[ml][0] = acc[ml][1] = 0ull;
+          }
         }
       }
       if (VARIANT != kGen) {
@@ -435,6 +442,7 @@ void team_by_rank(TeamQuery& q, int rank_ct) {
     case 4: team_run<VARIANT, WBITS, 4, OUTB>(q); break;
     case 8: team_run<VARIANT, WBITS, 8, OUTB>(q); break;
     case 16: team_run<VARIANT, WBITS, 16, OUTB>(q); break;
+    case -1: team_run<VARIANT, WBITS, -1, OUTB>(q); break;
     default: team_run<VARIANT, WBITS, 0, OUTB>(q); break;
   }
 }

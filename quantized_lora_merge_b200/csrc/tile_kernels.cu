@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
     const int rows = static_cast<int>(min64(L.m, L.d - row0));
     const int64_t col0 = static_cast<int64_t>(crank) * L.n_c;
     const int ncols = static_cast<int>(max64(0, min64(L.n_c, L.n - col0)));
-    const int r = (VARIANT == kGen) ? 1 : (RANK > 0 ? RANK : L.r);
+    // RANK > 0: fixed rank; 0: any rank; < 0: A B precomputed (L.T)
+    const int r = (VARIANT == kGen) ? 1 : (RANK < 0 ? 0 : (RANK > 0 ? RANK : L.r));
     const int m = L.m;
     const int n_c = L.n_c;
     // per-layer values used inside the item loops, read once per tile
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
         row_z[rr] = rr < rows ? clamp_i(__ldg(L.z + row0 + rr), 0, (1 << p.w_bits) - 1) : 0;
       }
       // A rows of the tile, read along the rank (coalesced), stored k-major
-      for (int idx = tid; idx < r * m; idx += kTileThreads) {
+      for (int idx = tid; RANK >= 0 && idx < r * m; idx += kTileThreads) {
         const int rr = idx / r, k = idx - rr * r;
         At[k * m + rr] = rr < rows ? __ldg(L.A + (row0 + rr) * static_cast<int64_t>(L.r) + k) : 0.0f;
       }
@@ -303,8 +304,21 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
             cw[ml] = load_codes<WBITS, ALIGNED>(src + i * ld_src, j, vcols);
           }
         }
-        // T = A B on the item (CUDA-core FMA)
-        if (VARIANT != kGen) {
+        // T = A B on the item: precomputed on the tensor cores, or CUDA-core FMA
+        if (VARIANT != kGen && RANK < 0) {
+#pragma unroll
+          for (int ml = 0; ml < RPI; ++ml) {
+            const float* trow = L.T + (row0 + min(w.g * RPI + ml, rows - 1)) * n;
+            if (ALIGNED) {
+              const float4 t4 = __ldg(reinterpret_cast<const float4*>(trow + j));
+              acc[ml][0] = t4.x; acc[ml][1] = t4.y; acc[ml][2] = t4.z; acc[ml][3] = t4.w;
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                if (c < vcols) acc[ml][c] = __ldg(trow + j + c);
+            }
+          }
+        } else if (VARIANT != kGen) {
           if (streamed) {
 #pragma unroll
             for (int ml = 0; ml < RPI; ++ml) {
@@ -571,6 +585,7 @@ void by_rank(TileQuery& q, int rank_ct) {
     case 4: run_query<VARIANT, WBITS, 4, OUTB, ALIGNED>(q); break;
     case 8: run_query<VARIANT, WBITS, 8, OUTB, ALIGNED>(q); break;
     case 16: run_query<VARIANT, WBITS, 16, OUTB, ALIGNED>(q); break;
+    case -1: run_query<VARIANT, WBITS, -1, OUTB, ALIGNED>(q); break;
     default: run_query<VARIANT, WBITS, 0, OUTB, ALIGNED>(q); break;
   }
 }

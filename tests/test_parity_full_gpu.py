@@ -43,7 +43,7 @@ def _synthetic_prepared(spec):
                 sigma_r=1.4142)
 
 
-def _check_prepare(specs, rows_per_layer=6):
+def _check_prepare(specs):
     dev = _dev()
     states = []
     for spec in specs:
@@ -93,10 +93,11 @@ def _run_merge(specs):
     variant, bits = specs[0].variant, specs[0].out_bits
     layers = [st.layer() for st in states]
     outs = [st.merge_out() for st in states]
+    ws = P.workspace(B.intlora_merge_workspace_size(layers), dev)   # tensor-core A B at r >= 32
     if variant == "mul":
-        B.intlora_merge_mul_batched(layers, outs, bits, None)
+        B.intlora_merge_mul_batched(layers, outs, bits, ws)
     else:
-        B.intlora_merge_shift_batched(layers, outs, bits, None)
+        B.intlora_merge_shift_batched(layers, outs, bits, ws)
     torch.cuda.synchronize()
     return states, inps
 

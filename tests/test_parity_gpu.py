@@ -110,6 +110,11 @@ MUL_CASES = [
     (130, 5120, 4, 4, 4),     # FF width 4d at d = 1280
     (1, 8, 1, 4, 4),          # single row, rank 1
     (17, 64, 8, 8, 6),        # 6-bit U quantizer (int16 products)
+    # ranks 32..64: A B from the tensor cores (tf32 three-term split)
+    (100, 1024, 32, 8, 8),
+    (129, 256, 33, 8, 8),     # ragged rank (padded to 64) and row block
+    (33, 8200, 64, 4, 4),     # wider than the team kernels: row-tile kernels read T
+    (7, 100, 48, 4, 4),
 ]
 
 
@@ -136,6 +141,24 @@ def test_merge_shift_parity(d, n, r, w_bits, shift_bits):
     inp = _oracle_prepared(spec)
     got = gpu_merge([spec], [inp])[0]
     _check_shift(spec, inp, got)
+
+
+@pytest.mark.parametrize("variant", ["mul", "shift"])
+def test_merge_tensor_core_t_and_cuda_core_t_agree(monkeypatch, variant):
+    """The same layers with A B from the tensor cores and from the CUDA cores:
+    both meet the oracle, and their codes differ only where a value sits
+    within the tolerance window of a rounding boundary."""
+    specs = [spec_for(d, n, r, 4, variant, 4, sid=300 + k)
+             for k, (d, n, r) in enumerate([(64, 3072, 64), (40, 640, 32), (12, 6400, 64)])]
+    inps = [_oracle_prepared(s) for s in specs]
+    res = {}
+    for kernel in ("auto", "cuda"):
+        monkeypatch.setenv("INTLORA_T_KERNEL", kernel)
+        res[kernel] = gpu_merge(specs, inps, batched=True)
+        for spec, inp, got in zip(specs, inps, res[kernel]):
+            (_check_mul if variant == "mul" else _check_shift)(spec, inp, got)
+    for x, y in zip(res["auto"], res["cuda"]):
+        assert np.mean(x["out"] != y["out"]) < 1e-3
 
 
 def test_merge_reduces_sigma_r_on_device_when_not_given():

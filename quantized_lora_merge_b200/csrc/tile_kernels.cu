@@ -218,8 +218,9 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
         row_z[rr] = rr < rows ? clamp_i(__ldg(L.z + row0 + rr), 0, (1 << p.w_bits) - 1) : 0;
       }
       // A rows of the tile, read along the rank (coalesced), stored k-major
-      for (int idx = tid; RANK >= 0 && idx < r * m; idx += kTileThreads) {
-        const int rr = idx / r, k = idx - rr * r;
+      const int rdiv = r > 0 ? r : 1;
+      for (int idx = tid; idx < r * m; idx += kTileThreads) {
+        const int rr = idx / rdiv, k = idx - rr * r;
         At[k * m + rr] = rr < rows ? __ldg(L.A + (row0 + rr) * static_cast<int64_t>(L.r) + k) : 0.0f;
       }
     }

@@ -762,11 +762,25 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
       ok = ste_tc_supported(s);
     }
     if (ok) {
-      b.count = count;
-      cudaError_t e = launch_ste_zero(b, st);
-      if (e != cudaSuccess) return cuda_fail(e, "STE zero launch");
-      e = launch_ste_tc(b.job, count, st);
-      if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE kernel launch");
+      // ranks >= 64: two passes, each product reduced inside a CTA; the rest
+      // one pass with reductions into zeroed outputs
+      SteBatch one;
+      std::memset(&one, 0, sizeof one);
+      std::vector<SteJob> wide;
+      for (int32_t k = 0; k < count; ++k) {
+        if (ste_wide_supported(b.job[k])) wide.push_back(b.job[k]);
+        else one.job[one.count++] = b.job[k];
+      }
+      if (!wide.empty()) {
+        cudaError_t e = launch_ste_wide(wide.data(), static_cast<int>(wide.size()), st);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE (two-pass) launch");
+      }
+      if (one.count > 0) {
+        cudaError_t e = launch_ste_zero(one, st);
+        if (e != cudaSuccess) return cuda_fail(e, "STE zero launch");
+        e = launch_ste_tc(one.job, one.count, st);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE kernel launch");
+      }
       return INTLORA_OK;
     }
   }
@@ -864,7 +878,9 @@ const char* intlora_last_error(void) { return g_last_error; }
 
 int intlora_version(void) { return 100; }
 
-uint32_t intlora_device_timeouts(void) { return intlora::ste_tc_timeouts() + intlora::t_gemm_timeouts(); }
+uint32_t intlora_device_timeouts(void) {
+  return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts();
+}
 
 int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits) {
   if ((variant != 0 && variant != 1) || (w_bits != 4 && w_bits != 8)) return 0;

@@ -187,6 +187,12 @@ constexpr int kSteTcMaxRank = 128;
 bool ste_tc_supported(const SteJob& j);
 cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s);
 unsigned int ste_tc_timeouts();
+// Ranks 64..128 (r % 8 == 0): two tensor-core passes over G, each product
+// reduced inside one CTA (no atomics, no zeroing).
+constexpr int kSteWideMinRank = 64;
+bool ste_wide_supported(const SteJob& j);
+cudaError_t launch_ste_wide(const SteJob* jobs, int count, cudaStream_t s);
+unsigned int ste_wide_timeouts();
 
 // T = A B on the tensor cores (tf32 three-term split) for ranks in
 // [kTensorTMinRank, kTensorTMaxRank]: the row kernels then read T instead of

@@ -207,7 +207,9 @@ def test_ste_parity(d, n, r):
 
 
 @pytest.mark.parametrize("d,n,r", [(100, 304, 128), (257, 1032, 33), (129, 136, 1), (1, 8, 4),
-                                   (4096, 1024, 64), (130, 4104, 8)])
+                                   (4096, 1024, 64), (130, 4104, 8),
+                                   # ranks >= 64: two passes, each output written once
+                                   (257, 1032, 96), (130, 4104, 64), (3, 8, 128)])
 def test_ste_tensor_core_parity(d, n, r):
     """Shapes the tensor-core pass takes (n % 8 == 0, r <= 128): ragged row
     blocks and column tiles, padded ranks (1, 8, 33 -> 16, 16, 48)."""
@@ -226,7 +228,8 @@ def test_ste_batched_mixed_ranks_both_kernels(monkeypatch):
     """One batched call over layers of different shapes and ranks, through the
     tensor-core pass and through the CUDA-core kernels: both match the oracle."""
     specs = [spec_for(d, n, r, 8, sid=40 + k) for k, (d, n, r) in
-             enumerate([(320, 320, 4), (200, 768, 8), (64, 1280, 16), (384, 256, 2)])]
+             enumerate([(320, 320, 4), (200, 768, 8), (64, 1280, 16), (384, 256, 2),
+                        (96, 512, 64), (40, 136, 128)])]
     host = [(wl.host_G_bits(s), wl.to_bf16_bits(wl.host_A(s)), wl.to_bf16_bits(wl.host_B(s)))
             for s in specs]
     for kernel in ("auto", "cuda"):

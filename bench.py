@@ -110,16 +110,19 @@ ALU_LANES_PER_SM_CLK = 128       # FP32/INT32 lanes per SM per clock on sm_100
 NUM_SMS = 148
 
 
+# sources the dominant (team) kernel is compiled from
+DOMINANT_SOURCES = ("team_kernels.cu", "intlora_device.cuh", "intlora_kernels.h")
+
+
 def csrc_hash():
-    """Hash of the CUDA sources, so a stored ncu traffic figure is only used
-    while the kernels it was taken on are unchanged."""
+    """Hash of the dominant kernel's CUDA sources, so a stored ncu traffic
+    figure is only used while the kernel it was taken on is unchanged."""
     import hashlib
     h = hashlib.sha256()
     root = Path(__file__).resolve().parent / "quantized_lora_merge_b200" / "csrc"
-    for p in sorted(root.iterdir()):
-        if p.suffix in (".cu", ".cuh", ".h"):
-            h.update(p.name.encode())
-            h.update(p.read_bytes())
+    for name in DOMINANT_SOURCES:
+        h.update(name.encode())
+        h.update((root / name).read_bytes())
     return h.hexdigest()
 
 

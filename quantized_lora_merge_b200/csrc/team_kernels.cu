@@ -39,6 +39,19 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// 4 x the 4-bit code c of a packed word (a byte offset into a 16-entry table).
+__device__ __forceinline__ uint32_t nib4_x4(uint32_t packed, int c) {
+  return c == 0 ? (packed << 2) & 0x3Cu : (packed >> (4 * c - 2)) & 0x3Cu;
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 template <int WBITS>
 __device__ __forceinline__ int32_t nib(uint32_t packed, int c) {
   return WBITS == 8 ? static_cast<int32_t>((packed >> (8 * c)) & 0xFFu)
@@ -71,6 +84,11 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
   // row extrema of every warp: [2][warps][2 kTeamRows] (double buffered)
   uint32_t* slots = Cbuf + (VARIANT == kGen ? 0 : smax * kTeamRows * kTeamThreads);
   float* rcp_tab = reinterpret_cast<float*>(slots + 2 * kTeamWarps * kSlotWords);   // 1/D, D in [-255, 255]
+  // 4-bit merges: each warp's 1/(code - z) for its 4 rows x 16 codes (256-byte
+  // aligned, so a row entry's address is base | code * 4 + row * 64)
+  const uint32_t lut_base =
+      (static_cast<uint32_t>(__cvta_generic_to_shared(rcp_tab + 512)) + 255u) & ~255u;
+  const uint32_t my_lut = lut_base + static_cast<uint32_t>(threadIdx.x >> 5) * 256u;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int qmax = (1 << p.bits) - 1;
@@ -164,6 +182,15 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
     }
 #endif
 
+    if (VARIANT != kGen && WBITS == 4) {
+      __syncwarp();
+      for (int e = lane; e < kTeamRows * 16; e += 32) {
+        const int32_t zr = pick_row(zv, e >> 4);
+        st_shared_f32(my_lut + 4u * static_cast<uint32_t>(e), rcp_tab[(e & 15) - zr + 255]);
+      }
+      __syncwarp();
+    }
+
     // ---- phase A
     float hi[kTeamRows], lo[kTeamRows];
 #pragma unroll
@@ -237,10 +264,17 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
             vp = f2_fma(lg, ncs, acc[ml][h]);
           } else {
             const uint64_t cs = f2_pack(laplace_sign(wa, c_ln2), laplace_sign(wb, c_ln2));
-            const int32_t d0 = nib<WBITS>(cw[ml], 2 * h) - zv[ml];
-            const int32_t d1 = nib<WBITS>(cw[ml], 2 * h + 1) - zv[ml];
-            vp = f2_fma(f2_fma(lg, cs, acc[ml][h]), f2_pack(rcp_tab[d0 + 255], rcp_tab[d1 + 255]),
-                        f2_pack(sv[ml], sv[ml]));
+            float r0, r1;
+            if (WBITS == 4) {
+              // code c's entry: base | c * 4 (one shift and one 3-input logic op)
+              const uint32_t row_lut = my_lut + static_cast<uint32_t>(ml) * 64u;   // 64-byte aligned
+              r0 = ld_shared_f32(row_lut | nib4_x4(cw[ml], 2 * h));
+              r1 = ld_shared_f32(row_lut | nib4_x4(cw[ml], 2 * h + 1));
+            } else {
+              r0 = rcp_tab[nib<WBITS>(cw[ml], 2 * h) - zv[ml] + 255];
+              r1 = rcp_tab[nib<WBITS>(cw[ml], 2 * h + 1) - zv[ml] + 255];
+            }
+            vp = f2_fma(f2_fma(lg, cs, acc[ml][h]), f2_pack(r0, r1), f2_pack(sv[ml], sv[ml]));
           }
           v[2 * h] = f2_lo(vp);
           v[2 * h + 1] = f2_hi(vp);
@@ -469,7 +503,8 @@ void team_dispatch(TeamQuery& q, int variant, int w_bits, int rank_ct, int out_b
 size_t team_smem_bytes(int variant, int sweeps_max) {
   const size_t per_sweep = static_cast<size_t>(kTeamRows) * kTeamThreads * 16 +
                            (variant == kGen ? 0 : static_cast<size_t>(kTeamRows) * kTeamThreads * 4);
-  return per_sweep * sweeps_max + 2 * kTeamWarps * kSlotWords * 4 + (variant == kGen ? 0 : 512 * 4);
+  return per_sweep * sweeps_max + 2 * kTeamWarps * kSlotWords * 4 +
+         (variant == kGen ? 0 : 512 * 4 + 256 + kTeamWarps * 256);
 }
 
 cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s) {

@@ -45,8 +45,8 @@ struct GroupSums {
 };
 
 template <bool HAS_W>
-__device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64_t group, float K,
-                                          int valid, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, const float* wgroup,
+                                          uint64_t group, float K, int valid, uint32_t k0, uint32_t k1) {
   const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
   uint64_t r01, r23;
   if (valid == 4) {
@@ -64,10 +64,9 @@ __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64
   g.r1 = f2_add(f2_add(g.r1, r01), r23);
   g.r2 = f2_fma(r23, r23, f2_fma(r01, r01, g.r2));
   if (HAS_W) {
-    const int64_t e = group << 2;
     uint64_t x01, x23;                   // W - K, elements past the tail left at 0
     if (valid == 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(J.W + e));
+      const float4 v = __ldg(reinterpret_cast<const float4*>(wgroup));
       const uint64_t nk = f2_pack(-K, -K);
       x01 = f2_add(f2_pack(v.x, v.y), nk);
       x23 = f2_add(f2_pack(v.z, v.w), nk);
@@ -75,7 +74,7 @@ __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, int64
       float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (c < valid) x[c] = __ldg(J.W + e + c) - K;
+        if (c < valid) x[c] = __ldg(wgroup + c) - K;
       x01 = f2_pack(x[0], x[1]);
       x23 = f2_pack(x[2], x[3]);
     }
@@ -95,11 +94,20 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int64_t full = J.numel >> 2;                 // complete groups
   const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
   const float K = HAS_W ? __ldg(J.W) : 0.0f;
-  int64_t g = local * kStatsThreads + threadIdx.x;
-  while (g < full) {
+  const int64_t g0 = local * kStatsThreads + threadIdx.x;
+  // this thread's groups g0, g0 + stride, ...: a 32-bit trip count, the group
+  // index (Philox counter) and the W pointer advance by the stride
+  const int32_t count = g0 < full ? static_cast<int32_t>((full - 1 - g0) / stride + 1) : 0;
+  uint64_t g = static_cast<uint64_t>(g0);
+  const float* wp = HAS_W ? J.W + 4 * g0 : nullptr;
+  for (int32_t k = 0; k < count;) {
     GroupSums s;
+    const int32_t kend = min(count, k + kFlush);
 #pragma unroll 2
-    for (int u = 0; u < kFlush && g < full; ++u, g += stride) add_group<HAS_W>(s, J, g, K, 4, k0, k1);
+    for (; k < kend; ++k, g += stride) {
+      add_group<HAS_W>(s, J, wp, g, K, 4, k0, k1);
+      if (HAS_W) wp += 4 * stride;
+    }
     acc[0] += f2_sum(s.w1);
     acc[1] += f2_sum(s.w2);
     acc[2] += f2_sum(s.r1);
@@ -108,7 +116,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
-    add_group<HAS_W>(s, J, full, K, tail, k0, k1);
+    add_group<HAS_W>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1);
     acc[0] += f2_sum(s.w1);
     acc[1] += f2_sum(s.w2);
     acc[2] += f2_sum(s.r1);

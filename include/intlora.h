@@ -218,6 +218,17 @@ typedef struct intlora_merge_out {
 /* Bytes per element of `out`: MUL (variant 0) or SHIFT (variant 1). */
 int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits);
 
+/* Workspace of a merge call (16-byte aligned device memory, caller-owned):
+ *  - for each layer with sigma_r == NULL: the scratch of its sigma_R reduction;
+ *  - for each layer with r in [32, 64] and n % 4 == 0 (on a device with the
+ *    tensor-map driver entry point): its product T = A B (d x n fp32) and the
+ *    exact tf32 hi/lo splits of A and B^T that the tensor cores multiply
+ *    (4 (d + n) kp x 2 bytes, kp = 32 or 64) -- [IntLoRA paper notes, method
+ *    section 2: U = s + (R* + A B) / D].
+ * A call given at least the sigma part but less than the whole still runs: it
+ * then forms A B on the CUDA cores inside the merge kernels (same results up
+ * to fp32 rounding order, slower at these ranks). Less than the sigma part:
+ * INTLORA_ERR_WORKSPACE. */
 size_t intlora_merge_workspace_size(const intlora_layer* layers, int32_t count);
 
 /* IntLoRA_MUL, u_bits in [2, 8]. */

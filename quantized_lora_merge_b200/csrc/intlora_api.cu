@@ -163,6 +163,7 @@ bool team_path_enabled() {
 bool team_eligible(int variant, const TileLayer& l) {
   if (l.n % 4 != 0 || l.n > kTeamMaxCols) return false;
   if (l.d > (int64_t{1} << 24)) return false;      // keeps tile indices of a batch in int32
+  if (l.d * l.n >= (int64_t{1} << 34)) return false; // Philox block index fits 32 bits
   if (variant != kGen && l.r > 0 && !aligned16(l.B)) return false;
   if (l.T != nullptr && !aligned16(l.T)) return false;
   return true;

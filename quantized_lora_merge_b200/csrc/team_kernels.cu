@@ -191,6 +191,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       __syncwarp();
     }
 
+    uint32_t ctr0[kTeamRows];                   // Philox block of (row, quad 0)
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) ctr0[ml] = static_cast<uint32_t>(irow[ml] * quads);
+
     // ---- phase A
     float hi[kTeamRows], lo[kTeamRows];
 #pragma unroll
@@ -248,7 +252,9 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       }
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml) {
-        const uint4 w4 = aux_block(static_cast<uint64_t>(irow[ml] * quads + q), sid, p.key0, p.key1);
+        // layers here have fewer than 2^34 elements: the block index fits the
+        // low counter word and the high word is 0 (rounds 0-1 partly uniform)
+        const uint4 w4 = philox10(ctr0[ml] + static_cast<uint32_t>(q), 0u, sid, 0u, p.key0, p.key1);
         const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
         float v[4];
 #pragma unroll

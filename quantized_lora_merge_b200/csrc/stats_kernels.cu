@@ -44,10 +44,12 @@ struct GroupSums {
   uint64_t w1 = 0, w2 = 0, r1 = 0, r2 = 0;
 };
 
-template <bool HAS_W>
+template <bool HAS_W, bool SMALL>
 __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, const float* wgroup,
                                           uint64_t group, float K, int valid, uint32_t k0, uint32_t k1) {
-  const uint4 w = aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
+  // SMALL: fewer than 2^34 elements, so the block index's high word is 0
+  const uint4 w = SMALL ? philox10(static_cast<uint32_t>(group), 0u, J.stream_id, 0u, k0, k1)
+                        : aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
   uint64_t r01, r23;
   if (valid == 4) {
     const uint64_t l01 = laplace_log2_x2(w.x, w.y), l23 = laplace_log2_x2(w.z, w.w);
@@ -87,7 +89,7 @@ __device__ __forceinline__ double f2_sum(uint64_t v) {
   return static_cast<double>(f2_lo(v)) + static_cast<double>(f2_hi(v));
 }
 
-template <bool HAS_W>
+template <bool HAS_W, bool SMALL>
 __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4],
                                            uint32_t k0, uint32_t k1) {
   constexpr int kFlush = 8;   // groups per fp32 partial
@@ -105,7 +107,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
     const int32_t kend = min(count, k + kFlush);
 #pragma unroll 2
     for (; k < kend; ++k, g += stride) {
-      add_group<HAS_W>(s, J, wp, g, K, 4, k0, k1);
+      add_group<HAS_W, SMALL>(s, J, wp, g, K, 4, k0, k1);
       if (HAS_W) wp += 4 * stride;
     }
     acc[0] += f2_sum(s.w1);
@@ -116,7 +118,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
-    add_group<HAS_W>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1);
+    add_group<HAS_W, SMALL>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1);
     acc[0] += f2_sum(s.w1);
     acc[1] += f2_sum(s.w2);
     acc[2] += f2_sum(s.r1);
@@ -132,8 +134,14 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_const
   const StatsJob& J = b.job[j];
   const int64_t local = bid - J.block_begin;
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  if (J.W != nullptr) stats_body<true>(J, local, acc, b.key0, b.key1);
-  else stats_body<false>(J, local, acc, b.key0, b.key1);
+  const bool small = J.numel < (int64_t{1} << 34);
+  if (J.W != nullptr) {
+    if (small) stats_body<true, true>(J, local, acc, b.key0, b.key1);
+    else stats_body<true, false>(J, local, acc, b.key0, b.key1);
+  } else {
+    if (small) stats_body<false, true>(J, local, acc, b.key0, b.key1);
+    else stats_body<false, false>(J, local, acc, b.key0, b.key1);
+  }
   block_sum4(acc, red);
   if (threadIdx.x == 0)
     for (int q = 0; q < 4; ++q) J.partial[local * 4 + q] = acc[q];

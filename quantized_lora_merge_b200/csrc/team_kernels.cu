@@ -369,6 +369,9 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
 
     // ---- phase B: quantize the parked values and store
     if (VARIANT == kGen && L.out == nullptr) continue;
+    int32_t gen_lo[kTeamRows];                 // base quantization: bias - z per row
+#pragma unroll
+    for (int ml = 0; ml < kTeamRows; ++ml) gen_lo[ml] = kRoundBiasBits - zq[ml];
     for (int k = 0; k < S; ++k) {
       const int q = lt + k * LT;
       if (q >= quads) break;
@@ -399,17 +402,23 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
             res[c] = centred * (nib<WBITS>(cw[ml], c) - zv[ml]);
             code8[c] = static_cast<uint32_t>(centred + zq[ml]);
           } else {
-            code8[c] = static_cast<uint32_t>(clamp_i(rne_scaled(uv[c], inv[ml]) + zq[ml], 0, qmax));
+            // the biased rounding word clamped straight to the code range
+            // [bias - z, bias - z + qmax]; the bias comes off once per word below
+            code8[c] = static_cast<uint32_t>(
+                clamp_i(__float_as_int(fmaf(uv[c], inv[ml], kRoundBias)), gen_lo[ml], gen_lo[ml] + qmax));
             res[c] = 0;
           }
         }
         if (VARIANT == kGen) {
+          // sum_c (word_c - lo) 2^(bits c), modulo 2^32 (multiply-adds)
           uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
+          const uint32_t lo = static_cast<uint32_t>(gen_lo[ml]);
           if (WBITS == 8)
-            *reinterpret_cast<uint32_t*>(orow + j) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
+            *reinterpret_cast<uint32_t*>(orow + j) =
+                code8[0] + code8[1] * 0x100u + code8[2] * 0x10000u + code8[3] * 0x1000000u - lo * 0x01010101u;
           else
-            *reinterpret_cast<uint16_t*>(orow + (j >> 1)) =
-                static_cast<uint16_t>(code8[0] | (code8[1] << 4) | (code8[2] << 8) | (code8[3] << 12));
+            *reinterpret_cast<uint16_t*>(orow + (j >> 1)) = static_cast<uint16_t>(
+                code8[0] + code8[1] * 16u + code8[2] * 256u + code8[3] * 4096u - lo * 0x1111u);
           continue;
         }
         const int64_t e0 = i * n + j;

@@ -367,6 +367,9 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
   b.out_bytes = out_bytes;
   b.key0 = static_cast<uint32_t>(seed);
   b.key1 = static_cast<uint32_t>(seed >> 32);
+  b.small = 1;
+  for (auto& l : L)
+    if (l.d * l.n >= (int64_t{1} << 34)) b.small = 0;
   cudaError_t e = launch_tiles(b, rank_ct, aligned, stream);
   if (e != cudaSuccess) return cuda_fail(e, "row-tile kernel launch");
   return INTLORA_OK;

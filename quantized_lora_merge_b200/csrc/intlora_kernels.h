@@ -86,6 +86,7 @@ struct TileBatch {
   int32_t smem_u;            // floats of the tile buffer (>= m n_c of every layer)
   int32_t smem_b;            // floats of the B buffer
   int32_t smem_a;            // floats of the A-rows buffer (>= r m)
+  int32_t small;             // every layer below 2^34 elements (32-bit Philox block index)
 };
 
 constexpr int kTileThreads = 256;

@@ -348,7 +348,9 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
           const int64_t e0 = (row0 + min(rr, rows - 1)) * n + j;
           uint32_t words[4];
           if (ALIGNED) {
-            const uint4 w4 = aux_block(static_cast<uint64_t>(blk0 + ml * nq), sid, p.key0, p.key1);
+            // layers below 2^34 elements: block index in the low counter word
+            const uint4 w4 = p.small ? philox10(static_cast<uint32_t>(blk0 + ml * nq), 0u, sid, 0u, p.key0, p.key1)
+                                     : aux_block(static_cast<uint64_t>(blk0 + ml * nq), sid, p.key0, p.key1);
             words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
           } else {
 #pragma unroll

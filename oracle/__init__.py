@@ -74,6 +74,8 @@ def _load():
         "orc_ste_backward": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _ptr]),
         "orc_ste_sampled": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _i64, _ptr, _i64,
                                    _ptr, _ptr]),
+        "orc_int_digits": (_i64, [_ptr, _i64, _i64, _int, _ptr]),
+        "orc_int_gemm_rows": (None, [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_num_threads": (_int, []),
     }
     for name, (res, args) in sig.items():
@@ -288,6 +290,40 @@ def ste_sampled(G_bits, A_bits, B_bits, rows, cols):
     _load().orc_ste_sampled(_p(g), _p(a), _p(b), d, n, r, _p(rw), rw.size, _p(cl), cl.size,
                             _p(dA), _p(dB))
     return dA, dB.T.copy()
+
+
+# --------------------------------------------------------------------------
+# Integer inference GEMM on the merged weights (Y = X W'^T)
+# --------------------------------------------------------------------------
+def int_planes(max_abs: int) -> int:
+    """Base-128 digit planes that hold every integer weight with |w| <= max_abs."""
+    for p in (1, 2, 3):
+        if max_abs <= 2 ** (7 * p) - 1:
+            return p
+    return 0
+
+
+def int_digits(W, planes: int):
+    """(digits [d][planes][n] int8, count of weights out of range)."""
+    w = _c(W, np.int64)
+    d, n = w.shape
+    out = np.zeros((d, planes, n), np.int8)
+    bad = _load().orc_int_digits(_p(w), d, n, planes, _p(out))
+    return out, int(bad)
+
+
+def int_gemm_rows(X, x_scale, W, w_scale, rows=None):
+    """Y rows (fp64) of the integer GEMM for the given token rows (all by default)."""
+    x = _c(X, np.int8)
+    xs = _c(x_scale, np.float64)
+    w = _c(W, np.int64)
+    ws = _c(w_scale, np.float64)
+    tokens, n = x.shape
+    d = w.shape[0]
+    rw = _c(np.arange(tokens) if rows is None else rows, np.int64)
+    Y = np.zeros((rw.size, d), np.float64)
+    _load().orc_int_gemm_rows(_p(x), _p(xs), _p(w), _p(ws), tokens, d, n, _p(rw), rw.size, _p(Y))
+    return Y
 
 
 def num_threads() -> int:

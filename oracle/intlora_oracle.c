@@ -31,7 +31,9 @@
  *   - rounding is to nearest, ties to even (C nearbyint in the default mode);
  *   - SHIFT: V = U / max_j |U_ij|, shift = nearest integer to -log2|V|,
  *     clamped to [0, 2^b - 1], and ">>" is an arithmetic (floor) shift;
- *   - the STE backward is the plain pair dA = G B^T, dB = A^T G.
+ *   - the STE backward is the plain pair dA = G B^T, dB = A^T G;
+ *   - the integer inference GEMM takes int8 activations with a per-token
+ *     scale and the merged integer weights with their per-row scale s_bar.
  *
  * Parity pins: every exported function is pinned by a test that does not
  * retype its formula (brute-force enumeration, closed forms, exact rational
@@ -442,6 +444,45 @@ void orc_ste_sampled(const uint16_t* G, const uint16_t* A, const uint16_t* B, in
                 acc += bf16_value(A[i * r + k]) * bf16_value(G[i * n + j]);
             dB_cols[t * r + k] = acc;
         }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Integer inference on the merged weights [IntLoRA notes, "两种实现版本" and */
+/* the efficiency table: the merged weight s_bar_i Q_ij is already integer,   */
+/* so a layer runs as an integer GEMM with no post-training quantization].    */
+/* ------------------------------------------------------------------------ */
+
+/* Digits of an integer weight in base 128 for an 8-bit integer MMA: with P
+ * planes, digit k < P-1 is (w >> 7k) & 127 and the top digit is w >> 7(P-1)
+ * (arithmetic shift), so w = sum_k 128^k digit_k. Layout [d][P][n]. Returns
+ * the number of weights whose top digit leaves [-128, 127] (stored truncated). */
+int64_t orc_int_digits(const int64_t* w, int64_t d, int64_t n, int planes, int8_t* out) {
+    int64_t bad = 0;
+    for (int64_t i = 0; i < d; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t v = w[i * n + j];
+            for (int k = 0; k < planes; ++k) {
+                int64_t digit = k < planes - 1 ? (v >> (7 * k)) & 127 : v >> (7 * k);
+                if (k == planes - 1 && (digit < -128 || digit > 127)) ++bad;
+                out[(i * planes + k) * n + j] = (int8_t)digit;
+            }
+        }
+    return bad;
+}
+
+/* Y[t][i] = x_scale[t] * w_scale[i] * sum_j X[t][j] W[i][j] for the listed
+ * token rows: the integer sum is exact (int64), the scaling is fp64. */
+void orc_int_gemm_rows(const int8_t* X, const double* x_scale, const int64_t* W,
+                       const double* w_scale, int64_t tokens, int64_t d, int64_t n,
+                       const int64_t* rows, int64_t n_rows, double* Y) {
+    (void)tokens;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t q = 0; q < n_rows * d; ++q) {
+        int64_t t = rows[q / d], i = q % d;
+        int64_t acc = 0;
+        for (int64_t j = 0; j < n; ++j) acc += (int64_t)X[t * n + j] * W[i * n + j];
+        Y[q] = (double)acc * x_scale[t] * w_scale[i];
     }
 }
 

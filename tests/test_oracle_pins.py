@@ -412,3 +412,75 @@ def test_ste_backward_against_numpy():
     sA, sB = oracle.ste_sampled(Gb, Ab, Bb, rows, cols)
     np.testing.assert_allclose(sA, dA[rows], rtol=1e-12, atol=1e-18)
     np.testing.assert_allclose(sB, dB[:, cols], rtol=1e-12, atol=1e-18)
+
+
+# ---------------------------------------------------------------------------
+# Integer inference GEMM on the merged weights (Y = X W'^T)
+# ---------------------------------------------------------------------------
+def test_int_planes_bounds():
+    assert [oracle.int_planes(v) for v in (0, 127, 128, 16383, 16384, 2**21 - 1, 2**21)] == \
+        [1, 1, 2, 2, 3, 3, 0]
+    # merged-weight bounds: |P| <= (2^b_W - 1)(2^b_U - 1) (MUL), |M| <= 2^b_W - 1 (SHIFT)
+    assert oracle.int_planes(15 * 15) == 2 and oracle.int_planes(255 * 255) == 3
+    assert oracle.int_planes(15) == 1 and oracle.int_planes(255) == 2
+
+
+@pytest.mark.parametrize("planes,lo,hi", [(1, -128, 127), (2, -16384, 16383)])
+def test_int_digits_exhaustive(planes, lo, hi):
+    """Every w in range: the digits rebuild w in base 128, lower digits lie in
+    [0, 127] and the top digit in [-128, 127] (which makes them unique)."""
+    w = np.arange(lo, hi + 1, dtype=np.int64).reshape(1, -1)
+    dig, bad = oracle.int_digits(w, planes)
+    assert bad == 0
+    dig = dig[0].astype(np.int64)                     # [planes][n]
+    rebuilt = sum(dig[k] * 128**k for k in range(planes))
+    assert np.array_equal(rebuilt, w[0])
+    for k in range(planes - 1):
+        assert dig[k].min() >= 0 and dig[k].max() <= 127
+
+
+def test_int_digits_three_planes_and_overflow():
+    rng = np.random.default_rng(5)
+    w = np.concatenate([rng.integers(-2**21, 2**21, 4000), [-2**21, 2**21 - 1, 0, -1, 127, -128]])
+    dig, bad = oracle.int_digits(w.reshape(2, -1), 3)
+    assert bad == 0
+    d = dig.astype(np.int64)
+    assert np.array_equal(d[:, 0] + 128 * d[:, 1] + 16384 * d[:, 2], w.reshape(2, -1))
+    for planes, out in ((1, [128, -129, 5]), (2, [16384, -16385, 3])):
+        _, bad = oracle.int_digits(np.array([out], np.int64), planes)
+        assert bad == 2
+
+
+def test_int_gemm_brute_force_tiny():
+    rng = np.random.default_rng(8)
+    X = rng.integers(-128, 128, (3, 5)).astype(np.int8)
+    W = rng.integers(-300, 300, (4, 5))
+    xs, ws = rng.uniform(0.01, 1, 3), rng.uniform(0.01, 1, 4)
+    Y = oracle.int_gemm_rows(X, xs, W, ws)
+    for t in range(3):
+        for i in range(4):
+            acc = sum(int(X[t, j]) * int(W[i, j]) for j in range(5))
+            assert Y[t, i] == acc * xs[t] * ws[i]
+    np.testing.assert_array_equal(oracle.int_gemm_rows(X, xs, W, ws, rows=[2, 0]), Y[[2, 0]])
+
+
+def test_int_gemm_is_the_dequantized_matmul_of_merged_weights():
+    """Y equals numpy's fp64 matmul of the dequantized activations with the
+    merged weight W' = s_bar P of an oracle MUL merge, and equals the sum of
+    the digit-plane products scaled by 128^k."""
+    spec, W, A, B, g = _prepared(12, 40, 4, 4, sid=3)
+    s32 = g["s"].astype(np.float32)
+    m = oracle.merge_mul(g["codes"], s32, g["z"], A, B, spec.seed, 3, g["sigma_w"], g["sigma_r"],
+                         spec.alpha, 4)
+    P, sbar = m["P"], m["sbar"]
+    rng = np.random.default_rng(4)
+    X = rng.integers(-127, 128, (7, 40)).astype(np.int8)
+    xs = rng.uniform(1e-3, 1e-2, 7)
+    Y = oracle.int_gemm_rows(X, xs, P, sbar)
+    Wm = sbar[:, None] * P
+    np.testing.assert_allclose(Y, (xs[:, None] * X) @ Wm.T, rtol=1e-12, atol=1e-300)
+    planes = oracle.int_planes(int(np.abs(P).max()))
+    dig, bad = oracle.int_digits(P, planes)
+    assert bad == 0
+    acc = sum(128**k * (X.astype(np.int64) @ dig[:, k, :].astype(np.int64).T) for k in range(planes))
+    np.testing.assert_allclose(Y, acc * xs[:, None] * sbar[None, :], rtol=1e-15, atol=0)

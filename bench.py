@@ -48,6 +48,13 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--op", default="step", choices=["step", "int_gemm"],
+                    help="step: the merge hot path (default); int_gemm: the integer "
+                         "inference GEMM on merged weights")
+    ap.add_argument("--planes", type=int, default=1, choices=[1, 2, 3],
+                    help="int_gemm: digit planes of the merged weights (1: SHIFT of 4-bit "
+                         "codes, 2: MUL of 4-bit codes, 3: MUL of 8-bit codes)")
+    ap.add_argument("--tokens", type=int, default=4096)
     return ap.parse_args()
 
 
@@ -280,6 +287,9 @@ def run_reference(args, layers, desc):
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
+    if args.op == "int_gemm":
+        bench_int_gemm(args)
+        return
     from quantized_lora_merge_b200 import workloads as wl
     layers_base = wl.CONFIGS[args.config]()
     desc = workload_desc(args.config, layers_base)
@@ -496,6 +506,144 @@ def e2e(layers, path, arena_in, arena_out, device, steps, world, elements):
     return {"value": elements / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "pipelined": "2 device copies, 3 streams"}
+
+
+# ---------------------------------------------------------------------------
+# integer inference GEMM on merged weights (--op int_gemm)
+# ---------------------------------------------------------------------------
+GEMM_METRIC = "integer GEMM on merged weights: tensor ops/s (int8 MMA), 1 GPU"
+GEMM_UNIT = "Top/s"
+# DiT-3072 block linears (qkv, attention out, fc1, fc2) as (d, n)
+GEMM_SHAPES = [(9216, 3072), (3072, 3072), (12288, 3072), (3072, 12288)]
+GEMM_KIND = {1: "shift4", 2: "mul4", 3: "mul8"}
+
+
+def bf16_peak_tflops():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        for k in ("bf16_tflops", "bf16_tflops_burst"):
+            if k in d:
+                return float(d[k]), "measured"
+    return 1590.0, "fallback"
+
+
+def bench_int_gemm(args):
+    """One step = the four DiT-3072 block GEMMs Y = X W'^T at `tokens` tokens
+    (one batched call): int8 activations x merged integer weights held as
+    `planes` int8 digit planes. Metric: int8 tensor ops per second executed
+    (2 tokens d n planes per step); algorithmic ops (2 tokens d n) beside it."""
+    import torch
+
+    from quantized_lora_merge_b200 import binding as B
+    from quantized_lora_merge_b200 import build as qbuild
+    from quantized_lora_merge_b200 import workloads as wl
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    qbuild.build()
+    P, T = args.planes, args.tokens
+    bound = wl.INT_GEMM_BOUNDS[GEMM_KIND[P]]
+    jobs, host = [], []
+    for k, (d, n) in enumerate(GEMM_SHAPES):
+        X, xs, Q, ws = wl.int_gemm_device(T, d, n, bound, device, salt=k)
+        packed = torch.empty((d, P, n), dtype=torch.int8, device=device)
+        B.intlora_int_pack(Q, P, packed)
+        del Q
+        jobs.append(B.IntGemmJob(X, xs, packed, ws, torch.empty((T, d), device=device)))
+        host.append((d, n))
+    desc_jobs = B.Descriptors(jobs)
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    tensor_ops = sum(2 * T * d * n * P for d, n in host)
+    alg_ops = sum(2 * T * d * n for d, n in host)
+    in_bytes = sum(T * n + d * n * P + 4 * (T + d) for d, n in host)
+    out_bytes = sum(4 * T * d for d, n in host)
+    for _ in range(max(3, args.warmup)):
+        B.intlora_int_gemm_batched(desc_jobs, P)
+    torch.cuda.synchronize(device)
+    steps = args.steps if args.steps != 1000 else 200
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    a.record(stream)
+    for _ in range(steps):
+        B.intlora_int_gemm_batched(desc_jobs, P)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    ms = a.elapsed_time(b) / steps
+    achieved = tensor_ops / (ms / 1e3) / 1e12
+    bf16, kind = bf16_peak_tflops()
+    peak = 2.0 * bf16                       # int8 dense = 2 x bf16 dense (nominal ratio)
+    # end to end: X from pinned host memory, Y back, through the same call
+    hx = [torch.empty_like(j.X, device="cpu").pin_memory() for j in jobs]
+    hy = [torch.empty_like(j.Y, device="cpu").pin_memory() for j in jobs]
+    for h, j in zip(hx, jobs):
+        h.copy_(j.X)
+    e2e_steps = 5
+    ea = torch.cuda.Event(enable_timing=True)
+    eb = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        for h, j in zip(hx, jobs):
+            j.X.copy_(h, non_blocking=True)
+        B.intlora_int_gemm_batched(desc_jobs, P)
+        for h, j in zip(hy, jobs):
+            h.copy_(j.Y, non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = ea.elapsed_time(eb) / e2e_steps
+    line = {
+        "metric": GEMM_METRIC, "value": achieved, "unit": GEMM_UNIT, "n_gpus": 1,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8 x s8 -> s32", "data": "synthetic",
+        "config": {"workload": f"DiT-3072 block linears (qkv 9216x3072, out 3072x3072, fc1 "
+                               f"12288x3072, fc2 3072x12288) at {T} tokens, W'={GEMM_KIND[P]} "
+                               f"merged weights as {P} int8 digit plane(s), int8 activations",
+                   "tokens": T, "planes": P,
+                   "l2": f"inputs {in_bytes / 1e6:.0f} MB + outputs {out_bytes / 1e6:.0f} MB per "
+                         f"step, larger than L2"},
+        "algorithmic_Top_s": alg_ops / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "int_gemm_kernel (tcgen05 kind::i8)",
+                     "achieved": achieved, "peak": peak, "unit": "Top/s",
+                     "frac": achieved / peak,
+                     "peak_source": f"2 x {kind} bf16 dense {bf16:.0f} TFLOP/s (int8/bf16 "
+                                    f"nominal ratio 4.5/2.25)",
+                     "traffic": None},
+        "clocks": clk, "gpu_launches": steps,
+        "e2e": {"value": tensor_ops / (e2e_ms / 1e3) / 1e12, "unit": GEMM_UNIT,
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": sum(j.X.numel() for j in jobs),
+                "d2h_bytes_per_step": sum(4 * j.Y.numel() for j in jobs)},
+    }
+    if not args.no_cpu_baseline:
+        import numpy as np
+
+        import oracle
+        X0, xs0, Q0, ws0 = wl.int_gemm_host(T, *GEMM_SHAPES[0], bound)
+        t0 = time.perf_counter()
+        rows, done = 0, 0
+        while time.perf_counter() - t0 < min(args.cpu_seconds, 10.0) and rows < T:
+            oracle.int_gemm_rows(X0, xs0.astype(np.float64), Q0, ws0.astype(np.float64),
+                                 np.arange(rows, rows + 4))
+            rows += 4
+        dt = time.perf_counter() - t0
+        done = 2 * rows * GEMM_SHAPES[0][0] * GEMM_SHAPES[0][1]
+        line["cpu_baseline"] = {"value": done / dt / 1e12, "unit": "Top/s (algorithmic)",
+                                "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"{rows} token rows of the qkv GEMM "
+                                          f"({GEMM_SHAPES[0][0]}x{GEMM_SHAPES[0][1]}), "
+                                          f"exact int64 sums, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
 
 
 if __name__ == "__main__":

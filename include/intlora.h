@@ -16,7 +16,9 @@
  *                           Hadamard product;
  *   - intlora_merge_shift   IntLoRA_SHIFT: U quantized by a log2 quantizer,
  *                           merged by arithmetic shifts;
- *   - intlora_ste_backward  straight-through backward dA = G B^T, dB = A^T G.
+ *   - intlora_ste_backward  straight-through backward dA = G B^T, dB = A^T G;
+ *   - intlora_int_gemm      integer inference GEMM on the merged weights
+ *                           (int8 activations x integer merged weights).
  *
  * Sources, cited by page title and section:
  *   [notes]   "IntLoRA: Integral Low-rank Adaptation of Quantized Diffusion
@@ -274,6 +276,58 @@ intlora_status intlora_ste_backward(const void* G, const void* A, const void* B,
                                     size_t ws_bytes, void* stream);
 intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t count,
                                             void* ws, size_t ws_bytes, void* stream);
+
+/* --------------------------------------------------------------------------
+ * Integer inference on the merged weights [notes, 两种实现版本 and the
+ * training/inference efficiency table: the merged weight is s_bar_i Q_ij with
+ * Q integer (IntLoRA_MUL: Q = P = (U_round - z_bar) D; IntLoRA_SHIFT:
+ * Q = M = sign(V) (D >> shift)), so the merged layer runs as an integer GEMM
+ * (W8A8 / W4A8) with no post-training quantization step]:
+ *
+ *   Y[t][i] = x_scale[t] * w_scale[i] * sum_j X[t][j] Q[i][j]
+ *
+ * X: int8 activations, tokens x n row-major, with a per-token scale (the
+ * activation quantizer is the caller's). w_scale: s_bar of the merged layer.
+ *
+ * Q reaches the tensor cores as P base-128 digit planes of int8:
+ *   digit_k = (Q >> 7k) & 127 for k < P - 1, digit_{P-1} = Q >> 7(P-1)
+ * (arithmetic shift), Q = sum_k 128^k digit_k. P = 1 holds |Q| <= 127 (SHIFT
+ * of 4-bit codes), 2 holds |Q| <= 16383 (MUL of 4-bit codes, SHIFT of 8-bit
+ * codes), 3 holds |Q| <= 2^21 - 1 (MUL of 8-bit codes); each plane costs one
+ * int8 GEMM.
+ * ------------------------------------------------------------------------ */
+
+/* Digit planes needed for |Q| <= max_abs: 1, 2 or 3; 0 if above 2^21 - 1. */
+int32_t intlora_int_planes(int64_t max_abs);
+
+/* Packs Q (d x n row-major; q_bytes = 1, 2 or 4: int8, int16 or int32, the
+ * merge outputs) into `packed`, laid out [d][planes][n] int8 (plane k of row i
+ * at packed + (i * planes + k) * n). n % 16 == 0; packed 16-byte aligned.
+ * If `overflow` (a device int32, may be NULL) is given, the number of values
+ * whose top digit leaves [-128, 127] is added to it (those are stored
+ * truncated). Asynchronous on `stream`. */
+intlora_status intlora_int_pack(const void* q, int32_t q_bytes, int64_t d, int64_t n,
+                                int32_t planes, int8_t* packed, int32_t* overflow,
+                                void* stream);
+
+typedef struct intlora_int_gemm_job {
+    const int8_t* X;          /* tokens x n, 16-byte aligned */
+    const float* x_scale;     /* [tokens] */
+    const int8_t* W;          /* packed digit planes [d][planes][n], 16-byte aligned */
+    const float* w_scale;     /* [d] */
+    int64_t tokens, d, n;     /* n % 16 == 0; tokens, d * planes <= 2^31 */
+    float* Y;                 /* tokens x d row-major, 16-byte aligned (overwritten) */
+} intlora_int_gemm_job;
+
+/* Every job of one call uses the same plane count. The integer sums are
+ * exact (s32 per plane, planes added in 64-bit integers); the result is
+ * fp32(sum) * fp32(x_scale[t] * w_scale[i]), three fp32 roundings. Jobs with
+ * n = 0 get Y = 0. Asynchronous on `stream`; no workspace. */
+intlora_status intlora_int_gemm_batched(const intlora_int_gemm_job* jobs, int32_t count,
+                                        int32_t planes, void* stream);
+intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int8_t* W,
+                                const float* w_scale, int64_t tokens, int64_t d, int64_t n,
+                                int32_t planes, float* Y, void* stream);
 
 /* Number of bounded device-side waits that gave up since the library was
  * loaded: 0 in a healthy run. The tensor-core STE kernel bounds every wait on

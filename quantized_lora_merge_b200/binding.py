@@ -55,6 +55,11 @@ class intlora_ste_job(ctypes.Structure):
                 ("r", _c_i32), ("dA", _c_ptr), ("dB", _c_ptr)]
 
 
+class intlora_int_gemm_job(ctypes.Structure):
+    _fields_ = [("X", _c_ptr), ("x_scale", _c_ptr), ("W", _c_ptr), ("w_scale", _c_ptr),
+                ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("Y", _c_ptr)]
+
+
 _P = ctypes.POINTER
 _SIGNATURES = {
     "intlora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -85,6 +90,13 @@ _SIGNATURES = {
                                             _c_ptr, _c_ptr, _c_ptr, _c_size, _c_ptr]),
     "intlora_ste_backward_batched": (ctypes.c_int, [_P(intlora_ste_job), _c_i32, _c_ptr,
                                                     _c_size, _c_ptr]),
+    "intlora_int_planes": (_c_i32, [_c_i64]),
+    "intlora_int_pack": (ctypes.c_int, [_c_ptr, _c_i32, _c_i64, _c_i64, _c_i32, _c_ptr, _c_ptr,
+                                        _c_ptr]),
+    "intlora_int_gemm_batched": (ctypes.c_int, [_P(intlora_int_gemm_job), _c_i32, _c_i32,
+                                                _c_ptr]),
+    "intlora_int_gemm": (ctypes.c_int, [_c_ptr, _c_ptr, _c_ptr, _c_ptr, _c_i64, _c_i64, _c_i64,
+                                        _c_i32, _c_ptr, _c_ptr]),
 }
 
 _lib = None
@@ -212,6 +224,20 @@ class SteJob:
                                _ptr(self.dA), _ptr(self.dB))
 
 
+@dataclass
+class IntGemmJob:
+    X: object                       # int8 [tokens, n]
+    x_scale: object                 # fp32 [tokens]
+    W: object                       # int8 [d, planes, n] digit planes
+    w_scale: object                 # fp32 [d]
+    Y: object                       # fp32 [tokens, d]
+
+    def to_c(self) -> intlora_int_gemm_job:
+        tokens, n = self.X.shape
+        return intlora_int_gemm_job(_ptr(self.X), _ptr(self.x_scale), _ptr(self.W),
+                                    _ptr(self.w_scale), tokens, self.W.shape[0], n, _ptr(self.Y))
+
+
 def _array(struct, items):
     if isinstance(items, Descriptors):
         if items.struct is not struct:
@@ -247,7 +273,8 @@ class Descriptors:
 
 
 Descriptors._STRUCT = {AuxJob: intlora_aux_job, Layer: intlora_layer,
-                       MergeOut: intlora_merge_out, SteJob: intlora_ste_job}
+                       MergeOut: intlora_merge_out, SteJob: intlora_ste_job,
+                       IntGemmJob: intlora_int_gemm_job}
 
 
 # ---------------------------------------------------------------------------
@@ -343,3 +370,26 @@ def intlora_ste_backward_batched(jobs: Sequence[SteJob], ws=None, stream=None) -
     p, nb = _ws(ws)
     _check(lib().intlora_ste_backward_batched(_array(intlora_ste_job, jobs), len(jobs), p, nb,
                                               _stream(stream)))
+
+
+def intlora_int_planes(max_abs: int) -> int:
+    return lib().intlora_int_planes(max_abs)
+
+
+def intlora_int_pack(q, planes: int, packed, overflow=None, stream=None) -> None:
+    """Packs the merged integer weights q (int8/int16/int32 [d, n]) into
+    base-128 digit planes packed (int8 [d, planes, n])."""
+    d, n = q.shape
+    _check(lib().intlora_int_pack(_ptr(q), q.element_size(), d, n, planes, _ptr(packed),
+                                  _ptr(overflow), _stream(stream)))
+
+
+def intlora_int_gemm_batched(jobs: Sequence[IntGemmJob], planes: int, stream=None) -> None:
+    _check(lib().intlora_int_gemm_batched(_array(intlora_int_gemm_job, jobs), len(jobs), planes,
+                                          _stream(stream)))
+
+
+def intlora_int_gemm(job: IntGemmJob, planes: int, stream=None) -> None:
+    c = job.to_c()
+    _check(lib().intlora_int_gemm(c.X, c.x_scale, c.W, c.w_scale, c.tokens, c.d, c.n, planes,
+                                  c.Y, _stream(stream)))

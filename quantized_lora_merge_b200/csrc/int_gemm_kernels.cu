@@ -1,0 +1,402 @@
+// Integer inference on merged IntLoRA weights: Y = X W'^T with W' = s_bar Q
+// [IntLoRA paper notes (ICML2025), section 两种实现版本: the merged weight of
+// IntLoRA_MUL is s_bar (U_round - z_bar) (.) (W_round - z) and that of
+// IntLoRA_SHIFT is s_bar sign(V) (.) ((W_round - z) >> shift), i.e. an
+// integer matrix Q times a per-row scale; the efficiency table runs the merged
+// model as W8A8 / W4A8 with no post-training quantization].
+//
+//   Y[t][i] = x_scale[t] * w_scale[i] * sum_j X[t][j] Q[i][j]
+//
+// X is int8 (tokens x n). Q is held as P base-128 digit planes of int8
+// (P = 1 when |Q| <= 127, the SHIFT merge of 4-bit codes; 2 for the MUL
+// merge of 4-bit codes, |P| <= 225; 3 for 8-bit codes), packed channel-major
+// [d][P][n] so that one TMA box of P C rows holds all planes of C channels.
+//
+// The GEMM runs on the 5th-generation tensor cores: tcgen05.mma.kind::i8
+// (signed x signed, s32 accumulate in TMEM), M = 128 tokens, N = P C <= 256
+// digit rows, K = 32 bytes per instruction, 128-byte K slices per pipeline
+// stage staged by TMA with the 128-byte swizzle. A persistent CTA per SM:
+// warp 0 issues the TMA loads, warp 1 the MMAs, warps 4-11 drain the
+// double-buffered accumulator (tcgen05.ld; two warps per 32-lane TMEM
+// quarter, each taking half of the tile's channels), add the planes exactly
+// in 64-bit integers and scale in fp32. The integer part is exact; the only roundings
+// are the int -> fp32 conversion, the scale product and the final multiply.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "intlora_device.cuh"
+#include "intlora_kernels.h"
+#include "tcgen05_util.cuh"
+
+namespace intlora {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kIgThreads = 384;
+constexpr int kIgEpiThreads = 256;            // warps 4-11
+constexpr int kIgRows = 128;                    // tokens per tile (M, TMEM lanes)
+constexpr int kIgMaxN = 256;                    // digit rows per tile (N)
+constexpr int kIgK = 128;                       // K bytes per stage (one swizzle row)
+constexpr uint32_t kIgABytes = kIgRows * kIgK;  // 16 KB
+constexpr int kMaxIgJobs = 48;
+
+__device__ unsigned int g_ig_timeouts;
+
+__device__ __forceinline__ bool wait_ig(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait(bar, parity, abort_flag, &g_ig_timeouts);
+}
+
+struct alignas(64) IgJob {
+  CUtensorMap x_map;          // {n, tokens} int8, box {128, 128}
+  CUtensorMap w_map;          // {n, d P} int8, box {128, C P}
+  const float* x_scale;
+  const float* w_scale;
+  float* Y;
+  int64_t tokens, d, n;
+  int32_t m_tiles, n_tiles, k_stages, pad;
+  int64_t tile_begin;
+};
+struct IgBatch {
+  IgJob job[kMaxIgJobs];
+  int32_t count;
+  int32_t planes;             // P
+  int32_t chans;              // C: channels per tile
+  int32_t stages;
+  int64_t total_tiles;
+};
+
+struct IgTile {
+  int job;
+  int64_t t0, i0;
+};
+__device__ __forceinline__ IgTile ig_tile(const IgBatch& b, int64_t u) {
+  int j = 0;
+  while (j + 1 < b.count && b.job[j + 1].tile_begin <= u) ++j;
+  const IgJob& J = b.job[j];
+  const int64_t local = u - J.tile_begin;
+  const int64_t nt = local / J.m_tiles;
+  IgTile x;
+  x.job = j;
+  x.t0 = (local - nt * J.m_tiles) * kIgRows;
+  x.i0 = nt * b.chans;
+  return x;
+}
+
+__device__ __forceinline__ void tc_mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// kind::i8: D s32, A and B signed 8-bit, both K-major, M = 128, N = nrows.
+__device__ __forceinline__ uint32_t ig_idesc(int nrows) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nrows >> 3) << 17) |
+         (static_cast<uint32_t>(kIgRows >> 4) << 24);
+}
+
+template <int P>
+__device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J, int64_t t, float xs,
+                                                  int64_t i, bool row_ok) {
+  float raw[16 * P];
+#pragma unroll
+  for (int q = 0; q < P; ++q) tmem_ld16(taddr + static_cast<uint32_t>(16 * q), raw + 16 * q);
+  tmem_ld_wait();
+  if (!row_ok || i >= J.d) return;
+  float y[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    float v;
+    if (P == 1) {
+      v = static_cast<float>(__float_as_int(raw[c]));
+    } else {
+      int64_t s = 0;
+#pragma unroll
+      for (int p = 0; p < P; ++p) s += static_cast<int64_t>(__float_as_int(raw[c * P + p])) << (7 * p);
+      v = static_cast<float>(s);
+    }
+    y[c] = v;
+  }
+  float ws[16];
+  if (i + 16 <= J.d && (reinterpret_cast<uintptr_t>(J.w_scale) & 15u) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 w4 = __ldg(reinterpret_cast<const float4*>(J.w_scale + i) + q);
+      ws[4 * q] = w4.x;
+      ws[4 * q + 1] = w4.y;
+      ws[4 * q + 2] = w4.z;
+      ws[4 * q + 3] = w4.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) ws[c] = i + c < J.d ? __ldg(J.w_scale + i + c) : 0.0f;
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) y[c] *= xs * ws[c];
+  float* dst = J.Y + t * J.d + i;
+  if (i + 16 <= J.d && (J.d & 3) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      reinterpret_cast<float4*>(dst)[q] = make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 16; ++c)
+      if (i + c < J.d) dst[c] = y[c];
+  }
+}
+
+template <int P>
+__global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_constant__ IgBatch b) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
+  const int S = b.stages;
+  const int nrows = P * b.chans;                        // digit rows of a tile
+  const uint32_t b_bytes = static_cast<uint32_t>(nrows) * kIgK;
+  const uint32_t stage_bytes = kIgABytes + b_bytes;     // multiple of 1024
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* d_full = bars + 2 * S;                      // [2]
+  uint64_t* d_empty = d_full + 2;                       // [2]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&d_full[q], 1);
+      mbar_init(&d_empty[q], kIgEpiThreads);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(&tmem_slot)), "r"(2 * kIgMaxN) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;                      // accumulator q at column q * 256
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < b.total_tiles && ok && !abort_flag; u += gridDim.x) {
+        const IgTile x = ig_tile(b, u);
+        const IgJob& J = b.job[x.job];
+        const int32_t ty = static_cast<int32_t>(x.t0);
+        const int32_t wy = static_cast<int32_t>(x.i0 * P);
+        for (int kb = 0; kb < J.k_stages; ++kb) {
+          if (!wait_ig(&empty[stage], ph ^ 1u, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_tx(&full[stage], stage_bytes);
+          uint8_t* dst = base + stage * stage_bytes;
+          tma_load_2d(dst, &J.x_map, kb * kIgK, ty, &full[stage]);
+          tma_load_2d(dst + kIgABytes, &J.w_map, kb * kIgK, wy, &full[stage]);
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0, buf = 0;
+      uint32_t ph = 0, bph = 0;
+      const uint32_t idesc = ig_idesc(nrows);
+      bool ok = true;
+      for (int64_t u = blockIdx.x; u < b.total_tiles && ok && !abort_flag; u += gridDim.x) {
+        const IgTile x = ig_tile(b, u);
+        const int kst = b.job[x.job].k_stages;
+        if (!wait_ig(&d_empty[buf], bph ^ 1u, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t dt = tmem + static_cast<uint32_t>(buf * kIgMaxN);
+        for (int kb = 0; kb < kst; ++kb) {
+          if (!wait_ig(&full[stage], ph, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t a0 = kmajor_desc(smem_u32(base + stage * stage_bytes));
+          const uint64_t b0 = kmajor_desc(smem_u32(base + stage * stage_bytes + kIgABytes));
+#pragma unroll
+          for (int ks = 0; ks < kIgK / 32; ++ks)      // 32 bytes (16-byte units x 2) per MMA
+            tc_mma_i8(dt, a0 + 2 * ks, b0 + 2 * ks, idesc, (kb | ks) != 0 ? 1u : 0u);
+          tc_commit(&empty[stage]);
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&d_full[buf]);
+        if (++buf == 2) {
+          buf = 0;
+          bph ^= 1u;
+        }
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------- epilogue: TMEM lane = token row of the tile
+    const int e = (warp & 3) * 32 + lane;                 // row of the tile
+    const int half = (warp - 4) >> 2;                     // channel half of the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int buf = 0;
+    uint32_t bph = 0;
+    for (int64_t u = blockIdx.x; u < b.total_tiles && !abort_flag; u += gridDim.x) {
+      const IgTile x = ig_tile(b, u);
+      const IgJob& J = b.job[x.job];
+      const int64_t t = x.t0 + e;
+      const bool row_ok = t < J.tokens;
+      const float xs = row_ok ? __ldg(J.x_scale + t) : 0.0f;
+      if (!wait_ig(&d_full[buf], bph, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(buf * kIgMaxN);
+      const int cbeg = half * (b.chans >> 1), cend = cbeg + (b.chans >> 1);
+      for (int c0 = cbeg; c0 < cend; c0 += 16)
+        ig_epilogue_chunk<P>(tb + static_cast<uint32_t>(c0 * P), J, t, xs, x.i0 + c0, row_ok);
+      tc_fence_before();
+      mbar_arrive(&d_empty[buf]);
+      if (++buf == 2) {
+        buf = 0;
+        bph ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (abort_flag) {
+      for (int k = 0; k < 2000; ++k) __nanosleep(1000);   // let copies in flight land
+    }
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kIgMaxN)
+                 : "memory");
+  }
+}
+
+size_t ig_smem_bytes(int planes, int stages) {
+  const size_t stage = kIgABytes + static_cast<size_t>(planes * int_gemm_chans(planes)) * kIgK;
+  return 1024 + static_cast<size_t>(stages) * stage + (2 * stages + 4) * 8;
+}
+
+// ---- digit planes ----------------------------------------------------------------
+__global__ void int_pack_kernel(const void* w, int w_bytes, int64_t d, int64_t n, int planes, int8_t* out,
+                                int32_t* overflow) {
+  const int64_t total = d * n;
+  int32_t bad = 0;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    int64_t v;
+    if (w_bytes == 1) v = static_cast<const int8_t*>(w)[e];
+    else if (w_bytes == 2) v = static_cast<const int16_t*>(w)[e];
+    else v = static_cast<const int32_t*>(w)[e];
+    const int64_t i = e / n, j = e - i * n;
+    int8_t* o = out + i * planes * n + j;
+    for (int k = 0; k < planes; ++k) {
+      const int64_t digit = k < planes - 1 ? (v >> (7 * k)) & 127 : v >> (7 * k);
+      if (k == planes - 1 && (digit < -128 || digit > 127)) ++bad;
+      o[k * n] = static_cast<int8_t>(digit);
+    }
+  }
+  if (overflow != nullptr && bad != 0) atomicAdd(overflow, bad);
+}
+
+}  // namespace
+
+int int_gemm_chans(int planes) { return planes == 1 ? 256 : planes == 2 ? 128 : 64; }
+
+bool int_gemm_supported() { return tc::encode_fn() != nullptr; }
+
+cudaError_t launch_int_pack(const void* w, int w_bytes, int64_t d, int64_t n, int planes, int8_t* out,
+                            int32_t* overflow, cudaStream_t s) {
+  const int64_t total = d * n;
+  if (total <= 0) return cudaSuccess;
+  const int64_t blocks = min64((total + 255) / 256, 148 * 16);
+  int_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, w_bytes, d, n, planes, out, overflow);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  static thread_local IgBatch b;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int chans = int_gemm_chans(planes);
+  for (int k0 = 0; k0 < count; k0 += kMaxIgJobs) {
+    const int m = count - k0 < kMaxIgJobs ? count - k0 : kMaxIgJobs;
+    std::memset(&b, 0, sizeof b);
+    int64_t tiles = 0;
+    for (int k = 0; k < m; ++k) {
+      const IntGemmJob& j = jobs[k0 + k];
+      IgJob& t = b.job[k];
+      const bool ok =
+          tc::encode_2d(&t.x_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.X, j.tokens, j.n, kIgK, kIgRows) &&
+          tc::encode_2d(&t.w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.W, j.d * planes, j.n, kIgK, chans * planes);
+      if (!ok) return cudaErrorInvalidValue;
+      t.x_scale = j.x_scale;
+      t.w_scale = j.w_scale;
+      t.Y = j.Y;
+      t.tokens = j.tokens;
+      t.d = j.d;
+      t.n = j.n;
+      t.m_tiles = static_cast<int32_t>((j.tokens + kIgRows - 1) / kIgRows);
+      t.n_tiles = static_cast<int32_t>((j.d + chans - 1) / chans);
+      t.k_stages = static_cast<int32_t>((j.n + kIgK - 1) / kIgK);
+      t.tile_begin = tiles;
+      tiles += static_cast<int64_t>(t.m_tiles) * t.n_tiles;
+    }
+    b.count = m;
+    b.planes = planes;
+    b.chans = chans;
+    int stages = 8;
+    while (stages > 2 && ig_smem_bytes(planes, stages) > 232448) --stages;
+    b.stages = stages;
+    b.total_tiles = tiles;
+    const size_t smem = ig_smem_bytes(planes, stages);
+    const void* fn = planes == 1 ? reinterpret_cast<const void*>(int_gemm_kernel<1>)
+                     : planes == 2 ? reinterpret_cast<const void*>(int_gemm_kernel<2>)
+                                   : reinterpret_cast<const void*>(int_gemm_kernel<3>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+    if (planes == 1) int_gemm_kernel<1><<<grid, kIgThreads, smem, s>>>(b);
+    else if (planes == 2) int_gemm_kernel<2><<<grid, kIgThreads, smem, s>>>(b);
+    else int_gemm_kernel<3><<<grid, kIgThreads, smem, s>>>(b);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+unsigned int int_gemm_timeouts() {
+  unsigned int v = 0;
+  cudaMemcpyFromSymbol(&v, g_ig_timeouts, sizeof v);
+  return v;
+}
+
+}  // namespace intlora

@@ -883,7 +883,77 @@ const char* intlora_last_error(void) { return g_last_error; }
 int intlora_version(void) { return 100; }
 
 uint32_t intlora_device_timeouts(void) {
-  return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts();
+  return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts() +
+         intlora::int_gemm_timeouts();
+}
+
+int32_t intlora_int_planes(int64_t max_abs) {
+  if (max_abs < 0) return 0;
+  for (int32_t p = 1; p <= 3; ++p)
+    if (max_abs <= (int64_t{1} << (7 * p)) - 1) return p;
+  return 0;
+}
+
+intlora_status intlora_int_pack(const void* q, int32_t q_bytes, int64_t d, int64_t n, int32_t planes,
+                                int8_t* packed, int32_t* overflow, void* stream) {
+  g_last_error[0] = '\0';
+  if (q_bytes != 1 && q_bytes != 2 && q_bytes != 4)
+    return fail(INTLORA_ERR_INVALID_ARG, "q_bytes must be 1, 2 or 4");
+  if (planes < 1 || planes > 3) return fail(INTLORA_ERR_INVALID_ARG, "planes must be 1, 2 or 3");
+  if (d < 0 || n < 0 || n % 16 != 0) return fail(INTLORA_ERR_INVALID_ARG, "d >= 0, n >= 0 and n % 16 == 0 required");
+  if (n > 0 && d > kMaxElements / n) return fail(INTLORA_ERR_INVALID_ARG, "d*n exceeds 2^40");
+  if (d * n == 0) return INTLORA_OK;
+  if (q == nullptr || packed == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "q and packed are required");
+  if (!aligned16(packed)) return fail(INTLORA_ERR_INVALID_ARG, "packed must be 16-byte aligned");
+  const cudaError_t e = launch_int_pack(q, q_bytes, d, n, planes, packed, overflow, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INTLORA_OK : cuda_fail(e, "int pack launch");
+}
+
+intlora_status intlora_int_gemm_batched(const intlora_int_gemm_job* jobs, int32_t count, int32_t planes,
+                                        void* stream) {
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  if (planes < 1 || planes > 3) return fail(INTLORA_ERR_INVALID_ARG, "planes must be 1, 2 or 3");
+  std::vector<IntGemmJob> work;
+  std::vector<int32_t> zero_jobs;
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_int_gemm_job& j = jobs[k];
+    if (j.tokens < 0 || j.d < 0 || j.n < 0 || j.n % 16 != 0)
+      return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: tokens, d, n >= 0 and n %% 16 == 0 required", k);
+    if (j.tokens > (int64_t{1} << 31) || j.d * planes > (int64_t{1} << 31) || j.n > (int64_t{1} << 31))
+      return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: tokens, d * planes, n must be <= 2^31", k);
+    if (j.tokens == 0 || j.d == 0) continue;
+    if (j.Y == nullptr || !aligned16(j.Y))
+      return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: Y is required, 16-byte aligned", k);
+    if (j.n == 0) {
+      zero_jobs.push_back(k);
+      continue;
+    }
+    if (j.X == nullptr || j.W == nullptr || j.x_scale == nullptr || j.w_scale == nullptr)
+      return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: X, x_scale, W, w_scale are required", k);
+    if (!aligned16(j.X) || !aligned16(j.W))
+      return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: X and W must be 16-byte aligned", k);
+    work.push_back(IntGemmJob{j.X, j.x_scale, j.W, j.w_scale, j.tokens, j.d, j.n, j.Y});
+  }
+  if (!work.empty() && !int_gemm_supported())
+    return fail(INTLORA_ERR_UNSUPPORTED, "int GEMM: the driver's tensor-map encoder is unavailable");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t k : zero_jobs) {
+    const cudaError_t e = launch_zero(jobs[k].Y, jobs[k].tokens * jobs[k].d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "int GEMM zero fill");
+  }
+  if (!work.empty()) {
+    const cudaError_t e = launch_int_gemm(work.data(), static_cast<int>(work.size()), planes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "int GEMM launch");
+  }
+  return INTLORA_OK;
+}
+
+intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int8_t* W, const float* w_scale,
+                                int64_t tokens, int64_t d, int64_t n, int32_t planes, float* Y, void* stream) {
+  intlora_int_gemm_job j{X, x_scale, W, w_scale, tokens, d, n, Y};
+  return intlora_int_gemm_batched(&j, 1, planes, stream);
 }
 
 int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bits) {

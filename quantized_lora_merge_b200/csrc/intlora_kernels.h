@@ -217,6 +217,23 @@ cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s);
 unsigned int t_gemm_timeouts();
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 
+// Integer inference GEMM on merged weights (tcgen05 kind::i8): Y = diag(x_scale)
+// X Q^T diag(w_scale) with Q held as base-128 int8 digit planes [d][P][n].
+struct IntGemmJob {
+  const int8_t* X;           // tokens x n, 16-byte aligned, n % 16 == 0
+  const float* x_scale;      // [tokens]
+  const int8_t* W;           // [d][planes][n] digit planes, 16-byte aligned
+  const float* w_scale;      // [d]
+  int64_t tokens, d, n;
+  float* Y;                  // tokens x d
+};
+int int_gemm_chans(int planes);          // output channels per tile: 256 / 128 / 64
+bool int_gemm_supported();
+cudaError_t launch_int_pack(const void* w, int w_bytes, int64_t d, int64_t n, int planes, int8_t* out,
+                            int32_t* overflow, cudaStream_t s);
+cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaStream_t s);
+unsigned int int_gemm_timeouts();
+
 // Sets the calling thread's intlora_last_error() message.
 void set_last_error(const char* message);
 

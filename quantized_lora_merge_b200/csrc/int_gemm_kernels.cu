@@ -19,7 +19,10 @@
 // warp 0 issues the TMA loads, warp 1 the MMAs, warps 4-11 drain the
 // double-buffered accumulator (tcgen05.ld; two warps per 32-lane TMEM
 // quarter, each taking half of the tile's channels), add the planes exactly
-// in 64-bit integers and scale in fp32. The integer part is exact; the only roundings
+// in 64-bit integers, scale in fp32 and hand each 32-row x 16-channel block
+// of Y to a TMA store through a double-buffered shared-memory stage (64-byte
+// swizzle, so the row-per-lane writes are free of bank conflicts and the
+// global writes are whole lines instead of 32 scattered rows). The integer part is exact; the only roundings
 // are the int -> fp32 conversion, the scale product and the final multiply.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -45,6 +48,8 @@ constexpr int kIgMaxN = 256;                    // digit rows per tile (N)
 constexpr int kIgK = 128;                       // K bytes per stage (one swizzle row)
 constexpr uint32_t kIgABytes = kIgRows * kIgK;  // 16 KB
 constexpr int kMaxIgJobs = 48;
+constexpr uint32_t kIgYBox = 32 * 16 * 4;        // one Y block: 32 rows x 16 fp32
+constexpr uint32_t kIgYStage = 8 * 2 * kIgYBox;  // 8 epilogue warps x 2 buffers
 
 __device__ unsigned int g_ig_timeouts;
 
@@ -55,11 +60,12 @@ __device__ __forceinline__ bool wait_ig(uint64_t* bar, uint32_t parity, volatile
 struct alignas(64) IgJob {
   CUtensorMap x_map;          // {n, tokens} int8, box {128, 128}
   CUtensorMap w_map;          // {n, d P} int8, box {128, C P}
+  CUtensorMap y_map;          // {d, tokens} fp32, box {16, 32}, 64-byte swizzle (when y_tma)
   const float* x_scale;
   const float* w_scale;
   float* Y;
   int64_t tokens, d, n;
-  int32_t m_tiles, n_tiles, k_stages, pad;
+  int32_t m_tiles, n_tiles, k_stages, y_tma;
   int64_t tile_begin;
 };
 struct IgBatch {
@@ -104,14 +110,18 @@ __device__ __forceinline__ uint32_t ig_idesc(int nrows) {
          (static_cast<uint32_t>(kIgRows >> 4) << 24);
 }
 
+// One 16-channel block of a tile for the calling warp's 32 rows (t = this
+// lane's row). ystage: the warp's shared-memory buffer for a TMA store, or
+// nullptr for direct stores.
 template <int P>
 __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J, int64_t t, float xs,
-                                                  int64_t i, bool row_ok) {
+                                                  int64_t i, bool row_ok, uint8_t* ystage, int lane) {
   float raw[16 * P];
 #pragma unroll
   for (int q = 0; q < P; ++q) tmem_ld16(taddr + static_cast<uint32_t>(16 * q), raw + 16 * q);
   tmem_ld_wait();
-  if (!row_ok || i >= J.d) return;
+  if (i >= J.d) return;                                  // warp-uniform
+  if (ystage == nullptr ? !row_ok : t - lane >= J.tokens) return;   // no row of the block in Y
   float y[16];
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
@@ -142,6 +152,27 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
   }
 #pragma unroll
   for (int c = 0; c < 16; ++c) y[c] *= xs * ws[c];
+  if (ystage != nullptr) {
+    // the buffer's previous store (two blocks ago) has finished reading it
+    if (lane == 0) bulk_wait_read<1>();
+    __syncwarp();
+    // row `lane`, 16-byte unit q at lane * 64 + 16 (q ^ ((lane >> 1) & 3))
+    const uint32_t row = smem_u32(ystage) + static_cast<uint32_t>(lane) * 64u;
+    const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                   ::"r"(row + 16u * (static_cast<uint32_t>(q) ^ sw)), "f"(y[4 * q]), "f"(y[4 * q + 1]),
+                     "f"(y[4 * q + 2]), "f"(y[4 * q + 3])
+                   : "memory");
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&J.y_map, ystage, static_cast<int32_t>(i), static_cast<int32_t>(t - lane));
+      bulk_commit();
+    }
+    return;
+  }
   float* dst = J.Y + t * J.d + i;
   if (i + 16 <= J.d && (J.d & 3) == 0) {
 #pragma unroll
@@ -164,7 +195,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
   const int nrows = P * b.chans;                        // digit rows of a tile
   const uint32_t b_bytes = static_cast<uint32_t>(nrows) * kIgK;
   const uint32_t stage_bytes = kIgABytes + b_bytes;     // multiple of 1024
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * stage_bytes);
+  uint8_t* ystage = base + S * stage_bytes;              // [8 warps][2][32 x 16 fp32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ystage + kIgYStage);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* d_full = bars + 2 * S;                      // [2]
@@ -264,7 +296,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
     const int half = (warp - 4) >> 2;                     // channel half of the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int buf = 0;
-    uint32_t bph = 0;
+    uint32_t bph = 0, nstore = 0;
+    uint8_t* my_stage = ystage + (warp - 4) * 2 * kIgYBox;
     for (int64_t u = blockIdx.x; u < b.total_tiles && !abort_flag; u += gridDim.x) {
       const IgTile x = ig_tile(b, u);
       const IgJob& J = b.job[x.job];
@@ -275,8 +308,10 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
       tc_fence_after();
       const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(buf * kIgMaxN);
       const int cbeg = half * (b.chans >> 1), cend = cbeg + (b.chans >> 1);
-      for (int c0 = cbeg; c0 < cend; c0 += 16)
-        ig_epilogue_chunk<P>(tb + static_cast<uint32_t>(c0 * P), J, t, xs, x.i0 + c0, row_ok);
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
+        uint8_t* ys = J.y_tma ? my_stage + (nstore++ & 1u) * kIgYBox : nullptr;
+        ig_epilogue_chunk<P>(tb + static_cast<uint32_t>(c0 * P), J, t, xs, x.i0 + c0, row_ok, ys, lane);
+      }
       tc_fence_before();
       mbar_arrive(&d_empty[buf]);
       if (++buf == 2) {
@@ -286,6 +321,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
     }
   }
 
+  if (warp >= 4 && lane == 0) bulk_wait<0>();           // this warp's Y stores are done
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -300,7 +336,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
 
 size_t ig_smem_bytes(int planes, int stages) {
   const size_t stage = kIgABytes + static_cast<size_t>(planes * int_gemm_chans(planes)) * kIgK;
-  return 1024 + static_cast<size_t>(stages) * stage + (2 * stages + 4) * 8;
+  return 1024 + static_cast<size_t>(stages) * stage + kIgYStage + (2 * stages + 4) * 8;
 }
 
 // ---- digit planes ----------------------------------------------------------------
@@ -358,6 +394,10 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
           tc::encode_2d(&t.x_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.X, j.tokens, j.n, kIgK, kIgRows) &&
           tc::encode_2d(&t.w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.W, j.d * planes, j.n, kIgK, chans * planes);
       if (!ok) return cudaErrorInvalidValue;
+      // Y through TMA stores when its rows are 16-byte multiples
+      t.y_tma = (j.d % 4 == 0) &&
+                tc::encode_2d_swz(&t.y_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.Y, j.tokens, j.d, 16, 32,
+                                  CU_TENSOR_MAP_SWIZZLE_64B) ? 1 : 0;
       t.x_scale = j.x_scale;
       t.w_scale = j.w_scale;
       t.Y = j.Y;

@@ -1,5 +1,5 @@
 // Shared PTX building blocks of the tensor-core kernels (sm_100a): mbarriers
-// with bounded waits, TMA tile loads, tcgen05 MMA / commit / fences / TMEM
+// with bounded waits, TMA tile loads and stores, tcgen05 MMA / commit / fences / TMEM
 // loads, shared-memory matrix descriptors, and the host-side tensor-map
 // encoder (through the driver entry point, so no libcuda link is needed).
 #pragma once
@@ -70,6 +70,26 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+// Tile store from shared memory (bulk-group completion) and its bookkeeping.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// at most N of this thread's bulk groups still reading shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// generic-proxy shared-memory writes made visible to the async (TMA) proxy
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
@@ -138,10 +158,12 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Row-major rows x cols matrix of `dtype` (element size esize bytes), box
-// {box_cols, box_rows} with the 128-byte swizzle (box_cols x esize must be
-// 128), zero fill outside the matrix.
-inline bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* ptr,
-                      int64_t rows, int64_t cols, int box_cols, int box_rows) {
+// {box_cols, box_rows} with the given swizzle (box_cols x esize must not
+// exceed the swizzle span), zero fill outside the matrix on loads, clipping
+// on stores.
+inline bool encode_2d_swz(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* ptr,
+                          int64_t rows, int64_t cols, int box_cols, int box_rows,
+                          CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -149,8 +171,13 @@ inline bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, co
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   return fn(map, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// The same with the 128-byte swizzle (box_cols x esize must be 128): the
+// operand layout of the tcgen05 K-major descriptors.
+inline bool encode_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* ptr,
+                      int64_t rows, int64_t cols, int box_cols, int box_rows) {
+  return encode_2d_swz(map, dtype, esize, ptr, rows, cols, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace tc

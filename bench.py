@@ -121,19 +121,19 @@ NUM_SMS = 148
 DOMINANT_SOURCES = ("team_kernels.cu", "intlora_device.cuh", "intlora_kernels.h")
 
 
-def csrc_hash():
+def csrc_hash(sources=None):
     """Hash of the dominant kernel's CUDA sources, so a stored ncu traffic
     figure is only used while the kernel it was taken on is unchanged."""
     import hashlib
     h = hashlib.sha256()
     root = Path(__file__).resolve().parent / "quantized_lora_merge_b200" / "csrc"
-    for name in DOMINANT_SOURCES:
+    for name in (sources or DOMINANT_SOURCES):
         h.update(name.encode())
         h.update((root / name).read_bytes())
     return h.hexdigest()
 
 
-def profiled_traffic(name):
+def profiled_traffic(name, sources=None):
     """dram__bytes_read.sum + dram__bytes_write.sum per launch from the ncu
     summary profiles/<name>.md, or None when absent or when the kernels have
     changed since it was taken."""
@@ -145,7 +145,7 @@ def profiled_traffic(name):
         if ":" in line:
             k, v = line.split(":", 1)
             fields[k.strip().strip("-* `")] = v.strip().strip("` ")
-    if fields.get("csrc_sha256") != csrc_hash():
+    if fields.get("csrc_sha256") != csrc_hash(sources):
         return None
     try:
         return float(fields["dram_bytes_per_launch"])
@@ -516,6 +516,7 @@ GEMM_UNIT = "Top/s"
 # DiT-3072 block linears (qkv, attention out, fc1, fc2) as (d, n)
 GEMM_SHAPES = [(9216, 3072), (3072, 3072), (12288, 3072), (3072, 12288)]
 GEMM_KIND = {1: "shift4", 2: "mul4", 3: "mul8"}
+GEMM_SOURCES = ("int_gemm_kernels.cu", "tcgen05_util.cuh", "intlora_kernels.h")
 
 
 def bf16_peak_tflops():
@@ -618,7 +619,9 @@ def bench_int_gemm(args):
                      "frac": achieved / peak,
                      "peak_source": f"2 x {kind} bf16 dense {bf16:.0f} TFLOP/s (int8/bf16 "
                                     f"nominal ratio 4.5/2.25)",
-                     "traffic": None},
+                     "traffic": profiled_traffic(f"int_gemm_kernel_dit_{GEMM_KIND[P]}",
+                                                 GEMM_SOURCES),
+                     "traffic_unit": "bytes per launch (one step)"},
         "clocks": clk, "gpu_launches": steps,
         "e2e": {"value": tensor_ops / (e2e_ms / 1e3) / 1e12, "unit": GEMM_UNIT,
                 "ms_per_step": e2e_ms,

@@ -74,6 +74,11 @@ def _load():
         "orc_ste_backward": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _ptr]),
         "orc_ste_sampled": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _i64, _ptr, _i64,
                                    _ptr, _ptr]),
+        "orc_quantize_rows": (None, [_ptr, _i64, _u64, _u32, _dbl, _int, _i64, _i64, _ptr, _ptr,
+                                     _ptr, _ptr, _ptr]),
+        "orc_merge_mul_rows": (None, [_ptr, _i64, _ptr, _ptr, _ptr, _ptr, _i64, _int, _u64, _u32,
+                                      _dbl, _int, _i64, _i64, _ptr, _ptr, _ptr, _ptr, _ptr,
+                                      _ptr]),
         "orc_int_digits": (_i64, [_ptr, _i64, _i64, _int, _ptr]),
         "orc_int_gemm_rows": (None, [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_num_threads": (_int, []),
@@ -189,6 +194,23 @@ def gen_aux(W, seed: int, stream_id: int, alpha: float, w_bits: int, row_begin: 
                 codes=codes, s=s, z=z, pre=pre, zpre=zpre)
 
 
+def quantize_rows(W_rows, seed: int, stream_id: int, c: float, w_bits: int,
+                  row_begin: int) -> dict:
+    """Base quantization of rows [row_begin, row_begin + len(W_rows)) of a layer
+    from those rows of W alone, with the VMC factor c given (layers too large
+    to hold or reduce on the host)."""
+    w = _c(W_rows, np.float32)
+    rc, n = w.shape
+    codes = np.zeros((rc, n), np.int32)
+    s = np.zeros(rc, np.float64)
+    z = np.zeros(rc, np.int32)
+    pre = np.zeros((rc, n), np.float64)
+    zpre = np.zeros(rc, np.float64)
+    _load().orc_quantize_rows(_p(w), n, seed, stream_id, c, w_bits, row_begin, rc, _p(codes),
+                              _p(s), _p(z), _p(pre), _p(zpre))
+    return dict(codes=codes, s=s, z=z, pre=pre, zpre=zpre)
+
+
 # --------------------------------------------------------------------------
 # a4-a7: the merges
 # --------------------------------------------------------------------------
@@ -231,6 +253,29 @@ def merge_mul(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, u_bi
                           sigma_w, sigma_r_, alpha, u_bits, row_begin, rc, _p(U), _p(ur),
                           _p(sbar), _p(zbar), _p(P), _p(pre), _p(zpre))
     return dict(U=U, u_round=ur, sbar=sbar, zbar=zbar, P=P, pre=pre, zpre=zpre)
+
+
+def merge_mul_rows(codes_rows, s_rows, z_rows, A_rows, B, seed, stream_id, c, u_bits,
+                   row_begin) -> dict:
+    """MUL merge of rows [row_begin, row_begin + len(codes_rows)) from those
+    rows' inputs alone, with the VMC factor c given."""
+    cd = _c(codes_rows, np.int32)
+    sf = _c(s_rows, np.float32)
+    zi = _c(z_rows, np.int32)
+    Af = _c(A_rows, np.float32)
+    Bf = _c(B, np.float32)
+    rc, n = cd.shape
+    r = Af.shape[1]
+    ur = np.zeros((rc, n), np.int32)
+    sbar = np.zeros(rc, np.float64)
+    zbar = np.zeros(rc, np.int32)
+    P = np.zeros((rc, n), np.int64)
+    pre = np.zeros((rc, n), np.float64)
+    zpre = np.zeros(rc, np.float64)
+    _load().orc_merge_mul_rows(_p(cd), n, _p(sf), _p(zi), _p(Af), _p(Bf), n, r, seed, stream_id,
+                               c, u_bits, row_begin, rc, _p(ur), _p(sbar), _p(zbar), _p(P),
+                               _p(pre), _p(zpre))
+    return dict(u_round=ur, sbar=sbar, zbar=zbar, P=P, pre=pre, zpre=zpre)
 
 
 def shift_quantize_row(U, D, shift_bits: int) -> dict:

@@ -244,6 +244,21 @@ void orc_affine_quantize_row(const double* x, int64_t n, int bits, double* scale
 /* for those rows (row-major, row_count x n). sigma values cover the whole   */
 /* d x n layer.                                                              */
 /* ------------------------------------------------------------------------ */
+/* One row i of the base quantization: X_j = W_ij - c R_ij (flat index
+ * e = i n + j), then the affine quantizer of the row. */
+static void quantize_row(const float* W_row, int64_t n, uint64_t seed, uint32_t stream_id, double c,
+                         int w_bits, int64_t i, double* r_star_row, int32_t* codes_row,
+                         double* s_out, int32_t* z_out, double* pre_row, double* zpre) {
+    double* x = (double*)malloc(sizeof(double) * (size_t)n);
+    for (int64_t j = 0; j < n; ++j) {
+        double r_star = c * orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
+        if (r_star_row) r_star_row[j] = r_star;
+        x[j] = (double)W_row[j] - r_star;
+    }
+    orc_affine_quantize_row(x, n, w_bits, s_out, z_out, codes_row, pre_row, zpre);
+    free(x);
+}
+
 void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t stream_id,
                  double alpha, int w_bits, int64_t row_begin, int64_t row_count,
                  double* sigma_w_out, double* sigma_r_out, double* c_out,
@@ -256,18 +271,23 @@ void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t s
     *sigma_r_out = sigma_r;
     *c_out = c;
 #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t t = 0; t < row_count; ++t) {
-        int64_t i = row_begin + t;
-        double* x = (double*)malloc(sizeof(double) * (size_t)n);
-        for (int64_t j = 0; j < n; ++j) {
-            double r_star = c * orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
-            if (r_star_out) r_star_out[t * n + j] = r_star;
-            x[j] = (double)W[i * n + j] - r_star;
-        }
-        orc_affine_quantize_row(x, n, w_bits, &s_out[t], &z_out[t], &codes[t * n],
-                                pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
-        free(x);
-    }
+    for (int64_t t = 0; t < row_count; ++t)
+        quantize_row(&W[(row_begin + t) * n], n, seed, stream_id, c, w_bits, row_begin + t,
+                     r_star_out ? &r_star_out[t * n] : NULL, &codes[t * n], &s_out[t], &z_out[t],
+                     pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
+}
+
+/* The same row quantization for rows whose W is given alone (W_rows holds
+ * rows [row_begin, row_begin + row_count) of the layer) and whose VMC factor
+ * c is given: layers too large to hold or reduce on the host. */
+void orc_quantize_rows(const float* W_rows, int64_t n, uint64_t seed, uint32_t stream_id, double c,
+                       int w_bits, int64_t row_begin, int64_t row_count, int32_t* codes,
+                       double* s_out, int32_t* z_out, double* pre, double* zpre) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < row_count; ++t)
+        quantize_row(&W_rows[t * n], n, seed, stream_id, c, w_bits, row_begin + t, NULL,
+                     &codes[t * n], &s_out[t], &z_out[t], pre ? &pre[t * n] : NULL,
+                     zpre ? &zpre[t] : NULL);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -276,15 +296,15 @@ void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t s
 /* with the quotient taken as 0 where W_round - z = 0. Computes U and the    */
 /* integer term D = W_round - z for one row i.                               */
 /* ------------------------------------------------------------------------ */
-static void adaptation_row(const int32_t* codes, int64_t ld_codes, const float* s, const int32_t* z,
-                           const float* A, const float* B, int64_t n, int r, uint64_t seed,
-                           uint32_t stream_id, double c, int64_t i, double* U, int64_t* D) {
-    double s_i = (double)s[i];
+static void adaptation_row(const int32_t* codes_row, float s_i32, int32_t z_i, const float* A_row,
+                           const float* B, int64_t n, int r, uint64_t seed, uint32_t stream_id,
+                           double c, int64_t i, double* U, int64_t* D) {
+    double s_i = (double)s_i32;
     for (int64_t j = 0; j < n; ++j) {
         double r_star = c * orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
         double ab = 0.0;
-        for (int k = 0; k < r; ++k) ab += (double)A[i * r + k] * (double)B[(int64_t)k * n + j];
-        int64_t dij = (int64_t)codes[i * ld_codes + j] - (int64_t)z[i];
+        for (int k = 0; k < r; ++k) ab += (double)A_row[k] * (double)B[(int64_t)k * n + j];
+        int64_t dij = (int64_t)codes_row[j] - (int64_t)z_i;
         D[j] = dij;
         U[j] = (dij != 0) ? s_i + (r_star + ab) / (double)dij : s_i;
     }
@@ -300,7 +320,8 @@ void orc_mla_rows(const int32_t* codes, int64_t ld_codes, const float* s, const 
     double c = orc_vmc_scale(sigma_w, sigma_r, alpha);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < row_count; ++t)
-        adaptation_row(codes, ld_codes, s, z, A, B, n, r, seed, stream_id, c, row_begin + t,
+        adaptation_row(&codes[(row_begin + t) * ld_codes], s[row_begin + t], z[row_begin + t],
+                       &A[(row_begin + t) * r], B, n, r, seed, stream_id, c, row_begin + t,
                        &U_out[t * n], &D_out[t * n]);
 }
 
@@ -311,6 +332,12 @@ void orc_mla_rows(const int32_t* codes, int64_t ld_codes, const float* s, const 
 /*   W' = s_bar * (U_round - z_bar) * (W_round - z), kept as the integer     */
 /*   product P = (U_round - z_bar) * D and the per-row scale s_bar.          */
 /* ------------------------------------------------------------------------ */
+void orc_merge_mul_rows(const int32_t* codes_rows, int64_t ld_codes, const float* s_rows,
+                        const int32_t* z_rows, const float* A_rows, const float* B, int64_t n,
+                        int r, uint64_t seed, uint32_t stream_id, double c, int u_bits,
+                        int64_t row_begin, int64_t row_count, int32_t* u_round, double* sbar,
+                        int32_t* zbar, int64_t* P, double* pre, double* zpre);
+
 void orc_merge_mul(const int32_t* codes, int64_t ld_codes, const float* s, const int32_t* z,
                    const float* A, const float* B, int64_t d, int64_t n, int r, uint64_t seed,
                    uint32_t stream_id, double sigma_w, double sigma_r, double alpha, int u_bits,
@@ -323,13 +350,37 @@ void orc_merge_mul(const int32_t* codes, int64_t ld_codes, const float* s, const
         int64_t i = row_begin + t;
         double* U = (double*)malloc(sizeof(double) * (size_t)n);
         int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
-        adaptation_row(codes, ld_codes, s, z, A, B, n, r, seed, stream_id, c, i, U, D);
+        adaptation_row(&codes[i * ld_codes], s[i], z[i], &A[i * r], B, n, r, seed, stream_id, c, i,
+                       U, D);
         orc_affine_quantize_row(U, n, u_bits, &sbar[t], &zbar[t], &u_round[t * n],
                                 pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
         for (int64_t j = 0; j < n; ++j) {
             if (U_out) U_out[t * n + j] = U[j];
             P[t * n + j] = ((int64_t)u_round[t * n + j] - (int64_t)zbar[t]) * D[j];
         }
+        free(U);
+        free(D);
+    }
+}
+
+/* The MUL merge of rows whose inputs are given alone (codes_rows, s_rows,
+ * z_rows, A_rows hold rows [row_begin, row_begin + row_count) of the layer)
+ * and whose VMC factor c is given: layers too large for the host. */
+void orc_merge_mul_rows(const int32_t* codes_rows, int64_t ld_codes, const float* s_rows,
+                        const int32_t* z_rows, const float* A_rows, const float* B, int64_t n,
+                        int r, uint64_t seed, uint32_t stream_id, double c, int u_bits,
+                        int64_t row_begin, int64_t row_count, int32_t* u_round, double* sbar,
+                        int32_t* zbar, int64_t* P, double* pre, double* zpre) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < row_count; ++t) {
+        double* U = (double*)malloc(sizeof(double) * (size_t)n);
+        int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
+        adaptation_row(&codes_rows[t * ld_codes], s_rows[t], z_rows[t], &A_rows[t * r], B, n, r,
+                       seed, stream_id, c, row_begin + t, U, D);
+        orc_affine_quantize_row(U, n, u_bits, &sbar[t], &zbar[t], &u_round[t * n],
+                                pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
+        for (int64_t j = 0; j < n; ++j)
+            P[t * n + j] = ((int64_t)u_round[t * n + j] - (int64_t)zbar[t]) * D[j];
         free(U);
         free(D);
     }
@@ -379,7 +430,8 @@ void orc_merge_shift(const int32_t* codes, int64_t ld_codes, const float* s, con
         int64_t i = row_begin + t;
         double* U = (double*)malloc(sizeof(double) * (size_t)n);
         int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
-        adaptation_row(codes, ld_codes, s, z, A, B, n, r, seed, stream_id, c, i, U, D);
+        adaptation_row(&codes[i * ld_codes], s[i], z[i], &A[i * r], B, n, r, seed, stream_id, c, i,
+                       U, D);
         orc_shift_quantize_row(U, D, n, shift_bits, &sbar[t], &shift[t * n], &M[t * n],
                                pre ? &pre[t * n] : NULL);
         if (U_out)

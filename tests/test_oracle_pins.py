@@ -484,3 +484,20 @@ def test_int_gemm_is_the_dequantized_matmul_of_merged_weights():
     assert bad == 0
     acc = sum(128**k * (X.astype(np.int64) @ dig[:, k, :].astype(np.int64).T) for k in range(planes))
     np.testing.assert_allclose(Y, acc * xs[:, None] * sbar[None, :], rtol=1e-15, atol=0)
+
+
+def test_row_views_equal_whole_layer_functions():
+    """quantize_rows / merge_mul_rows (rows given alone, c given) reproduce the
+    pinned whole-layer functions on a slice of rows, flat index included."""
+    spec, W, A, B, g = _prepared(21, 36, 4, 4, sid=13)
+    rows = slice(7, 15)
+    q = oracle.quantize_rows(W[rows], spec.seed, 13, g["c"], 4, 7)
+    for k in ("codes", "s", "z", "pre", "zpre"):
+        np.testing.assert_array_equal(q[k], g[k][rows])
+    s32 = g["s"].astype(np.float32)
+    m = oracle.merge_mul(g["codes"], s32, g["z"], A, B, spec.seed, 13, g["sigma_w"], g["sigma_r"],
+                         spec.alpha, 4)
+    mr = oracle.merge_mul_rows(g["codes"][rows], s32[rows], g["z"][rows], A[rows], B, spec.seed,
+                               13, g["c"], 4, 7)
+    for k in ("u_round", "sbar", "zbar", "P", "pre", "zpre"):
+        np.testing.assert_array_equal(mr[k], m[k][rows])

@@ -191,3 +191,84 @@ def test_rank_sweep_full_size(r):
         _verify_merge(spec, st, inp)
     del mstates, inps
     _run_and_verify_ste(specs)
+
+
+# ---------------------------------------------------------------------------
+# maximum size: a layer past 2^34 elements, where the Philox block index
+# e / 4 needs the counter's high word (rows from 2^20 on, at n = 16384)
+# ---------------------------------------------------------------------------
+HUGE_D, HUGE_N = 2**20 + 1, 16384           # 2^34 + 16384 elements
+
+
+def _huge_rows():
+    return [0, 12345, 2**19, 2**20 - 1, 2**20]   # the last row lies wholly past 2^34
+
+
+def test_layer_beyond_2_34_elements():
+    dev = _dev()
+    if torch.cuda.mem_get_info(dev)[0] < 90 * 2**30:
+        pytest.skip("needs ~80 GB of free device memory")
+    d, n = HUGE_D, HUGE_N
+    assert d * n > 2**34
+    # preparation with alpha = 0 (c = 1, no sigma needed on the host): W is a
+    # seeded device draw; the sampled rows go to the oracle
+    spec = wl.LayerSpec("huge", d, n, 4, 4, "mul", 4, alpha=0.0, stream_id=77)
+    g = torch.Generator(device=dev)
+    g.manual_seed(2026)
+    W = torch.randn(d, n, generator=g, device=dev).mul_(wl.W_STD)
+    sigma = torch.zeros(2, dtype=torch.float64, device=dev)
+    w_round = torch.zeros(d, P.code_row_bytes(n, 4), dtype=torch.uint8, device=dev)
+    s_d = torch.zeros(d, dtype=torch.float32, device=dev)
+    z_d = torch.zeros(d, dtype=torch.int32, device=dev)
+    job = B.AuxJob(W, spec.seed, spec.stream_id, spec.alpha, 4, sigma[0:1], sigma[1:2], None,
+                   w_round, s_d, z_d)
+    ws = P.workspace(B.intlora_gen_aux_workspace_size([job]), dev)
+    B.intlora_gen_aux_batched([job], ws)
+    torch.cuda.synchronize()
+    rows = _huge_rows()
+    idx = torch.tensor(rows, device=dev)
+    W_rows = W[idx].cpu().numpy()
+    codes = wl.unpack_codes(w_round[idx].cpu().numpy(), n, 4)
+    s, z = s_d[idx].cpu().numpy(), z_d[idx].cpu().numpy()
+    sig = sigma.cpu().numpy()
+    assert np.all(np.isfinite(sig)) and np.all(sig > 0)
+    del W, w_round, s_d, z_d, job, ws
+    torch.cuda.empty_cache()
+    for k, i in enumerate(rows):
+        o = oracle.quantize_rows(W_rows[k:k + 1], spec.seed, spec.stream_id, 1.0, 4, i)
+        assert_scale("s", s[k:k + 1], o["s"])
+        assert_affine(f"W_round row {i}", codes[k:k + 1], z[k:k + 1], o["codes"], o["z"], o["pre"],
+                      o["zpre"], 15)
+
+    # MUL merge with alpha = 1.5 on a seeded synthetic prepared layer
+    mspec = wl.LayerSpec("huge", d, n, 4, 4, "mul", 4, alpha=1.5, stream_id=78)
+    A = torch.randn(d, 4, generator=g, device=dev).mul_(wl.AB_STD)
+    Bm = torch.randn(4, n, generator=g, device=dev).mul_(wl.AB_STD)
+    st = P.allocate(mspec, None, A, Bm, dev, want_code=True)
+    st.w_round.copy_(torch.randint(0, 256, st.w_round.shape, generator=g, device=dev,
+                                   dtype=torch.uint8))
+    st.s.copy_(torch.empty(d, device=dev).uniform_(0.5, 1.5, generator=g) * (0.08 / 15))
+    st.z.copy_(torch.randint(4, 12, (d,), generator=g, device=dev, dtype=torch.int32))
+    sw, sr = 0.02, 1.4142
+    st.sigma.copy_(torch.tensor([sw, sr], dtype=torch.float64))
+    layers, outs = [st.layer()], [st.merge_out()]
+    mws = P.workspace(B.intlora_merge_workspace_size(layers), dev)
+    B.intlora_merge_mul_batched(layers, outs, 4, mws)
+    torch.cuda.synchronize()
+    c = oracle.vmc_scale(sw, sr, 1.5)
+    in_codes = wl.unpack_codes(st.w_round[idx].cpu().numpy(), n, 4)
+    in_s, in_z = st.s[idx].cpu().numpy(), st.z[idx].cpu().numpy()
+    A_rows, B_h = A[idx].cpu().numpy(), Bm.cpu().numpy()
+    out = st.out[idx].cpu().numpy().astype(np.int64)
+    code = st.code[idx].cpu().numpy()
+    sbar, zbar = st.sbar[idx].cpu().numpy(), st.zbar[idx].cpu().numpy()
+    del st, mws, A, Bm
+    torch.cuda.empty_cache()
+    for k, i in enumerate(rows):
+        o = oracle.merge_mul_rows(in_codes[k:k + 1], in_s[k:k + 1], in_z[k:k + 1], A_rows[k:k + 1],
+                                  B_h, mspec.seed, mspec.stream_id, c, 4, i)
+        assert_scale("s_bar", sbar[k:k + 1], o["sbar"])
+        assert_affine(f"U_round row {i}", code[k:k + 1], zbar[k:k + 1], o["u_round"], o["zbar"],
+                      o["pre"], o["zpre"], 15)
+        D = in_codes[k].astype(np.int64) - in_z[k]
+        assert np.array_equal(out[k], (code[k].astype(np.int64) - zbar[k]) * D)

@@ -40,6 +40,59 @@ __device__ __forceinline__ uint4 philox10(uint32_t c0, uint32_t c1, uint32_t c2,
   return make_uint4(c0, c1, c2, c3);
 }
 
+// Philox4x32-10 for counters (c0, 0, sid, 0) under a fixed key and stream id
+// (layers below 2^34 elements): everything that does not depend on c0 is
+// formed once per layer. Round 0 multiplies sid (the same for the whole
+// layer), so its word-0 output u0 and word-1 output u1 are constants; round 1
+// multiplies u0, so its high and low products are constants too. The round
+// keys k + r W of rounds 2-9 are formed here as well. Bit-identical to
+// philox10(c0, 0, sid, 0, k0, k1).
+struct PhiloxSmall {
+  uint32_t u0, u1;           // words 0 and 1 after round 0
+  uint32_t x1, y1, l1;       // round 1: u1 ^ key0(1), hi(M0 u0) ^ key1(1), lo(M0 u0)
+  uint32_t k1;               // key word 1 (round 0)
+  uint32_t rk0[8], rk1[8];   // round keys of rounds 2-9: k + r W
+};
+__device__ __forceinline__ PhiloxSmall philox_small_setup(uint32_t sid, uint32_t k0, uint32_t k1) {
+  PhiloxSmall p;
+  const uint64_t q = static_cast<uint64_t>(kPhiloxM1) * sid;
+  p.u0 = static_cast<uint32_t>(q >> 32) ^ k0;          // c1 = 0
+  p.u1 = static_cast<uint32_t>(q);
+  const uint64_t h = static_cast<uint64_t>(kPhiloxM0) * p.u0;
+  p.x1 = p.u1 ^ (k0 + kPhiloxW0);
+  p.y1 = static_cast<uint32_t>(h >> 32) ^ (k1 + kPhiloxW1);
+  p.l1 = static_cast<uint32_t>(h);
+  p.k1 = k1;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    p.rk0[r] = k0 + static_cast<uint32_t>(r + 2) * kPhiloxW0;
+    p.rk1[r] = k1 + static_cast<uint32_t>(r + 2) * kPhiloxW1;
+  }
+  return p;
+}
+__device__ __forceinline__ uint4 philox10_small(uint32_t c0, const PhiloxSmall& p) {
+  // round 0: word 2 from the product of c0 (c3 = 0)
+  const uint64_t a = static_cast<uint64_t>(kPhiloxM0) * c0;
+  const uint32_t c2 = static_cast<uint32_t>(a >> 32) ^ p.k1;
+  const uint32_t c3 = static_cast<uint32_t>(a);
+  // round 1: the product of word 0 (= u0) is a layer constant
+  const uint64_t b = static_cast<uint64_t>(kPhiloxM1) * c2;
+  uint32_t w0 = static_cast<uint32_t>(b >> 32) ^ p.x1;
+  uint32_t w1 = static_cast<uint32_t>(b);
+  uint32_t w2 = c3 ^ p.y1;
+  uint32_t w3 = p.l1;
+#pragma unroll
+  for (int round = 2; round < 10; ++round) {
+    const uint64_t p0 = static_cast<uint64_t>(kPhiloxM0) * w0;
+    const uint64_t p1 = static_cast<uint64_t>(kPhiloxM1) * w2;
+    w0 = static_cast<uint32_t>(p1 >> 32) ^ w1 ^ p.rk0[round - 2];
+    w2 = static_cast<uint32_t>(p0 >> 32) ^ w3 ^ p.rk1[round - 2];
+    w1 = static_cast<uint32_t>(p1);
+    w3 = static_cast<uint32_t>(p0);
+  }
+  return make_uint4(w0, w1, w2, w3);
+}
+
 // Four consecutive words of the auxiliary stream, starting at a flat index
 // that is a multiple of 4: block = e / 4, counter (block lo, block hi,
 // stream id, 0).

@@ -46,9 +46,10 @@ struct GroupSums {
 
 template <bool HAS_W, bool SMALL>
 __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, const float* wgroup,
-                                          uint64_t group, float K, int valid, uint32_t k0, uint32_t k1) {
+                                          uint64_t group, float K, int valid, uint32_t k0, uint32_t k1,
+                                          const PhiloxSmall& ph) {
   // SMALL: fewer than 2^34 elements, so the block index's high word is 0
-  const uint4 w = SMALL ? philox10(static_cast<uint32_t>(group), 0u, J.stream_id, 0u, k0, k1)
+  const uint4 w = SMALL ? philox10_small(static_cast<uint32_t>(group), ph)
                         : aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
   uint64_t r01, r23;
   if (valid == 4) {
@@ -102,12 +103,13 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int32_t count = g0 < full ? static_cast<int32_t>((full - 1 - g0) / stride + 1) : 0;
   uint64_t g = static_cast<uint64_t>(g0);
   const float* wp = HAS_W ? J.W + 4 * g0 : nullptr;
+  const PhiloxSmall ph = philox_small_setup(J.stream_id, k0, k1);
   for (int32_t k = 0; k < count;) {
     GroupSums s;
     const int32_t kend = min(count, k + kFlush);
 #pragma unroll 2
     for (; k < kend; ++k, g += stride) {
-      add_group<HAS_W, SMALL>(s, J, wp, g, K, 4, k0, k1);
+      add_group<HAS_W, SMALL>(s, J, wp, g, K, 4, k0, k1, ph);
       if (HAS_W) wp += 4 * stride;
     }
     acc[0] += f2_sum(s.w1);
@@ -118,7 +120,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
-    add_group<HAS_W, SMALL>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1);
+    add_group<HAS_W, SMALL>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1, ph);
     acc[0] += f2_sum(s.w1);
     acc[1] += f2_sum(s.w2);
     acc[2] += f2_sum(s.r1);

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
     const uint8_t* __restrict__ src = static_cast<const uint8_t*>(L.src);
     const int64_t ld_src = L.ld_src;
     const uint32_t sid = L.stream_id;
+    const PhiloxSmall ph = philox_small_setup(sid, p.key0, p.key1);
     // RANK > 0: fixed rank; 0: any rank; < 0: A B precomputed (L.T), no rank loop
     const int r = (VARIANT == kGen || RANK < 0) ? 0 : (RANK > 0 ? RANK : L.r);
 
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       for (int ml = 0; ml < kTeamRows; ++ml) {
         // layers here have fewer than 2^34 elements: the block index fits the
         // low counter word and the high word is 0 (rounds 0-1 partly uniform)
-        const uint4 w4 = philox10(ctr0[ml] + static_cast<uint32_t>(q), 0u, sid, 0u, p.key0, p.key1);
+        const uint4 w4 = philox10_small(ctr0[ml] + static_cast<uint32_t>(q), ph);
         const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
         float v[4];
 #pragma unroll

@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
     const int64_t ld_src = L.ld_src;
     const uint8_t* __restrict__ src = static_cast<const uint8_t*>(L.src);
     const uint32_t sid = L.stream_id;
+    const PhiloxSmall ph = philox_small_setup(sid, p.key0, p.key1);
     void* const out = L.out;
     uint8_t* const code_out = VARIANT == kGen ? nullptr : L.code_out;
     const int64_t ld_out = L.ld_out;
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
           uint32_t words[4];
           if (ALIGNED) {
             // layers below 2^34 elements: block index in the low counter word
-            const uint4 w4 = p.small ? philox10(static_cast<uint32_t>(blk0 + ml * nq), 0u, sid, 0u, p.key0, p.key1)
+            const uint4 w4 = p.small ? philox10_small(static_cast<uint32_t>(blk0 + ml * nq), ph)
                                      : aux_block(static_cast<uint64_t>(blk0 + ml * nq), sid, p.key0, p.key1);
             words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
           } else {

@@ -4,7 +4,8 @@
 //
 // One pass reads W (16-byte vector loads) and regenerates R (Philox + Laplace)
 // for the same elements; each CTA accumulates shifted sums in fp64 (shift K =
-// W[0] for W, 0 for R, whose mean is 0 by symmetry), writes one partial, and
+// W[0] for W, 0 for R, whose mean is 0 by symmetry; R's sums are taken of
+// R / ln 2 and scaled back when sigma is formed), writes one partial, and
 // a finalize kernel adds the partials in a fixed order, so sigma does not
 // depend on scheduling. var = (S2 - S1^2 / N) / N.
 #include <cuda_runtime.h>
@@ -19,7 +20,7 @@ namespace intlora {
 namespace {
 
 constexpr int kStatsThreads = 256;
-constexpr float kLn2f = 0.693147180559945309f;
+constexpr double kLn2d = 0.693147180559945309417232121458;
 
 __device__ __forceinline__ void block_sum4(double v[4], double* red /* [4][32] */) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -51,21 +52,23 @@ __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, const
   // SMALL: fewer than 2^34 elements, so the block index's high word is 0
   const uint4 w = SMALL ? philox10_small(static_cast<uint32_t>(group), ph)
                         : aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
-  uint64_t r01, r23;
+  // R / ln 2 = +-log2(w): the sums run in the log2 domain (the sign is a
+  // factor of +-1, R^2 needs none) and the finalize kernel scales by ln 2
   if (valid == 4) {
     const uint64_t l01 = laplace_log2_x2(w.x, w.y), l23 = laplace_log2_x2(w.z, w.w);
-    r01 = f2_mul(l01, f2_pack(laplace_sign(w.x, kLn2f), laplace_sign(w.y, kLn2f)));
-    r23 = f2_mul(l23, f2_pack(laplace_sign(w.z, kLn2f), laplace_sign(w.w, kLn2f)));
+    const uint64_t s01 = f2_pack(laplace_sign(w.x, 1.0f), laplace_sign(w.y, 1.0f));
+    const uint64_t s23 = f2_pack(laplace_sign(w.z, 1.0f), laplace_sign(w.w, 1.0f));
+    g.r1 = f2_fma(l23, s23, f2_fma(l01, s01, g.r1));
+    g.r2 = f2_fma(l23, l23, f2_fma(l01, l01, g.r2));
   } else {
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     float rv[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) rv[c] = c < valid ? laplace_scaled(words[c], kLn2f) : 0.0f;
-    r01 = f2_pack(rv[0], rv[1]);
-    r23 = f2_pack(rv[2], rv[3]);
+    for (int c = 0; c < 4; ++c) rv[c] = c < valid ? laplace_scaled(words[c], 1.0f) : 0.0f;
+    const uint64_t r01 = f2_pack(rv[0], rv[1]), r23 = f2_pack(rv[2], rv[3]);
+    g.r1 = f2_add(f2_add(g.r1, r01), r23);
+    g.r2 = f2_fma(r23, r23, f2_fma(r01, r01, g.r2));
   }
-  g.r1 = f2_add(f2_add(g.r1, r01), r23);
-  g.r2 = f2_fma(r23, r23, f2_fma(r01, r01, g.r2));
   if (HAS_W) {
     uint64_t x01, x23;                   // W - K, elements past the tail left at 0
     if (valid == 4) {
@@ -163,8 +166,8 @@ __global__ void __launch_bounds__(kStatsThreads) stats_finalize_kernel(const __g
       *J.sigma_w_out = sqrt(fmax(var, 0.0));
     }
     if (J.sigma_r_out != nullptr) {
-      const double var = (acc[3] - acc[2] * acc[2] / N) / N;
-      *J.sigma_r_out = sqrt(fmax(var, 0.0));
+      const double var = (acc[3] - acc[2] * acc[2] / N) / N;   // of R / ln 2
+      *J.sigma_r_out = kLn2d * sqrt(fmax(var, 0.0));
     }
   }
 }

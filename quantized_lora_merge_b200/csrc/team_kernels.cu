@@ -255,7 +255,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       for (int ml = 0; ml < kTeamRows; ++ml) {
         // layers here have fewer than 2^34 elements: the block index fits the
         // low counter word and the high word is 0 (rounds 0-1 partly uniform)
-        const uint4 w4 = philox10_small(ctr0[ml] + static_cast<uint32_t>(q), ph);
+        // the folded form measured slower where A is read from L1 (ranks above 8)
+        const uint4 w4 = (VARIANT == kGen || (RANK > 0 && RANK <= 8) || RANK < 0)
+                             ? philox10_small(ctr0[ml] + static_cast<uint32_t>(q), ph)
+                             : philox10(ctr0[ml] + static_cast<uint32_t>(q), 0u, sid, 0u, p.key0, p.key1);
         const uint32_t words[4] = {w4.x, w4.y, w4.z, w4.w};
         float v[4];
 #pragma unroll

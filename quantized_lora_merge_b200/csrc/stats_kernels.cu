@@ -96,7 +96,7 @@ __device__ __forceinline__ double f2_sum(uint64_t v) {
 template <bool HAS_W, bool SMALL>
 __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4],
                                            uint32_t k0, uint32_t k1) {
-  constexpr int kFlush = 8;   // groups per fp32 partial
+  constexpr int kFlush = 16;  // groups per fp32 partial
   const int64_t full = J.numel >> 2;                 // complete groups
   const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
   const float K = HAS_W ? __ldg(J.W) : 0.0f;
@@ -110,7 +110,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   for (int32_t k = 0; k < count;) {
     GroupSums s;
     const int32_t kend = min(count, k + kFlush);
-#pragma unroll 2
+#pragma unroll 4
     for (; k < kend; ++k, g += stride) {
       add_group<HAS_W, SMALL>(s, J, wp, g, K, 4, k0, k1, ph);
       if (HAS_W) wp += 4 * stride;

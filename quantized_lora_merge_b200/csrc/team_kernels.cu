@@ -170,9 +170,16 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         const int nrows = static_cast<int>(min64(kTeamRows, L.d - nrow0));
         const int64_t row_bytes = VARIANT == kGen ? 4 * n : (WBITS == 8 ? n : n / 2);
         const int lines = static_cast<int>((row_bytes + 127) / 128);
-        for (int idx = lt; idx < nrows * lines; idx += LT) {
-          const int rr = idx / lines;
-          prefetch_l2(src + (nrow0 + rr) * ld_src + static_cast<int64_t>(idx - rr * lines) * 128);
+        if (VARIANT == kGen) {
+          // fp32 rows: many lines per row, walked row by row without a division
+          const uint8_t* nsrc = src + nrow0 * ld_src;
+          for (int rr = 0; rr < nrows; ++rr, nsrc += ld_src)
+            for (int line = lt; line < lines; line += LT) prefetch_l2(nsrc + static_cast<int64_t>(line) * 128);
+        } else {
+          for (int idx = lt; idx < nrows * lines; idx += LT) {
+            const int rr = idx / lines;
+            prefetch_l2(src + (nrow0 + rr) * ld_src + static_cast<int64_t>(idx - rr * lines) * 128);
+          }
         }
         if (VARIANT != kGen && lt == 0) {
           prefetch_l2(L.s + nrow0);

@@ -54,31 +54,32 @@ def _load():
         "orc_philox4x32_10": (None, [_ptr, _ptr, _ptr]),
         "orc_aux_word": (_u32, [_u64, _u32, _i64]),
         "orc_laplace_from_word": (_dbl, [_u32]),
-        "orc_aux_block": (None, [_u64, _u32, _i64, _i64, _ptr]),
+        "orc_aux_block": (None, [_u64, _u32, _i64, _i64, _ptr, _int]),
+        "orc_aux_value": (_dbl, [_u64, _u32, _i64, _int]),
         "orc_population_std": (_dbl, [_ptr, _i64]),
         "orc_std_f32": (_dbl, [_ptr, _i64, _i64]),
-        "orc_sigma_r": (_dbl, [_i64, _i64, _u64, _u32]),
+        "orc_sigma_r": (_dbl, [_i64, _i64, _u64, _u32, _int]),
         "orc_vmc_scale": (_dbl, [_dbl, _dbl, _dbl]),
         "orc_affine_quantize_row": (None, [_ptr, _i64, _int, _ptr, _ptr, _ptr, _ptr, _ptr]),
         "orc_gen_aux": (None, [_ptr, _i64, _i64, _u64, _u32, _dbl, _int, _i64, _i64,
-                               _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr]),
+                               _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _ptr, _int]),
         "orc_mla_rows": (None, [_ptr, _i64, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _int, _u64,
-                                _u32, _dbl, _dbl, _dbl, _i64, _i64, _ptr, _ptr]),
+                                _u32, _dbl, _dbl, _dbl, _i64, _i64, _ptr, _ptr, _int]),
         "orc_merge_mul": (None, [_ptr, _i64, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _int, _u64,
                                  _u32, _dbl, _dbl, _dbl, _int, _i64, _i64, _ptr, _ptr, _ptr,
-                                 _ptr, _ptr, _ptr, _ptr]),
+                                 _ptr, _ptr, _ptr, _ptr, _int]),
         "orc_merge_shift": (None, [_ptr, _i64, _ptr, _ptr, _ptr, _ptr, _i64, _i64, _int, _u64,
                                    _u32, _dbl, _dbl, _dbl, _int, _i64, _i64, _ptr, _ptr, _ptr,
-                                   _ptr, _ptr]),
+                                   _ptr, _ptr, _int]),
         "orc_shift_quantize_row": (None, [_ptr, _ptr, _i64, _int, _ptr, _ptr, _ptr, _ptr]),
         "orc_ste_backward": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _ptr]),
         "orc_ste_sampled": (None, [_ptr, _ptr, _ptr, _i64, _i64, _int, _ptr, _i64, _ptr, _i64,
                                    _ptr, _ptr]),
         "orc_quantize_rows": (None, [_ptr, _i64, _u64, _u32, _dbl, _int, _i64, _i64, _ptr, _ptr,
-                                     _ptr, _ptr, _ptr]),
+                                     _ptr, _ptr, _ptr, _int]),
         "orc_merge_mul_rows": (None, [_ptr, _i64, _ptr, _ptr, _ptr, _ptr, _i64, _int, _u64, _u32,
                                       _dbl, _int, _i64, _i64, _ptr, _ptr, _ptr, _ptr, _ptr,
-                                      _ptr]),
+                                      _ptr, _int]),
         "orc_int_digits": (_i64, [_ptr, _i64, _i64, _int, _ptr]),
         "orc_int_gemm_rows": (None, [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_num_threads": (_int, []),
@@ -117,6 +118,14 @@ def aux_word(seed: int, stream_id: int, e: int) -> int:
     return int(_load().orc_aux_word(seed, stream_id, e))
 
 
+LAPLACE, GAUSSIAN, CAUCHY, STUDENT_T2 = 0, 1, 2, 3     # auxiliary laws
+
+
+def aux_value(seed: int, stream_id: int, e: int, dist: int) -> float:
+    """Element e of the auxiliary matrix under law `dist`."""
+    return float(_load().orc_aux_value(seed, stream_id, e, dist))
+
+
 def laplace_from_word(x) -> np.ndarray:
     lib = _load()
     xs = np.atleast_1d(np.asarray(x, dtype=np.uint32))
@@ -124,11 +133,11 @@ def laplace_from_word(x) -> np.ndarray:
 
 
 def aux_R(d: int, n: int, seed: int, stream_id: int, row_begin: int = 0,
-          row_count: int | None = None) -> np.ndarray:
+          row_count: int | None = None, dist: int = 0) -> np.ndarray:
     """Rows [row_begin, row_begin+row_count) of the d x n Laplace matrix R."""
     rc = d - row_begin if row_count is None else row_count
     out = np.zeros((rc, n), np.float64)
-    _load().orc_aux_block(seed, stream_id, row_begin * n, rc * n, _p(out))
+    _load().orc_aux_block(seed, stream_id, row_begin * n, rc * n, _p(out), dist)
     return out
 
 
@@ -146,8 +155,8 @@ def std_f32(W) -> float:
     return float(_load().orc_std_f32(_p(w), d, n))
 
 
-def sigma_r(d: int, n: int, seed: int, stream_id: int) -> float:
-    return float(_load().orc_sigma_r(d, n, seed, stream_id))
+def sigma_r(d: int, n: int, seed: int, stream_id: int, dist: int = 0) -> float:
+    return float(_load().orc_sigma_r(d, n, seed, stream_id, dist))
 
 
 def vmc_scale(sigma_w: float, sigma_r_: float, alpha: float) -> float:
@@ -175,7 +184,7 @@ def affine_quantize_row(x, bits: int):
 # a1-a3: layer preparation
 # --------------------------------------------------------------------------
 def gen_aux(W, seed: int, stream_id: int, alpha: float, w_bits: int, row_begin: int = 0,
-            row_count: int | None = None, want_r_star: bool = False) -> dict:
+            row_count: int | None = None, want_r_star: bool = False, dist: int = 0) -> dict:
     w = _c(W, np.float32)
     d, n = w.shape
     rc = d - row_begin if row_count is None else row_count
@@ -189,13 +198,14 @@ def gen_aux(W, seed: int, stream_id: int, alpha: float, w_bits: int, row_begin: 
     pre = np.zeros((rc, n), np.float64)
     zpre = np.zeros(rc, np.float64)
     _load().orc_gen_aux(_p(w), d, n, seed, stream_id, alpha, w_bits, row_begin, rc, _p(sw),
-                        _p(sr), _p(cc), _p(r_star), _p(codes), _p(s), _p(z), _p(pre), _p(zpre))
+                        _p(sr), _p(cc), _p(r_star), _p(codes), _p(s), _p(z), _p(pre), _p(zpre),
+                        dist)
     return dict(sigma_w=float(sw[0]), sigma_r=float(sr[0]), c=float(cc[0]), r_star=r_star,
                 codes=codes, s=s, z=z, pre=pre, zpre=zpre)
 
 
 def quantize_rows(W_rows, seed: int, stream_id: int, c: float, w_bits: int,
-                  row_begin: int) -> dict:
+                  row_begin: int, dist: int = 0) -> dict:
     """Base quantization of rows [row_begin, row_begin + len(W_rows)) of a layer
     from those rows of W alone, with the VMC factor c given (layers too large
     to hold or reduce on the host)."""
@@ -207,7 +217,7 @@ def quantize_rows(W_rows, seed: int, stream_id: int, c: float, w_bits: int,
     pre = np.zeros((rc, n), np.float64)
     zpre = np.zeros(rc, np.float64)
     _load().orc_quantize_rows(_p(w), n, seed, stream_id, c, w_bits, row_begin, rc, _p(codes),
-                              _p(s), _p(z), _p(pre), _p(zpre))
+                              _p(s), _p(z), _p(pre), _p(zpre), dist)
     return dict(codes=codes, s=s, z=z, pre=pre, zpre=zpre)
 
 
@@ -227,19 +237,19 @@ def _merge_inputs(codes, s, z, A, B):
 
 
 def mla_rows(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, row_begin=0,
-             row_count=None):
+             row_count=None, dist=0):
     """U and D for the given rows (U * D is the pre-quantization merged weight)."""
     cd, sf, zi, Af, Bf, d, n, r = _merge_inputs(codes, s, z, A, B)
     rc = d - row_begin if row_count is None else row_count
     U = np.zeros((rc, n), np.float64)
     D = np.zeros((rc, n), np.int64)
     _load().orc_mla_rows(_p(cd), n, _p(sf), _p(zi), _p(Af), _p(Bf), d, n, r, seed, stream_id,
-                         sigma_w, sigma_r_, alpha, row_begin, rc, _p(U), _p(D))
+                         sigma_w, sigma_r_, alpha, row_begin, rc, _p(U), _p(D), dist)
     return U, D
 
 
 def merge_mul(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, u_bits,
-              row_begin=0, row_count=None) -> dict:
+              row_begin=0, row_count=None, dist=0) -> dict:
     cd, sf, zi, Af, Bf, d, n, r = _merge_inputs(codes, s, z, A, B)
     rc = d - row_begin if row_count is None else row_count
     U = np.zeros((rc, n), np.float64)
@@ -251,12 +261,12 @@ def merge_mul(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, u_bi
     zpre = np.zeros(rc, np.float64)
     _load().orc_merge_mul(_p(cd), n, _p(sf), _p(zi), _p(Af), _p(Bf), d, n, r, seed, stream_id,
                           sigma_w, sigma_r_, alpha, u_bits, row_begin, rc, _p(U), _p(ur),
-                          _p(sbar), _p(zbar), _p(P), _p(pre), _p(zpre))
+                          _p(sbar), _p(zbar), _p(P), _p(pre), _p(zpre), dist)
     return dict(U=U, u_round=ur, sbar=sbar, zbar=zbar, P=P, pre=pre, zpre=zpre)
 
 
 def merge_mul_rows(codes_rows, s_rows, z_rows, A_rows, B, seed, stream_id, c, u_bits,
-                   row_begin) -> dict:
+                   row_begin, dist=0) -> dict:
     """MUL merge of rows [row_begin, row_begin + len(codes_rows)) from those
     rows' inputs alone, with the VMC factor c given."""
     cd = _c(codes_rows, np.int32)
@@ -274,7 +284,7 @@ def merge_mul_rows(codes_rows, s_rows, z_rows, A_rows, B, seed, stream_id, c, u_
     zpre = np.zeros(rc, np.float64)
     _load().orc_merge_mul_rows(_p(cd), n, _p(sf), _p(zi), _p(Af), _p(Bf), n, r, seed, stream_id,
                                c, u_bits, row_begin, rc, _p(ur), _p(sbar), _p(zbar), _p(P),
-                               _p(pre), _p(zpre))
+                               _p(pre), _p(zpre), dist)
     return dict(u_round=ur, sbar=sbar, zbar=zbar, P=P, pre=pre, zpre=zpre)
 
 
@@ -292,7 +302,7 @@ def shift_quantize_row(U, D, shift_bits: int) -> dict:
 
 
 def merge_shift(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, shift_bits,
-                row_begin=0, row_count=None) -> dict:
+                row_begin=0, row_count=None, dist=0) -> dict:
     cd, sf, zi, Af, Bf, d, n, r = _merge_inputs(codes, s, z, A, B)
     rc = d - row_begin if row_count is None else row_count
     U = np.zeros((rc, n), np.float64)
@@ -302,7 +312,7 @@ def merge_shift(codes, s, z, A, B, seed, stream_id, sigma_w, sigma_r_, alpha, sh
     pre = np.zeros((rc, n), np.float64)
     _load().orc_merge_shift(_p(cd), n, _p(sf), _p(zi), _p(Af), _p(Bf), d, n, r, seed, stream_id,
                             sigma_w, sigma_r_, alpha, shift_bits, row_begin, rc, _p(U), _p(sbar),
-                            _p(shift), _p(M), _p(pre))
+                            _p(shift), _p(M), _p(pre), dist)
     return dict(U=U, sbar=sbar, shift=shift, M=M, pre=pre)
 
 

@@ -112,10 +112,49 @@ double orc_laplace_from_word(uint32_t x) {
     return -sign_v * log(1.0 - 2.0 * fabs(v));
 }
 
+/* ------------------------------------------------------------------------ */
+/* The auxiliary laws the ablation compares with Laplace [IntLoRA summary,   */
+/* Measured effects: Gaussian, Cauchy and Student-t auxiliary matrices].     */
+/* Each maps the same Philox words through u = (2 (x >> 9) + 1) 2^-24:      */
+/*   Gaussian N(0,1): Box-Muller on the word pair (2p, 2p + 1) of a block,  */
+/*     rho = sqrt(-2 ln u_2p); word 2p gets rho cos(2 pi u_2p+1), word 2p+1 */
+/*     gets rho sin(2 pi u_2p+1);                                            */
+/*   Cauchy(0,1): tan(pi (u - 1/2)) (inverse CDF);                           */
+/*   Student-t with 2 degrees of freedom: (2u - 1) / sqrt(2 u (1 - u))       */
+/*     (inverse CDF; the pages give no degrees of freedom: reading taken).   */
+/* ------------------------------------------------------------------------ */
+#define PI_F64 3.14159265358979323846264338327950288
+#define DIST_LAPLACE 0
+#define DIST_GAUSSIAN 1
+#define DIST_CAUCHY 2
+#define DIST_STUDENT_T2 3
+
+static double unit_from_word(uint32_t x) { return (2.0 * (double)(x >> 9) + 1.0) * 0x1p-24; }
+
+double orc_aux_value(uint64_t seed, uint32_t stream_id, int64_t e, int dist) {
+    if (dist == DIST_LAPLACE) return orc_laplace_from_word(orc_aux_word(seed, stream_id, e));
+    uint64_t block = (uint64_t)e >> 2;
+    uint32_t ctr[4] = {(uint32_t)block, (uint32_t)(block >> 32), stream_id, 0u};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    orc_philox4x32_10(ctr, key, w);
+    int c = (int)(e & 3);
+    double u = unit_from_word(w[c]);
+    if (dist == DIST_GAUSSIAN) {
+        int p = c & ~1;
+        double rho = sqrt(-2.0 * log(unit_from_word(w[p])));
+        double theta = 2.0 * PI_F64 * unit_from_word(w[p + 1]);
+        return (c & 1) ? rho * sin(theta) : rho * cos(theta);
+    }
+    if (dist == DIST_CAUCHY) return tan(PI_F64 * (u - 0.5));
+    if (dist == DIST_STUDENT_T2) return (2.0 * u - 1.0) / sqrt(2.0 * u * (1.0 - u));
+    return NAN;
+}
+
 /* R for count consecutive flat indices starting at e0. */
-void orc_aux_block(uint64_t seed, uint32_t stream_id, int64_t e0, int64_t count, double* out) {
-    for (int64_t t = 0; t < count; ++t)
-        out[t] = orc_laplace_from_word(orc_aux_word(seed, stream_id, e0 + t));
+void orc_aux_block(uint64_t seed, uint32_t stream_id, int64_t e0, int64_t count, double* out,
+                   int dist) {
+    for (int64_t t = 0; t < count; ++t) out[t] = orc_aux_value(seed, stream_id, e0 + t, dist);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -162,14 +201,14 @@ double orc_std_f32(const float* x, int64_t d, int64_t n) {
 
 /* sigma_R of the regenerated d x n auxiliary matrix (two passes, each one
  * regenerating R; nothing is stored). */
-double orc_sigma_r(int64_t d, int64_t n, uint64_t seed, uint32_t stream_id) {
+double orc_sigma_r(int64_t d, int64_t n, uint64_t seed, uint32_t stream_id, int dist) {
     double* row_acc = (double*)malloc(sizeof(double) * (size_t)d);
     double total = 0.0;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < d; ++i) {
         double acc = 0.0;
         for (int64_t j = 0; j < n; ++j)
-            acc += orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
+            acc += orc_aux_value(seed, stream_id, i * n + j, dist);
         row_acc[i] = acc;
     }
     for (int64_t i = 0; i < d; ++i) total += row_acc[i];
@@ -178,7 +217,7 @@ double orc_sigma_r(int64_t d, int64_t n, uint64_t seed, uint32_t stream_id) {
     for (int64_t i = 0; i < d; ++i) {
         double acc = 0.0;
         for (int64_t j = 0; j < n; ++j) {
-            double dev = orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j)) - mean;
+            double dev = orc_aux_value(seed, stream_id, i * n + j, dist) - mean;
             acc += dev * dev;
         }
         row_acc[i] = acc;
@@ -248,10 +287,10 @@ void orc_affine_quantize_row(const double* x, int64_t n, int bits, double* scale
  * e = i n + j), then the affine quantizer of the row. */
 static void quantize_row(const float* W_row, int64_t n, uint64_t seed, uint32_t stream_id, double c,
                          int w_bits, int64_t i, double* r_star_row, int32_t* codes_row,
-                         double* s_out, int32_t* z_out, double* pre_row, double* zpre) {
+                         double* s_out, int32_t* z_out, double* pre_row, double* zpre, int dist) {
     double* x = (double*)malloc(sizeof(double) * (size_t)n);
     for (int64_t j = 0; j < n; ++j) {
-        double r_star = c * orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
+        double r_star = c * orc_aux_value(seed, stream_id, i * n + j, dist);
         if (r_star_row) r_star_row[j] = r_star;
         x[j] = (double)W_row[j] - r_star;
     }
@@ -263,9 +302,9 @@ void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t s
                  double alpha, int w_bits, int64_t row_begin, int64_t row_count,
                  double* sigma_w_out, double* sigma_r_out, double* c_out,
                  double* r_star_out, int32_t* codes, double* s_out, int32_t* z_out,
-                 double* pre, double* zpre) {
+                 double* pre, double* zpre, int dist) {
     double sigma_w = orc_std_f32(W, d, n);
-    double sigma_r = orc_sigma_r(d, n, seed, stream_id);
+    double sigma_r = orc_sigma_r(d, n, seed, stream_id, dist);
     double c = orc_vmc_scale(sigma_w, sigma_r, alpha);
     *sigma_w_out = sigma_w;
     *sigma_r_out = sigma_r;
@@ -274,7 +313,7 @@ void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t s
     for (int64_t t = 0; t < row_count; ++t)
         quantize_row(&W[(row_begin + t) * n], n, seed, stream_id, c, w_bits, row_begin + t,
                      r_star_out ? &r_star_out[t * n] : NULL, &codes[t * n], &s_out[t], &z_out[t],
-                     pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
+                     pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL, dist);
 }
 
 /* The same row quantization for rows whose W is given alone (W_rows holds
@@ -282,12 +321,12 @@ void orc_gen_aux(const float* W, int64_t d, int64_t n, uint64_t seed, uint32_t s
  * c is given: layers too large to hold or reduce on the host. */
 void orc_quantize_rows(const float* W_rows, int64_t n, uint64_t seed, uint32_t stream_id, double c,
                        int w_bits, int64_t row_begin, int64_t row_count, int32_t* codes,
-                       double* s_out, int32_t* z_out, double* pre, double* zpre) {
+                       double* s_out, int32_t* z_out, double* pre, double* zpre, int dist) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < row_count; ++t)
         quantize_row(&W_rows[t * n], n, seed, stream_id, c, w_bits, row_begin + t, NULL,
                      &codes[t * n], &s_out[t], &z_out[t], pre ? &pre[t * n] : NULL,
-                     zpre ? &zpre[t] : NULL);
+                     zpre ? &zpre[t] : NULL, dist);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -298,10 +337,10 @@ void orc_quantize_rows(const float* W_rows, int64_t n, uint64_t seed, uint32_t s
 /* ------------------------------------------------------------------------ */
 static void adaptation_row(const int32_t* codes_row, float s_i32, int32_t z_i, const float* A_row,
                            const float* B, int64_t n, int r, uint64_t seed, uint32_t stream_id,
-                           double c, int64_t i, double* U, int64_t* D) {
+                           double c, int64_t i, double* U, int64_t* D, int dist) {
     double s_i = (double)s_i32;
     for (int64_t j = 0; j < n; ++j) {
-        double r_star = c * orc_laplace_from_word(orc_aux_word(seed, stream_id, i * n + j));
+        double r_star = c * orc_aux_value(seed, stream_id, i * n + j, dist);
         double ab = 0.0;
         for (int k = 0; k < r; ++k) ab += (double)A_row[k] * (double)B[(int64_t)k * n + j];
         int64_t dij = (int64_t)codes_row[j] - (int64_t)z_i;
@@ -315,14 +354,14 @@ static void adaptation_row(const int32_t* codes_row, float s_i32, int32_t z_i, c
 void orc_mla_rows(const int32_t* codes, int64_t ld_codes, const float* s, const int32_t* z,
                   const float* A, const float* B, int64_t d, int64_t n, int r, uint64_t seed,
                   uint32_t stream_id, double sigma_w, double sigma_r, double alpha,
-                  int64_t row_begin, int64_t row_count, double* U_out, int64_t* D_out) {
+                  int64_t row_begin, int64_t row_count, double* U_out, int64_t* D_out, int dist) {
     (void)d;
     double c = orc_vmc_scale(sigma_w, sigma_r, alpha);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < row_count; ++t)
         adaptation_row(&codes[(row_begin + t) * ld_codes], s[row_begin + t], z[row_begin + t],
                        &A[(row_begin + t) * r], B, n, r, seed, stream_id, c, row_begin + t,
-                       &U_out[t * n], &D_out[t * n]);
+                       &U_out[t * n], &D_out[t * n], dist);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -336,13 +375,13 @@ void orc_merge_mul_rows(const int32_t* codes_rows, int64_t ld_codes, const float
                         const int32_t* z_rows, const float* A_rows, const float* B, int64_t n,
                         int r, uint64_t seed, uint32_t stream_id, double c, int u_bits,
                         int64_t row_begin, int64_t row_count, int32_t* u_round, double* sbar,
-                        int32_t* zbar, int64_t* P, double* pre, double* zpre);
+                        int32_t* zbar, int64_t* P, double* pre, double* zpre, int dist);
 
 void orc_merge_mul(const int32_t* codes, int64_t ld_codes, const float* s, const int32_t* z,
                    const float* A, const float* B, int64_t d, int64_t n, int r, uint64_t seed,
                    uint32_t stream_id, double sigma_w, double sigma_r, double alpha, int u_bits,
                    int64_t row_begin, int64_t row_count, double* U_out, int32_t* u_round,
-                   double* sbar, int32_t* zbar, int64_t* P, double* pre, double* zpre) {
+                   double* sbar, int32_t* zbar, int64_t* P, double* pre, double* zpre, int dist) {
     (void)d;
     double c = orc_vmc_scale(sigma_w, sigma_r, alpha);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -351,7 +390,7 @@ void orc_merge_mul(const int32_t* codes, int64_t ld_codes, const float* s, const
         double* U = (double*)malloc(sizeof(double) * (size_t)n);
         int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
         adaptation_row(&codes[i * ld_codes], s[i], z[i], &A[i * r], B, n, r, seed, stream_id, c, i,
-                       U, D);
+                       U, D, dist);
         orc_affine_quantize_row(U, n, u_bits, &sbar[t], &zbar[t], &u_round[t * n],
                                 pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
         for (int64_t j = 0; j < n; ++j) {
@@ -370,13 +409,13 @@ void orc_merge_mul_rows(const int32_t* codes_rows, int64_t ld_codes, const float
                         const int32_t* z_rows, const float* A_rows, const float* B, int64_t n,
                         int r, uint64_t seed, uint32_t stream_id, double c, int u_bits,
                         int64_t row_begin, int64_t row_count, int32_t* u_round, double* sbar,
-                        int32_t* zbar, int64_t* P, double* pre, double* zpre) {
+                        int32_t* zbar, int64_t* P, double* pre, double* zpre, int dist) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t t = 0; t < row_count; ++t) {
         double* U = (double*)malloc(sizeof(double) * (size_t)n);
         int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
         adaptation_row(&codes_rows[t * ld_codes], s_rows[t], z_rows[t], &A_rows[t * r], B, n, r,
-                       seed, stream_id, c, row_begin + t, U, D);
+                       seed, stream_id, c, row_begin + t, U, D, dist);
         orc_affine_quantize_row(U, n, u_bits, &sbar[t], &zbar[t], &u_round[t * n],
                                 pre ? &pre[t * n] : NULL, zpre ? &zpre[t] : NULL);
         for (int64_t j = 0; j < n; ++j)
@@ -422,7 +461,7 @@ void orc_merge_shift(const int32_t* codes, int64_t ld_codes, const float* s, con
                      const float* A, const float* B, int64_t d, int64_t n, int r, uint64_t seed,
                      uint32_t stream_id, double sigma_w, double sigma_r, double alpha,
                      int shift_bits, int64_t row_begin, int64_t row_count, double* U_out,
-                     double* sbar, int32_t* shift, int64_t* M, double* pre) {
+                     double* sbar, int32_t* shift, int64_t* M, double* pre, int dist) {
     (void)d;
     double c = orc_vmc_scale(sigma_w, sigma_r, alpha);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -431,7 +470,7 @@ void orc_merge_shift(const int32_t* codes, int64_t ld_codes, const float* s, con
         double* U = (double*)malloc(sizeof(double) * (size_t)n);
         int64_t* D = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
         adaptation_row(&codes[i * ld_codes], s[i], z[i], &A[i * r], B, n, r, seed, stream_id, c, i,
-                       U, D);
+                       U, D, dist);
         orc_shift_quantize_row(U, D, n, shift_bits, &sbar[t], &shift[t * n], &M[t * n],
                                pre ? &pre[t * n] : NULL);
         if (U_out)

@@ -501,3 +501,80 @@ def test_row_views_equal_whole_layer_functions():
                                13, g["c"], 4, 7)
     for k in ("u_round", "sbar", "zbar", "P", "pre", "zpre"):
         np.testing.assert_array_equal(mr[k], m[k][rows])
+
+
+# ---------------------------------------------------------------------------
+# auxiliary laws of the ablation: Gaussian, Cauchy, Student-t (2 dof)
+# ---------------------------------------------------------------------------
+def _law_sample(dist):
+    return oracle.aux_R(1024, 1024, 1, 3, dist=dist).ravel()
+
+
+def _frac_close(frac, p, n, z=4.5):
+    return abs(frac - p) <= z * math.sqrt(p * (1 - p) / n)
+
+
+def test_gaussian_law_moments_and_tails():
+    x = _law_sample(oracle.GAUSSIAN)
+    n = x.size
+    assert abs(x.mean()) < 4.5 / math.sqrt(n)
+    assert abs(x.var() - 1.0) < 4.5 * math.sqrt(2.0 / n)
+    k = ((x - x.mean()) ** 4).mean() / x.var() ** 2
+    assert abs(k - 3.0) < 4.5 * math.sqrt(24.0 / n)
+    for t in (0.5, 1.0, 1.96, 3.0):      # P(|Z| > t) = erfc(t / sqrt 2)
+        assert _frac_close(np.mean(np.abs(x) > t), math.erfc(t / math.sqrt(2.0)), n)
+    # Box-Muller pairs: words 2p and 2p+1 share the radius, so the pair's
+    # squared norm is -2 ln u of word 2p, independent of the angle word
+    pairs = x.reshape(-1, 2)
+    r2 = (pairs ** 2).sum(axis=1)
+    assert abs(np.mean(r2) - 2.0) < 4.5 * 2.0 / math.sqrt(r2.size)   # chi-square(2): mean 2, sd 2
+    assert _frac_close(np.mean(r2 > 2.0), math.exp(-1.0), r2.size)   # P(chi2_2 > t) = e^(-t/2)
+
+
+def test_cauchy_law_cdf_and_symmetry():
+    x = _law_sample(oracle.CAUCHY)
+    n = x.size
+    for t in (-10.0, -1.0, -0.25, 0.0, 0.5, 1.0, 3.0, 50.0):   # F(t) = 1/2 + atan(t) / pi
+        assert _frac_close(np.mean(x <= t), 0.5 + math.atan(t) / math.pi, n)
+    assert _frac_close(np.mean(np.abs(x) < 1.0), 0.5, n)         # quartiles at -1, +1
+
+
+def test_student_t2_law_cdf():
+    x = _law_sample(oracle.STUDENT_T2)
+    n = x.size
+    for t in (-5.0, -2.0, -0.5, 0.0, 1.0, 3.0, 20.0):   # F(t) = 1/2 + t / (2 sqrt(2 + t^2))
+        assert _frac_close(np.mean(x <= t), 0.5 + t / (2.0 * math.sqrt(2.0 + t * t)), n)
+
+
+def test_laws_share_the_laplace_stream_and_layout():
+    """Law 0 is the pinned Laplace sampler; every law reads element e from
+    block e / 4 (a different element of the same block changes the value)."""
+    np.testing.assert_array_equal(oracle.aux_R(3, 8, 1, 5, dist=oracle.LAPLACE),
+                                  oracle.aux_R(3, 8, 1, 5))
+    for dist in (oracle.GAUSSIAN, oracle.CAUCHY, oracle.STUDENT_T2):
+        a = oracle.aux_R(3, 8, 1, 5, dist=dist)
+        assert np.all(np.isfinite(a))
+        assert [oracle.aux_value(1, 5, e, dist) for e in range(24)] == a.ravel().tolist()
+
+
+@pytest.mark.parametrize("dist", [1, 2, 3])
+def test_gen_aux_and_merge_compose_under_other_laws(dist):
+    """sigma_R is the population std of the law's R; the base quantization and
+    the MUL merge use c = (sigma_W / sigma_R)^alpha and R of that law."""
+    spec, W, A, B = _small_layer(10, 24, 4, 4, 19)
+    g = oracle.gen_aux(W, spec.seed, 19, spec.alpha, 4, want_r_star=True, dist=dist)
+    R = oracle.aux_R(10, 24, spec.seed, 19, dist=dist)
+    assert abs(g["sigma_r"] - np.std(R)) <= 1e-12 * np.std(R)
+    assert abs(g["sigma_r"] - oracle.sigma_r(10, 24, spec.seed, 19, dist=dist)) <= 1e-12 * g["sigma_r"]
+    c = oracle.vmc_scale(np.std(W.astype(np.float64)), np.std(R), spec.alpha)
+    np.testing.assert_allclose(g["r_star"], c * R, rtol=1e-12)
+    for i in range(10):
+        q = oracle.affine_quantize_row(W[i].astype(np.float64) - g["r_star"][i], 4)
+        assert g["codes"][i].tolist() == q["codes"].tolist()
+    s32 = g["s"].astype(np.float32)
+    U, D = oracle.mla_rows(g["codes"], s32, g["z"], A, B, spec.seed, 19, g["sigma_w"], g["sigma_r"],
+                           spec.alpha, dist=dist)
+    AB = A.astype(np.float64) @ B.astype(np.float64)
+    nz = D != 0
+    np.testing.assert_allclose((U * D)[nz], (s32.astype(np.float64)[:, None] * D + g["r_star"] + AB)[nz],
+                               rtol=1e-11, atol=1e-14)

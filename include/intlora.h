@@ -101,6 +101,23 @@ const char* intlora_last_error(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int intlora_version(void);
 
+/* Auxiliary law of R [summary, "Measured effects": the ablation compares
+ * Laplace, the method's choice, with Gaussian, Cauchy and Student-t auxiliary
+ * matrices]. Every law reads element e from word e mod 4 of Philox block e / 4
+ * through u = (2 (x >> 9) + 1) 2^-24:
+ *   LAPLACE     -sign(u - 1/2) ln(1 - 2 |u - 1/2|)
+ *   GAUSSIAN    Box-Muller on the word pair (2p, 2p + 1) of the block: word 2p
+ *               gets sqrt(-2 ln u_2p) cos(2 pi u_2p+1), word 2p + 1 the sine
+ *   CAUCHY      tan(pi (u - 1/2))
+ *   STUDENT_T2  (2u - 1) / sqrt(2 u (1 - u)): Student-t with 2 degrees of
+ *               freedom (the pages give none; 2 has a closed-form inverse CDF)
+ * Layers with a law other than Laplace run on the general row-tile kernels
+ * with A B on the CUDA cores. */
+#define INTLORA_DIST_LAPLACE 0
+#define INTLORA_DIST_GAUSSIAN 1
+#define INTLORA_DIST_CAUCHY 2
+#define INTLORA_DIST_STUDENT_T2 3
+
 /* Limits of this build. */
 #define INTLORA_MAX_RANK 256
 #define INTLORA_MAX_BATCH 128     /* descriptors per batched call */
@@ -135,6 +152,7 @@ typedef struct intlora_aux_job {
     int64_t ld_w_out;
     float* s_out;
     int32_t* z_out;
+    int32_t distribution;       /* INTLORA_DIST_*; intlora_gen_aux(_noalloc) use LAPLACE */
 } intlora_aux_job;
 
 size_t intlora_gen_aux_workspace_size(const intlora_aux_job* jobs, int32_t count);
@@ -200,6 +218,7 @@ typedef struct intlora_layer {
     float alpha;                /* VMC exponent */
     const double* sigma_w;      /* device scalar */
     const double* sigma_r;      /* device scalar or NULL */
+    int32_t distribution;       /* INTLORA_DIST_*: the law R was drawn from in gen_aux */
 } intlora_layer;
 
 /* Outputs of one merge.

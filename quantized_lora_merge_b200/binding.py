@@ -21,6 +21,8 @@ HEADER = PKG.parent / "include" / "intlora.h"
 _c_i64, _c_i32, _c_u64, _c_u32 = ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64, ctypes.c_uint32
 _c_f32, _c_ptr, _c_size = ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
+DIST_LAPLACE, DIST_GAUSSIAN, DIST_CAUCHY, DIST_STUDENT_T2 = 0, 1, 2, 3   # INTLORA_DIST_*
+
 STATUS = {0: "INTLORA_OK", 1: "INTLORA_ERR_INVALID_ARG", 2: "INTLORA_ERR_UNSUPPORTED",
           3: "INTLORA_ERR_WORKSPACE", 4: "INTLORA_ERR_CUDA", 5: "INTLORA_ERR_TIMEOUT"}
 
@@ -36,14 +38,15 @@ class intlora_aux_job(ctypes.Structure):
                 ("stream_id", _c_u32), ("alpha", _c_f32), ("w_bits", _c_i32),
                 ("sigma_w_out", _c_ptr), ("sigma_r_out", _c_ptr), ("r_star_out", _c_ptr),
                 ("w_round_out", _c_ptr), ("ld_w_out", _c_i64), ("s_out", _c_ptr),
-                ("z_out", _c_ptr)]
+                ("z_out", _c_ptr), ("distribution", _c_i32)]
 
 
 class intlora_layer(ctypes.Structure):
     _fields_ = [("d", _c_i64), ("n", _c_i64), ("r", _c_i32), ("w_bits", _c_i32),
                 ("w_round", _c_ptr), ("ld_w", _c_i64), ("s", _c_ptr), ("z", _c_ptr),
                 ("A", _c_ptr), ("B", _c_ptr), ("seed", _c_u64), ("stream_id", _c_u32),
-                ("alpha", _c_f32), ("sigma_w", _c_ptr), ("sigma_r", _c_ptr)]
+                ("alpha", _c_f32), ("sigma_w", _c_ptr), ("sigma_r", _c_ptr),
+                ("distribution", _c_i32)]
 
 
 class intlora_merge_out(ctypes.Structure):
@@ -165,6 +168,7 @@ class AuxJob:
     w_round: object = None          # uint8 [d, ld]
     s: object = None
     z: object = None
+    distribution: int = 0           # INTLORA_DIST_*
 
     def to_c(self) -> intlora_aux_job:
         d, n = self.W.shape
@@ -172,7 +176,7 @@ class AuxJob:
         return intlora_aux_job(_ptr(self.W), d, n, self.seed, self.stream_id, self.alpha,
                                self.w_bits, _ptr(self.sigma_w), _ptr(self.sigma_r),
                                _ptr(self.r_star), _ptr(self.w_round), ld, _ptr(self.s),
-                               _ptr(self.z))
+                               _ptr(self.z), self.distribution)
 
 
 @dataclass
@@ -189,13 +193,14 @@ class Layer:
     alpha: float
     sigma_w: object
     sigma_r: object = None
+    distribution: int = 0           # INTLORA_DIST_*
 
     def to_c(self) -> intlora_layer:
         d = self.w_round.shape[0]
         return intlora_layer(d, self.n, self.A.shape[1], self.w_bits, _ptr(self.w_round),
                              self.w_round.shape[1], _ptr(self.s), _ptr(self.z), _ptr(self.A),
                              _ptr(self.B), self.seed, self.stream_id, self.alpha,
-                             _ptr(self.sigma_w), _ptr(self.sigma_r))
+                             _ptr(self.sigma_w), _ptr(self.sigma_r), self.distribution)
 
 
 @dataclass

@@ -290,7 +290,7 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
 }
 
 intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bits, int w_bits,
-                                 int out_bytes, uint64_t seed, cudaStream_t stream) {
+                                 int out_bytes, uint64_t seed, int dist, cudaStream_t stream) {
   // layers whose A B was precomputed run in launches of their own (the
   // kernels' rank-free specialisation)
   bool any_t = false, all_t = true;
@@ -301,12 +301,13 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
   if (any_t && !all_t) {
     std::vector<TileLayer> with_t, without;
     for (auto& l : L) (l.T != nullptr ? with_t : without).push_back(l);
-    const intlora_status s = launch_tile_batch(variant, with_t, bits, w_bits, out_bytes, seed, stream);
+    const intlora_status s = launch_tile_batch(variant, with_t, bits, w_bits, out_bytes, seed, dist, stream);
     if (s != INTLORA_OK) return s;
-    return launch_tile_batch(variant, without, bits, w_bits, out_bytes, seed, stream);
+    return launch_tile_batch(variant, without, bits, w_bits, out_bytes, seed, dist, stream);
   }
   // layers the team kernel takes go there (one launch); the rest stay here
-  if (team_path_enabled()) {
+  // (the team kernels draw Laplace R only)
+  if (team_path_enabled() && dist == INTLORA_DIST_LAPLACE) {
     std::vector<TileLayer> team, rest;
     for (auto& l : L) (team_eligible(variant, l) ? team : rest).push_back(l);
     if (!team.empty()) {
@@ -332,6 +333,7 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
     if (rank_ct != 4 && rank_ct != 8 && rank_ct != 16) rank_ct = 0;
     if (all_t) rank_ct = -1;
   }
+  if (dist != INTLORA_DIST_LAPLACE) rank_ct = -2;    // any rank, another auxiliary law
   bool aligned = true;
   for (auto& l : L) aligned = aligned && (l.n % 4 == 0);
   TileBatch b;
@@ -370,6 +372,7 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
   b.small = 1;
   for (auto& l : L)
     if (l.d * l.n >= (int64_t{1} << 34)) b.small = 0;
+  b.dist = dist;
   cudaError_t e = launch_tiles(b, rank_ct, aligned, stream);
   if (e != cudaSuccess) return cuda_fail(e, "row-tile kernel launch");
   return INTLORA_OK;
@@ -393,6 +396,8 @@ intlora_status check_aux_job(const intlora_aux_job& j, int idx) {
     return fail(INTLORA_ERR_INVALID_ARG, "job %d: alpha must be finite and >= 0", idx);
   if (j.sigma_w_out == nullptr || j.sigma_r_out == nullptr)
     return fail(INTLORA_ERR_INVALID_ARG, "job %d: sigma outputs are required", idx);
+  if (j.distribution < INTLORA_DIST_LAPLACE || j.distribution > INTLORA_DIST_STUDENT_T2)
+    return fail(INTLORA_ERR_INVALID_ARG, "job %d: distribution must be one of INTLORA_DIST_*", idx);
   if (!aligned16(j.W)) return fail(INTLORA_ERR_INVALID_ARG, "job %d: W must be 16-byte aligned", idx);
   if (j.r_star_out != nullptr && !aligned16(j.r_star_out))
     return fail(INTLORA_ERR_INVALID_ARG, "job %d: r_star_out must be 16-byte aligned", idx);
@@ -416,17 +421,19 @@ size_t aux_ws_bytes(const intlora_aux_job* jobs, int32_t count) {
   return total;
 }
 
-// Indices of `count` items grouped by seed, in first-appearance order: every
-// launch carries one Philox key at batch level (uniform round keys).
+// Indices of `count` items grouped by (seed, auxiliary law), in
+// first-appearance order: every launch carries one Philox key (uniform round
+// keys) and one law at batch level.
 template <typename T>
 std::vector<std::vector<int32_t>> group_by_seed(const T* items, int32_t count) {
-  std::vector<uint64_t> seeds;
+  std::vector<std::pair<uint64_t, int32_t>> keys;
   std::vector<std::vector<int32_t>> groups;
   for (int32_t k = 0; k < count; ++k) {
+    const std::pair<uint64_t, int32_t> key(items[k].seed, items[k].distribution);
     size_t g = 0;
-    while (g < seeds.size() && seeds[g] != items[k].seed) ++g;
-    if (g == seeds.size()) {
-      seeds.push_back(items[k].seed);
+    while (g < keys.size() && keys[g] != key) ++g;
+    if (g == keys.size()) {
+      keys.push_back(key);
       groups.emplace_back();
     }
     groups[g].push_back(k);
@@ -463,6 +470,7 @@ intlora_status gen_aux_chunk(const intlora_aux_job* jobs, int32_t count, char* w
     sb.count = static_cast<int32_t>(grp.size());
     sb.key0 = lo32(jobs[grp[0]].seed);
     sb.key1 = hi32(jobs[grp[0]].seed);
+    sb.dist = jobs[grp[0]].distribution;
     cudaError_t e = launch_stats(sb, blocks, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
     e = launch_stats_finalize(sb, st);
@@ -492,7 +500,8 @@ intlora_status gen_aux_chunk(const intlora_aux_job* jobs, int32_t count, char* w
         L.push_back(l);
       }
       if (L.empty()) continue;
-      const intlora_status s = launch_tile_batch(kGen, L, wb, wb, 1, jobs[grp[0]].seed, st);
+      const intlora_status s =
+          launch_tile_batch(kGen, L, wb, wb, 1, jobs[grp[0]].seed, jobs[grp[0]].distribution, st);
       if (s != INTLORA_OK) return s;
     }
   }
@@ -522,6 +531,8 @@ intlora_status check_layer(const intlora_layer* l, int idx) {
   if (!aligned16(l->w_round)) return fail(INTLORA_ERR_INVALID_ARG, "layer %d: w_round must be 16-byte aligned", idx);
   if (!(l->alpha >= 0.0f) || !std::isfinite(l->alpha))
     return fail(INTLORA_ERR_INVALID_ARG, "layer %d: alpha must be finite and >= 0", idx);
+  if (l->distribution < INTLORA_DIST_LAPLACE || l->distribution > INTLORA_DIST_STUDENT_T2)
+    return fail(INTLORA_ERR_INVALID_ARG, "layer %d: distribution must be one of INTLORA_DIST_*", idx);
   return INTLORA_OK;
 }
 
@@ -543,7 +554,7 @@ bool tensor_t_enabled() {
   return v == nullptr || std::strcmp(v, "cuda") != 0;
 }
 bool uses_tensor_t(const intlora_layer& l) {
-  return tensor_t_enabled() && t_gemm_supported(l.d, l.n, l.r);
+  return tensor_t_enabled() && l.distribution == INTLORA_DIST_LAPLACE && t_gemm_supported(l.d, l.n, l.r);
 }
 // A call whose workspace does not cover the tensor-core T buffers still runs,
 // with A B on the CUDA cores (set per call by merge_batched).
@@ -639,6 +650,7 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
       sb.count = ns;
       sb.key0 = lo32(layers[grp[0]].seed);
       sb.key1 = hi32(layers[grp[0]].seed);
+      sb.dist = layers[grp[0]].distribution;
       cudaError_t e = launch_stats(sb, blocks, st);
       if (e != cudaSuccess) return cuda_fail(e, "statistics kernel launch");
       e = launch_stats_finalize(sb, st);
@@ -678,7 +690,7 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
       if (L.empty()) continue;
       const intlora_status s = launch_tile_batch(variant, L, bits, wb,
                                                  out_bytes_for(variant == kMul ? 0 : 1, wb, bits),
-                                                 layers[grp[0]].seed, st);
+                                                 layers[grp[0]].seed, layers[grp[0]].distribution, st);
       if (s != INTLORA_OK) return s;
     }
   }
@@ -1007,6 +1019,7 @@ intlora_status intlora_gen_aux(const float* W, int64_t d, int64_t n, uint64_t se
   j.ld_w_out = ld_w_out;
   j.s_out = s_out;
   j.z_out = z_out;
+  j.distribution = INTLORA_DIST_LAPLACE;
   return intlora_gen_aux_batched(&j, 1, ws, ws_bytes, stream);
 }
 

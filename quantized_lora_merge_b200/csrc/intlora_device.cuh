@@ -135,6 +135,36 @@ __device__ __forceinline__ float laplace_scaled(uint32_t x, float c_ln2) {
   return laplace_log2(x) * laplace_sign(x, c_ln2);
 }
 
+// The auxiliary laws the ablation compares with Laplace (IntLoRA summary,
+// "Measured effects": Gaussian, Cauchy and Student-t auxiliary matrices),
+// read from the same Philox words through u = (2 (x >> 9) + 1) 2^-24:
+//   Gaussian: Box-Muller on the word pair (2p, 2p + 1) of a block: radius
+//     sqrt(-2 ln u_2p), angle 2 pi u_2p+1; word 2p takes the cosine, word
+//     2p + 1 the sine;
+//   Cauchy: tan(pi (u - 1/2)) = -cos(pi u) / sin(pi u) (sinpi / cospi keep
+//     the argument exact near the poles);
+//   Student-t with 2 degrees of freedom: (2u - 1) / sqrt(2 u (1 - u)).
+constexpr int kDistLaplace = 0;
+constexpr int kDistGaussian = 1;
+constexpr int kDistCauchy = 2;
+constexpr int kDistStudentT2 = 3;
+
+// u of a word, exactly: 1 + k 2^-23 built from the bits, minus (1 - 2^-24).
+__device__ __forceinline__ float unit_from_word(uint32_t x) {
+  return __uint_as_float(0x3F800000u | (x >> 9)) - 0.999999940395355224609375f;
+}
+// R of the element whose word is word `odd` of the pair (w_even, w_odd).
+__device__ __forceinline__ float aux_value_generic(int dist, uint32_t w_even, uint32_t w_odd, bool odd) {
+  if (dist == kDistGaussian) {
+    const float rho = sqrtf(-2.0f * logf(unit_from_word(w_even)));
+    const float t = 2.0f * unit_from_word(w_odd);
+    return odd ? rho * sinpif(t) : rho * cospif(t);
+  }
+  const float u = unit_from_word(odd ? w_odd : w_even);
+  if (dist == kDistCauchy) return -cospif(u) / sinpif(u);
+  return (2.0f * u - 1.0f) / sqrtf(2.0f * u * (1.0f - u));
+}
+
 // Packed pairs of fp32 (sm_100 f32x2 instructions): two lanes' worth of
 // fma/add/mul per instruction, each half rounded exactly like its scalar
 // counterpart (round to nearest even).

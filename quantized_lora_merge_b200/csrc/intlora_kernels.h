@@ -31,6 +31,7 @@ struct StatsBatch {
   int32_t count;
   uint32_t key0, key1;       // Philox key shared by every job of the batch (kept
                              // at batch level so the round keys stay uniform)
+  int32_t dist;              // auxiliary law of every job (kDistLaplace, ...)
 };
 
 // ---------------------------------------------------------------------------
@@ -87,6 +88,7 @@ struct TileBatch {
   int32_t smem_b;            // floats of the B buffer
   int32_t smem_a;            // floats of the A-rows buffer (>= r m)
   int32_t small;             // every layer below 2^34 elements (32-bit Philox block index)
+  int32_t dist;              // auxiliary law (other than Laplace: the RANK = -2 kernels)
 };
 
 constexpr int kTileThreads = 256;

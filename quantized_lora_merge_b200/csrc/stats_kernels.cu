@@ -45,16 +45,26 @@ struct GroupSums {
   uint64_t w1 = 0, w2 = 0, r1 = 0, r2 = 0;
 };
 
-template <bool HAS_W, bool SMALL>
+template <bool HAS_W, bool SMALL, bool GENERIC>
 __device__ __forceinline__ void add_group(GroupSums& g, const StatsJob& J, const float* wgroup,
                                           uint64_t group, float K, int valid, uint32_t k0, uint32_t k1,
-                                          const PhiloxSmall& ph) {
+                                          const PhiloxSmall& ph, int dist) {
   // SMALL: fewer than 2^34 elements, so the block index's high word is 0
   const uint4 w = SMALL ? philox10_small(static_cast<uint32_t>(group), ph)
                         : aux_block(static_cast<uint64_t>(group), J.stream_id, k0, k1);
-  // R / ln 2 = +-log2(w): the sums run in the log2 domain (the sign is a
-  // factor of +-1, R^2 needs none) and the finalize kernel scales by ln 2
-  if (valid == 4) {
+  if (GENERIC) {
+    // another auxiliary law: R itself is summed
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    float rv[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      rv[c] = c < valid ? aux_value_generic(dist, words[c & 2], words[c | 1], (c & 1) != 0) : 0.0f;
+    const uint64_t r01 = f2_pack(rv[0], rv[1]), r23 = f2_pack(rv[2], rv[3]);
+    g.r1 = f2_add(f2_add(g.r1, r01), r23);
+    g.r2 = f2_fma(r23, r23, f2_fma(r01, r01, g.r2));
+  } else if (valid == 4) {
+    // R / ln 2 = +-log2(w): the sums run in the log2 domain (the sign is a
+    // factor of +-1, R^2 needs none) and the finalize kernel scales by ln 2
     const uint64_t l01 = laplace_log2_x2(w.x, w.y), l23 = laplace_log2_x2(w.z, w.w);
     const uint64_t s01 = f2_pack(laplace_sign(w.x, 1.0f), laplace_sign(w.y, 1.0f));
     const uint64_t s23 = f2_pack(laplace_sign(w.z, 1.0f), laplace_sign(w.w, 1.0f));
@@ -93,9 +103,9 @@ __device__ __forceinline__ double f2_sum(uint64_t v) {
   return static_cast<double>(f2_lo(v)) + static_cast<double>(f2_hi(v));
 }
 
-template <bool HAS_W, bool SMALL>
+template <bool HAS_W, bool SMALL, bool GENERIC>
 __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, double acc[4],
-                                           uint32_t k0, uint32_t k1) {
+                                           uint32_t k0, uint32_t k1, int dist) {
   constexpr int kFlush = 16;  // groups per fp32 partial
   const int64_t full = J.numel >> 2;                 // complete groups
   const int64_t stride = static_cast<int64_t>(J.nblocks) * kStatsThreads;
@@ -112,7 +122,7 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
     const int32_t kend = min(count, k + kFlush);
 #pragma unroll 4
     for (; k < kend; ++k, g += stride) {
-      add_group<HAS_W, SMALL>(s, J, wp, g, K, 4, k0, k1, ph);
+      add_group<HAS_W, SMALL, GENERIC>(s, J, wp, g, K, 4, k0, k1, ph, dist);
       if (HAS_W) wp += 4 * stride;
     }
     acc[0] += f2_sum(s.w1);
@@ -123,7 +133,8 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   const int tail = static_cast<int>(J.numel & 3);
   if (tail != 0 && local == 0 && threadIdx.x == 0) {
     GroupSums s;
-    add_group<HAS_W, SMALL>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1, ph);
+    add_group<HAS_W, SMALL, GENERIC>(s, J, HAS_W ? J.W + 4 * full : nullptr, full, K, tail, k0, k1, ph,
+                                     dist);
     acc[0] += f2_sum(s.w1);
     acc[1] += f2_sum(s.w2);
     acc[2] += f2_sum(s.r1);
@@ -131,6 +142,8 @@ __device__ __forceinline__ void stats_body(const StatsJob& J, int64_t local, dou
   }
 }
 
+// GENERIC: an auxiliary law other than Laplace (b.dist)
+template <bool GENERIC>
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_constant__ StatsBatch b) {
   __shared__ double red[4 * 32];
   const int64_t bid = blockIdx.x;
@@ -141,11 +154,11 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const __grid_const
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
   const bool small = J.numel < (int64_t{1} << 34);
   if (J.W != nullptr) {
-    if (small) stats_body<true, true>(J, local, acc, b.key0, b.key1);
-    else stats_body<true, false>(J, local, acc, b.key0, b.key1);
+    if (small) stats_body<true, true, GENERIC>(J, local, acc, b.key0, b.key1, b.dist);
+    else stats_body<true, false, GENERIC>(J, local, acc, b.key0, b.key1, b.dist);
   } else {
-    if (small) stats_body<false, true>(J, local, acc, b.key0, b.key1);
-    else stats_body<false, false>(J, local, acc, b.key0, b.key1);
+    if (small) stats_body<false, true, GENERIC>(J, local, acc, b.key0, b.key1, b.dist);
+    else stats_body<false, false, GENERIC>(J, local, acc, b.key0, b.key1, b.dist);
   }
   block_sum4(acc, red);
   if (threadIdx.x == 0)
@@ -166,8 +179,8 @@ __global__ void __launch_bounds__(kStatsThreads) stats_finalize_kernel(const __g
       *J.sigma_w_out = sqrt(fmax(var, 0.0));
     }
     if (J.sigma_r_out != nullptr) {
-      const double var = (acc[3] - acc[2] * acc[2] / N) / N;   // of R / ln 2
-      *J.sigma_r_out = kLn2d * sqrt(fmax(var, 0.0));
+      const double var = (acc[3] - acc[2] * acc[2] / N) / N;   // Laplace: of R / ln 2
+      *J.sigma_r_out = (b.dist == kDistLaplace ? kLn2d : 1.0) * sqrt(fmax(var, 0.0));
     }
   }
 }
@@ -181,7 +194,10 @@ __global__ void zero_kernel(float* p, int64_t count) {
 }  // namespace
 
 cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t s) {
-  stats_kernel<<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
+  if (b.dist == kDistLaplace)
+    stats_kernel<false><<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
+  else
+    stats_kernel<true><<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
   return cudaGetLastError();
 }
 

@@ -182,8 +182,9 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
     const int rows = static_cast<int>(min64(L.m, L.d - row0));
     const int64_t col0 = static_cast<int64_t>(crank) * L.n_c;
     const int ncols = static_cast<int>(max64(0, min64(L.n_c, L.n - col0)));
-    // RANK > 0: fixed rank; 0: any rank; < 0: A B precomputed (L.T)
-    const int r = (VARIANT == kGen) ? 1 : (RANK < 0 ? 0 : (RANK > 0 ? RANK : L.r));
+    // RANK > 0: fixed rank; 0: any rank; -1: A B precomputed (L.T); -2: any
+    // rank with an auxiliary law other than Laplace (p.dist)
+    const int r = (VARIANT == kGen) ? 1 : (RANK == -1 ? 0 : (RANK > 0 ? RANK : L.r));
     const int m = L.m;
     const int n_c = L.n_c;
     // per-layer values used inside the item loops, read once per tile
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
     if (li != cur) {
       if (tid == 0) {
         const double c = pow(*L.sigma_w / *L.sigma_r, static_cast<double>(L.alpha));
-        s_cln2 = static_cast<float>(c * kLn2);
+        s_cln2 = static_cast<float>(RANK == -2 ? c : c * kLn2);   // -2: c itself
       }
       if (VARIANT != kGen && L.b_resident) {
         for (int idx = tid; idx < r * n_c; idx += kTileThreads) {
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
           }
         }
         // T = A B on the item: precomputed on the tensor cores, or CUDA-core FMA
-        if (VARIANT != kGen && RANK < 0) {
+        if (VARIANT != kGen && RANK == -1) {
 #pragma unroll
           for (int ml = 0; ml < RPI; ++ml) {
             const float* trow = L.T + (row0 + min(w.g * RPI + ml, rows - 1)) * n;
@@ -353,11 +354,29 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
             const uint4 w4 = p.small ? philox10_small(static_cast<uint32_t>(blk0 + ml * nq), ph)
                                      : aux_block(static_cast<uint64_t>(blk0 + ml * nq), sid, p.key0, p.key1);
             words[0] = w4.x; words[1] = w4.y; words[2] = w4.z; words[3] = w4.w;
-          } else {
+          } else if (RANK != -2) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               words[c] = c < vcols ? aux_word(static_cast<uint64_t>(e0 + c), sid, p.key0, p.key1)
                                    : 0u;
+          }
+          float rv[4];                                   // RANK -2: R of each element
+          if (RANK == -2) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              if (ALIGNED) {
+                rv[c] = aux_value_generic(p.dist, words[c & 2], words[c | 1], (c & 1) != 0);
+              } else if (c < vcols) {
+                // the element's block (the Gaussian pairs words within it)
+                const uint64_t e = static_cast<uint64_t>(e0 + c);
+                const uint4 bw = aux_block(e >> 2, sid, p.key0, p.key1);
+                const uint32_t ww[4] = {bw.x, bw.y, bw.z, bw.w};
+                const int cc = static_cast<int>(e & 3u);
+                rv[c] = aux_value_generic(p.dist, ww[cc & 2], ww[cc | 1], (cc & 1) != 0);
+              } else {
+                rv[c] = 0.0f;
+              }
+            }
           }
           float sv = 0.0f;
           int32_t zv = 0;
@@ -368,14 +387,24 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
           float v[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const float lg = laplace_log2(words[c]);
-            const float cs = laplace_sign(words[c], c_ln2);   // +-c ln2
             float x;
-            if (VARIANT == kGen) {
-              x = fmaf(-lg, cs, acc[ml][c]);                   // W - R*
+            if (RANK == -2) {
+              // c_ln2 holds c: R* = c R
+              if (VARIANT == kGen) {
+                x = fmaf(-c_ln2, rv[c], acc[ml][c]);
+              } else {
+                const int32_t dcode = code_at<WBITS>(cw[ml], c) - zv;
+                x = fmaf(fmaf(c_ln2, rv[c], acc[ml][c]), rcp_tab[dcode + 255], sv);
+              }
             } else {
-              const int32_t dcode = code_at<WBITS>(cw[ml], c) - zv;
-              x = fmaf(fmaf(lg, cs, acc[ml][c]), rcp_tab[dcode + 255], sv);
+              const float lg = laplace_log2(words[c]);
+              const float cs = laplace_sign(words[c], c_ln2);   // +-c ln2
+              if (VARIANT == kGen) {
+                x = fmaf(-lg, cs, acc[ml][c]);                   // W - R*
+              } else {
+                const int32_t dcode = code_at<WBITS>(cw[ml], c) - zv;
+                x = fmaf(fmaf(lg, cs, acc[ml][c]), rcp_tab[dcode + 255], sv);
+              }
             }
             // columns past a ragged layer's end must not reach the extrema
             v[c] = (ALIGNED || c < vcols) ? x : 0.0f;
@@ -384,7 +413,8 @@ __global__ void __launch_bounds__(kTileThreads, 3) tile_kernel(const __grid_cons
           if (VARIANT != kGen) Cs[rr * quads + w.q] = cw[ml];
           if (VARIANT == kGen && r_star_out != nullptr && rr < rows) {
             for (int c = 0; c < vcols; ++c)
-              r_star_out[e0 + c] = laplace_log2(words[c]) * laplace_sign(words[c], c_ln2);
+              r_star_out[e0 + c] = RANK == -2 ? c_ln2 * rv[c]
+                                              : laplace_log2(words[c]) * laplace_sign(words[c], c_ln2);
           }
         }
       }
@@ -590,6 +620,7 @@ void by_rank(TileQuery& q, int rank_ct) {
     case 8: run_query<VARIANT, WBITS, 8, OUTB, ALIGNED>(q); break;
     case 16: run_query<VARIANT, WBITS, 16, OUTB, ALIGNED>(q); break;
     case -1: run_query<VARIANT, WBITS, -1, OUTB, ALIGNED>(q); break;
+    case -2: run_query<VARIANT, WBITS, -2, OUTB, ALIGNED>(q); break;
     default: run_query<VARIANT, WBITS, 0, OUTB, ALIGNED>(q); break;
   }
 }
@@ -597,8 +628,14 @@ void by_rank(TileQuery& q, int rank_ct) {
 template <bool ALIGNED>
 void by_variant(TileQuery& q, int variant, int w_bits, int rank_ct, int out_bytes) {
   if (variant == kGen) {
-    if (w_bits == 8) run_query<kGen, 8, 0, 1, ALIGNED>(q);
-    else run_query<kGen, 4, 0, 1, ALIGNED>(q);
+    if (rank_ct == -2) {
+      if (w_bits == 8) run_query<kGen, 8, -2, 1, ALIGNED>(q);
+      else run_query<kGen, 4, -2, 1, ALIGNED>(q);
+    } else if (w_bits == 8) {
+      run_query<kGen, 8, 0, 1, ALIGNED>(q);
+    } else {
+      run_query<kGen, 4, 0, 1, ALIGNED>(q);
+    }
   } else if (variant == kMul) {
     if (w_bits == 8) {
       if (out_bytes == 4) by_rank<kMul, 8, 4, ALIGNED>(q, rank_ct);

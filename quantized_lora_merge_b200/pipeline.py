@@ -48,13 +48,13 @@ class LayerState:
     def aux_job(self) -> B.AuxJob:
         sp = self.spec
         return B.AuxJob(self.W, sp.seed, sp.stream_id, sp.alpha, sp.w_bits, self.sigma[0:1],
-                        self.sigma[1:2], None, self.w_round, self.s, self.z)
+                        self.sigma[1:2], None, self.w_round, self.s, self.z, sp.distribution)
 
     def layer(self, pass_sigma_r: bool = True) -> B.Layer:
         sp = self.spec
         return B.Layer(self.w_round, sp.n, sp.w_bits, self.s, self.z, self.A, self.B, sp.seed,
                        sp.stream_id, sp.alpha, self.sigma[0:1],
-                       self.sigma[1:2] if pass_sigma_r else None)
+                       self.sigma[1:2] if pass_sigma_r else None, sp.distribution)
 
     def merge_out(self) -> B.MergeOut:
         return B.MergeOut(self.out, self.sbar, self.zbar if self.spec.variant == "mul" else None,

@@ -2,6 +2,7 @@
 seeded inputs, through the C ABI. Each stage is fed the oracle's inputs, so a
 difference in one stage cannot cascade into the next."""
 import numpy as np
+from dataclasses import replace
 import pytest
 import torch
 
@@ -64,7 +65,7 @@ def test_gen_aux_batched_equals_single():
 # ---------------------------------------------------------------------------
 def _oracle_prepared(spec):
     W = wl.host_W(spec)
-    g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits)
+    g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits, dist=spec.distribution)
     return dict(codes=g["codes"], s=g["s"].astype(np.float32), z=g["z"], A=wl.host_A(spec),
                 B=wl.host_B(spec), sigma_w=g["sigma_w"], sigma_r=g["sigma_r"])
 
@@ -72,7 +73,7 @@ def _oracle_prepared(spec):
 def _check_mul(spec, inp, got):
     o = oracle.merge_mul(inp["codes"], inp["s"], inp["z"], inp["A"], inp["B"], spec.seed,
                          spec.stream_id, inp["sigma_w"], inp["sigma_r"], spec.alpha,
-                         spec.out_bits)
+                         spec.out_bits, dist=spec.distribution)
     qmax = 2**spec.out_bits - 1
     assert_scale("s_bar", got["sbar"], o["sbar"])
     assert_affine("U_round", got["code"], got["zbar"], o["u_round"], o["zbar"], o["pre"],
@@ -89,7 +90,7 @@ def _check_mul(spec, inp, got):
 def _check_shift(spec, inp, got):
     o = oracle.merge_shift(inp["codes"], inp["s"], inp["z"], inp["A"], inp["B"], spec.seed,
                            spec.stream_id, inp["sigma_w"], inp["sigma_r"], spec.alpha,
-                           spec.out_bits)
+                           spec.out_bits, dist=spec.distribution)
     assert_scale("s_bar", got["sbar"], o["sbar"])
     assert_shift("shift", got["code"], o["shift"], o["pre"], 2**spec.out_bits - 1)
     D = inp["codes"].astype(np.int64) - inp["z"][:, None]
@@ -308,3 +309,56 @@ def test_batches_with_mixed_seeds():
     for spec, inp, x, y in zip(specs, inps, a, b):
         assert np.array_equal(x["out"], y["out"])
         _check_mul(spec, inp, x)
+
+
+# ---------------------------------------------------------------------------
+# auxiliary laws of the ablation (Gaussian, Cauchy, Student-t 2 dof): the
+# statistics pass and the row-tile kernels' general-law path
+# ---------------------------------------------------------------------------
+LAWS = [1, 2, 3]
+
+
+@pytest.mark.parametrize("dist", LAWS)
+@pytest.mark.parametrize("d,n,w_bits", [(64, 768, 4), (33, 100, 8), (7, 10, 4), (5, 6, 8)])
+def test_gen_aux_parity_other_laws(dist, d, n, w_bits):
+    spec = replace(spec_for(d, n, 4, w_bits, sid=d + n + dist), distribution=dist)
+    W = wl.host_W(spec)
+    g = gpu_gen_aux([spec], [W], want_r_star=True)[0]
+    o = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, w_bits, want_r_star=True, dist=dist)
+    assert_scale("sigma_w", g["sigma_w"], o["sigma_w"])
+    assert_scale("sigma_r", g["sigma_r"], o["sigma_r"])
+    assert_scale("s", g["s"], o["s"])
+    assert_affine("W_round", g["codes"], g["z"], o["codes"], o["z"], o["pre"], o["zpre"],
+                  2**w_bits - 1)
+    err = np.abs(g["r_star"].astype(np.float64) - o["r_star"])
+    assert np.max(err / np.maximum(np.abs(o["r_star"]), 1e-3 * o["c"])) < 2e-6
+
+
+@pytest.mark.parametrize("dist", LAWS)
+@pytest.mark.parametrize("d,n,r,w_bits,bits", [(40, 264, 4, 4, 4), (9, 50, 3, 8, 8), (17, 1024, 16, 8, 8)])
+def test_merge_mul_parity_other_laws(dist, d, n, r, w_bits, bits):
+    spec = replace(spec_for(d, n, r, w_bits, "mul", bits, sid=3 + d + dist), distribution=dist)
+    inp = _oracle_prepared(spec)
+    _check_mul(spec, inp, gpu_merge([spec], [inp])[0])
+
+
+@pytest.mark.parametrize("dist", LAWS)
+@pytest.mark.parametrize("d,n,r,w_bits,bits", [(24, 320, 8, 4, 4), (5, 6, 2, 4, 2)])
+def test_merge_shift_parity_other_laws(dist, d, n, r, w_bits, bits):
+    spec = replace(spec_for(d, n, r, w_bits, "shift", bits, sid=5 + d + dist), distribution=dist)
+    inp = _oracle_prepared(spec)
+    _check_shift(spec, inp, gpu_merge([spec], [inp])[0])
+
+
+def test_mixed_laws_in_one_batch():
+    """A batch mixing laws is split by law on the host: each layer equals its
+    own single-layer result, and sigma_R reduced on the device follows the law."""
+    specs = [replace(spec_for(20, 128, 4, 4, "mul", 4, sid=60 + k), distribution=k % 4)
+             for k in range(6)]
+    inps = [_oracle_prepared(s) for s in specs]
+    a = gpu_merge(specs, inps, batched=True, pass_sigma_r=False)
+    for k, spec in enumerate(specs):
+        b = gpu_merge([spec], [inps[k]], batched=False, pass_sigma_r=False)[0]
+        for key in ("out", "sbar", "zbar", "code"):
+            assert np.array_equal(a[k][key], b[key]), (spec.distribution, key)
+        _check_mul(spec, inps[k], a[k])

@@ -55,6 +55,12 @@ def parse():
                     help="int_gemm: digit planes of the merged weights (1: SHIFT of 4-bit "
                          "codes, 2: MUL of 4-bit codes, 3: MUL of 8-bit codes)")
     ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--dist", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="auxiliary law of R for every layer: 0 Laplace (the method's), 1 Gaussian, "
+                         "2 Cauchy, 3 Student-t with 2 degrees of freedom (the ablation's laws)")
+    ap.add_argument("--shard", action="store_true",
+                    help="strong scaling: split the model's layers across the ranks (greedy by "
+                         "element count) instead of giving every rank its own copy")
     return ap.parse_args()
 
 
@@ -223,14 +229,17 @@ def oracle_sample(layers, seconds):
         Gb = wl.host_G_bits(spec)
         A16, B16 = wl.to_bf16_bits(A), wl.to_bf16_bits(Bm)
         t0 = time.perf_counter()
-        g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits)
+        g = oracle.gen_aux(W, spec.seed, spec.stream_id, spec.alpha, spec.w_bits,
+                           dist=spec.distribution)
         s32 = g["s"].astype(np.float32)
         if spec.variant == "mul":
             oracle.merge_mul(g["codes"], s32, g["z"], A, Bm, spec.seed, spec.stream_id,
-                             g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits)
+                             g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits,
+                             dist=spec.distribution)
         else:
             oracle.merge_shift(g["codes"], s32, g["z"], A, Bm, spec.seed, spec.stream_id,
-                               g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits)
+                               g["sigma_w"], g["sigma_r"], spec.alpha, spec.out_bits,
+                               dist=spec.distribution)
         oracle.ste_backward(wl.bf16_bits_to_f32(Gb).astype(np.float64),
                             wl.bf16_bits_to_f32(A16).astype(np.float64),
                             wl.bf16_bits_to_f32(B16).astype(np.float64))
@@ -292,7 +301,12 @@ def main():
         return
     from quantized_lora_merge_b200 import workloads as wl
     layers_base = wl.CONFIGS[args.config]()
+    if args.dist:
+        from dataclasses import replace as _replace
+        layers_base = [_replace(l, distribution=args.dist) for l in layers_base]
     desc = workload_desc(args.config, layers_base)
+    if args.dist:
+        desc["auxiliary_law"] = ["laplace", "gaussian", "cauchy", "student_t2"][args.dist]
     if args.impl == "reference":
         run_reference(args, layers_base, desc)
         return
@@ -315,8 +329,17 @@ def main():
     from quantized_lora_merge_b200 import build as qbuild
     from quantized_lora_merge_b200 import pipeline as P
     qbuild.build()
-    # weak scaling: every rank owns its own copy of the workload (own R streams)
-    layers = [replace(l, stream_id=l.stream_id + 1000 * rank, ste=True) for l in layers_base]
+    if args.shard:
+        # strong scaling: the model's layers are split across the ranks, no
+        # collective on the data path
+        from quantized_lora_merge_b200.sharding import shard_layers
+        if world > len(layers_base):
+            raise SystemExit(f"--shard needs at most {len(layers_base)} ranks for this model")
+        owned = shard_layers([l.numel for l in layers_base], world)[rank]
+        layers = [replace(layers_base[k], ste=True) for k in owned]
+    else:
+        # weak scaling: every rank owns its own copy of the workload (own R streams)
+        layers = [replace(l, stream_id=l.stream_id + 1000 * rank, ste=True) for l in layers_base]
 
     states = []
     for spec in layers:
@@ -370,7 +393,8 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
 
-    elements = sum(l.numel for l in layers) * world
+    elements = (sum(l.numel for l in layers_base) if args.shard
+                else sum(l.numel for l in layers) * world)
     value = elements / (ms_step / 1000.0)
     hbm_peak, peak_kind = peaks()
 
@@ -397,18 +421,22 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": desc,
+        "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": dict(desc, sharding="layers split across ranks"
+                                            if args.shard else "one copy per rank"),
         "hbm_GB_s_merge": stages["merge"]["GB_s"],
         "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
-        "roofline": {"bound": "alu", "kernel": "merge team kernel (MUL, 1 launch per step)",
+        "roofline": {"bound": "alu", "kernel": ("merge team kernel (MUL, 1 launch per step)"
+                                                if not args.dist else
+                                                "merge row-tile kernel (general auxiliary law)"),
                      "achieved": alu_achieved, "peak": alu_peak, "unit": "Top/s",
                      "frac": alu_achieved / alu_peak,
                      "peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
                      "ops_per_element": merge_ops(layers[0]) / layers[0].numel,
                      "hbm_achieved_GB_s": stages["merge"]["GB_s"], "hbm_peak_GB_s": hbm_peak,
                      "hbm_peak_source": peak_kind, "hbm_frac": stages["merge"]["frac_of_hbm"],
-                     "traffic": profiled_traffic("team_kernel_mul_sd_unet")},
+                     "traffic": (profiled_traffic("team_kernel_mul_sd_unet")
+                                 if not args.dist else None)},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": args.steps * sum(launches_per_step.values()),

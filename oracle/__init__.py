@@ -381,5 +381,22 @@ def int_gemm_rows(X, x_scale, W, w_scale, rows=None):
     return Y
 
 
+def ste_mask(codes, z):
+    """[D != 0] with D = W_round - z: where the masked STE keeps G."""
+    return np.asarray(codes, np.int64) != np.asarray(z, np.int64)[:, None]
+
+
+def ste_backward_masked(G, A, B, codes, z):
+    """Masked STE: dA and dB of G (.) [W_round != z]."""
+    return ste_backward(np.asarray(G, np.float64) * ste_mask(codes, z), A, B)
+
+
+def ste_sampled_masked(G_bits, A_bits, B_bits, codes, z, rows, cols):
+    """Sampled rows of dA and columns of dB of the masked STE (bf16 inputs;
+    masked elements of G become +0)."""
+    g = np.where(ste_mask(codes, z), np.asarray(G_bits, np.uint16), np.uint16(0))
+    return ste_sampled(g, A_bits, B_bits, rows, cols)
+
+
 def num_threads() -> int:
     return int(_load().orc_num_threads())

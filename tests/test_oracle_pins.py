@@ -578,3 +578,30 @@ def test_gen_aux_and_merge_compose_under_other_laws(dist):
     nz = D != 0
     np.testing.assert_allclose((U * D)[nz], (s32.astype(np.float64)[:, None] * D + g["r_star"] + AB)[nz],
                                rtol=1e-11, atol=1e-14)
+
+
+def test_ste_masked_pins():
+    """The masked STE is the plain one on G (.) [W_round != z]: all-kept
+    equals the plain STE, all-masked gives zero, and a random mask equals
+    numpy's matmul of the masked gradient; the sampled form agrees."""
+    spec = wl.LayerSpec("t", 11, 24, 4, 4, "mul", 4, stream_id=23)
+    Gb = wl.host_G_bits(spec)
+    Ab = wl.to_bf16_bits(wl.host_A(spec))
+    Bb = wl.to_bf16_bits(wl.host_B(spec))
+    G, A, B = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+    rng = np.random.default_rng(31)
+    codes = rng.integers(0, 16, (11, 24))
+    z = rng.integers(0, 16, 11)
+    never = np.broadcast_to((z[:, None] + 1) % 16, (11, 24))        # never equal to z
+    for a, b in zip(oracle.ste_backward_masked(G, A, B, never, z), oracle.ste_backward(G, A, B)):
+        np.testing.assert_array_equal(a, b)
+    dA0, dB0 = oracle.ste_backward_masked(G, A, B, np.repeat(z[:, None], 24, axis=1), z)
+    assert not dA0.any() and not dB0.any()
+    M = (codes != z[:, None]).astype(np.float64)
+    dA, dB = oracle.ste_backward_masked(G, A, B, codes, z)
+    np.testing.assert_allclose(dA, (G * M) @ B.T, rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(dB, A.T @ (G * M), rtol=1e-12, atol=1e-18)
+    rows, cols = np.array([0, 4, 10]), np.array([1, 23])
+    sA, sB = oracle.ste_sampled_masked(Gb, Ab, Bb, codes, z, rows, cols)
+    np.testing.assert_allclose(sA, dA[rows], rtol=1e-12, atol=1e-18)
+    np.testing.assert_allclose(sB, dB[:, cols], rtol=1e-12, atol=1e-18)

@@ -286,6 +286,18 @@ typedef struct intlora_ste_job {
     int32_t r;
     float* dA;
     float* dB;
+    /* Masked STE (optional; mask_codes NULL = the plain STE above). Where
+     * D_ij = W_round_ij - z_i = 0 the adaptation term is U = s_i whatever A B
+     * is [notes, MLA, with the zero-divisor rule], so the exact derivative of
+     * the pre-quantization weight U (.) D with respect to A B is the mask
+     * [D != 0]; the masked STE uses G (.) [D != 0] in both products.
+     * mask_codes: the layer's W_round (mask_bits 4: packed nibbles, low nibble
+     * = even column; 8: bytes), row i at byte i * mask_ld, 16-byte aligned;
+     * mask_z: [d] int32 zero-points. Masked jobs run on the CUDA cores. */
+    const void* mask_codes;
+    int64_t mask_ld;
+    int32_t mask_bits;
+    const int32_t* mask_z;
 } intlora_ste_job;
 
 size_t intlora_ste_workspace_size(const intlora_ste_job* jobs, int32_t count);

@@ -55,7 +55,8 @@ class intlora_merge_out(ctypes.Structure):
 
 class intlora_ste_job(ctypes.Structure):
     _fields_ = [("G", _c_ptr), ("A", _c_ptr), ("B", _c_ptr), ("d", _c_i64), ("n", _c_i64),
-                ("r", _c_i32), ("dA", _c_ptr), ("dB", _c_ptr)]
+                ("r", _c_i32), ("dA", _c_ptr), ("dB", _c_ptr), ("mask_codes", _c_ptr),
+                ("mask_ld", _c_i64), ("mask_bits", _c_i32), ("mask_z", _c_ptr)]
 
 
 class intlora_int_gemm_job(ctypes.Structure):
@@ -222,11 +223,16 @@ class SteJob:
     B: object                       # bf16 [r, n]
     dA: object                      # fp32 [d, r]
     dB: object                      # fp32 [r, n]
+    mask_codes: object = None       # masked STE: W_round uint8 [d, ld] (None: plain STE)
+    mask_bits: int = 0
+    mask_z: object = None           # int32 [d]
 
     def to_c(self) -> intlora_ste_job:
         d, n = self.G.shape
+        ld = self.mask_codes.shape[1] if self.mask_codes is not None else 0
         return intlora_ste_job(_ptr(self.G), _ptr(self.A), _ptr(self.B), d, n, self.A.shape[1],
-                               _ptr(self.dA), _ptr(self.dB))
+                               _ptr(self.dA), _ptr(self.dB), _ptr(self.mask_codes), ld,
+                               self.mask_bits, _ptr(self.mask_z))
 
 
 @dataclass

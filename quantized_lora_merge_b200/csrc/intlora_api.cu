@@ -746,7 +746,38 @@ intlora_status check_ste(const intlora_ste_job& j, int idx) {
     return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: r must be in [1, %d]", idx, INTLORA_MAX_RANK);
   if (!aligned16(j.G) || !aligned16(j.A) || !aligned16(j.B))
     return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: G, A, B must be 16-byte aligned", idx);
+  if (j.mask_codes != nullptr) {
+    if (j.mask_bits != 4 && j.mask_bits != 8)
+      return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: mask_bits must be 4 or 8", idx);
+    if (j.mask_bits == 4 && j.n % 2 != 0)
+      return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: n must be even for 4-bit mask codes", idx);
+    const int64_t need = j.mask_bits == 8 ? j.n : j.n / 2;
+    if (j.mask_ld < need || j.mask_ld % 16 != 0 || !aligned16(j.mask_codes))
+      return fail(INTLORA_ERR_INVALID_ARG,
+                  "STE job %d: mask_codes must be 16-byte aligned with mask_ld >= %lld, a multiple of 16",
+                  idx, static_cast<long long>(need));
+    if (j.mask_z == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "STE job %d: mask_z is required", idx);
+  }
   return INTLORA_OK;
+}
+
+// The kernels' descriptor of one STE job (tiling fields left 0).
+SteJob ste_job_of(const intlora_ste_job& j) {
+  SteJob s;
+  std::memset(&s, 0, sizeof s);
+  s.G = static_cast<const uint16_t*>(j.G);
+  s.A = static_cast<const uint16_t*>(j.A);
+  s.B = static_cast<const uint16_t*>(j.B);
+  s.d = j.d;
+  s.n = j.n;
+  s.r = j.r;
+  s.dA = j.dA;
+  s.dB = j.dB;
+  s.mcodes = static_cast<const uint8_t*>(j.mask_codes);
+  s.mld = j.mask_ld;
+  s.mbits = j.mask_bits;
+  s.mz = j.mask_z;
+  return s;
 }
 
 constexpr int kSteBM = 64, kSteRB = 32, kSteTargetCtas = 148 * 4;
@@ -759,7 +790,9 @@ bool ste_tc_enabled() {
 }
 
 intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_t st) {
-  if (ste_tc_enabled()) {
+  bool masked = false;                     // masked jobs run on the CUDA cores
+  for (int32_t k = 0; k < count; ++k) masked = masked || jobs[k].mask_codes != nullptr;
+  if (ste_tc_enabled() && !masked) {
     // tensor-core pass: both products from one read of G
     SteBatch b;
     std::memset(&b, 0, sizeof b);
@@ -767,14 +800,7 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
     for (int32_t k = 0; k < count && ok; ++k) {
       const intlora_ste_job& j = jobs[k];
       SteJob& s = b.job[k];
-      s.G = static_cast<const uint16_t*>(j.G);
-      s.A = static_cast<const uint16_t*>(j.A);
-      s.B = static_cast<const uint16_t*>(j.B);
-      s.d = j.d;
-      s.n = j.n;
-      s.r = j.r;
-      s.dA = j.dA;
-      s.dB = j.dB;
+      s = ste_job_of(j);
       ok = ste_tc_supported(s);
     }
     if (ok) {
@@ -815,14 +841,7 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
     for (int32_t k = 0; k < count; ++k) {
       const intlora_ste_job& j = jobs[k];
       SteJob& s = b.job[k];
-      s.G = static_cast<const uint16_t*>(j.G);
-      s.A = static_cast<const uint16_t*>(j.A);
-      s.B = static_cast<const uint16_t*>(j.B);
-      s.d = j.d;
-      s.n = j.n;
-      s.r = j.r;
-      s.dA = j.dA;
-      s.dB = j.dB;
+      s = ste_job_of(j);
       const int64_t strips = ceil_div(j.n, 128);
       // row ranges of at least 256 rows, enough CTAs to fill the GPU a few times
       int64_t ranges = std::max<int64_t>(1, ceil_div(kSteTargetCtas * 2, strips));
@@ -845,14 +864,7 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
     for (int32_t k = 0; k < count; ++k) {
       const intlora_ste_job& j = jobs[k];
       SteJob& s = b.job[k];
-      s.G = static_cast<const uint16_t*>(j.G);
-      s.A = static_cast<const uint16_t*>(j.A);
-      s.B = static_cast<const uint16_t*>(j.B);
-      s.d = j.d;
-      s.n = j.n;
-      s.r = j.r;
-      s.dA = j.dA;
-      s.dB = j.dB;
+      s = ste_job_of(j);
       const int64_t M = dir ? j.n : j.d, K = dir ? j.d : j.n;
       const int64_t base = ceil_div(M, kSteBM) * ceil_div(j.r, kSteRB);
       int64_t ks = std::max<int64_t>(1, ceil_div(kSteTargetCtas, base));
@@ -1077,10 +1089,17 @@ intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t
     const intlora_status s = check_ste(jobs[k], k);
     if (s != INTLORA_OK) return s;
   }
-  for (int32_t k0 = 0; k0 < count; k0 += kMaxBatch) {
-    const int32_t c = std::min<int32_t>(kMaxBatch, count - k0);
-    const intlora_status s = ste_chunk(jobs + k0, c, static_cast<cudaStream_t>(stream));
-    if (s != INTLORA_OK) return s;
+  // masked and plain jobs go to separate launches (the plain ones keep the
+  // tensor-core path)
+  std::vector<intlora_ste_job> plain, masked;
+  for (int32_t k = 0; k < count; ++k) (jobs[k].mask_codes != nullptr ? masked : plain).push_back(jobs[k]);
+  for (const auto* list : {&plain, &masked}) {
+    const int32_t total = static_cast<int32_t>(list->size());
+    for (int32_t k0 = 0; k0 < total; k0 += kMaxBatch) {
+      const int32_t c = std::min<int32_t>(kMaxBatch, total - k0);
+      const intlora_status s = ste_chunk(list->data() + k0, c, static_cast<cudaStream_t>(stream));
+      if (s != INTLORA_OK) return s;
+    }
   }
   return INTLORA_OK;
 }
@@ -1088,7 +1107,7 @@ intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t
 intlora_status intlora_ste_backward(const void* G, const void* A, const void* B, int64_t d, int64_t n,
                                     int32_t r, float* dA, float* dB, void* ws, size_t ws_bytes,
                                     void* stream) {
-  intlora_ste_job j{G, A, B, d, n, r, dA, dB};
+  intlora_ste_job j{G, A, B, d, n, r, dA, dB, nullptr, 0, 0, nullptr};
   return intlora_ste_backward_batched(&j, 1, ws, ws_bytes, stream);
 }
 

@@ -162,6 +162,10 @@ struct SteJob {
   int32_t r;
   float* dA;
   float* dB;
+  const uint8_t* mcodes;     // masked STE: W_round (nullptr: no mask), row stride mld
+  int64_t mld;
+  int32_t mbits;             // 4 or 8
+  const int32_t* mz;         // zero-points: G is used only where code != z
   int64_t tile_begin;        // first CTA of this job in the grid
   int32_t ksplit;            // CTAs sharing one output tile (split reduction); fused
                              // pass: row ranges per column strip

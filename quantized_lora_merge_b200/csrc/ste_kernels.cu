@@ -31,6 +31,33 @@ __device__ __forceinline__ float bf16f(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);
 }
 
+// Masked STE: the base code of element (row, col) and whether G is kept there
+// (code != z: D != 0).
+__device__ __forceinline__ bool mask_keep(const SteJob& J, int64_t row, int64_t col) {
+  const uint8_t* rp = J.mcodes + row * J.mld;
+  const int32_t code = J.mbits == 8 ? static_cast<int32_t>(__ldg(rp + col))
+                                    : static_cast<int32_t>((__ldg(rp + (col >> 1)) >> (4 * (col & 1))) & 0xFu);
+  return code != __ldg(J.mz + row);
+}
+// The same for the 4 consecutive columns c0..c0+3 (c0 % 4 == 0) of a row,
+// applied to their bf16 values (2 per word).
+__device__ __forceinline__ uint2 mask_bf16x4(const SteJob& J, int64_t row, int64_t c0, uint2 g) {
+  const uint8_t* rp = J.mcodes + row * J.mld;
+  uint32_t codes;
+  if (J.mbits == 8) {
+    codes = __ldg(reinterpret_cast<const uint32_t*>(rp + c0));
+  } else {
+    const uint32_t h = __ldg(reinterpret_cast<const uint16_t*>(rp + (c0 >> 1)));
+    codes = (h & 0xFu) | ((h & 0xF0u) << 4) | ((h & 0xF00u) << 8) | ((h & 0xF000u) << 12);
+  }
+  const uint32_t z = static_cast<uint32_t>(__ldg(J.mz + row));
+  const uint32_t k0 = ((codes & 0xFFu) != z) ? 0x0000FFFFu : 0u;
+  const uint32_t k1 = (((codes >> 8) & 0xFFu) != z) ? 0xFFFF0000u : 0u;
+  const uint32_t k2 = (((codes >> 16) & 0xFFu) != z) ? 0x0000FFFFu : 0u;
+  const uint32_t k3 = ((codes >> 24) != z) ? 0xFFFF0000u : 0u;
+  return make_uint2(g.x & (k0 | k1), g.y & (k2 | k3));
+}
+
 template <bool TRANS>
 __global__ void __launch_bounds__(kSteThreads) ste_gemm_kernel(const __grid_constant__ SteBatch b) {
   __shared__ __align__(16) float Xs[kBK][kBM + 4];
@@ -69,7 +96,11 @@ __global__ void __launch_bounds__(kSteThreads) ste_gemm_kernel(const __grid_cons
       else { mm = idx / kBK; kk = idx % kBK; }         // coalesced along k (= G column)
       const int64_t m = m0 + mm, k = kb + kk;
       float v = 0.0f;
-      if (m < M && k < kend) v = TRANS ? bf16f(J.G[k * J.n + m]) : bf16f(J.G[m * J.n + k]);
+      if (m < M && k < kend) {
+        const int64_t row = TRANS ? k : m, col = TRANS ? m : k;
+        v = bf16f(J.G[row * J.n + col]);
+        if (J.mcodes != nullptr && !mask_keep(J, row, col)) v = 0.0f;
+      }
       Xs[kk][mm] = v;
     }
     // stage Y tile: Ys[kk][c] = Y[kb + kk][k0r + c]
@@ -216,6 +247,7 @@ __global__ void __launch_bounds__(kSteThreads, 2) ste_fused_kernel(const __grid_
       const int64_t i = i0 + u;
       graw[u] = (i < i_end && col_ok) ? __ldg(reinterpret_cast<const uint2*>(G + i * n + c0))
                                       : make_uint2(0u, 0u);
+      if (J.mcodes != nullptr && i < i_end && col_ok) graw[u] = mask_bf16x4(J, i, c0, graw[u]);
     }
 #pragma unroll
     for (int u = 0; u < RG; ++u) {

@@ -362,3 +362,71 @@ def test_mixed_laws_in_one_batch():
         for key in ("out", "sbar", "zbar", "code"):
             assert np.array_equal(a[k][key], b[key]), (spec.distribution, key)
         _check_mul(spec, inps[k], a[k])
+
+
+# ---------------------------------------------------------------------------
+# masked STE: G restricted to D = W_round - z != 0
+# ---------------------------------------------------------------------------
+def _masked_inputs(spec, w_bits):
+    Gb = wl.host_G_bits(spec)
+    Ab = wl.to_bf16_bits(wl.host_A(spec))
+    Bb = wl.to_bf16_bits(wl.host_B(spec))
+    rng = np.random.default_rng([12, spec.stream_id])
+    qmax = 2**w_bits - 1
+    z = rng.integers(0, qmax + 1, spec.d).astype(np.int32)
+    # codes near z so that a sizeable share of D is 0 (1 in 3)
+    codes = np.clip(z[:, None] + rng.integers(-1, 2, (spec.d, spec.n)), 0, qmax).astype(np.int32)
+    return Gb, Ab, Bb, codes, z
+
+
+def _gpu_ste_masked(jobs_host, w_bits):
+    jobs = []
+    for Gb, Ab, Bb, codes, z in jobs_host:
+        d, n = Gb.shape
+        r = Ab.shape[1]
+        t = [torch.from_numpy(x.view(np.int16)).to(dev()).view(torch.bfloat16) for x in (Gb, Ab, Bb)]
+        jobs.append(B.SteJob(t[0], t[1], t[2],
+                             torch.full((d, r), np.nan, dtype=torch.float32, device=dev()),
+                             torch.full((r, n), np.nan, dtype=torch.float32, device=dev()),
+                             torch.from_numpy(wl.pack_codes(codes, w_bits)).to(dev()), w_bits,
+                             torch.from_numpy(z).to(dev())))
+    B.intlora_ste_backward_batched(jobs)
+    torch.cuda.synchronize()
+    return [(j.dA.cpu().numpy(), j.dB.cpu().numpy()) for j in jobs]
+
+
+@pytest.mark.parametrize("d,n,r,w_bits", [(320, 320, 4, 4), (200, 768, 8, 8), (64, 1280, 16, 4),
+                                          (33, 50, 3, 8), (9, 1032, 33, 4), (1, 8, 1, 8)])
+def test_ste_masked_parity(d, n, r, w_bits):
+    spec = spec_for(d, n, r, w_bits, sid=70 + d)
+    h = _masked_inputs(spec, w_bits)
+    (dA, dB), = _gpu_ste_masked([h], w_bits)
+    Gb, Ab, Bb, codes, z = h
+    G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
+    oA, oB = oracle.ste_backward_masked(G, A, Bm, codes, z)
+    assert rel_fro(dA, oA) < STE_RTOL
+    assert rel_fro(dB, oB) < STE_RTOL
+    if d * n >= 1000:      # the mask matters: the plain STE is far outside the tolerance
+        pA, _ = oracle.ste_backward(G, A, Bm)
+        assert rel_fro(pA, oA) > 10 * STE_RTOL
+
+
+def test_ste_masked_and_plain_jobs_in_one_call():
+    specs = [spec_for(128, 512, 4, 4, sid=90), spec_for(96, 256, 8, 4, sid=91)]
+    hs = [_masked_inputs(s, 4) for s in specs]
+    (mA, mB), = _gpu_ste_masked([hs[0]], 4)
+    Gb, Ab, Bb, _, _ = hs[1]
+    pA, pB = gpu_ste(Gb, Ab, Bb)
+    # the same two jobs in one batched call, one masked and one plain
+    t0 = [torch.from_numpy(x.view(np.int16)).to(dev()).view(torch.bfloat16) for x in hs[0][:3]]
+    t1 = [torch.from_numpy(x.view(np.int16)).to(dev()).view(torch.bfloat16) for x in hs[1][:3]]
+    j0 = B.SteJob(t0[0], t0[1], t0[2], torch.empty((128, 4), device=dev()),
+                  torch.empty((4, 512), device=dev()),
+                  torch.from_numpy(wl.pack_codes(hs[0][3], 4)).to(dev()), 4,
+                  torch.from_numpy(hs[0][4]).to(dev()))
+    j1 = B.SteJob(t1[0], t1[1], t1[2], torch.empty((96, 8), device=dev()),
+                  torch.empty((8, 256), device=dev()))
+    B.intlora_ste_backward_batched([j0, j1])
+    torch.cuda.synchronize()
+    assert rel_fro(j0.dA.cpu().numpy(), mA) < 1e-6 and rel_fro(j0.dB.cpu().numpy(), mB) < 1e-6
+    assert rel_fro(j1.dA.cpu().numpy(), pA) < 1e-6 and rel_fro(j1.dB.cpu().numpy(), pB) < 1e-6

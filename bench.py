@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--dist", type=int, default=0, choices=[0, 1, 2, 3],
                     help="auxiliary law of R for every layer: 0 Laplace (the method's), 1 Gaussian, "
                          "2 Cauchy, 3 Student-t with 2 degrees of freedom (the ablation's laws)")
+    ap.add_argument("--masked-ste", action="store_true",
+                    help="STE backward restricted to D = W_round - z != 0 (the layers' own codes)")
     ap.add_argument("--shard", action="store_true",
                     help="strong scaling: split the model's layers across the ranks (greedy by "
                          "element count) instead of giving every rank its own copy")
@@ -307,6 +309,8 @@ def main():
     desc = workload_desc(args.config, layers_base)
     if args.dist:
         desc["auxiliary_law"] = ["laplace", "gaussian", "cauchy", "student_t2"][args.dist]
+    if args.masked_ste:
+        desc["ste"] = "masked: G kept where W_round != z"
     if args.impl == "reference":
         run_reference(args, layers_base, desc)
         return
@@ -350,7 +354,7 @@ def main():
     # them with one host<->device copy per direction
     arena_in, arena_out = P.pack_io(states, device)
     torch.cuda.empty_cache()
-    path = P.Path(states, device)
+    path = P.Path(states, device, masked_ste=args.masked_ste)
     stream = torch.cuda.current_stream(device)
 
     def barrier():
@@ -477,7 +481,7 @@ def e2e(layers, path, arena_in, arena_out, device, steps, world, elements):
                for l in layers]
     in2, out2 = P.pack_io(states2, device)
     assert in2.numel() == arena_in.numel() and out2.numel() == arena_out.numel()
-    path2 = P.Path(states2, device)
+    path2 = P.Path(states2, device, masked_ste=path.masked_ste)
     sets = [(path, arena_in, arena_out), (path2, in2, out2)]
 
     host_in = torch.empty(arena_in.numel(), dtype=torch.uint8, pin_memory=True)

@@ -293,7 +293,11 @@ typedef struct intlora_ste_job {
      * [D != 0]; the masked STE uses G (.) [D != 0] in both products.
      * mask_codes: the layer's W_round (mask_bits 4: packed nibbles, low nibble
      * = even column; 8: bytes), row i at byte i * mask_ld, 16-byte aligned;
-     * mask_z: [d] int32 zero-points. Masked jobs run on the CUDA cores. */
+     * mask_z: [d] int32 zero-points. Given the workspace that
+     * intlora_ste_workspace_size asks for (a bf16 copy of G per masked job),
+     * a masked job zeroes the masked elements into that copy and takes the
+     * plain path; without it the CUDA-core kernels apply the mask as they
+     * read G (slower, same results up to fp32 summation order). */
     const void* mask_codes;
     int64_t mask_ld;
     int32_t mask_bits;

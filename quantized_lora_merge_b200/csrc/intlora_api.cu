@@ -1073,15 +1073,15 @@ intlora_status intlora_merge_shift(const intlora_layer* layer, int32_t shift_bit
 }
 
 size_t intlora_ste_workspace_size(const intlora_ste_job* jobs, int32_t count) {
-  (void)jobs;
-  (void)count;
-  return 0;
+  // masked jobs: a bf16 copy of G with the masked elements zeroed
+  size_t total = 0;
+  for (int32_t k = 0; k < count && jobs != nullptr; ++k)
+    if (jobs[k].mask_codes != nullptr) total += round256(static_cast<size_t>(jobs[k].d * jobs[k].n) * 2);
+  return total;
 }
 
 intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t count, void* ws,
                                             size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   g_last_error[0] = '\0';
   if (count < 0 || (count > 0 && jobs == nullptr))
     return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
@@ -1090,9 +1090,35 @@ intlora_status intlora_ste_backward_batched(const intlora_ste_job* jobs, int32_t
     if (s != INTLORA_OK) return s;
   }
   // masked and plain jobs go to separate launches (the plain ones keep the
-  // tensor-core path)
+  // tensor-core path). With the workspace of intlora_ste_workspace_size the
+  // masked jobs become plain jobs on a masked copy of G; without it they run
+  // on the CUDA-core kernels, which apply the mask as they read G.
   std::vector<intlora_ste_job> plain, masked;
-  for (int32_t k = 0; k < count; ++k) (jobs[k].mask_codes != nullptr ? masked : plain).push_back(jobs[k]);
+  const size_t need = intlora_ste_workspace_size(jobs, count);
+  const bool copy = need > 0 && ws != nullptr && ws_bytes >= need && aligned16(ws);
+  std::vector<MaskJob> mjobs;
+  char* wp = static_cast<char*>(ws);
+  for (int32_t k = 0; k < count; ++k) {
+    if (jobs[k].mask_codes == nullptr) {
+      plain.push_back(jobs[k]);
+    } else if (copy) {
+      intlora_ste_job j = jobs[k];
+      MaskJob m{static_cast<const uint16_t*>(j.G), reinterpret_cast<uint16_t*>(wp),
+                static_cast<const uint8_t*>(j.mask_codes), j.mask_ld, j.mask_bits, j.mask_z, j.d, j.n};
+      mjobs.push_back(m);
+      j.G = wp;
+      j.mask_codes = nullptr;
+      plain.push_back(j);
+      wp += round256(static_cast<size_t>(j.d * j.n) * 2);
+    } else {
+      masked.push_back(jobs[k]);
+    }
+  }
+  if (!mjobs.empty()) {
+    const cudaError_t e = launch_mask_g(mjobs.data(), static_cast<int>(mjobs.size()),
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "STE mask launch");
+  }
   for (const auto* list : {&plain, &masked}) {
     const int32_t total = static_cast<int32_t>(list->size());
     for (int32_t k0 = 0; k0 < total; k0 += kMaxBatch) {

@@ -188,6 +188,18 @@ cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_by
 int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s);   // dA and dB of every job
+// Masked STE with a workspace: G' = G where W_round != z, else 0 (bf16 copy),
+// after which the plain (tensor-core) path runs on G'.
+struct MaskJob {
+  const uint16_t* G;
+  uint16_t* out;
+  const uint8_t* codes;
+  int64_t ld;
+  int32_t bits;
+  const int32_t* z;
+  int64_t d, n;
+};
+cudaError_t launch_mask_g(const MaskJob* jobs, int count, cudaStream_t s);
 // tcgen05 path of the STE backward (one pass over G, both products on the
 // tensor cores); outputs must be zeroed first.
 constexpr int kSteTcMaxRank = 128;

@@ -331,6 +331,92 @@ __global__ void __launch_bounds__(256) zero_segments_kernel(const __grid_constan
 
 }  // namespace
 
+namespace {
+constexpr int kMaskChunk = 256 * 8;      // octets per CTA step
+
+struct MaskBatch {
+  MaskJob job[kMaxBatch];
+  int64_t chunk_begin[kMaxBatch + 1];     // CTA steps before job k
+  int32_t count;
+};
+
+// Octets (8 consecutive elements of a row) in chunks of kMaskChunk, each
+// chunk inside one job: a 16-byte load of G and of its codes' bytes when the
+// row allows it, else element by element.
+__global__ void __launch_bounds__(256) mask_g_kernel(const __grid_constant__ MaskBatch b) {
+  const int64_t total = b.chunk_begin[b.count];
+  int k = 0;
+  for (int64_t c = blockIdx.x; c < total; c += gridDim.x) {
+    while (k + 1 < b.count && b.chunk_begin[k + 1] <= c) ++k;       // chunks only increase
+    const MaskJob& J = b.job[k];
+    const int64_t per_row = (J.n + 7) / 8;
+    const int64_t octets = J.d * per_row;
+    const int64_t o_begin = (c - b.chunk_begin[k]) * kMaskChunk;
+    const int64_t o_end = min64(octets, o_begin + kMaskChunk);
+    for (int64_t o = o_begin + threadIdx.x; o < o_end; o += blockDim.x) {
+      const int64_t i = o / per_row;
+      const int64_t j0 = (o - i * per_row) * 8;
+      const uint8_t* crow = J.codes + i * J.ld;
+      const uint32_t z = static_cast<uint32_t>(__ldg(J.z + i));
+      const uint16_t* src = J.G + i * J.n + j0;
+      uint16_t* dst = J.out + i * J.n + j0;
+      if (J.n % 8 == 0) {
+        uint4 g = __ldg(reinterpret_cast<const uint4*>(src));
+        uint32_t c[8];
+        if (J.bits == 8) {
+          const uint2 cb = __ldg(reinterpret_cast<const uint2*>(crow + j0));
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            c[q] = (cb.x >> (8 * q)) & 0xFFu;
+            c[q + 4] = (cb.y >> (8 * q)) & 0xFFu;
+          }
+        } else {
+          const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(crow + (j0 >> 1)));
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) c[q] = (cw >> (4 * q)) & 0xFu;
+        }
+        uint32_t* gw = reinterpret_cast<uint32_t*>(&g);
+  #pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t lo = c[2 * q] != z ? 0x0000FFFFu : 0u;
+          const uint32_t hi = c[2 * q + 1] != z ? 0xFFFF0000u : 0u;
+          gw[q] &= lo | hi;
+        }
+        *reinterpret_cast<uint4*>(dst) = g;
+      } else {
+        for (int q = 0; q < 8 && j0 + q < J.n; ++q) {
+          const int64_t j = j0 + q;
+          const uint32_t code = J.bits == 8 ? crow[j] : (crow[j >> 1] >> (4 * (j & 1))) & 0xFu;
+          dst[q] = code != z ? src[q] : static_cast<uint16_t>(0);
+        }
+      }
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_mask_g(const MaskJob* jobs, int count, cudaStream_t s) {
+  static thread_local MaskBatch b;
+  for (int k0 = 0; k0 < count; k0 += kMaxBatch) {
+    const int m = count - k0 < kMaxBatch ? count - k0 : kMaxBatch;
+    std::memset(&b, 0, sizeof b);
+    int64_t chunks = 0;
+    for (int k = 0; k < m; ++k) {
+      b.job[k] = jobs[k0 + k];
+      b.chunk_begin[k] = chunks;
+      chunks += (jobs[k0 + k].d * ((jobs[k0 + k].n + 7) / 8) + kMaskChunk - 1) / kMaskChunk;
+    }
+    b.chunk_begin[m] = chunks;
+    b.count = m;
+    if (chunks == 0) continue;
+    const int64_t blocks = min64(chunks, 148 * 8);
+    mask_g_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(b);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s) {
   if (b.count <= 0) return cudaSuccess;
   ZeroBatch z;

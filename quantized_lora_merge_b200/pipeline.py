@@ -60,7 +60,11 @@ class LayerState:
         return B.MergeOut(self.out, self.sbar, self.zbar if self.spec.variant == "mul" else None,
                           self.code)
 
-    def ste_job(self) -> B.SteJob:
+    def ste_job(self, masked: bool = False) -> B.SteJob:
+        """masked: G is kept only where W_round != z (the layer's own codes)."""
+        if masked:
+            return B.SteJob(self.G, self.A16, self.B16, self.dA, self.dB, self.w_round,
+                            self.spec.w_bits, self.z)
         return B.SteJob(self.G, self.A16, self.B16, self.dA, self.dB)
 
 
@@ -131,9 +135,10 @@ class Path:
     quantization), merge (MUL or SHIFT) and, where requested, the STE
     backward; each stage is one batched call (a handful of launches)."""
 
-    def __init__(self, states: list[LayerState], device):
+    def __init__(self, states: list[LayerState], device, masked_ste: bool = False):
         self.states = states
         self.device = device
+        self.masked_ste = masked_ste
         self.mul = [s for s in states if s.spec.variant == "mul"]
         self.shift = [s for s in states if s.spec.variant == "shift"]
         self.ste = [s for s in states if s.G is not None]
@@ -150,7 +155,10 @@ class Path:
         self.merge_groups = [(kind, bits, B.Descriptors(s.layer() for s in sts),
                               B.Descriptors(s.merge_out() for s in sts))
                              for (kind, bits), sts in groups.items()]
-        self.ste_jobs = B.Descriptors(s.ste_job() for s in self.ste) if self.ste else None
+        self.ste_jobs = (B.Descriptors(s.ste_job(masked_ste) for s in self.ste)
+                         if self.ste else None)
+        self.ws_ste = (workspace(B.intlora_ste_workspace_size(self.ste_jobs), device)
+                       if self.ste else None)
 
     def prepare(self, stream=None):
         B.intlora_gen_aux_batched(self.aux_jobs, self.ws_aux, stream)
@@ -164,7 +172,7 @@ class Path:
 
     def backward(self, stream=None):
         if self.ste_jobs is not None:
-            B.intlora_ste_backward_batched(self.ste_jobs, None, stream)
+            B.intlora_ste_backward_batched(self.ste_jobs, self.ws_ste, stream)
 
     def step(self, stream=None):
         self.prepare(stream)

@@ -8,6 +8,7 @@ import torch
 
 import oracle
 from quantized_lora_merge_b200 import binding as B
+from quantized_lora_merge_b200 import pipeline as P
 from quantized_lora_merge_b200 import workloads as wl
 
 from .parity import (STE_RTOL, assert_affine, assert_scale, assert_shift, dev, gpu_gen_aux,
@@ -379,7 +380,7 @@ def _masked_inputs(spec, w_bits):
     return Gb, Ab, Bb, codes, z
 
 
-def _gpu_ste_masked(jobs_host, w_bits):
+def _gpu_ste_masked(jobs_host, w_bits, with_ws=True):
     jobs = []
     for Gb, Ab, Bb, codes, z in jobs_host:
         d, n = Gb.shape
@@ -390,17 +391,21 @@ def _gpu_ste_masked(jobs_host, w_bits):
                              torch.full((r, n), np.nan, dtype=torch.float32, device=dev()),
                              torch.from_numpy(wl.pack_codes(codes, w_bits)).to(dev()), w_bits,
                              torch.from_numpy(z).to(dev())))
-    B.intlora_ste_backward_batched(jobs)
+    # with the workspace: a masked copy of G on the plain (tensor-core) path;
+    # without: the CUDA-core kernels mask G as they read it
+    ws = P.workspace(B.intlora_ste_workspace_size(jobs), dev()) if with_ws else None
+    B.intlora_ste_backward_batched(jobs, ws)
     torch.cuda.synchronize()
     return [(j.dA.cpu().numpy(), j.dB.cpu().numpy()) for j in jobs]
 
 
 @pytest.mark.parametrize("d,n,r,w_bits", [(320, 320, 4, 4), (200, 768, 8, 8), (64, 1280, 16, 4),
                                           (33, 50, 3, 8), (9, 1032, 33, 4), (1, 8, 1, 8)])
-def test_ste_masked_parity(d, n, r, w_bits):
+@pytest.mark.parametrize("with_ws", [True, False])
+def test_ste_masked_parity(d, n, r, w_bits, with_ws):
     spec = spec_for(d, n, r, w_bits, sid=70 + d)
     h = _masked_inputs(spec, w_bits)
-    (dA, dB), = _gpu_ste_masked([h], w_bits)
+    (dA, dB), = _gpu_ste_masked([h], w_bits, with_ws)
     Gb, Ab, Bb, codes, z = h
     G, A, Bm = (wl.bf16_bits_to_f32(x).astype(np.float64) for x in (Gb, Ab, Bb))
     oA, oB = oracle.ste_backward_masked(G, A, Bm, codes, z)

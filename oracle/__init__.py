@@ -81,6 +81,8 @@ def _load():
                                       _dbl, _int, _i64, _i64, _ptr, _ptr, _ptr, _ptr, _ptr,
                                       _ptr, _int]),
         "orc_int_digits": (_i64, [_ptr, _i64, _i64, _int, _ptr]),
+        "orc_fakequant_bf16": (None, [_ptr, _ptr, _i64, _i64, _ptr]),
+        "orc_linear_rows": (None, [_ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_int_gemm_rows": (None, [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_num_threads": (_int, []),
     }
@@ -396,6 +398,31 @@ def ste_sampled_masked(G_bits, A_bits, B_bits, codes, z, rows, cols):
     masked elements of G become +0)."""
     g = np.where(ste_mask(codes, z), np.asarray(G_bits, np.uint16), np.uint16(0))
     return ste_sampled(g, A_bits, B_bits, rows, cols)
+
+
+# --------------------------------------------------------------------------
+# Training forward on the merged weights
+# --------------------------------------------------------------------------
+def fakequant_bf16(Q, sbar):
+    """bf16 bit patterns of fp32(sbar_i * Q_ij)."""
+    q = _c(Q, np.int64)
+    sb = _c(sbar, np.float32)
+    d, n = q.shape
+    out = np.zeros((d, n), np.uint16)
+    _load().orc_fakequant_bf16(_p(q), _p(sb), d, n, _p(out))
+    return out
+
+
+def linear_rows(X_bits, W_bits, rows=None):
+    """Y rows (fp64) of X W^T for bf16 patterns X (tokens x n), W (d x n)."""
+    x = _c(X_bits, np.uint16)
+    w = _c(W_bits, np.uint16)
+    tokens, n = x.shape
+    d = w.shape[0]
+    rw = _c(np.arange(tokens) if rows is None else rows, np.int64)
+    Y = np.zeros((rw.size, d), np.float64)
+    _load().orc_linear_rows(_p(x), _p(w), tokens, d, n, _p(rw), rw.size, _p(Y))
+    return Y
 
 
 def num_threads() -> int:

@@ -577,6 +577,50 @@ void orc_int_gemm_rows(const int8_t* X, const double* x_scale, const int64_t* W,
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Training forward on the merged weights [IntLoRA notes, 两种实现版本 and    */
+/* the efficiency table]: the merged weight enters the layer GEMM as bf16.   */
+/* ------------------------------------------------------------------------ */
+
+/* bf16 of an fp32 value: round to nearest with ties to even on the upper 16
+ * bits of the pattern (finite values). */
+static uint16_t bf16_rne(float f) {
+    uint32_t b;
+    memcpy(&b, &f, sizeof b);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return (uint16_t)(b >> 16);
+}
+
+/* W'_bf16[i][j] = bf16(fp32(s_bar_i * Q_ij)): the fp32 product, then bf16. */
+void orc_fakequant_bf16(const int64_t* Q, const float* sbar, int64_t d, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < d; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            float w = sbar[i] * (float)Q[i * n + j];
+            out[i * n + j] = bf16_rne(w);
+        }
+}
+
+static double bf16_to_f64(uint16_t h) {
+    uint32_t b = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &b, sizeof f);
+    return (double)f;
+}
+
+/* Y[t][i] = sum_j X[t][j] W[i][j] in fp64 for the listed token rows (X, W
+ * bf16 patterns). */
+void orc_linear_rows(const uint16_t* X, const uint16_t* W, int64_t tokens, int64_t d, int64_t n,
+                     const int64_t* rows, int64_t n_rows, double* Y) {
+    (void)tokens;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t q = 0; q < n_rows * d; ++q) {
+        int64_t t = rows[q / d], i = q % d;
+        double acc = 0.0;
+        for (int64_t j = 0; j < n; ++j) acc += bf16_to_f64(X[t * n + j]) * bf16_to_f64(W[i * n + j]);
+        Y[q] = acc;
+    }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -605,3 +605,48 @@ def test_ste_masked_pins():
     sA, sB = oracle.ste_sampled_masked(Gb, Ab, Bb, codes, z, rows, cols)
     np.testing.assert_allclose(sA, dA[rows], rtol=1e-12, atol=1e-18)
     np.testing.assert_allclose(sB, dB[:, cols], rtol=1e-12, atol=1e-18)
+
+
+# ---------------------------------------------------------------------------
+# training forward: fake-quantized bf16 merged weight and the layer GEMM
+# ---------------------------------------------------------------------------
+def _bf16_nearest_even(x32):
+    """bf16 pattern of an fp32 value by exact comparison with its two bf16
+    neighbours (ties to the even pattern)."""
+    bits = int(np.float32(x32).view(np.uint32))
+    lo = bits >> 16
+    hi = lo + 1
+    val = Fraction(float(np.float32(x32)))
+    f = lambda p: Fraction(float(np.array([p << 16], np.uint32).view(np.float32)[0]))
+    dl, dh = abs(val - f(lo)), abs(f(hi) - val)
+    if dl < dh or (dl == dh and lo % 2 == 0):
+        return lo
+    return hi
+
+
+def test_fakequant_bf16_rounding_brute_force():
+    rng = np.random.default_rng(17)
+    Q = rng.integers(-65025, 65026, (6, 40))
+    sbar = rng.uniform(1e-5, 1e-2, 6).astype(np.float32)
+    Q[0, :3] = [0, 1, -1]
+    got = oracle.fakequant_bf16(Q, sbar)
+    for i in range(6):
+        for j in range(40):
+            prod = np.float32(sbar[i]) * np.float32(Q[i, j])      # one fp32 rounding
+            assert got[i, j] == _bf16_nearest_even(prod)
+    # exact ties: 1 + 2^-8 (+ 2^-7) sit halfway between bf16 neighbours
+    ties = oracle.fakequant_bf16(np.array([[257, 259]]), np.array([2.0**-8], np.float32))
+    assert ties.tolist() == [[0x3F80, 0x3F82]]
+
+
+def test_linear_rows_brute_force_and_numpy():
+    rng = np.random.default_rng(18)
+    X = wl.to_bf16_bits(rng.standard_normal((3, 16)).astype(np.float32))
+    W = wl.to_bf16_bits(rng.standard_normal((5, 16)).astype(np.float32))
+    Y = oracle.linear_rows(X, W)
+    xf, wf = wl.bf16_bits_to_f32(X).astype(np.float64), wl.bf16_bits_to_f32(W).astype(np.float64)
+    for t in range(3):
+        for i in range(5):
+            assert abs(Y[t, i] - sum(float(xf[t, j]) * float(wf[i, j]) for j in range(16))) < 1e-12
+    np.testing.assert_allclose(Y, xf @ wf.T, rtol=1e-13, atol=1e-13)
+    np.testing.assert_array_equal(oracle.linear_rows(X, W, rows=[2]), Y[[2]])

@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--op", default="step", choices=["step", "int_gemm"],
+    ap.add_argument("--op", default="step", choices=["step", "int_gemm", "train_forward"],
                     help="step: the merge hot path (default); int_gemm: the integer "
                          "inference GEMM on merged weights")
     ap.add_argument("--planes", type=int, default=1, choices=[1, 2, 3],
@@ -300,6 +300,9 @@ def main():
     args = parse()
     if args.op == "int_gemm":
         bench_int_gemm(args)
+        return
+    if args.op == "train_forward":
+        bench_train_forward(args)
         return
     from quantized_lora_merge_b200 import workloads as wl
     layers_base = wl.CONFIGS[args.config]()
@@ -678,6 +681,97 @@ def bench_int_gemm(args):
                                 "sample": f"{rows} token rows of the qkv GEMM "
                                           f"({GEMM_SHAPES[0][0]}x{GEMM_SHAPES[0][1]}), "
                                           f"exact int64 sums, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# training forward on merged weights (--op train_forward)
+# ---------------------------------------------------------------------------
+def bench_train_forward(args):
+    """One step = the training forward of every SD-UNet linear at `tokens`
+    tokens: the MUL merge (all layers, one batched call), the bf16
+    fake-quantization of the merged weights, and Y = X W'^T for every layer
+    (batched bf16 GEMMs on the tensor cores). Metric: GEMM TFLOP/s of the
+    whole step (2 tokens d n per layer over the step time)."""
+    import torch
+
+    from quantized_lora_merge_b200 import binding as B
+    from quantized_lora_merge_b200 import build as qbuild
+    from quantized_lora_merge_b200 import pipeline as P
+    from quantized_lora_merge_b200 import workloads as wl
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    qbuild.build()
+    T = args.tokens
+    layers = wl.CONFIGS["sd_unet"]()
+    states = []
+    for spec in layers:
+        t = wl.device_inputs(spec, device, salt=0)
+        states.append(P.allocate(spec, t["W"], t["A"], t["B"], device))
+    path = P.Path(states, device)
+    path.prepare()
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    wq = [torch.empty(l.d, l.n, dtype=torch.bfloat16, device=device) for l in layers]
+    lin = B.Descriptors(B.LinearJob(torch.randn(T, l.n, generator=g, device=device).to(torch.bfloat16),
+                                    w, torch.empty(T, l.d, device=device)) for l, w in zip(layers, wq))
+    stream = torch.cuda.current_stream(device)
+
+    fq = B.Descriptors(B.FakeQuantJob(st.out, st.sbar, w) for st, w in zip(states, wq))
+
+    def step():
+        path.merge()
+        B.intlora_fakequant_bf16_batched(fq)
+        B.intlora_linear_bf16_batched(lin)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    steps = args.steps if args.steps != 1000 else 20
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gemm_ms = 0.0
+    torch.cuda.synchronize(device)
+    a.record(stream)
+    for _ in range(steps):
+        path.merge()
+        ev[0].record(stream)
+        B.intlora_fakequant_bf16_batched(fq)
+        ev[1].record(stream)
+        B.intlora_linear_bf16_batched(lin)
+        ev[2].record(stream)
+        ev[2].synchronize()
+        gemm_ms += ev[1].elapsed_time(ev[2])
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    ms = a.elapsed_time(b) / steps
+    gemm_ms /= steps
+    flops = sum(2 * T * l.d * l.n for l in layers)
+    bf16, kind = bf16_peak_tflops()
+    gemm_tf = flops / (gemm_ms / 1e3) / 1e12
+    line = {
+        "metric": "training forward on merged weights: GEMM TFLOP/s per step (bf16), 1 GPU",
+        "value": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
+        "config": {"workload": f"SD-UNet 128 linears at {T} tokens: MUL merge (4-bit) + bf16 "
+                               f"fake-quantization + Y = X W'^T per layer", "tokens": T},
+        "gemm_ms": gemm_ms,
+        "roofline": {"bound": "tensor", "kernel": "int_gemm_kernel<0> (tcgen05 kind::f16)",
+                     "achieved": gemm_tf, "peak": bf16, "unit": "TFLOP/s", "frac": gemm_tf / bf16,
+                     "peak_source": f"{kind} bf16 dense", "traffic": None},
+        "clocks": clk,
+        "gpu_launches": steps * (2 + (len(layers) + 47) // 48),
+    }
     print(json.dumps(line), flush=True)
 
 

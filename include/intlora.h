@@ -364,6 +364,46 @@ intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int
                                 const float* w_scale, int64_t tokens, int64_t d, int64_t n,
                                 int32_t planes, float* Y, void* stream);
 
+/* --------------------------------------------------------------------------
+ * Training forward on the merged weights [notes, 两种实现版本 and the
+ * efficiency table: IntLoRA trains with the merged weight quantized in the
+ * forward pass (fake quantization) and the STE in the backward]:
+ *
+ *   W'_bf16 = bf16(fp32(s_bar_i) * Q_ij)          (intlora_fakequant_bf16)
+ *   Y = X W'^T,  X bf16 tokens x n, fp32 accumulation, Y fp32 tokens x d
+ *                                                 (intlora_linear_bf16_batched)
+ *
+ * Q: the merge output (q_bytes 1, 2 or 4); the product is rounded once to
+ * fp32 and then to bf16 (nearest, ties to even). The GEMM runs on the tensor
+ * cores (tcgen05 kind::f16, the integer GEMM's pipeline with bf16 operands).
+ * Requirements: n % 8 == 0; X, W, Y, w_out 16-byte aligned. Y is
+ * overwritten (zero when n = 0). Asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+intlora_status intlora_fakequant_bf16(const void* q, int32_t q_bytes, const float* sbar, int64_t d,
+                                      int64_t n, void* w_out, void* stream);
+
+typedef struct intlora_fakequant_job {
+    const void* q;            /* merged integer weights, d x n, 16-byte aligned */
+    int32_t q_bytes;          /* 1, 2 or 4 */
+    const float* sbar;        /* [d] */
+    int64_t d, n;
+    void* w_out;              /* bf16 d x n, 16-byte aligned */
+} intlora_fakequant_job;
+
+/* Many layers in one launch. */
+intlora_status intlora_fakequant_bf16_batched(const intlora_fakequant_job* jobs, int32_t count,
+                                              void* stream);
+
+typedef struct intlora_linear_job {
+    const void* X;            /* bf16 tokens x n */
+    const void* W;            /* bf16 d x n (the fake-quantized merged weight) */
+    int64_t tokens, d, n;
+    float* Y;                 /* tokens x d */
+} intlora_linear_job;
+
+intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32_t count,
+                                           void* stream);
+
 /* Number of bounded device-side waits that gave up since the library was
  * loaded: 0 in a healthy run. The tensor-core STE kernel bounds every wait on
  * an mbarrier (2 s); a wait that gives up is counted here, the CTA stops, releases its

@@ -59,6 +59,16 @@ class intlora_ste_job(ctypes.Structure):
                 ("mask_ld", _c_i64), ("mask_bits", _c_i32), ("mask_z", _c_ptr)]
 
 
+class intlora_fakequant_job(ctypes.Structure):
+    _fields_ = [("q", _c_ptr), ("q_bytes", _c_i32), ("sbar", _c_ptr), ("d", _c_i64), ("n", _c_i64),
+                ("w_out", _c_ptr)]
+
+
+class intlora_linear_job(ctypes.Structure):
+    _fields_ = [("X", _c_ptr), ("W", _c_ptr), ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64),
+                ("Y", _c_ptr)]
+
+
 class intlora_int_gemm_job(ctypes.Structure):
     _fields_ = [("X", _c_ptr), ("x_scale", _c_ptr), ("W", _c_ptr), ("w_scale", _c_ptr),
                 ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("Y", _c_ptr)]
@@ -95,6 +105,10 @@ _SIGNATURES = {
     "intlora_ste_backward_batched": (ctypes.c_int, [_P(intlora_ste_job), _c_i32, _c_ptr,
                                                     _c_size, _c_ptr]),
     "intlora_int_planes": (_c_i32, [_c_i64]),
+    "intlora_fakequant_bf16": (ctypes.c_int, [_c_ptr, _c_i32, _c_ptr, _c_i64, _c_i64, _c_ptr,
+                                              _c_ptr]),
+    "intlora_linear_bf16_batched": (ctypes.c_int, [_P(intlora_linear_job), _c_i32, _c_ptr]),
+    "intlora_fakequant_bf16_batched": (ctypes.c_int, [_P(intlora_fakequant_job), _c_i32, _c_ptr]),
     "intlora_int_pack": (ctypes.c_int, [_c_ptr, _c_i32, _c_i64, _c_i64, _c_i32, _c_ptr, _c_ptr,
                                         _c_ptr]),
     "intlora_int_gemm_batched": (ctypes.c_int, [_P(intlora_int_gemm_job), _c_i32, _c_i32,
@@ -249,6 +263,30 @@ class IntGemmJob:
                                     _ptr(self.w_scale), tokens, self.W.shape[0], n, _ptr(self.Y))
 
 
+@dataclass
+class FakeQuantJob:
+    q: object                       # merged integer weights [d, n] (int8/int16/int32)
+    sbar: object                    # fp32 [d]
+    w_out: object                   # bf16 [d, n]
+
+    def to_c(self) -> intlora_fakequant_job:
+        d, n = self.q.shape
+        return intlora_fakequant_job(_ptr(self.q), self.q.element_size(), _ptr(self.sbar), d, n,
+                                     _ptr(self.w_out))
+
+
+@dataclass
+class LinearJob:
+    X: object                       # bf16 [tokens, n]
+    W: object                       # bf16 [d, n]
+    Y: object                       # fp32 [tokens, d]
+
+    def to_c(self) -> intlora_linear_job:
+        tokens, n = self.X.shape
+        return intlora_linear_job(_ptr(self.X), _ptr(self.W), tokens, self.W.shape[0], n,
+                                  _ptr(self.Y))
+
+
 def _array(struct, items):
     if isinstance(items, Descriptors):
         if items.struct is not struct:
@@ -285,7 +323,8 @@ class Descriptors:
 
 Descriptors._STRUCT = {AuxJob: intlora_aux_job, Layer: intlora_layer,
                        MergeOut: intlora_merge_out, SteJob: intlora_ste_job,
-                       IntGemmJob: intlora_int_gemm_job}
+                       IntGemmJob: intlora_int_gemm_job, LinearJob: intlora_linear_job,
+                       FakeQuantJob: intlora_fakequant_job}
 
 
 # ---------------------------------------------------------------------------
@@ -404,3 +443,20 @@ def intlora_int_gemm(job: IntGemmJob, planes: int, stream=None) -> None:
     c = job.to_c()
     _check(lib().intlora_int_gemm(c.X, c.x_scale, c.W, c.w_scale, c.tokens, c.d, c.n, planes,
                                   c.Y, _stream(stream)))
+
+
+def intlora_fakequant_bf16(q, sbar, w_out, stream=None) -> None:
+    """w_out (bf16 [d, n]) = bf16(fp32(sbar_i) * q_ij) for merged weights q."""
+    d, n = q.shape
+    _check(lib().intlora_fakequant_bf16(_ptr(q), q.element_size(), _ptr(sbar), d, n, _ptr(w_out),
+                                        _stream(stream)))
+
+
+def intlora_linear_bf16_batched(jobs: Sequence[LinearJob], stream=None) -> None:
+    _check(lib().intlora_linear_bf16_batched(_array(intlora_linear_job, jobs), len(jobs),
+                                             _stream(stream)))
+
+
+def intlora_fakequant_bf16_batched(jobs: Sequence[FakeQuantJob], stream=None) -> None:
+    _check(lib().intlora_fakequant_bf16_batched(_array(intlora_fakequant_job, jobs), len(jobs),
+                                                _stream(stream)))

@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cuda_bf16.h>
+
 #include <cstdint>
 #include <cstring>
 
@@ -109,16 +111,23 @@ __device__ __forceinline__ uint32_t ig_idesc(int nrows) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nrows >> 3) << 17) |
          (static_cast<uint32_t>(kIgRows >> 4) << 24);
 }
+// kind::f16: D f32, A and B bf16, both K-major, M = 128, N = nrows.
+__device__ __forceinline__ uint32_t ig_idesc_bf16(int nrows) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nrows >> 3) << 17) |
+         (static_cast<uint32_t>(kIgRows >> 4) << 24);
+}
 
 // One 16-channel block of a tile for the calling warp's 32 rows (t = this
 // lane's row). ystage: the warp's shared-memory buffer for a TMA store, or
 // nullptr for direct stores.
+// P = 0: the bf16 GEMM (fp32 accumulators, no scales).
 template <int P>
 __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J, int64_t t, float xs,
                                                   int64_t i, bool row_ok, uint8_t* ystage, int lane) {
-  float raw[16 * P];
+  constexpr int NP = P == 0 ? 1 : P;
+  float raw[16 * NP];
 #pragma unroll
-  for (int q = 0; q < P; ++q) tmem_ld16(taddr + static_cast<uint32_t>(16 * q), raw + 16 * q);
+  for (int q = 0; q < NP; ++q) tmem_ld16(taddr + static_cast<uint32_t>(16 * q), raw + 16 * q);
   tmem_ld_wait();
   if (i >= J.d) return;                                  // warp-uniform
   if (ystage == nullptr ? !row_ok : t - lane >= J.tokens) return;   // no row of the block in Y
@@ -126,7 +135,9 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
     float v;
-    if (P == 1) {
+    if (P == 0) {
+      v = raw[c];
+    } else if (P == 1) {
       v = static_cast<float>(__float_as_int(raw[c]));
     } else {
       int64_t s = 0;
@@ -137,7 +148,10 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
     y[c] = v;
   }
   float ws[16];
-  if (i + 16 <= J.d && (reinterpret_cast<uintptr_t>(J.w_scale) & 15u) == 0) {
+  if (P == 0) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) ws[c] = 1.0f;
+  } else if (i + 16 <= J.d && (reinterpret_cast<uintptr_t>(J.w_scale) & 15u) == 0) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 w4 = __ldg(reinterpret_cast<const float4*>(J.w_scale + i) + q);
@@ -150,8 +164,10 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
 #pragma unroll
     for (int c = 0; c < 16; ++c) ws[c] = i + c < J.d ? __ldg(J.w_scale + i + c) : 0.0f;
   }
+  if (P != 0) {
 #pragma unroll
-  for (int c = 0; c < 16; ++c) y[c] *= xs * ws[c];
+    for (int c = 0; c < 16; ++c) y[c] *= xs * ws[c];
+  }
   if (ystage != nullptr) {
     // the buffer's previous store (two blocks ago) has finished reading it
     if (lane == 0) bulk_wait_read<1>();
@@ -192,7 +208,9 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
   __shared__ volatile int abort_flag;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   const int S = b.stages;
-  const int nrows = P * b.chans;                        // digit rows of a tile
+  constexpr int NP = P == 0 ? 1 : P;                    // P = 0: bf16 operands
+  constexpr int kElems = P == 0 ? kIgK / 2 : kIgK;      // K elements per stage
+  const int nrows = NP * b.chans;                       // digit rows of a tile
   const uint32_t b_bytes = static_cast<uint32_t>(nrows) * kIgK;
   const uint32_t stage_bytes = kIgABytes + b_bytes;     // multiple of 1024
   uint8_t* ystage = base + S * stage_bytes;              // [8 warps][2][32 x 16 fp32]
@@ -235,7 +253,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
         const IgTile x = ig_tile(b, u);
         const IgJob& J = b.job[x.job];
         const int32_t ty = static_cast<int32_t>(x.t0);
-        const int32_t wy = static_cast<int32_t>(x.i0 * P);
+        const int32_t wy = static_cast<int32_t>(x.i0 * NP);
         for (int kb = 0; kb < J.k_stages; ++kb) {
           if (!wait_ig(&empty[stage], ph ^ 1u, &abort_flag)) {
             ok = false;
@@ -243,8 +261,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
           }
           mbar_arrive_tx(&full[stage], stage_bytes);
           uint8_t* dst = base + stage * stage_bytes;
-          tma_load_2d(dst, &J.x_map, kb * kIgK, ty, &full[stage]);
-          tma_load_2d(dst + kIgABytes, &J.w_map, kb * kIgK, wy, &full[stage]);
+          tma_load_2d(dst, &J.x_map, kb * kElems, ty, &full[stage]);
+          tma_load_2d(dst + kIgABytes, &J.w_map, kb * kElems, wy, &full[stage]);
           if (++stage == S) {
             stage = 0;
             ph ^= 1u;
@@ -257,7 +275,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
     if (lane == 0) {
       int stage = 0, buf = 0;
       uint32_t ph = 0, bph = 0;
-      const uint32_t idesc = ig_idesc(nrows);
+      const uint32_t idesc = P == 0 ? ig_idesc_bf16(nrows) : ig_idesc(nrows);
       bool ok = true;
       for (int64_t u = blockIdx.x; u < b.total_tiles && ok && !abort_flag; u += gridDim.x) {
         const IgTile x = ig_tile(b, u);
@@ -274,8 +292,10 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
           const uint64_t a0 = kmajor_desc(smem_u32(base + stage * stage_bytes));
           const uint64_t b0 = kmajor_desc(smem_u32(base + stage * stage_bytes + kIgABytes));
 #pragma unroll
-          for (int ks = 0; ks < kIgK / 32; ++ks)      // 32 bytes (16-byte units x 2) per MMA
-            tc_mma_i8(dt, a0 + 2 * ks, b0 + 2 * ks, idesc, (kb | ks) != 0 ? 1u : 0u);
+          for (int ks = 0; ks < kIgK / 32; ++ks) {    // 32 bytes (16-byte units x 2) per MMA
+            if (P == 0) tc_mma(dt, a0 + 2 * ks, b0 + 2 * ks, idesc, (kb | ks) != 0 ? 1u : 0u);
+            else tc_mma_i8(dt, a0 + 2 * ks, b0 + 2 * ks, idesc, (kb | ks) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
@@ -303,14 +323,14 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
       const IgJob& J = b.job[x.job];
       const int64_t t = x.t0 + e;
       const bool row_ok = t < J.tokens;
-      const float xs = row_ok ? __ldg(J.x_scale + t) : 0.0f;
+      const float xs = (P != 0 && row_ok) ? __ldg(J.x_scale + t) : 0.0f;
       if (!wait_ig(&d_full[buf], bph, &abort_flag)) break;
       tc_fence_after();
       const uint32_t tb = tmem + lane_base + static_cast<uint32_t>(buf * kIgMaxN);
       const int cbeg = half * (b.chans >> 1), cend = cbeg + (b.chans >> 1);
       for (int c0 = cbeg; c0 < cend; c0 += 16) {
         uint8_t* ys = J.y_tma ? my_stage + (nstore++ & 1u) * kIgYBox : nullptr;
-        ig_epilogue_chunk<P>(tb + static_cast<uint32_t>(c0 * P), J, t, xs, x.i0 + c0, row_ok, ys, lane);
+        ig_epilogue_chunk<P>(tb + static_cast<uint32_t>(c0 * NP), J, t, xs, x.i0 + c0, row_ok, ys, lane);
       }
       tc_fence_before();
       mbar_arrive(&d_empty[buf]);
@@ -335,7 +355,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
 }
 
 size_t ig_smem_bytes(int planes, int stages) {
-  const size_t stage = kIgABytes + static_cast<size_t>(planes * int_gemm_chans(planes)) * kIgK;
+  const int np = planes == 0 ? 1 : planes;                // 0: bf16
+  const size_t stage = kIgABytes + static_cast<size_t>(np * int_gemm_chans(planes)) * kIgK;
   return 1024 + static_cast<size_t>(stages) * stage + kIgYStage + (2 * stages + 4) * 8;
 }
 
@@ -361,9 +382,92 @@ __global__ void int_pack_kernel(const void* w, int w_bytes, int64_t d, int64_t n
   if (overflow != nullptr && bad != 0) atomicAdd(overflow, bad);
 }
 
+// W'_bf16 = bf16(fp32(s_bar_i) * q_ij): the merged weight as the bf16 operand
+// of a training forward (one fp32 product rounded to nearest, then to bf16
+// with ties to even). A CTA takes rows of one job (kFqRows per step); its
+// threads walk the row in 4-element groups.
+constexpr int kFqRows = 4;
+
+struct FqBatch {
+  FakeQuantJob job[kMaxBatch];
+  int64_t step_begin[kMaxBatch + 1];   // CTA steps before job k
+  int32_t count;
+};
+
+__device__ __forceinline__ int32_t q_at(const void* q, int q_bytes, int64_t e) {
+  if (q_bytes == 1) return static_cast<const int8_t*>(q)[e];
+  if (q_bytes == 2) return static_cast<const int16_t*>(q)[e];
+  return static_cast<const int32_t*>(q)[e];
+}
+__device__ __forceinline__ uint16_t fq_one(float s, int32_t v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(s, static_cast<float>(v))));
+}
+
+__global__ void __launch_bounds__(256) fakequant_kernel(const __grid_constant__ FqBatch b) {
+  const int64_t total = b.step_begin[b.count];
+  int k = 0;
+  for (int64_t c = blockIdx.x; c < total; c += gridDim.x) {
+    while (k + 1 < b.count && b.step_begin[k + 1] <= c) ++k;
+    const FakeQuantJob& J = b.job[k];
+    const int64_t r0 = (c - b.step_begin[k]) * kFqRows;
+    for (int64_t i = r0; i < min64(J.d, r0 + kFqRows); ++i) {
+      const float s = __ldg(J.sbar + i);
+      const int64_t e0 = i * J.n;
+      if (J.n % 4 == 0) {
+        for (int64_t j = 4 * static_cast<int64_t>(threadIdx.x); j < J.n; j += 4 * blockDim.x) {
+          int32_t v[4];
+          if (J.q_bytes == 1) {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const int8_t*>(J.q) + e0 + j);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) v[t] = static_cast<int8_t>(w >> (8 * t));
+          } else if (J.q_bytes == 2) {
+            const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const int16_t*>(J.q) + e0 + j);
+            v[0] = static_cast<int16_t>(w.x);
+            v[1] = static_cast<int16_t>(w.x >> 16);
+            v[2] = static_cast<int16_t>(w.y);
+            v[3] = static_cast<int16_t>(w.y >> 16);
+          } else {
+            const int4 w = *reinterpret_cast<const int4*>(static_cast<const int32_t*>(J.q) + e0 + j);
+            v[0] = w.x;
+            v[1] = w.y;
+            v[2] = w.z;
+            v[3] = w.w;
+          }
+          const uint2 o = make_uint2(fq_one(s, v[0]) | (static_cast<uint32_t>(fq_one(s, v[1])) << 16),
+                                     fq_one(s, v[2]) | (static_cast<uint32_t>(fq_one(s, v[3])) << 16));
+          *reinterpret_cast<uint2*>(J.out + e0 + j) = o;
+        }
+      } else {
+        for (int64_t j = threadIdx.x; j < J.n; j += blockDim.x) J.out[e0 + j] = fq_one(s, q_at(J.q, J.q_bytes, e0 + j));
+      }
+    }
+  }
+}
+
 }  // namespace
 
-int int_gemm_chans(int planes) { return planes == 1 ? 256 : planes == 2 ? 128 : 64; }
+cudaError_t launch_fakequant(const FakeQuantJob* jobs, int count, cudaStream_t s) {
+  static thread_local FqBatch b;
+  for (int k0 = 0; k0 < count; k0 += kMaxBatch) {
+    const int m = count - k0 < kMaxBatch ? count - k0 : kMaxBatch;
+    std::memset(&b, 0, sizeof b);
+    int64_t steps = 0;
+    for (int k = 0; k < m; ++k) {
+      b.job[k] = jobs[k0 + k];
+      b.step_begin[k] = steps;
+      steps += (jobs[k0 + k].d + kFqRows - 1) / kFqRows;
+    }
+    b.step_begin[m] = steps;
+    b.count = m;
+    if (steps == 0) continue;
+    fakequant_kernel<<<static_cast<unsigned>(min64(steps, 148 * 8)), 256, 0, s>>>(b);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+int int_gemm_chans(int planes) { return planes <= 1 ? 256 : planes == 2 ? 128 : 64; }
 
 bool int_gemm_supported() { return tc::encode_fn() != nullptr; }
 
@@ -376,8 +480,14 @@ cudaError_t launch_int_pack(const void* w, int w_bytes, int64_t d, int64_t n, in
   return cudaGetLastError();
 }
 
+// planes = 0: the bf16 GEMM Y = X W^T (X, W bf16 bit patterns, scales unused).
 cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaStream_t s) {
   if (count <= 0) return cudaSuccess;
+  const bool bf16 = planes == 0;
+  const int np = bf16 ? 1 : planes;
+  const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const int esize = bf16 ? 2 : 1;
+  const int kelems = kIgK / esize;            // K elements per 128-byte stage
   static thread_local IgBatch b;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
@@ -391,8 +501,8 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
       const IntGemmJob& j = jobs[k0 + k];
       IgJob& t = b.job[k];
       const bool ok =
-          tc::encode_2d(&t.x_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.X, j.tokens, j.n, kIgK, kIgRows) &&
-          tc::encode_2d(&t.w_map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, j.W, j.d * planes, j.n, kIgK, chans * planes);
+          tc::encode_2d(&t.x_map, dt, esize, j.X, j.tokens, j.n, kelems, kIgRows) &&
+          tc::encode_2d(&t.w_map, dt, esize, j.W, j.d * np, j.n, kelems, chans * np);
       if (!ok) return cudaErrorInvalidValue;
       // Y through TMA stores when its rows are 16-byte multiples
       t.y_tma = (j.d % 4 == 0) &&
@@ -406,7 +516,7 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
       t.n = j.n;
       t.m_tiles = static_cast<int32_t>((j.tokens + kIgRows - 1) / kIgRows);
       t.n_tiles = static_cast<int32_t>((j.d + chans - 1) / chans);
-      t.k_stages = static_cast<int32_t>((j.n + kIgK - 1) / kIgK);
+      t.k_stages = static_cast<int32_t>((j.n + kelems - 1) / kelems);
       t.tile_begin = tiles;
       tiles += static_cast<int64_t>(t.m_tiles) * t.n_tiles;
     }
@@ -418,13 +528,15 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
     b.stages = stages;
     b.total_tiles = tiles;
     const size_t smem = ig_smem_bytes(planes, stages);
-    const void* fn = planes == 1 ? reinterpret_cast<const void*>(int_gemm_kernel<1>)
+    const void* fn = planes == 0   ? reinterpret_cast<const void*>(int_gemm_kernel<0>)
+                     : planes == 1 ? reinterpret_cast<const void*>(int_gemm_kernel<1>)
                      : planes == 2 ? reinterpret_cast<const void*>(int_gemm_kernel<2>)
                                    : reinterpret_cast<const void*>(int_gemm_kernel<3>);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
-    if (planes == 1) int_gemm_kernel<1><<<grid, kIgThreads, smem, s>>>(b);
+    if (planes == 0) int_gemm_kernel<0><<<grid, kIgThreads, smem, s>>>(b);
+    else if (planes == 1) int_gemm_kernel<1><<<grid, kIgThreads, smem, s>>>(b);
     else if (planes == 2) int_gemm_kernel<2><<<grid, kIgThreads, smem, s>>>(b);
     else int_gemm_kernel<3><<<grid, kIgThreads, smem, s>>>(b);
     e = cudaGetLastError();

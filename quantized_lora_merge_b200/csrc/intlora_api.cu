@@ -974,6 +974,74 @@ intlora_status intlora_int_gemm_batched(const intlora_int_gemm_job* jobs, int32_
   return INTLORA_OK;
 }
 
+intlora_status intlora_fakequant_bf16_batched(const intlora_fakequant_job* jobs, int32_t count, void* stream) {
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  std::vector<FakeQuantJob> work;
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_fakequant_job& j = jobs[k];
+    if (j.q_bytes != 1 && j.q_bytes != 2 && j.q_bytes != 4)
+      return fail(INTLORA_ERR_INVALID_ARG, "fake-quantization job %d: q_bytes must be 1, 2 or 4", k);
+    if (j.d < 0 || j.n < 0) return fail(INTLORA_ERR_INVALID_ARG, "fake-quantization job %d: d, n must be >= 0", k);
+    if (j.n > 0 && j.d > kMaxElements / j.n)
+      return fail(INTLORA_ERR_INVALID_ARG, "fake-quantization job %d: d*n exceeds 2^40", k);
+    if (j.d * j.n == 0) continue;
+    if (j.q == nullptr || j.sbar == nullptr || j.w_out == nullptr || !aligned16(j.q) || !aligned16(j.w_out))
+      return fail(INTLORA_ERR_INVALID_ARG, "fake-quantization job %d: q, sbar, w_out are required; q and "
+                  "w_out 16-byte aligned", k);
+    work.push_back(FakeQuantJob{j.q, j.q_bytes, j.sbar, j.d, j.n, static_cast<uint16_t*>(j.w_out)});
+  }
+  if (work.empty()) return INTLORA_OK;
+  const cudaError_t e = launch_fakequant(work.data(), static_cast<int>(work.size()),
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? INTLORA_OK : cuda_fail(e, "fake-quantization launch");
+}
+
+intlora_status intlora_fakequant_bf16(const void* q, int32_t q_bytes, const float* sbar, int64_t d, int64_t n,
+                                      void* w_out, void* stream) {
+  intlora_fakequant_job j{q, q_bytes, sbar, d, n, w_out};
+  return intlora_fakequant_bf16_batched(&j, 1, stream);
+}
+
+intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32_t count, void* stream) {
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  std::vector<IntGemmJob> work;
+  std::vector<int32_t> zero_jobs;
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_linear_job& j = jobs[k];
+    if (j.tokens < 0 || j.d < 0 || j.n < 0 || j.n % 8 != 0)
+      return fail(INTLORA_ERR_INVALID_ARG, "linear job %d: tokens, d, n >= 0 and n %% 8 == 0 required", k);
+    if (j.tokens > (int64_t{1} << 31) || j.d > (int64_t{1} << 31) || j.n > (int64_t{1} << 31))
+      return fail(INTLORA_ERR_INVALID_ARG, "linear job %d: tokens, d, n must be <= 2^31", k);
+    if (j.tokens == 0 || j.d == 0) continue;
+    if (j.Y == nullptr || !aligned16(j.Y))
+      return fail(INTLORA_ERR_INVALID_ARG, "linear job %d: Y is required, 16-byte aligned", k);
+    if (j.n == 0) {
+      zero_jobs.push_back(k);
+      continue;
+    }
+    if (j.X == nullptr || j.W == nullptr || !aligned16(j.X) || !aligned16(j.W))
+      return fail(INTLORA_ERR_INVALID_ARG, "linear job %d: X and W are required, 16-byte aligned", k);
+    work.push_back(IntGemmJob{static_cast<const int8_t*>(j.X), nullptr, static_cast<const int8_t*>(j.W),
+                              nullptr, j.tokens, j.d, j.n, j.Y});
+  }
+  if (!work.empty() && !int_gemm_supported())
+    return fail(INTLORA_ERR_UNSUPPORTED, "bf16 GEMM: the driver's tensor-map encoder is unavailable");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int32_t k : zero_jobs) {
+    const cudaError_t e = launch_zero(jobs[k].Y, jobs[k].tokens * jobs[k].d, st);
+    if (e != cudaSuccess) return cuda_fail(e, "linear zero fill");
+  }
+  if (!work.empty()) {
+    const cudaError_t e = launch_int_gemm(work.data(), static_cast<int>(work.size()), 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "bf16 GEMM launch");
+  }
+  return INTLORA_OK;
+}
+
 intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int8_t* W, const float* w_scale,
                                 int64_t tokens, int64_t d, int64_t n, int32_t planes, float* Y, void* stream) {
   intlora_int_gemm_job j{X, x_scale, W, w_scale, tokens, d, n, Y};

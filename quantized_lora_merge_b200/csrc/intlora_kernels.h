@@ -250,6 +250,15 @@ bool int_gemm_supported();
 cudaError_t launch_int_pack(const void* w, int w_bytes, int64_t d, int64_t n, int planes, int8_t* out,
                             int32_t* overflow, cudaStream_t s);
 cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaStream_t s);
+// planes = 0 above: the bf16 GEMM Y = X W^T (X tokens x n, W d x n bf16).
+struct FakeQuantJob {
+  const void* q;             // merged integer weights (q_bytes 1, 2 or 4), d x n, 16-byte aligned
+  int32_t q_bytes;
+  const float* sbar;
+  int64_t d, n;
+  uint16_t* out;             // bf16 d x n, 16-byte aligned
+};
+cudaError_t launch_fakequant(const FakeQuantJob* jobs, int count, cudaStream_t s);
 unsigned int int_gemm_timeouts();
 
 // Sets the calling thread's intlora_last_error() message.

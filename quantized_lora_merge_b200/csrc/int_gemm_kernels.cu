@@ -384,9 +384,10 @@ __global__ void int_pack_kernel(const void* w, int w_bytes, int64_t d, int64_t n
 
 // W'_bf16 = bf16(fp32(s_bar_i) * q_ij): the merged weight as the bf16 operand
 // of a training forward (one fp32 product rounded to nearest, then to bf16
-// with ties to even). A CTA takes rows of one job (kFqRows per step); its
-// threads walk the row in 4-element groups.
-constexpr int kFqRows = 4;
+// with ties to even). A CTA step covers kFqRows rows of one job; its threads
+// walk those rows' 4-element groups as one flat range (n % 4 == 0), else
+// element by element.
+constexpr int kFqRows = 8;
 
 struct FqBatch {
   FakeQuantJob job[kMaxBatch];
@@ -410,35 +411,45 @@ __global__ void __launch_bounds__(256) fakequant_kernel(const __grid_constant__ 
     while (k + 1 < b.count && b.step_begin[k + 1] <= c) ++k;
     const FakeQuantJob& J = b.job[k];
     const int64_t r0 = (c - b.step_begin[k]) * kFqRows;
-    for (int64_t i = r0; i < min64(J.d, r0 + kFqRows); ++i) {
-      const float s = __ldg(J.sbar + i);
-      const int64_t e0 = i * J.n;
-      if (J.n % 4 == 0) {
-        for (int64_t j = 4 * static_cast<int64_t>(threadIdx.x); j < J.n; j += 4 * blockDim.x) {
-          int32_t v[4];
-          if (J.q_bytes == 1) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const int8_t*>(J.q) + e0 + j);
+    const int rows = static_cast<int>(min64(J.d - r0, kFqRows));
+    if (J.n % 4 == 0) {
+      const int64_t nq = J.n >> 2;                                // groups per row
+      const int64_t groups = nq * rows;
+      const bool narrow = groups < (int64_t{1} << 31);             // 32-bit division
+      for (int64_t g = threadIdx.x; g < groups; g += blockDim.x) {
+        const int64_t rr = narrow ? static_cast<int64_t>(static_cast<uint32_t>(g) / static_cast<uint32_t>(nq))
+                                  : g / nq;
+        const int64_t i = r0 + rr;
+        const int64_t e = i * J.n + 4 * (g - rr * nq);
+        const float s = __ldg(J.sbar + i);
+        int32_t v[4];
+        if (J.q_bytes == 1) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(static_cast<const int8_t*>(J.q) + e);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) v[t] = static_cast<int8_t>(w >> (8 * t));
-          } else if (J.q_bytes == 2) {
-            const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const int16_t*>(J.q) + e0 + j);
-            v[0] = static_cast<int16_t>(w.x);
-            v[1] = static_cast<int16_t>(w.x >> 16);
-            v[2] = static_cast<int16_t>(w.y);
-            v[3] = static_cast<int16_t>(w.y >> 16);
-          } else {
-            const int4 w = *reinterpret_cast<const int4*>(static_cast<const int32_t*>(J.q) + e0 + j);
-            v[0] = w.x;
-            v[1] = w.y;
-            v[2] = w.z;
-            v[3] = w.w;
-          }
-          const uint2 o = make_uint2(fq_one(s, v[0]) | (static_cast<uint32_t>(fq_one(s, v[1])) << 16),
-                                     fq_one(s, v[2]) | (static_cast<uint32_t>(fq_one(s, v[3])) << 16));
-          *reinterpret_cast<uint2*>(J.out + e0 + j) = o;
+          for (int t = 0; t < 4; ++t) v[t] = static_cast<int8_t>(w >> (8 * t));
+        } else if (J.q_bytes == 2) {
+          const uint2 w = *reinterpret_cast<const uint2*>(static_cast<const int16_t*>(J.q) + e);
+          v[0] = static_cast<int16_t>(w.x);
+          v[1] = static_cast<int16_t>(w.x >> 16);
+          v[2] = static_cast<int16_t>(w.y);
+          v[3] = static_cast<int16_t>(w.y >> 16);
+        } else {
+          const int4 w = *reinterpret_cast<const int4*>(static_cast<const int32_t*>(J.q) + e);
+          v[0] = w.x;
+          v[1] = w.y;
+          v[2] = w.z;
+          v[3] = w.w;
         }
-      } else {
-        for (int64_t j = threadIdx.x; j < J.n; j += blockDim.x) J.out[e0 + j] = fq_one(s, q_at(J.q, J.q_bytes, e0 + j));
+        *reinterpret_cast<uint2*>(J.out + e) =
+            make_uint2(fq_one(s, v[0]) | (static_cast<uint32_t>(fq_one(s, v[1])) << 16),
+                       fq_one(s, v[2]) | (static_cast<uint32_t>(fq_one(s, v[3])) << 16));
+      }
+    } else {
+      for (int rr = 0; rr < rows; ++rr) {
+        const int64_t i = r0 + rr;
+        const float s = __ldg(J.sbar + i);
+        for (int64_t j = threadIdx.x; j < J.n; j += blockDim.x)
+          J.out[i * J.n + j] = fq_one(s, q_at(J.q, J.q_bytes, i * J.n + j));
       }
     }
   }

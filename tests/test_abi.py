@@ -130,3 +130,78 @@ def test_empty_batches_are_no_ops(lib):
     assert lib.intlora_gen_aux_batched(None, 0, None, 0, None) == 0
     assert lib.intlora_merge_mul_batched(None, None, 0, 8, None, 0, None) == 0
     assert lib.intlora_ste_backward_batched(None, 0, None, 0, None) == 0
+
+
+# ---------------------------------------------------------------------------
+# widened entry points: host-side validation only (no launch is reached)
+# ---------------------------------------------------------------------------
+def test_int_planes(lib):
+    cases = {0: 1, 127: 1, 128: 2, 16383: 2, 16384: 3, 2**21 - 1: 3, 2**21: 0, -1: 0}
+    for v, p in cases.items():
+        assert lib.intlora_int_planes(v) == p
+
+
+def test_int_pack_rejects(lib):
+    assert lib.intlora_int_pack(FAKE, 3, 4, 16, 1, FAKE, None, None) == 1      # q_bytes
+    assert lib.intlora_int_pack(FAKE, 2, 4, 16, 4, FAKE, None, None) == 1      # planes
+    assert lib.intlora_int_pack(FAKE, 2, 4, 24, 2, FAKE, None, None) == 1      # n % 16
+    assert lib.intlora_int_pack(FAKE, 2, 4, 16, 2, FAKE + 8, None, None) == 1  # alignment
+    assert lib.intlora_int_pack(None, 2, 0, 16, 2, None, None, None) == 0      # empty: no-op
+
+
+def _igjob(**kw):
+    j = B.intlora_int_gemm_job(X=FAKE, x_scale=FAKE, W=FAKE, w_scale=FAKE, tokens=4, d=8, n=32, Y=FAKE)
+    for k, v in kw.items():
+        setattr(j, k, v)
+    return (B.intlora_int_gemm_job * 1)(j)
+
+
+@pytest.mark.parametrize("field,value", [("n", 24), ("X", FAKE + 4), ("Y", None), ("W", None),
+                                         ("tokens", 2**31 + 1), ("n", -16)])
+def test_int_gemm_rejects(lib, field, value):
+    assert lib.intlora_int_gemm_batched(_igjob(**{field: value}), 1, 1, None) == 1
+
+
+def test_int_gemm_rejects_planes(lib):
+    assert lib.intlora_int_gemm_batched(_igjob(), 1, 0, None) == 1
+    assert lib.intlora_int_gemm_batched(_igjob(), 1, 4, None) == 1
+    assert lib.intlora_int_gemm_batched(_igjob(tokens=0), 1, 1, None) == 0    # empty: no-op
+
+
+def test_fakequant_and_linear_reject(lib):
+    assert lib.intlora_fakequant_bf16(FAKE, 3, FAKE, 4, 8, FAKE, None) == 1
+    assert lib.intlora_fakequant_bf16(FAKE, 2, FAKE, 4, 8, FAKE + 2, None) == 1
+    assert lib.intlora_fakequant_bf16(FAKE, 2, None, 4, 8, FAKE, None) == 1
+    assert lib.intlora_fakequant_bf16(None, 2, None, 0, 8, None, None) == 0   # empty: no-op
+    bad_n = (B.intlora_linear_job * 1)(B.intlora_linear_job(X=FAKE, W=FAKE, tokens=4, d=4, n=12, Y=FAKE))
+    assert lib.intlora_linear_bf16_batched(bad_n, 1, None) == 1
+    no_x = (B.intlora_linear_job * 1)(B.intlora_linear_job(X=None, W=FAKE, tokens=4, d=4, n=16, Y=FAKE))
+    assert lib.intlora_linear_bf16_batched(no_x, 1, None) == 1
+
+
+def test_distribution_is_validated(lib):
+    for bad in (-1, 4):
+        jobs = (B.intlora_aux_job * 1)(_aux(distribution=bad))
+        assert lib.intlora_gen_aux_batched(jobs, 1, None, 0, None) == 1
+        assert "distribution" in lib.intlora_last_error().decode()
+        layer = _layer(distribution=bad)
+        assert lib.intlora_merge_mul(ctypes.byref(layer), 8, FAKE, FAKE, FAKE, None, None, 0, None) == 1
+
+
+def _ste(**kw):
+    j = B.intlora_ste_job(G=FAKE, A=FAKE, B=FAKE, d=4, n=8, r=4, dA=FAKE, dB=FAKE, mask_codes=FAKE,
+                          mask_ld=16, mask_bits=4, mask_z=FAKE)
+    for k, v in kw.items():
+        setattr(j, k, v)
+    return (B.intlora_ste_job * 1)(j)
+
+
+@pytest.mark.parametrize("field,value", [("mask_bits", 5), ("mask_codes", FAKE + 8), ("mask_z", None),
+                                         ("mask_ld", 8), ("n", 7)])
+def test_masked_ste_rejects(lib, field, value):
+    assert lib.intlora_ste_backward_batched(_ste(**{field: value}), 1, None, 0, None) == 1
+
+
+def test_masked_ste_workspace_size(lib):
+    assert lib.intlora_ste_workspace_size(_ste(d=100, n=24), 1) == (100 * 24 * 2 + 255) // 256 * 256
+    assert lib.intlora_ste_workspace_size(_ste(mask_codes=None), 1) == 0

@@ -88,7 +88,7 @@ extern "C" {
 typedef enum intlora_status {
     INTLORA_OK = 0,
     INTLORA_ERR_INVALID_ARG = 1,  /* bad pointer, size, bit width, alignment */
-    INTLORA_ERR_UNSUPPORTED = 2,  /* valid but outside what this build handles */
+    INTLORA_ERR_UNSUPPORTED = 2,  /* valid but outside what this library handles */
     INTLORA_ERR_WORKSPACE = 3,    /* ws NULL or ws_bytes below the query's value */
     INTLORA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
     INTLORA_ERR_TIMEOUT = 5       /* a bounded device wait gave up */
@@ -118,7 +118,7 @@ int intlora_version(void);
 #define INTLORA_DIST_CAUCHY 2
 #define INTLORA_DIST_STUDENT_T2 3
 
-/* Limits of this build. */
+/* Limits of this library. */
 #define INTLORA_MAX_RANK 256
 #define INTLORA_MAX_BATCH 128     /* descriptors per batched call */
 

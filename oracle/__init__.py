@@ -1,6 +1,6 @@
 """CPU oracle for the IntLoRA integer low-rank merge (test infrastructure).
 
-TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+TEST INFRASTRUCTURE ONLY: the tests, the repository smoke check and the
 CPU-baseline leg of ``bench.py`` import this package; the CUDA library and its
 Python binding never do. The arithmetic lives in ``intlora_oracle.c`` (plain
 fp64 C, its own Philox4x32-10); this module only builds that file with gcc and

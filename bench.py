@@ -55,6 +55,7 @@ def parse():
                     help="int_gemm: digit planes of the merged weights (1: SHIFT of 4-bit "
                          "codes, 2: MUL of 4-bit codes, 3: MUL of 8-bit codes)")
     ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--y-bf16", action="store_true", help="int_gemm: write Y in bf16")
     ap.add_argument("--dist", type=int, default=0, choices=[0, 1, 2, 3],
                     help="auxiliary law of R for every layer: 0 Laplace (the method's), 1 Gaussian, "
                          "2 Cauchy, 3 Student-t with 2 degrees of freedom (the ablation's laws)")
@@ -590,7 +591,8 @@ def bench_int_gemm(args):
         packed = torch.empty((d, P, n), dtype=torch.int8, device=device)
         B.intlora_int_pack(Q, P, packed)
         del Q
-        jobs.append(B.IntGemmJob(X, xs, packed, ws, torch.empty((T, d), device=device)))
+        jobs.append(B.IntGemmJob(X, xs, packed, ws, torch.empty(
+            (T, d), dtype=torch.bfloat16 if args.y_bf16 else torch.float32, device=device)))
         host.append((d, n))
     desc_jobs = B.Descriptors(jobs)
     torch.cuda.synchronize(device)
@@ -598,7 +600,7 @@ def bench_int_gemm(args):
     tensor_ops = sum(2 * T * d * n * P for d, n in host)
     alg_ops = sum(2 * T * d * n for d, n in host)
     in_bytes = sum(T * n + d * n * P + 4 * (T + d) for d, n in host)
-    out_bytes = sum(4 * T * d for d, n in host)
+    out_bytes = sum((2 if args.y_bf16 else 4) * T * d for d, n in host)
     for _ in range(max(3, args.warmup)):
         B.intlora_int_gemm_batched(desc_jobs, P)
     torch.cuda.synchronize(device)
@@ -645,7 +647,7 @@ def bench_int_gemm(args):
         "config": {"workload": f"DiT-3072 block linears (qkv 9216x3072, out 3072x3072, fc1 "
                                f"12288x3072, fc2 3072x12288) at {T} tokens, W'={GEMM_KIND[P]} "
                                f"merged weights as {P} int8 digit plane(s), int8 activations",
-                   "tokens": T, "planes": P,
+                   "tokens": T, "planes": P, "y": "bf16" if args.y_bf16 else "fp32",
                    "l2": f"inputs {in_bytes / 1e6:.0f} MB + outputs {out_bytes / 1e6:.0f} MB per "
                          f"step, larger than L2"},
         "algorithmic_Top_s": alg_ops / (ms / 1e3) / 1e12,
@@ -661,7 +663,7 @@ def bench_int_gemm(args):
         "e2e": {"value": tensor_ops / (e2e_ms / 1e3) / 1e12, "unit": GEMM_UNIT,
                 "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": sum(j.X.numel() for j in jobs),
-                "d2h_bytes_per_step": sum(4 * j.Y.numel() for j in jobs)},
+                "d2h_bytes_per_step": sum(j.Y.element_size() * j.Y.numel() for j in jobs)},
     }
     if not args.no_cpu_baseline:
         import numpy as np
@@ -718,8 +720,10 @@ def bench_train_forward(args):
     g = torch.Generator(device=device)
     g.manual_seed(11)
     wq = [torch.empty(l.d, l.n, dtype=torch.bfloat16, device=device) for l in layers]
+    # activations and outputs in bf16 (a training forward's layer outputs)
     lin = B.Descriptors(B.LinearJob(torch.randn(T, l.n, generator=g, device=device).to(torch.bfloat16),
-                                    w, torch.empty(T, l.d, device=device)) for l, w in zip(layers, wq))
+                                    w, torch.empty(T, l.d, dtype=torch.bfloat16, device=device))
+                        for l, w in zip(layers, wq))
     stream = torch.cuda.current_stream(device)
 
     fq = B.Descriptors(B.FakeQuantJob(st.out, st.sbar, w) for st, w in zip(states, wq))
@@ -764,7 +768,8 @@ def bench_train_forward(args):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16 x bf16 -> f32", "data": "synthetic",
         "config": {"workload": f"SD-UNet 128 linears at {T} tokens: MUL merge (4-bit) + bf16 "
-                               f"fake-quantization + Y = X W'^T per layer", "tokens": T},
+                               f"fake-quantization + Y = X W'^T per layer (bf16 X and Y)",
+                   "tokens": T},
         "gemm_ms": gemm_ms,
         "roofline": {"bound": "tensor", "kernel": "int_gemm_kernel<0> (tcgen05 kind::f16)",
                      "achieved": gemm_tf, "peak": bf16, "unit": "TFLOP/s", "frac": gemm_tf / bf16,

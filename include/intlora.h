@@ -351,7 +351,8 @@ typedef struct intlora_int_gemm_job {
     const int8_t* W;          /* packed digit planes [d][planes][n], 16-byte aligned */
     const float* w_scale;     /* [d] */
     int64_t tokens, d, n;     /* n % 16 == 0; tokens, d * planes <= 2^31 */
-    float* Y;                 /* tokens x d row-major, 16-byte aligned (overwritten) */
+    void* Y;                  /* tokens x d row-major, 16-byte aligned (overwritten) */
+    int32_t y_bf16;           /* 0: Y fp32; 1: Y bf16 (nearest, ties to even) */
 } intlora_int_gemm_job;
 
 /* Every job of one call uses the same plane count. The integer sums are
@@ -398,7 +399,8 @@ typedef struct intlora_linear_job {
     const void* X;            /* bf16 tokens x n */
     const void* W;            /* bf16 d x n (the fake-quantized merged weight) */
     int64_t tokens, d, n;
-    float* Y;                 /* tokens x d */
+    void* Y;                  /* tokens x d: fp32, or bf16 when y_bf16 */
+    int32_t y_bf16;
 } intlora_linear_job;
 
 intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32_t count,

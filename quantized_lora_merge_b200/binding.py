@@ -66,12 +66,13 @@ class intlora_fakequant_job(ctypes.Structure):
 
 class intlora_linear_job(ctypes.Structure):
     _fields_ = [("X", _c_ptr), ("W", _c_ptr), ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64),
-                ("Y", _c_ptr)]
+                ("Y", _c_ptr), ("y_bf16", _c_i32)]
 
 
 class intlora_int_gemm_job(ctypes.Structure):
     _fields_ = [("X", _c_ptr), ("x_scale", _c_ptr), ("W", _c_ptr), ("w_scale", _c_ptr),
-                ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("Y", _c_ptr)]
+                ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("Y", _c_ptr),
+                ("y_bf16", _c_i32)]
 
 
 _P = ctypes.POINTER
@@ -255,12 +256,14 @@ class IntGemmJob:
     x_scale: object                 # fp32 [tokens]
     W: object                       # int8 [d, planes, n] digit planes
     w_scale: object                 # fp32 [d]
-    Y: object                       # fp32 [tokens, d]
+    Y: object                       # fp32 or bf16 [tokens, d]
 
     def to_c(self) -> intlora_int_gemm_job:
+        import torch
         tokens, n = self.X.shape
         return intlora_int_gemm_job(_ptr(self.X), _ptr(self.x_scale), _ptr(self.W),
-                                    _ptr(self.w_scale), tokens, self.W.shape[0], n, _ptr(self.Y))
+                                    _ptr(self.w_scale), tokens, self.W.shape[0], n, _ptr(self.Y),
+                                    int(self.Y.dtype == torch.bfloat16))
 
 
 @dataclass
@@ -279,12 +282,13 @@ class FakeQuantJob:
 class LinearJob:
     X: object                       # bf16 [tokens, n]
     W: object                       # bf16 [d, n]
-    Y: object                       # fp32 [tokens, d]
+    Y: object                       # fp32 or bf16 [tokens, d]
 
     def to_c(self) -> intlora_linear_job:
+        import torch
         tokens, n = self.X.shape
         return intlora_linear_job(_ptr(self.X), _ptr(self.W), tokens, self.W.shape[0], n,
-                                  _ptr(self.Y))
+                                  _ptr(self.Y), int(self.Y.dtype == torch.bfloat16))
 
 
 def _array(struct, items):
@@ -440,7 +444,10 @@ def intlora_int_gemm_batched(jobs: Sequence[IntGemmJob], planes: int, stream=Non
 
 
 def intlora_int_gemm(job: IntGemmJob, planes: int, stream=None) -> None:
+    """Single-layer call (fp32 Y; a bf16 Y goes through intlora_int_gemm_batched)."""
     c = job.to_c()
+    if c.y_bf16:
+        raise TypeError("intlora_int_gemm writes fp32 Y; use intlora_int_gemm_batched for bf16 Y")
     _check(lib().intlora_int_gemm(c.X, c.x_scale, c.W, c.w_scale, c.tokens, c.d, c.n, planes,
                                   c.Y, _stream(stream)))
 

@@ -62,12 +62,14 @@ __device__ __forceinline__ bool wait_ig(uint64_t* bar, uint32_t parity, volatile
 struct alignas(64) IgJob {
   CUtensorMap x_map;          // {n, tokens} int8, box {128, 128}
   CUtensorMap w_map;          // {n, d P} int8, box {128, C P}
-  CUtensorMap y_map;          // {d, tokens} fp32, box {16, 32}, 64-byte swizzle (when y_tma)
+  CUtensorMap y_map;          // {d, tokens} fp32 box {16, 32} 64-byte swizzle, or bf16 box
+                              // {16, 32} 32-byte swizzle (when y_tma)
   const float* x_scale;
   const float* w_scale;
-  float* Y;
+  void* Y;                    // fp32, or bf16 when y_bf16
   int64_t tokens, d, n;
   int32_t m_tiles, n_tiles, k_stages, y_tma;
+  int32_t y_bf16, pad;
   int64_t tile_begin;
 };
 struct IgBatch {
@@ -168,19 +170,39 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
 #pragma unroll
     for (int c = 0; c < 16; ++c) y[c] *= xs * ws[c];
   }
+  uint32_t yb[8];                                        // bf16 output: pairs, nearest even
+  if (J.y_bf16) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * q], y[2 * q + 1]);
+      yb[q] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
   if (ystage != nullptr) {
     // the buffer's previous store (two blocks ago) has finished reading it
     if (lane == 0) bulk_wait_read<1>();
     __syncwarp();
-    // row `lane`, 16-byte unit q at lane * 64 + 16 (q ^ ((lane >> 1) & 3))
-    const uint32_t row = smem_u32(ystage) + static_cast<uint32_t>(lane) * 64u;
-    const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+    if (J.y_bf16) {
+      // 32-byte rows: unit q of row `lane` at lane * 32 + 16 (q ^ ((lane >> 2) & 1))
+      const uint32_t row = smem_u32(ystage) + static_cast<uint32_t>(lane) * 32u;
+      const uint32_t sw = static_cast<uint32_t>((lane >> 2) & 1);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
-                   ::"r"(row + 16u * (static_cast<uint32_t>(q) ^ sw)), "f"(y[4 * q]), "f"(y[4 * q + 1]),
-                     "f"(y[4 * q + 2]), "f"(y[4 * q + 3])
-                   : "memory");
+      for (int q = 0; q < 2; ++q)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(row + 16u * (static_cast<uint32_t>(q) ^ sw)), "r"(yb[4 * q]), "r"(yb[4 * q + 1]),
+                       "r"(yb[4 * q + 2]), "r"(yb[4 * q + 3])
+                     : "memory");
+    } else {
+      // row `lane`, 16-byte unit q at lane * 64 + 16 (q ^ ((lane >> 1) & 3))
+      const uint32_t row = smem_u32(ystage) + static_cast<uint32_t>(lane) * 64u;
+      const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(row + 16u * (static_cast<uint32_t>(q) ^ sw)), "f"(y[4 * q]), "f"(y[4 * q + 1]),
+                       "f"(y[4 * q + 2]), "f"(y[4 * q + 3])
+                     : "memory");
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -189,7 +211,19 @@ __device__ __forceinline__ void ig_epilogue_chunk(uint32_t taddr, const IgJob& J
     }
     return;
   }
-  float* dst = J.Y + t * J.d + i;
+  if (J.y_bf16) {
+    uint16_t* dst = static_cast<uint16_t*>(J.Y) + t * J.d + i;
+    if (i + 16 <= J.d && (J.d & 7) == 0) {
+      reinterpret_cast<uint4*>(dst)[0] = make_uint4(yb[0], yb[1], yb[2], yb[3]);
+      reinterpret_cast<uint4*>(dst)[1] = make_uint4(yb[4], yb[5], yb[6], yb[7]);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        if (i + c < J.d) dst[c] = static_cast<uint16_t>(yb[c >> 1] >> (16 * (c & 1)));
+    }
+    return;
+  }
+  float* dst = static_cast<float*>(J.Y) + t * J.d + i;
   if (i + 16 <= J.d && (J.d & 3) == 0) {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
@@ -516,9 +550,15 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
           tc::encode_2d(&t.w_map, dt, esize, j.W, j.d * np, j.n, kelems, chans * np);
       if (!ok) return cudaErrorInvalidValue;
       // Y through TMA stores when its rows are 16-byte multiples
-      t.y_tma = (j.d % 4 == 0) &&
-                tc::encode_2d_swz(&t.y_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.Y, j.tokens, j.d, 16, 32,
-                                  CU_TENSOR_MAP_SWIZZLE_64B) ? 1 : 0;
+      t.y_bf16 = j.y_bf16;
+      if (j.y_bf16)
+        t.y_tma = (j.d % 8 == 0) &&
+                  tc::encode_2d_swz(&t.y_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, j.Y, j.tokens, j.d, 16, 32,
+                                    CU_TENSOR_MAP_SWIZZLE_32B) ? 1 : 0;
+      else
+        t.y_tma = (j.d % 4 == 0) &&
+                  tc::encode_2d_swz(&t.y_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.Y, j.tokens, j.d, 16, 32,
+                                    CU_TENSOR_MAP_SWIZZLE_64B) ? 1 : 0;
       t.x_scale = j.x_scale;
       t.w_scale = j.w_scale;
       t.Y = j.Y;

@@ -958,13 +958,14 @@ intlora_status intlora_int_gemm_batched(const intlora_int_gemm_job* jobs, int32_
       return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: X, x_scale, W, w_scale are required", k);
     if (!aligned16(j.X) || !aligned16(j.W))
       return fail(INTLORA_ERR_INVALID_ARG, "int GEMM job %d: X and W must be 16-byte aligned", k);
-    work.push_back(IntGemmJob{j.X, j.x_scale, j.W, j.w_scale, j.tokens, j.d, j.n, j.Y});
+    work.push_back(IntGemmJob{j.X, j.x_scale, j.W, j.w_scale, j.tokens, j.d, j.n, j.Y, j.y_bf16 != 0});
   }
   if (!work.empty() && !int_gemm_supported())
     return fail(INTLORA_ERR_UNSUPPORTED, "int GEMM: the driver's tensor-map encoder is unavailable");
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int32_t k : zero_jobs) {
-    const cudaError_t e = launch_zero(jobs[k].Y, jobs[k].tokens * jobs[k].d, st);
+    const size_t bytes = static_cast<size_t>(jobs[k].tokens * jobs[k].d) * (jobs[k].y_bf16 ? 2 : 4);
+    const cudaError_t e = cudaMemsetAsync(jobs[k].Y, 0, bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "int GEMM zero fill");
   }
   if (!work.empty()) {
@@ -1026,13 +1027,14 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
     if (j.X == nullptr || j.W == nullptr || !aligned16(j.X) || !aligned16(j.W))
       return fail(INTLORA_ERR_INVALID_ARG, "linear job %d: X and W are required, 16-byte aligned", k);
     work.push_back(IntGemmJob{static_cast<const int8_t*>(j.X), nullptr, static_cast<const int8_t*>(j.W),
-                              nullptr, j.tokens, j.d, j.n, j.Y});
+                              nullptr, j.tokens, j.d, j.n, j.Y, j.y_bf16 != 0});
   }
   if (!work.empty() && !int_gemm_supported())
     return fail(INTLORA_ERR_UNSUPPORTED, "bf16 GEMM: the driver's tensor-map encoder is unavailable");
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   for (int32_t k : zero_jobs) {
-    const cudaError_t e = launch_zero(jobs[k].Y, jobs[k].tokens * jobs[k].d, st);
+    const size_t bytes = static_cast<size_t>(jobs[k].tokens * jobs[k].d) * (jobs[k].y_bf16 ? 2 : 4);
+    const cudaError_t e = cudaMemsetAsync(jobs[k].Y, 0, bytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "linear zero fill");
   }
   if (!work.empty()) {
@@ -1044,7 +1046,7 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
 
 intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int8_t* W, const float* w_scale,
                                 int64_t tokens, int64_t d, int64_t n, int32_t planes, float* Y, void* stream) {
-  intlora_int_gemm_job j{X, x_scale, W, w_scale, tokens, d, n, Y};
+  intlora_int_gemm_job j{X, x_scale, W, w_scale, tokens, d, n, Y, 0};
   return intlora_int_gemm_batched(&j, 1, planes, stream);
 }
 

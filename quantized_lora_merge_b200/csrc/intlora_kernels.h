@@ -243,7 +243,8 @@ struct IntGemmJob {
   const int8_t* W;           // [d][planes][n] digit planes, 16-byte aligned
   const float* w_scale;      // [d]
   int64_t tokens, d, n;
-  float* Y;                  // tokens x d
+  void* Y;                   // tokens x d: fp32, or bf16 when y_bf16
+  int32_t y_bf16;
 };
 int int_gemm_chans(int planes);          // output channels per tile: 256 / 128 / 64
 bool int_gemm_supported();

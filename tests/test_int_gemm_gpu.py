@@ -179,3 +179,20 @@ def test_int_gemm_full_size_sampled(planes, bound, tokens, d, n):
                               Qd.cpu().numpy(), wsd.cpu().numpy().astype(np.float64), rows)
     _assert_y(Y[torch.from_numpy(rows).to(dev())].cpu().numpy().astype(np.float64), Yo)
     assert B.intlora_device_timeouts() == 0
+
+
+@pytest.mark.parametrize("planes,bound,tokens,d,n", [(1, 15, 200, 304, 144), (2, 225, 129, 257, 272),
+                                                     (1, 15, 33, 12, 64)])
+def test_int_gemm_bf16_output(planes, bound, tokens, d, n):
+    """Y in bf16 (TMA-stored when d % 8 == 0, else stored directly) is the
+    fp32 result rounded to nearest even, from the same accumulators."""
+    X, xs, Q, ws = wl.int_gemm_host(tokens, d, n, bound, salt=4)
+    packed, _ = _pack(Q, planes)
+    Xd, xsd, wsd = _t(X), _t(xs), _t(ws)
+    Y32 = torch.empty((tokens, d), device=dev())
+    Y16 = torch.full((tokens, d), float("nan"), dtype=torch.bfloat16, device=dev())
+    B.intlora_int_gemm_batched([B.IntGemmJob(Xd, xsd, packed, wsd, Y32)], planes)
+    B.intlora_int_gemm_batched([B.IntGemmJob(Xd, xsd, packed, wsd, Y16)], planes)
+    torch.cuda.synchronize()
+    assert torch.equal(Y16.view(torch.int16), Y32.to(torch.bfloat16).view(torch.int16))
+    _assert_y(Y32.cpu().numpy().astype(np.float64), oracle.int_gemm_rows(X, xs, Q, ws))

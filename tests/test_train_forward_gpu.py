@@ -120,3 +120,17 @@ def test_fakequant_batched_and_ragged():
     torch.cuda.synchronize()
     for j, w in zip(jobs, want):
         assert np.array_equal(_bits(j.w_out), w)
+
+
+@pytest.mark.parametrize("tokens,d,n", [(200, 304, 136), (77, 100, 64)])
+def test_linear_bf16_output(tokens, d, n):
+    rng = np.random.default_rng([tokens, d])
+    Xb = wl.to_bf16_bits(rng.standard_normal((tokens, n)).astype(np.float32))
+    Wb = wl.to_bf16_bits((rng.standard_normal((d, n)) * 0.05).astype(np.float32))
+    Y32 = torch.empty((tokens, d), device=dev())
+    Y16 = torch.full((tokens, d), float("nan"), dtype=torch.bfloat16, device=dev())
+    B.intlora_linear_bf16_batched([B.LinearJob(_bf16(Xb), _bf16(Wb), Y32),
+                                   B.LinearJob(_bf16(Xb), _bf16(Wb), Y16)])
+    torch.cuda.synchronize()
+    assert torch.equal(Y16.view(torch.int16), Y32.to(torch.bfloat16).view(torch.int16))
+    _check_y(Y32.cpu().numpy().astype(np.float64), Xb, Wb)

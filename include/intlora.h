@@ -357,8 +357,10 @@ typedef struct intlora_int_gemm_job {
 
 /* Every job of one call uses the same plane count. The integer sums are
  * exact (s32 per plane, planes added in 64-bit integers); the result is
- * fp32(sum) * fp32(x_scale[t] * w_scale[i]), three fp32 roundings. Jobs with
- * n = 0 get Y = 0. Asynchronous on `stream`; no workspace. */
+ * fp32(sum) * fp32(x_scale[t] * w_scale[i]), three fp32 roundings, then
+ * rounded to bf16 (nearest, ties to even) when y_bf16. Jobs with n = 0 get
+ * Y = 0. Asynchronous on `stream`; no workspace. The single-layer call
+ * writes fp32 Y. */
 intlora_status intlora_int_gemm_batched(const intlora_int_gemm_job* jobs, int32_t count,
                                         int32_t planes, void* stream);
 intlora_status intlora_int_gemm(const int8_t* X, const float* x_scale, const int8_t* W,

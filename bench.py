@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--dist", type=int, default=0, choices=[0, 1, 2, 3],
                     help="auxiliary law of R for every layer: 0 Laplace (the method's), 1 Gaussian, "
                          "2 Cauchy, 3 Student-t with 2 degrees of freedom (the ablation's laws)")
+    ap.add_argument("--rank", type=int, default=0,
+                    help="keep only the layers of this LoRA rank (e.g. one point of --config rank_sweep)")
     ap.add_argument("--masked-ste", action="store_true",
                     help="STE backward restricted to D = W_round - z != 0 (the layers' own codes)")
     ap.add_argument("--shard", action="store_true",
@@ -307,6 +309,10 @@ def main():
         return
     from quantized_lora_merge_b200 import workloads as wl
     layers_base = wl.CONFIGS[args.config]()
+    if args.rank:
+        layers_base = [l for l in layers_base if l.r == args.rank]
+        if not layers_base:
+            raise SystemExit(f"no layer of rank {args.rank} in {args.config}")
     if args.dist:
         from dataclasses import replace as _replace
         layers_base = [_replace(l, distribution=args.dist) for l in layers_base]

@@ -21,6 +21,13 @@
 
 using namespace intlora;
 
+// Two-pass tensor-core A B helpers (tgemm_kernels.cu).
+namespace intlora {
+cudaError_t launch_copy_cols(const float* src, int64_t ld_src, int32_t col0, int32_t cols, int64_t d, float* dst,
+                             cudaStream_t s);
+cudaError_t launch_add_f32(float* t, const float* t2, int64_t count, cudaStream_t s);
+}  // namespace intlora
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -553,28 +560,40 @@ bool tensor_t_enabled() {
   const char* v = std::getenv("INTLORA_T_KERNEL");
   return v == nullptr || std::strcmp(v, "cuda") != 0;
 }
+// Ranks in (kTensorTMaxRank, 2 kTensorTMaxRank] take two tensor-core passes
+// over the rank (the second product added into T).
+constexpr int32_t kTwoPassMaxRank = 2 * kTensorTMaxRank;
+bool two_pass_t(const intlora_layer& l) { return l.r > kTensorTMaxRank; }
 bool uses_tensor_t(const intlora_layer& l) {
-  return tensor_t_enabled() && l.distribution == INTLORA_DIST_LAPLACE && t_gemm_supported(l.d, l.n, l.r);
+  if (!tensor_t_enabled() || l.distribution != INTLORA_DIST_LAPLACE) return false;
+  if (l.r > kTensorTMaxRank && l.r <= kTwoPassMaxRank)
+    return t_gemm_supported(l.d, l.n, kTensorTMaxRank);
+  return t_gemm_supported(l.d, l.n, l.r);
 }
 // A call whose workspace does not cover the tensor-core T buffers still runs,
 // with A B on the CUDA cores (set per call by merge_batched).
 thread_local bool g_t_allowed = true;
 
 // Workspace of one layer of a merge: the sigma_R scratch when sigma_r is not
-// passed, then (tensor-core T) T, A_hi, A_lo, B^T_hi, B^T_lo.
+// passed, then (tensor-core T) T, A_hi, A_lo, B^T_hi, B^T_lo; for two-pass
+// ranks also the second product T2 and A's two column blocks (d x 64 each).
 struct MergeWs {
-  size_t sigma, T, a, bt, total;
+  size_t sigma, T, a, bt, t2, ablk, total;
 };
 MergeWs merge_ws_layout(const intlora_layer& l) {
-  MergeWs w{0, 0, 0, 0, 0};
+  MergeWs w{0, 0, 0, 0, 0, 0, 0};
   if (l.sigma_r == nullptr) w.sigma = 256 + stats_partial_bytes(l.d * l.n);
   if (g_t_allowed && uses_tensor_t(l)) {
-    const int64_t kp = t_gemm_kp(l.r);
+    const int64_t kp = t_gemm_kp(std::min(l.r, kTensorTMaxRank));
     w.T = round256(static_cast<size_t>(l.d * l.n) * 4);
     w.a = round256(static_cast<size_t>(l.d * kp) * 4);
     w.bt = round256(static_cast<size_t>(l.n * kp) * 4);
+    if (two_pass_t(l)) {
+      w.t2 = w.T;
+      w.ablk = round256(static_cast<size_t>(l.d * kTensorTMaxRank) * 4);
+    }
   }
-  w.total = w.sigma + w.T + 2 * w.a + 2 * w.bt;
+  w.total = w.sigma + w.T + 2 * w.a + 2 * w.bt + w.t2 + 2 * w.ablk;
   return w;
 }
 
@@ -597,26 +616,49 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
   std::vector<const double*> sig_r(count);
   std::vector<size_t> offset(count);
   std::vector<const float*> t_of(count, nullptr);
-  std::vector<TGemmJob> tjobs;
+  std::vector<TGemmJob> tjobs, tjobs2;        // second passes of two-pass ranks
+  std::vector<std::pair<float*, const float*>> adds;   // T += T2 after the passes
+  std::vector<int64_t> add_count;
   size_t off = 0;
   for (int32_t k = 0; k < count; ++k) {
     sig_r[k] = layers[k].sigma_r;
     offset[k] = off;
     const MergeWs w = merge_ws_layout(layers[k]);
     if (w.T > 0) {
+      const intlora_layer& y = layers[k];
       char* p = ws + off + w.sigma;
       TGemmJob j;
-      j.A = layers[k].A;
-      j.B = layers[k].B;
-      j.d = layers[k].d;
-      j.n = layers[k].n;
-      j.r = layers[k].r;
-      j.kp = static_cast<int32_t>(t_gemm_kp(layers[k].r));
+      j.A = y.A;
+      j.B = y.B;
+      j.d = y.d;
+      j.n = y.n;
+      j.r = std::min(y.r, kTensorTMaxRank);
+      j.kp = static_cast<int32_t>(t_gemm_kp(j.r));
       j.T = reinterpret_cast<float*>(p);
       j.a_hi = reinterpret_cast<float*>(p + w.T);
       j.a_lo = reinterpret_cast<float*>(p + w.T + w.a);
       j.b_hi = reinterpret_cast<float*>(p + w.T + 2 * w.a);
       j.b_lo = reinterpret_cast<float*>(p + w.T + 2 * w.a + w.bt);
+      if (two_pass_t(y)) {
+        // A's column blocks [0, 64) and [64, r) as dense matrices; the second
+        // pass reuses the split buffers after the first has run
+        float* t2 = reinterpret_cast<float*>(p + w.T + 2 * w.a + 2 * w.bt);
+        float* a1 = reinterpret_cast<float*>(p + w.T + 2 * w.a + 2 * w.bt + w.t2);
+        float* a2 = reinterpret_cast<float*>(p + w.T + 2 * w.a + 2 * w.bt + w.t2 + w.ablk);
+        cudaError_t e = launch_copy_cols(y.A, y.r, 0, kTensorTMaxRank, y.d, a1, st);
+        if (e == cudaSuccess) e = launch_copy_cols(y.A, y.r, kTensorTMaxRank, y.r - kTensorTMaxRank, y.d, a2, st);
+        if (e != cudaSuccess) return cuda_fail(e, "A column copy launch");
+        j.A = a1;
+        TGemmJob j2 = j;
+        j2.A = a2;
+        j2.B = y.B + static_cast<int64_t>(kTensorTMaxRank) * y.n;
+        j2.r = y.r - kTensorTMaxRank;
+        j2.kp = static_cast<int32_t>(t_gemm_kp(j2.r));
+        j2.T = t2;
+        tjobs2.push_back(j2);
+        adds.emplace_back(j.T, t2);
+        add_count.push_back(y.d * y.n);
+      }
       t_of[k] = j.T;
       tjobs.push_back(j);
     }
@@ -625,6 +667,14 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
   if (!tjobs.empty()) {
     cudaError_t e = launch_t_gemm(tjobs.data(), static_cast<int>(tjobs.size()), st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor-core A B launch");
+  }
+  if (!tjobs2.empty()) {
+    cudaError_t e = launch_t_gemm(tjobs2.data(), static_cast<int>(tjobs2.size()), st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor-core A B (second pass) launch");
+    for (size_t q = 0; q < adds.size(); ++q) {
+      e = launch_add_f32(adds[q].first, adds[q].second, add_count[q], st);
+      if (e != cudaSuccess) return cuda_fail(e, "A B pass add launch");
+    }
   }
   for (const auto& grp : group_by_seed(layers, count)) {
     // sigma_R on the device for layers that did not pass it in

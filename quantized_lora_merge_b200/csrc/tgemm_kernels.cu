@@ -343,6 +343,53 @@ size_t tg_smem_bytes(int kp_max, int stages) {
 
 }  // namespace
 
+// Ranks in (64, 128] run as two passes over the rank: T = A[:, :64] B[:64]
+// written into T, A[:, 64:] B[64:] into a second buffer, then added. These
+// copy a column block of A into a dense buffer and add the second product.
+__global__ void copy_cols_kernel(const float* src, int64_t ld_src, int32_t col0, int32_t cols, int64_t d,
+                                 float* dst) {
+  const int64_t total = d * cols;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / cols;
+    dst[e] = __ldg(src + i * ld_src + col0 + (e - i * cols));
+  }
+}
+
+__global__ void add_f32_kernel(float* t, const float* t2, int64_t count) {
+  const int64_t quads = count >> 2;
+  for (int64_t q = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; q < quads;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 a = reinterpret_cast<float4*>(t)[q];
+    const float4 b = __ldg(reinterpret_cast<const float4*>(t2) + q);
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    reinterpret_cast<float4*>(t)[q] = a;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (count & 3)) {
+    const int64_t e = (quads << 2) + threadIdx.x;
+    t[e] += t2[e];
+  }
+}
+
+cudaError_t launch_copy_cols(const float* src, int64_t ld_src, int32_t col0, int32_t cols, int64_t d, float* dst,
+                             cudaStream_t s) {
+  const int64_t total = d * cols;
+  if (total <= 0) return cudaSuccess;
+  copy_cols_kernel<<<static_cast<unsigned>(min64((total + 255) / 256, 148 * 8)), 256, 0, s>>>(src, ld_src, col0,
+                                                                                             cols, d, dst);
+  return cudaGetLastError();
+}
+
+// t and t2 16-byte aligned.
+cudaError_t launch_add_f32(float* t, const float* t2, int64_t count, cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  add_f32_kernel<<<static_cast<unsigned>(min64((count / 4 + 255) / 256 + 1, 148 * 16)), 256, 0, s>>>(t, t2, count);
+  return cudaGetLastError();
+}
+
 int64_t t_gemm_kp(int32_t r) { return r <= 32 ? 32 : 64; }
 
 bool t_gemm_supported(int64_t d, int64_t n, int32_t r) {

@@ -117,6 +117,10 @@ MUL_CASES = [
     (129, 256, 33, 8, 8),     # ragged rank (padded to 64) and row block
     (33, 8200, 64, 4, 4),     # wider than the team kernels: row-tile kernels read T
     (7, 100, 48, 4, 4),
+    # ranks 65..128: two tensor-core passes over the rank, second product added
+    (100, 1024, 96, 8, 8),
+    (33, 520, 72, 4, 4),      # second pass of rank 8 (padded to 32)
+    (129, 8200, 128, 8, 8),
 ]
 
 
@@ -130,6 +134,7 @@ def test_merge_mul_parity(d, n, r, w_bits, u_bits):
 
 SHIFT_CASES = [
     (32, 3072, 64, 4, 4),     # DiT width, r = 64, 4-bit base, 4-bit shift
+    (16, 3072, 128, 4, 4),    # two tensor-core passes
     (16, 12288, 64, 4, 4),    # DiT fc2 width
     (48, 320, 4, 8, 4),       # 8-bit base: int16 merged codes
     (5, 6, 2, 4, 2),          # ragged, 2-bit shift code (clamps at 3)
@@ -151,7 +156,7 @@ def test_merge_tensor_core_t_and_cuda_core_t_agree(monkeypatch, variant):
     both meet the oracle, and their codes differ only where a value sits
     within the tolerance window of a rounding boundary."""
     specs = [spec_for(d, n, r, 4, variant, 4, sid=300 + k)
-             for k, (d, n, r) in enumerate([(64, 3072, 64), (40, 640, 32), (12, 6400, 64)])]
+             for k, (d, n, r) in enumerate([(64, 3072, 64), (40, 640, 32), (12, 6400, 64), (24, 1024, 128)])]
     inps = [_oracle_prepared(s) for s in specs]
     res = {}
     for kernel in ("auto", "cuda"):

@@ -241,11 +241,13 @@ int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bit
 
 /* Workspace of a merge call (16-byte aligned device memory, caller-owned):
  *  - for each layer with sigma_r == NULL: the scratch of its sigma_R reduction;
- *  - for each layer with r in [32, 64] and n % 4 == 0 (on a device with the
- *    tensor-map driver entry point): its product T = A B (d x n fp32) and the
- *    exact tf32 hi/lo splits of A and B^T that the tensor cores multiply
- *    (4 (d + n) kp x 2 bytes, kp = 32 or 64) -- [IntLoRA paper notes, method
- *    section 2: U = s + (R* + A B) / D].
+ *  - for each Laplace layer with r in [32, 128] and n % 4 == 0 (on a device
+ *    with the tensor-map driver entry point): its product T = A B (d x n fp32)
+ *    and the exact tf32 hi/lo splits of A and B^T that the tensor cores
+ *    multiply (4 (d + n) kp x 2 bytes, kp = 32 or 64); for r above 64 (two
+ *    passes over the rank) also the second product (d x n fp32) and A's two
+ *    column blocks (2 x d x 64 fp32) -- [IntLoRA paper notes, method section
+ *    2: U = s + (R* + A B) / D].
  * A call given at least the sigma part but less than the whole still runs: it
  * then forms A B on the CUDA cores inside the merge kernels (same results up
  * to fp32 rounding order, slower at these ranks). Less than the sigma part:

@@ -954,7 +954,7 @@ const char* intlora_status_string(int status) {
 
 const char* intlora_last_error(void) { return g_last_error; }
 
-int intlora_version(void) { return 100; }
+int intlora_version(void) { return 200; }   // 0.2.0: descriptors gained trailing fields
 
 uint32_t intlora_device_timeouts(void) {
   return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts() +

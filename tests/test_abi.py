@@ -205,3 +205,30 @@ def test_masked_ste_rejects(lib, field, value):
 def test_masked_ste_workspace_size(lib):
     assert lib.intlora_ste_workspace_size(_ste(d=100, n=24), 1) == (100 * 24 * 2 + 255) // 256 * 256
     assert lib.intlora_ste_workspace_size(_ste(mask_codes=None), 1) == 0
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/intlora.h compiles as C11 with warnings as errors, and the
+    descriptor layouts accept positional initializers in declared order."""
+    import shutil
+    import subprocess
+    from pathlib import Path
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    inc = Path(__file__).resolve().parents[1] / "include"
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include "intlora.h"
+int use(void* p) {
+  intlora_aux_job a = {0, 4, 8, 1, 0, 1.5f, 4, 0, 0, 0, p, 16, 0, 0, INTLORA_DIST_CAUCHY};
+  intlora_layer l = {4, 8, 4, 4, p, 16, 0, 0, 0, 0, 1, 0, 1.5f, 0, 0, INTLORA_DIST_LAPLACE};
+  intlora_ste_job s = {p, p, p, 4, 8, 4, 0, 0, p, 16, 4, 0};
+  intlora_int_gemm_job g = {0, 0, 0, 0, 1, 1, 16, p, 1};
+  intlora_linear_job f = {p, p, 1, 1, 8, p, 0};
+  intlora_fakequant_job q = {p, 2, 0, 1, 8, p};
+  return (int)(a.distribution + l.distribution + s.mask_bits + g.y_bf16 + f.y_bf16 + q.q_bytes);
+}
+''')
+    res = subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-c", str(src), "-I", str(inc),
+                          "-o", str(tmp_path / "use.o")], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr

@@ -425,5 +425,16 @@ def linear_rows(X_bits, W_bits, rows=None):
     return Y
 
 
+def train_backward(X_bits, dY_bits, W_bits, A_bits, B_bits) -> dict:
+    """Backward of one IntLoRA linear Y = X W'^T through the STE, in fp64 from
+    bf16 patterns: G = dY^T X (the gradient on W', d x n), dX = dY W'
+    (tokens x n), and the STE products dA = G B^T, dB = A^T G."""
+    f = lambda b: (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    X, dY, W, A, B = (f(b) for b in (X_bits, dY_bits, W_bits, A_bits, B_bits))
+    G = dY.T @ X
+    dA, dB = ste_backward(G, A, B)
+    return dict(G=G, dX=dY @ W, dA=dA, dB=dB)
+
+
 def num_threads() -> int:
     return int(_load().orc_num_threads())

@@ -650,3 +650,23 @@ def test_linear_rows_brute_force_and_numpy():
             assert abs(Y[t, i] - sum(float(xf[t, j]) * float(wf[i, j]) for j in range(16))) < 1e-12
     np.testing.assert_allclose(Y, xf @ wf.T, rtol=1e-13, atol=1e-13)
     np.testing.assert_array_equal(oracle.linear_rows(X, W, rows=[2]), Y[[2]])
+
+
+def test_train_backward_brute_force_and_reassociation():
+    """G = dY^T X, dX = dY W', dA = G B^T, dB = A^T G: brute force on a tiny
+    case, and the low-rank reassociation dA = dY^T (X B^T), dB = (dY A)^T X
+    that a fused backward would use holds to rounding."""
+    rng = np.random.default_rng(44)
+    T, d, n, r = 3, 4, 5, 2
+    bits = lambda *shape: wl.to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+    Xb, dYb, Wb, Ab, Bb = bits(T, n), bits(T, d), bits(d, n), bits(d, r), bits(r, n)
+    o = oracle.train_backward(Xb, dYb, Wb, Ab, Bb)
+    X, dY, W, A, B = (wl.bf16_bits_to_f32(b).astype(np.float64) for b in (Xb, dYb, Wb, Ab, Bb))
+    for i in range(d):
+        for j in range(n):
+            assert abs(o["G"][i, j] - sum(dY[t, i] * X[t, j] for t in range(T))) < 1e-12
+    for t in range(T):
+        for j in range(n):
+            assert abs(o["dX"][t, j] - sum(dY[t, i] * W[i, j] for i in range(d))) < 1e-12
+    np.testing.assert_allclose(o["dA"], dY.T @ (X @ B.T), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(o["dB"], (dY @ A).T @ X, rtol=1e-12, atol=1e-14)

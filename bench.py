@@ -6,13 +6,14 @@ layer preparation (Philox/Laplace R, sigma_W and sigma_R, VMC, base
 quantization of W - R*), the merge (MUL for the default workload) and the STE
 backward (dA = G B^T, dB = A^T G), each stage one batched call of the C ABI.
 
-Default workload: 128 SD-v1.5-UNet-shaped linears (16 transformer blocks, 8
-linears each), int4 base codes, rank 4, alpha 1.5, MUL with a 4-bit U
-quantizer, 217,415,680 merged weight elements per step (synthetic inputs drawn
-on the device). Metric: merged weight elements per second (whole job). The
-roofline line is the merge kernel's: it is bound by lane issue (Philox and the
-Laplace inverse CDF per element), so it is reported against the SM lane-issue
-rate at the sampled SM clock, with its HBM fraction beside it.
+Default workload: the 224 linears of a Llama-3-8B-shaped decoder (32 layers:
+q, o 4096x4096; k, v 1024x4096; gate, up 14336x4096; down 4096x14336), int8
+base codes, rank 16, alpha 1.5, MUL with an 8-bit U quantizer: 6,979,321,856
+merged weight elements per step, the largest of the workloads that fits one
+GPU (synthetic inputs drawn on the device). `--config sd_unet`, `dit_3072`,
+`rank_sweep` and `linear320` select the other workloads. Metric: merged weight
+elements per second (whole job); the merge stage's achieved HBM GB/s and its
+fraction of the measured copy peak beside it.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: one process per GPU under torch.distributed.run; every rank runs its
@@ -44,7 +45,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="sd_unet")
+    ap.add_argument("--config", default="llama3_8b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -381,8 +382,10 @@ def main():
     clocks.start()
     time.sleep(0.3)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    from quantized_lora_merge_b200 import binding as Bnd
     barrier()
     torch.cuda.synchronize(device)
+    launches0 = Bnd.intlora_kernel_launches()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -395,6 +398,7 @@ def main():
         path.backward()
         ev[k][3].record(stream)
     t_end.record(stream)
+    launches = Bnd.intlora_kernel_launches() - launches0
     torch.cuda.synchronize(device)
     barrier()
     clk = clocks.stop()
@@ -427,17 +431,13 @@ def main():
     sm_mhz = clk.get("sm_mhz") or 1965.0
     alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
     alu_achieved = sum(merge_ops(l) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
-    # prepare: statistics + finalize + base quantization; merge: one team
-    # launch; STE: zeroing + one tensor-core launch per 64 layers
-    launches_per_step = {"prepare": 3, "merge": 1,
-                         "ste_backward": 1 + (len(layers) + 63) // 64}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.shard else "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": dict(desc, sharding="layers split across ranks"
-                                            if args.shard else "one copy per rank"),
+        "data": "synthetic", "config": desc,
+        "sharding": "layers split across ranks" if args.shard else "one copy of the workload per rank",
         "hbm_GB_s_merge": stages["merge"]["GB_s"],
         "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
         "roofline": {"bound": "alu", "kernel": ("merge team kernel (MUL, 1 launch per step)"
@@ -453,12 +453,12 @@ def main():
                                  if not args.dist else None)},
         "stages": stages,
         "clocks": clk,
-        "gpu_launches": args.steps * sum(launches_per_step.values()),
+        "gpu_launches": launches,
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e(layers, path, arena_in, arena_out, device,
-                          max(4, min(args.steps, 10)), world, elements)
+        line["e2e"] = e2e(states, arena_in, arena_out, device, max(4, min(args.steps, 10)),
+                          world, elements, masked_ste=args.masked_ste)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
     if rank == 0:
@@ -467,87 +467,116 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e(layers, path, arena_in, arena_out, device, steps, world, elements):
-    """Same step through the public API with HOST buffers: every step copies
-    the step's inputs (one pinned host arena holding every layer's W, A, B, G
-    and bf16 A, B) to the device, runs the path and reads the merged weights,
-    scales, zero-points and gradients back (one arena).
+def pinned_host(nbytes):
+    """Page-locked host buffer of exactly `nbytes` (numpy memory registered
+    with the CUDA runtime; torch's pinned allocator would round a 40 GB request
+    up to the next power of two). Returns (tensor, release)."""
+    import numpy as np
+    import torch
+    a = np.empty(max(nbytes, 1), dtype=np.uint8)
+    rt = torch.cuda.cudart()
+    rc = rt.cudaHostRegister(a.ctypes.data, a.nbytes, 0)
+    if int(rc) != 0:
+        raise RuntimeError(f"cudaHostRegister of {nbytes} bytes failed ({rc})")
+    t = torch.from_numpy(a)
+    assert t.is_pinned()
 
-    Steps are pipelined over two device copies of the workload and three
-    streams, as a streaming caller would run them: the inputs of step k+1
-    travel host->device while step k computes and step k-1's results travel
-    device->host. Every step still moves all of its bytes both ways inside
-    the timed region."""
+    def release():
+        rt.cudaHostUnregister(a.ctypes.data)
+    return t, release
+
+
+def layer_groups(states, budget_bytes=3 << 30):
+    """Consecutive runs of layers whose input bytes stay within the budget
+    (at least one layer each): the units the end-to-end leg streams."""
+    groups, cur, size = [], [], 0
+    for st in states:
+        lo, hi = st.extra["in"]
+        if cur and size + (hi - lo) > budget_bytes:
+            groups.append(cur)
+            cur, size = [], 0
+        cur.append(st)
+        size += hi - lo
+    if cur:
+        groups.append(cur)
+    return groups
+
+
+def e2e(states, arena_in, arena_out, device, steps, world, elements, masked_ste=False):
+    """The same step through the public API with HOST buffers: every step
+    copies all of its inputs (W, A, B, G and bf16 A, B of every layer, held in
+    one pinned host arena) to the device, runs the path and copies every
+    merged weight, scale, zero-point and gradient back (one pinned arena).
+
+    The model is streamed as a caller merging it would run it: the layers go
+    in consecutive groups of at most ~3 GB of inputs, each group's inputs
+    travel host->device on one stream, its three stages run on a second (one
+    batched call each) and its results travel device->host on a third, so
+    group g+1 goes up while group g computes and group g-1 comes down. The
+    device buffers are the ones the device-resident leg uses; every step
+    moves all of its bytes both ways inside the timed region."""
     import torch
     import torch.distributed as dist
     from quantized_lora_merge_b200 import pipeline as P
-    # second device copy of the workload (same layers, own buffers)
-    states2 = [P.allocate(l, torch.empty(l.d, l.n, device=device),
-                          torch.empty(l.d, l.r, device=device),
-                          torch.empty(l.r, l.n, device=device), device,
-                          G=torch.empty(l.d, l.n, dtype=torch.bfloat16, device=device),
-                          A16=torch.empty(l.d, l.r, dtype=torch.bfloat16, device=device),
-                          B16=torch.empty(l.r, l.n, dtype=torch.bfloat16, device=device))
-               for l in layers]
-    in2, out2 = P.pack_io(states2, device)
-    assert in2.numel() == arena_in.numel() and out2.numel() == arena_out.numel()
-    path2 = P.Path(states2, device, masked_ste=path.masked_ste)
-    sets = [(path, arena_in, arena_out), (path2, in2, out2)]
-
-    host_in = torch.empty(arena_in.numel(), dtype=torch.uint8, pin_memory=True)
+    groups = layer_groups(states)
+    paths = [P.Path(g, device, masked_ste=masked_ste) for g in groups]
+    rng_in = [(g[0].extra["in"][0], g[-1].extra["in"][1]) for g in groups]
+    rng_out = [(g[0].extra["out"][0], g[-1].extra["out"][1]) for g in groups]
+    host_in, rel_in = pinned_host(arena_in.numel())
+    host_out, rel_out = pinned_host(arena_out.numel())
     host_in.copy_(arena_in)
-    host_out = [torch.empty(arena_out.numel(), dtype=torch.uint8, pin_memory=True)
-                for _ in range(2)]
-    h2d = host_in.numel()
-    d2h = arena_out.numel()
+    h2d = sum(hi - lo for lo, hi in rng_in)
+    d2h = sum(hi - lo for lo, hi in rng_out)
     s_h2d, s_run, s_d2h = (torch.cuda.Stream(device) for _ in range(3))
-    ev = lambda: torch.cuda.Event()                       # noqa: E731
-    copied_in = [ev(), ev()]
-    computed = [ev(), ev()]
-    copied_out = [ev(), ev()]
-    used = [False, False]
+    ng = len(groups)
+    copied_in = [torch.cuda.Event() for _ in range(ng)]
+    computed = [torch.cuda.Event() for _ in range(ng)]
+    copied_out = [torch.cuda.Event() for _ in range(ng)]
+    used = [False] * ng
 
-    def one(k):
-        q = k & 1
-        pth, a_in, a_out = sets[q]
-        with torch.cuda.stream(s_h2d):
-            if used[q]:
-                s_h2d.wait_event(computed[q])             # step k-2 has read its inputs
-            a_in.copy_(host_in, non_blocking=True)
-            copied_in[q].record(s_h2d)
-        with torch.cuda.stream(s_run):
-            s_run.wait_event(copied_in[q])
-            if used[q]:
-                s_run.wait_event(copied_out[q])           # step k-2's outputs are home
-            pth.step()
-            computed[q].record(s_run)
-        with torch.cuda.stream(s_d2h):
-            s_d2h.wait_event(computed[q])
-            host_out[q].copy_(a_out, non_blocking=True)
-            copied_out[q].record(s_d2h)
-        used[q] = True
+    def one_step():
+        for g in range(ng):
+            (ilo, ihi), (olo, ohi) = rng_in[g], rng_out[g]
+            with torch.cuda.stream(s_h2d):
+                if used[g]:
+                    s_h2d.wait_event(computed[g])         # the last step has read them
+                arena_in[ilo:ihi].copy_(host_in[ilo:ihi], non_blocking=True)
+                copied_in[g].record(s_h2d)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(copied_in[g])
+                if used[g]:
+                    s_run.wait_event(copied_out[g])       # the last step's results are home
+                paths[g].step(s_run)
+                computed[g].record(s_run)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(computed[g])
+                host_out[olo:ohi].copy_(arena_out[olo:ohi], non_blocking=True)
+                copied_out[g].record(s_d2h)
+            used[g] = True
 
-    for k in range(2):
-        one(k)
+    one_step()                                            # untimed
     torch.cuda.synchronize(device)
     if world > 1:
         dist.barrier()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(s_h2d)
-    for k in range(steps):
-        one(k)
-    s_d2h.wait_event(copied_out[(steps - 2) & 1])
+    for _ in range(steps):
+        one_step()
+    s_d2h.wait_event(copied_out[ng - 1])
     b.record(s_d2h)
     torch.cuda.synchronize(device)
     ms = a.elapsed_time(b) / steps
+    rel_in()
+    rel_out()
     if world > 1:
         t = torch.tensor([ms], device=device, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
     return {"value": elements / (ms / 1000.0), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
-            "pipelined": "2 device copies, 3 streams"}
+            "pipelined": f"{ng} layer groups per step streamed over 3 streams (pinned host "
+                         f"arenas, one copy per group and direction)"}
 
 
 # ---------------------------------------------------------------------------

@@ -418,6 +418,12 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
  * word); the library has no counterpart of this on the pages. */
 uint32_t intlora_device_timeouts(void);
 
+/* Number of kernels this library has enqueued (every entry point, every
+ * thread) since it was loaded; a launch that the CUDA runtime refused is not
+ * counted. Host-side counter, never synchronizes. The pages have no
+ * counterpart of this; it lets a caller count the GPU launches of a region. */
+uint64_t intlora_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

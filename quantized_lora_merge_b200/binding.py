@@ -81,6 +81,7 @@ _SIGNATURES = {
     "intlora_last_error": (ctypes.c_char_p, []),
     "intlora_version": (ctypes.c_int, []),
     "intlora_device_timeouts": (_c_u32, []),
+    "intlora_kernel_launches": (_c_u64, []),
     "intlora_merge_out_bytes": (_c_i32, [_c_i32, _c_i32, _c_i32]),
     "intlora_gen_aux_workspace_size": (_c_size, [_P(intlora_aux_job), _c_i32]),
     "intlora_gen_aux": (ctypes.c_int, [_c_ptr, _c_i64, _c_i64, _c_u64, _c_u32, _c_f32, _c_i32,
@@ -341,6 +342,11 @@ def intlora_version() -> int:
 def intlora_device_timeouts() -> int:
     """Bounded device waits that gave up since the library was loaded."""
     return lib().intlora_device_timeouts()
+
+
+def intlora_kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded (host counter)."""
+    return lib().intlora_kernel_launches()
 
 
 def intlora_merge_out_bytes(variant: int, w_bits: int, out_bits: int) -> int:

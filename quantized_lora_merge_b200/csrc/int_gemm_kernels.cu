@@ -506,7 +506,7 @@ cudaError_t launch_fakequant(const FakeQuantJob* jobs, int count, cudaStream_t s
     b.count = m;
     if (steps == 0) continue;
     fakequant_kernel<<<static_cast<unsigned>(min64(steps, 148 * 8)), 256, 0, s>>>(b);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -522,7 +522,7 @@ cudaError_t launch_int_pack(const void* w, int w_bytes, int64_t d, int64_t n, in
   if (total <= 0) return cudaSuccess;
   const int64_t blocks = min64((total + 255) / 256, 148 * 16);
   int_pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(w, w_bytes, d, n, planes, out, overflow);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 // planes = 0: the bf16 GEMM Y = X W^T (X, W bf16 bit patterns, scales unused).
@@ -590,7 +590,7 @@ cudaError_t launch_int_gemm(const IntGemmJob* jobs, int count, int planes, cudaS
     else if (planes == 1) int_gemm_kernel<1><<<grid, kIgThreads, smem, s>>>(b);
     else if (planes == 2) int_gemm_kernel<2><<<grid, kIgThreads, smem, s>>>(b);
     else int_gemm_kernel<3><<<grid, kIgThreads, smem, s>>>(b);
-    e = cudaGetLastError();
+    e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

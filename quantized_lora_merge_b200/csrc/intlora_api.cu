@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -938,6 +939,11 @@ void intlora::set_last_error(const char* message) {
   snprintf(g_last_error, sizeof g_last_error, "%s", message);
 }
 
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void intlora::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 extern "C" {
 
 const char* intlora_status_string(int status) {
@@ -955,6 +961,8 @@ const char* intlora_status_string(int status) {
 const char* intlora_last_error(void) { return g_last_error; }
 
 int intlora_version(void) { return 200; }   // 0.2.0: descriptors gained trailing fields
+
+uint64_t intlora_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 uint32_t intlora_device_timeouts(void) {
   return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts() +

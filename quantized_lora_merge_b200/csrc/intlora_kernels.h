@@ -265,4 +265,12 @@ unsigned int int_gemm_timeouts();
 // Sets the calling thread's intlora_last_error() message.
 void set_last_error(const char* message);
 
+// Count of kernel launches this library has enqueued (all threads, since it
+// was loaded); `counted` adds one when a launch returned cudaSuccess.
+void note_launch();
+inline cudaError_t counted(cudaError_t e) {
+  if (e == cudaSuccess) note_launch();
+  return e;
+}
+
 }  // namespace intlora

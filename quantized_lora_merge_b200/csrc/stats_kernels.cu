@@ -198,19 +198,19 @@ cudaError_t launch_stats(const StatsBatch& b, int64_t total_blocks, cudaStream_t
     stats_kernel<false><<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
   else
     stats_kernel<true><<<static_cast<unsigned>(total_blocks), kStatsThreads, 0, s>>>(b);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_stats_finalize(const StatsBatch& b, cudaStream_t s) {
   stats_finalize_kernel<<<static_cast<unsigned>(b.count), kStatsThreads, 0, s>>>(b);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s) {
   if (count <= 0) return cudaSuccess;
   const int64_t blocks = min64((count + 255) / 256, 148 * 8);
   zero_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p, count);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace intlora

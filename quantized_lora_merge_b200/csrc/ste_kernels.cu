@@ -411,7 +411,7 @@ cudaError_t launch_mask_g(const MaskJob* jobs, int count, cudaStream_t s) {
     if (chunks == 0) continue;
     const int64_t blocks = min64(chunks, 148 * 8);
     mask_g_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(b);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -439,7 +439,7 @@ cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s) {
   z.block_begin[seg] = blocks;
   if (blocks == 0) return cudaSuccess;
   zero_segments_kernel<<<blocks, 256, 0, s>>>(z);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s) {
@@ -451,16 +451,20 @@ cudaError_t launch_ste(const SteBatch& b, cudaStream_t s) {
       ste_fused_kernel<4><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
     else
       ste_fused_kernel<8><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
   }
   bool any_split = false;
   for (int j = 0; j < b.count; ++j) any_split = any_split || b.job[j].ksplit > 1;
-  if (any_split) ste_zero_kernel<<<148 * 4, 256, 0, s>>>(b);
+  if (any_split) {
+    ste_zero_kernel<<<148 * 4, 256, 0, s>>>(b);
+    const cudaError_t e = counted(cudaGetLastError());
+    if (e != cudaSuccess) return e;
+  }
   if (!b.transposed)
     ste_gemm_kernel<false><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
   else
     ste_gemm_kernel<true><<<static_cast<unsigned>(b.total_tiles), kSteThreads, 0, s>>>(b);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 }  // namespace intlora

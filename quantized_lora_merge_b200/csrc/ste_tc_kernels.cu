@@ -411,7 +411,7 @@ cudaError_t launch_ste_tc(const SteJob* jobs, int count, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int64_t grid = units < int64_t{per_sm} * sms ? units : int64_t{per_sm} * sms;
     ste_tc_kernel<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(b);
-    e = cudaGetLastError();
+    e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

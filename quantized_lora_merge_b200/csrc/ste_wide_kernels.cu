@@ -340,7 +340,7 @@ cudaError_t launch_ste_wide(const SteJob* jobs, int count, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int64_t grid = u2 < sms ? u2 : sms;
     ste_wide_kernel<<<static_cast<unsigned>(grid), kWThreads, smem, s>>>(b);
-    e = cudaGetLastError();
+    e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

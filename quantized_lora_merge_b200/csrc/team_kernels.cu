@@ -469,7 +469,7 @@ struct TeamLaunch {
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     kernel()<<<b.num_ctas, kTeamThreads, smem, s>>>(b);
-    return cudaGetLastError();
+    return counted(cudaGetLastError());
   }
   static int max_ctas(size_t smem) {
     if (cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,

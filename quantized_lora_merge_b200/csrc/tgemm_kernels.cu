@@ -380,14 +380,14 @@ cudaError_t launch_copy_cols(const float* src, int64_t ld_src, int32_t col0, int
   if (total <= 0) return cudaSuccess;
   copy_cols_kernel<<<static_cast<unsigned>(min64((total + 255) / 256, 148 * 8)), 256, 0, s>>>(src, ld_src, col0,
                                                                                              cols, d, dst);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 // t and t2 16-byte aligned.
 cudaError_t launch_add_f32(float* t, const float* t2, int64_t count, cudaStream_t s) {
   if (count <= 0) return cudaSuccess;
   add_f32_kernel<<<static_cast<unsigned>(min64((count / 4 + 255) / 256 + 1, 148 * 16)), 256, 0, s>>>(t, t2, count);
-  return cudaGetLastError();
+  return counted(cudaGetLastError());
 }
 
 int64_t t_gemm_kp(int32_t r) { return r <= 32 ? 32 : 64; }
@@ -423,7 +423,7 @@ cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s) {
     sb.count = count;
     sb.total_blocks = blocks;
     t_split_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(sb);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   // 2. the products, up to kMaxTgJobs layers per launch
@@ -467,7 +467,7 @@ cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const int64_t grid = units < sms ? units : sms;
     t_gemm_kernel<<<static_cast<unsigned>(grid), kTgThreads, smem, s>>>(b);
-    e = cudaGetLastError();
+    e = counted(cudaGetLastError());
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -576,7 +576,7 @@ struct TileLaunch {
     if (err != cudaSuccess) return err;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = config(b.num_clusters * b.cluster, b.cluster, smem, s, attr);
-    return cudaLaunchKernelEx(&cfg, kernel(), b);
+    return counted(cudaLaunchKernelEx(&cfg, kernel(), b));
   }
 
   static int max_clusters(int cluster, size_t smem) {

@@ -90,10 +90,11 @@ def allocate(spec: LayerSpec, W, A, Bm, device, G=None, A16=None, B16=None,
     return st
 
 
-def arena(tensors: list[torch.Tensor], device) -> tuple[torch.Tensor, list[torch.Tensor]]:
+def arena(tensors: list[torch.Tensor], device) -> tuple[torch.Tensor, list[torch.Tensor], list[int]]:
     """One device buffer holding copies of `tensors` (each at a 256-byte
-    aligned offset) and views of it with the tensors' shapes and dtypes: a
-    host mirror of the buffer then moves with one copy per direction."""
+    aligned offset), views of it with the tensors' shapes and dtypes, and the
+    byte offset of each view: a host mirror of the buffer then moves with one
+    copy per direction (or one per contiguous run of views)."""
     offsets, total = [], 0
     for t in tensors:
         offsets.append(total)
@@ -105,21 +106,25 @@ def arena(tensors: list[torch.Tensor], device) -> tuple[torch.Tensor, list[torch
         v = buf[off:off + nb].view(t.dtype).view(t.shape)
         v.copy_(t)
         views.append(v)
-    return buf, views
+    return buf, views, offsets
 
 
 def pack_io(states: list[LayerState], device) -> tuple[torch.Tensor, torch.Tensor]:
     """Moves every layer's inputs (W, A, B and the STE operands) into one
     arena and its outputs (merged weights, scales, zero-points, gradients)
-    into another; returns (inputs, outputs). Build the Path afterwards."""
+    into another; returns (inputs, outputs). A layer's views are contiguous in
+    each arena, layers in list order: st.extra["in"] and st.extra["out"] hold
+    each layer's [begin, end) byte range. Build the Path afterwards."""
     in_keys = ("W", "A", "B", "G", "A16", "B16")
     out_keys = ("out", "sbar", "zbar", "dA", "dB")
     groups = []
-    for keys in (in_keys, out_keys):
+    for tag, keys in (("in", in_keys), ("out", out_keys)):
         slots = [(st, k) for st in states for k in keys if getattr(st, k) is not None]
-        buf, views = arena([getattr(st, k) for st, k in slots], device)
-        for (st, k), v in zip(slots, views):
+        buf, views, offsets = arena([getattr(st, k) for st, k in slots], device)
+        for (st, k), v, off in zip(slots, views, offsets):
             setattr(st, k, v)
+            lo, hi = st.extra.get(tag, (off, off))
+            st.extra[tag] = (min(lo, off), max(hi, off + v.numel() * v.element_size()))
         groups.append(buf)
     return groups[0], groups[1]
 

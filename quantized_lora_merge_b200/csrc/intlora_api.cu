@@ -571,7 +571,31 @@ bool uses_tensor_t(const intlora_layer& l) {
     return t_gemm_supported(l.d, l.n, kTensorTMaxRank);
   return t_gemm_supported(l.d, l.n, l.r);
 }
-// A call whose workspace does not cover the tensor-core T buffers still runs,
+// INTLORA_MERGE_KERNEL=rows keeps every merge on the row kernels (team and
+// row-tile kernels, A B on the CUDA cores or from the tensor-core T pass);
+// "tc" sends every layer the fused tensor-core kernel takes there, whatever
+// its rank; unset or "auto": the fused kernel takes the layers it supports
+// from rank kMergeTcAutoMinRank up (below it the CUDA-core FMAs of the team
+// kernels cost less than the tensor-core hand-offs).
+constexpr int32_t kMergeTcAutoMinRank = 8;
+int merge_kernel_mode() {
+  const char* v = std::getenv("INTLORA_MERGE_KERNEL");
+  if (v == nullptr) return 0;
+  if (std::strcmp(v, "rows") == 0) return 1;
+  if (std::strcmp(v, "tc") == 0) return 2;
+  return 0;
+}
+bool uses_merge_tc(const intlora_layer& l) {
+  const int mode = merge_kernel_mode();
+  if (mode == 1 || l.distribution != INTLORA_DIST_LAPLACE) return false;
+  if (mode == 0 && l.r < kMergeTcAutoMinRank) return false;
+  // 32-bit Philox block index and tensor-map extents
+  if (l.d * l.n >= (int64_t{1} << 34) || l.d >= (int64_t{1} << 31)) return false;
+  MtcPlan plan;
+  return merge_tc_plan(l.n, l.r, &plan) && t_gemm_supported(l.d, l.n, kTensorTMinRank);
+}
+
+// A call whose workspace does not cover the tensor-core buffers still runs,
 // with A B on the CUDA cores (set per call by merge_batched).
 thread_local bool g_t_allowed = true;
 
@@ -580,11 +604,17 @@ thread_local bool g_t_allowed = true;
 // ranks also the second product T2 and A's two column blocks (d x 64 each).
 struct MergeWs {
   size_t sigma, T, a, bt, t2, ablk, total;
+  bool tc;                   // fused tensor-core merge: only the split A, B^T
 };
 MergeWs merge_ws_layout(const intlora_layer& l) {
-  MergeWs w{0, 0, 0, 0, 0, 0, 0};
+  MergeWs w{0, 0, 0, 0, 0, 0, 0, false};
   if (l.sigma_r == nullptr) w.sigma = 256 + stats_partial_bytes(l.d * l.n);
-  if (g_t_allowed && uses_tensor_t(l)) {
+  if (g_t_allowed && uses_merge_tc(l)) {
+    const int64_t kp = merge_tc_kp(l.r);
+    w.tc = true;
+    w.a = round256(static_cast<size_t>(l.d * kp) * 4);
+    w.bt = round256(static_cast<size_t>(l.n * kp) * 4);
+  } else if (g_t_allowed && uses_tensor_t(l)) {
     const int64_t kp = t_gemm_kp(std::min(l.r, kTensorTMaxRank));
     w.T = round256(static_cast<size_t>(l.d * l.n) * 4);
     w.a = round256(static_cast<size_t>(l.d * kp) * 4);
@@ -598,10 +628,17 @@ MergeWs merge_ws_layout(const intlora_layer& l) {
   return w;
 }
 
-size_t merge_ws_bytes(const intlora_layer* layers, int32_t count) {
+// Per-layer regions in order, then (when a layer takes the fused kernel) the
+// fused kernel's exchange area.
+size_t merge_layers_ws_bytes(const intlora_layer* layers, int32_t count) {
   size_t total = 0;
   for (int32_t k = 0; k < count; ++k) total += merge_ws_layout(layers[k]).total;
   return total;
+}
+size_t merge_ws_bytes(const intlora_layer* layers, int32_t count) {
+  bool tc = false;
+  for (int32_t k = 0; k < count && !tc; ++k) tc = merge_ws_layout(layers[k]).tc;
+  return merge_layers_ws_bytes(layers, count) + (tc ? round256(merge_tc_exchange_bytes()) : 0);
 }
 
 int32_t out_bytes_for(int variant, int w_bits, int out_bits) {
@@ -618,6 +655,8 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
   std::vector<size_t> offset(count);
   std::vector<const float*> t_of(count, nullptr);
   std::vector<TGemmJob> tjobs, tjobs2;        // second passes of two-pass ranks
+  std::vector<TGemmJob> sjobs;                // split operands of the fused-kernel layers
+  std::vector<const TGemmJob*> split_of(count, nullptr);
   std::vector<std::pair<float*, const float*>> adds;   // T += T2 after the passes
   std::vector<int64_t> add_count;
   size_t off = 0;
@@ -625,7 +664,23 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
     sig_r[k] = layers[k].sigma_r;
     offset[k] = off;
     const MergeWs w = merge_ws_layout(layers[k]);
-    if (w.T > 0) {
+    if (w.tc) {
+      const intlora_layer& y = layers[k];
+      char* p = ws + off + w.sigma;
+      TGemmJob j;
+      std::memset(&j, 0, sizeof j);
+      j.A = y.A;
+      j.B = y.B;
+      j.d = y.d;
+      j.n = y.n;
+      j.r = y.r;
+      j.kp = static_cast<int32_t>(merge_tc_kp(y.r));
+      j.a_hi = reinterpret_cast<float*>(p);
+      j.a_lo = reinterpret_cast<float*>(p + w.a);
+      j.b_hi = reinterpret_cast<float*>(p + 2 * w.a);
+      j.b_lo = reinterpret_cast<float*>(p + 2 * w.a + w.bt);
+      sjobs.push_back(j);
+    } else if (w.T > 0) {
       const intlora_layer& y = layers[k];
       char* p = ws + off + w.sigma;
       TGemmJob j;
@@ -664,6 +719,15 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
       tjobs.push_back(j);
     }
     off += w.total;
+  }
+  {
+    size_t q = 0;
+    for (int32_t k = 0; k < count; ++k)
+      if (merge_ws_layout(layers[k]).tc) split_of[k] = &sjobs[q++];
+  }
+  if (!sjobs.empty()) {
+    cudaError_t e = launch_t_split(sjobs.data(), static_cast<int>(sjobs.size()), st);
+    if (e != cudaSuccess) return cuda_fail(e, "A B operand split launch");
   }
   if (!tjobs.empty()) {
     cudaError_t e = launch_t_gemm(tjobs.data(), static_cast<int>(tjobs.size()), st);
@@ -707,11 +771,55 @@ intlora_status merge_chunk(int variant, const intlora_layer* layers, const intlo
       e = launch_stats_finalize(sb, st);
       if (e != cudaSuccess) return cuda_fail(e, "statistics finalize launch");
     }
+    // fused tensor-core merge: one launch per (geometry, code width)
+    {
+      std::map<std::tuple<int, int, int>, std::vector<MtcJob>> tc_groups;
+      for (int32_t k : grp) {
+        if (split_of[k] == nullptr) continue;
+        const intlora_layer& y = layers[k];
+        const TGemmJob& sj = *split_of[k];
+        MtcPlan plan;
+        merge_tc_plan(y.n, y.r, &plan);
+        MtcJob j;
+        std::memset(&j, 0, sizeof j);
+        j.codes = static_cast<const uint8_t*>(y.w_round);
+        j.ld_w = y.ld_w;
+        j.s = y.s;
+        j.z = y.z;
+        j.a_hi = sj.a_hi;
+        j.a_lo = sj.a_lo;
+        j.b_hi = sj.b_hi;
+        j.b_lo = sj.b_lo;
+        j.sigma_w = y.sigma_w;
+        j.sigma_r = sig_r[k];
+        j.alpha = y.alpha;
+        j.stream_id = y.stream_id;
+        j.out = outs[k].out;
+        j.scale_out = outs[k].sbar;
+        j.zero_out = variant == kMul ? outs[k].zbar : nullptr;
+        j.code_out = outs[k].code;
+        j.d = y.d;
+        j.n = y.n;
+        j.kp = sj.kp;
+        tc_groups[std::make_tuple(plan.group, static_cast<int>(plan.slice), y.w_bits)].push_back(j);
+      }
+      for (auto& kv : tc_groups) {
+        MtcPlan plan;
+        plan.group = std::get<0>(kv.first);
+        plan.slice = std::get<1>(kv.first);
+        const int wb = std::get<2>(kv.first);
+        const int ob = out_bytes_for(variant == kMul ? 0 : 1, wb, bits);
+        cudaError_t e = launch_merge_tc(kv.second.data(), static_cast<int>(kv.second.size()), variant, wb, ob, bits,
+                                        lo32(layers[grp[0]].seed), hi32(layers[grp[0]].seed), plan,
+                                        ws + merge_layers_ws_bytes(layers, count), st);
+        if (e != cudaSuccess) return cuda_fail(e, "fused tensor-core merge launch");
+      }
+    }
     for (int wb : {4, 8}) {
       std::vector<TileLayer> L;
       for (int32_t k : grp) {
         const intlora_layer& y = layers[k];
-        if (y.w_bits != wb) continue;
+        if (y.w_bits != wb || split_of[k] != nullptr) continue;
         TileLayer l;
         std::memset(&l, 0, sizeof l);
         l.src = y.w_round;
@@ -966,7 +1074,7 @@ uint64_t intlora_kernel_launches(void) { return g_launches.load(std::memory_orde
 
 uint32_t intlora_device_timeouts(void) {
   return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts() +
-         intlora::int_gemm_timeouts();
+         intlora::int_gemm_timeouts() + intlora::merge_tc_timeouts();
 }
 
 int32_t intlora_int_planes(int64_t max_abs) {

@@ -233,6 +233,52 @@ int64_t t_gemm_kp(int32_t r);
 bool t_gemm_supported(int64_t d, int64_t n, int32_t r);
 cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s);
 unsigned int t_gemm_timeouts();
+// The split pass alone: A_hi, A_lo (d x kp) and B^T_hi, B^T_lo (n x kp) of
+// every job (T and r above kp unused), one launch.
+cudaError_t launch_t_split(const TGemmJob* jobs, int count, cudaStream_t s);
+
+// Fused merge with A B on the tensor cores (merge_tc_kernels.cu): T = A B
+// (tf32 three-term split) lands in tensor memory, U is formed and parked
+// there, the row extrema are combined across the group of CTAs that shares a
+// row (through an exchange area of the workspace), and the merged weights are
+// stored; no other intermediate goes to global memory.
+constexpr int32_t kMergeTcMaxRank = 128;
+constexpr int kMergeTcMaxGroup = 64;        // CTAs per row: rows of up to 64 x 512 columns
+constexpr int kMergeTcMaxCtas = 256;        // CTAs of one launch (one per SM)
+struct MtcJob {
+  const uint8_t* codes;      // W_round, row stride ld_w bytes (multiple of 16)
+  int64_t ld_w;
+  const float* s;
+  const int32_t* z;
+  const float* a_hi;         // d x kp split operands (workspace, 16-byte aligned)
+  const float* a_lo;
+  const float* b_hi;         // n x kp (B transposed)
+  const float* b_lo;
+  const double* sigma_w;
+  const double* sigma_r;
+  float alpha;
+  uint32_t stream_id;
+  void* out;                 // P or M, d x n dense
+  float* scale_out;
+  int32_t* zero_out;         // MUL only (may be nullptr)
+  uint8_t* code_out;         // optional U_round / shift codes
+  int64_t d, n;
+  int32_t kp;                // merge_tc_kp(r)
+};
+struct MtcPlan {
+  int group;                 // CTAs sharing one row (G)
+  int32_t slice;             // columns per CTA (multiple of 32, <= 512)
+};
+int64_t merge_tc_kp(int32_t r);
+// Geometry for rows of n columns at rank r, or false when the fused kernel
+// does not take such a layer (n % 32 != 0, r outside [1, kMergeTcMaxRank],
+// rows longer than kMergeTcMaxGroup x 512 columns).
+bool merge_tc_plan(int64_t n, int32_t r, MtcPlan* plan);
+// Bytes of the exchange area a launch needs (16-byte aligned, any contents).
+size_t merge_tc_exchange_bytes();
+cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bits, int out_bytes, int bits,
+                            uint32_t key0, uint32_t key1, const MtcPlan& plan, void* exchange, cudaStream_t s);
+unsigned int merge_tc_timeouts();
 cudaError_t launch_zero(float* p, int64_t count, cudaStream_t s);
 
 // Integer inference GEMM on merged weights (tcgen05 kind::i8): Y = diag(x_scale)

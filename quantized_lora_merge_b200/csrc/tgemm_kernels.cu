@@ -397,9 +397,8 @@ bool t_gemm_supported(int64_t d, int64_t n, int32_t r) {
          n <= (int64_t{1} << 31) && tc::encode_fn() != nullptr;
 }
 
-cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s) {
+cudaError_t launch_t_split(const TGemmJob* jobs, int count, cudaStream_t s) {
   if (count <= 0) return cudaSuccess;
-  // 1. split the operands (one launch for the whole batch)
   {
     static thread_local SplitBatch sb;
     std::memset(&sb, 0, sizeof sb);
@@ -424,6 +423,16 @@ cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s) {
     sb.total_blocks = blocks;
     t_split_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(sb);
     cudaError_t e = counted(cudaGetLastError());
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_t_gemm(const TGemmJob* jobs, int count, cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  // 1. split the operands (one launch for the whole batch)
+  {
+    cudaError_t e = launch_t_split(jobs, count, s);
     if (e != cudaSuccess) return e;
   }
   // 2. the products, up to kMaxTgJobs layers per launch

@@ -182,8 +182,10 @@ intlora_status intlora_gen_aux_batched(const intlora_aux_job* jobs, int32_t coun
  * intlora_last_error(). Allocates nothing.
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture. All calls share the one array: calls whose GPU work can overlap
+ * device current) and caches it for the life of the process; make that first
+ * call before any stream capture, and do not reset the device
+ * (cudaDeviceReset) between calls, since the cached address would then be
+ * stale. All calls share the one array: calls whose GPU work can overlap
  * (different streams without ordering) race on it and must be serialized by
  * the caller. Nothing in the array needs clearing between calls.
  * ------------------------------------------------------------------------ */
@@ -417,6 +419,23 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
  * wrong outputs instead of a hung device. Synchronous (reads one device
  * word); the library has no counterpart of this on the pages. */
 uint32_t intlora_device_timeouts(void);
+
+/* Device health check: synchronizes the device, then returns
+ * INTLORA_ERR_TIMEOUT (with the count in intlora_last_error()) when bounded
+ * device-side waits gave up since the previous intlora_device_status() call
+ * (the results of the calls in between are not valid), a CUDA error as
+ * INTLORA_ERR_CUDA, else INTLORA_OK. Each timeout is reported once. The pages
+ * have no counterpart of this; it is how the library's failure detection
+ * reaches the caller without a device trap. */
+intlora_status intlora_device_status(void);
+
+/* Self-test of that failure path: enqueues on `stream` one kernel that waits,
+ * through the same bounded mbarrier wait the tensor-core kernels use, on a
+ * barrier nothing will complete, for limit_us microseconds (1 .. 1,000,000).
+ * No copy or tensor-core product is in flight; the wait gives up, is counted,
+ * and the kernel returns, leaving the context usable. A following
+ * intlora_device_status() returns INTLORA_ERR_TIMEOUT. */
+intlora_status intlora_selftest_bounded_wait(uint32_t limit_us, void* stream);
 
 /* Number of kernels this library has enqueued (every entry point, every
  * thread) since it was loaded; a launch that the CUDA runtime refused is not

@@ -82,6 +82,8 @@ _SIGNATURES = {
     "intlora_version": (ctypes.c_int, []),
     "intlora_device_timeouts": (_c_u32, []),
     "intlora_kernel_launches": (_c_u64, []),
+    "intlora_device_status": (ctypes.c_int, []),
+    "intlora_selftest_bounded_wait": (ctypes.c_int, [_c_u32, _c_ptr]),
     "intlora_merge_out_bytes": (_c_i32, [_c_i32, _c_i32, _c_i32]),
     "intlora_gen_aux_workspace_size": (_c_size, [_P(intlora_aux_job), _c_i32]),
     "intlora_gen_aux": (ctypes.c_int, [_c_ptr, _c_i64, _c_i64, _c_u64, _c_u32, _c_f32, _c_i32,
@@ -342,6 +344,18 @@ def intlora_version() -> int:
 def intlora_device_timeouts() -> int:
     """Bounded device waits that gave up since the library was loaded."""
     return lib().intlora_device_timeouts()
+
+
+def intlora_device_status() -> int:
+    """INTLORA_OK, or INTLORA_ERR_TIMEOUT when bounded device waits gave up
+    since the last check (synchronizes the device). Returns the status code
+    (no exception), so callers can tell the two apart."""
+    return lib().intlora_device_status()
+
+
+def intlora_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    """Enqueues the self-test kernel whose bounded wait runs out."""
+    _check(lib().intlora_selftest_bounded_wait(limit_us, _stream(stream)))
 
 
 def intlora_kernel_launches() -> int:

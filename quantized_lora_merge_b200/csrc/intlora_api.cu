@@ -50,16 +50,14 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 constexpr int64_t kMaxElements = int64_t{1} << 40;
-constexpr int kStatsThreadsHost = 256;
-constexpr int kStatsGroupsPerThread = 64;
 constexpr int kStatsMaxBlocksPerJob = 148 * 8;
 
 int64_t stats_blocks(int64_t numel) {
-  const int64_t groups = ceil_div(numel, 4);
-  return std::min<int64_t>(kStatsMaxBlocksPerJob,
-                           std::max<int64_t>(1, ceil_div(groups, kStatsThreadsHost * kStatsGroupsPerThread)));
+  return std::min<int64_t>(kStatsMaxBlocksPerJob, std::max<int64_t>(1, ceil_div(numel, kStatsElementsPerCta)));
 }
-size_t stats_partial_bytes(int64_t numel) { return round256(static_cast<size_t>(stats_blocks(numel)) * 4 * sizeof(double)); }
+size_t stats_partial_bytes(int64_t numel) {
+  return round256(static_cast<size_t>(stats_blocks(numel)) * kStatsPartialBytes);
+}
 
 // ------------------------------------------------------------------------
 // tile geometry: cluster size, column slice, rows per tile
@@ -1074,7 +1072,38 @@ uint64_t intlora_kernel_launches(void) { return g_launches.load(std::memory_orde
 
 uint32_t intlora_device_timeouts(void) {
   return intlora::ste_tc_timeouts() + intlora::ste_wide_timeouts() + intlora::t_gemm_timeouts() +
-         intlora::int_gemm_timeouts() + intlora::merge_tc_timeouts();
+         intlora::int_gemm_timeouts() + intlora::merge_tc_timeouts() + intlora::selftest_timeouts();
+}
+
+namespace {
+std::mutex g_status_mutex;
+uint32_t g_timeouts_reported = 0;
+}
+
+intlora_status intlora_device_status(void) {
+  const cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "device synchronization");
+  const uint32_t now = intlora_device_timeouts();
+  std::lock_guard<std::mutex> lock(g_status_mutex);
+  if (now != g_timeouts_reported) {
+    const uint32_t fresh = now - g_timeouts_reported;
+    g_timeouts_reported = now;
+    return fail(INTLORA_ERR_TIMEOUT,
+                "%u bounded device wait(s) gave up since the last check; the results of the "
+                "calls in between are not valid",
+                fresh);
+  }
+  return INTLORA_OK;
+}
+
+intlora_status intlora_selftest_bounded_wait(uint32_t limit_us, void* stream) {
+  g_last_error[0] = '\0';
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(INTLORA_ERR_INVALID_ARG, "limit_us must be in [1, 1000000]");
+  const cudaError_t e = intlora::launch_selftest_wait(uint64_t{limit_us} * 1000u, nullptr,
+                                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test kernel launch");
+  return INTLORA_OK;
 }
 
 int32_t intlora_int_planes(int64_t max_abs) {

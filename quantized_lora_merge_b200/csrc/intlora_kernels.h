@@ -26,6 +26,12 @@ struct StatsJob {
   double* sigma_w_out;       // may be nullptr
   double* sigma_r_out;
 };
+// Elements one statistics CTA reduces (256 threads x 64 groups of 4) and the
+// bytes of its fp64 partial (four sums), when a layer spans enough CTAs.
+constexpr int kStatsThreadsPerCta = 256;
+constexpr int kStatsGroupsPerThread = 64;
+constexpr int64_t kStatsElementsPerCta = int64_t{4} * kStatsThreadsPerCta * kStatsGroupsPerThread;
+constexpr size_t kStatsPartialBytes = 4 * sizeof(double);
 struct StatsBatch {
   StatsJob job[kMaxBatch];
   int32_t count;
@@ -310,6 +316,12 @@ unsigned int int_gemm_timeouts();
 
 // Sets the calling thread's intlora_last_error() message.
 void set_last_error(const char* message);
+
+// Self-test of the bounded waits: one mbarrier that nothing completes, waited
+// on for limit_ns (selftest_kernels.cu); *completed (device int, optional)
+// receives 0 when the wait gave up.
+cudaError_t launch_selftest_wait(uint64_t limit_ns, int* completed, cudaStream_t s);
+unsigned int selftest_timeouts();
 
 // Count of kernel launches this library has enqueued (all threads, since it
 // was loaded); `counted` adds one when a launch returned cudaSuccess.

@@ -27,10 +27,14 @@
 
 namespace {
 
-// 512 CTA partials of four fp64 sums: enough for any layer of at most
-// INTLORA_NOALLOC_MAX_ELEMENTS elements (the statistics kernel uses one CTA per
-// 8192 elements up to its cap).
+// The statistics pass gives each CTA kStatsElementsPerCta (65,536) elements
+// and one partial of kStatsPartialBytes (four fp64 sums, 32 bytes), so a layer
+// of INTLORA_NOALLOC_MAX_ELEMENTS (4,194,304) elements needs 64 partials,
+// 2 KB rounded to 256 bytes. The array holds 16 KB: room for 512 partials.
 constexpr size_t kScratchBytes = 16384;
+static_assert(((INTLORA_NOALLOC_MAX_ELEMENTS + intlora::kStatsElementsPerCta - 1) / intlora::kStatsElementsPerCta) *
+                      intlora::kStatsPartialBytes <= kScratchBytes,
+              "the built-in scratch must hold the partials of the largest layer this entry point accepts");
 static __device__ __align__(256) double g_scratch[kScratchBytes / sizeof(double)];
 
 constexpr int kMaxDevices = 64;

@@ -45,23 +45,27 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait: false once kWaitNs have passed (the wait is counted in a
+// Bounded wait: false once limit_ns have passed (the wait is counted in a
 // device word and the CTA is told to stop) or when another role of the CTA
 // has given up already.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* timeouts) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              unsigned int* timeouts, uint64_t limit_ns) {
   if (mbar_try(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitNs) break;
+      if (global_ns() - t0 > limit_ns) break;
     }
   }
   atomicAdd(timeouts, 1u);
   *abort_flag = 1;
   return false;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* timeouts) {
+  return mbar_wait_for(bar, parity, abort_flag, timeouts, kWaitNs);
 }
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {

@@ -36,7 +36,9 @@ def _near_half(x: np.ndarray) -> np.ndarray:
 
 
 def _allowed_mismatches(n: int) -> int:
-    return max(1, int(np.floor((1.0 - MIN_EXACT) * n)))
+    """Codes that may differ among n: at most 0.01 % (exactly, in integers),
+    so none at all below 10,000 codes."""
+    return n // 10000
 
 
 def assert_scale(name, gpu, ora):

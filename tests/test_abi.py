@@ -232,3 +232,16 @@ int use(void* p) {
     res = subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-c", str(src), "-I", str(inc),
                           "-o", str(tmp_path / "use.o")], capture_output=True, text=True)
     assert res.returncode == 0, res.stderr
+
+
+def test_selftest_wait_rejects_bad_limits(lib):
+    """The bounded-wait self-test validates its limit before launching."""
+    assert lib.intlora_selftest_bounded_wait(0, None) == 1
+    assert lib.intlora_selftest_bounded_wait(2_000_000, None) == 1
+    assert "limit_us" in lib.intlora_last_error().decode()
+
+
+def test_launch_counter_is_monotonic(lib):
+    a = lib.intlora_kernel_launches()
+    lib.intlora_merge_out_bytes(0, 8, 8)           # launches nothing
+    assert lib.intlora_kernel_launches() == a

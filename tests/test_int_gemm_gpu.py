@@ -178,7 +178,7 @@ def test_int_gemm_full_size_sampled(planes, bound, tokens, d, n):
     Yo = oracle.int_gemm_rows(Xd.cpu().numpy(), xsd.cpu().numpy().astype(np.float64),
                               Qd.cpu().numpy(), wsd.cpu().numpy().astype(np.float64), rows)
     _assert_y(Y[torch.from_numpy(rows).to(dev())].cpu().numpy().astype(np.float64), Yo)
-    assert B.intlora_device_timeouts() == 0
+    assert B.intlora_device_status() == 0
 
 
 @pytest.mark.parametrize("planes,bound,tokens,d,n", [(1, 15, 200, 304, 144), (2, 225, 129, 257, 272),

@@ -103,4 +103,4 @@ def test_fused_without_code_output_and_repeat():
 
 
 def test_fused_no_device_wait_gave_up():
-    assert B.intlora_device_timeouts() == 0
+    assert B.intlora_device_status() == 0

@@ -100,7 +100,7 @@ def test_linear_bf16_full_size_sampled():
     rows = np.array([0, 1, 127, 128, 2049, tokens - 1])
     Xb, Wb = _bits(X), _bits(Wt)
     _check_y(Y[torch.from_numpy(rows).to(dev())].cpu().numpy().astype(np.float64), Xb, Wb, rows)
-    assert B.intlora_device_timeouts() == 0
+    assert B.intlora_device_status() == 0
 
 
 def test_fakequant_batched_and_ragged():

@@ -50,6 +50,7 @@ constexpr int kIgMaxN = 256;                    // digit rows per tile (N)
 constexpr int kIgK = 128;                       // K bytes per stage (one swizzle row)
 constexpr uint32_t kIgABytes = kIgRows * kIgK;  // 16 KB
 constexpr int kMaxIgJobs = 48;
+constexpr int kIgMaxStages = 8;                 // pipeline stages at most (host picks 2-8)
 constexpr uint32_t kIgYBox = 32 * 16 * 4;        // one Y block: 32 rows x 16 fp32
 constexpr uint32_t kIgYStage = 8 * 2 * kIgYBox;  // 8 epilogue warps x 2 buffers
 
@@ -240,6 +241,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ __align__(8) uint64_t drain_bar;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   const int S = b.stages;
   constexpr int NP = P == 0 ? 1 : P;                    // P = 0: bf16 operands
@@ -265,6 +267,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
       mbar_init(&d_empty[q], kIgEpiThreads);
     }
     abort_flag = 0;
+    mbar_init(&drain_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -283,6 +286,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
       int stage = 0;
       uint32_t ph = 0;
       bool ok = true;
+      int armed[kIgMaxStages];               // parity last armed per stage (-1: never)
+      for (int q = 0; q < kIgMaxStages; ++q) armed[q] = -1;
       for (int64_t u = blockIdx.x; u < b.total_tiles && ok && !abort_flag; u += gridDim.x) {
         const IgTile x = ig_tile(b, u);
         const IgJob& J = b.job[x.job];
@@ -294,6 +299,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
             break;
           }
           mbar_arrive_tx(&full[stage], stage_bytes);
+          armed[stage] = static_cast<int>(ph);
           uint8_t* dst = base + stage * stage_bytes;
           tma_load_2d(dst, &J.x_map, kb * kElems, ty, &full[stage]);
           tma_load_2d(dst + kIgABytes, &J.w_map, kb * kElems, wy, &full[stage]);
@@ -303,6 +309,8 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
           }
         }
       }
+      if (abort_flag)        // copies in flight land before the CTA goes away
+        for (int q = 0; q < S; ++q) drain_phase(&full[q], armed[q]);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -343,6 +351,7 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
           bph ^= 1u;
         }
       }
+      if (abort_flag) drain_mma(&drain_bar);   // products in flight complete first
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: TMEM lane = token row of the tile
@@ -379,9 +388,6 @@ __global__ void __launch_bounds__(kIgThreads, 1) int_gemm_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (abort_flag) {
-      for (int k = 0; k < 2000; ++k) __nanosleep(1000);   // let copies in flight land
-    }
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kIgMaxN)
                  : "memory");

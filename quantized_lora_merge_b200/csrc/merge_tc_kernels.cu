@@ -422,19 +422,32 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       }
 
       // ---- phase A: T -> U, row extrema, U parked in tensor memory
+      // This thread's 16-column groups are g = 0 .. ng - 1 at slice column
+      // 32 g + 16 member, in part order; each group's codes are loaded two
+      // groups ahead (the loads are the longest latency of the loop).
+      const int ng = cols >> 5;
       float hi = 0.0f, lo = 0.0f;
       bool ok = true;
-      for (int p = 0; p < NP; ++p) {
-        if (!wait_m(&t_full[p], up, &abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int pc = min(static_cast<int>(kPartCols), cols - p * static_cast<int>(kPartCols));
-        for (int c = 16 * member; c < pc; c += 32) {
-          const int cc = p * static_cast<int>(kPartCols) + c;             // column in the slice
+      {
+        uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
+        if (ng > 0) cw0 = load_codes16<WBITS>(crow + (((col0 + 16 * member) * WBITS) >> 3));
+        if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + 32 + 16 * member) * WBITS) >> 3));
+        int have_part = -1;
+        for (int g = 0; g < ng; ++g) {
+          const int cc = 32 * g + 16 * member;                 // column in the slice
+          const int p = cc >> 7;
+          if (p != have_part) {
+            if (!wait_m(&t_full[p], up, &abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            have_part = p;
+          }
           const int64_t j = col0 + cc;
-          const uint4 cw = load_codes16<WBITS>(crow + ((j * WBITS) >> 3));
+          const uint4 cw = cw0;
+          cw0 = cw1;
+          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 64) * WBITS) >> 3));
           float v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();
@@ -535,12 +548,18 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       uint8_t* orow = static_cast<uint8_t*>(L.out) + rrow * n * OUTB;
       const int32_t bias_lo = kRoundBiasBits - zero;
       const int32_t bias_hi = bias_lo + qmax;
+      uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
+      if (ng > 0) cw0 = load_codes16<WBITS>(crow + (((col0 + 16 * member) * WBITS) >> 3));
+      if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + 32 + 16 * member) * WBITS) >> 3));
+      int g = 0;
       for (int p = 0; p < NP; ++p) {
         const int pc = min(static_cast<int>(kPartCols), cols - p * static_cast<int>(kPartCols));
-        for (int c = 16 * member; c < pc; c += 32) {
+        for (int c = 16 * member; c < pc; c += 32, ++g) {
           const int cc = p * static_cast<int>(kPartCols) + c;
           const int64_t j = col0 + cc;
-          const uint4 cw = load_codes16<WBITS>(crow + ((j * WBITS) >> 3));
+          const uint4 cw = cw0;
+          cw0 = cw1;
+          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 64) * WBITS) >> 3));
           float v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();

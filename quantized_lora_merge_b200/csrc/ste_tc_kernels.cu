@@ -39,6 +39,7 @@ constexpr uint32_t kGBytes = kTileRows * kTileCols * 2;
 constexpr uint32_t kBoxBytes = kTileRows * 64 * 2;    // one 64-column box of the G tile
 constexpr int kMaxTcJobs = 64;
 constexpr int kMaxD2 = 8;                      // D2 accumulators (tile epilogues in flight)
+constexpr int kMaxStages = 4;                  // pipeline stages at most (host picks 2-4)
 
 struct alignas(64) SteTcJob {
   CUtensorMap g_map;          // G: dims {n, d}, box {64, 128}, 128B swizzle
@@ -111,6 +112,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ __align__(8) uint64_t drain_bar;
   // operands want 1024-byte alignment (the 128-byte swizzle repeats every 8 rows)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   const int RP = b.rp, S = b.stages;
@@ -146,6 +148,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
       mbar_init(&a_empty[q], 1);
     }
     abort_flag = 0;
+    mbar_init(&drain_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -166,12 +169,15 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
+      int armed[kMaxStages];
+      for (int q = 0; q < kMaxStages; ++q) armed[q] = -1;
       for (int64_t u = blockIdx.x; u < b.total_units && !abort_flag; u += gridDim.x) {
         const Unit x = decode_unit(b, u);
         const SteTcJob& J = b.job[x.job];
         for (int ct = x.ct0; ct < x.ct1; ++ct) {
           if (!mbar_wait_c(&empty[stage], ph ^ 1u, &abort_flag)) break;
           mbar_arrive_tx(&full[stage], kGBytes + b_bytes);
+          armed[stage] = static_cast<int>(ph);
           uint8_t* g = sG + stage * kGBytes;
           uint8_t* bt = sB + stage * b_bytes;
           const int32_t x0 = ct * kTileCols;
@@ -186,6 +192,8 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
           }
         }
       }
+      if (abort_flag)        // copies in flight land before the CTA goes away
+        for (int q = 0; q < S; ++q) drain_phase(&full[q], armed[q]);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -246,6 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
         tc_commit(&d1_full[ab]);
         tc_commit(&a_empty[ab]);
       }
+      if (abort_flag) drain_mma(&drain_bar);   // products in flight complete first
     }
   } else if (warp < 4) {
     // ---------------- A-block staging (64 threads, two rows each)
@@ -328,10 +337,6 @@ __global__ void __launch_bounds__(kTcThreads, 2) ste_tc_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (abort_flag) {
-      // let copies and products already in flight land before the memory goes
-      for (int k = 0; k < 2000; ++k) __nanosleep(1000);
-    }
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(b.tmem_cols)
                  : "memory");

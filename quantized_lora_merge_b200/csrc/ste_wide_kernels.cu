@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ __align__(8) uint64_t drain_bar;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   const int RP = b.rp, S = b.stages;
   // a stage: the G tile, then the pass's second operand (B tile: RP rows x
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
       mbar_init(&d_empty[q], 128);
     }
     abort_flag = 0;
+    mbar_init(&drain_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   const uint32_t tmem_cols = static_cast<uint32_t>(2 * RP);   // 128 or 256 (power of two)
@@ -144,6 +146,7 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
+      int armed[4] = {-1, -1, -1, -1};      // parity last armed per stage (host picks 2-4 stages)
       for (int64_t u = blockIdx.x; u < b.total_units && !abort_flag; u += gridDim.x) {
         const WUnit x = w_unit(b, u);
         const WJob& J = b.job[x.job];
@@ -156,6 +159,7 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
           const int32_t rb = static_cast<int32_t>(x.pass == 1 ? x.fixed : st);
           const int32_t ct = static_cast<int32_t>(x.pass == 1 ? st : x.fixed);
           mbar_arrive_tx(&full[stage], stage_bytes);
+          armed[stage] = static_cast<int>(ph);
           uint8_t* g = base + stage * stage_bytes;
           tma_load_2d(g, &J.g_map, ct * kWCols, rb * kWRows, &full[stage]);
           tma_load_2d(g + kWBox, &J.g_map, ct * kWCols + 64, rb * kWRows, &full[stage]);
@@ -176,6 +180,8 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
         }
         if (!ok) break;
       }
+      if (abort_flag)        // copies in flight land before the CTA goes away
+        for (int q = 0; q < S; ++q) drain_phase(&full[q], armed[q]);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -229,6 +235,7 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
           bph ^= 1u;
         }
       }
+      if (abort_flag) drain_mma(&drain_bar);   // products in flight complete first
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: TMEM lane = row of dA (pass 1) / column of dB (pass 2)
@@ -271,9 +278,6 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (abort_flag) {
-      for (int k = 0; k < 2000; ++k) __nanosleep(1000);
-    }
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
   }

@@ -67,6 +67,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           unsigned int* timeouts) {
   return mbar_wait_for(bar, parity, abort_flag, timeouts, kWaitNs);
 }
+// Drain helpers for a CTA that gave up. A TMA copy completes on the mbarrier
+// phase it was armed on: wait (bounded) for the last phase armed on `bar`
+// (parity 0 or 1; -1 = never armed). tcgen05.commit arrives once every
+// tensor-core operation the calling thread issued has completed: commit to
+// a fresh single-arrival barrier and wait (bounded) for its first phase.
+__device__ __forceinline__ void drain_phase(uint64_t* bar, int parity) {
+  if (parity < 0) return;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try(bar, static_cast<uint32_t>(parity)) && global_ns() - t0 < kWaitNs) {
+  }
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar);
+__device__ __forceinline__ void drain_mma(uint64_t* fresh_bar) {
+  tc_commit(fresh_bar);
+  drain_phase(fresh_bar, 0);
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {
   asm volatile(

@@ -41,6 +41,7 @@ constexpr int kTgRows = 128;                      // tile rows (M)
 constexpr int kTgCols = 128;                      // tile columns (N)
 constexpr uint32_t kAtomBytes = kTgRows * 128;    // 128 rows x 32 fp32 (one K atom)
 constexpr int kMaxTgJobs = 48;
+constexpr int kTgMaxStages = 6;                   // pipeline stages at most (host picks 2-6)
 
 __device__ unsigned int g_tg_timeouts;
 
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ __align__(8) uint64_t drain_bar;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t{1023});
   const int S = b.stages;
   const uint32_t op_bytes = static_cast<uint32_t>(b.kp_max / 32) * kAtomBytes;   // one operand tile
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
       mbar_init(&d_empty[q], 128);
     }
     abort_flag = 0;
+    mbar_init(&drain_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -201,6 +204,8 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
     if (lane == 0) {
       int stage = 0, ucount = 0;
       uint32_t ph = 0;
+      int armed[kTgMaxStages], armed_a = -1;     // parity last armed per barrier (-1: never)
+      for (int q = 0; q < kTgMaxStages; ++q) armed[q] = -1;
       for (int64_t u = blockIdx.x; u < b.total_units && !abort_flag; u += gridDim.x, ++ucount) {
         const TgUnit x = tg_unit(b, u);
         const TgJob& J = b.job[x.job];
@@ -208,6 +213,7 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
         const int32_t y0 = static_cast<int32_t>(x.i0);
         if (!wait_c(a_empty, (static_cast<uint32_t>(ucount) & 1u) ^ 1u, &abort_flag)) break;
         mbar_arrive_tx(a_full, 2u * atoms * kAtomBytes);
+        armed_a = ucount & 1;
         for (int at = 0; at < atoms; ++at) {
           tma_load_2d(sA + at * kAtomBytes, &J.a_hi, at * 32, y0, a_full);
           tma_load_2d(sA + op_bytes + at * kAtomBytes, &J.a_lo, at * 32, y0, a_full);
@@ -219,6 +225,7 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
             break;
           }
           mbar_arrive_tx(&full[stage], 2u * atoms * kAtomBytes);
+          armed[stage] = static_cast<int>(ph);
           uint8_t* dst = sB + stage * 2 * op_bytes;
           for (int at = 0; at < atoms; ++at) {
             tma_load_2d(dst + at * kAtomBytes, &J.b_hi, at * 32, ct * kTgCols, &full[stage]);
@@ -230,6 +237,10 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
           }
         }
         if (!ok) break;
+      }
+      if (abort_flag) {      // copies in flight land before the CTA goes away
+        for (int q = 0; q < S; ++q) drain_phase(&full[q], armed[q]);
+        drain_phase(a_full, armed_a);
       }
     }
   } else if (warp == 1) {
@@ -276,6 +287,7 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
         if (!ok) break;
         tc_commit(a_empty);
       }
+      if (abort_flag) drain_mma(&drain_bar);   // products in flight complete first
     }
   } else if (warp >= 4) {
     // ---------------- epilogue: TMEM lane = tile row
@@ -327,9 +339,6 @@ __global__ void __launch_bounds__(kTgThreads, 1) t_gemm_kernel(const __grid_cons
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    if (abort_flag) {
-      for (int k = 0; k < 2000; ++k) __nanosleep(1000);
-    }
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * kTgCols)
                  : "memory");

@@ -179,7 +179,7 @@ def test_merge_with_zero_adapter(monkeypatch, kernel, d, n, r, w_bits, out_bits,
     ([notes] section 1, AQS), so A B = 0 and U = s + R* / D exactly. Through
     both kernel families."""
     monkeypatch.setenv("INTLORA_MERGE_KERNEL", kernel)
-    spec = spec_for(d, n, r, w_bits, variant, out_bits, sid=900 + d)
+    spec = spec_for(d, n, r, w_bits, variant, out_bits if variant == "mul" else 4, sid=900 + d)
     inp = _oracle_prepared(spec)
     inp["A"] = np.zeros_like(inp["A"])
     got = gpu_merge([spec], [inp])[0]

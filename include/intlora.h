@@ -420,6 +420,44 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
  * word); the library has no counterpart of this on the pages. */
 uint32_t intlora_device_timeouts(void);
 
+/* --------------------------------------------------------------------------
+ * Training backward of one IntLoRA linear Y = X W'^T, W' the fake-quantized
+ * merged weight of the forward (intlora_fakequant_bf16), the gradient
+ * reaching the low-rank factors through the straight-through estimator
+ * [notes, 两种实现版本: training passes the quantizers with the STE; the
+ * efficiency table times these steps]. Per job, from bf16 inputs:
+ *     dX = dY W'                       (tokens x n)
+ *     dA = G B^T,  dB = A^T G,  G = dY^T X  (the gradient on W', d x n)
+ * G is never formed: with Z1 = X B^T and Z2 = dY A (tokens x r),
+ * dA = dY^T Z1 and dB = Z2^T X, every product on the tensor cores with fp32
+ * accumulation (Z enters the last products as two exact bf16 halves, so
+ * they stay fp32-faithful).
+ *
+ * X: bf16 tokens x n; dY: bf16 tokens x d; W: bf16 d x n; A: bf16 d x r;
+ * B: bf16 r x n; all row-major, X, dY, W, B 16-byte aligned. Outputs (fp32,
+ * row-major, 16-byte aligned): dX tokens x n, dA d x r, dB r x n; written,
+ * not accumulated. Requires tokens >= 1, d and n multiples of 8, 1 <= r <= 64.
+ * The workspace (intlora_train_backward_workspace_size, 256-byte aligned
+ * regions per job) holds W'^T, A^T, Z1, Z2 and the halves' products.
+ * ------------------------------------------------------------------------ */
+typedef struct intlora_train_backward_job {
+    const void* X;
+    const void* dY;
+    const void* W;
+    const void* A;
+    const void* B;
+    int64_t tokens, d, n;
+    int32_t r;
+    float* dX;
+    float* dA;
+    float* dB;
+} intlora_train_backward_job;
+
+size_t intlora_train_backward_workspace_size(const intlora_train_backward_job* jobs, int32_t count);
+
+intlora_status intlora_train_backward_batched(const intlora_train_backward_job* jobs, int32_t count,
+                                              void* ws, size_t ws_bytes, void* stream);
+
 /* Device health check: synchronizes the device, then returns
  * INTLORA_ERR_TIMEOUT (with the count in intlora_last_error()) when bounded
  * device-side waits gave up since the previous intlora_device_status() call

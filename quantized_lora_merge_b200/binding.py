@@ -69,6 +69,12 @@ class intlora_linear_job(ctypes.Structure):
                 ("Y", _c_ptr), ("y_bf16", _c_i32)]
 
 
+class intlora_train_backward_job(ctypes.Structure):
+    _fields_ = [("X", _c_ptr), ("dY", _c_ptr), ("W", _c_ptr), ("A", _c_ptr), ("B", _c_ptr),
+                ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("r", _c_i32),
+                ("dX", _c_ptr), ("dA", _c_ptr), ("dB", _c_ptr)]
+
+
 class intlora_int_gemm_job(ctypes.Structure):
     _fields_ = [("X", _c_ptr), ("x_scale", _c_ptr), ("W", _c_ptr), ("w_scale", _c_ptr),
                 ("tokens", _c_i64), ("d", _c_i64), ("n", _c_i64), ("Y", _c_ptr),
@@ -112,6 +118,9 @@ _SIGNATURES = {
     "intlora_fakequant_bf16": (ctypes.c_int, [_c_ptr, _c_i32, _c_ptr, _c_i64, _c_i64, _c_ptr,
                                               _c_ptr]),
     "intlora_linear_bf16_batched": (ctypes.c_int, [_P(intlora_linear_job), _c_i32, _c_ptr]),
+    "intlora_train_backward_workspace_size": (_c_size, [_P(intlora_train_backward_job), _c_i32]),
+    "intlora_train_backward_batched": (ctypes.c_int, [_P(intlora_train_backward_job), _c_i32,
+                                                      _c_ptr, _c_size, _c_ptr]),
     "intlora_fakequant_bf16_batched": (ctypes.c_int, [_P(intlora_fakequant_job), _c_i32, _c_ptr]),
     "intlora_int_pack": (ctypes.c_int, [_c_ptr, _c_i32, _c_i64, _c_i64, _c_i32, _c_ptr, _c_ptr,
                                         _c_ptr]),
@@ -294,6 +303,25 @@ class LinearJob:
                                   _ptr(self.Y), int(self.Y.dtype == torch.bfloat16))
 
 
+@dataclass
+class TrainBackwardJob:
+    X: object                       # bf16 [tokens, n]
+    dY: object                      # bf16 [tokens, d]
+    W: object                       # bf16 [d, n] (fake-quantized merged weight)
+    A: object                       # bf16 [d, r]
+    B: object                       # bf16 [r, n]
+    dX: object                      # fp32 [tokens, n]
+    dA: object                      # fp32 [d, r]
+    dB: object                      # fp32 [r, n]
+
+    def to_c(self) -> intlora_train_backward_job:
+        tokens, n = self.X.shape
+        d, r = self.A.shape
+        return intlora_train_backward_job(_ptr(self.X), _ptr(self.dY), _ptr(self.W), _ptr(self.A),
+                                          _ptr(self.B), tokens, d, n, r, _ptr(self.dX),
+                                          _ptr(self.dA), _ptr(self.dB))
+
+
 def _array(struct, items):
     if isinstance(items, Descriptors):
         if items.struct is not struct:
@@ -331,7 +359,8 @@ class Descriptors:
 Descriptors._STRUCT = {AuxJob: intlora_aux_job, Layer: intlora_layer,
                        MergeOut: intlora_merge_out, SteJob: intlora_ste_job,
                        IntGemmJob: intlora_int_gemm_job, LinearJob: intlora_linear_job,
-                       FakeQuantJob: intlora_fakequant_job}
+                       FakeQuantJob: intlora_fakequant_job,
+                       TrainBackwardJob: intlora_train_backward_job}
 
 
 # ---------------------------------------------------------------------------
@@ -482,6 +511,17 @@ def intlora_fakequant_bf16(q, sbar, w_out, stream=None) -> None:
 def intlora_linear_bf16_batched(jobs: Sequence[LinearJob], stream=None) -> None:
     _check(lib().intlora_linear_bf16_batched(_array(intlora_linear_job, jobs), len(jobs),
                                              _stream(stream)))
+
+
+def intlora_train_backward_workspace_size(jobs: Sequence[TrainBackwardJob]) -> int:
+    return lib().intlora_train_backward_workspace_size(_array(intlora_train_backward_job, jobs),
+                                                       len(jobs))
+
+
+def intlora_train_backward_batched(jobs: Sequence[TrainBackwardJob], ws=None, stream=None) -> None:
+    p, nb = _ws(ws)
+    _check(lib().intlora_train_backward_batched(_array(intlora_train_backward_job, jobs), len(jobs),
+                                                p, nb, _stream(stream)))
 
 
 def intlora_fakequant_bf16_batched(jobs: Sequence[FakeQuantJob], stream=None) -> None:

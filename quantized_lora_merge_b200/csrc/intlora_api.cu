@@ -1076,6 +1076,43 @@ uint32_t intlora_device_timeouts(void) {
 }
 
 namespace {
+
+// Workspace regions of one training-backward job, in order (each 256-byte aligned).
+struct TbWs {
+  size_t wt, at, z1, z2, zs1, zs2, b0, o1, o2, j1, j2, total;
+};
+TbWs tb_ws_layout(const intlora_train_backward_job& j) {
+  TbWs w;
+  const size_t T = static_cast<size_t>(j.tokens), d = static_cast<size_t>(j.d), n = static_cast<size_t>(j.n);
+  const size_t r = static_cast<size_t>(j.r);
+  w.wt = round256(n * d * 2);
+  w.at = round256(r * d * 2);
+  w.z1 = w.z2 = round256(T * r * 4);
+  w.zs1 = w.zs2 = round256(T * 2 * r * 2);
+  w.b0 = round256(2 * r * std::max(d, n) * 2);
+  w.o1 = round256(2 * r * d * 4);
+  w.o2 = round256(2 * r * n * 4);
+  w.j1 = w.j2 = round256(T * 2 * r * 4);
+  w.total = w.wt + w.at + w.z1 + w.z2 + w.zs1 + w.zs2 + w.b0 + w.o1 + w.o2 + w.j1 + w.j2;
+  return w;
+}
+
+intlora_status check_tb(const intlora_train_backward_job& j, int k) {
+  if (j.tokens < 1 || j.d < 8 || j.n < 8 || j.d % 8 != 0 || j.n % 8 != 0)
+    return fail(INTLORA_ERR_INVALID_ARG, "train-backward job %d: tokens >= 1, d and n multiples of 8 required", k);
+  if (j.r < 1 || j.r > 64)
+    return fail(INTLORA_ERR_INVALID_ARG, "train-backward job %d: r must be in [1, 64]", k);
+  if (j.tokens > (int64_t{1} << 31) || j.d > (int64_t{1} << 31) || j.n > (int64_t{1} << 31))
+    return fail(INTLORA_ERR_INVALID_ARG, "train-backward job %d: tokens, d, n must be <= 2^31", k);
+  if (j.X == nullptr || j.dY == nullptr || j.W == nullptr || j.A == nullptr || j.B == nullptr ||
+      j.dX == nullptr || j.dA == nullptr || j.dB == nullptr)
+    return fail(INTLORA_ERR_INVALID_ARG, "train-backward job %d: every pointer is required", k);
+  if (!aligned16(j.X) || !aligned16(j.dY) || !aligned16(j.W) || !aligned16(j.B) || !aligned16(j.dX) ||
+      !aligned16(j.dA) || !aligned16(j.dB) || (reinterpret_cast<uintptr_t>(j.A) & 1u) != 0)
+    return fail(INTLORA_ERR_INVALID_ARG, "train-backward job %d: X, dY, W, B and outputs must be 16-byte aligned", k);
+  return INTLORA_OK;
+}
+
 std::mutex g_status_mutex;
 uint32_t g_timeouts_reported = 0;
 }
@@ -1093,6 +1130,85 @@ intlora_status intlora_device_status(void) {
                 "calls in between are not valid",
                 fresh);
   }
+  return INTLORA_OK;
+}
+
+size_t intlora_train_backward_workspace_size(const intlora_train_backward_job* jobs, int32_t count) {
+  size_t total = 0;
+  for (int32_t k = 0; k < count && jobs != nullptr; ++k) total += tb_ws_layout(jobs[k]).total;
+  return total;
+}
+
+intlora_status intlora_train_backward_batched(const intlora_train_backward_job* jobs, int32_t count, void* ws,
+                                              size_t ws_bytes, void* stream) {
+  g_last_error[0] = '\0';
+  if (count < 0 || (count > 0 && jobs == nullptr))
+    return fail(INTLORA_ERR_INVALID_ARG, "jobs must be a non-NULL array, count >= 0");
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_status s = check_tb(jobs[k], k);
+    if (s != INTLORA_OK) return s;
+  }
+  if (count == 0) return INTLORA_OK;
+  const size_t need = intlora_train_backward_workspace_size(jobs, count);
+  if (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(INTLORA_ERR_WORKSPACE, "workspace of %zu bytes (256-byte aligned) required", need);
+  if (!int_gemm_supported())
+    return fail(INTLORA_ERR_UNSUPPORTED, "training backward: the driver's tensor-map encoder is unavailable");
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<TransposeJob> tr;
+  std::vector<intlora_linear_job> lin;
+  std::vector<SplitZJob> split;
+  std::vector<intlora_ste_job> ste;
+  std::vector<CombineJob> comb;
+  char* p = static_cast<char*>(ws);
+  for (int32_t k = 0; k < count; ++k) {
+    const intlora_train_backward_job& j = jobs[k];
+    const TbWs w = tb_ws_layout(j);
+    uint16_t* wt = reinterpret_cast<uint16_t*>(p);
+    uint16_t* at = reinterpret_cast<uint16_t*>(p + w.wt);
+    float* z1 = reinterpret_cast<float*>(p + w.wt + w.at);
+    float* z2 = reinterpret_cast<float*>(p + w.wt + w.at + w.z1);
+    uint16_t* zs1 = reinterpret_cast<uint16_t*>(p + w.wt + w.at + w.z1 + w.z2);
+    uint16_t* zs2 = reinterpret_cast<uint16_t*>(p + w.wt + w.at + w.z1 + w.z2 + w.zs1);
+    char* b0 = p + w.wt + w.at + w.z1 + w.z2 + w.zs1 + w.zs2;
+    float* o1 = reinterpret_cast<float*>(b0 + w.b0);
+    float* o2 = reinterpret_cast<float*>(b0 + w.b0 + w.o1);
+    float* j1 = reinterpret_cast<float*>(b0 + w.b0 + w.o1 + w.o2);
+    float* j2 = reinterpret_cast<float*>(b0 + w.b0 + w.o1 + w.o2 + w.j1);
+    // W'^T (n x d) and A^T (r x d): every GEMM operand K-major
+    tr.push_back(TransposeJob{static_cast<const uint16_t*>(j.W), wt, j.d, j.n, 0});
+    tr.push_back(TransposeJob{static_cast<const uint16_t*>(j.A), at, j.d, j.r, 0});
+    // dX = dY W' (K = d), Z1 = X B^T (K = n), Z2 = dY A (K = d), fp32 out
+    lin.push_back(intlora_linear_job{j.dY, wt, j.tokens, j.n, j.d, j.dX, 0});
+    lin.push_back(intlora_linear_job{j.X, j.B, j.tokens, j.r, j.n, z1, 0});
+    lin.push_back(intlora_linear_job{j.dY, at, j.tokens, j.r, j.d, z2, 0});
+    split.push_back(SplitZJob{z1, zs1, j.tokens, j.r});
+    split.push_back(SplitZJob{z2, zs2, j.tokens, j.r});
+    // one pass over dY: [Z1_hi | Z1_lo]^T dY (2r x d); one over X: [Z2_hi | Z2_lo]^T X (2r x n);
+    // the STE kernel's other product (against the zero B) is discarded
+    intlora_ste_job s1;
+    std::memset(&s1, 0, sizeof s1);
+    s1.G = j.dY; s1.A = zs1; s1.B = b0; s1.d = j.tokens; s1.n = j.d; s1.r = 2 * j.r; s1.dA = j1; s1.dB = o1;
+    intlora_ste_job s2 = s1;
+    s2.G = j.X; s2.A = zs2; s2.n = j.n; s2.dA = j2; s2.dB = o2;
+    ste.push_back(s1);
+    ste.push_back(s2);
+    comb.push_back(CombineJob{o1, j.dA, j.d, j.r, 1});     // dA = (top + bottom)^T
+    comb.push_back(CombineJob{o2, j.dB, j.n, j.r, 0});     // dB = top + bottom
+    const cudaError_t e = cudaMemsetAsync(b0, 0, w.b0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "zero operand fill");
+    p += w.total;
+  }
+  cudaError_t e = launch_transpose_bf16(tr.data(), static_cast<int>(tr.size()), st);
+  if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
+  intlora_status s = intlora_linear_bf16_batched(lin.data(), static_cast<int32_t>(lin.size()), stream);
+  if (s != INTLORA_OK) return s;
+  e = launch_split_hilo(split.data(), static_cast<int>(split.size()), st);
+  if (e != cudaSuccess) return cuda_fail(e, "split launch");
+  s = intlora_ste_backward_batched(ste.data(), static_cast<int32_t>(ste.size()), nullptr, 0, stream);
+  if (s != INTLORA_OK) return s;
+  e = launch_combine_halves(comb.data(), static_cast<int>(comb.size()), st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
   return INTLORA_OK;
 }
 

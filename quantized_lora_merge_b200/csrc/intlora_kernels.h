@@ -317,6 +317,30 @@ unsigned int int_gemm_timeouts();
 // Sets the calling thread's intlora_last_error() message.
 void set_last_error(const char* message);
 
+// Glue kernels of the training backward (train_backward_kernels.cu).
+struct TransposeJob {        // out (cols x rows) = in (rows x cols)^T, bf16
+  const uint16_t* in;
+  uint16_t* out;
+  int64_t rows, cols;
+  int64_t block_begin;       // set by the launcher
+};
+struct SplitZJob {           // zs (rows x 2r bf16) = [hi | lo] of z (rows x r fp32)
+  const float* z;
+  uint16_t* zs;
+  int64_t rows;
+  int32_t r;
+};
+struct CombineJob {          // out = in[0:r] + in[r:2r] (in: 2r x cols fp32); transposed: out is cols x r
+  const float* in;
+  float* out;
+  int64_t cols;
+  int32_t r;
+  int32_t transposed;
+};
+cudaError_t launch_transpose_bf16(const TransposeJob* jobs, int count, cudaStream_t s);
+cudaError_t launch_split_hilo(const SplitZJob* jobs, int count, cudaStream_t s);
+cudaError_t launch_combine_halves(const CombineJob* jobs, int count, cudaStream_t s);
+
 // Self-test of the bounded waits: one mbarrier that nothing completes, waited
 // on for limit_ns (selftest_kernels.cu); *completed (device int, optional)
 // receives 0 when the wait gave up.

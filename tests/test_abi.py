@@ -245,3 +245,28 @@ def test_launch_counter_is_monotonic(lib):
     a = lib.intlora_kernel_launches()
     lib.intlora_merge_out_bytes(0, 8, 8)           # launches nothing
     assert lib.intlora_kernel_launches() == a
+
+
+def _tb_job(**kw):
+    fake = 0x100000
+    f = dict(X=fake, dY=fake, W=fake, A=fake, B=fake, tokens=64, d=64, n=128, r=4,
+             dX=fake, dA=fake, dB=fake)
+    f.update(kw)
+    return B.intlora_train_backward_job(**f)
+
+
+@pytest.mark.parametrize("field,value", [("d", 12), ("n", 0), ("tokens", 0), ("r", 0), ("r", 65),
+                                         ("X", None), ("dB", None), ("W", 0x100008)])
+def test_train_backward_rejects(lib, field, value):
+    job = _tb_job(**{field: value})
+    st = lib.intlora_train_backward_batched(ctypes.byref(job), 1, 0x100000, 1 << 30, None)
+    assert st == 1, lib.intlora_last_error()
+
+
+def test_train_backward_workspace_checked(lib):
+    job = _tb_job()
+    need = lib.intlora_train_backward_workspace_size(ctypes.byref(job), 1)
+    assert need > 0 and need % 256 == 0
+    assert lib.intlora_train_backward_batched(ctypes.byref(job), 1, None, 0, None) == 3
+    assert lib.intlora_train_backward_batched(ctypes.byref(job), 1, 0x100000, need - 1, None) == 3
+    assert lib.intlora_train_backward_batched(ctypes.byref(job), 0, None, 0, None) == 0

@@ -61,7 +61,11 @@ namespace {
 using namespace tc;
 
 constexpr double kLn2 = 0.69314718055994530942;
-constexpr int kQuantWarps = 8;
+#ifndef INTLORA_MTC_QUANT_WARPS
+#define INTLORA_MTC_QUANT_WARPS 8
+#endif
+constexpr int kQuantWarps = INTLORA_MTC_QUANT_WARPS;   // a multiple of 4: kMembers warps per lane quarter
+constexpr int kMembers = kQuantWarps / 4;
 constexpr int kQuantThreads = 32 * kQuantWarps;
 constexpr int kMtcThreads = 32 * (4 + kQuantWarps);
 constexpr int kRows = 128;                               // rows per unit = tensor-memory lanes
@@ -203,8 +207,8 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
   const int G = b.group;
   uint8_t* sA = base;                                                   // [atom][hi, lo]
   uint8_t* sB = sA + static_cast<size_t>(b.atoms_max) * 2 * kABytes;  // [stage][hi, lo]
-  uint2* ext = reinterpret_cast<uint2*>(sB + static_cast<size_t>(NS) * 2 * kBPart);   // [2][128]
-  float* rcp_tab = reinterpret_cast<float*>(ext + 2 * kRows);          // 1/D, D in [-255, 255]
+  uint2* ext = reinterpret_cast<uint2*>(sB + static_cast<size_t>(NS) * 2 * kBPart);   // [kMembers][128]
+  float* rcp_tab = reinterpret_cast<float*>(ext + kMembers * kRows);   // 1/D, D in [-255, 255]
   uint64_t* bars = reinterpret_cast<uint64_t*>(rcp_tab + 512);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
@@ -372,7 +376,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
   } else if (warp >= 4) {
     // ---------------- quantizers: lane i of quarter q = row 32 q + i of the unit
     const int quarter = warp & 3;
-    const int member = (warp - 4) >> 2;            // 0 or 1: alternate 16-column groups
+    const int member = (warp - 4) >> 2;            // 0 .. kMembers - 1: every kMembers-th 16-column group
     const int row_u = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int qmax = (1 << b.bits) - 1;
@@ -416,25 +420,26 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
           if (nrow < L2.d && ncol0 < L2.n) {
             const int64_t bytes = (min64(S, L2.n - ncol0) * WBITS) >> 3;
             const uint8_t* q = L2.codes + nrow * L2.ld_w + ((ncol0 * WBITS) >> 3);
-            for (int64_t o = member * 128; o < bytes; o += 256) prefetch_l2(q + o);
+            for (int64_t o = member * 128; o < bytes; o += 128 * kMembers) prefetch_l2(q + o);
           }
         }
       }
 
       // ---- phase A: T -> U, row extrema, U parked in tensor memory
       // This thread's 16-column groups are g = 0 .. ng - 1 at slice column
-      // 32 g + 16 member, in part order; each group's codes are loaded two
-      // groups ahead (the loads are the longest latency of the loop).
-      const int ng = cols >> 5;
+      // 16 (kMembers g + member), in part order; each group's codes are
+      // loaded two groups ahead (the loads are the longest latency of the loop).
+      constexpr int kStep = 16 * kMembers;                      // columns between a thread's groups
+      const int ng = (cols >> 4) > member ? ((cols >> 4) - member + kMembers - 1) / kMembers : 0;
       float hi = 0.0f, lo = 0.0f;
       bool ok = true;
       {
         uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
         if (ng > 0) cw0 = load_codes16<WBITS>(crow + (((col0 + 16 * member) * WBITS) >> 3));
-        if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + 32 + 16 * member) * WBITS) >> 3));
+        if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + kStep + 16 * member) * WBITS) >> 3));
         int have_part = -1;
         for (int g = 0; g < ng; ++g) {
-          const int cc = 32 * g + 16 * member;                 // column in the slice
+          const int cc = kStep * g + 16 * member;              // column in the slice
           const int p = cc >> 7;
           if (p != have_part) {
             if (!wait_m(&t_full[p], up, &abort_flag)) {
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
           const int64_t j = col0 + cc;
           const uint4 cw = cw0;
           cw0 = cw1;
-          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 64) * WBITS) >> 3));
+          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 2 * kStep) * WBITS) >> 3));
           float v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();
@@ -484,14 +489,19 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       tmem_st_wait();
       if (!valid) hi = lo = 0.0f;
 
-      // ---- row extrema: the two members of this CTA, then the group
+      // ---- row extrema: the members of this CTA, then the group
       ext[member * kRows + row_u] = make_uint2(ord_abs(hi), ord_abs(lo));
       mbar_arrive(ext_bar);
       if (!wait_m(ext_bar, up, &abort_flag) || !ok) break;
       const uint32_t tag = static_cast<uint32_t>(ucount) + 1u;
       if (sender) {
-        const uint2 e0 = ext[row_u], e1 = ext[kRows + row_u];
-        my_slots[(static_cast<int64_t>(up) * G + rank) * kRows + row_u] = make_uint2(max(e0.x, e1.x), max(e0.y, e1.y));
+        uint2 e = ext[row_u];
+#pragma unroll
+        for (int m = 1; m < kMembers; ++m) {
+          const uint2 f = ext[m * kRows + row_u];
+          e = make_uint2(max(e.x, f.x), max(e.y, f.y));
+        }
+        my_slots[(static_cast<int64_t>(up) * G + rank) * kRows + row_u] = e;
         __threadfence();
         mbar_arrive(sent_bar);
         if (row_u == 0) {
@@ -550,16 +560,16 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       const int32_t bias_hi = bias_lo + qmax;
       uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
       if (ng > 0) cw0 = load_codes16<WBITS>(crow + (((col0 + 16 * member) * WBITS) >> 3));
-      if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + 32 + 16 * member) * WBITS) >> 3));
+      if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + kStep + 16 * member) * WBITS) >> 3));
       int g = 0;
       for (int p = 0; p < NP; ++p) {
         const int pc = min(static_cast<int>(kPartCols), cols - p * static_cast<int>(kPartCols));
-        for (int c = 16 * member; c < pc; c += 32, ++g) {
+        for (int c = 16 * member; c < pc; c += kStep, ++g) {
           const int cc = p * static_cast<int>(kPartCols) + c;
           const int64_t j = col0 + cc;
           const uint4 cw = cw0;
           cw0 = cw1;
-          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 64) * WBITS) >> 3));
+          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 2 * kStep) * WBITS) >> 3));
           float v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();
@@ -630,7 +640,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
 // share an SM: each allocates all 512 tensor-memory columns.
 size_t mtc_smem_bytes(int atoms_max, int stages) {
   const size_t need = 1024 + static_cast<size_t>(atoms_max) * 2 * kABytes + static_cast<size_t>(stages) * 2 * kBPart +
-                      2 * kRows * 8 + 512 * 4 + (6 + 2 * kMaxParts + 2 * stages) * 8;
+                      kMembers * kRows * 8 + 512 * 4 + (6 + 2 * kMaxParts + 2 * stages) * 8;
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
 

@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--config", default="llama3_8b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the integer-GEMM and training-step legs of the default line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--op", default="step", choices=["step", "int_gemm", "train_forward"],
                     help="step: the merge hot path (default); int_gemm: the integer "
@@ -129,8 +131,10 @@ ALU_LANES_PER_SM_CLK = 128       # FP32/INT32 lanes per SM per clock on sm_100
 NUM_SMS = 148
 
 
-# sources the dominant (team) kernel is compiled from
-DOMINANT_SOURCES = ("team_kernels.cu", "intlora_device.cuh", "intlora_kernels.h")
+# sources the fused merge kernel is compiled from (a stored ncu figure is used
+# only while they hash to the value recorded beside it)
+MERGE_TC_SOURCES = ("merge_tc_kernels.cu", "intlora_device.cuh", "tcgen05_util.cuh", "intlora_kernels.h")
+DOMINANT_SOURCES = MERGE_TC_SOURCES
 
 
 def csrc_hash(sources=None):
@@ -145,10 +149,11 @@ def csrc_hash(sources=None):
     return h.hexdigest()
 
 
-def profiled_traffic(name, sources=None):
-    """dram__bytes_read.sum + dram__bytes_write.sum per launch from the ncu
-    summary profiles/<name>.md, or None when absent or when the kernels have
-    changed since it was taken."""
+def profiled_traffic(name, sources=None, field="dram_bytes_per_launch"):
+    """dram__bytes_read.sum + dram__bytes_write.sum (per launch, or per element
+    with field="dram_bytes_per_element") from the ncu summary
+    profiles/<name>.md, or None when absent or when the kernels have changed
+    since it was taken."""
     p = Path(__file__).resolve().parent / "profiles" / f"{name}.md"
     if not p.exists():
         return None
@@ -160,7 +165,7 @@ def profiled_traffic(name, sources=None):
     if fields.get("csrc_sha256") != csrc_hash(sources):
         return None
     try:
-        return float(fields["dram_bytes_per_launch"])
+        return float(fields[field])
     except (KeyError, ValueError):
         return None
 
@@ -425,12 +430,25 @@ def main():
         stages[name] = {"ms": ms, "algorithmic_GB": per_stage_bytes[name] / 1e9,
                         "GB_s": gbs, "frac_of_hbm": gbs / hbm_peak}
     stages["merge"]["elements_per_s"] = sum(l.numel for l in layers) / (stage_ms["merge"] / 1e3)
-    # dominant kernel: the merge's team kernel (one launch per step); it is
-    # bound by ALU issue (Philox + Laplace per element), so its roofline is the
-    # SM lane-issue rate at the measured SM clock; HBM fraction reported beside
+    # The metric's kernel: the merge stage. Layers of rank >= 16 whose rows are a
+    # multiple of 32 columns run on the fused tensor-core merge kernel (one
+    # cooperative launch per row width), the rest on the team / row-tile
+    # kernels (the library's routing). Its roofline is HBM (algorithmic bytes
+    # of W_round, A, B and the outputs); the lane-issue view (modelled
+    # operations per element over the SM lane rate at the sampled clock)
+    # is reported beside it.
     sm_mhz = clk.get("sm_mhz") or 1965.0
     alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
     alu_achieved = sum(merge_ops(l) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
+    fused = (not args.dist) and all(l.r >= 16 and l.n % 32 == 0 for l in layers)
+    kernel_name = ("merge_tc_kernel (fused tensor-core merge)" if fused else
+                   "team / row-tile merge kernels" if not args.dist else
+                   "merge row-tile kernel (general auxiliary law)")
+    traffic = None
+    if fused:
+        per_el = profiled_traffic(f"merge_tc_kernel_{args.config}", MERGE_TC_SOURCES, "dram_bytes_per_element")
+        if per_el is not None:
+            traffic = per_el * sum(l.numel for l in layers)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -440,17 +458,17 @@ def main():
         "sharding": "layers split across ranks" if args.shard else "one copy of the workload per rank",
         "hbm_GB_s_merge": stages["merge"]["GB_s"],
         "hbm_frac_merge": stages["merge"]["frac_of_hbm"],
-        "roofline": {"bound": "alu", "kernel": ("merge team kernel (MUL, 1 launch per step)"
-                                                if not args.dist else
-                                                "merge row-tile kernel (general auxiliary law)"),
-                     "achieved": alu_achieved, "peak": alu_peak, "unit": "Top/s",
-                     "frac": alu_achieved / alu_peak,
-                     "peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
-                     "ops_per_element": merge_ops(layers[0]) / layers[0].numel,
-                     "hbm_achieved_GB_s": stages["merge"]["GB_s"], "hbm_peak_GB_s": hbm_peak,
-                     "hbm_peak_source": peak_kind, "hbm_frac": stages["merge"]["frac_of_hbm"],
-                     "traffic": (profiled_traffic("team_kernel_mul_sd_unet")
-                                 if not args.dist else None)},
+        "roofline": {"bound": "hbm", "kernel": kernel_name, "stage": "merge (every launch of the stage)",
+                     "achieved": stages["merge"]["GB_s"], "peak": hbm_peak, "unit": "GB/s",
+                     "frac": stages["merge"]["frac_of_hbm"],
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_step": per_stage_bytes["merge"],
+                     "traffic": traffic,
+                     "traffic_unit": "DRAM bytes per step of the stage (ncu bytes per element x elements)",
+                     "alu_achieved_Top_s": alu_achieved, "alu_peak_Top_s": alu_peak,
+                     "alu_frac_modelled": alu_achieved / alu_peak,
+                     "alu_peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
+                     "ops_per_element_modelled": merge_ops(layers[0]) / layers[0].numel},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": launches,
@@ -461,10 +479,136 @@ def main():
                           world, elements, masked_ste=args.masked_ste)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
+    if not args.no_extra:
+        # the next rows of the path, measured on the same GPU after the main
+        # workload is released: every rank runs them (no collective inside)
+        del path, states, arena_in, arena_out
+        torch.cuda.empty_cache()
+        launches0 = Bnd.intlora_kernel_launches()
+        line["next_int_gemm"] = int_gemm_leg(device, planes=1, tokens=4096, steps=50)
+        line["next_train_step"] = train_step_leg(device, tokens=4096, steps=10)
+        line["next_legs_gpu_launches"] = Bnd.intlora_kernel_launches() - launches0
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def int_gemm_leg(device, planes, tokens, steps):
+    """Integer inference GEMM on merged weights (the four DiT-3072 block
+    linears at `tokens` tokens, merged weights as `planes` int8 digit planes,
+    one batched call per step); CUDA-event time, int8 tensor Top/s and the
+    fraction of 2 x the measured bf16 dense peak."""
+    import torch
+
+    from quantized_lora_merge_b200 import binding as B
+    from quantized_lora_merge_b200 import workloads as wl
+    bound = wl.INT_GEMM_BOUNDS[GEMM_KIND[planes]]
+    jobs, shapes = [], []
+    for k, (d, n) in enumerate(GEMM_SHAPES):
+        X, xs, Q, ws = wl.int_gemm_device(tokens, d, n, bound, device, salt=k)
+        packed = torch.empty((d, planes, n), dtype=torch.int8, device=device)
+        B.intlora_int_pack(Q, planes, packed)
+        del Q
+        jobs.append(B.IntGemmJob(X, xs, packed, ws, torch.empty((tokens, d), device=device)))
+        shapes.append((d, n))
+    desc = B.Descriptors(jobs)
+    for _ in range(3):
+        B.intlora_int_gemm_batched(desc, planes)
+    stream = torch.cuda.current_stream(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+    a.record(stream)
+    for _ in range(steps):
+        B.intlora_int_gemm_batched(desc, planes)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    ops = sum(2 * tokens * d * n * planes for d, n in shapes)
+    bf16, kind = bf16_peak_tflops()
+    top_s = ops / (ms / 1e3) / 1e12
+    del jobs, desc
+    torch.cuda.empty_cache()
+    return {"workload": f"DiT-3072 block GEMMs at {tokens} tokens, {planes} int8 digit plane(s), fp32 Y",
+            "ms": ms, "steps": steps, "tensor_Top_s": top_s, "peak_Top_s": 2.0 * bf16,
+            "frac_of_int8_peak": top_s / (2.0 * bf16),
+            "peak_source": f"2 x {kind} bf16 dense (nominal int8/bf16 ratio 2)",
+            "kernel": "int_gemm_kernel (tcgen05 kind::i8)"}
+
+
+def train_step_leg(device, tokens, steps):
+    """One IntLoRA training step of every SD-UNet linear at `tokens` tokens:
+    the MUL merge, the bf16 fake-quantized merged weight, the forward GEMM
+    Y = X W'^T and the backward (dX = dY W', dA and dB through the STE
+    without the weight gradient in HBM), each one batched call. CUDA-event
+    times per stage; bf16 tensor TFLOP/s of the two layer-sized GEMMs
+    (forward and dX, 4 tokens d n per layer) against the measured peak."""
+    import torch
+
+    from quantized_lora_merge_b200 import binding as B
+    from quantized_lora_merge_b200 import pipeline as P
+    from quantized_lora_merge_b200 import workloads as wl
+    layers = wl.CONFIGS["sd_unet"]()
+    states = []
+    for spec in layers:
+        t = wl.device_inputs(spec, device, with_grad=True, salt=0)
+        states.append(P.allocate(spec, t["W"], t["A"], t["B"], device, G=t["G"], A16=t["A16"],
+                                 B16=t["B16"]))
+    path = P.Path(states, device)
+    path.prepare()
+    g = torch.Generator(device=device)
+    g.manual_seed(17)
+    wq = [torch.empty(l.d, l.n, dtype=torch.bfloat16, device=device) for l in layers]
+    X = [torch.randn(tokens, l.n, generator=g, device=device).to(torch.bfloat16) for l in layers]
+    dY = [(torch.randn(tokens, l.d, generator=g, device=device) * 1e-3).to(torch.bfloat16)
+          for l in layers]
+    fq = B.Descriptors(B.FakeQuantJob(st.out, st.sbar, w) for st, w in zip(states, wq))
+    lin = B.Descriptors(B.LinearJob(x, w, torch.empty(tokens, l.d, dtype=torch.bfloat16,
+                                                      device=device))
+                        for l, x, w in zip(layers, X, wq))
+    bwd_jobs = [B.TrainBackwardJob(x, dy, w, st.A16, st.B16,
+                                   torch.empty(tokens, l.n, device=device), st.dA, st.dB)
+                for l, st, x, dy, w in zip(layers, states, X, dY, wq)]
+    bwd = B.Descriptors(bwd_jobs)
+    ws = torch.empty(max(256, B.intlora_train_backward_workspace_size(bwd_jobs)), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        path.merge()
+        if ev: ev[0].record(stream)
+        B.intlora_fakequant_bf16_batched(fq)
+        if ev: ev[1].record(stream)
+        B.intlora_linear_bf16_batched(lin)
+        if ev: ev[2].record(stream)
+        B.intlora_train_backward_batched(bwd, ws)
+        if ev: ev[3].record(stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for k in range(steps):
+        step(evs[k])
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    fwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+    gemm_flops = sum(4 * tokens * l.d * l.n for l in layers)
+    bf16, kind = bf16_peak_tflops()
+    tf = gemm_flops / ((fwd_ms + bwd_ms) / 1e3) / 1e12
+    del states, path, wq, X, dY, fq, lin, bwd, bwd_jobs, ws
+    torch.cuda.empty_cache()
+    return {"workload": f"SD-UNet 128 linears at {tokens} tokens: MUL merge + fake-quantization + "
+                        f"Y = X W'^T + backward (dX, dA, dB)",
+            "ms": ms, "steps": steps, "forward_gemm_ms": fwd_ms, "backward_ms": bwd_ms,
+            "gemm_TFLOP_s": tf, "peak_TFLOP_s": bf16, "frac_of_bf16_peak": tf / bf16,
+            "peak_source": f"{kind} bf16 dense",
+            "note": "TFLOP/s counts the forward and dX GEMMs (4 tokens d n per layer) over the "
+                    "forward-GEMM plus backward time; the backward also forms dA and dB"}
 
 
 def pinned_host(nbytes):

@@ -575,7 +575,7 @@ bool uses_tensor_t(const intlora_layer& l) {
 // its rank; unset or "auto": the fused kernel takes the layers it supports
 // from rank kMergeTcAutoMinRank up (below it the CUDA-core FMAs of the team
 // kernels cost less than the tensor-core hand-offs).
-constexpr int32_t kMergeTcAutoMinRank = 8;
+constexpr int32_t kMergeTcAutoMinRank = 16;   // measured: the team kernels win at r = 8, the fused kernel at r = 16
 int merge_kernel_mode() {
   const char* v = std::getenv("INTLORA_MERGE_KERNEL");
   if (v == nullptr) return 0;

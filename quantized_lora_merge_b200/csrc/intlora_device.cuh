@@ -110,6 +110,16 @@ __device__ __forceinline__ uint32_t aux_word(uint64_t e, uint32_t stream_id, uin
   return sel == 0 ? w.x : sel == 1 ? w.y : sel == 2 ? w.z : w.w;
 }
 
+// Base-2 logarithm on the special-function unit for a normal, positive
+// argument (flush-to-zero form: no denormal guard around the instruction;
+// the Laplace argument below is at least 2^-23, so it is never denormal and
+// the result is the one the guarded form gives).
+__device__ __forceinline__ float lg2_normal(float w) {
+  float r;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(w));
+  return r;
+}
+
 // c * R for the Laplace sample of word x, with c_ln2 = c * ln 2 (fp32).
 //
 // With k = x >> 9 (23 bits), u = (2k + 1) 2^-24 and v = u - 1/2, the inverse
@@ -125,7 +135,7 @@ __device__ __forceinline__ float laplace_log2(uint32_t x) {
   const float f = __uint_as_float(__funnelshift_r(x, 0x7Fu, 9));
   const float u2 = fmaf(2.0f, f, -1.99999988079071044921875f);   // -(2 - 2^-23)
   const float w = 1.0f - fabsf(u2 - 1.0f);
-  return __log2f(w);                                              // log2(1 - 2|v|) < 0
+  return lg2_normal(w);                                           // log2(1 - 2|v|) < 0
 }
 // +-c ln2: the factor that turns laplace_log2(x) into c * R.
 __device__ __forceinline__ float laplace_sign(uint32_t x, float c_ln2) {
@@ -203,7 +213,7 @@ __device__ __forceinline__ uint64_t laplace_log2_x2(uint32_t x, uint32_t y) {
   const uint64_t u2 = f2_fma(f2_pack(2.0f, 2.0f), f, f2_pack(-1.99999988079071044921875f,
                                                            -1.99999988079071044921875f));
   const uint64_t t = f2_add(u2, f2_pack(-1.0f, -1.0f));
-  return f2_pack(__log2f(1.0f - fabsf(f2_lo(t))), __log2f(1.0f - fabsf(f2_hi(t))));
+  return f2_pack(lg2_normal(1.0f - fabsf(f2_lo(t))), lg2_normal(1.0f - fabsf(f2_hi(t))));
 }
 
 // Round to nearest, ties to even, for |x| < 2^22, via the 1.5 * 2^23 bias:

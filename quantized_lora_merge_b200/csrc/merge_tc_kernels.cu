@@ -74,17 +74,27 @@ constexpr int kMaxParts = 4;
 constexpr uint32_t kABytes = kRows * 128;                // one tf32 part of one K atom of A (16 KB)
 constexpr uint32_t kBPart = kPartCols * 128;             // one tf32 part of a B^T stage (16 KB)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxMtcJobs = 40;
+constexpr int kMaxMtcJobs = 32;
+constexpr uint32_t kOutStage = 2048;                     // one 32 x 16 output block (int32), 1 KB aligned
 
 __device__ unsigned int g_mtc_timeouts;
 
+// Every wait of this kernel sleeps between checks: a waiting warp (the TMA
+// and MMA threads wait most of the time) takes no issue slots from the
+// quantizer warps that share its scheduler.
 __device__ __forceinline__ bool wait_m(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  return mbar_wait(bar, parity, abort_flag, &g_mtc_timeouts);
+  return mbar_wait_sleep(bar, parity, abort_flag, &g_mtc_timeouts);
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
 }
 
 struct alignas(64) MtcLayerDev {
   CUtensorMap a_hi, a_lo;        // {kp, d}, box {32, 128}, 128B swizzle
   CUtensorMap b_hi, b_lo;        // {kp, n}, box {32, 128}, 128B swizzle
+  CUtensorMap out_map;           // {n, d} of P or M, box {16, 32}, swizzle = row bytes (16 B: none)
   const uint8_t* codes;
   int64_t ld_w;
   const float* s;
@@ -113,6 +123,7 @@ struct MtcBatch {
   int32_t slice;                 // S: columns per CTA (multiple of 32, <= 512)
   int32_t atoms_max;
   int32_t stages;
+  int32_t obufs;                 // output staging blocks per quantizer warp (2, or 1 at rank > 64)
   int32_t num_groups;
   int64_t total_units;
 };
@@ -175,8 +186,9 @@ __device__ __forceinline__ uint4 load_codes16(const uint8_t* p) {
 template <int WBITS>
 __device__ __forceinline__ int32_t code_at(const uint4& c, int k) {
   if (WBITS == 8) {
+    // byte k & 3 of the word, zero-extended (one byte permute)
     const uint32_t w = k < 4 ? c.x : k < 8 ? c.y : k < 12 ? c.z : c.w;
-    return static_cast<int32_t>((w >> (8 * (k & 3))) & 0xFFu);
+    return static_cast<int32_t>(__byte_perm(w, 0u, 0x4440u | static_cast<uint32_t>(k & 3)));
   }
   const uint32_t w = k < 8 ? c.x : c.y;
   return static_cast<int32_t>((w >> (4 * (k & 7))) & 0xFu);
@@ -207,7 +219,8 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
   const int G = b.group;
   uint8_t* sA = base;                                                   // [atom][hi, lo]
   uint8_t* sB = sA + static_cast<size_t>(b.atoms_max) * 2 * kABytes;  // [stage][hi, lo]
-  uint2* ext = reinterpret_cast<uint2*>(sB + static_cast<size_t>(NS) * 2 * kBPart);   // [kMembers][128]
+  uint8_t* ostage = sB + static_cast<size_t>(NS) * 2 * kBPart;           // [quantizer warp][2] output blocks
+  uint2* ext = reinterpret_cast<uint2*>(ostage + static_cast<size_t>(kQuantWarps) * b.obufs * kOutStage);   // [kMembers][128]
   float* rcp_tab = reinterpret_cast<float*>(ext + kMembers * kRows);   // 1/D, D in [-255, 255]
   uint64_t* bars = reinterpret_cast<uint64_t*>(rcp_tab + 512);
   uint64_t* a_full = bars;
@@ -384,6 +397,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
     uint32_t* my_flags = b.flags + static_cast<int64_t>(grp) * G;
     uint2* my_slots = b.slots + static_cast<int64_t>(grp) * 2 * G * kRows;
     int cur = -1, ucount = 0;
+    uint32_t nstore = 0;                           // output blocks this warp has sent
     float c_ln2 = 0.0f;
     PhiloxSmall ph{};
     for (int64_t u = grp; u < b.total_units && !abort_flag; u += b.num_groups, ++ucount) {
@@ -404,7 +418,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       const int cols = col0 < n ? static_cast<int>(min64(S, n - col0)) : 0;   // multiple of 32
       const float sv = __ldg(L.s + rrow);
       const int32_t zv = clamp_i(__ldg(L.z + rrow), 0, (1 << WBITS) - 1);
-      const float* rb = rcp_tab + (255 - zv);
+      const uint32_t rb = smem_u32(rcp_tab) + 4u * static_cast<uint32_t>(255 - zv);   // 1/(code - z) at rb + 4 code
       const uint8_t* crow = L.codes + rrow * L.ld_w;
       const uint32_t ctr_row = static_cast<uint32_t>(rrow * (n >> 2));
       const uint64_t s2 = f2_pack(sv, sv);
@@ -467,8 +481,8 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
               const int k0 = 4 * q + 2 * h;
               const uint64_t lg = laplace_log2_x2(wa, wb);
               const uint64_t cs = f2_pack(laplace_sign(wa, c_ln2), laplace_sign(wb, c_ln2));
-              const float r0 = rb[code_at<WBITS>(cw, k0)];
-              const float r1 = rb[code_at<WBITS>(cw, k0 + 1)];
+              const float r0 = ld_shared_f32(rb + 4u * static_cast<uint32_t>(code_at<WBITS>(cw, k0)));
+              const float r1 = ld_shared_f32(rb + 4u * static_cast<uint32_t>(code_at<WBITS>(cw, k0 + 1)));
               const uint64_t vp = f2_fma(f2_fma(lg, cs, f2_pack(v[k0], v[k0 + 1])), f2_pack(r0, r1), s2);
               v[k0] = f2_lo(vp);
               v[k0 + 1] = f2_hi(vp);
@@ -518,6 +532,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
         if (!seen) {
           const uint64_t t0 = global_ns();
           for (uint32_t it = 1; !seen; ++it) {
+            __nanosleep(64);                     // poll the flag without flooding L2
             seen = ld_acquire_gpu(f) >= tag;
             if (!seen && (it & 63u) == 0u) {
               if (abort_flag) break;
@@ -555,7 +570,6 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       }
 
       // ---- phase B: quantize the parked U and store the row's merged weights
-      uint8_t* orow = static_cast<uint8_t*>(L.out) + rrow * n * OUTB;
       const int32_t bias_lo = kRoundBiasBits - zero;
       const int32_t bias_hi = bias_lo + qmax;
       uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
@@ -591,27 +605,59 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
               code8[k] = static_cast<uint32_t>(cb - bias_lo);
             }
           }
-          if (valid) {
-            uint8_t* op = orow + j * OUTB;
-            if (OUTB == 4) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                reinterpret_cast<int4*>(op)[q] = make_int4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
-            } else if (OUTB == 2) {
-              uint32_t wv[8];
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                wv[q] = (static_cast<uint32_t>(res[2 * q]) & 0xFFFFu) | (static_cast<uint32_t>(res[2 * q + 1]) << 16);
-              reinterpret_cast<uint4*>(op)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-              reinterpret_cast<uint4*>(op)[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-            } else {
+          if (OUTB == 1) {
+            // 16 bytes per row and group: one direct store per lane
+            if (valid) {
               uint32_t wv[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q)
                 wv[q] = (static_cast<uint32_t>(res[4 * q]) & 0xFFu) | ((static_cast<uint32_t>(res[4 * q + 1]) & 0xFFu) << 8) |
                         ((static_cast<uint32_t>(res[4 * q + 2]) & 0xFFu) << 16) | (static_cast<uint32_t>(res[4 * q + 3]) << 24);
-              reinterpret_cast<uint4*>(op)[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+              *reinterpret_cast<uint4*>(static_cast<uint8_t*>(L.out) + row * n + j) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
+          } else {
+            // the warp's 32 rows x 16 columns go out as one TMA store through a
+            // swizzled staging block (double-buffered when shared memory
+            // allows), one whole 32- or 64-byte segment per row
+            const bool two = b.obufs == 2;
+            uint8_t* stage = ostage + static_cast<size_t>(warp - 4) * b.obufs * kOutStage + (two ? (nstore & 1u) : 0u) * kOutStage;
+            if (lane == 0) {                         // this block's last store has read it
+              if (two) bulk_wait_read<1>();
+              else bulk_wait_read<0>();
+            }
+            __syncwarp();
+            const uint32_t rowp = smem_u32(stage) + static_cast<uint32_t>(lane) * (16u * OUTB);
+            if (OUTB == 4) {
+              const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);     // 64-byte swizzle
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                             ::"r"(rowp + 16u * (static_cast<uint32_t>(q) ^ sw)), "r"(res[4 * q]), "r"(res[4 * q + 1]),
+                               "r"(res[4 * q + 2]), "r"(res[4 * q + 3])
+                             : "memory");
+            } else {
+              uint32_t wv[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                wv[q] = (static_cast<uint32_t>(res[2 * q]) & 0xFFFFu) | (static_cast<uint32_t>(res[2 * q + 1]) << 16);
+              const uint32_t sw = static_cast<uint32_t>((lane >> 2) & 1);     // 32-byte swizzle
+#pragma unroll
+              for (int q = 0; q < 2; ++q)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                             ::"r"(rowp + 16u * (static_cast<uint32_t>(q) ^ sw)), "r"(wv[4 * q]), "r"(wv[4 * q + 1]),
+                               "r"(wv[4 * q + 2]), "r"(wv[4 * q + 3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              // rows past d are clipped by the tensor map
+              tma_store_2d(&L.out_map, stage, static_cast<int32_t>(j), static_cast<int32_t>(x.i0 + quarter * 32));
+              bulk_commit();
+            }
+            ++nstore;
+          }
+          if (valid) {
             if (L.code_out != nullptr) {
               uint32_t cv[4];
 #pragma unroll
@@ -626,6 +672,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
         mbar_arrive(&t_empty[p]);
       }
     }
+    if (lane == 0) bulk_wait<0>();                 // this warp's output stores are done
   }
 
   tc_fence_before();
@@ -638,9 +685,12 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
 
 // Dynamic shared memory of a launch. At least 120 KB, so that two CTAs never
 // share an SM: each allocates all 512 tensor-memory columns.
+int mtc_obufs(int atoms_max) { return atoms_max > 2 ? 1 : 2; }
+
 size_t mtc_smem_bytes(int atoms_max, int stages) {
   const size_t need = 1024 + static_cast<size_t>(atoms_max) * 2 * kABytes + static_cast<size_t>(stages) * 2 * kBPart +
-                      kMembers * kRows * 8 + 512 * 4 + (6 + 2 * kMaxParts + 2 * stages) * 8;
+                      static_cast<size_t>(kQuantWarps) * mtc_obufs(atoms_max) * kOutStage + kMembers * kRows * 8 +
+                      512 * 4 + (6 + 2 * kMaxParts + 2 * stages) * 8;
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
 
@@ -764,7 +814,12 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
                       tc::encode_2d(&t.a_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.a_lo, j.d, kp, 32, kRows) &&
                       tc::encode_2d(&t.b_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.b_hi, j.n, kp, 32, kPartCols) &&
                       tc::encode_2d(&t.b_lo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, j.b_lo, j.n, kp, 32, kPartCols);
-      if (!ok) return cudaErrorInvalidValue;
+      const CUtensorMapDataType odt = out_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                      : out_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+      const CUtensorMapSwizzle osw = out_bytes == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                     : out_bytes == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
+      if (!ok || !tc::encode_2d_swz(&t.out_map, odt, out_bytes, j.out, j.d, j.n, 16, 32, osw))
+        return cudaErrorInvalidValue;
       t.codes = j.codes;
       t.ld_w = j.ld_w;
       t.s = j.s;
@@ -792,6 +847,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     b.slice = plan.slice;
     b.atoms_max = atoms_max;
     b.stages = mtc_stages(atoms_max);
+    b.obufs = mtc_obufs(atoms_max);
     if (b.stages == 0) return cudaErrorInvalidValue;
     b.total_units = units;
     const size_t smem = mtc_smem_bytes(atoms_max, b.stages);

@@ -40,6 +40,19 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread sleeps (issues nothing) until
+// the phase completes or about hint_ns pass.
+__device__ __forceinline__ bool mbar_try_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -66,6 +79,23 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, vo
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* timeouts) {
   return mbar_wait_for(bar, parity, abort_flag, timeouts, kWaitNs);
+}
+// The same bounded wait for threads that can afford to sleep between
+// checks (a waiting warp then takes no issue slots from working warps).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                unsigned int* timeouts) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_hint(bar, parity, 2000u)) return true;
+    if ((it & 15u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitNs) break;
+    }
+  }
+  atomicAdd(timeouts, 1u);
+  *abort_flag = 1;
+  return false;
 }
 // Drain helpers for a CTA that gave up. A TMA copy completes on the mbarrier
 // phase it was armed on: wait (bounded) for the last phase armed on `bar`

@@ -116,15 +116,16 @@ def prepare_bytes(l):
     return l.numel * (4 + 4 + code) + l.d * 8
 
 
-def merge_ops(l):
+def merge_ops(l, fused=False):
     """Algorithmic lane operations of the merge kernel, per element x numel:
     Philox4x32-10 share (10 rounds x 4 ops / 4 words = 10), Laplace inverse CDF
-    (6: shift, int->float, fma, log2, scale, sign), T = A.B (r FMAs), U (4: add,
-    fma, reciprocal multiply, select), row extrema (2), quantize + product
-    (MUL 5.5: fma, round, clamp x2, sub, half an IMAD; SHIFT 8: abs, exponent,
+    (6: shift, int->float, fma, log2, scale, sign), T = A.B (r FMAs on the
+    CUDA cores; none where the tensor cores form it), U (4: add, fma,
+    reciprocal multiply, select), row extrema (2), quantize + product (MUL
+    5.5: fma, round, clamp x2, sub, half an IMAD; SHIFT 8: abs, exponent,
     mantissa compare, clamps, shift, sign)."""
     quant = 5.5 if l.variant == "mul" else 8.0
-    return l.numel * (10 + 6 + l.r + 4 + 2 + quant)
+    return l.numel * (10 + 6 + (0 if fused else l.r) + 4 + 2 + quant)
 
 
 ALU_LANES_PER_SM_CLK = 128       # FP32/INT32 lanes per SM per clock on sm_100
@@ -439,8 +440,8 @@ def main():
     # is reported beside it.
     sm_mhz = clk.get("sm_mhz") or 1965.0
     alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
-    alu_achieved = sum(merge_ops(l) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
     fused = (not args.dist) and all(l.r >= 16 and l.n % 32 == 0 for l in layers)
+    alu_achieved = sum(merge_ops(l, fused) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
     kernel_name = ("merge_tc_kernel (fused tensor-core merge)" if fused else
                    "team / row-tile merge kernels" if not args.dist else
                    "merge row-tile kernel (general auxiliary law)")
@@ -468,7 +469,7 @@ def main():
                      "alu_achieved_Top_s": alu_achieved, "alu_peak_Top_s": alu_peak,
                      "alu_frac_modelled": alu_achieved / alu_peak,
                      "alu_peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
-                     "ops_per_element_modelled": merge_ops(layers[0]) / layers[0].numel},
+                     "ops_per_element_modelled": merge_ops(layers[0], fused) / layers[0].numel},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": launches,

@@ -35,11 +35,12 @@
 // MMA issuer part by part as the quantizers finish reading U, so the next
 // unit's products overlap the current unit's last parts.
 //
-// Roles (12 warps): warp 0 issues TMA loads (the unit's A tile once, B^T
+// Roles (16 warps): warp 0 issues TMA loads (the unit's A tile once, B^T
 // tiles through a ring of stages), warp 1 allocates tensor memory and issues
-// the MMAs (one thread), warps 4-11 quantize: warps 4 + q and 8 + q serve
-// lane quarter q (rows 32 q .. 32 q + 31) and take alternate 16-column
-// groups of every part. Every wait is bounded (2 s); a wait that gives up is
+// the MMAs (one thread), warps 4-15 quantize: warps 4 + q, 8 + q and 12 + q
+// serve lane quarter q (rows 32 q .. 32 q + 31) and take every third
+// 16-column group (three warps per scheduler keep the issue slots busier
+// than two; 128 registers a thread suffice without spills). Every wait is bounded (2 s); a wait that gives up is
 // counted, the CTA drains its copies and products and returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -62,9 +63,10 @@ using namespace tc;
 
 constexpr double kLn2 = 0.69314718055994530942;
 #ifndef INTLORA_MTC_QUANT_WARPS
-#define INTLORA_MTC_QUANT_WARPS 8
+#define INTLORA_MTC_QUANT_WARPS 12
 #endif
 constexpr int kQuantWarps = INTLORA_MTC_QUANT_WARPS;   // a multiple of 4: kMembers warps per lane quarter
+static_assert(kQuantWarps % 4 == 0 && kQuantWarps >= 4 && kQuantWarps <= 16, "quantizer warps: 4, 8, 12 or 16");
 constexpr int kMembers = kQuantWarps / 4;
 constexpr int kQuantThreads = 32 * kQuantWarps;
 constexpr int kMtcThreads = 32 * (4 + kQuantWarps);
@@ -572,18 +574,34 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       // ---- phase B: quantize the parked U and store the row's merged weights
       const int32_t bias_lo = kRoundBiasBits - zero;
       const int32_t bias_hi = bias_lo + qmax;
-      uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
-      if (ng > 0) cw0 = load_codes16<WBITS>(crow + (((col0 + 16 * member) * WBITS) >> 3));
-      if (ng > 1) cw1 = load_codes16<WBITS>(crow + (((col0 + kStep + 16 * member) * WBITS) >> 3));
-      int g = 0;
-      for (int p = 0; p < NP; ++p) {
+      // Each part in turn: this thread's groups of the part (16-column groups
+      // 16 member + kStep i), their codes loaded one part ahead; the part of
+      // tensor memory goes back to the MMA issuer once they have been read.
+      constexpr int kGpp = (static_cast<int>(kPartCols) / 16 + kMembers - 1) / kMembers;   // groups per part, at most
+      uint4 cwn[kGpp];
+      auto load_part = [&](int p) {
         const int pc = min(static_cast<int>(kPartCols), cols - p * static_cast<int>(kPartCols));
-        for (int c = 16 * member; c < pc; c += kStep, ++g) {
+#pragma unroll
+        for (int i = 0; i < kGpp; ++i) {
+          const int c = 16 * member + kStep * i;
+          cwn[i] = c < pc ? load_codes16<WBITS>(crow + (((col0 + p * static_cast<int>(kPartCols) + c) * WBITS) >> 3))
+                          : make_uint4(0u, 0u, 0u, 0u);
+        }
+      };
+      if (NP > 0) load_part(0);
+      for (int p = 0; p < NP; ++p) {
+        uint4 cwc[kGpp];
+#pragma unroll
+        for (int i = 0; i < kGpp; ++i) cwc[i] = cwn[i];
+        if (p + 1 < NP) load_part(p + 1);
+        const int pc = min(static_cast<int>(kPartCols), cols - p * static_cast<int>(kPartCols));
+#pragma unroll
+        for (int i = 0; i < kGpp; ++i) {
+          const int c = 16 * member + kStep * i;
+          if (c >= pc) break;
           const int cc = p * static_cast<int>(kPartCols) + c;
           const int64_t j = col0 + cc;
-          const uint4 cw = cw0;
-          cw0 = cw1;
-          if (g + 2 < ng) cw1 = load_codes16<WBITS>(crow + (((j + 2 * kStep) * WBITS) >> 3));
+          const uint4 cw = cwc[i];
           float v[16];
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();
@@ -667,7 +685,6 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
             }
           }
         }
-        // this part of tensor memory is free for the next unit's products
         tc_fence_before();
         mbar_arrive(&t_empty[p]);
       }

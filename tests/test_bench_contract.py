@@ -40,3 +40,5 @@ def test_algorithmic_counts(cfg):
         assert bench.ste_bytes(l) == 2 * l.numel + 6 * l.r * (l.d + l.n)
         assert bench.merge_bytes(l) > l.numel * code
         assert bench.merge_ops(l) == l.numel * (22 + l.r + (5.5 if l.variant == "mul" else 8.0))
+        # the tensor cores form A B in the fused kernel: no rank term on the lanes
+        assert bench.merge_ops(l, True) == l.numel * (22 + (5.5 if l.variant == "mul" else 8.0))

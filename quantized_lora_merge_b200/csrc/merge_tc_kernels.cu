@@ -16,9 +16,12 @@
 // columns per tcgen05.ld: four Philox blocks of that row), forms U, keeps the
 // row's running extrema in registers and writes U back in place
 // (tcgen05.st). The extrema of the G CTAs are combined through a small
-// exchange area in the caller's workspace (each CTA publishes its 128 row
-// extrema and a release flag; the group's CTAs acquire all G flags), then the
-// same thread reads U back, quantizes it and stores its row's merged weights.
+// exchange area in the caller's workspace: each CTA stores its 128 row
+// extrema as tagged 64-bit words (tag = the unit's number in the launch), and
+// the quantizer threads of a row read the other CTAs' words, several in
+// flight at once, until every tag matches; no fence, flag or extra barrier
+// hop lies on that path. Then the same thread reads U back, quantizes it and
+// stores its row's merged weights.
 // Nothing else of the merge touches global memory.
 //
 // The launch is cooperative (every CTA resident, one per SM), so a CTA may
@@ -78,6 +81,10 @@ constexpr uint32_t kBPart = kPartCols * 128;             // one tf32 part of a B
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxMtcJobs = 32;
 constexpr uint32_t kOutStage = 2048;                     // one 32 x 16 output block (int32), 1 KB aligned
+#ifndef INTLORA_MTC_GATHER
+#define INTLORA_MTC_GATHER 2
+#endif
+constexpr int kGather = INTLORA_MTC_GATHER;              // exchange slots in flight per thread
 
 __device__ unsigned int g_mtc_timeouts;
 
@@ -116,8 +123,7 @@ struct alignas(64) MtcLayerDev {
 };
 struct MtcBatch {
   MtcLayerDev layer[kMaxMtcJobs];
-  uint32_t* flags;               // [groups][G] unit counters (zeroed before the launch)
-  uint2* slots;                  // [groups][2][G][128] row extrema
+  ulonglong2* slots;             // [groups][2][G][128] tagged row extrema (zeroed before the launch)
   int32_t count;
   uint32_t key0, key1;
   int32_t bits;                  // MUL: u_bits; SHIFT: shift_bits
@@ -159,18 +165,16 @@ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// Exchange area accesses: L2-coherent (another SM wrote them).
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Exchange area accesses, L2-coherent (another SM wrote them). A slot is two
+// 64-bit words, each (tag << 32) | value: an aligned 64-bit access is single-
+// copy atomic, so a word whose tag matches carries its own value and no fence
+// or flag is needed to publish it.
+__device__ __forceinline__ void st_slot(ulonglong2* p, uint64_t w0, uint64_t w1) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
 }
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint2* p) {
-  uint2 v;
-  asm volatile("ld.relaxed.gpu.global.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
+__device__ __forceinline__ ulonglong2 ld_slot(const ulonglong2* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
@@ -223,13 +227,12 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
   uint8_t* sB = sA + static_cast<size_t>(b.atoms_max) * 2 * kABytes;  // [stage][hi, lo]
   uint8_t* ostage = sB + static_cast<size_t>(NS) * 2 * kBPart;           // [quantizer warp][2] output blocks
   uint2* ext = reinterpret_cast<uint2*>(ostage + static_cast<size_t>(kQuantWarps) * b.obufs * kOutStage);   // [kMembers][128]
-  float* rcp_tab = reinterpret_cast<float*>(ext + kMembers * kRows);   // 1/D, D in [-255, 255]
+  float* rcp_tab = reinterpret_cast<float*>(ext + 2 * kMembers * kRows);   // 1/D, D in [-255, 255]; ext, then gat
   uint64_t* bars = reinterpret_cast<uint64_t*>(rcp_tab + 512);
   uint64_t* a_full = bars;
   uint64_t* a_empty = bars + 1;
   uint64_t* ext_bar = bars + 2;            // the quantizers' partial extrema are in ext
-  uint64_t* sent_bar = bars + 3;           // the senders' slot stores are done
-  uint64_t* got_bar = bars + 4;            // every flag of the group is in
+  uint64_t* got_bar = bars + 4;            // every member's share of the group's extrema is in gat
   uint64_t* drain = bars + 5;
   uint64_t* t_full = bars + 6;             // [kMaxParts]
   uint64_t* t_empty = t_full + kMaxParts;  // [kMaxParts]
@@ -244,8 +247,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
     mbar_init(a_full, 1);
     mbar_init(a_empty, 1);
     mbar_init(ext_bar, kQuantThreads);
-    mbar_init(sent_bar, kRows);
-    mbar_init(got_bar, static_cast<uint32_t>(G));
+    mbar_init(got_bar, kQuantThreads);
     mbar_init(drain, 1);
     for (int p = 0; p < kMaxParts; ++p) {
       mbar_init(&t_full[p], 1);
@@ -396,8 +398,8 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int qmax = (1 << b.bits) - 1;
     const bool sender = member == 0;
-    uint32_t* my_flags = b.flags + static_cast<int64_t>(grp) * G;
-    uint2* my_slots = b.slots + static_cast<int64_t>(grp) * 2 * G * kRows;
+    ulonglong2* my_slots = b.slots + static_cast<int64_t>(grp) * 2 * G * kRows;
+    uint2* gat = ext + kMembers * kRows;           // [kMembers][128] partial group extrema
     int cur = -1, ucount = 0;
     uint32_t nstore = 0;                           // output blocks this warp has sent
     float c_ln2 = 0.0f;
@@ -509,51 +511,61 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
       ext[member * kRows + row_u] = make_uint2(ord_abs(hi), ord_abs(lo));
       mbar_arrive(ext_bar);
       if (!wait_m(ext_bar, up, &abort_flag) || !ok) break;
-      const uint32_t tag = static_cast<uint32_t>(ucount) + 1u;
-      if (sender) {
-        uint2 e = ext[row_u];
+      // this CTA's extrema of the row (every member reads them from ext)
+      uint2 own = ext[row_u];
 #pragma unroll
-        for (int m = 1; m < kMembers; ++m) {
-          const uint2 f = ext[m * kRows + row_u];
-          e = make_uint2(max(e.x, f.x), max(e.y, f.y));
-        }
-        my_slots[(static_cast<int64_t>(up) * G + rank) * kRows + row_u] = e;
-        __threadfence();
-        mbar_arrive(sent_bar);
-        if (row_u == 0) {
-          // publish once every sender's store is in (CTA acquire, GPU release)
-          if (!wait_m(sent_bar, up, &abort_flag)) break;
-          st_release_gpu(my_flags + rank, tag);
-        }
+      for (int m = 1; m < kMembers; ++m) {
+        const uint2 f = ext[m * kRows + row_u];
+        own = make_uint2(max(own.x, f.x), max(own.y, f.y));
       }
-      // G threads wait for the group's flags, then release the others
-      const int qt = threadIdx.x - 128;
-      if (qt < G) {
-        const uint32_t* f = my_flags + qt;
-        bool seen = ld_acquire_gpu(f) >= tag;
-        if (!seen) {
-          const uint64_t t0 = global_ns();
-          for (uint32_t it = 1; !seen; ++it) {
-            __nanosleep(64);                     // poll the flag without flooding L2
-            seen = ld_acquire_gpu(f) >= tag;
-            if (!seen && (it & 63u) == 0u) {
-              if (abort_flag) break;
-              if (global_ns() - t0 > kWaitNs) {
-                atomicAdd(&g_mtc_timeouts, 1u);
-                abort_flag = 1;
-                break;
+      const uint32_t want = static_cast<uint32_t>(ucount) + 1u;      // this unit's tag
+      if (sender)
+        st_slot(my_slots + (static_cast<int64_t>(up) * G + rank) * kRows + row_u,
+                (static_cast<uint64_t>(want) << 32) | own.x, (static_cast<uint64_t>(want) << 32) | own.y);
+      // member m gathers the other CTAs k = m, m + kMembers, ... of the group,
+      // kGather slots in flight at a time; a slot is read again (sleeping
+      // between reads, bounded) until both words carry this unit's tag
+      uint2 part = own;
+      {
+        const ulonglong2* sp = my_slots + static_cast<int64_t>(up) * G * kRows + row_u;
+        uint64_t t0 = 0;
+        for (int k0 = member; k0 < G && !abort_flag; k0 += kGather * kMembers) {
+          ulonglong2 e[kGather];
+#pragma unroll
+          for (int i = 0; i < kGather; ++i) {
+            const int k = k0 + i * kMembers;
+            if (k < G && k != rank) e[i] = ld_slot(sp + static_cast<int64_t>(k) * kRows);
+          }
+#pragma unroll
+          for (int i = 0; i < kGather; ++i) {
+            const int k = k0 + i * kMembers;
+            if (k >= G || k == rank) continue;
+            for (uint32_t it = 1; static_cast<uint32_t>(e[i].x >> 32) != want || static_cast<uint32_t>(e[i].y >> 32) != want; ++it) {
+              __nanosleep(64);
+              e[i] = ld_slot(sp + static_cast<int64_t>(k) * kRows);
+              if ((it & 63u) == 0u) {
+                if (t0 == 0) {
+                  t0 = global_ns();
+                } else if (global_ns() - t0 > kWaitNs) {
+                  atomicAdd(&g_mtc_timeouts, 1u);
+                  abort_flag = 1;
+                }
+                if (abort_flag) break;
               }
             }
+            part = make_uint2(max(part.x, static_cast<uint32_t>(e[i].x)), max(part.y, static_cast<uint32_t>(e[i].y)));
           }
         }
-        if (seen) mbar_arrive(got_bar);
       }
-      if (!wait_m(got_bar, up, &abort_flag)) break;
-      uint32_t top_b = 0u, negb_b = 0u;
-      for (int k = 0; k < G; ++k) {
-        const uint2 e = ld_relaxed_gpu_v2(my_slots + (static_cast<int64_t>(up) * G + k) * kRows + row_u);
-        top_b = max(top_b, e.x);
-        negb_b = max(negb_b, e.y);
+      gat[member * kRows + row_u] = part;
+      mbar_arrive(got_bar);
+      if (!wait_m(got_bar, up, &abort_flag) || abort_flag) break;
+      uint32_t top_b = part.x, negb_b = part.y;
+#pragma unroll
+      for (int m = 0; m < kMembers; ++m) {
+        const uint2 f = gat[m * kRows + row_u];
+        top_b = max(top_b, f.x);
+        negb_b = max(negb_b, f.y);
       }
       const float top = __uint_as_float(top_b), neg_bottom = __uint_as_float(negb_b);
       float scale = 1.0f;
@@ -706,7 +718,7 @@ int mtc_obufs(int atoms_max) { return atoms_max > 2 ? 1 : 2; }
 
 size_t mtc_smem_bytes(int atoms_max, int stages) {
   const size_t need = 1024 + static_cast<size_t>(atoms_max) * 2 * kABytes + static_cast<size_t>(stages) * 2 * kBPart +
-                      static_cast<size_t>(kQuantWarps) * mtc_obufs(atoms_max) * kOutStage + kMembers * kRows * 8 +
+                      static_cast<size_t>(kQuantWarps) * mtc_obufs(atoms_max) * kOutStage + 2 * kMembers * kRows * 8 +
                       512 * 4 + (6 + 2 * kMaxParts + 2 * stages) * 8;
   return need < 120 * 1024 ? 120 * 1024 : need;
 }
@@ -808,9 +820,8 @@ bool merge_tc_plan(int64_t n, int32_t r, MtcPlan* plan) {
 }
 
 size_t merge_tc_exchange_bytes() {
-  // flags, then the double-buffered row extrema, of up to kMergeTcMaxCtas CTAs
-  return ((static_cast<size_t>(kMergeTcMaxCtas) * 4 + 255) & ~size_t{255}) +
-         static_cast<size_t>(kMergeTcMaxCtas) * 2 * kRows * 8;
+  // the double-buffered tagged row extrema of up to kMergeTcMaxCtas CTAs
+  return static_cast<size_t>(kMergeTcMaxCtas) * 2 * kRows * sizeof(ulonglong2);
 }
 
 cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bits, int out_bytes, int bits,
@@ -875,11 +886,9 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     const int64_t fit = std::min<int64_t>(num_sms(), kMergeTcMaxCtas) / G;
     if (fit < 1) return cudaErrorInvalidConfiguration;
     b.num_groups = static_cast<int32_t>(units < fit ? units : fit);
-    const int64_t ngr = kMergeTcMaxCtas / G;
-    b.flags = reinterpret_cast<uint32_t*>(exchange);
-    b.slots = reinterpret_cast<uint2*>(static_cast<char*>(exchange) +
-                                       ((static_cast<size_t>(ngr) * G * 4 + 255) & ~size_t{255}));
-    cudaError_t e = cudaMemsetAsync(b.flags, 0, static_cast<size_t>(b.num_groups) * G * 4, s);
+    // tags restart at 1 with every launch: the slots this launch uses start zeroed
+    b.slots = static_cast<ulonglong2*>(exchange);
+    cudaError_t e = cudaMemsetAsync(b.slots, 0, static_cast<size_t>(b.num_groups) * G * 2 * kRows * sizeof(ulonglong2), s);
     if (e != cudaSuccess) return e;
     q.op = 0;
     q.batch = &b;

@@ -961,8 +961,11 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
       ok = ste_tc_supported(s);
     }
     if (ok) {
-      // ranks >= 64: two passes, each product reduced inside a CTA; the rest
-      // one pass with reductions into zeroed outputs
+      // ranks >= 64: two passes over L2-sized regions; the rest one pass.
+      // Both reduce into outputs zeroed first.
+      b.count = count;
+      cudaError_t e = launch_ste_zero(b, st);
+      if (e != cudaSuccess) return cuda_fail(e, "STE zero launch");
       SteBatch one;
       std::memset(&one, 0, sizeof one);
       std::vector<SteJob> wide;
@@ -971,12 +974,10 @@ intlora_status ste_chunk(const intlora_ste_job* jobs, int32_t count, cudaStream_
         else one.job[one.count++] = b.job[k];
       }
       if (!wide.empty()) {
-        cudaError_t e = launch_ste_wide(wide.data(), static_cast<int>(wide.size()), st);
+        e = launch_ste_wide(wide.data(), static_cast<int>(wide.size()), st);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE (two-pass) launch");
       }
       if (one.count > 0) {
-        cudaError_t e = launch_ste_zero(one, st);
-        if (e != cudaSuccess) return cuda_fail(e, "STE zero launch");
         e = launch_ste_tc(one.job, one.count, st);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core STE kernel launch");
       }

@@ -5,17 +5,21 @@
 // The one-pass kernel (ste_tc_kernels.cu) reduces every tile's 128 x r block
 // of dB^T into global memory with fp32 reductions: at r >= 64 that is one
 // reduction per 2 elements of G or more, and the reductions, not HBM, set its
-// pace. Here the two products take separate passes over G instead, each with
-// its reduction dimension inside one CTA, so every output element is written
-// exactly once (no atomics, no zeroing):
-//   pass 1  unit = 128 rows of one layer:  D1 += G_tile B_tile^T over all
-//           column tiles (both operands K-major), then D1 -> dA rows;
-//   pass 2  unit = 128 columns of one layer: D2 += G_tile^T A_tile over all
+// pace. Here the two products take separate passes, each accumulating over
+// many tiles inside one CTA before it reduces into the (zeroed) outputs. A
+// layer is cut into regions of up to 16 row blocks x 16 column tiles (8 MB of
+// G); a region's units are
+//   pass 1  one per row block: D1 += G_tile B_tile^T over the region's
+//           column tiles (both operands K-major), then D1 -> dA rows (+=);
+//   pass 2  one per column tile: D2 += G_tile^T A_tile over the region's
 //           row blocks (G tile MN-major, the A tile loaded by TMA straight
-//           from the row-major A as an MN-major operand), then D2 -> dB.
-// Both passes share one launch (their units are one index space). G is read
-// twice; at r >= 64 the arithmetic intensity of the single pass (2r flop/B)
-// is near or above the tensor/HBM ridge anyway.
+//           from the row-major A as an MN-major operand), then D2 -> dB (+=).
+// Units are numbered region by region and the persistent CTAs walk them in
+// that order, so both passes over a region run close together in time and
+// the second read of its G tiles is served by L2: HBM sees G about once.
+// Every unit is at most 16 tile steps (balanced across the CTAs), and the
+// reductions add 128 r fp32 per unit against 16 tiles of G (an eighth of
+// G's bytes at r = 128).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -45,19 +49,24 @@ __device__ __forceinline__ bool wait_w(uint64_t* bar, uint32_t parity, volatile 
   return mbar_wait(bar, parity, abort_flag, &g_sw_timeouts);
 }
 
+constexpr int kRegionBlocks = 16;                // row blocks per region
+constexpr int kRegionTiles = 16;                 // column tiles per region
+
 struct alignas(64) WJob {
   CUtensorMap g_map;          // G: dims {n, d}, box {64, 128}
   CUtensorMap b_map;          // B: dims {n, r}, box {64, RP}
   CUtensorMap a_map;          // A: dims {r, d}, box {64, 128}
-  float* dA;
-  float* dB;
+  float* dA;                  // zeroed before the launch
+  float* dB;                  // zeroed before the launch
   int64_t d, n;
   int32_t r;
   int32_t row_blocks;
   int32_t col_tiles;
+  int32_t bands;              // region rows: ceil(row_blocks / kRegionBlocks)
+  int32_t chunks;             // region columns: ceil(col_tiles / kRegionTiles)
   int32_t pad;
-  int64_t unit1_begin;        // pass-1 units of this job
-  int64_t unit2_begin;        // pass-2 units of this job
+  int64_t band_units;         // units of a full band: chunks kRegionBlocks + col_tiles
+  int64_t unit_begin;         // first unit of this job
 };
 struct WBatch {
   WJob job[kMaxWJobs];
@@ -65,7 +74,6 @@ struct WBatch {
   int32_t rp;                 // r rounded up to 64 (MMA N)
   int32_t stages;
   int32_t pad;
-  int64_t units1;             // pass-1 units of the batch; pass-2 units follow
   int64_t total_units;
 };
 
@@ -73,22 +81,37 @@ struct WUnit {
   int job;
   int pass;                   // 1 or 2
   int64_t fixed;              // pass 1: row block; pass 2: column tile
+  int64_t start;              // pass 1: first column tile; pass 2: first row block
   int steps;                  // pass 1: column tiles; pass 2: row blocks
 };
+__device__ __forceinline__ int64_t wmin(int64_t a, int64_t b) { return a < b ? a : b; }
+// Unit u: its job, band (region row), chunk (region column), then the
+// region's pass-1 units (one per row block) followed by its pass-2 units
+// (one per column tile).
 __device__ __forceinline__ WUnit w_unit(const WBatch& b, int64_t u) {
-  WUnit x;
-  x.pass = u < b.units1 ? 1 : 2;
   int j = 0;
-  if (x.pass == 1) {
-    while (j + 1 < b.count && b.job[j + 1].unit1_begin <= u) ++j;
-    x.fixed = u - b.job[j].unit1_begin;
-    x.steps = b.job[j].col_tiles;
-  } else {
-    while (j + 1 < b.count && b.job[j + 1].unit2_begin <= u) ++j;
-    x.fixed = u - b.job[j].unit2_begin;
-    x.steps = b.job[j].row_blocks;
-  }
+  while (j + 1 < b.count && b.job[j + 1].unit_begin <= u) ++j;
+  const WJob& J = b.job[j];
+  int64_t local = u - J.unit_begin;
+  const int64_t bi = wmin(local / J.band_units, J.bands - 1);
+  local -= bi * J.band_units;
+  const int64_t rcount = wmin(kRegionBlocks, J.row_blocks - bi * kRegionBlocks);
+  const int64_t ci = wmin(local / (rcount + kRegionTiles), J.chunks - 1);
+  local -= ci * (rcount + kRegionTiles);
+  const int64_t tcount = wmin(kRegionTiles, J.col_tiles - ci * kRegionTiles);
+  WUnit x;
   x.job = j;
+  if (local < rcount) {
+    x.pass = 1;
+    x.fixed = bi * kRegionBlocks + local;
+    x.start = ci * kRegionTiles;
+    x.steps = static_cast<int>(tcount);
+  } else {
+    x.pass = 2;
+    x.fixed = ci * kRegionTiles + (local - rcount);
+    x.start = bi * kRegionBlocks;
+    x.steps = static_cast<int>(rcount);
+  }
   return x;
 }
 
@@ -156,8 +179,8 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
             ok = false;
             break;
           }
-          const int32_t rb = static_cast<int32_t>(x.pass == 1 ? x.fixed : st);
-          const int32_t ct = static_cast<int32_t>(x.pass == 1 ? st : x.fixed);
+          const int32_t rb = static_cast<int32_t>(x.pass == 1 ? x.fixed : x.start + st);
+          const int32_t ct = static_cast<int32_t>(x.pass == 1 ? x.start + st : x.fixed);
           mbar_arrive_tx(&full[stage], stage_bytes);
           armed[stage] = static_cast<int>(ph);
           uint8_t* g = base + stage * stage_bytes;
@@ -258,12 +281,12 @@ __global__ void __launch_bounds__(kWThreads, 1) ste_wide_kernel(const __grid_con
           if (idx < J.d) {
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-              if (c0 + k < r) J.dA[idx * r + c0 + k] = v[k];
+              if (c0 + k < r) red_add(J.dA + idx * r + c0 + k, v[k]);
           }
         } else if (idx < J.n) {
 #pragma unroll
           for (int k = 0; k < 16; ++k)
-            if (c0 + k < r) J.dB[static_cast<int64_t>(c0 + k) * J.n + idx] = v[k];
+            if (c0 + k < r) red_add(J.dB + static_cast<int64_t>(c0 + k) * J.n + idx, v[k]);
         }
       }
       tc_fence_before();
@@ -307,7 +330,7 @@ cudaError_t launch_ste_wide(const SteJob* jobs, int count, cudaStream_t s) {
     int max_r = 64;
     for (int k = 0; k < m; ++k) max_r = jobs[k0 + k].r > max_r ? jobs[k0 + k].r : max_r;
     const int rp = (max_r + 63) / 64 * 64;
-    int64_t u1 = 0;
+    int64_t units = 0;
     for (int k = 0; k < m; ++k) {
       const SteJob& j = jobs[k0 + k];
       WJob& t = b.job[k];
@@ -323,18 +346,19 @@ cudaError_t launch_ste_wide(const SteJob* jobs, int count, cudaStream_t s) {
       t.r = j.r;
       t.row_blocks = static_cast<int32_t>((j.d + kWRows - 1) / kWRows);
       t.col_tiles = static_cast<int32_t>((j.n + kWCols - 1) / kWCols);
-      t.unit1_begin = u1;
-      u1 += t.row_blocks;
-    }
-    int64_t u2 = u1;
-    for (int k = 0; k < m; ++k) {
-      b.job[k].unit2_begin = u2;
-      u2 += b.job[k].col_tiles;
+      t.bands = (t.row_blocks + kRegionBlocks - 1) / kRegionBlocks;
+      t.chunks = (t.col_tiles + kRegionTiles - 1) / kRegionTiles;
+      t.band_units = static_cast<int64_t>(t.chunks) * kRegionBlocks + t.col_tiles;
+      t.unit_begin = units;
+      // every band but the last is full; a band's units are its chunks' row
+      // blocks plus all the column tiles
+      const int64_t last_rows = t.row_blocks - static_cast<int64_t>(t.bands - 1) * kRegionBlocks;
+      units += static_cast<int64_t>(t.bands - 1) * t.band_units + t.chunks * last_rows + t.col_tiles;
     }
     b.count = m;
     b.rp = rp;
-    b.units1 = u1;
-    b.total_units = u2;
+    b.total_units = units;
+    const int64_t u2 = units;
     int stages = 4;
     while (stages > 2 && w_smem_bytes(rp, stages) > 232448) --stages;
     b.stages = stages;

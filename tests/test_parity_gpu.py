@@ -308,8 +308,10 @@ def test_ste_parity(d, n, r):
 
 @pytest.mark.parametrize("d,n,r", [(100, 304, 128), (257, 1032, 33), (129, 136, 1), (1, 8, 4),
                                    (4096, 1024, 64), (130, 4104, 8),
-                                   # ranks >= 64: two passes, each output written once
-                                   (257, 1032, 96), (130, 4104, 64), (3, 8, 128)])
+                                   # ranks >= 64: two passes over L2-sized regions (up to
+                                   # 16 row blocks x 16 column tiles), reduced into dA, dB
+                                   (257, 1032, 96), (130, 4104, 64), (3, 8, 128),
+                                   (2100, 2600, 128), (2200, 2056, 64)])
 def test_ste_tensor_core_parity(d, n, r):
     """Shapes the tensor-core pass takes (n % 8 == 0, r <= 128): ragged row
     blocks and column tiles, padded ranks (1, 8, 33 -> 16, 16, 48)."""

@@ -166,8 +166,14 @@ bool team_path_enabled() {
   return v == nullptr || std::strcmp(v, "tile") != 0;
 }
 
+// Base quantization of a row wider than kTeamMaxCols that is a whole number
+// of 8-warp sweeps: the team kernel with tensor-memory parking takes it.
+bool team_wide(int variant, const TileLayer& l) {
+  return variant == kGen && l.n > kTeamMaxCols && l.n <= kTeamWideMaxCols && l.n % (4 * kTeamThreads) == 0;
+}
+
 bool team_eligible(int variant, const TileLayer& l) {
-  if (l.n % 4 != 0 || l.n > kTeamMaxCols) return false;
+  if (l.n % 4 != 0 || (l.n > kTeamMaxCols && !team_wide(variant, l))) return false;
   if (l.d > (int64_t{1} << 24)) return false;      // keeps tile indices of a batch in int32
   if (l.d * l.n >= (int64_t{1} << 34)) return false; // Philox block index fits 32 bits
   if (variant != kGen && l.r > 0 && !aligned16(l.B)) return false;
@@ -197,29 +203,29 @@ void team_shape(int64_t n, int* tw_out, int* sweeps_out) {
   *sweeps_out = best_s;
 }
 
-int team_ctas_cached(int variant, int w_bits, int rank_ct, int out_bytes, int sweeps_max) {
+int team_ctas_cached(int variant, int w_bits, int rank_ct, int out_bytes, int sweeps_max, bool wide) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int, int>, int> cache;
+  static std::map<std::tuple<int, int, int, int, int, int, bool>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, out_bytes, sweeps_max);
+  const auto key = std::make_tuple(dev, variant, w_bits, rank_ct, out_bytes, sweeps_max, wide);
   {
     std::lock_guard<std::mutex> g(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
   }
   const int v = team_max_active_ctas(variant, w_bits, rank_ct, out_bytes,
-                                     team_smem_bytes(variant, sweeps_max));
+                                     team_smem_bytes(variant, sweeps_max), wide);
   std::lock_guard<std::mutex> g(mu);
   cache[key] = v;
   return v;
 }
 
 intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, int rank_ct, int bits,
-                                 int w_bits, int out_bytes, uint64_t seed, cudaStream_t stream) {
+                                 int w_bits, int out_bytes, uint64_t seed, cudaStream_t stream, bool wide = false) {
   static thread_local TeamBatch b;
   std::memset(&b, 0, sizeof b);
-  int smax = 1;
+  int smax = wide ? 0 : 1;
   int64_t tiles = 0;
   std::vector<double> layer_cost(L.size()), tile_cost(L.size());
   std::vector<int64_t> layer_tiles(L.size());
@@ -247,8 +253,15 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
     t.d = s.d;
     t.n = s.n;
     t.r = s.r;
-    team_shape(s.n, &t.team_warps, &t.sweeps);
-    smax = std::max(smax, t.sweeps);
+    if (wide) {
+      // the whole CTA is the team; sweeps past the tensor-memory ones in shared memory
+      t.team_warps = kTeamWarps;
+      t.sweeps = static_cast<int32_t>(s.n / (4 * kTeamThreads));
+      smax = std::max(smax, t.sweeps - kTeamTmemSweeps);
+    } else {
+      team_shape(s.n, &t.team_warps, &t.sweeps);
+      smax = std::max(smax, t.sweeps);
+    }
     const int64_t groups = ceil_div(s.d, kTeamRows);
     const int64_t teams = kTeamWarps / t.team_warps;
     t.tile_begin = tiles;
@@ -259,7 +272,7 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
     layer_cost[k] = tile_cost[k] * static_cast<double>(layer_tiles[k]);
     total_cost += layer_cost[k];
   }
-  const int resident = team_ctas_cached(variant, w_bits, rank_ct, out_bytes, smax);
+  const int resident = team_ctas_cached(variant, w_bits, rank_ct, out_bytes, smax, wide);
   if (resident <= 0) return fail(INTLORA_ERR_UNSUPPORTED, "team kernel cannot be made resident");
   const int ctas = static_cast<int>(std::min<int64_t>({int64_t{resident}, int64_t{kTeamMaxCtas}, tiles}));
   // contiguous tile ranges of about equal cost, one per CTA
@@ -288,6 +301,7 @@ intlora_status launch_team_batch(int variant, const std::vector<TileLayer>& L, i
   b.bits = bits;
   b.w_bits = w_bits;
   b.sweeps_max = smax;
+  b.tmem_sweeps = wide ? kTeamTmemSweeps : 0;
   b.num_ctas = ctas;
   b.total_tiles = tiles;
   cudaError_t e = launch_team(b, variant, rank_ct, out_bytes, stream);
@@ -314,8 +328,12 @@ intlora_status launch_tile_batch(int variant, std::vector<TileLayer>& L, int bit
   // layers the team kernel takes go there (one launch); the rest stay here
   // (the team kernels draw Laplace R only)
   if (team_path_enabled() && dist == INTLORA_DIST_LAPLACE) {
-    std::vector<TileLayer> team, rest;
-    for (auto& l : L) (team_eligible(variant, l) ? team : rest).push_back(l);
+    std::vector<TileLayer> team, rest, wide;
+    for (auto& l : L) (team_eligible(variant, l) ? (team_wide(variant, l) ? wide : team) : rest).push_back(l);
+    if (!wide.empty()) {
+      const intlora_status s = launch_team_batch(variant, wide, 0, bits, w_bits, out_bytes, seed, stream, true);
+      if (s != INTLORA_OK) return s;
+    }
     if (!team.empty()) {
       int rank_t = 0;
       if (variant != kGen) {

@@ -118,6 +118,12 @@ constexpr int kTeamRows = 4;
 constexpr int kTeamMaxSweeps = 6;
 constexpr int64_t kTeamMaxCols = int64_t{4} * kTeamThreads * kTeamMaxSweeps;
 constexpr int kTeamMaxCtas = 148 * 4;
+// Base quantization of wider rows (n up to 4 x 256 x (kTeamMaxSweeps +
+// kTeamTmemSweeps), a whole number of sweeps of the 8-warp team): the first
+// kTeamTmemSweeps sweeps of every lane are parked in tensor memory (256
+// columns per CTA, two CTAs per SM), the rest in shared memory.
+constexpr int kTeamTmemSweeps = 8;
+constexpr int64_t kTeamWideMaxCols = int64_t{4} * kTeamThreads * (kTeamMaxSweeps + kTeamTmemSweeps);
 
 struct TeamLayer {
   const void* src;           // kGen: fp32 W; merges: W_round codes
@@ -150,6 +156,7 @@ struct TeamBatch {
   int32_t bits;              // kGen: w_bits; kMul: u_bits; kShift: shift_bits
   int32_t w_bits;
   int32_t sweeps_max;        // shared memory is carved for this many sweeps
+  int32_t tmem_sweeps;       // 0, or kTeamTmemSweeps: sweeps parked in tensor memory (kGen)
   int32_t num_ctas;
   int64_t total_tiles;
   int32_t cta_begin[kTeamMaxCtas + 1];   // tiles of CTA k: [cta_begin[k], cta_begin[k+1])
@@ -191,7 +198,7 @@ cudaError_t launch_tiles(const TileBatch& b, int rank_ct, bool aligned, cudaStre
 int tile_max_active_clusters(int variant, int w_bits, int rank_ct, int out_bytes, bool aligned,
                              int cluster, size_t smem);
 cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s);
-int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem);
+int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem, bool tmem_park = false);
 cudaError_t launch_ste(const SteBatch& b, cudaStream_t s);
 cudaError_t launch_ste_zero(const SteBatch& b, cudaStream_t s);   // dA and dB of every job
 // Masked STE with a workspace: G' = G where W_round != z, else 0 (bf16 copy),

@@ -20,6 +20,7 @@
 
 #include "intlora_device.cuh"
 #include "intlora_kernels.h"
+#include "tcgen05_util.cuh"
 
 namespace intlora {
 
@@ -74,9 +75,17 @@ __device__ __forceinline__ T pick_row(const T v[kTeamRows], int k) {
   return x;
 }
 
-template <int VARIANT, int WBITS, int RANK, int OUTB>
+// TMS > 0 (base quantization of wide rows only): sweeps k < TMS of a lane are
+// parked in tensor memory, lane 32 (warp % 4) + lane, columns
+// 128 (warp / 4) + 16 k .. + 15 (its 4 rows x 4 values); the later sweeps in
+// shared memory as usual. Every lane then has the same number of sweeps
+// (the host takes only rows that are a whole number of sweeps), so the
+// warp-collective tensor-memory accesses are never divergent.
+template <int VARIANT, int WBITS, int RANK, int OUTB, int TMS>
 __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_constant__ TeamBatch p) {
+  static_assert(TMS == 0 || (VARIANT == kGen && TMS * kTeamRows * 4 * 2 <= 256), "tensor-memory parking: kGen, 256 columns");
   extern __shared__ __align__(16) float4 smem4[];
+  __shared__ uint32_t tmem_slot;
   const int smax = p.sweeps_max;
   float4* Ubuf = smem4;                                              // [smax][4][256]
   // code words of the merges: [smax][kTeamRows][256]
@@ -95,7 +104,20 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
   if (VARIANT != kGen)
     for (int k = tid; k < 511; k += kTeamThreads)
       rcp_tab[k] = (k == 255) ? 0.0f : __frcp_rn(static_cast<float>(k - 255));
+  uint32_t tpark = 0;                      // this thread's first parking column in tensor memory
+  if (TMS > 0) {
+    if (warp == 0) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                   ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(&tmem_slot))), "r"(256u) : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc::tc_fence_before();
+  }
   __syncthreads();
+  if (TMS > 0) {
+    tc::tc_fence_after();
+    tpark = tmem_slot + ((static_cast<uint32_t>(warp & 3) * 32u) << 16) + static_cast<uint32_t>(warp >> 2) * 128u;
+  }
 
   const int64_t t_begin = p.cta_begin[blockIdx.x];
   const int64_t t_end = p.cta_begin[blockIdx.x + 1];
@@ -310,7 +332,10 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
             lo[ml] = fminf(lo[ml], v[c]);
           }
         }
-        Ubuf[(k * kTeamRows + ml) * kTeamThreads + tid] = make_float4(v[0], v[1], v[2], v[3]);
+        if (TMS > 0 && k < TMS)
+          tc::tmem_st4(tpark + static_cast<uint32_t>((k * kTeamRows + ml) * 4), make_float4(v[0], v[1], v[2], v[3]));
+        else
+          Ubuf[((k - TMS) * kTeamRows + ml) * kTeamThreads + tid] = make_float4(v[0], v[1], v[2], v[3]);
         if (VARIANT == kGen && L.r_star_out != nullptr && ml < rows) {
           float* rs = L.r_star_out + irow[ml] * n + j;
           *reinterpret_cast<float4*>(rs) =
@@ -323,6 +348,8 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
         for (int ml = 0; ml < kTeamRows; ++ml) Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] = cw[ml];
       }
     }
+
+    if (TMS > 0) tc::tmem_st_wait_all();        // this warp's parked values are in
 
     // ---- row extrema: over the warp (REDUX), then over the team
     uint32_t ehi[kTeamRows], elo[kTeamRows];
@@ -400,10 +427,17 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml)
         cw[ml] = VARIANT != kGen ? Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] : 0u;
+      float parked[TMS > 0 ? 16 : 1];             // the sweep's 4 rows from tensor memory
+      if (TMS > 0 && k < TMS) {
+        tc::tmem_ld16(tpark + static_cast<uint32_t>(k * kTeamRows * 4), parked);
+        tc::tmem_ld_wait();
+      }
 #pragma unroll
       for (int ml = 0; ml < kTeamRows; ++ml) {
         if (ml >= rows) break;
-        const float4 u4 = Ubuf[(k * kTeamRows + ml) * kTeamThreads + tid];
+        const float4 u4 = (TMS > 0 && k < TMS)
+                              ? make_float4(parked[4 * ml], parked[4 * ml + 1], parked[4 * ml + 2], parked[4 * ml + 3])
+                              : Ubuf[((k - TMS) * kTeamRows + ml) * kTeamThreads + tid];
         const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
         const int64_t i = row0 + ml;
         int32_t res[4];
@@ -458,11 +492,19 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       }
     }
   }
+  if (TMS > 0) {
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+      tc::tc_fence_after();
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_slot), "r"(256u) : "memory");
+    }
+  }
 }
 
-template <int VARIANT, int WBITS, int RANK, int OUTB>
+template <int VARIANT, int WBITS, int RANK, int OUTB, int TMS = 0>
 struct TeamLaunch {
-  static constexpr auto kernel() { return team_kernel<VARIANT, WBITS, RANK, OUTB>; }
+  static constexpr auto kernel() { return team_kernel<VARIANT, WBITS, RANK, OUTB, TMS>; }
   static cudaError_t launch(const TeamBatch& b, cudaStream_t s) {
     const size_t smem = team_smem_bytes(VARIANT, b.sweeps_max);
     cudaError_t err = cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -482,9 +524,21 @@ struct TeamLaunch {
       cudaGetLastError();
       return 0;
     }
-    int dev = 0, sms = 0;
+    int dev = 0, sms = 0, smem_sm = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (TMS > 0 && per_sm < 2) {
+      // The occupancy query answers one CTA per SM for the tensor-memory
+      // variant at any shared-memory size, yet two fit: 2 x 256 threads x
+      // 128 registers is the register file, each CTA takes 256 of the 512
+      // tensor-memory columns, and the shared memory is checked here
+      // (measured on the 4096 x 14336 layers: 1.27x faster with two).
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kernel()) == cudaSuccess && fa.numRegs * kTeamThreads * 2 <= 65536 &&
+          2 * (smem + fa.sharedSizeBytes + 1024) <= static_cast<size_t>(smem_sm))
+        per_sm = 2;
+    }
     return per_sm * sms;
   }
 };
@@ -498,9 +552,9 @@ struct TeamQuery {
   cudaError_t err;
 };
 
-template <int VARIANT, int WBITS, int RANK, int OUTB>
+template <int VARIANT, int WBITS, int RANK, int OUTB, int TMS = 0>
 void team_run(TeamQuery& q) {
-  using T = TeamLaunch<VARIANT, WBITS, RANK, OUTB>;
+  using T = TeamLaunch<VARIANT, WBITS, RANK, OUTB, TMS>;
   if (q.op == 0) q.err = T::launch(*q.batch, q.stream);
   else q.result = T::max_ctas(q.smem);
 }
@@ -516,10 +570,16 @@ void team_by_rank(TeamQuery& q, int rank_ct) {
   }
 }
 
-void team_dispatch(TeamQuery& q, int variant, int w_bits, int rank_ct, int out_bytes) {
+void team_dispatch(TeamQuery& q, int variant, int w_bits, int rank_ct, int out_bytes, bool tmem_park) {
   if (variant == kGen) {
-    if (w_bits == 8) team_run<kGen, 8, 0, 1>(q);
-    else team_run<kGen, 4, 0, 1>(q);
+    if (tmem_park) {
+      if (w_bits == 8) team_run<kGen, 8, 0, 1, kTeamTmemSweeps>(q);
+      else team_run<kGen, 4, 0, 1, kTeamTmemSweeps>(q);
+    } else if (w_bits == 8) {
+      team_run<kGen, 8, 0, 1>(q);
+    } else {
+      team_run<kGen, 4, 0, 1>(q);
+    }
   } else if (variant == kMul) {
     if (w_bits == 8) {
       if (out_bytes == 4) team_by_rank<kMul, 8, 4>(q, rank_ct);
@@ -544,13 +604,13 @@ size_t team_smem_bytes(int variant, int sweeps_max) {
 
 cudaError_t launch_team(const TeamBatch& b, int variant, int rank_ct, int out_bytes, cudaStream_t s) {
   TeamQuery q{0, 0, &b, s, 0, cudaSuccess};
-  team_dispatch(q, variant, variant == kGen ? b.bits : b.w_bits, rank_ct, out_bytes);
+  team_dispatch(q, variant, variant == kGen ? b.bits : b.w_bits, rank_ct, out_bytes, b.tmem_sweeps > 0);
   return q.err;
 }
 
-int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem) {
+int team_max_active_ctas(int variant, int w_bits, int rank_ct, int out_bytes, size_t smem, bool tmem_park) {
   TeamQuery q{1, smem, nullptr, nullptr, 0, cudaSuccess};
-  team_dispatch(q, variant, w_bits, rank_ct, out_bytes);
+  team_dispatch(q, variant, w_bits, rank_ct, out_bytes, tmem_park);
   return q.result;
 }
 

@@ -35,7 +35,10 @@ def test_aux_matrix_matches_oracle(d, n):
 # a1-a3: layer preparation
 # ---------------------------------------------------------------------------
 GEN_SHAPES = [(320, 320, 8), (64, 768, 4), (33, 100, 8), (7, 10, 4), (5, 6, 8), (1, 4, 8),
-              (130, 5120, 4), (20, 14336, 8), (9, 2, 4)]
+              (130, 5120, 4), (20, 14336, 8), (9, 2, 4),
+              # rows of whole 8-warp sweeps past 6144 columns: tensor-memory parking
+              # (7 and 8 sweeps: all in tensor memory; 12 and 14: the rest in shared memory)
+              (13, 14336, 4), (70, 12288, 8), (9, 7168, 8), (6, 8192, 4)]
 
 
 @pytest.mark.parametrize("d,n,w_bits", GEN_SHAPES)
@@ -49,6 +52,21 @@ def test_gen_aux_parity(d, n, w_bits):
     assert_scale("s", g["s"], o["s"])
     assert_affine("W_round", g["codes"], g["z"], o["codes"], o["z"], o["pre"], o["zpre"],
                   2**w_bits - 1)
+
+
+def test_gen_aux_wide_rows_team_equals_tile(monkeypatch):
+    """The tensor-memory-parked team kernel and the row-tile kernels give the
+    same codes, scales and zero-points on wide rows (one batch of mixed widths)."""
+    specs = [spec_for(d, n, 4, b, sid=60 + k) for k, (d, n, b) in
+             enumerate([(21, 14336, 8), (8, 12288, 4), (5, 7168, 8), (12, 4096, 8)])]
+    Ws = [wl.host_W(s) for s in specs]
+    monkeypatch.setenv("INTLORA_ROW_KERNEL", "tile")
+    tile = gpu_gen_aux(specs, Ws, batched=True)
+    monkeypatch.setenv("INTLORA_ROW_KERNEL", "auto")
+    team = gpu_gen_aux(specs, Ws, batched=True)
+    for x, y in zip(team, tile):
+        assert np.array_equal(x["codes"], y["codes"])
+        assert np.array_equal(x["s"], y["s"]) and np.array_equal(x["z"], y["z"])
 
 
 def test_gen_aux_batched_equals_single():

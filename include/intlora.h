@@ -431,14 +431,17 @@ uint32_t intlora_device_timeouts(void);
  * G is never formed: with Z1 = X B^T and Z2 = dY A (tokens x r),
  * dA = dY^T Z1 and dB = Z2^T X, every product on the tensor cores with fp32
  * accumulation (Z enters the last products as two exact bf16 halves, so
- * they stay fp32-faithful).
+ * they stay fp32-faithful). Besides the dX GEMM, X is streamed twice and dY
+ * once (X -> Z1; dY -> Z2 and dA; X -> dB), each pass forming both of its
+ * products from one read.
  *
  * X: bf16 tokens x n; dY: bf16 tokens x d; W: bf16 d x n; A: bf16 d x r;
  * B: bf16 r x n; all row-major, X, dY, W, B 16-byte aligned. Outputs (fp32,
  * row-major, 16-byte aligned): dX tokens x n, dA d x r, dB r x n; written,
  * not accumulated. Requires tokens >= 1, d and n multiples of 8, 1 <= r <= 64.
  * The workspace (intlora_train_backward_workspace_size, 256-byte aligned
- * regions per job) holds W'^T, A^T, Z1, Z2 and the halves' products.
+ * regions per job) holds W'^T, A^T and B padded with r zero rows, Z1 and Z2
+ * with their bf16 halves, and the halves' products.
  * ------------------------------------------------------------------------ */
 typedef struct intlora_train_backward_job {
     const void* X;

@@ -1096,23 +1096,26 @@ uint32_t intlora_device_timeouts(void) {
 
 namespace {
 
-// Workspace regions of one training-backward job, in order (each 256-byte aligned).
+// Workspace regions of one training-backward job, in order (each 256-byte aligned):
+// W'^T, [A^T; 0], [B; 0], a zero tokens x 2r operand, the tokens x 2r fp32
+// product of the current pass, the two split operands, the two 2r-row
+// products that become dA and dB.
 struct TbWs {
-  size_t wt, at, z1, z2, zs1, zs2, b0, o1, o2, j1, j2, total;
+  size_t wt, at, bp, zz, zw, zs1, zs2, o1, o2, total;
 };
 TbWs tb_ws_layout(const intlora_train_backward_job& j) {
   TbWs w;
   const size_t T = static_cast<size_t>(j.tokens), d = static_cast<size_t>(j.d), n = static_cast<size_t>(j.n);
   const size_t r = static_cast<size_t>(j.r);
   w.wt = round256(n * d * 2);
-  w.at = round256(r * d * 2);
-  w.z1 = w.z2 = round256(T * r * 4);
+  w.at = round256(2 * r * d * 2);
+  w.bp = round256(2 * r * n * 2);
+  w.zz = round256(T * 2 * r * 2);
+  w.zw = round256(T * 2 * r * 4);
   w.zs1 = w.zs2 = round256(T * 2 * r * 2);
-  w.b0 = round256(2 * r * std::max(d, n) * 2);
   w.o1 = round256(2 * r * d * 4);
   w.o2 = round256(2 * r * n * 4);
-  w.j1 = w.j2 = round256(T * 2 * r * 4);
-  w.total = w.wt + w.at + w.z1 + w.z2 + w.zs1 + w.zs2 + w.b0 + w.o1 + w.o2 + w.j1 + w.j2;
+  w.total = w.wt + w.at + w.bp + w.zz + w.zw + w.zs1 + w.zs2 + w.o1 + w.o2;
   return w;
 }
 
@@ -1176,55 +1179,70 @@ intlora_status intlora_train_backward_batched(const intlora_train_backward_job* 
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   std::vector<TransposeJob> tr;
   std::vector<intlora_linear_job> lin;
-  std::vector<SplitZJob> split;
-  std::vector<intlora_ste_job> ste;
+  std::vector<intlora_ste_job> pass_x1, pass_y, pass_x2;
+  std::vector<SplitZJob> split1, split2;
   std::vector<CombineJob> comb;
   char* p = static_cast<char*>(ws);
   for (int32_t k = 0; k < count; ++k) {
     const intlora_train_backward_job& j = jobs[k];
     const TbWs w = tb_ws_layout(j);
-    uint16_t* wt = reinterpret_cast<uint16_t*>(p);
-    uint16_t* at = reinterpret_cast<uint16_t*>(p + w.wt);
-    float* z1 = reinterpret_cast<float*>(p + w.wt + w.at);
-    float* z2 = reinterpret_cast<float*>(p + w.wt + w.at + w.z1);
-    uint16_t* zs1 = reinterpret_cast<uint16_t*>(p + w.wt + w.at + w.z1 + w.z2);
-    uint16_t* zs2 = reinterpret_cast<uint16_t*>(p + w.wt + w.at + w.z1 + w.z2 + w.zs1);
-    char* b0 = p + w.wt + w.at + w.z1 + w.z2 + w.zs1 + w.zs2;
-    float* o1 = reinterpret_cast<float*>(b0 + w.b0);
-    float* o2 = reinterpret_cast<float*>(b0 + w.b0 + w.o1);
-    float* j1 = reinterpret_cast<float*>(b0 + w.b0 + w.o1 + w.o2);
-    float* j2 = reinterpret_cast<float*>(b0 + w.b0 + w.o1 + w.o2 + w.j1);
-    // W'^T (n x d) and A^T (r x d): every GEMM operand K-major
+    char* q = p;
+    uint16_t* wt = reinterpret_cast<uint16_t*>(q);
+    q += w.wt;
+    uint16_t* at = reinterpret_cast<uint16_t*>(q);      // [A^T; 0]: 2r x d
+    q += w.at;
+    uint16_t* bp = reinterpret_cast<uint16_t*>(q);      // [B; 0]: 2r x n
+    q += w.bp;
+    uint16_t* zz = reinterpret_cast<uint16_t*>(q);      // zeros: tokens x 2r
+    q += w.zz;
+    float* zw = reinterpret_cast<float*>(q);            // tokens x 2r: [Z1 | 0], then [Z2 | 0]
+    q += w.zw;
+    uint16_t* zs1 = reinterpret_cast<uint16_t*>(q);
+    q += w.zs1;
+    uint16_t* zs2 = reinterpret_cast<uint16_t*>(q);
+    q += w.zs2;
+    float* o1 = reinterpret_cast<float*>(q);            // [Z1_hi | Z1_lo]^T dY: 2r x d
+    q += w.o1;
+    float* o2 = reinterpret_cast<float*>(q);            // [Z2_hi | Z2_lo]^T X: 2r x n
+    // the padded operands: zero rows r .. 2r - 1, then A^T and B in rows 0 .. r - 1
+    cudaError_t e = cudaMemsetAsync(at, 0, w.at + w.bp + w.zz, st);
+    if (e != cudaSuccess) return cuda_fail(e, "zero operand fill");
+    e = cudaMemcpyAsync(bp, j.B, static_cast<size_t>(j.r) * j.n * 2, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "B operand copy");
     tr.push_back(TransposeJob{static_cast<const uint16_t*>(j.W), wt, j.d, j.n, 0});
     tr.push_back(TransposeJob{static_cast<const uint16_t*>(j.A), at, j.d, j.r, 0});
-    // dX = dY W' (K = d), Z1 = X B^T (K = n), Z2 = dY A (K = d), fp32 out
+    // dX = dY W' (K = d), fp32 out
     lin.push_back(intlora_linear_job{j.dY, wt, j.tokens, j.n, j.d, j.dX, 0});
-    lin.push_back(intlora_linear_job{j.X, j.B, j.tokens, j.r, j.n, z1, 0});
-    lin.push_back(intlora_linear_job{j.dY, at, j.tokens, j.r, j.d, z2, 0});
-    split.push_back(SplitZJob{z1, zs1, j.tokens, j.r});
-    split.push_back(SplitZJob{z2, zs2, j.tokens, j.r});
-    // one pass over dY: [Z1_hi | Z1_lo]^T dY (2r x d); one over X: [Z2_hi | Z2_lo]^T X (2r x n);
-    // the STE kernel's other product (against the zero B) is discarded
-    intlora_ste_job s1;
-    std::memset(&s1, 0, sizeof s1);
-    s1.G = j.dY; s1.A = zs1; s1.B = b0; s1.d = j.tokens; s1.n = j.d; s1.r = 2 * j.r; s1.dA = j1; s1.dB = o1;
-    intlora_ste_job s2 = s1;
-    s2.G = j.X; s2.A = zs2; s2.n = j.n; s2.dA = j2; s2.dB = o2;
-    ste.push_back(s1);
-    ste.push_back(s2);
+    // pass over X: its product with [B; 0] is [Z1 | 0] (the other product, against zeros, is discarded)
+    intlora_ste_job s;
+    std::memset(&s, 0, sizeof s);
+    s.G = j.X; s.A = zz; s.B = bp; s.d = j.tokens; s.n = j.n; s.r = 2 * j.r; s.dA = zw; s.dB = o2;
+    pass_x1.push_back(s);
+    split1.push_back(SplitZJob{zw, zs1, j.tokens, j.r, 2 * j.r});
+    // pass over dY: [Z2 | 0] = dY [A^T; 0]^T and [Z1_hi | Z1_lo]^T dY (-> dA)
+    s.G = j.dY; s.A = zs1; s.B = at; s.n = j.d; s.dA = zw; s.dB = o1;
+    pass_y.push_back(s);
+    split2.push_back(SplitZJob{zw, zs2, j.tokens, j.r, 2 * j.r});
+    // pass over X: [Z2_hi | Z2_lo]^T X (-> dB); the other product is discarded
+    s.G = j.X; s.A = zs2; s.B = bp; s.n = j.n; s.dA = zw; s.dB = o2;
+    pass_x2.push_back(s);
     comb.push_back(CombineJob{o1, j.dA, j.d, j.r, 1});     // dA = (top + bottom)^T
     comb.push_back(CombineJob{o2, j.dB, j.n, j.r, 0});     // dB = top + bottom
-    const cudaError_t e = cudaMemsetAsync(b0, 0, w.b0, st);
-    if (e != cudaSuccess) return cuda_fail(e, "zero operand fill");
     p += w.total;
   }
   cudaError_t e = launch_transpose_bf16(tr.data(), static_cast<int>(tr.size()), st);
   if (e != cudaSuccess) return cuda_fail(e, "transpose launch");
   intlora_status s = intlora_linear_bf16_batched(lin.data(), static_cast<int32_t>(lin.size()), stream);
   if (s != INTLORA_OK) return s;
-  e = launch_split_hilo(split.data(), static_cast<int>(split.size()), st);
+  s = intlora_ste_backward_batched(pass_x1.data(), static_cast<int32_t>(pass_x1.size()), nullptr, 0, stream);
+  if (s != INTLORA_OK) return s;
+  e = launch_split_hilo(split1.data(), static_cast<int>(split1.size()), st);
   if (e != cudaSuccess) return cuda_fail(e, "split launch");
-  s = intlora_ste_backward_batched(ste.data(), static_cast<int32_t>(ste.size()), nullptr, 0, stream);
+  s = intlora_ste_backward_batched(pass_y.data(), static_cast<int32_t>(pass_y.size()), nullptr, 0, stream);
+  if (s != INTLORA_OK) return s;
+  e = launch_split_hilo(split2.data(), static_cast<int>(split2.size()), st);
+  if (e != cudaSuccess) return cuda_fail(e, "split launch");
+  s = intlora_ste_backward_batched(pass_x2.data(), static_cast<int32_t>(pass_x2.size()), nullptr, 0, stream);
   if (s != INTLORA_OK) return s;
   e = launch_combine_halves(comb.data(), static_cast<int>(comb.size()), st);
   if (e != cudaSuccess) return cuda_fail(e, "combine launch");

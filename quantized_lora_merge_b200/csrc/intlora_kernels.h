@@ -331,11 +331,12 @@ struct TransposeJob {        // out (cols x rows) = in (rows x cols)^T, bf16
   int64_t rows, cols;
   int64_t block_begin;       // set by the launcher
 };
-struct SplitZJob {           // zs (rows x 2r bf16) = [hi | lo] of z (rows x r fp32)
+struct SplitZJob {           // zs (rows x 2r bf16) = [hi | lo] of z (rows x r fp32, row stride ld)
   const float* z;
   uint16_t* zs;
   int64_t rows;
   int32_t r;
+  int32_t ld;                // floats between rows of z (>= r)
 };
 struct CombineJob {          // out = in[0:r] + in[r:2r] (in: 2r x cols fp32); transposed: out is cols x r
   const float* in;

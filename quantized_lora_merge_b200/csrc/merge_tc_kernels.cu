@@ -213,7 +213,9 @@ __device__ __forceinline__ Unit unit_of(const MtcBatch& b, int64_t u) {
   return x;
 }
 
-template <int VARIANT, int WBITS, int OUTB>
+// CODE: some layer of the launch asks for the U codes as well (code_out);
+// the instantiation without it forms no code bytes at all.
+template <int VARIANT, int WBITS, int OUTB, bool CODE>
 __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_constant__ MtcBatch b) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t tmem_slot;
@@ -618,7 +620,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
           tmem_ld16(tmem + lane_base + static_cast<uint32_t>(cc), v);
           tmem_ld_wait();
           int32_t res[16];
-          uint32_t code8[16];
+          uint32_t code8[CODE ? 16 : 1];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int32_t dcode = code_at<WBITS>(cw, k) - zv;
@@ -627,12 +629,12 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
               const int32_t sh = clamp_i(neg_log2_round(vn), 0, qmax);
               const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
               res[k] = sgn * (dcode >> sh);
-              code8[k] = static_cast<uint32_t>(sh);
+              if (CODE) code8[CODE ? k : 0] = static_cast<uint32_t>(sh);
             } else {
               // biased rounding word clamped to the code range, bias taken off after
               const int32_t cb = clamp_i(__float_as_int(fmaf(v[k], inv, kRoundBias)), bias_lo, bias_hi);
               res[k] = (cb - kRoundBiasBits) * dcode;
-              code8[k] = static_cast<uint32_t>(cb - bias_lo);
+              if (CODE) code8[CODE ? k : 0] = static_cast<uint32_t>(cb - bias_lo);
             }
           }
           if (OUTB == 1) {
@@ -687,12 +689,15 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
             }
             ++nstore;
           }
-          if (valid) {
+          if (CODE && valid) {
             if (L.code_out != nullptr) {
               uint32_t cv[4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                cv[q] = code8[4 * q] | (code8[4 * q + 1] << 8) | (code8[4 * q + 2] << 16) | (code8[4 * q + 3] << 24);
+              for (int q = 0; q < 4; ++q) {
+                const int k0 = CODE ? 4 * q : 0;
+                cv[q] = code8[k0] | (code8[k0 + (CODE ? 1 : 0)] << 8) | (code8[k0 + (CODE ? 2 : 0)] << 16) |
+                        (code8[k0 + (CODE ? 3 : 0)] << 24);
+              }
               *reinterpret_cast<uint4*>(L.code_out + row * n + j) = make_uint4(cv[0], cv[1], cv[2], cv[3]);
             }
           }
@@ -731,9 +736,9 @@ int mtc_stages(int atoms_max) {
 
 int mtc_atoms(int32_t r) { return r <= 32 ? 1 : (r <= 64 ? 2 : 4); }
 
-template <int VARIANT, int WBITS, int OUTB>
+template <int VARIANT, int WBITS, int OUTB, bool CODE>
 struct MtcLaunch {
-  static constexpr auto kernel() { return merge_tc_kernel<VARIANT, WBITS, OUTB>; }
+  static constexpr auto kernel() { return merge_tc_kernel<VARIANT, WBITS, OUTB, CODE>; }
   static int blocks_per_sm(size_t smem) {
     if (cudaFuncSetAttribute(kernel(), cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess) {
@@ -773,20 +778,26 @@ struct MtcQuery {
   cudaError_t err;
 };
 template <int VARIANT, int WBITS, int OUTB>
-void mtc_run(MtcQuery& q) {
-  using T = MtcLaunch<VARIANT, WBITS, OUTB>;
-  if (q.op == 0) q.err = T::launch(*q.batch, q.smem, q.stream);
-  else q.result = T::blocks_per_sm(q.smem);
+void mtc_run(MtcQuery& q, bool code) {
+  if (code) {
+    using T = MtcLaunch<VARIANT, WBITS, OUTB, true>;
+    if (q.op == 0) q.err = T::launch(*q.batch, q.smem, q.stream);
+    else q.result = T::blocks_per_sm(q.smem);
+  } else {
+    using T = MtcLaunch<VARIANT, WBITS, OUTB, false>;
+    if (q.op == 0) q.err = T::launch(*q.batch, q.smem, q.stream);
+    else q.result = T::blocks_per_sm(q.smem);
+  }
 }
-bool mtc_dispatch(MtcQuery& q, int variant, int w_bits, int out_bytes) {
+bool mtc_dispatch(MtcQuery& q, int variant, int w_bits, int out_bytes, bool code) {
   if (variant == kMul) {
-    if (w_bits == 8 && out_bytes == 4) mtc_run<kMul, 8, 4>(q);
-    else if (w_bits == 8 && out_bytes == 2) mtc_run<kMul, 8, 2>(q);
-    else if (w_bits == 4 && out_bytes == 2) mtc_run<kMul, 4, 2>(q);
+    if (w_bits == 8 && out_bytes == 4) mtc_run<kMul, 8, 4>(q, code);
+    else if (w_bits == 8 && out_bytes == 2) mtc_run<kMul, 8, 2>(q, code);
+    else if (w_bits == 4 && out_bytes == 2) mtc_run<kMul, 4, 2>(q, code);
     else return false;
   } else {
-    if (w_bits == 4 && out_bytes == 1) mtc_run<kShift, 4, 1>(q);
-    else if (w_bits == 8 && out_bytes == 2) mtc_run<kShift, 8, 2>(q);
+    if (w_bits == 4 && out_bytes == 1) mtc_run<kShift, 4, 1>(q, code);
+    else if (w_bits == 8 && out_bytes == 2) mtc_run<kShift, 8, 2>(q, code);
     else return false;
   }
   return true;
@@ -834,6 +845,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     std::memset(&b, 0, sizeof b);
     int atoms_max = 1;
     int64_t units = 0;
+    bool code = false;
     for (int k = 0; k < m; ++k) {
       const MtcJob& j = jobs[k0 + k];
       MtcLayerDev& t = b.layer[k];
@@ -858,6 +870,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
       t.scale_out = j.scale_out;
       t.zero_out = j.zero_out;
       t.code_out = j.code_out;
+      code = code || j.code_out != nullptr;
       t.d = j.d;
       t.n = j.n;
       t.unit_begin = units;
@@ -880,7 +893,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     b.total_units = units;
     const size_t smem = mtc_smem_bytes(atoms_max, b.stages);
     MtcQuery q{1, smem, nullptr, s, 0, cudaSuccess};
-    if (!mtc_dispatch(q, variant, w_bits, out_bytes)) return cudaErrorInvalidValue;
+    if (!mtc_dispatch(q, variant, w_bits, out_bytes, code)) return cudaErrorInvalidValue;
     if (q.result < 1) return cudaErrorInvalidConfiguration;
     // one CTA per SM (shared memory and tensor memory allow no more)
     const int64_t fit = std::min<int64_t>(num_sms(), kMergeTcMaxCtas) / G;
@@ -892,7 +905,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     if (e != cudaSuccess) return e;
     q.op = 0;
     q.batch = &b;
-    mtc_dispatch(q, variant, w_bits, out_bytes);
+    mtc_dispatch(q, variant, w_bits, out_bytes, code);
     if (q.err != cudaSuccess) return q.err;
   }
   return cudaSuccess;

@@ -440,9 +440,13 @@ def main():
     # is reported beside it.
     sm_mhz = clk.get("sm_mhz") or 1965.0
     alu_peak = NUM_SMS * ALU_LANES_PER_SM_CLK * sm_mhz * 1e6 / 1e12          # Top/s
-    fused = (not args.dist) and all(l.r >= 16 and l.n % 32 == 0 for l in layers)
-    alu_achieved = sum(merge_ops(l, fused) for l in layers) / (stage_ms["merge"] / 1e3) / 1e12
+    # the library's routing: the fused kernel from rank 16, and at any rank for
+    # rows wider than the team kernels take (6144 columns)
+    on_tc = [(not args.dist) and l.n % 32 == 0 and (l.r >= 16 or l.n > 6144) for l in layers]
+    fused = all(on_tc)
+    alu_achieved = sum(merge_ops(l, f) for l, f in zip(layers, on_tc)) / (stage_ms["merge"] / 1e3) / 1e12
     kernel_name = ("merge_tc_kernel (fused tensor-core merge)" if fused else
+                   "merge_tc_kernel (wide rows) + team kernels" if any(on_tc) else
                    "team / row-tile merge kernels" if not args.dist else
                    "merge row-tile kernel (general auxiliary law)")
     traffic = None
@@ -469,7 +473,7 @@ def main():
                      "alu_achieved_Top_s": alu_achieved, "alu_peak_Top_s": alu_peak,
                      "alu_frac_modelled": alu_achieved / alu_peak,
                      "alu_peak_source": f"148 SMs x 128 lanes x measured {sm_mhz:.0f} MHz",
-                     "ops_per_element_modelled": merge_ops(layers[0], fused) / layers[0].numel},
+                     "ops_per_element_modelled": merge_ops(layers[0], on_tc[0]) / layers[0].numel},
         "stages": stages,
         "clocks": clk,
         "gpu_launches": launches,

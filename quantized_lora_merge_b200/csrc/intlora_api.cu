@@ -592,7 +592,9 @@ bool uses_tensor_t(const intlora_layer& l) {
 // "tc" sends every layer the fused tensor-core kernel takes there, whatever
 // its rank; unset or "auto": the fused kernel takes the layers it supports
 // from rank kMergeTcAutoMinRank up (below it the CUDA-core FMAs of the team
-// kernels cost less than the tensor-core hand-offs).
+// kernels cost less than the tensor-core hand-offs), and at any rank the rows
+// too wide for the team kernels (the row-tile kernels are slower than the
+// fused one there: measured on 4096 x 14336 layers at r = 4 and 8).
 constexpr int32_t kMergeTcAutoMinRank = 16;   // measured: the team kernels win at r = 8, the fused kernel at r = 16
 int merge_kernel_mode() {
   const char* v = std::getenv("INTLORA_MERGE_KERNEL");
@@ -604,7 +606,7 @@ int merge_kernel_mode() {
 bool uses_merge_tc(const intlora_layer& l) {
   const int mode = merge_kernel_mode();
   if (mode == 1 || l.distribution != INTLORA_DIST_LAPLACE) return false;
-  if (mode == 0 && l.r < kMergeTcAutoMinRank) return false;
+  if (mode == 0 && l.r < kMergeTcAutoMinRank && l.n <= kTeamMaxCols) return false;
   // 32-bit Philox block index and tensor-map extents
   if (l.d * l.n >= (int64_t{1} << 34) || l.d >= (int64_t{1} << 31)) return false;
   MtcPlan plan;

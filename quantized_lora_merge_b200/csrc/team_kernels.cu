@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "intlora_device.cuh"
 #include "intlora_kernels.h"
@@ -419,78 +420,85 @@ __global__ void __launch_bounds__(kTeamThreads, 2) team_kernel(const __grid_cons
       gen_lo[ml] = kRoundBiasBits - zq[ml];
       orow[ml] = static_cast<uint8_t*>(L.out) + irow[ml] * n * static_cast<int64_t>(OUTB);
     }
-    for (int k = 0; k < S; ++k) {
-      const int q = lt + k * LT;
-      if (q >= quads) break;
-      const int64_t j = 4 * static_cast<int64_t>(q);
-      uint32_t cw[kTeamRows];
-#pragma unroll
-      for (int ml = 0; ml < kTeamRows; ++ml)
-        cw[ml] = VARIANT != kGen ? Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] : 0u;
-      float parked[TMS > 0 ? 16 : 1];             // the sweep's 4 rows from tensor memory
-      if (TMS > 0 && k < TMS) {
-        tc::tmem_ld16(tpark + static_cast<uint32_t>(k * kTeamRows * 4), parked);
-        tc::tmem_ld_wait();
-      }
-#pragma unroll
-      for (int ml = 0; ml < kTeamRows; ++ml) {
-        if (ml >= rows) break;
-        const float4 u4 = (TMS > 0 && k < TMS)
-                              ? make_float4(parked[4 * ml], parked[4 * ml + 1], parked[4 * ml + 2], parked[4 * ml + 3])
-                              : Ubuf[((k - TMS) * kTeamRows + ml) * kTeamThreads + tid];
-        const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
-        const int64_t i = row0 + ml;
-        int32_t res[4];
-        uint32_t code8[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (VARIANT == kShift) {
-            const float vn = uv[c] * inv[ml];
-            const int32_t sh = clamp_i(neg_log2_round(vn), 0, qmax);
-            const int32_t dcode = nib<WBITS>(cw[ml], c) - zv[ml];
-            const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
-            res[c] = sgn * (dcode >> sh);
-            code8[c] = static_cast<uint32_t>(sh);
-          } else if (VARIANT == kMul) {
-            const int32_t centred = clamp_i(rne_scaled(uv[c], inv[ml]), -zq[ml], qmax - zq[ml]);
-            res[c] = centred * (nib<WBITS>(cw[ml], c) - zv[ml]);
-            code8[c] = static_cast<uint32_t>(centred + zq[ml]);
-          } else {
-            // the biased rounding word clamped straight to the code range
-            // [bias - z, bias - z + qmax]; the bias comes off once per word below
-            code8[c] = static_cast<uint32_t>(
-                clamp_i(__float_as_int(fmaf(uv[c], inv[ml], kRoundBias)), gen_lo[ml], gen_lo[ml] + qmax));
-            res[c] = 0;
+    // the merges form the U code bytes only when the layer asks for them
+    // (two copies of the loop; the base quantization's output is the codes)
+    auto phase_b = [&](auto want_code) {
+      constexpr bool WC = decltype(want_code)::value;
+      for (int k = 0; k < S; ++k) {
+        const int q = lt + k * LT;
+        if (q >= quads) break;
+        const int64_t j = 4 * static_cast<int64_t>(q);
+        uint32_t cw[kTeamRows];
+  #pragma unroll
+        for (int ml = 0; ml < kTeamRows; ++ml)
+          cw[ml] = VARIANT != kGen ? Cbuf[(k * kTeamRows + ml) * kTeamThreads + tid] : 0u;
+        float parked[TMS > 0 ? 16 : 1];             // the sweep's 4 rows from tensor memory
+        if (TMS > 0 && k < TMS) {
+          tc::tmem_ld16(tpark + static_cast<uint32_t>(k * kTeamRows * 4), parked);
+          tc::tmem_ld_wait();
+        }
+  #pragma unroll
+        for (int ml = 0; ml < kTeamRows; ++ml) {
+          if (ml >= rows) break;
+          const float4 u4 = (TMS > 0 && k < TMS)
+                                ? make_float4(parked[4 * ml], parked[4 * ml + 1], parked[4 * ml + 2], parked[4 * ml + 3])
+                                : Ubuf[((k - TMS) * kTeamRows + ml) * kTeamThreads + tid];
+          const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+          const int64_t i = row0 + ml;
+          int32_t res[4];
+          uint32_t code8[4];
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (VARIANT == kShift) {
+              const float vn = uv[c] * inv[ml];
+              const int32_t sh = clamp_i(neg_log2_round(vn), 0, qmax);
+              const int32_t dcode = nib<WBITS>(cw[ml], c) - zv[ml];
+              const int32_t sgn = vn > 0.0f ? 1 : (vn < 0.0f ? -1 : 0);
+              res[c] = sgn * (dcode >> sh);
+              if (WC) code8[c] = static_cast<uint32_t>(sh);
+            } else if (VARIANT == kMul) {
+              const int32_t centred = clamp_i(rne_scaled(uv[c], inv[ml]), -zq[ml], qmax - zq[ml]);
+              res[c] = centred * (nib<WBITS>(cw[ml], c) - zv[ml]);
+              if (WC) code8[c] = static_cast<uint32_t>(centred + zq[ml]);
+            } else {
+              // the biased rounding word clamped straight to the code range
+              // [bias - z, bias - z + qmax]; the bias comes off once per word below
+              code8[c] = static_cast<uint32_t>(
+                  clamp_i(__float_as_int(fmaf(uv[c], inv[ml], kRoundBias)), gen_lo[ml], gen_lo[ml] + qmax));
+              res[c] = 0;
+            }
           }
+          if (VARIANT == kGen) {
+            // sum_c (word_c - lo) 2^(bits c), modulo 2^32 (multiply-adds)
+            uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
+            const uint32_t lo = static_cast<uint32_t>(gen_lo[ml]);
+            if (WBITS == 8)
+              *reinterpret_cast<uint32_t*>(orow + j) =
+                  code8[0] + code8[1] * 0x100u + code8[2] * 0x10000u + code8[3] * 0x1000000u - lo * 0x01010101u;
+            else
+              *reinterpret_cast<uint16_t*>(orow + (j >> 1)) = static_cast<uint16_t>(
+                  code8[0] + code8[1] * 16u + code8[2] * 256u + code8[3] * 4096u - lo * 0x1111u);
+            continue;
+          }
+          uint8_t* const op = orow[ml] + j * OUTB;
+          if (OUTB == 4) {
+            *reinterpret_cast<int4*>(op) = make_int4(res[0], res[1], res[2], res[3]);
+          } else if (OUTB == 2) {
+            const uint32_t w0 = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
+            const uint32_t w1 = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
+            *reinterpret_cast<uint2*>(op) = make_uint2(w0, w1);
+          } else {
+            *reinterpret_cast<uint32_t*>(op) =
+                (static_cast<uint32_t>(res[0]) & 0xFFu) | ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
+                ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) | (static_cast<uint32_t>(res[3]) << 24);
+          }
+          if (WC)
+            *reinterpret_cast<uint32_t*>(L.code_out + i * n + j) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
         }
-        if (VARIANT == kGen) {
-          // sum_c (word_c - lo) 2^(bits c), modulo 2^32 (multiply-adds)
-          uint8_t* orow = static_cast<uint8_t*>(L.out) + i * L.ld_out;
-          const uint32_t lo = static_cast<uint32_t>(gen_lo[ml]);
-          if (WBITS == 8)
-            *reinterpret_cast<uint32_t*>(orow + j) =
-                code8[0] + code8[1] * 0x100u + code8[2] * 0x10000u + code8[3] * 0x1000000u - lo * 0x01010101u;
-          else
-            *reinterpret_cast<uint16_t*>(orow + (j >> 1)) = static_cast<uint16_t>(
-                code8[0] + code8[1] * 16u + code8[2] * 256u + code8[3] * 4096u - lo * 0x1111u);
-          continue;
-        }
-        uint8_t* const op = orow[ml] + j * OUTB;
-        if (OUTB == 4) {
-          *reinterpret_cast<int4*>(op) = make_int4(res[0], res[1], res[2], res[3]);
-        } else if (OUTB == 2) {
-          const uint32_t w0 = (static_cast<uint32_t>(res[0]) & 0xFFFFu) | (static_cast<uint32_t>(res[1]) << 16);
-          const uint32_t w1 = (static_cast<uint32_t>(res[2]) & 0xFFFFu) | (static_cast<uint32_t>(res[3]) << 16);
-          *reinterpret_cast<uint2*>(op) = make_uint2(w0, w1);
-        } else {
-          *reinterpret_cast<uint32_t*>(op) =
-              (static_cast<uint32_t>(res[0]) & 0xFFu) | ((static_cast<uint32_t>(res[1]) & 0xFFu) << 8) |
-              ((static_cast<uint32_t>(res[2]) & 0xFFu) << 16) | (static_cast<uint32_t>(res[3]) << 24);
-        }
-        if (L.code_out != nullptr)
-          *reinterpret_cast<uint32_t*>(L.code_out + i * n + j) = code8[0] | (code8[1] << 8) | (code8[2] << 16) | (code8[3] << 24);
       }
-    }
+    };
+    if (VARIANT == kGen || L.code_out != nullptr) phase_b(std::true_type{});
+    else phase_b(std::false_type{});
   }
   if (TMS > 0) {
     tc::tc_fence_before();

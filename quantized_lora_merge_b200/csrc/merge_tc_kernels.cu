@@ -123,7 +123,7 @@ struct alignas(64) MtcLayerDev {
 };
 struct MtcBatch {
   MtcLayerDev layer[kMaxMtcJobs];
-  ulonglong2* slots;             // [groups][2][G][128] tagged row extrema (zeroed before the launch)
+  uint64_t* slots;               // [groups][2][G][128] tagged row extrema (zeroed before the launch)
   int32_t count;
   uint32_t key0, key1;
   int32_t bits;                  // MUL: u_bits; SHIFT: shift_bits
@@ -165,16 +165,20 @@ __device__ __forceinline__ uint32_t idesc_tf32(uint32_t n) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
-// Exchange area accesses, L2-coherent (another SM wrote them). A slot is two
-// 64-bit words, each (tag << 32) | value: an aligned 64-bit access is single-
-// copy atomic, so a word whose tag matches carries its own value and no fence
-// or flag is needed to publish it.
-__device__ __forceinline__ void st_slot(ulonglong2* p, uint64_t w0, uint64_t w1) {
-  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+// Exchange area accesses, L2-coherent (another SM wrote them). A slot is one
+// 64-bit word: the row maximum and negated minimum as |value| bit patterns
+// (31 bits each) and a 2-bit tag. An aligned 64-bit access is single-copy
+// atomic, so a word whose tag matches carries its own values and no fence or
+// flag is needed to publish it.
+__device__ __forceinline__ uint64_t slot_word(uint32_t top, uint32_t negb, uint32_t tag) {
+  return (static_cast<uint64_t>(top) << 33) | (static_cast<uint64_t>(negb) << 2) | tag;
 }
-__device__ __forceinline__ ulonglong2 ld_slot(const ulonglong2* p) {
-  ulonglong2 v;
-  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+__device__ __forceinline__ void st_slot(uint64_t* p, uint64_t w) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ uint64_t ld_slot(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int qmax = (1 << b.bits) - 1;
     const bool sender = member == 0;
-    ulonglong2* my_slots = b.slots + static_cast<int64_t>(grp) * 2 * G * kRows;
+    uint64_t* my_slots = b.slots + static_cast<int64_t>(grp) * 2 * G * kRows;
     uint2* gat = ext + kMembers * kRows;           // [kMembers][128] partial group extrema
     int cur = -1, ucount = 0;
     uint32_t nstore = 0;                           // output blocks this warp has sent
@@ -520,19 +524,20 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
         const uint2 f = ext[m * kRows + row_u];
         own = make_uint2(max(own.x, f.x), max(own.y, f.y));
       }
-      const uint32_t want = static_cast<uint32_t>(ucount) + 1u;      // this unit's tag
-      if (sender)
-        st_slot(my_slots + (static_cast<int64_t>(up) * G + rank) * kRows + row_u,
-                (static_cast<uint64_t>(want) << 32) | own.x, (static_cast<uint64_t>(want) << 32) | own.y);
+      // this unit's tag: the slot set (parity) alternates every unit, so the
+      // stale word a slot can hold is the unit two back's (other tag) or the
+      // launch's zero fill (tag 0)
+      const uint32_t want = ((static_cast<uint32_t>(ucount) >> 1) & 1u) + 1u;
+      if (sender) st_slot(my_slots + (static_cast<int64_t>(up) * G + rank) * kRows + row_u, slot_word(own.x, own.y, want));
       // member m gathers the other CTAs k = m, m + kMembers, ... of the group,
       // kGather slots in flight at a time; a slot is read again (sleeping
-      // between reads, bounded) until both words carry this unit's tag
+      // between reads, bounded) until it carries this unit's tag
       uint2 part = own;
       {
-        const ulonglong2* sp = my_slots + static_cast<int64_t>(up) * G * kRows + row_u;
+        const uint64_t* sp = my_slots + static_cast<int64_t>(up) * G * kRows + row_u;
         uint64_t t0 = 0;
         for (int k0 = member; k0 < G && !abort_flag; k0 += kGather * kMembers) {
-          ulonglong2 e[kGather];
+          uint64_t e[kGather];
 #pragma unroll
           for (int i = 0; i < kGather; ++i) {
             const int k = k0 + i * kMembers;
@@ -542,7 +547,7 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
           for (int i = 0; i < kGather; ++i) {
             const int k = k0 + i * kMembers;
             if (k >= G || k == rank) continue;
-            for (uint32_t it = 1; static_cast<uint32_t>(e[i].x >> 32) != want || static_cast<uint32_t>(e[i].y >> 32) != want; ++it) {
+            for (uint32_t it = 1; static_cast<uint32_t>(e[i] & 3u) != want; ++it) {
               __nanosleep(64);
               e[i] = ld_slot(sp + static_cast<int64_t>(k) * kRows);
               if ((it & 63u) == 0u) {
@@ -555,7 +560,8 @@ __global__ void __launch_bounds__(kMtcThreads, 1) merge_tc_kernel(const __grid_c
                 if (abort_flag) break;
               }
             }
-            part = make_uint2(max(part.x, static_cast<uint32_t>(e[i].x)), max(part.y, static_cast<uint32_t>(e[i].y)));
+            part = make_uint2(max(part.x, static_cast<uint32_t>(e[i] >> 33)),
+                              max(part.y, static_cast<uint32_t>(e[i] >> 2) & 0x7FFFFFFFu));
           }
         }
       }
@@ -832,7 +838,7 @@ bool merge_tc_plan(int64_t n, int32_t r, MtcPlan* plan) {
 
 size_t merge_tc_exchange_bytes() {
   // the double-buffered tagged row extrema of up to kMergeTcMaxCtas CTAs
-  return static_cast<size_t>(kMergeTcMaxCtas) * 2 * kRows * sizeof(ulonglong2);
+  return static_cast<size_t>(kMergeTcMaxCtas) * 2 * kRows * sizeof(uint64_t);
 }
 
 cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bits, int out_bytes, int bits,
@@ -900,8 +906,8 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     if (fit < 1) return cudaErrorInvalidConfiguration;
     b.num_groups = static_cast<int32_t>(units < fit ? units : fit);
     // tags restart at 1 with every launch: the slots this launch uses start zeroed
-    b.slots = static_cast<ulonglong2*>(exchange);
-    cudaError_t e = cudaMemsetAsync(b.slots, 0, static_cast<size_t>(b.num_groups) * G * 2 * kRows * sizeof(ulonglong2), s);
+    b.slots = static_cast<uint64_t*>(exchange);
+    cudaError_t e = cudaMemsetAsync(b.slots, 0, static_cast<size_t>(b.num_groups) * G * 2 * kRows * sizeof(uint64_t), s);
     if (e != cudaSuccess) return e;
     q.op = 0;
     q.batch = &b;

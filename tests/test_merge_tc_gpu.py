@@ -102,5 +102,24 @@ def test_fused_without_code_output_and_repeat():
     assert np.array_equal(b["code"], c["code"]) and np.array_equal(b["sbar"], c["sbar"])
 
 
+@pytest.mark.parametrize("r", [4, 8])
+def test_wide_low_rank_rows_route_to_fused(monkeypatch, r):
+    """Rows wider than the team kernels take (n > 6144) go to the fused kernel
+    at any rank under the default routing (a batch with a narrow layer of the
+    same rank beside it): both layers meet the oracle, and the wide one agrees
+    with the rows path (A B on the CUDA cores) up to the rounding-boundary
+    codes the two ways of forming A B may split differently."""
+    specs = [spec_for(70, 8192, r, 8, "mul", 8, sid=90 + r), spec_for(64, 1024, r, 8, "mul", 8, sid=91 + r)]
+    inps = [_oracle_prepared(sp) for sp in specs]
+    monkeypatch.setenv("INTLORA_MERGE_KERNEL", "auto")
+    auto = gpu_merge(specs, inps, batched=True)
+    monkeypatch.setenv("INTLORA_MERGE_KERNEL", "rows")
+    rows = gpu_merge(specs, inps, batched=True)
+    for sp, inp, x, y in zip(specs, inps, auto, rows):
+        assert np.mean(x["out"] != y["out"]) < 1e-3
+        assert np.max(np.abs(x["sbar"] / y["sbar"] - 1)) < 1e-6
+        _check_mul(sp, inp, x)
+
+
 def test_fused_no_device_wait_gave_up():
     assert B.intlora_device_status() == 0

@@ -17,10 +17,11 @@
 // row's running extrema in registers and writes U back in place
 // (tcgen05.st). The extrema of the G CTAs are combined through a small
 // exchange area in the caller's workspace: each CTA stores its 128 row
-// extrema as tagged 64-bit words (tag = the unit's number in the launch), and
-// the quantizer threads of a row read the other CTAs' words, several in
-// flight at once, until every tag matches; no fence, flag or extra barrier
-// hop lies on that path. Then the same thread reads U back, quantizes it and
+// extrema as one 64-bit word per row (both extrema and a 2-bit tag that
+// tells this unit from the one two back, which used the same slot set), and
+// the quantizer threads of a row read the other CTAs' words, two in flight
+// at a time, until every tag matches; no fence, flag or extra barrier hop
+// lies on that path. Then the same thread reads U back, quantizes it and
 // stores its row's merged weights.
 // Nothing else of the merge touches global memory.
 //
@@ -905,7 +906,7 @@ cudaError_t launch_merge_tc(const MtcJob* jobs, int count, int variant, int w_bi
     const int64_t fit = std::min<int64_t>(num_sms(), kMergeTcMaxCtas) / G;
     if (fit < 1) return cudaErrorInvalidConfiguration;
     b.num_groups = static_cast<int32_t>(units < fit ? units : fit);
-    // tags restart at 1 with every launch: the slots this launch uses start zeroed
+    // tag 0 matches no unit: the slots this launch uses start zeroed
     b.slots = static_cast<uint64_t*>(exchange);
     cudaError_t e = cudaMemsetAsync(b.slots, 0, static_cast<size_t>(b.num_groups) * G * 2 * kRows * sizeof(uint64_t), s);
     if (e != cudaSuccess) return e;

@@ -480,8 +480,20 @@ def main():
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e(states, arena_in, arena_out, device, max(4, min(args.steps, 10)),
-                          world, elements, masked_ste=args.masked_ste)
+        ok, why = host_room(arena_in.numel() + arena_out.numel(),
+                            int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
+        if world > 1:
+            # every rank takes the same branch (the leg holds collectives)
+            f = torch.tensor([1 if ok else 0], device=device, dtype=torch.int32)
+            dist.all_reduce(f, op=dist.ReduceOp.MIN)
+            if ok and int(f.item()) == 0:
+                why = "another rank's node lacks the host memory for its pinned arenas"
+            ok = int(f.item()) == 1
+        if ok:
+            line["e2e"] = e2e(states, arena_in, arena_out, device, max(4, min(args.steps, 10)),
+                              world, elements, masked_ste=args.masked_ste)
+        else:
+            line["e2e"] = {"value": None, "unit": UNIT, "unavailable": why}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layers_base, args.cpu_seconds)
     if not args.no_extra:
@@ -633,6 +645,22 @@ def pinned_host(nbytes):
     def release():
         rt.cudaHostUnregister(a.ctypes.data)
     return t, release
+
+
+def host_room(need_bytes, local_ranks, meminfo="/proc/meminfo"):
+    """Whether this node's available host memory holds the end-to-end leg's
+    pinned arenas for every rank on it (need_bytes each, 10 % margin).
+    Returns (ok, reason)."""
+    try:
+        with open(meminfo) as f:
+            avail = next(int(line.split()[1]) * 1024 for line in f if line.startswith("MemAvailable:"))
+    except (OSError, StopIteration, ValueError, IndexError):
+        return True, ""                 # unknown: let cudaHostRegister decide
+    total = need_bytes * max(1, local_ranks)
+    if total * 1.1 <= avail:
+        return True, ""
+    return False, (f"pinned host arenas of {local_ranks} rank(s) x {need_bytes / 1e9:.1f} GB exceed "
+                   f"the node's {avail / 1e9:.1f} GB of available host memory")
 
 
 def layer_groups(states, budget_bytes=3 << 30):

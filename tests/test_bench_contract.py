@@ -42,3 +42,18 @@ def test_algorithmic_counts(cfg):
         assert bench.merge_ops(l) == l.numel * (22 + l.r + (5.5 if l.variant == "mul" else 8.0))
         # the tensor cores form A B in the fused kernel: no rank term on the lanes
         assert bench.merge_ops(l, True) == l.numel * (22 + (5.5 if l.variant == "mul" else 8.0))
+
+
+def test_host_room_for_pinned_arenas(tmp_path):
+    """The end-to-end leg's pinned arenas are checked against the node's
+    available host memory for every rank on the node (10 % margin)."""
+    mi = tmp_path / "meminfo"
+    mi.write_text("MemTotal:       209715200 kB\nMemAvailable:   104857600 kB\n")   # 100 GiB free
+    need = 40 << 30
+    assert bench.host_room(need, 1, str(mi)) == (True, "")
+    assert bench.host_room(need, 2, str(mi)) == (True, "")        # 80 GiB x 1.1 < 100 GiB
+    ok, why = bench.host_room(need, 3, str(mi))
+    assert not ok and "3 rank(s)" in why
+    # no MemAvailable line: nothing to compare against, the leg runs
+    mi.write_text("MemTotal:       209715200 kB\n")
+    assert bench.host_room(need, 8, str(mi)) == (True, "")

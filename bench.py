@@ -480,10 +480,13 @@ def main():
     }
 
     if not args.no_e2e:
-        ok, why = host_room(arena_in.numel() + arena_out.numel(),
-                            int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
+        ok, why = True, ""
         if world > 1:
+            # several ranks pin their arenas on one node: check the node's
+            # memory first (one rank alone leaves it to cudaHostRegister), and
             # every rank takes the same branch (the leg holds collectives)
+            ok, why = host_room(arena_in.numel() + arena_out.numel(),
+                                int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
             f = torch.tensor([1 if ok else 0], device=device, dtype=torch.int32)
             dist.all_reduce(f, op=dist.ReduceOp.MIN)
             if ok and int(f.item()) == 0:

@@ -263,12 +263,33 @@ def oracle_sample(layers, seconds):
     return done, t_total, names
 
 
+def single_core(layers):
+    """The oracle on one host thread over the config's smallest layer (whole
+    path, repeated until a second has passed), beside the all-core figure."""
+    import oracle
+    small = min(layers, key=lambda l: l.numel)
+    threads = oracle.num_threads()
+    oracle.set_num_threads(1)
+    done, t, passes = 0, 0.0, 0
+    try:
+        cores = oracle.num_threads()
+        while t < 1.0:
+            d, tt, _ = oracle_sample([small], 0.0)
+            done, t, passes = done + d, t + tt, passes + 1
+    finally:
+        oracle.set_num_threads(threads)
+    return {"value": done / t, "unit": UNIT, "cores": cores,
+            "sample": f"layer {small.name} ({small.d}x{small.n}, the config's smallest) x {passes}, "
+                      f"prepare + merge + STE, {t:.1f} s"}
+
+
 def cpu_baseline(layers, seconds):
     import oracle
     done, t, names = oracle_sample(layers, seconds)
     return {"value": done / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"first {len(names)} of {len(layers)} layers in workload order "
-                      f"({done} merged elements, prepare + merge + STE, {t:.1f} s)"}
+                      f"({done} merged elements, prepare + merge + STE, {t:.1f} s)",
+            "single_core": single_core(layers)}
 
 
 # ---------------------------------------------------------------------------
@@ -297,7 +318,8 @@ def run_reference(args, layers, desc):
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle",
                              "sample": f"each step: first {len(names)} layers in workload "
-                                       f"order, prepare + merge + STE"},
+                                       f"order, prepare + merge + STE",
+                             "single_core": single_core(layers)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -15,6 +15,7 @@ matmul). No function is "parity unpinned".
 from __future__ import annotations
 
 import ctypes
+import hashlib
 import os
 import subprocess
 from pathlib import Path
@@ -35,13 +36,19 @@ _ptr = ctypes.c_void_p
 
 
 def build(force: bool = False) -> Path:
-    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE: no fast-math)."""
-    if force or not _LIB_PATH.exists() or _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE: no fast-math).
+    The library is rebuilt whenever the source's hash differs from the one
+    recorded beside it (copies of the tree need not keep file times)."""
+    digest = hashlib.sha256(_SRC.read_bytes()).hexdigest()
+    stamp = _LIB_PATH.with_name(_LIB_PATH.name + ".sha256")
+    fresh = _LIB_PATH.exists() and stamp.exists() and stamp.read_text().strip() == digest
+    if force or not fresh:
         tmp = _LIB_PATH.with_suffix(f".so.tmp{os.getpid()}")
         cmd = ["gcc", "-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp",
                "-fPIC", "-shared", str(_SRC), "-o", str(tmp), "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB_PATH)
+        stamp.write_text(digest + "\n")
     return _LIB_PATH
 
 
@@ -85,6 +92,7 @@ def _load():
         "orc_linear_rows": (None, [_ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_int_gemm_rows": (None, [_ptr, _ptr, _ptr, _ptr, _i64, _i64, _i64, _ptr, _i64, _ptr]),
         "orc_num_threads": (_int, []),
+        "orc_set_num_threads": (None, [_int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -438,3 +446,8 @@ def train_backward(X_bits, dY_bits, W_bits, A_bits, B_bits) -> dict:
 
 def num_threads() -> int:
     return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads of the oracle's later calls from this thread."""
+    _load().orc_set_num_threads(int(n))

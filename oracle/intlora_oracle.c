@@ -628,3 +628,14 @@ int orc_num_threads(void) {
     return 1;
 #endif
 }
+
+/* Threads of the calling thread's later parallel regions (n >= 1); the
+ * benchmark's single-core figure uses it. No arithmetic depends on it: every
+ * parallel loop above writes disjoint outputs, each computed in one thread. */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -28,6 +28,8 @@ def test_reference_arm_json_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    one = line["cpu_baseline"]["single_core"]
+    assert one["cores"] == 1 and one["value"] > 0 and one["unit"] == line["unit"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
 
 

@@ -503,6 +503,31 @@ def test_row_views_equal_whole_layer_functions():
         np.testing.assert_array_equal(mr[k], m[k][rows])
 
 
+def test_results_do_not_depend_on_the_thread_count():
+    """One host thread and all of them give the same bits: the statistics add
+    row sums in row order and every parallel loop writes its own outputs (the
+    benchmark's single-core figure relies on this)."""
+    spec, W, A, B, g = _prepared(37, 52, 8, 8, sid=17)
+    s32 = g["s"].astype(np.float32)
+    many = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        assert oracle.num_threads() == 1
+        g1 = oracle.gen_aux(W, spec.seed, 17, spec.alpha, 8)
+        m1 = oracle.merge_mul(g1["codes"], g1["s"].astype(np.float32), g1["z"], A, B, spec.seed, 17,
+                              g1["sigma_w"], g1["sigma_r"], spec.alpha, 8)
+    finally:
+        oracle.set_num_threads(many)
+    assert oracle.num_threads() == many
+    m = oracle.merge_mul(g["codes"], s32, g["z"], A, B, spec.seed, 17, g["sigma_w"], g["sigma_r"],
+                         spec.alpha, 8)
+    assert g1["sigma_w"] == g["sigma_w"] and g1["sigma_r"] == g["sigma_r"]
+    for k in ("codes", "s", "z"):
+        np.testing.assert_array_equal(g1[k], g[k])
+    for k in ("u_round", "sbar", "zbar", "P"):
+        np.testing.assert_array_equal(m1[k], m[k])
+
+
 # ---------------------------------------------------------------------------
 # auxiliary laws of the ablation: Gaussian, Cauchy, Student-t (2 dof)
 # ---------------------------------------------------------------------------

@@ -38,7 +38,7 @@ def test_package_never_imports_the_oracle():
 def test_bench_uses_the_oracle_only_for_its_cpu_legs():
     src = (ROOT / "bench.py").read_text()
     tree = ast.parse(src)
-    allowed_functions = {"oracle_sample", "cpu_baseline", "run_reference"}
+    allowed_functions = {"oracle_sample", "single_core", "cpu_baseline", "run_reference"}
     parents = {}
     for node in ast.walk(tree):
         for child in ast.iter_child_nodes(node):

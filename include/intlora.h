@@ -243,17 +243,19 @@ int32_t intlora_merge_out_bytes(int32_t variant, int32_t w_bits, int32_t out_bit
 
 /* Workspace of a merge call (16-byte aligned device memory, caller-owned):
  *  - for each layer with sigma_r == NULL: the scratch of its sigma_R reduction;
- *  - for each Laplace layer with r in [32, 128] and n % 4 == 0 (on a device
- *    with the tensor-map driver entry point): its product T = A B (d x n fp32)
- *    and the exact tf32 hi/lo splits of A and B^T that the tensor cores
- *    multiply (4 (d + n) kp x 2 bytes, kp = 32 or 64); for r above 64 (two
- *    passes over the rank) also the second product (d x n fp32) and A's two
- *    column blocks (2 x d x 64 fp32) -- [IntLoRA paper notes, method section
- *    2: U = s + (R* + A B) / D].
+ *  - for each Laplace layer the fused tensor-core merge takes (n % 32 == 0,
+ *    and r >= 16 or n > 6144): the exact tf32 hi/lo splits of A and B^T that
+ *    the tensor cores multiply (4 (d + n) kp x 2 bytes, kp = 32, 64 or 128),
+ *    plus, once per call, the kernel's row-exchange area (512 KiB);
+ *  - for each other Laplace layer with r in [32, 128] and n % 4 == 0: its
+ *    product T = A B (d x n fp32) and the same splits (kp = 32 or 64); for r
+ *    above 64 (two passes over the rank) also the second product (d x n
+ *    fp32) and A's two column blocks (2 x d x 64 fp32)
+ *  -- [IntLoRA paper notes, method section 2: U = s + (R* + A B) / D].
  * A call given at least the sigma part but less than the whole still runs: it
- * then forms A B on the CUDA cores inside the merge kernels (same results up
- * to fp32 rounding order, slower at these ranks). Less than the sigma part:
- * INTLORA_ERR_WORKSPACE. */
+ * then forms A B on the CUDA cores inside the row merge kernels (same results
+ * up to fp32 rounding order, slower at these ranks). Less than the sigma
+ * part: INTLORA_ERR_WORKSPACE. */
 size_t intlora_merge_workspace_size(const intlora_layer* layers, int32_t count);
 
 /* IntLoRA_MUL, u_bits in [2, 8]. */
@@ -413,11 +415,13 @@ intlora_status intlora_linear_bf16_batched(const intlora_linear_job* jobs, int32
                                            void* stream);
 
 /* Number of bounded device-side waits that gave up since the library was
- * loaded: 0 in a healthy run. The tensor-core STE kernel bounds every wait on
- * an mbarrier (2 s); a wait that gives up is counted here, the CTA stops, releases its
+ * loaded: 0 in a healthy run. Every kernel that waits on an mbarrier or on
+ * another CTA (the tensor-core STE kernels, the T GEMM, the integer GEMM,
+ * the fused merge and its row exchange) bounds each wait (2 s); a wait that
+ * gives up is counted here, the CTA drains what it started, releases its
  * tensor memory and returns, so a broken run shows up as a nonzero count and
- * wrong outputs instead of a hung device. Synchronous (reads one device
- * word); the library has no counterpart of this on the pages. */
+ * wrong outputs instead of a hung device. Synchronous (reads the device
+ * counters); the library has no counterpart of this on the pages. */
 uint32_t intlora_device_timeouts(void);
 
 /* --------------------------------------------------------------------------

@@ -69,7 +69,9 @@
  *   - Every call validates its arguments on the host and returns a status
  *     before launching anything. Work is then enqueued asynchronously on
  *     `stream` (a cudaStream_t; NULL = legacy default stream). A launch
- *     failure returns INTLORA_ERR_CUDA. No call synchronizes the device.
+ *     failure returns INTLORA_ERR_CUDA. No call synchronizes the device,
+ *     except the status queries intlora_device_status and
+ *     intlora_device_timeouts, which say so.
  *   - Outputs must not alias inputs. Calls on different streams that share a
  *     workspace race.
  *   - intlora_last_error() returns a thread-local description of the most

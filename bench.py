@@ -502,18 +502,7 @@ def main():
     }
 
     if not args.no_e2e:
-        ok, why = True, ""
-        if world > 1:
-            # several ranks pin their arenas on one node: check the node's
-            # memory first (one rank alone leaves it to cudaHostRegister), and
-            # every rank takes the same branch (the leg holds collectives)
-            ok, why = host_room(arena_in.numel() + arena_out.numel(),
-                                int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
-            f = torch.tensor([1 if ok else 0], device=device, dtype=torch.int32)
-            dist.all_reduce(f, op=dist.ReduceOp.MIN)
-            if ok and int(f.item()) == 0:
-                why = "another rank's node lacks the host memory for its pinned arenas"
-            ok = int(f.item()) == 1
+        ok, why = e2e_allowed(arena_in.numel() + arena_out.numel(), world, device)
         if ok:
             line["e2e"] = e2e(states, arena_in, arena_out, device, max(4, min(args.steps, 10)),
                               world, elements, masked_ste=args.masked_ste)
@@ -686,6 +675,25 @@ def host_room(need_bytes, local_ranks, meminfo="/proc/meminfo"):
         return True, ""
     return False, (f"pinned host arenas of {local_ranks} rank(s) x {need_bytes / 1e9:.1f} GB exceed "
                    f"the node's {avail / 1e9:.1f} GB of available host memory")
+
+
+def e2e_allowed(need_bytes, world, device, meminfo="/proc/meminfo"):
+    """Whether the end-to-end leg runs. One rank alone leaves the question to
+    cudaHostRegister; several ranks check their node's memory for every
+    local rank's arenas (host_room) and agree by a MIN all-reduce, so every
+    rank takes the same branch (the leg holds collectives). Returns
+    (ok, reason)."""
+    if world <= 1:
+        return True, ""
+    import torch
+    import torch.distributed as dist
+    ok, why = host_room(need_bytes, int(os.environ.get("LOCAL_WORLD_SIZE", "1")), meminfo)
+    f = torch.tensor([1 if ok else 0], device=device, dtype=torch.int32)
+    dist.all_reduce(f, op=dist.ReduceOp.MIN)
+    agreed = int(f.item()) == 1
+    if ok and not agreed:
+        why = "another rank's node lacks the host memory for its pinned arenas"
+    return agreed, why
 
 
 def layer_groups(states, budget_bytes=3 << 30):

@@ -84,3 +84,46 @@ def test_two_rank_sharded_results_equal_single_rank():
     for k, spec in enumerate(layers):
         assert np.array_equal(merged[k], _layer_result(spec))
     assert tmax == 2.0
+
+
+def _e2e_worker(rank, world, port, mem_kb, tmpdir, out_q):
+    import datetime
+    import sys
+    from pathlib import Path
+    sys.path.insert(0, str(Path(__file__).resolve().parents[1]))
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    os.environ["LOCAL_WORLD_SIZE"] = "1"
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        mi = Path(tmpdir) / f"meminfo{rank}"
+        mi.write_text(f"MemTotal: {2 * mem_kb[rank]} kB\nMemAvailable: {mem_kb[rank]} kB\n")
+        ok, why = bench.e2e_allowed(40 << 30, world, torch.device("cpu"), meminfo=str(mi))
+        out_q.put((rank, ok, why))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mem_gib,expect", [((200, 200), True), ((200, 10), False)])
+def test_end_to_end_leg_is_skipped_by_every_rank_or_none(tmp_path, mem_gib, expect):
+    """bench.py's end-to-end leg holds collectives, so the host-memory check
+    is agreed across ranks: one short node makes every rank skip it."""
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    mem_kb = [g << 20 for g in mem_gib]
+    procs = [ctx.Process(target=_e2e_worker, args=(r, 2, port, mem_kb, str(tmp_path), q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict((r, (ok, why)) for r, ok, why in (q.get(timeout=300) for _ in range(2)))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    assert got[0][0] == got[1][0] == expect
+    if not expect:
+        assert "rank(s)" in got[1][1] and "another rank" in got[0][1]

@@ -7,6 +7,7 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 from pathlib import Path
 
 PKG = Path(__file__).resolve().parent
@@ -38,14 +39,14 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> Path:
         return LIB
     objdir = ROOT / "_build"
     objdir.mkdir(exist_ok=True)
-    objs = []
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
-    for src in sources():
-        obj = objdir / (src.stem + ".o")
-        cmd = [NVCC, *ARCH, *FLAGS, *extra, "-I", str(INCLUDE), "-I", str(CSRC), "-c", str(src),
-               "-o", str(obj)]
-        subprocess.run(cmd, check=True)
-        objs.append(str(obj))
+    objs = [str(objdir / (src.stem + ".o")) for src in sources()]
+    cmds = [[NVCC, *ARCH, *FLAGS, *extra, "-I", str(INCLUDE), "-I", str(CSRC), "-c", str(src),
+             "-o", obj] for src, obj in zip(sources(), objs)]
+    # the translation units are independent: compile them side by side
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for done in [pool.submit(subprocess.run, cmd, check=True) for cmd in cmds]:
+            done.result()
     tmp = LIB.with_suffix(f".so.tmp{os.getpid()}")
     subprocess.run([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", *objs, "-o", str(tmp)],
                    check=True)

@@ -1274,7 +1274,7 @@ intlora_status intlora_int_pack(const void* q, int32_t q_bytes, int64_t d, int64
   if (q_bytes != 1 && q_bytes != 2 && q_bytes != 4)
     return fail(INTLORA_ERR_INVALID_ARG, "q_bytes must be 1, 2 or 4");
   if (planes < 1 || planes > 3) return fail(INTLORA_ERR_INVALID_ARG, "planes must be 1, 2 or 3");
-  if (d < 0 || n < 0 || n % 16 != 0) return fail(INTLORA_ERR_INVALID_ARG, "d >= 0, n >= 0 and n % 16 == 0 required");
+  if (d < 0 || n < 0 || n % 16 != 0) return fail(INTLORA_ERR_INVALID_ARG, "d >= 0, n >= 0 and n %% 16 == 0 required");
   if (n > 0 && d > kMaxElements / n) return fail(INTLORA_ERR_INVALID_ARG, "d*n exceeds 2^40");
   if (d * n == 0) return INTLORA_OK;
   if (q == nullptr || packed == nullptr) return fail(INTLORA_ERR_INVALID_ARG, "q and packed are required");

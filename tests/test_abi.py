@@ -145,6 +145,7 @@ def test_int_pack_rejects(lib):
     assert lib.intlora_int_pack(FAKE, 3, 4, 16, 1, FAKE, None, None) == 1      # q_bytes
     assert lib.intlora_int_pack(FAKE, 2, 4, 16, 4, FAKE, None, None) == 1      # planes
     assert lib.intlora_int_pack(FAKE, 2, 4, 24, 2, FAKE, None, None) == 1      # n % 16
+    assert lib.intlora_last_error() == b"d >= 0, n >= 0 and n % 16 == 0 required"
     assert lib.intlora_int_pack(FAKE, 2, 4, 16, 2, FAKE + 8, None, None) == 1  # alignment
     assert lib.intlora_int_pack(None, 2, 0, 16, 2, None, None, None) == 0      # empty: no-op
 

@@ -3,7 +3,9 @@ the oracle library given on the command line (a build with AddressSanitizer
 and UndefinedBehaviorSanitizer, see tests/test_oracle_sanitized.py). Checks
 nothing itself: the sanitizers abort the process on an out-of-bounds access,
 a use after free or undefined behaviour, and the test reads the exit status.
-Prints "done" when every call returned."""
+Prints "done" when every call returned. With --pins it runs the oracle's pin
+suite (tests/test_oracle_pins.py) on the same library instead, except the
+comparison with Triton's Philox, which runs in an interpreter of its own."""
 import sys
 from pathlib import Path
 
@@ -93,4 +95,10 @@ def main():
 
 
 if __name__ == "__main__":
+    if "--pins" in sys.argv[2:]:
+        import pytest
+        # -s: a sanitizer report goes straight to stderr instead of a capture file
+        sys.exit(pytest.main(["-q", "-x", "-s", "-p", "no:cacheprovider",
+                              str(Path(__file__).resolve().parent / "test_oracle_pins.py"),
+                              "-k", "not philox_matches_independent_implementation"]))
     main()

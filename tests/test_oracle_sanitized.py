@@ -31,8 +31,14 @@ def test_oracle_under_address_and_undefined_behaviour_sanitizers(tmp_path):
                     "-lm"], check=True, timeout=300)
     env = dict(os.environ, LD_PRELOAD=asan, ASAN_OPTIONS="detect_leaks=0",
                UBSAN_OPTIONS="print_stacktrace=1")
-    res = subprocess.run([sys.executable, str(ROOT / "tests" / "oracle_sanitize_run.py"), str(lib)],
-                         env=env, capture_output=True, text=True, timeout=600, cwd=str(ROOT))
+    run = [sys.executable, str(ROOT / "tests" / "oracle_sanitize_run.py"), str(lib)]
+    res = subprocess.run(run, env=env, capture_output=True, text=True, timeout=600, cwd=str(ROOT))
     assert res.returncode == 0, res.stderr[-3000:]
     assert res.stdout.strip().endswith("done")
+    assert "runtime error" not in res.stderr and "AddressSanitizer" not in res.stderr
+    # the pin suite's own calls (large draws, brute force, worked examples)
+    res = subprocess.run(run + ["--pins"], env=env, capture_output=True, text=True, timeout=900,
+                         cwd=str(ROOT))
+    assert res.returncode == 0, (res.stdout[-2000:], res.stderr[-3000:])
+    assert " passed" in res.stdout
     assert "runtime error" not in res.stderr and "AddressSanitizer" not in res.stderr

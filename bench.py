@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the integer-GEMM and training-step legs of the default line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="--impl reference: oracle seconds over the whole run (warm-up and timed "
+                         "steps), split evenly across the steps")
     ap.add_argument("--op", default="step", choices=["step", "int_gemm", "train_forward"],
                     help="step: the merge hot path (default); int_gemm: the integer "
                          "inference GEMM on merged weights")
@@ -296,17 +299,39 @@ def cpu_baseline(layers, seconds):
 # ---------------------------------------------------------------------------
 # reference arm: the oracle as it stands on the host cores
 # ---------------------------------------------------------------------------
+def reference_sample(layers, budget):
+    """The per-step sample of the reference arm: whole layers in workload
+    order while one still fits the per-step budget (seconds), else a block of
+    the first layer's leading rows taken as a layer of its own (whole path,
+    sigma over the block), sized by timing a 16-row block. Returns (layers
+    to run, description)."""
+    from dataclasses import replace
+    first = layers[0]
+    probe = replace(first, d=min(first.d, 16))
+    done, t, _ = oracle_sample([probe], 0.0)
+    per_row = t / probe.d
+    if per_row * first.d <= budget:
+        return layers, "first {count} layers in workload order, prepare + merge + STE"
+    rows = max(1, min(first.d, int(budget / per_row)))
+    return ([replace(first, d=rows)],
+            f"the first {rows} of {first.d} rows of {first.name} ({first.d}x{first.n}) taken as one "
+            f"layer, prepare + merge + STE")
+
+
 def run_reference(args, layers, desc):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    per_step_seconds = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # the whole run's oracle work stays near args.reference_seconds
+    budget = args.reference_seconds / max(1, args.steps + args.warmup)
+    per_step_seconds = min(20.0, budget)
+    sample, what = reference_sample(layers, per_step_seconds)
     for _ in range(args.warmup):
-        oracle_sample(layers, per_step_seconds)
+        oracle_sample(sample, per_step_seconds)
     done = t = 0.0
     names = []
     for _ in range(args.steps):
-        d, tt, names = oracle_sample(layers, per_step_seconds)
+        d, tt, names = oracle_sample(sample, per_step_seconds)
         done += d
         t += tt
     import oracle
@@ -318,8 +343,7 @@ def run_reference(args, layers, desc):
             "config": desc,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
                              "kind": "oracle",
-                             "sample": f"each step: first {len(names)} layers in workload "
-                                       f"order, prepare + merge + STE",
+                             "sample": "each step: " + what.format(count=len(names)),
                              "single_core": single_core(layers)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}

@@ -33,6 +33,19 @@ def test_reference_arm_json_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
 
 
+def test_reference_arm_bounds_its_steps_with_a_row_block():
+    """Many steps on a large config: each step's sample shrinks to a block of
+    the first layer's rows, so the run stays near --reference-seconds."""
+    res = subprocess.run([sys.executable, str(ROOT / "bench.py"), "--impl", "reference", "--steps", "4",
+                          "--warmup", "1", "--config", "llama3_8b", "--reference-seconds", "2"],
+                         capture_output=True, text=True, timeout=600, cwd=str(ROOT))
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = json.loads(res.stdout.strip().splitlines()[-1])
+    assert line["steps"] == 4 and line["value"] > 0
+    assert "rows of layer0.q (4096x4096) taken as one layer" in line["cpu_baseline"]["sample"]
+    assert line["ms_per_step"] < 2000.0
+
+
 @pytest.mark.parametrize("cfg", ["sd_unet", "llama3_8b", "dit_3072"])
 def test_algorithmic_counts(cfg):
     layers = wl.CONFIGS[cfg]()
